@@ -1,0 +1,423 @@
+"""Pins of the CPU oracle to facts fixed outside it.
+
+Each ``check_*`` function compares the oracle with something it does not
+share code with: a library routine (torch's bfloat16 cast, the RoPE of
+transformers' Llama, torch's scaled_dot_product_attention and topk), a closed
+form (complex rotation, relative-position dependence of an FC's share), an
+invariant (orthogonal FC decomposition sums to the dot product, GQA
+linearity, norm preservation) or brute force on tiny inputs. The mutation test
+at the bottom plants plausible mistakes in the oracle and checks that at least
+one pin fails for each.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.fasa_oracle as O
+
+RNG = np.random.default_rng(12345)
+
+
+def _close(a, b, rtol=1e-12, atol=1e-12):
+    return np.allclose(a, b, rtol=rtol, atol=atol)
+
+
+# ------------------------------------------------------------ bf16 storage
+
+def check_bf16_vs_torch(m):
+    x = (RNG.standard_normal(20000) * np.exp(RNG.uniform(-20, 20, 20000))).astype(np.float32)
+    x[:4] = [0.0, -0.0, 1.0, -3.5]
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = m.f64_to_bf16_bits(x.astype(np.float64))
+    return np.array_equal(got, want)
+
+
+def _exact_bf16(v: Fraction) -> Fraction:
+    """Nearest bfloat16 (8 significant bits), ties to even, by exact arithmetic."""
+    if v == 0:
+        return Fraction(0)
+    sgn = -1 if v < 0 else 1
+    a = abs(v)
+    e = 0
+    while a >= 2:
+        a /= 2
+        e += 1
+    while a < 1:
+        a *= 2
+        e -= 1
+    scaled = a * 128                      # in [128, 256)
+    lo = scaled.numerator // scaled.denominator
+    frac = scaled - lo
+    if frac > Fraction(1, 2) or (frac == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return sgn * Fraction(lo, 128) * Fraction(2) ** e
+
+
+def check_bf16_halfway_exact(m):
+    # values exactly at, and a hair (below float32 resolution) around, bf16 ties
+    vals = []
+    for mant in [128, 129, 200, 255]:
+        for e in [-10, 0, 3]:
+            tie = Fraction(2 * mant + 1, 256) * Fraction(2) ** e
+            for eps in [Fraction(0), Fraction(1, 2 ** 40), -Fraction(1, 2 ** 40)]:
+                vals.append(tie + eps * Fraction(2) ** e)
+    xs = np.array([float(v) for v in vals], dtype=np.float64)
+    got = m.to_f64(m.f64_to_bf16_bits(xs))
+    want = np.array([float(_exact_bf16(Fraction(float(v)))) for v in vals])
+    return np.array_equal(got, want)
+
+
+# ------------------------------------------------------------------- RoPE
+
+def check_rope_vs_complex(m):
+    base = 5e5
+    x = RNG.standard_normal((6, 128))
+    pos = np.array([0, 1, 5, 4096, 32768, 131071])
+    got = m.rope_rotate(x, pos, base)
+    theta = 1.0 / base ** (np.arange(0, 128, 2, dtype=np.float64) / 128)
+    z = (x[:, :64] + 1j * x[:, 64:]) * np.exp(1j * pos[:, None] * theta)
+    want = np.concatenate([z.real, z.imag], axis=1)
+    return _close(got, want, rtol=1e-9, atol=1e-9)
+
+
+_HF = {}
+
+
+def _hf_rope(base):
+    if base not in _HF:
+        from transformers import LlamaConfig
+        from transformers.models.llama.modeling_llama import LlamaRotaryEmbedding, apply_rotary_pos_emb
+        cfg = LlamaConfig(hidden_size=256, num_attention_heads=2, head_dim=128,
+                          rope_theta=float(base), max_position_embeddings=1 << 20)
+        _HF[base] = (LlamaRotaryEmbedding(cfg), apply_rotary_pos_emb)
+    return _HF[base]
+
+
+def check_rope_vs_transformers(m):
+    ok = True
+    for base in (1e4, 5e5):
+        rot, apply = _hf_rope(base)
+        # the library evaluates angles in float32, so compare at small positions
+        pos = torch.tensor([[0, 1, 2, 3, 17, 63, 100]])
+        x = torch.from_numpy(RNG.standard_normal((1, 1, 7, 128)))
+        cos, sin = rot(x, pos)
+        want, _ = apply(x, x, cos, sin)
+        got = m.rope_rotate(x.numpy()[0, 0], pos.numpy()[0], base)
+        ok &= _close(got, want.numpy()[0, 0], rtol=0, atol=2e-5)
+        ok &= _close(m.rope_frequencies(base), rot.inv_freq.double().numpy(), rtol=2e-6, atol=0)
+    return bool(ok)
+
+
+def check_rope_invariants(m):
+    x = RNG.standard_normal((9, 128))
+    ok = _close(m.rope_rotate(x, 0, 1e4), x)                      # identity at 0
+    r = m.rope_rotate(x, 777, 1e4)
+    n0 = x[:, :64] ** 2 + x[:, 64:] ** 2
+    n1 = r[:, :64] ** 2 + r[:, 64:] ** 2
+    ok &= _close(n0, n1, rtol=1e-12)                               # per-FC norm kept
+    ok &= _close(m.rope_rotate(m.rope_rotate(x, 300, 1e4), 477, 1e4), r, rtol=1e-9, atol=1e-9)
+    return bool(ok)
+
+
+# -------------------------------------------------------------- FC shares
+
+def check_fc_partials_sum_to_dot(m):
+    q = RNG.standard_normal((5, 128))
+    k = RNG.standard_normal((5, 128))
+    P = m.fc_partials(q, k)
+    return P.shape == (5, 64) and _close(P.sum(-1), np.einsum("ij,ij->i", q, k))
+
+
+def check_fc_partial_closed_form(m):
+    base = 1e4
+    q = RNG.standard_normal(128)
+    k = RNG.standard_normal(128)
+    ok = True
+    th = 1.0 / base ** (np.arange(0, 128, 2) / 128.0)
+    qc = q[:64] + 1j * q[64:]
+    kc = k[:64] + 1j * k[64:]
+    for p, t in [(4096, 0), (4096, 4095), (100, 37), (37, 100)]:
+        P = m.fc_partials(m.rope_rotate(q, p, base), m.rope_rotate(k, t, base))
+        want = np.real(qc * np.conj(kc) * np.exp(1j * (p - t) * th))
+        ok &= _close(P, want, rtol=1e-9, atol=1e-9)
+        # only the relative position matters
+        P2 = m.fc_partials(m.rope_rotate(q, p + 500, base), m.rope_rotate(k, t + 500, base))
+        ok &= _close(P, P2, rtol=1e-8, atol=1e-8)
+    return bool(ok)
+
+
+# -------------------------------------------------------------------- TIP
+
+def _head(L=40, G=3, base=1e4, seed=0, dtype="f32"):
+    r = np.random.default_rng(seed)
+    qpre = r.standard_normal((G, 128)).astype(np.float32)
+    kpre = r.standard_normal((L, 128)).astype(np.float32)
+    v = r.standard_normal((L, 128)).astype(np.float32)
+    if dtype == "bf16":
+        qpre = O.f64_to_bf16_bits(qpre.astype(np.float64))
+        kpre = O.f64_to_bf16_bits(kpre.astype(np.float64))
+        v = O.f64_to_bf16_bits(v.astype(np.float64))
+    return qpre, kpre, v
+
+
+def check_tip_all_fcs_is_dot(m):
+    qpre, kpre, v = _head()
+    dom = np.arange(64)
+    k_rot, _, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    qr = m.rotate_queries(qpre, 40, 1e4)
+    s = m.tip_scores(qr, sk, dom)
+    want = (qr @ m.to_f64(k_rot).T).sum(0)
+    return _close(s, want, rtol=1e-10, atol=1e-10)
+
+
+def check_tip_subset_is_partial_sum(m):
+    qpre, kpre, v = _head(seed=1)
+    dom = np.array([5, 63, 0, 17, 40])
+    k_rot, _, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    qr = m.rotate_queries(qpre, 40, 1e4)
+    P = m.fc_partials(qr[:, None, :], m.to_f64(k_rot)[None, :, :])   # [G, L, 64]
+    want = P[:, :, dom].sum(axis=(0, 2))
+    return _close(m.tip_scores(qr, sk, dom), want, rtol=1e-10, atol=1e-10)
+
+
+def check_tip_gqa_linear(m):
+    qpre, kpre, v = _head(seed=2, G=4)
+    dom = np.array([3, 9, 27])
+    _, _, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    qr = m.rotate_queries(qpre, 40, 1e4)
+    s_group = m.tip_scores(qr, sk, dom)
+    s_sum = m.tip_scores(qr.sum(0, keepdims=True), sk, dom)
+    return _close(s_group, s_sum, rtol=1e-10, atol=1e-10)
+
+
+def check_tip_brute_force(m):
+    qpre, kpre, v = _head(L=12, G=2, seed=3)
+    dom = [7, 1, 50]
+    k_rot, _, sk = m.append_kv(kpre, v, 0, 1e4, np.array(dom), "f32")
+    qr = m.rotate_queries(qpre, 12, 1e4)
+    kr = m.to_f64(k_rot)
+    want = []
+    for t in range(12):
+        acc = 0.0
+        for h in range(2):
+            for i in dom:
+                acc += qr[h][i] * kr[t][i] + qr[h][i + 64] * kr[t][i + 64]
+        want.append(acc)
+    return _close(m.tip_scores(qr, sk, np.array(dom)), np.array(want), rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- select
+
+def check_select_brute_force(m):
+    ok = True
+    r = np.random.default_rng(4)
+    for L, k in [(1, 1), (7, 3), (20, 5), (33, 33), (10, 25), (40, 1)]:
+        s = r.integers(-3, 4, L).astype(np.float64)          # many exact ties
+        want = []
+        for t in range(L):
+            rank = sum(1 for u in range(L) if s[u] > s[t] or (s[u] == s[t] and u < t))
+            if rank < min(k, L):
+                want.append(t)
+        got = m.select_critical_set(s, k)
+        ok &= list(got) == want
+    return bool(ok)
+
+
+def check_select_permutation(m):
+    r = np.random.default_rng(5)
+    s = r.standard_normal(200)
+    perm = r.permutation(200)
+    a = set(m.select_critical_set(s, 17).tolist())
+    b = set(perm[m.select_critical_set(s[perm], 17)].tolist())
+    return a == b and len(a) == 17
+
+
+# -------------------------------------------------------------------- FAC
+
+def _sdpa(q, K, V):
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+
+
+def check_dense_vs_sdpa(m):
+    r = np.random.default_rng(6)
+    q = r.standard_normal((4, 128)) * 0.3
+    K = r.standard_normal((50, 128))
+    V = r.standard_normal((50, 128))
+    return _close(m.dense_attention(q, K, V), _sdpa(q, K, V), rtol=1e-10, atol=1e-12)
+
+
+def check_focused_special_cases(m):
+    r = np.random.default_rng(7)
+    q = r.standard_normal((3, 128)) * 0.3
+    K = r.standard_normal((30, 128))
+    V = r.standard_normal((30, 128))
+    ok = _close(m.focused_attention(q, K, V, np.arange(30)), m.dense_attention(q, K, V))
+    idx = np.array([2, 9, 11, 20])
+    o = m.focused_attention(q, K, V, idx)
+    ok &= _close(o, _sdpa(q, K[idx], V[idx]), rtol=1e-10, atol=1e-12)
+    ok &= bool(np.all(o <= V[idx].max(0) + 1e-12) and np.all(o >= V[idx].min(0) - 1e-12))
+    one = m.focused_attention(q, K, V, np.array([13]))
+    ok &= _close(one, np.repeat(V[13][None], 3, 0))
+    return bool(ok)
+
+
+# ------------------------------------------------------------- end to end
+
+def check_e2e_all_fc_full_k_is_dense(m):
+    qpre, kpre, v = _head(L=64, G=2, seed=8)
+    dom = np.arange(64)
+    k_rot, v_st, sk = m.append_kv(kpre, v, 0, 5e5, dom, "f32")
+    idx, out, _ = m.decode_head(qpre, 64, k_rot, v_st, sk, dom, 64, 5e5)
+    qr = m.rope_rotate(m.to_f64(qpre), 64, 5e5)
+    want = _sdpa(qr, m.to_f64(k_rot), m.to_f64(v_st))
+    return list(idx) == list(range(64)) and _close(out, want, rtol=1e-9, atol=1e-12)
+
+
+def check_e2e_all_fc_topk_exact(m):
+    qpre, kpre, v = _head(L=64, G=1, seed=9)
+    dom = np.arange(64)
+    k_rot, v_st, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    idx, out, _ = m.decode_head(qpre, 64, k_rot, v_st, sk, dom, 9, 1e4)
+    qr = m.rope_rotate(m.to_f64(qpre), 64, 1e4)
+    logits = torch.from_numpy(qr @ m.to_f64(k_rot).T)[0]
+    top = np.sort(torch.topk(logits, 9).indices.numpy())
+    want = _sdpa(qr, m.to_f64(k_rot)[top], m.to_f64(v_st)[top])
+    return list(idx) == list(top) and _close(out, want, rtol=1e-9, atol=1e-12)
+
+
+def check_append_positions(m):
+    qpre, kpre, v = _head(L=30, seed=10, dtype="bf16")
+    dom = np.array([0, 2, 4])
+    a = m.append_kv(kpre, v, 0, 1e4, dom, "bf16")
+    b1 = m.append_kv(kpre[:11], v[:11], 0, 1e4, dom, "bf16")
+    b2 = m.append_kv(kpre[11:], v[11:], 11, 1e4, dom, "bf16")
+    ok = all(np.array_equal(x, np.concatenate([y, z])) for x, y, z in zip(a, b1, b2))
+    # slot t holds the key rotated at absolute position t
+    t = 23
+    ok &= np.array_equal(a[0][t], m.store(m.rope_rotate(m.to_f64(kpre[t]), t, 1e4), "bf16"))
+    return bool(ok)
+
+
+PINS = [check_bf16_vs_torch, check_bf16_halfway_exact, check_rope_vs_complex,
+        check_rope_vs_transformers, check_rope_invariants, check_fc_partials_sum_to_dot,
+        check_fc_partial_closed_form, check_tip_all_fcs_is_dot, check_tip_subset_is_partial_sum,
+        check_tip_gqa_linear, check_tip_brute_force, check_select_brute_force,
+        check_select_permutation, check_dense_vs_sdpa, check_focused_special_cases,
+        check_e2e_all_fc_full_k_is_dense, check_e2e_all_fc_topk_exact, check_append_positions]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_oracle_pin(pin):
+    assert pin(O)
+
+
+def test_golden_fixture_matches_oracle():
+    """Regression fixture written by tests/golden/make_golden.py (oracle only)."""
+    import json, os
+    from tests.golden.make_golden import compute_golden
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_decode.json")
+    with open(path) as f:
+        stored = json.load(f)
+    fresh = compute_golden()
+    assert stored["idx"] == fresh["idx"]
+    np.testing.assert_allclose(stored["out"], fresh["out"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(stored["scores"], fresh["scores"], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------- mutations
+
+def _mut_rope_sign(x, pos, base):
+    x = np.asarray(x, dtype=np.float64)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * O.rope_frequencies(base, x.shape[-1])
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :64], x[..., 64:]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
+
+
+def _mut_rope_adjacent(x, pos, base):
+    x = np.asarray(x, dtype=np.float64)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * O.rope_frequencies(base, x.shape[-1])
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    x1, x2 = x[..., 0::2], x[..., 1::2]
+    out[..., 0::2] = x1 * c - x2 * s
+    out[..., 1::2] = x2 * c + x1 * s
+    return out
+
+
+def _mut_freq(base, d=128):
+    return np.power(float(base), -1.0 * np.arange(d // 2) / d)
+
+
+def _mut_partials(qr, kr):
+    return qr[..., :64] * kr[..., :64]
+
+
+def _mut_tip_head0(q_rot, sketch, dom):
+    return _orig_tip(q_rot[:1], sketch, dom)
+
+
+def _mut_select_high_tie(scores, k):
+    s = np.asarray(scores, dtype=np.float64)
+    order = np.lexsort((-np.arange(len(s)), -s))
+    return np.sort(order[:min(k, len(s))])
+
+
+def _mut_no_scale(q_rot, k_rot, v, idx):
+    idx = np.asarray(idx)
+    K, V = O.to_f64(k_rot)[idx], O.to_f64(v)[idx]
+    z = q_rot @ K.T
+    p = np.exp(z - z.max(-1, keepdims=True))
+    return (p / p.sum(-1, keepdims=True)) @ V
+
+
+def _mut_sketch(k_rot, dom):
+    dom = np.asarray(dom)
+    out = np.empty(k_rot.shape[:-1] + (2 * len(dom),), dtype=k_rot.dtype)
+    out[..., 0::2] = k_rot[..., dom]
+    out[..., 1::2] = k_rot[..., (dom + 1) % 128]
+    return out
+
+
+def _mut_append_pos(k_pre, v, pos0, base, dom, dtype):
+    return _orig_append(k_pre, v, pos0 + 1, base, dom, dtype)
+
+
+def _mut_bf16_trunc(x):
+    x = np.asarray(x, np.float64).astype(np.float32)
+    return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+
+_orig_append = O.append_kv
+_orig_tip = O.tip_scores
+
+MUTANTS = {
+    "rope_rotates_backwards": ("rope_rotate", _mut_rope_sign),
+    "rope_adjacent_pairs": ("rope_rotate", _mut_rope_adjacent),
+    "rope_theta_exponent": ("rope_frequencies", _mut_freq),
+    "fc_partial_drops_half": ("fc_partials", _mut_partials),
+    "tip_drops_group_heads": ("tip_scores", _mut_tip_head0),
+    "select_ties_to_higher_index": ("select_critical_set", _mut_select_high_tie),
+    "attention_without_scale": ("focused_attention", _mut_no_scale),
+    "sketch_wrong_pair": ("sketch_rows", _mut_sketch),
+    "append_position_off_by_one": ("append_kv", _mut_append_pos),
+    "bf16_truncates": ("f64_to_bf16_bits", _mut_bf16_trunc),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for pin in PINS:
+        try:
+            ok = pin(O)
+        except Exception:
+            ok = False
+        if not ok:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
