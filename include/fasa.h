@@ -1,0 +1,228 @@
+/*
+ * fasa.h -- C ABI of the FASA decode hot path on NVIDIA B200 (sm_100a).
+ *
+ * FASA ("FASA: Frequency-aware Sparse Attention", Wang et al.) predicts which
+ * cached tokens matter for the current query from a few RoPE frequency chunks
+ * (FCs), keeps the top-k of them, and runs exact softmax attention over only
+ * those rows. Citations below name the page and section that define each step:
+ *
+ *   [abstract]  chatpaper.ai page "FASA: Frequency-aware Sparse Attention",
+ *               English abstract.
+ *   [tech §2]   gist.science page "FASA: Frequency-aware Sparse Attention",
+ *               "Resumo Técnico" (technical summary), §2 "Metodologia e
+ *               Insight Central": "A Descoberta" (FCs), the TIP bullets
+ *               (offline calibration, online prediction), the FAC bullets,
+ *               and "Variantes de Implementação" (FASA-M / FASA-C).
+ *
+ * Notation: B batch, Hq query heads, Hkv KV heads, G = Hq / Hkv query heads
+ * per KV head (query head h belongs to KV head h / G), d = 128 head dim,
+ * 64 FCs; FC i is the dim pair (i, i + 64) ("rotate-half" pairing) rotated at
+ * theta_i = rope_base^(-2i/128). A cached token in slot t sits at absolute
+ * position t. "dtype" is the cache dtype, used for keys, values, queries and
+ * outputs alike.
+ *
+ * Conventions shared by every call:
+ *  - All pointers are DEVICE pointers owned by the caller, 16-byte aligned,
+ *    tensors dense and row-major as documented. The library allocates no
+ *    memory; fasa_decode takes a caller-owned workspace.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and do not
+ *    synchronize, except fasa_device_status.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call launches nothing and returns an error status. A CUDA launch
+ *    failure returns FASA_ERR_CUDA. No call aborts, throws, or traps the GPU.
+ *  - Problems only the device can see (an out-of-range token index given to
+ *    fasa_sparse_attend, an out-of-range dominant-FC index, a bounded wait
+ *    that gave up) are recorded in a sticky per-device status word, read by
+ *    fasa_device_status. The offending element is skipped, never accessed.
+ *  - Thread safety: calls may be made from several host threads; the only
+ *    library state is the per-device status word and cached device attributes.
+ */
+#ifndef FASA_H_
+#define FASA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FASA_ABI_VERSION 1
+#define FASA_HEAD_DIM 128
+#define FASA_NUM_FC 64
+#define FASA_MAX_GROUP 16          /* largest G = Hq / Hkv */
+#define FASA_MAX_LEN (1 << 19)     /* largest cached length a decode call accepts */
+#define FASA_MAX_K (1 << 17)       /* largest kept-token budget */
+
+typedef enum fasa_status {
+  FASA_OK = 0,
+  FASA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or range */
+  FASA_ERR_UNSUPPORTED = 2,   /* head_dim != 128, G > 16, len > FASA_MAX_LEN, ... */
+  FASA_ERR_CAPACITY = 3,      /* write or read beyond max_len */
+  FASA_ERR_WORKSPACE = 4,     /* workspace missing or too small */
+  FASA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  FASA_ERR_TIMEOUT = 6,       /* device: a bounded wait gave up (status word) */
+  FASA_ERR_BAD_INDEX = 7      /* device: an index outside its range was skipped */
+} fasa_status;
+
+typedef enum fasa_dtype { FASA_F32 = 0, FASA_BF16 = 1 } fasa_dtype;
+
+/*
+ * A KV cache of one attention layer, with its dominant-FC key sketch.
+ *
+ *  k, v    : [B][Hkv][max_len][128] dtype. Slot t of (b, g) holds the key
+ *            rotated at position t (RoPE applied at append time) and the
+ *            unrotated value.
+ *  sketch  : [B][Hkv][max_len][sketch_stride] dtype. Row t of (b, g) holds,
+ *            for j = 0 .. n_dom-1, element 2j = k[b][g][t][dom[g][j]] and
+ *            element 2j+1 = k[b][g][t][dom[g][j] + 64] (the two dims of
+ *            dominant FC j, copied from the stored rotated key); elements
+ *            2*n_dom .. sketch_stride-1 are zero. It is what TIP reads, so a
+ *            decode step streams 2*n_dom values per token instead of 256
+ *            ([tech §2] FASA-C reads only a sparse subset of key state;
+ *            FASA-M keeps the dominant key parts on the GPU apart from the
+ *            rest).
+ *  dom_idx : [Hkv][n_dom] int32, the dominant FCs I_dom of each KV head from
+ *            offline calibration ([tech §2] TIP, first bullet): distinct,
+ *            each in [0, 64). fasa_check_dom_idx validates a host copy.
+ *  sketch_stride must equal fasa_sketch_stride(n_dom, dtype).
+ */
+typedef struct fasa_cache {
+  int32_t batch;          /* B >= 1 */
+  int32_t n_q_heads;      /* Hq, a multiple of Hkv */
+  int32_t n_kv_heads;     /* Hkv >= 1 */
+  int32_t head_dim;       /* must be 128 */
+  int32_t n_dom;          /* 1 .. 64 */
+  int32_t max_len;        /* capacity in tokens, 1 .. 2^30 */
+  int32_t dtype;          /* fasa_dtype */
+  int32_t sketch_stride;  /* elements per sketch row */
+  double rope_base;       /* > 1 */
+  void* k;
+  void* v;
+  void* sketch;
+  const int32_t* dom_idx;
+} fasa_cache;
+
+/* ABI version (FASA_ABI_VERSION of the built library). */
+int32_t fasa_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fasa_status_string(int32_t status);
+
+/* Sketch row length in elements for n_dom dominant FCs: 2*n_dom rounded up
+ * so that a row is a power-of-two number of 16-byte chunks (so a 16-byte load
+ * never straddles two tokens). Returns -1 for n_dom outside 1..64 or an
+ * unknown dtype. */
+int32_t fasa_sketch_stride(int32_t n_dom, int32_t dtype);
+
+/* Host-side check of a HOST copy of dom_idx ([Hkv][n_dom]): FASA_OK when
+ * every row holds distinct values in [0, 64), else FASA_ERR_INVALID_ARG. */
+fasa_status fasa_check_dom_idx(const int32_t* dom_idx_host, int32_t n_kv_heads, int32_t n_dom);
+
+/*
+ * Append n_new tokens at positions pos0 .. pos0+n_new-1 of every sequence.
+ * [tech §2] "A Descoberta" (RoPE rotates each FC at its own frequency) and
+ * FAC (positions are kept absolute): each key is rotated at its own position
+ * once, here, and stored rotated.
+ *
+ *  k_new, v_new : [B][Hkv][n_new][128] dtype, pre-RoPE keys and values.
+ *  Writes k, v and sketch rows pos0 .. pos0+n_new-1 of every (b, g).
+ *  Arithmetic: cos/sin and the rotation in float64, rounded once to dtype
+ *  (round to nearest even).
+ *  Errors: FASA_ERR_CAPACITY when pos0 + n_new > max_len; n_new == 0 is a
+ *  no-op returning FASA_OK.
+ */
+fasa_status fasa_append_kv(const fasa_cache* cache, const void* k_new, const void* v_new,
+                           int32_t n_new, int32_t pos0, cudaStream_t stream);
+
+/*
+ * TIP online prediction ([tech §2] TIP, second bullet; [abstract]: the
+ * dominant FCs are a computationally free proxy for token importance).
+ * For every sequence b, KV head g and cached token t < len:
+ *   scores[b][g][t] = sum over the G query heads h of g, and over the
+ *   dominant FCs i of g, of  q'_h[i] k[t][i] + q'_h[i+64] k[t][i+64],
+ * where q'_h is query h rotated at position q_pos.
+ *
+ *  q      : [B][Hq][128] dtype, pre-RoPE queries.
+ *  scores : [B][Hkv][len] float32 (row stride len).
+ *  Arithmetic: query rotation and the sum in float64, rounded once to float32.
+ *  len may be 0 (nothing is written). Errors: FASA_ERR_CAPACITY if
+ *  len > max_len.
+ */
+fasa_status fasa_score(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
+                       float* scores, cudaStream_t stream);
+
+/*
+ * Critical-set selection T_t ([tech §2] FAC, first bullet): for each of
+ * n_rows score rows, the indices of the k_eff = min(k, len) largest scores;
+ * equal scores go to the lower index (-0.0 counts as +0.0); indices are
+ * written in ascending order. Exact (radix select on order-preserving keys).
+ *
+ *  scores : [n_rows][len] float32, finite.
+ *  idx    : [n_rows][k_eff] int32.
+ *  Errors: k < 1, len < 1 or n_rows < 1 -> FASA_ERR_INVALID_ARG;
+ *  len > FASA_MAX_LEN or k > FASA_MAX_K -> FASA_ERR_UNSUPPORTED.
+ */
+fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, int32_t k,
+                             int32_t* idx, cudaStream_t stream);
+
+/*
+ * Focused attention ([tech §2] FAC, second and third bullets): full softmax
+ * attention of each query head over only the given rows of its KV head,
+ * each row at its original absolute position (keys were rotated at append):
+ *   out[b][h] = sum_j softmax_j(q'_h . k[idx_j] / sqrt(128)) v[idx_j].
+ *
+ *  q    : [B][Hq][128] dtype, pre-RoPE (rotated here at q_pos).
+ *  idx  : [B][Hkv][n_idx] int32, each in [0, len); duplicates count twice.
+ *         An index outside [0, len) is skipped and recorded as
+ *         FASA_ERR_BAD_INDEX in the device status word.
+ *  out  : [B][Hq][128] dtype.
+ *  Arithmetic: float32 logits and online softmax, output rounded to dtype.
+ *  Errors: n_idx < 1 or len < 1 -> FASA_ERR_INVALID_ARG.
+ */
+fasa_status fasa_sparse_attend(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
+                               const int32_t* idx, int32_t n_idx, void* out, cudaStream_t stream);
+
+/* Workspace bytes fasa_decode needs for this cache at cached length len. */
+size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len);
+
+/*
+ * One FASA decode step over a layer: TIP (fasa_score) -> T_t
+ * (fasa_select_topk with k) -> FAC (fasa_sparse_attend), fused into two
+ * launches; scores stay in the workspace and the kept indices stay on chip.
+ *
+ *  out     : [B][Hq][128] dtype.
+ *  idx_out : nullable; [B][Hkv][min(k, len)] int32, the kept tokens in
+ *            ascending order.
+ *  workspace : caller-owned device memory of at least
+ *            fasa_decode_workspace_bytes(cache, len) bytes, 256-byte aligned;
+ *            its contents need no initialisation and are scratch.
+ *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;
+ *  FASA_ERR_WORKSPACE if the workspace is missing or too small.
+ */
+fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
+                        int32_t k, void* out, int32_t* idx_out, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Dense full-KV decode, the comparison path: the same attention as
+ * fasa_sparse_attend over all len cached rows (the upper bound in
+ * [tech §4] "Resultados Experimentais", full KV "FKV").
+ */
+fasa_status fasa_dense_decode(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
+                              void* out, cudaStream_t stream);
+
+/*
+ * Synchronizes the current device, then returns FASA_OK or the first
+ * device-side problem recorded since the status was last cleared
+ * (FASA_ERR_BAD_INDEX, FASA_ERR_TIMEOUT); clears it when clear != 0.
+ * Returns FASA_ERR_CUDA if the synchronization itself fails.
+ */
+fasa_status fasa_device_status(int32_t clear);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* FASA_H_ */

@@ -1,0 +1,461 @@
+// C ABI of the FASA decode hot path (declared in include/fasa.h).
+//
+// Host side only: argument validation (before any launch), launch-shape
+// choice, and dispatch to the kernels in append.cuh, score.cuh and
+// select_attend.cuh. Nothing here allocates device memory.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <unordered_map>
+
+#include "append.cuh"
+#include "fasa_device.cuh"
+#include "score.cuh"
+#include "select_attend.cuh"
+
+using namespace fasa;
+
+namespace {
+
+constexpr int kMaxChunkKeys = 32768;  // keys per CTA held in shared memory
+constexpr int kMaxSlice = 8192;       // kept indices per CTA
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+  bool ready = false;
+  int sms = 0;
+  int smem_optin = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+std::unordered_map<uint64_t, int> g_cache;  // (device, kernel, key) -> value
+
+fasa_status device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FASA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FASA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return FASA_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = d;
+  return FASA_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int pow2ceil(int64_t x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+inline int elem_bytes(int dtype) { return dtype == FASA_F32 ? 4 : 2; }
+
+void fill_theta(double* th, double base) {
+  for (int i = 0; i < kNFC; ++i) th[i] = std::pow(base, -2.0 * (double)i / (double)kD);
+}
+
+fasa_status check_cache(const fasa_cache* c) {
+  if (c == nullptr) return FASA_ERR_INVALID_ARG;
+  if (c->head_dim != kD) return FASA_ERR_UNSUPPORTED;
+  if (c->dtype != FASA_F32 && c->dtype != FASA_BF16) return FASA_ERR_UNSUPPORTED;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0)
+    return FASA_ERR_INVALID_ARG;
+  if (c->n_q_heads / c->n_kv_heads > FASA_MAX_GROUP) return FASA_ERR_UNSUPPORTED;
+  if ((int64_t)c->batch * c->n_kv_heads > 65535) return FASA_ERR_UNSUPPORTED;
+  if (c->n_dom < 1 || c->n_dom > kNFC) return FASA_ERR_INVALID_ARG;
+  if (c->sketch_stride != fasa_sketch_stride(c->n_dom, c->dtype)) return FASA_ERR_INVALID_ARG;
+  if (c->max_len < 1 || c->max_len > (1 << 30)) return FASA_ERR_INVALID_ARG;
+  if (!(c->rope_base > 1.0) || !std::isfinite(c->rope_base)) return FASA_ERR_INVALID_ARG;
+  if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->sketch, 16) || !aligned(c->dom_idx, 4))
+    return FASA_ERR_INVALID_ARG;
+  return FASA_OK;
+}
+
+fasa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FASA_OK;
+  (void)cudaGetLastError();  // clear a non-sticky launch error
+  return FASA_ERR_CUDA;
+}
+
+// Cached per (device, kernel, key) integer, computed once by `fn`.
+template <typename F>
+fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FASA_ERR_CUDA;
+  const uint64_t h = (reinterpret_cast<uint64_t>(kernel) * 1000003ull) ^ (key * 131ull) ^ (uint64_t)dev;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_cache.find(h);
+    if (it != g_cache.end()) {
+      *out = it->second;
+      return FASA_OK;
+    }
+  }
+  int v = 0;
+  const fasa_status st = fn(&v);
+  if (st != FASA_OK) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_cache[h] = v;
+  *out = v;
+  return FASA_OK;
+}
+
+// ------------------------------------------------------------ score
+
+template <typename T, int LPT>
+fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
+  auto kern = score_kernel<T, LPT>;
+  int occ = 0;
+  fasa_status s = cached_int((const void*)kern, 0, &occ, [&](int* v) {
+    return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kern, kScoreThreads, 0));
+  });
+  if (s != FASA_OK) return s;
+  const int64_t want = (int64_t)d.sms * (occ > 0 ? occ : 1);
+  const int64_t cap = ceil_div(p.total, 256);  // at least 256 tokens per CTA
+  const int grid = (int)std::max<int64_t>(1, std::min(want, cap));
+  kern<<<grid, kScoreThreads, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T>
+fasa_status launch_score_lpt(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
+  const int lpt = p.stride * (int)sizeof(T) / 16;
+  switch (lpt) {
+    case 1: return launch_score_t<T, 1>(p, d, st);
+    case 2: return launch_score_t<T, 2>(p, d, st);
+    case 4: return launch_score_t<T, 4>(p, d, st);
+    case 8: return launch_score_t<T, 8>(p, d, st);
+    case 16: return launch_score_t<T, 16>(p, d, st);
+    case 32: return launch_score_t<T, 32>(p, d, st);
+    default: return FASA_ERR_UNSUPPORTED;
+  }
+}
+
+fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
+                         cudaStream_t st) {
+  DevInfo d;
+  fasa_status s = device_info(&d);
+  if (s != FASA_OK) return s;
+  ScoreParams p{};
+  p.sketch = c->sketch;
+  p.q = q;
+  p.dom_idx = c->dom_idx;
+  p.scores = scores;
+  p.max_len = c->max_len;
+  p.total = (int64_t)c->batch * c->n_kv_heads * len;
+  p.len = len;
+  p.stride = c->sketch_stride;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.n_dom = c->n_dom;
+  p.q_pos = q_pos;
+  fill_theta(p.theta, c->rope_base);
+  return c->dtype == FASA_F32 ? launch_score_lpt<float>(p, d, st) : launch_score_lpt<__nv_bfloat16>(p, d, st);
+}
+
+// ---------------------------------------------------- select / attend
+
+struct SAShape {
+  int C, chunk, slice, smem;
+};
+
+inline int maxg_for(int g) { return g <= 4 ? 4 : (g <= 8 ? 8 : 16); }
+
+template <typename T, int MODE, int MAXG>
+fasa_status launch_sa_t(SAParams p, int rows, int C, bool pdl, cudaStream_t st, const DevInfo& d) {
+  auto kern = select_attend_kernel<T, MODE, MAXG>;
+  const SALayout L = sa_layout(MODE, (int)sizeof(T), p.chunk, p.slice, MAXG);
+  if (L.total > d.smem_optin) return FASA_ERR_UNSUPPORTED;
+  int set = 0;
+  fasa_status s = cached_int((const void*)kern, 1, &set, [&](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    *v = 1;
+    return cuda_status(e);
+  });
+  if (s != FASA_OK) return s;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[2];
+  cfg.gridDim = dim3((unsigned)C, (unsigned)rows, 1);
+  cfg.blockDim = dim3(kSAThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)L.total;
+  cfg.stream = st;
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = (unsigned)C;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  int na = 1;
+  if (pdl) {
+    attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
+
+  if (C > 8) {  // non-portable cluster size: make sure it can be co-scheduled
+    int nclus = 0;
+    s = cached_int((const void*)kern, 1000ull + (uint64_t)C * 1000003ull + (uint64_t)L.total, &nclus, [&](int* v) {
+      return cuda_status(cudaOccupancyMaxActiveClusters(v, kern, &cfg));
+    });
+    if (s != FASA_OK) return s;
+    if (nclus < 1) return FASA_ERR_UNSUPPORTED;
+  }
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
+}
+
+template <typename T, int MODE>
+fasa_status launch_sa_g(const SAParams& p, int rows, int C, bool pdl, cudaStream_t st, const DevInfo& d) {
+  switch (maxg_for(p.group)) {
+    case 4: return launch_sa_t<T, MODE, 4>(p, rows, C, pdl, st, d);
+    case 8: return launch_sa_t<T, MODE, 8>(p, rows, C, pdl, st, d);
+    default: return launch_sa_t<T, MODE, 16>(p, rows, C, pdl, st, d);
+  }
+}
+
+// Cluster size: enough CTAs to cover the GPU, within the shared-memory
+// limits on keys and kept indices per CTA.
+int choose_cluster(int mode, int rows, int64_t len, int64_t keep, int sms) {
+  int cmin = 1;
+  if (mode == kSelect || mode == kDecode) cmin = std::max(cmin, pow2ceil(ceil_div(len, kMaxChunkKeys)));
+  if (mode == kDecode || mode == kAttendIdx) cmin = std::max(cmin, pow2ceil(ceil_div(keep, kMaxSlice)));
+  const int64_t target = (mode == kDense ? 8 : 2) * (int64_t)sms;
+  const int cfill = pow2ceil(ceil_div(target, rows));
+  return std::max(cmin, std::min(cfill, kMaxCluster));
+}
+
+template <int MODE>
+fasa_status launch_sa(const fasa_cache* c, SAParams p, int rows, bool pdl, cudaStream_t st, int dtype) {
+  DevInfo d;
+  fasa_status s = device_info(&d);
+  if (s != FASA_OK) return s;
+  int C = choose_cluster(MODE, rows, p.len, p.n_keep, d.sms);
+  if (C > kMaxCluster) return FASA_ERR_UNSUPPORTED;
+  for (;;) {
+    p.chunk = (int)ceil_div(p.len, C);
+    p.slice = (int)ceil_div(p.n_keep, C);
+    if (c) fill_theta(p.theta, c->rope_base);
+    if constexpr (MODE == kSelect) {
+      s = launch_sa_t<float, MODE, 4>(p, rows, C, pdl, st, d);
+    } else {
+      if (dtype == FASA_F32)
+        s = launch_sa_g<float, MODE>(p, rows, C, pdl, st, d);
+      else
+        s = launch_sa_g<__nv_bfloat16, MODE>(p, rows, C, pdl, st, d);
+    }
+    // a 16-CTA cluster that cannot be co-scheduled: retry with 8 when allowed
+    if (s == FASA_ERR_UNSUPPORTED && C == 16) {
+      const int cmin = choose_cluster(MODE, 1 << 30, p.len, p.n_keep, d.sms);
+      if (cmin <= 8) {
+        C = 8;
+        continue;
+      }
+    }
+    return s;
+  }
+}
+
+size_t decode_ws(const fasa_cache* c, int32_t len) {
+  const size_t b = (size_t)c->batch * c->n_kv_heads * (size_t)std::max(len, 0) * sizeof(float);
+  return (b + 255) / 256 * 256 + 256;
+}
+
+}  // namespace
+
+// =================================================================== ABI
+
+extern "C" {
+
+int32_t fasa_abi_version(void) { return FASA_ABI_VERSION; }
+
+const char* fasa_status_string(int32_t s) {
+  switch (s) {
+    case FASA_OK: return "FASA_OK";
+    case FASA_ERR_INVALID_ARG: return "FASA_ERR_INVALID_ARG";
+    case FASA_ERR_UNSUPPORTED: return "FASA_ERR_UNSUPPORTED";
+    case FASA_ERR_CAPACITY: return "FASA_ERR_CAPACITY";
+    case FASA_ERR_WORKSPACE: return "FASA_ERR_WORKSPACE";
+    case FASA_ERR_CUDA: return "FASA_ERR_CUDA";
+    case FASA_ERR_TIMEOUT: return "FASA_ERR_TIMEOUT";
+    case FASA_ERR_BAD_INDEX: return "FASA_ERR_BAD_INDEX";
+    default: return "FASA_ERR_UNKNOWN";
+  }
+}
+
+int32_t fasa_sketch_stride(int32_t n_dom, int32_t dtype) {
+  if (n_dom < 1 || n_dom > kNFC) return -1;
+  if (dtype != FASA_F32 && dtype != FASA_BF16) return -1;
+  const int per16 = 16 / elem_bytes(dtype);
+  const int chunks = pow2ceil(ceil_div(2 * n_dom, per16));
+  return chunks * per16;
+}
+
+fasa_status fasa_check_dom_idx(const int32_t* dom, int32_t n_kv_heads, int32_t n_dom) {
+  if (dom == nullptr || n_kv_heads < 1 || n_dom < 1 || n_dom > kNFC) return FASA_ERR_INVALID_ARG;
+  for (int g = 0; g < n_kv_heads; ++g) {
+    bool seen[kNFC] = {false};
+    for (int j = 0; j < n_dom; ++j) {
+      const int v = dom[g * n_dom + j];
+      if (v < 0 || v >= kNFC || seen[v]) return FASA_ERR_INVALID_ARG;
+      seen[v] = true;
+    }
+  }
+  return FASA_OK;
+}
+
+fasa_status fasa_append_kv(const fasa_cache* c, const void* k_new, const void* v_new, int32_t n_new,
+                           int32_t pos0, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (n_new < 0 || pos0 < 0) return FASA_ERR_INVALID_ARG;
+  if ((int64_t)pos0 + n_new > c->max_len) return FASA_ERR_CAPACITY;
+  if (n_new == 0) return FASA_OK;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return FASA_ERR_INVALID_ARG;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return s;
+  AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k = c->k;
+  p.v = c->v;
+  p.sketch = c->sketch;
+  p.dom_idx = c->dom_idx;
+  p.max_len = c->max_len;
+  p.n_rows = c->batch * c->n_kv_heads;
+  p.n_kv_heads = c->n_kv_heads;
+  p.n_new = n_new;
+  p.pos0 = pos0;
+  p.n_dom = c->n_dom;
+  p.stride = c->sketch_stride;
+  fill_theta(p.theta, c->rope_base);
+  const int64_t tok_blocks = ceil_div(n_new, kAppendTok);
+  const int64_t groups = std::max<int64_t>(1, std::min<int64_t>(p.n_rows, ceil_div(4LL * d.sms, tok_blocks)));
+  p.heads_per_cta = (int)ceil_div(p.n_rows, groups);
+  const dim3 grid((unsigned)tok_blocks, (unsigned)ceil_div(p.n_rows, p.heads_per_cta), 1);
+  if (c->dtype == FASA_F32)
+    append_kernel<float><<<grid, kAppendThreads, 0, stream>>>(p);
+  else
+    append_kernel<__nv_bfloat16><<<grid, kAppendThreads, 0, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+fasa_status fasa_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
+                       cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 0 || q_pos < 0) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (len == 0) return FASA_OK;
+  if (!aligned(q, 16) || !aligned(scores, 4)) return FASA_ERR_INVALID_ARG;
+  return launch_score(c, len, q, q_pos, scores, stream);
+}
+
+fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, int32_t k, int32_t* idx,
+                             cudaStream_t stream) {
+  if (!aligned(scores, 4) || !aligned(idx, 4)) return FASA_ERR_INVALID_ARG;
+  if (n_rows < 1 || len < 1 || k < 1) return FASA_ERR_INVALID_ARG;
+  if (len > FASA_MAX_LEN || k > FASA_MAX_K || n_rows > 65535) return FASA_ERR_UNSUPPORTED;
+  SAParams p{};
+  p.scores = scores;
+  p.idx_out = idx;
+  p.len = len;
+  p.n_keep = std::min(k, len);
+  p.group = 1;
+  return launch_sa<kSelect>(nullptr, p, n_rows, false, stream, FASA_F32);
+}
+
+fasa_status fasa_sparse_attend(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos,
+                               const int32_t* idx, int32_t n_idx, void* out, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || q_pos < 0 || n_idx < 1) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (n_idx > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(idx, 4)) return FASA_ERR_INVALID_ARG;
+  SAParams p{};
+  p.idx_in = idx;
+  p.k = c->k;
+  p.v = c->v;
+  p.q = q;
+  p.out = out;
+  p.max_len = c->max_len;
+  p.len = len;
+  p.n_keep = n_idx;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.q_pos = q_pos;
+  return launch_sa<kAttendIdx>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype);
+}
+
+size_t fasa_decode_workspace_bytes(const fasa_cache* c, int32_t len) {
+  if (check_cache(c) != FASA_OK || len < 0) return 0;
+  return decode_ws(c, len);
+}
+
+fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k, void* out,
+                        int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (len > FASA_MAX_LEN || k > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  if (idx_out != nullptr && !aligned(idx_out, 4)) return FASA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < decode_ws(c, len))
+    return FASA_ERR_WORKSPACE;
+  float* scores = static_cast<float*>(workspace);
+  if ((s = launch_score(c, len, q, q_pos, scores, stream)) != FASA_OK) return s;
+  SAParams p{};
+  p.scores = scores;
+  p.idx_out = idx_out;
+  p.k = c->k;
+  p.v = c->v;
+  p.q = q;
+  p.out = out;
+  p.max_len = c->max_len;
+  p.len = len;
+  p.n_keep = std::min(k, len);
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.q_pos = q_pos;
+  return launch_sa<kDecode>(c, p, c->batch * c->n_kv_heads, true, stream, c->dtype);
+}
+
+fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, void* out,
+                              cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || q_pos < 0) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  SAParams p{};
+  p.k = c->k;
+  p.v = c->v;
+  p.q = q;
+  p.out = out;
+  p.max_len = c->max_len;
+  p.len = len;
+  p.n_keep = len;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.q_pos = q_pos;
+  return launch_sa<kDense>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype);
+}
+
+fasa_status fasa_device_status(int32_t clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FASA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return FASA_ERR_CUDA;
+  if (clear && v != 0) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_status, &z, sizeof(z)) != cudaSuccess) return FASA_ERR_CUDA;
+  }
+  return v == 0 ? FASA_OK : (fasa_status)v;
+}
+
+}  // extern "C"

@@ -1,0 +1,232 @@
+"""Python binding of the FASA C ABI (include/fasa.h): argument marshalling only.
+
+Every call passes device pointers, sizes and the current CUDA stream to
+libfasa.so; all arithmetic runs in the library's kernels. torch provides the
+device memory and the stream. There is no fallback: if the library is missing
+or a call fails, a FasaError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfasa.so")
+
+FASA_F32, FASA_BF16 = 0, 1
+HEAD_DIM = 128
+STATUS = {0: "FASA_OK", 1: "FASA_ERR_INVALID_ARG", 2: "FASA_ERR_UNSUPPORTED", 3: "FASA_ERR_CAPACITY",
+          4: "FASA_ERR_WORKSPACE", 5: "FASA_ERR_CUDA", 6: "FASA_ERR_TIMEOUT", 7: "FASA_ERR_BAD_INDEX"}
+
+_TORCH_DTYPE = {FASA_F32: torch.float32, FASA_BF16: torch.bfloat16}
+_DTYPE_CODE = {"f32": FASA_F32, "bf16": FASA_BF16, torch.float32: FASA_F32, torch.bfloat16: FASA_BF16}
+
+
+class FasaError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        super().__init__(f"{call}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class fasa_cache(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("n_dom", ctypes.c_int32), ("max_len", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("sketch_stride", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("sketch", ctypes.c_void_p),
+                ("dom_idx", ctypes.c_void_p)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_CP = ctypes.POINTER(fasa_cache)
+
+_SIGS = {
+    "fasa_abi_version": (_I, []),
+    "fasa_status_string": (ctypes.c_char_p, [_I]),
+    "fasa_sketch_stride": (_I, [_I, _I]),
+    "fasa_check_dom_idx": (_I, [_P, _I, _I]),
+    "fasa_append_kv": (_I, [_CP, _P, _P, _I, _I, _P]),
+    "fasa_score": (_I, [_CP, _I, _P, _I, _P, _P]),
+    "fasa_select_topk": (_I, [_P, _I, _I, _I, _P, _P]),
+    "fasa_sparse_attend": (_I, [_CP, _I, _P, _I, _P, _I, _P, _P]),
+    "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
+    "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
+    "fasa_device_status": (_I, [_I]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfasa.so (built in-tree by rope_frequency_chunk_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FasaError(5, f"libfasa.so not found at {LIB_PATH}; build it with "
+                               "`python -m rope_frequency_chunk_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, call: str):
+    if status != 0:
+        raise FasaError(status, call)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+# ------------------------------------------------------------------ cache
+
+def fasa_sketch_stride(n_dom: int, dtype) -> int:
+    return int(lib().fasa_sketch_stride(n_dom, _DTYPE_CODE[dtype]))
+
+
+def fasa_check_dom_idx(dom_idx_host) -> None:
+    import numpy as np
+    a = np.ascontiguousarray(dom_idx_host, dtype=np.int32)
+    _check(lib().fasa_check_dom_idx(a.ctypes.data, a.shape[0], a.shape[1]), "fasa_check_dom_idx")
+
+
+class KVCache:
+    """A layer's KV cache and dominant-FC key sketch, in caller-owned device memory."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, n_dom, max_len, dtype, rope_base, dom_idx,
+                 device="cuda"):
+        code = _DTYPE_CODE[dtype]
+        tdt = _TORCH_DTYPE[code]
+        stride = fasa_sketch_stride(n_dom, code)
+        if stride < 0:
+            raise FasaError(1, "fasa_sketch_stride")
+        fasa_check_dom_idx(dom_idx)
+        self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
+        self.n_dom, self.max_len, self.dtype, self.rope_base = n_dom, max_len, tdt, float(rope_base)
+        self.k = torch.empty(batch, n_kv_heads, max_len, HEAD_DIM, dtype=tdt, device=device)
+        self.v = torch.empty_like(self.k)
+        self.sketch = torch.empty(batch, n_kv_heads, max_len, stride, dtype=tdt, device=device)
+        self.dom_idx = torch.as_tensor(dom_idx, dtype=torch.int32).to(device).contiguous()
+        self.struct = fasa_cache(batch, n_q_heads, n_kv_heads, HEAD_DIM, n_dom, max_len, code, stride,
+                                 float(rope_base), self.k.data_ptr(), self.v.data_ptr(),
+                                 self.sketch.data_ptr(), self.dom_idx.data_ptr())
+        self.sketch_stride = stride
+
+    @property
+    def group(self):
+        return self.n_q_heads // self.n_kv_heads
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+# ------------------------------------------------------------------ calls
+
+def fasa_append_kv(cache: KVCache, k_new, v_new, pos0: int, stream=None) -> None:
+    _dev(k_new, "k_new", cache.dtype)
+    _dev(v_new, "v_new", cache.dtype)
+    n_new = k_new.shape[2]
+    if tuple(k_new.shape) != (cache.batch, cache.n_kv_heads, n_new, HEAD_DIM) or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new must be [B, Hkv, n_new, 128]")
+    _check(lib().fasa_append_kv(cache.ref(), k_new.data_ptr(), v_new.data_ptr(), n_new, pos0,
+                                _stream(stream)), "fasa_append_kv")
+
+
+def _q(cache, q):
+    _dev(q, "q", cache.dtype)
+    if tuple(q.shape) != (cache.batch, cache.n_q_heads, HEAD_DIM):
+        raise ValueError("q must be [B, Hq, 128]")
+    return q
+
+
+def fasa_score(cache: KVCache, length: int, q, q_pos: int, scores=None, stream=None):
+    _q(cache, q)
+    if scores is None:
+        scores = torch.empty(cache.batch, cache.n_kv_heads, length, dtype=torch.float32, device=q.device)
+    _dev(scores, "scores", torch.float32)
+    _check(lib().fasa_score(cache.ref(), length, q.data_ptr(), q_pos, scores.data_ptr(), _stream(stream)),
+           "fasa_score")
+    return scores
+
+
+def fasa_select_topk(scores, k: int, idx=None, stream=None):
+    _dev(scores, "scores", torch.float32)
+    length = scores.shape[-1]
+    rows = scores.numel() // max(length, 1)
+    k_eff = min(k, length)
+    if idx is None:
+        idx = torch.empty(*scores.shape[:-1], k_eff, dtype=torch.int32, device=scores.device)
+    _dev(idx, "idx", torch.int32)
+    _check(lib().fasa_select_topk(scores.data_ptr(), rows, length, k, idx.data_ptr(), _stream(stream)),
+           "fasa_select_topk")
+    return idx
+
+
+def fasa_sparse_attend(cache: KVCache, length: int, q, q_pos: int, idx, out=None, stream=None):
+    _q(cache, q)
+    _dev(idx, "idx", torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    _check(lib().fasa_sparse_attend(cache.ref(), length, q.data_ptr(), q_pos, idx.data_ptr(), idx.shape[-1],
+                                    out.data_ptr(), _stream(stream)), "fasa_sparse_attend")
+    return out
+
+
+def fasa_decode_workspace_bytes(cache: KVCache, length: int) -> int:
+    return int(lib().fasa_decode_workspace_bytes(cache.ref(), length))
+
+
+def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, idx_out=None,
+                workspace=None, stream=None):
+    """One FASA decode step; returns out (and fills idx_out when given)."""
+    _q(cache, q)
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    if idx_out is not None:
+        _dev(idx_out, "idx_out", torch.int32)
+    need = fasa_decode_workspace_bytes(cache, length)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_decode(cache.ref(), length, q.data_ptr(), q_pos, k, out.data_ptr(), _ptr(idx_out),
+                             workspace.data_ptr(), workspace.numel(), _stream(stream)), "fasa_decode")
+    return out
+
+
+def fasa_dense_decode(cache: KVCache, length: int, q, q_pos: int, out=None, stream=None):
+    _q(cache, q)
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    _check(lib().fasa_dense_decode(cache.ref(), length, q.data_ptr(), q_pos, out.data_ptr(), _stream(stream)),
+           "fasa_dense_decode")
+    return out
+
+
+def fasa_device_status(clear: bool = True) -> int:
+    """Synchronizes; returns the device status word (0 = OK)."""
+    return int(lib().fasa_device_status(1 if clear else 0))

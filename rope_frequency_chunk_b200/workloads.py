@@ -247,3 +247,24 @@ def layer_inputs(wl: Workload, layer: int = 0, n_dom: int | None = None,
     with ThreadPoolExecutor(_threads()) as ex:
         list(ex.map(work, range(B * H)))
     return LayerInputs(lp, q, k, v)
+
+
+def to_torch(a: np.ndarray, device="cpu"):
+    """Stored array (float32, or uint16 bf16 bits) -> torch tensor of the cache dtype."""
+    import torch
+
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.to(device)
+
+
+def from_torch(t) -> np.ndarray:
+    """torch tensor (float32 or bfloat16) -> stored numpy array (float32 or uint16 bits)."""
+    import torch
+
+    t = t.detach().to("cpu").contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16).copy()
+    return t.numpy().copy()

@@ -1,0 +1,102 @@
+"""The C-ABI library: it loads, exports every symbol the header declares, and
+rejects bad arguments on the host (no GPU needed: nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rope_frequency_chunk_b200 import fasa as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fasa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from rope_frequency_chunk_b200 import build
+    build.build()
+    return F.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fasa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["fasa_append_kv", "fasa_score", "fasa_select_topk", "fasa_sparse_attend", "fasa_decode",
+                 "fasa_dense_decode", "fasa_decode_workspace_bytes", "fasa_device_status"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing
+
+
+def test_version_and_strings(L):
+    assert L.fasa_abi_version() == 1
+    assert F.lib().fasa_status_string(0) == b"FASA_OK"
+    assert F.lib().fasa_status_string(7) == b"FASA_ERR_BAD_INDEX"
+    assert F.lib().fasa_status_string(99) == b"FASA_ERR_UNKNOWN"
+
+
+def test_sketch_stride(L):
+    s = F.fasa_sketch_stride
+    assert [s(n, "bf16") for n in (1, 4, 5, 8, 16, 32, 64)] == [8, 8, 16, 16, 32, 64, 128]
+    assert [s(n, "f32") for n in (1, 2, 3, 16, 64)] == [4, 4, 8, 32, 128]
+    assert s(0, "bf16") == -1 and s(65, "bf16") == -1
+    assert L.fasa_sketch_stride(16, 7) == -1
+
+
+def test_check_dom_idx(L):
+    F.fasa_check_dom_idx([[0, 5, 63], [1, 2, 3]])
+    for bad in ([[0, 0, 1]], [[0, 64, 1]], [[-1, 2, 3]]):
+        with pytest.raises(F.FasaError):
+            F.fasa_check_dom_idx(bad)
+
+
+def _fake_cache(**kw):
+    c = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, n_dom=16, max_len=1024, dtype=1,
+             sketch_stride=32, rope_base=1e4, k=0x10000, v=0x20000, sketch=0x30000, dom_idx=0x40000)
+    c.update(kw)
+    return F.fasa_cache(**c)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, 2), ("dtype", 3, 2), ("n_q_heads", 3, 1), ("n_q_heads", 64, 2), ("n_dom", 0, 1),
+    ("sketch_stride", 16, 1), ("max_len", 0, 1), ("rope_base", 1.0, 1), ("k", 0x10008, 1), ("v", 0, 1),
+])
+def test_cache_validation(L, field, value, status):
+    c = _fake_cache(**{field: value})
+    st = L.fasa_score(ctypes.byref(c), 10, 0x50000, 10, 0x60000, None)
+    assert st == status
+
+
+def test_call_validation_without_launch(L):
+    c = ctypes.byref(_fake_cache())
+    assert L.fasa_append_kv(c, 0x50000, 0x60000, 10, 1020, None) == 3          # beyond max_len
+    assert L.fasa_append_kv(c, 0x50000, 0x60000, 0, 5, None) == 0              # no-op
+    assert L.fasa_append_kv(c, 0x50008, 0x60000, 4, 0, None) == 1              # misaligned input
+    assert L.fasa_score(c, 2000, 0x50000, 0, 0x60000, None) == 3               # len > max_len
+    assert L.fasa_score(c, 0, 0x50000, 0, 0x60000, None) == 0                  # empty
+    assert L.fasa_select_topk(None, 1, 10, 2, 0x60000, None) == 1
+    assert L.fasa_select_topk(0x50000, 1, 10, 0, 0x60000, None) == 1           # k < 1
+    assert L.fasa_select_topk(0x50000, 1, (1 << 19) + 1, 5, 0x60000, None) == 2
+    assert L.fasa_sparse_attend(c, 10, 0x50000, 10, 0x60000, 0, 0x70000, None) == 1   # n_idx < 1
+    assert L.fasa_decode(c, 0, 0x50000, 0, 8, 0x70000, None, 0x80000, 1 << 20, None) == 1
+    assert L.fasa_decode(c, 100, 0x50000, 100, 8, 0x70000, None, None, 1 << 20, None) == 4
+    need = L.fasa_decode_workspace_bytes(c, 100)
+    assert need >= 2 * 100 * 4
+    assert L.fasa_decode(c, 100, 0x50000, 100, 8, 0x70000, None, 0x80000, need - 1, None) == 4
+    assert L.fasa_dense_decode(c, 0, 0x50000, 0, 0x70000, None) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(F, "_lib", None)
+    monkeypatch.setattr(F, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(F.FasaError):
+        F.lib()

@@ -1,0 +1,304 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle, through the C ABI.
+
+Stages are checked both alone (each fed the GPU's own output of the previous
+stage) and fused (fasa_decode). Small cases span several tiles with ragged
+tails; the full workload sizes are checked on sampled heads.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.fasa_oracle as O
+from rope_frequency_chunk_b200 import fasa as F
+from rope_frequency_chunk_b200 import workloads as W
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+C = W.CONFIGS
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    F.fasa_device_status(clear=True)
+    yield
+    assert F.fasa_device_status(clear=True) == 0
+
+
+# small variants: ragged lengths, every group size and n_dom family
+SMALL = {
+    "c1": C["c1"],
+    "c2_ragged": C["c2"].replace(ctx_len=5003),
+    "c4_g7": C["c4"].replace(ctx_len=3001, batch=2, k=567, n_dom=8),
+    "g16_f32": C["c1"].replace(name="g16", n_q_heads=32, n_kv_heads=2, ctx_len=1500, n_dom=5, k=100),
+    "g1_bf16_ndom64": C["c2"].replace(name="g1", n_q_heads=3, n_kv_heads=3, ctx_len=777, n_dom=64, k=64),
+    "bf16_ndom1": C["c2"].replace(name="nd1", batch=2, n_q_heads=8, n_kv_heads=2, ctx_len=2049, n_dom=1, k=31),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_append_matches_oracle(name):
+    wl = SMALL[name]
+    inp, cache, q = U.build(wl, chunks=None)
+    U.check_append(wl, inp, cache, U.all_heads(wl))
+
+
+def test_append_in_ragged_chunks_equals_one_shot():
+    wl = SMALL["c2_ragged"]
+    inp = W.layer_inputs(wl)
+    _, a, _ = U.build(wl, inp=inp)
+    _, b, _ = U.build(wl, inp=inp, chunks=[1, 2, 1000, 7, 3993], max_len=6000)
+    L = wl.ctx_len
+    assert torch.equal(a.k[:, :, :L], b.k[:, :, :L]) and torch.equal(a.v[:, :, :L], b.v[:, :, :L])
+    assert torch.equal(a.sketch[:, :, :L], b.sketch[:, :, :L])
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_score_matches_oracle(name):
+    wl = SMALL[name]
+    inp, cache, q = U.build(wl)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    for (b, g) in U.all_heads(wl):
+        _, ref, abs_sum = U.oracle_scores(wl, inp, cache, b, g)
+        U.check_scores(s[b, g], ref, abs_sum)
+
+
+def _select_cases():
+    r = np.random.default_rng(7)
+    cases = []
+    for rows, L, k in [(1, 1, 1), (1, 7, 3), (3, 100, 100), (3, 100, 250), (2, 4096, 256), (5, 40001, 1),
+                       (4, 40001, 5000), (1, 300000, 2048), (64, 16384, 1024), (2, 2 ** 19, 9000)]:
+        s = r.standard_normal((rows, L)).astype(np.float32)
+        cases.append((f"normal_{rows}x{L}_k{k}", s, k))
+    ties = r.integers(-3, 3, (3, 20000)).astype(np.float32)
+    ties[0, :50] = -0.0
+    ties[0, 50:100] = 0.0
+    cases.append(("many_ties", ties, 777))
+    cases.append(("all_equal", np.full((2, 5000), 1.5, np.float32), 300))
+    cases.append(("zeros_signed", np.where(r.random((1, 3000)) < 0.5, -0.0, 0.0).astype(np.float32), 10))
+    neg = -np.abs(r.standard_normal((2, 9999))).astype(np.float32)
+    cases.append(("all_negative", neg, 4000))
+    return cases
+
+
+@pytest.mark.parametrize("name,scores,k", _select_cases(), ids=[c[0] for c in _select_cases()])
+def test_select_is_exact(name, scores, k):
+    idx = F.fasa_select_topk(torch.from_numpy(scores).cuda(), k).cpu().numpy()
+    for r in range(scores.shape[0]):
+        want = O.select_critical_set(scores[r].astype(np.float64), k)
+        assert np.array_equal(idx[r], want), name
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_sparse_attend_matches_oracle(name):
+    wl = SMALL[name]
+    inp, cache, q = U.build(wl)
+    r = np.random.default_rng(3)
+    n_idx = min(wl.k, wl.ctx_len)
+    idx = np.stack([np.stack([r.choice(wl.ctx_len, n_idx, replace=False) for _ in range(wl.n_kv_heads)])
+                    for _ in range(wl.batch)]).astype(np.int32)
+    idx[0, 0, :3] = idx[0, 0, 0]  # duplicates count twice; order is free
+    out = F.fasa_sparse_attend(cache, wl.ctx_len, q, wl.q_pos, torch.from_numpy(idx).cuda())
+    out_np = U.stored(out)
+    G = wl.group
+    for (b, g) in U.all_heads(wl):
+        q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos, wl.rope_base)
+        ref = O.focused_attention(q_rot, U.stored(cache.k[b, g]), U.stored(cache.v[b, g]), idx[b, g])
+        U.check_out(wl, out_np[b, g * G:(g + 1) * G], ref)
+
+
+def test_sparse_attend_skips_bad_index():
+    wl = SMALL["c2_ragged"]
+    inp, cache, q = U.build(wl)
+    idx = np.tile(np.arange(0, 40, dtype=np.int32), (1, wl.n_kv_heads, 1))
+    idx[0, 1, 5] = wl.ctx_len        # out of range -> skipped, status recorded
+    idx[0, 2, 7] = -3
+    out = F.fasa_sparse_attend(cache, wl.ctx_len, q, wl.q_pos, torch.from_numpy(idx).cuda())
+    assert F.fasa_device_status(clear=True) == 7
+    G = wl.group
+    for g in (1, 2):
+        keep = [t for t in idx[0, g] if 0 <= t < wl.ctx_len]
+        q_rot = O.rotate_queries(inp.q[0, g * G:(g + 1) * G], wl.q_pos, wl.rope_base)
+        ref = O.focused_attention(q_rot, U.stored(cache.k[0, g]), U.stored(cache.v[0, g]), keep)
+        U.check_out(wl, U.stored(out)[0, g * G:(g + 1) * G], ref)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_dense_matches_oracle(name):
+    wl = SMALL[name]
+    inp, cache, q = U.build(wl)
+    out = U.stored(F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos))
+    G = wl.group
+    for (b, g) in U.all_heads(wl):
+        q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos, wl.rope_base)
+        ref = O.dense_attention(q_rot, U.stored(cache.k[b, g]), U.stored(cache.v[b, g]))
+        U.check_out(wl, out[b, g * G:(g + 1) * G], ref)
+
+
+def _decode(wl, cache, q, k, length=None):
+    L = length or wl.ctx_len
+    idx = torch.empty(wl.batch, wl.n_kv_heads, min(k, L), dtype=torch.int32, device="cuda")
+    out = F.fasa_decode(cache, L, q, L, k, idx_out=idx)
+    return out, idx
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_matches_oracle(name):
+    wl = SMALL[name]
+    inp, cache, q = U.build(wl)
+    out, idx = _decode(wl, cache, q, wl.k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
+
+
+@pytest.mark.parametrize("k_of_L", ["one", "equal", "more", "half"])
+def test_decode_budget_edges(k_of_L):
+    wl = SMALL["c2_ragged"].replace(ctx_len=1999)
+    L = wl.ctx_len
+    k = {"one": 1, "equal": L, "more": L + 500, "half": L // 2}[k_of_L]
+    inp, cache, q = U.build(wl)
+    out, idx = _decode(wl, cache, q, k)
+    U.check_decode_heads(wl, inp, cache, q, k, U.all_heads(wl), out, idx)
+    if k >= L:  # keeping every token is dense attention
+        dense = F.fasa_dense_decode(cache, L, q, L)
+        assert np.max(np.abs(W.stored_to_f64(U.stored(out)) - W.stored_to_f64(U.stored(dense)))) <= 2e-2
+
+
+def test_decode_single_token_cache():
+    wl = C["c2"].replace(ctx_len=1, batch=2)
+    inp, cache, q = U.build(wl)
+    out, idx = _decode(wl, cache, q, 256)
+    assert idx.cpu().numpy().ravel().tolist() == [0] * (2 * 8)
+    U.check_decode_heads(wl, inp, cache, q, 256, U.all_heads(wl), out, idx)
+
+
+def test_decode_all_fc_full_budget_is_dense():
+    """With every FC dominant and k = L, FASA is dense attention."""
+    wl = C["c2"].replace(ctx_len=3000, n_dom=64, k=3000)
+    inp, cache, q = U.build(wl)
+    out, idx = _decode(wl, cache, q, wl.k)
+    dense = F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos)
+    d = np.abs(W.stored_to_f64(U.stored(out)) - W.stored_to_f64(U.stored(dense)))
+    assert d.max() <= 2e-2
+
+
+def test_decode_with_tied_tokens():
+    """Tokens whose dominant dims are zero all score exactly 0; the budget is
+    placed inside that tie, so ties must go to the lower index."""
+    wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=4000)
+    inp = W.layer_inputs(wl)
+    dom = inp.params.dom_idx[0]
+    cols = np.concatenate([dom, dom + 64])
+    for c in cols:
+        inp.k[0, 0, 1000:3000, c] = 0          # +0.0
+    _, cache, q = U.build(wl, inp=inp)
+    _, s_ref, _ = U.oracle_scores(wl, inp, cache, 0, 0)
+    assert np.sum(s_ref == 0) >= 2000
+    k = int(np.sum(s_ref > 0)) + 37
+    out, idx = _decode(wl, cache, q, k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, k, [(0, 0)], out, idx, scores_gpu=s)
+    kept_zero = [t for t in idx.cpu().numpy()[0, 0] if s_ref[t] == 0]
+    assert kept_zero == list(range(1000, 1037))
+
+
+def test_decode_is_deterministic_and_capturable():
+    wl = SMALL["c2_ragged"]
+    inp, cache, q = U.build(wl)
+    ws = torch.empty(F.fasa_decode_workspace_bytes(cache, wl.ctx_len), dtype=torch.uint8, device="cuda")
+    out1 = torch.empty_like(q)
+    F.fasa_decode(cache, wl.ctx_len, q, wl.q_pos, wl.k, out=out1, workspace=ws)
+    s = torch.cuda.Stream()
+    out2 = torch.empty_like(q)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        F.fasa_decode(cache, wl.ctx_len, q, wl.q_pos, wl.k, out=out2, workspace=ws)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+# ------------------------------------------------------------ full sizes
+
+def test_full_c1():
+    wl = C["c1"]
+    inp, cache, q = U.build(wl)
+    U.check_append(wl, inp, cache, U.all_heads(wl))
+    out, idx = _decode(wl, cache, q, wl.k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
+
+
+def test_full_c2():
+    wl = C["c2"]
+    inp, cache, q = U.build(wl)
+    U.check_append(wl, inp, cache, U.sample_heads(wl, 2))
+    out, idx = _decode(wl, cache, q, wl.k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
+    dense = U.stored(F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos))
+    G = wl.group
+    for (b, g) in U.sample_heads(wl, 2, seed=1):
+        q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos, wl.rope_base)
+        ref = O.dense_attention(q_rot, U.stored(cache.k[b, g]), U.stored(cache.v[b, g]))
+        U.check_out(wl, dense[b, g * G:(g + 1) * G], ref)
+
+
+def test_full_c3_sampled():
+    wl = C["c3"]
+    inp, cache, q = U.build(wl)
+    heads = U.sample_heads(wl, 3)
+    U.check_append(wl, inp, cache, heads[:1])
+    out, idx = _decode(wl, cache, q, wl.k)
+    U.check_decode_heads(wl, inp, cache, q, wl.k, heads, out, idx)
+
+
+@pytest.fixture(scope="module")
+def c5_state():
+    state = U.build(C["c5"])
+    yield state
+    del state
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("k", W.C5_KS)
+def test_full_c5_sampled(k, c5_state):
+    wl = C["c5"]
+    inp, cache, q = c5_state
+    out, idx = _decode(wl, cache, q, k)
+    U.check_decode_heads(wl, inp, cache, q, k, U.sample_heads(wl, 3, seed=k), out, idx)
+    if k == W.C5_KS[-1]:
+        dense = U.stored(F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos))
+        G = wl.group
+        for (b, g) in U.sample_heads(wl, 2, seed=5):
+            q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos, wl.rope_base)
+            ref = O.dense_attention(q_rot, U.stored(cache.k[b, g]), U.stored(cache.v[b, g]))
+            U.check_out(wl, dense[b, g * G:(g + 1) * G], ref)
+
+
+@pytest.mark.parametrize("n_dom", W.C4_NDOMS)
+def test_full_c4_sweep_sampled(n_dom):
+    """Long-CoT sweep: 1K appends up to 32K; decode with k = 18.9% of L at several steps."""
+    wl = C["c4"]
+    inp = W.layer_inputs(wl, n_dom=n_dom)
+    lp = inp.params
+    cache = F.KVCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, n_dom, wl.ctx_len, wl.dtype, wl.rope_base,
+                      lp.dom_idx)
+    k_all = W.to_torch(inp.k, "cuda")
+    v_all = W.to_torch(inp.v, "cuda")
+    heads = U.sample_heads(wl, 2, seed=n_dom)
+    for step in range(W.C4_STEPS):
+        c0 = step * W.C4_APPEND_CHUNK
+        c1 = c0 + W.C4_APPEND_CHUNK
+        F.fasa_append_kv(cache, k_all[:, :, c0:c1].contiguous(), v_all[:, :, c0:c1].contiguous(), c0)
+        L = c1
+        if step in (0, 7, W.C4_STEPS - 1):
+            k = W.c4_budget(L)
+            q_np = np.stack([np.concatenate([W.head_q(wl, lp, 0, b, g, step=step) for g in range(wl.n_kv_heads)])
+                             for b in range(wl.batch)])
+            q = W.to_torch(q_np, "cuda")
+            sub = W.LayerInputs(lp, q_np, inp.k, inp.v)
+            out, idx = _decode(wl, cache, q, k, length=L)
+            U.check_decode_heads(wl, sub, cache, q, k, heads, out, idx, length=L)
+    U.check_append(wl, inp, cache, heads[:1])
