@@ -1,0 +1,407 @@
+"""Benchmark of the FASA decode hot path on B200 (prints one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--layers 32]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+A step is one FASA decode (fasa_decode: TIP score -> top-k -> focused
+attention) of every layer of a stack of independent layer caches, each
+holding the configuration's synthetic KV cache and dominant-FC sketch. The
+stack is larger than L2, so every layer's data comes from HBM. Steps are
+replayed from one CUDA graph. `value` is achieved HBM GB/s on the algorithmic
+(roofline) bytes: sketch of every cached token + K/V rows of the kept tokens +
+query and output. Multi-GPU runs are independent replicas (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rope_frequency_chunk_b200 import workloads as W  # noqa: E402
+
+METRIC = "fasa_decode µs/layer-step and achieved HBM GB/s vs peak (32K ctx, k=256)"
+L2_BYTES = 126 * 2 ** 20
+
+
+def roofline_bytes(wl: W.Workload, k: int | None = None, n_dom: int | None = None) -> int:
+    """Algorithmic bytes of one decode layer-step (sketch + kept K/V rows + q/out)."""
+    k = wl.k if k is None else k
+    n_dom = wl.n_dom if n_dom is None else n_dom
+    es = wl.elem_bytes
+    k_eff = min(k, wl.ctx_len)
+    sketch = wl.batch * wl.n_kv_heads * wl.ctx_len * 2 * n_dom * es
+    rows = wl.batch * wl.n_kv_heads * k_eff * 2 * W.HEAD_DIM * es
+    qo = 2 * wl.batch * wl.n_q_heads * W.HEAD_DIM * es
+    return sketch + rows + qo
+
+
+def sketch_bytes(wl: W.Workload) -> int:
+    return wl.batch * wl.n_kv_heads * wl.ctx_len * 2 * wl.n_dom * wl.elem_bytes
+
+
+def dense_bytes(wl: W.Workload) -> int:
+    es = wl.elem_bytes
+    return (wl.batch * wl.n_kv_heads * wl.ctx_len * 2 * W.HEAD_DIM * es
+            + 2 * wl.batch * wl.n_q_heads * W.HEAD_DIM * es)
+
+
+def default_layers(wl: W.Workload) -> int:
+    per_layer = roofline_bytes(wl)
+    n = 32 if wl.name in ("c1", "c2", "c4") else 2
+    while n * per_layer < 3 * L2_BYTES and n < 4096:
+        n *= 2
+    return n
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.25)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- oracle leg
+
+def oracle_units(wl: W.Workload, n: int):
+    """Prepare n distinct (layer, b, g) units for the oracle (untimed): inputs
+    from the generator, cache contents from the oracle's own append."""
+    import oracle.fasa_oracle as O
+    units = []
+    for u in range(n):
+        layer, rem = divmod(u, wl.batch * wl.n_kv_heads)
+        b, g = divmod(rem, wl.n_kv_heads)
+        lp = W.layer_params(wl, layer)
+        kk, vv = W.head_kv(wl, lp, layer, b, g)
+        qq = W.head_q(wl, lp, layer, b, g)
+        k_rot, v_st, sk = O.append_kv(kk, vv, 0, wl.rope_base, lp.dom_idx[g], wl.dtype)
+        units.append((qq, k_rot, v_st, sk, lp.dom_idx[g]))
+    return units
+
+
+def oracle_time(wl: W.Workload, units, k: int, budget_s: float = 0.0, calls: int | None = None):
+    """Time oracle decodes (one KV head each), cycling over prepared units,
+    single-threaded; returns (roofline bytes processed, seconds, calls)."""
+    import oracle.fasa_oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    per_unit = roofline_bytes(wl, k) / (wl.batch * wl.n_kv_heads)
+    done, spent = 0, 0.0
+    while (calls is None and spent < budget_s) or (calls is not None and done < calls):
+        qq, k_rot, v_st, sk, dom = units[done % len(units)]
+        t0 = time.perf_counter()
+        O.decode_head(qq, wl.q_pos, k_rot, v_st, sk, dom, k, wl.rope_base)
+        spent += time.perf_counter() - t0
+        done += 1
+    if limiter is not None:
+        limiter.unregister()
+    return per_unit * done, spent, done
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    k = args.k or wl.k
+    units = oracle_units(wl, min(4, wl.batch * wl.n_kv_heads))
+    oracle_time(wl, units, k, calls=args.warmup)
+    total_b, total_t, steps = 0.0, 0.0, 0
+    deadline = time.time() + 150.0
+    for _ in range(args.steps):
+        b, t, _ = oracle_time(wl, units, k, calls=1)
+        total_b += b
+        total_t += t
+        steps += 1
+        if time.time() > deadline:
+            break
+    gbs = total_b / total_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "ctx_len": wl.ctx_len, "k": k, "n_dom": wl.n_dom,
+                   "heads": f"{wl.n_q_heads}/{wl.n_kv_heads}"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{steps} steps, each the oracle decode of one (sequence, KV head) of "
+                                   f"{wl.name} (cycling over {len(units)} prepared heads), float64 numpy, 1 thread"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def build_stack(wl, n_layers, device):
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+    caches, qs = [], []
+    for layer in range(n_layers):
+        inp = W.layer_inputs(wl, layer=layer)
+        c = F.KVCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.n_dom, wl.ctx_len, wl.dtype, wl.rope_base,
+                      inp.params.dom_idx, device=device)
+        k = W.to_torch(inp.k, device)
+        v = W.to_torch(inp.v, device)
+        F.fasa_append_kv(c, k, v, 0)
+        del k, v
+        caches.append(c)
+        qs.append(W.to_torch(inp.q, device))
+        del inp
+    torch.cuda.synchronize()
+    return caches, qs
+
+
+def time_graph(fn, steps, warmup, stream, dist=None):
+    """Capture fn() (one step) in a CUDA graph; replay warmup + steps; return
+    device ms for the steps (events on the replay stream), max over ranks."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    torch.cuda.synchronize()
+    del g
+    return ms
+
+
+def run_fasa(args, wl):
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    device = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    F.lib()
+
+    k = args.k or wl.k
+    n_layers = args.layers or default_layers(wl)
+    caches, qs = build_stack(wl, n_layers, device)
+    outs = [torch.empty_like(q) for q in qs]
+    ws = torch.empty(max(F.fasa_decode_workspace_bytes(c, wl.ctx_len) for c in caches), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.Stream(device=device)
+    L = wl.ctx_len
+
+    def decode_step():
+        for c, q, o in zip(caches, qs, outs):
+            F.fasa_decode(c, L, q, wl.q_pos, k, out=o, workspace=ws)
+
+    scores = torch.empty(wl.batch, wl.n_kv_heads, L, dtype=torch.float32, device=device)
+
+    def score_step():
+        for c, q in zip(caches, qs):
+            F.fasa_score(c, L, q, wl.q_pos, scores=scores)
+
+    def dense_step():
+        for c, q, o in zip(caches, qs, outs):
+            F.fasa_dense_decode(c, L, q, wl.q_pos, out=o)
+
+    hbm_peak, peak_kind = peaks()
+    with ClockSampler(local) as clk:
+        ms = time_graph(decode_step, args.steps, args.warmup, stream, dist)
+    clocks = clk.summary()
+    status = F.fasa_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed decode")
+
+    per_layer_bytes = roofline_bytes(wl, k)
+    step_bytes = per_layer_bytes * n_layers
+    ms_step = ms / args.steps
+    us_layer = 1e3 * ms_step / n_layers
+    gbs = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # dominant kernel (TIP score stream), timed alone on the same stack
+    ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
+    score_gbs = sketch_bytes(wl) * n_layers / (ms_score * 1e-3) / 1e9
+
+    extra = {}
+    if not args.no_dense:
+        dsteps = max(3, args.steps // 8)
+        ms_dense = time_graph(dense_step, dsteps, args.warmup, stream, dist) / dsteps
+        extra["dense_us_per_layer_step"] = 1e3 * ms_dense / n_layers
+        extra["dense_gbs"] = dense_bytes(wl) * n_layers / (ms_dense * 1e-3) / 1e9
+        extra["speedup_vs_dense"] = ms_dense / ms_step
+
+    e2e = None
+    if not args.no_e2e:
+        q_host = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in qs]
+        for qh, q in zip(q_host, qs):
+            qh.copy_(q.cpu())
+        o_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+
+        def e2e_step():
+            for qh, q in zip(q_host, qs):
+                q.copy_(qh, non_blocking=True)
+            decode_step()
+            for oh, o in zip(o_host, outs):
+                oh.copy_(o, non_blocking=True)
+
+        esteps = max(3, args.steps // 4)
+        ms_e2e = time_graph(e2e_step, esteps, args.warmup, stream, dist) / esteps
+        h2d = sum(q.numel() * q.element_size() for q in qs)
+        e2e = {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d, "ms_per_step": ms_e2e}
+
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "heads": f"{wl.n_q_heads}/{wl.n_kv_heads}",
+                   "ctx_len": L, "k": k, "n_dom": wl.n_dom, "layers_per_step": n_layers,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2: {n_layers} layer caches "
+                         f"({step_bytes / 2**20:.0f} MiB of roofline bytes per step) stepped in order"},
+        "us_per_layer_step": us_layer,
+        "tokens_per_s": world * wl.batch / (us_layer * 1e-6),
+        "decode_roofline": {"achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": gbs / world / hbm_peak, "bytes_per_layer_step": per_layer_bytes,
+                            "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "score_kernel (TIP sketch stream)", "achieved": score_gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": score_gbs / hbm_peak,
+                     "traffic": None, "bytes_per_launch": sketch_bytes(wl), "peak_kind": peak_kind,
+                     "us_per_launch": 1e3 * ms_score / n_layers},
+        "clocks": clocks,
+        "gpu_launches": 2 * n_layers * args.steps,
+        "e2e": e2e,
+    }
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        units = oracle_units(wl, min(4, wl.batch * wl.n_kv_heads))
+        b, t, calls = oracle_time(wl, units, k, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{calls} oracle decodes of one (sequence, KV head) of {wl.name} each, "
+                                          f"cycling over {len(units)} prepared heads ({t:.1f} s), float64 numpy, "
+                                          f"1 thread"}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fasa", choices=["fasa", "reference"])
+    ap.add_argument("--config", default="c2", choices=sorted(W.CONFIGS))
+    ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--k", type=int, default=0)
+    ap.add_argument("--ctx-len", type=int, default=0)
+    ap.add_argument("--n-dom", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = W.CONFIGS[args.config]
+    if args.ctx_len:
+        wl = wl.replace(ctx_len=args.ctx_len, k=W.c4_budget(args.ctx_len) if wl.name == "c4" else wl.k)
+    if args.n_dom:
+        wl = wl.replace(n_dom=args.n_dom)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_fasa(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

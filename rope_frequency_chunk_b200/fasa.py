@@ -21,7 +21,8 @@ STATUS = {0: "FASA_OK", 1: "FASA_ERR_INVALID_ARG", 2: "FASA_ERR_UNSUPPORTED", 3:
           4: "FASA_ERR_WORKSPACE", 5: "FASA_ERR_CUDA", 6: "FASA_ERR_TIMEOUT", 7: "FASA_ERR_BAD_INDEX"}
 
 _TORCH_DTYPE = {FASA_F32: torch.float32, FASA_BF16: torch.bfloat16}
-_DTYPE_CODE = {"f32": FASA_F32, "bf16": FASA_BF16, torch.float32: FASA_F32, torch.bfloat16: FASA_BF16}
+_DTYPE_CODE = {"f32": FASA_F32, "bf16": FASA_BF16, torch.float32: FASA_F32, torch.bfloat16: FASA_BF16,
+               FASA_F32: FASA_F32, FASA_BF16: FASA_BF16}
 
 
 class FasaError(RuntimeError):

@@ -50,6 +50,7 @@ def test_sketch_stride(L):
     assert [s(n, "f32") for n in (1, 2, 3, 16, 64)] == [4, 4, 8, 32, 128]
     assert s(0, "bf16") == -1 and s(65, "bf16") == -1
     assert L.fasa_sketch_stride(16, 7) == -1
+    assert s(16, F.FASA_BF16) == s(16, "bf16") == s(16, __import__("torch").bfloat16) == 32
 
 
 def test_check_dom_idx(L):

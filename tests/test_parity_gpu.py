@@ -161,7 +161,7 @@ def test_decode_budget_edges(k_of_L):
     U.check_decode_heads(wl, inp, cache, q, k, U.all_heads(wl), out, idx)
     if k >= L:  # keeping every token is dense attention
         dense = F.fasa_dense_decode(cache, L, q, L)
-        assert np.max(np.abs(W.stored_to_f64(U.stored(out)) - W.stored_to_f64(U.stored(dense)))) <= 2e-2
+        assert U.ulp_diff_bf16(U.stored(out), U.stored(dense)).max() <= 1
 
 
 def test_decode_single_token_cache():
@@ -178,8 +178,7 @@ def test_decode_all_fc_full_budget_is_dense():
     inp, cache, q = U.build(wl)
     out, idx = _decode(wl, cache, q, wl.k)
     dense = F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos)
-    d = np.abs(W.stored_to_f64(U.stored(out)) - W.stored_to_f64(U.stored(dense)))
-    assert d.max() <= 2e-2
+    assert U.ulp_diff_bf16(U.stored(out), U.stored(dense)).max() <= 1
 
 
 def test_decode_with_tied_tokens():
