@@ -110,6 +110,10 @@ int32_t fasa_abi_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fasa_status_string(int32_t status);
 
+/* Description of the CUDA error behind the calling thread's most recent
+ * FASA_ERR_CUDA (static string, never NULL; "no error" before any). */
+const char* fasa_last_cuda_error(void);
+
 /* Sketch row length in elements for n_dom dominant FCs: 2*n_dom rounded up
  * so that a row is a power-of-two number of 16-byte chunks (so a 16-byte load
  * never straddles two tokens). Returns -1 for n_dom outside 1..64 or an

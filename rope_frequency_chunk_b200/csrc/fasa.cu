@@ -58,6 +58,17 @@ void fill_theta(double* th, double base) {
   for (int i = 0; i < kNFC; ++i) th[i] = std::pow(base, -2.0 * (double)i / (double)kD);
 }
 
+// cos / sin of the query's rotation angle pos * theta_i, float64 on the host.
+void fill_query_angle(double* cosv, double* sinv, double base, int32_t pos) {
+  double th[kNFC];
+  fill_theta(th, base);
+  for (int i = 0; i < kNFC; ++i) {
+    const double a = (double)pos * th[i];
+    cosv[i] = std::cos(a);
+    sinv[i] = std::sin(a);
+  }
+}
+
 fasa_status check_cache(const fasa_cache* c) {
   if (c == nullptr) return FASA_ERR_INVALID_ARG;
   if (c->head_dim != kD) return FASA_ERR_UNSUPPORTED;
@@ -75,8 +86,11 @@ fasa_status check_cache(const fasa_cache* c) {
   return FASA_OK;
 }
 
+thread_local const char* t_last_cuda_error = "no error";
+
 fasa_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return FASA_OK;
+  t_last_cuda_error = cudaGetErrorString(e);
   (void)cudaGetLastError();  // clear a non-sticky launch error
   return FASA_ERR_CUDA;
 }
@@ -109,15 +123,16 @@ fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
 template <typename T, int LPT>
 fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
   auto kern = score_kernel<T, LPT>;
-  int occ = 0;
-  fasa_status s = cached_int((const void*)kern, 0, &occ, [&](int* v) {
-    return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kern, kScoreThreads, 0));
+  const int smem = kScoreStages * kScoreStageBytes;
+  int set = 0;
+  fasa_status s = cached_int((const void*)kern, 0, &set, [&](int* v) {
+    *v = 1;
+    return cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   });
   if (s != FASA_OK) return s;
-  const int64_t want = (int64_t)d.sms * (occ > 0 ? occ : 1);
   const int64_t cap = ceil_div(p.total, 256);  // at least 256 tokens per CTA
-  const int grid = (int)std::max<int64_t>(1, std::min(want, cap));
-  kern<<<grid, kScoreThreads, 0, st>>>(p);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sms, cap));
+  kern<<<grid, kScoreThreads, smem, st>>>(p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -152,23 +167,25 @@ fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
   p.n_dom = c->n_dom;
-  p.q_pos = q_pos;
-  fill_theta(p.theta, c->rope_base);
+  fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   return c->dtype == FASA_F32 ? launch_score_lpt<float>(p, d, st) : launch_score_lpt<__nv_bfloat16>(p, d, st);
 }
 
 // ---------------------------------------------------- select / attend
 
-struct SAShape {
-  int C, chunk, slice, smem;
-};
+constexpr int kMaxCap = 16384;  // candidate keys per CTA in the sampled selection
 
 inline int maxg_for(int g) { return g <= 4 ? 4 : (g <= 8 ? 8 : 16); }
 
 template <typename T, int MODE, int MAXG>
 fasa_status launch_sa_t(SAParams p, int rows, int C, bool pdl, cudaStream_t st, const DevInfo& d) {
   auto kern = select_attend_kernel<T, MODE, MAXG>;
-  const SALayout L = sa_layout(MODE, (int)sizeof(T), p.chunk, p.slice, MAXG);
+  SALayout L = sa_layout(MODE, (int)sizeof(T), p.chunk, p.slice, p.cap, MAXG, p.n_stages);
+  // a smaller candidate buffer only sends more rows to the exact fallback
+  while (L.total > d.smem_optin && p.cap > 1024) {
+    p.cap /= 2;
+    L = sa_layout(MODE, (int)sizeof(T), p.chunk, p.slice, p.cap, MAXG, p.n_stages);
+  }
   if (L.total > d.smem_optin) return FASA_ERR_UNSUPPORTED;
   int set = 0;
   fasa_status s = cached_int((const void*)kern, 1, &set, [&](int* v) {
@@ -224,22 +241,46 @@ int choose_cluster(int mode, int rows, int64_t len, int64_t keep, int sms) {
   int cmin = 1;
   if (mode == kSelect || mode == kDecode) cmin = std::max(cmin, pow2ceil(ceil_div(len, kMaxChunkKeys)));
   if (mode == kDecode || mode == kAttendIdx) cmin = std::max(cmin, pow2ceil(ceil_div(keep, kMaxSlice)));
-  const int64_t target = (mode == kDense ? 8 : 2) * (int64_t)sms;
+  const int64_t target = (mode == kDense ? 1 : 2) * (int64_t)sms;
   const int cfill = pow2ceil(ceil_div(target, rows));
   return std::max(cmin, std::min(cfill, kMaxCluster));
 }
 
+// Sampling parameters of the selection: stride s (at most kMaxSamples samples
+// per row), rank j of the sample used as threshold (k_eff / s plus four
+// standard deviations and a constant), candidate capacity.
+void choose_sampling(SAParams& p) {
+  const int64_t len = p.len, k = p.n_keep;
+  int s = 8;
+  while (ceil_div(len, s) > kMaxSamples) s <<= 1;
+  const int64_t m = ceil_div(len, s);
+  const int64_t mu = ceil_div(k, s);
+  const int64_t j = mu + (int64_t)std::ceil(4.0 * std::sqrt((double)mu)) + 4;
+  p.sample_stride = s;
+  if (j >= m) {
+    p.sample_rank = (int)m;  // no sampling: every key is a candidate
+    p.cap = (int)std::min<int64_t>(kMaxCap, std::max<int64_t>(1024, pow2ceil(len)));
+  } else {
+    p.sample_rank = (int)j;
+    const int64_t expect = (j + (int64_t)std::ceil(3.0 * std::sqrt((double)j)) + 2) * s;
+    p.cap = (int)std::min<int64_t>(kMaxCap, std::max<int64_t>(1024, pow2ceil(expect)));
+  }
+}
+
 template <int MODE>
-fasa_status launch_sa(const fasa_cache* c, SAParams p, int rows, bool pdl, cudaStream_t st, int dtype) {
+fasa_status launch_sa(const fasa_cache* c, SAParams p, int rows, bool pdl, cudaStream_t st, int dtype,
+                      int32_t q_pos) {
   DevInfo d;
   fasa_status s = device_info(&d);
   if (s != FASA_OK) return s;
   int C = choose_cluster(MODE, rows, p.len, p.n_keep, d.sms);
   if (C > kMaxCluster) return FASA_ERR_UNSUPPORTED;
+  if (c) fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
+  if (MODE == kSelect || MODE == kDecode) choose_sampling(p);
+  p.n_stages = 4;
   for (;;) {
     p.chunk = (int)ceil_div(p.len, C);
     p.slice = (int)ceil_div(p.n_keep, C);
-    if (c) fill_theta(p.theta, c->rope_base);
     if constexpr (MODE == kSelect) {
       s = launch_sa_t<float, MODE, 4>(p, rows, C, pdl, st, d);
     } else {
@@ -272,6 +313,8 @@ size_t decode_ws(const fasa_cache* c, int32_t len) {
 extern "C" {
 
 int32_t fasa_abi_version(void) { return FASA_ABI_VERSION; }
+
+const char* fasa_last_cuda_error(void) { return t_last_cuda_error; }
 
 const char* fasa_status_string(int32_t s) {
   switch (s) {
@@ -366,7 +409,7 @@ fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, i
   p.len = len;
   p.n_keep = std::min(k, len);
   p.group = 1;
-  return launch_sa<kSelect>(nullptr, p, n_rows, false, stream, FASA_F32);
+  return launch_sa<kSelect>(nullptr, p, n_rows, false, stream, FASA_F32, 0);
 }
 
 fasa_status fasa_sparse_attend(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos,
@@ -388,8 +431,7 @@ fasa_status fasa_sparse_attend(const fasa_cache* c, int32_t len, const void* q, 
   p.n_keep = n_idx;
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
-  p.q_pos = q_pos;
-  return launch_sa<kAttendIdx>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype);
+  return launch_sa<kAttendIdx>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype, q_pos);
 }
 
 size_t fasa_decode_workspace_bytes(const fasa_cache* c, int32_t len) {
@@ -422,8 +464,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.n_keep = std::min(k, len);
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
-  p.q_pos = q_pos;
-  return launch_sa<kDecode>(c, p, c->batch * c->n_kv_heads, true, stream, c->dtype);
+  return launch_sa<kDecode>(c, p, c->batch * c->n_kv_heads, true, stream, c->dtype, q_pos);
 }
 
 fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, void* out,
@@ -443,8 +484,7 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
   p.n_keep = len;
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
-  p.q_pos = q_pos;
-  return launch_sa<kDense>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype);
+  return launch_sa<kDense>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype, q_pos);
 }
 
 fasa_status fasa_device_status(int32_t clear) {

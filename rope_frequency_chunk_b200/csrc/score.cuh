@@ -8,9 +8,13 @@
 // first (in float64) into one coefficient per sketch column, Q[c].
 //
 // Data path: the sketch holds 2*n_dom values per token, stride padded to a
-// power-of-two number of 16-byte chunks. A token is read by LPT lanes, one
-// 16-byte chunk each, so a warp's load covers 512 contiguous bytes. The grid
-// is persistent and splits the flattened (row, token) range evenly.
+// power-of-two number of 16-byte chunks. The grid is persistent (one CTA per
+// SM) and splits the flattened (row, token) range evenly. A producer warp
+// streams the CTA's contiguous range through a ring of shared-memory stages
+// with 1-D bulk copies (TMA engine, full/empty mbarriers, no multicast); 16
+// consumer warps score the tokens, each token read from shared memory by LPT
+// lanes, one 16-byte chunk each. The first stages are in flight before the
+// query coefficients are computed.
 //
 // Arithmetic: float64. Each stored element e is widened exactly to the double
 // e * 2^-896 by placing its sign, exponent and mantissa bits in the double's
@@ -24,8 +28,10 @@
 
 namespace fasa {
 
-constexpr int kScoreThreads = 256;
-constexpr int kScoreUnroll = 4;
+constexpr int kScoreConsumerWarps = 16;
+constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kScoreStages = 8;
+constexpr int kScoreStageBytes = 24576;
 
 struct ScoreParams {
   const void* sketch;    // [rows][max_len][stride]
@@ -39,8 +45,8 @@ struct ScoreParams {
   int32_t n_kv_heads;
   int32_t group;
   int32_t n_dom;
-  int32_t q_pos;
-  double theta[kNFC];
+  double cosv[kNFC];   // cos / sin of q_pos * theta_i (host, float64)
+  double sinv[kNFC];
 };
 
 // Widen the two bf16 halves of w to (value * 2^-896) doubles, exactly.
@@ -83,83 +89,117 @@ __device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double 
 }
 
 template <typename T, int LPT>
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScoreParams p) {
   constexpr int EPC = Elem<T>::kPer16;
-  constexpr int TPW = 32 / LPT;  // tokens per warp load
-  constexpr int U = kScoreUnroll;
+  constexpr int TPW = 32 / LPT;                 // tokens per warp load
+  constexpr int ROWB = LPT * 16;                // sketch row bytes
+  constexpr int TPS = kScoreStageBytes / ROWB;  // tokens per stage
+  constexpr int NCW = kScoreConsumerWarps;
+  extern __shared__ __align__(128) unsigned char ring[];  // kScoreStages x kScoreStageBytes
   __shared__ double s_q[kD];
+  __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
+  __shared__ int st_row[kScoreStages], st_t0[kScoreStages], st_n[kScoreStages];
   grid_dependency_wait();
   grid_dependents_launch();  // the selection kernel may be scheduled now; it waits for our results
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int nw = kScoreThreads / 32;
-  const int sub = lane % LPT, tl = lane / LPT;
-  const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
-
   const int64_t per = (p.total + gridDim.x - 1) / gridDim.x;
-  int64_t f = (int64_t)blockIdx.x * per;
-  const int64_t f_end = min(p.total, f + per);
+  const int64_t f_beg = min(p.total, (int64_t)blockIdx.x * per);
+  const int64_t f_end = min(p.total, f_beg + per);
+  const int64_t n_tok = f_end - f_beg;
 
-  while (f < f_end) {
-    const int row = (int)(f / p.len);
-    const int t0 = (int)(f % p.len);
-    const int t1 = (int)min((int64_t)p.len, (int64_t)t0 + (f_end - f));
-    const int b = row / p.n_kv_heads, g = row % p.n_kv_heads;
+  if (tid == 0) {
+    for (int b = 0; b < kScoreStages; ++b) {
+      mbar_init(&full[b], 1);
+      mbar_init(&empty[b], NCW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
 
-    __syncthreads();  // previous segment done with s_q
-    if (tid < p.stride) {
-      double acc = 0.0;
-      const int j = tid >> 1;
-      if (j < p.n_dom) {
-        const int i = p.dom_idx[g * p.n_dom + j];
-        if (i >= 0 && i < kNFC) {
-          double s, c;
-          sincos((double)p.q_pos * p.theta[i], &s, &c);
-          const T* qh = static_cast<const T*>(p.q) + ((int64_t)(b * p.n_kv_heads + g) * p.group) * kD;
-          for (int h = 0; h < p.group; ++h) {
-            const double x = to_float(qh[h * kD + i]);
-            const double y = to_float(qh[h * kD + i + kNFC]);
-            // rotated query, first (x) or second (y) dim of FC i
-            acc += (tid & 1) ? __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s))
-                             : __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
-          }
-        } else {
-          flag_status(FASA_ERR_BAD_INDEX);
+  if (warp == NCW) {
+    // ---------------- producer: one lane walks the range, stage by stage
+    if (lane == 0 && n_tok > 0) {
+      int row = (int)(f_beg / p.len), t = (int)(f_beg % p.len);
+      int64_t left = n_tok;
+      for (int j = 0; left > 0; ++j) {
+        const int b = j % kScoreStages;
+        if (j >= kScoreStages && !mbar_wait(&empty[b], (uint32_t)(((j / kScoreStages) - 1) & 1))) break;
+        const int n = (int)min((int64_t)min(TPS, p.len - t), left);
+        st_row[b] = row;
+        st_t0[b] = t;
+        st_n[b] = n;
+        mbar_arrive_expect_tx(&full[b], (uint32_t)(n * ROWB));
+        bulk_g2s(ring + (size_t)b * kScoreStageBytes,
+                 static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t) * ROWB, (uint32_t)(n * ROWB),
+                 &full[b]);
+        left -= n;
+        t += n;
+        if (t == p.len) {
+          t = 0;
+          ++row;
         }
       }
-      s_q[tid] = acc * two896;
     }
-    __syncthreads();
-    double qr[EPC];
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) qr[e] = s_q[sub * EPC + e];
+    return;
+  }
 
-    const char* base = static_cast<const char*>(p.sketch) +
-                       ((int64_t)row * p.max_len) * p.stride * (int64_t)sizeof(T) + sub * 16;
-    const int64_t row_bytes = (int64_t)p.stride * sizeof(T);
-    float* out = p.scores + (int64_t)row * p.len;
-    const int ngroups = (t1 - t0 + TPW - 1) / TPW;
-
-    for (int gi = warp; gi < ngroups; gi += nw * U) {
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tg = gi + u * nw;
-        const int t = t0 + tg * TPW + tl;
-        if (tg < ngroups && t < t1) v[u] = ld_stream16(base + (int64_t)t * row_bytes);
-        else v[u] = make_uint4(0, 0, 0, 0);
+  // ---------------- consumers
+  const int sub = lane % LPT, tl = lane / LPT;
+  const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
+  double qr[EPC];
+  int cur_row = -1;
+  float* out = p.scores;
+  int64_t done = 0;
+  for (int j = 0; done < n_tok; ++j) {
+    const int b = j % kScoreStages;
+    if (!mbar_wait(&full[b], (uint32_t)((j / kScoreStages) & 1))) break;  // status already recorded
+    const int row = st_row[b], t0 = st_t0[b], n = st_n[b];
+    if (row != cur_row) {
+      // new row: the group's rotated queries summed per sketch column (float64)
+      named_barrier_sync(1, NCW * 32);
+      if (tid < p.stride) {
+        const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
+        double acc = 0.0;
+        const int jj = tid >> 1;
+        if (jj < p.n_dom) {
+          const int i = p.dom_idx[g * p.n_dom + jj];
+          if (i >= 0 && i < kNFC) {
+            const double c = p.cosv[i], s = p.sinv[i];
+            const T* qh = static_cast<const T*>(p.q) + ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD;
+            for (int h = 0; h < p.group; ++h) {
+              const double x = to_float(qh[h * kD + i]);
+              const double y = to_float(qh[h * kD + i + kNFC]);
+              // rotated query, first (x) or second (y) dim of FC i
+              acc += (tid & 1) ? __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s))
+                               : __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
+            }
+          } else {
+            flag_status(FASA_ERR_BAD_INDEX);
+          }
+        }
+        s_q[tid] = acc * two896;
       }
+      named_barrier_sync(1, NCW * 32);
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tg = gi + u * nw;
-        const int t = t0 + tg * TPW + tl;
-        double acc = chunk_dot<T>(v[u], qr);
-#pragma unroll
-        for (int off = LPT / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-        if (sub == 0 && tg < ngroups && t < t1) out[t] = (float)acc;
-      }
+      for (int e = 0; e < EPC; ++e) qr[e] = s_q[sub * EPC + e];
+      cur_row = row;
+      out = p.scores + (int64_t)row * p.len + 0;
     }
-    f += (t1 - t0);
+    const unsigned char* buf = ring + (size_t)b * kScoreStageBytes;
+    const int ngroups = (n + TPW - 1) / TPW;
+    for (int gi = warp; gi < ngroups; gi += NCW) {
+      const int t = gi * TPW + tl;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t < n) v = *reinterpret_cast<const uint4*>(buf + t * ROWB + sub * 16);
+      double acc = chunk_dot<T>(v, qr);
+#pragma unroll
+      for (int off = LPT / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+      if (sub == 0 && t < n) out[t0 + t] = (float)acc;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[b]);
+    done += n;
   }
 }
 

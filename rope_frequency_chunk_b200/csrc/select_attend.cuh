@@ -12,20 +12,26 @@
 //   kAttendIdx  given idx -> attention -> out (fasa_sparse_attend)
 //   kDense      all rows -> attention -> out (fasa_dense_decode)
 //
-// Select: exact top-k by a 3-pass radix select (11, 11, 10 bits) on
-// order-preserving uint32 keys. The C CTAs of a cluster each hold a contiguous
-// chunk of the row's keys in shared memory; per-pass histograms are summed
-// into the leader CTA's shared memory over DSMEM and every CTA reads the
-// total back, so no pass touches global memory. Ties at the threshold key go
-// to the lower token index; the kept indices are emitted in ascending order
-// straight into the shared memory of the CTA that will attend over them.
-//
-// Attention: each CTA takes an equal slice of the kept indices, gathers their
-// K and V rows with 1-D bulk copies (TMA engine, mbarrier completion,
-// double-buffered, no multicast), computes float32 logits for the G query
-// heads with 8 lanes per row, keeps a float32 online softmax (base-2, scale
-// folded into q), and accumulates P.V per 4-dim quad. Partials (m, l, o) are
-// merged across the cluster over DSMEM.
+// Selection is exact: the k_eff largest order-preserving uint32 keys, ties to
+// the lower token index. The C CTAs of a cluster each hold a contiguous chunk
+// of the row's keys in shared memory.
+//  1. Threshold guess: every CTA reads the same strided sample of the whole
+//     row from L2 and takes a value t_lo at or below the sample's
+//     j-th largest (j a few standard deviations above k_eff / stride), so
+//     that about k_eff + margin keys are >= t_lo.
+//  2. Every CTA counts its keys >= t_lo (warp ballots) and tells the others;
+//     if the total is < k_eff or exceeds the candidate buffer, all CTAs take
+//     the exact fallback (3 below on all keys).
+//  3. Candidates (key, index) are written, in index order, into every CTA's
+//     shared memory; each CTA finds the exact k_eff-th key and the number of
+//     ties to keep with a radix select whose digit histograms are counted by
+//     warp ballots (no atomics), and extracts its own slice of the kept list.
+// Attention: each CTA gathers its slice's K and V rows with 16-byte cp.async
+// (double-buffered), computes float32 logits with the query in registers and
+// a butterfly transpose-reduce across the warp, keeps a base-2 online
+// softmax, accumulates P.V per 4-dim quad, and the cluster merges its
+// (m, l, o) partials over DSMEM. The dense mode streams contiguous rows with
+// 1-D bulk copies (TMA engine, mbarrier completion, no multicast).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -37,8 +43,9 @@ namespace cg = cooperative_groups;
 
 constexpr int kSAThreads = 512;
 constexpr int kSAWarps = kSAThreads / 32;
-constexpr int kBins = 2048;
 constexpr int kMaxCluster = 16;
+constexpr int kMaxSamples = 2048;
+constexpr int kStageBytes = 32768;  // K + V rows of one pipeline stage
 
 enum SAMode { kSelect = 0, kDecode = 1, kAttendIdx = 2, kDense = 3 };
 
@@ -57,96 +64,216 @@ struct SAParams {
   int32_t slice;             // kept indices attended per CTA
   int32_t n_kv_heads;
   int32_t group;
-  int32_t q_pos;
-  double theta[kNFC];
+  int32_t cap;               // candidate capacity per CTA
+  int32_t sample_stride;     // s: every s-th score is sampled
+  int32_t sample_rank;       // j: rank of the sample used as threshold
+  int32_t n_stages;          // attention pipeline depth
+  double cosv[kNFC];         // cos / sin of q_pos * theta_i (host, float64)
+  double sinv[kNFC];
 };
 
-// Rows per pipeline stage: 32 KB of K+V per stage.
-template <typename T> __host__ __device__ constexpr int stage_rows() { return 32768 / (2 * kD * (int)sizeof(T)); }
+template <typename T> __host__ __device__ constexpr int stage_rows() {
+  return kStageBytes / (2 * kD * (int)sizeof(T));
+}
 
-// Shared-memory layout, identical on host and device.
 struct SALayout {
-  int off_keys, off_stage, off_idx, off_hist, off_ghist, off_q, off_z, off_o, off_ml, off_cs, off_misc, off_bar, total;
+  int keys, stage, cand_key, cand_idx, samples, idx, rscr, chist, misc, qraw, qs, zs, acc, ml, mlall, red, bar, total;
 };
 
 __host__ __device__ inline int sa_align(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SALayout sa_layout(int mode, int elem_bytes, int chunk, int slice, int maxg) {
+// Region A holds the keys and, after them, the candidate buffer during
+// selection, and the attention stages afterwards.
+__host__ __device__ inline SALayout sa_layout(int mode, int elem_bytes, int chunk, int slice, int cap, int maxg,
+                                              int n_stages) {
   SALayout L;
-  const int rb = 32768 / (2 * kD * elem_bytes);
+  const int rb = kStageBytes / (2 * kD * elem_bytes);
   const bool sel = (mode == kSelect || mode == kDecode);
   const bool att = (mode != kSelect);
-  const int keys_bytes = sel ? chunk * 4 : 0;
-  const int stage_bytes = att ? 2 * 32768 : 0;
-  const int a_bytes = keys_bytes > stage_bytes ? keys_bytes : stage_bytes;
+  const int keys_bytes = sel ? sa_align(chunk * 4, 128) : 0;
+  const int cand_bytes = sel ? 2 * sa_align(cap * 4, 128) : 0;
+  const int stage_bytes = att ? n_stages * kStageBytes : 0;
   int off = 0;
-  L.off_keys = off;
-  L.off_stage = off;  // stages reuse the key region after selection
-  off = sa_align(off + a_bytes, 128);
-  L.off_idx = off;
+  L.keys = L.stage = 0;
+  L.cand_key = keys_bytes;
+  L.cand_idx = keys_bytes + cand_bytes / 2;
+  off = sa_align(keys_bytes + cand_bytes > stage_bytes ? keys_bytes + cand_bytes : stage_bytes, 128);
+  L.samples = off;
+  off = sa_align(off + (sel ? kMaxSamples * 4 : 0), 128);
+  L.idx = off;
   off = sa_align(off + ((mode == kDecode || mode == kAttendIdx) ? slice * 4 : 0), 128);
-  L.off_hist = off;
-  off = sa_align(off + (sel ? kBins * 4 : 0), 128);
-  L.off_ghist = off;
-  off = sa_align(off + (sel ? 3 * kBins * 4 : 0), 128);
-  L.off_q = off;
+  L.rscr = off;
+  off = sa_align(off + (sel ? (kSAWarps * 256 + 256 + 8) * 4 : 0), 128);
+  L.chist = off;
+  off = sa_align(off + (sel ? 4 * 256 * 4 : 0), 128);
+  L.misc = off;
+  off = sa_align(off + 128 * 4, 128);
+  L.qraw = off;
+  off = sa_align(off + (att ? maxg * kD * elem_bytes : 0), 128);
+  L.qs = off;
   off = sa_align(off + (att ? maxg * kD * 4 : 0), 128);
-  L.off_z = off;
+  L.zs = off;
   off = sa_align(off + (att ? maxg * rb * 4 : 0), 128);
-  L.off_o = off;
+  L.acc = off;
   off = sa_align(off + (att ? maxg * kD * 4 : 0), 128);
-  L.off_ml = off;
-  off = sa_align(off + (att ? 3 * maxg * 4 : 0), 128);
-  L.off_cs = off;
-  off = sa_align(off + (att ? 2 * kNFC * 8 : 0), 128);
-  L.off_misc = off;
-  off = sa_align(off + 256 * 4, 128);
-  L.off_bar = off;
-  off = sa_align(off + 2 * 8, 128);
+  L.ml = off;
+  off = sa_align(off + (att ? 4 * maxg * 4 : 0), 128);
+  L.mlall = off;
+  off = sa_align(off + (att ? kMaxCluster * 2 * maxg * 4 : 0), 128);
+  L.red = off;
+  off = sa_align(off + (att ? (maxg * kD + kMaxCluster) * 4 : 0), 128);
+  L.bar = off;
+  off = sa_align(off + 8 * 8, 128);
   L.total = off;
   return L;
 }
 
 // misc-area slots (uint32 words)
 enum : int {
-  kMiscWarpGt = 0,     // [16]
-  kMiscWarpEq = 16,    // [16]
-  kMiscCtaGt = 32,     // [16]  written remotely into the leader
-  kMiscCtaEq = 48,     // [16]
-  kMiscScan = 64,      // [16]  block-scan scratch
-  kMiscBin = 80,       // broadcast: selected bin
-  kMiscAbove = 81,     // broadcast: count above it
-  kMiscGtBefore = 82,
-  kMiscEqBefore = 83,
+  kMiscWarpA = 0,     // [16] per-warp counts / exclusive offsets
+  kMiscWarpB = 16,    // [16]
+  kMiscCtaA = 32,     // [16] per-CTA counts, written by every CTA into every CTA
+  kMiscCtaB = 48,     // [16]
+  kMiscScan = 64,     // [16] scratch
+  kMiscBcast = 80,    // [8]  broadcast values
 };
 
-// Inclusive scan of one value per thread (thread order), block-wide.
-__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* scratch) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// ----------------------------------------------------------- helpers
+
+// Exclusive scan of the 16 per-warp values in misc[base..base+16) in place;
+// returns the total. Call from one thread.
+__device__ __forceinline__ uint32_t warp_offsets_serial(uint32_t* misc, int base) {
+  uint32_t t = 0;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, v, off);
-    if (lane >= off) v += n;
+  for (int w = 0; w < kSAWarps; ++w) {
+    const uint32_t a = misc[base + w];
+    misc[base + w] = t;
+    t += a;
   }
-  if (lane == 31) scratch[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = lane < kSAWarps ? scratch[lane] : 0u;
+  return t;
+}
+
+// Exact radix select by 8-bit digits, most significant first, over
+// keys[0..n) in shared memory. Digit histograms are counted with warp
+// ballots, no atomics: one ballot per digit bit, and lane L counts bins
+// 8L..8L+7 by intersecting the ballots. After `passes` passes (4 = exact),
+// returns the prefix of the k-th largest key and how many keys equal to that
+// prefix must still be taken (ties to the lower position). With kCluster the
+// per-pass histograms are summed over the cluster in the leader's shared
+// memory.
+template <bool kCluster>
+__device__ void ballot_radix(const uint32_t* keys, int n, int k, int passes, uint32_t* rscr, uint32_t* chist,
+                             cg::cluster_group& cluster, uint32_t& out_prefix, int& out_krem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* tot = rscr + kSAWarps * 256;
+  uint32_t* bc = tot + 256;
+  uint32_t prefix = 0u, pmask = 0u;
+  int krem = k;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = 24 - 8 * pass;
+    uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    for (int base = warp * 32; base < n; base += kSAThreads) {
+      const int i = base + lane;
+      bool act = false;
+      uint32_t d = 0u;
+      if (i < n) {
+        const uint32_t x = keys[i];
+        act = (x & pmask) == prefix;
+        d = (x >> shift) & 255u;
+      }
+      unsigned b[8];
+      const unsigned a = __ballot_sync(0xFFFFFFFFu, act);
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t n = __shfl_up_sync(0xFFFFFFFFu, w, off);
-      if (lane >= off) w += n;
+      for (int j = 0; j < 8; ++j) b[j] = __ballot_sync(0xFFFFFFFFu, act && ((d >> j) & 1u));
+      unsigned m = a;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) m &= ((lane >> j) & 1) ? b[3 + j] : ~b[3 + j];
+      const unsigned n0 = ~b[0], n1 = ~b[1], n2 = ~b[2];
+      cnt[0] += __popc(m & n0 & n1 & n2);
+      cnt[1] += __popc(m & b[0] & n1 & n2);
+      cnt[2] += __popc(m & n0 & b[1] & n2);
+      cnt[3] += __popc(m & b[0] & b[1] & n2);
+      cnt[4] += __popc(m & n0 & n1 & b[2]);
+      cnt[5] += __popc(m & b[0] & n1 & b[2]);
+      cnt[6] += __popc(m & n0 & b[1] & b[2]);
+      cnt[7] += __popc(m & b[0] & b[1] & b[2]);
     }
-    if (lane < kSAWarps) scratch[lane] = w;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) rscr[warp * 256 + lane * 8 + u] = cnt[u];
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t sum = 0u;
+#pragma unroll
+      for (int w = 0; w < kSAWarps; ++w) sum += rscr[w * 256 + tid];
+      if (kCluster) {
+        if (sum) atomicAdd(cluster.map_shared_rank(chist + pass * 256, 0) + tid, sum);
+      } else {
+        tot[tid] = sum;
+      }
+    }
+    if (kCluster) {
+      cluster_arrive();
+      cluster_wait();
+      if (tid < 256) tot[tid] = cluster.map_shared_rank(chist + pass * 256, 0)[tid];
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t g[8], gs = 0u;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        g[u] = tot[lane * 8 + u];
+        gs += g[u];
+      }
+      // inclusive sum over this lane and all higher lanes (higher bins)
+      uint32_t incl = gs;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, off);
+        if (lane + off < 32) incl += v;
+      }
+      const uint32_t excl = incl - gs;
+      if (excl < (uint32_t)krem && (uint32_t)krem <= incl) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+          if (acc + g[u] >= (uint32_t)krem) {
+            bc[0] = (uint32_t)(lane * 8 + u);
+            bc[1] = acc;
+            break;
+          }
+          acc += g[u];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= bc[0] << shift;
+    pmask |= 255u << shift;
+    krem -= (int)bc[1];
   }
-  __syncthreads();
-  const uint32_t before = warp > 0 ? scratch[warp - 1] : 0u;
-  __syncthreads();
-  return v + before;
+  out_prefix = prefix;
+  out_krem = krem;
+}
+
+// Unrolled coalesced load of n score keys (global float -> order-preserving key).
+__device__ __forceinline__ void load_keys(uint32_t* dst, const float* src, int n) {
+  constexpr int U = 8;
+  for (int base = threadIdx.x; base < n; base += kSAThreads * U) {
+    float f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * kSAThreads;
+      f[u] = i < n ? __ldcg(src + i) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * kSAThreads;
+      if (i < n) dst[i] = score_key(f[u]);
+    }
+  }
 }
 
 template <typename T, int MODE, int MAXG>
-__global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend_kernel(const SAParams p) {
+__global__ void __launch_bounds__(kSAThreads, 1) select_attend_kernel(const SAParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   grid_dependency_wait();  // inputs of an earlier kernel in the stream are complete
   cg::cluster_group cluster = cg::this_cluster();
@@ -158,203 +285,257 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
   constexpr bool kAtt = (MODE != kSelect);
   constexpr int RB = stage_rows<T>();
   constexpr int ES = (int)sizeof(T);
+  constexpr int NV = (MAXG == 8) ? 32 : 16;  // partial logits per lane in one step
+  constexpr int RPW = NV / MAXG;              // rows per warp in one logit step
+  constexpr bool kQReg = MAXG <= 8;           // query slice held in registers
+  const unsigned lt = (1u << lane) - 1u;
 
-  const SALayout L = sa_layout(MODE, ES, p.chunk, p.slice, MAXG);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.off_keys);
-  T* stage = reinterpret_cast<T*>(smem + L.off_stage);
-  int32_t* idx_s = reinterpret_cast<int32_t*>(smem + L.off_idx);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.off_hist);
-  uint32_t* ghist = reinterpret_cast<uint32_t*>(smem + L.off_ghist);
-  float* qs = reinterpret_cast<float*>(smem + L.off_q);
-  float* zs = reinterpret_cast<float*>(smem + L.off_z);
-  float* os = reinterpret_cast<float*>(smem + L.off_o);
-  float* ml = reinterpret_cast<float*>(smem + L.off_ml);  // m[MAXG], l[MAXG], scale[MAXG]
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L.off_misc);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  const SALayout L = sa_layout(MODE, ES, p.chunk, p.slice, p.cap, MAXG, p.n_stages);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  unsigned char* stage = smem + L.stage;
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(smem + L.cand_key);
+  int32_t* cand_idx = reinterpret_cast<int32_t*>(smem + L.cand_idx);
+  uint32_t* samples = reinterpret_cast<uint32_t*>(smem + L.samples);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem + L.idx);
+  uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + L.rscr);
+  uint32_t* chist = reinterpret_cast<uint32_t*>(smem + L.chist);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L.misc);
+  float* qs = reinterpret_cast<float*>(smem + L.qs);
+  float* zs = reinterpret_cast<float*>(smem + L.zs);
+  float* acc_s = reinterpret_cast<float*>(smem + L.acc);
+  float* ml = reinterpret_cast<float*>(smem + L.ml);  // m[MAXG], l[MAXG], scale[MAXG], weight[MAXG]
+  float* mlall = reinterpret_cast<float*>(smem + L.mlall);
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  unsigned char* qraw = smem + L.qraw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
 
   const int G = p.group;
 
   // ------------------------------------------------------------ set-up
   if (kSel && rank == 0)
-    for (int i = tid; i < 3 * kBins; i += kSAThreads) ghist[i] = 0u;
+    for (int i = tid; i < 4 * 256; i += kSAThreads) chist[i] = 0u;
+  if (tid < 128) misc[tid] = 0u;
   if (MODE == kDecode)  // slots the selection never fills stay masked
     for (int i = tid; i < p.slice; i += kSAThreads) idx_s[i] = -1;
   if (kAtt) {
-    if (tid == 0) {
-      mbar_init(&bars[0], 1);
-      mbar_init(&bars[1], 1);
+    // prefetch the group's raw queries; rotated just before attention
+    const unsigned char* qsrc = static_cast<const unsigned char*>(p.q) + ((int64_t)row * G) * kD * ES;
+    for (int c = tid; c < G * kD * ES / 16; c += kSAThreads) cp_async16(qraw + c * 16, qsrc + c * 16);
+    cp_async_commit();
+    if (MODE == kDense && tid == 0) {
+      for (int s = 0; s < p.n_stages; ++s) mbar_init(&bars[s], 1);
       fence_mbar_init();
     }
-    for (int i = tid; i < MAXG * kD; i += kSAThreads) os[i] = 0.0f;
+    for (int i = tid; i < MAXG * kD; i += kSAThreads) acc_s[i] = 0.0f;
     if (tid < MAXG) {
       ml[tid] = -INFINITY;
       ml[MAXG + tid] = 0.0f;
       ml[2 * MAXG + tid] = 0.0f;
+      ml[3 * MAXG + tid] = 0.0f;
     }
-    // rotated, pre-scaled queries: q'_h * log2(e) / sqrt(128), float32
-    double* cs = reinterpret_cast<double*>(smem + L.off_cs);  // 64 x (cos, sin)
-    if (tid < kNFC) {
-      double s, c;
-      sincos((double)p.q_pos * p.theta[tid], &s, &c);
-      cs[2 * tid] = c;
-      cs[2 * tid + 1] = s;
-    }
-    __syncthreads();
-    const T* qh = static_cast<const T*>(p.q) + ((int64_t)row * G) * kD;
-    const double qscale = 1.4426950408889634 / 11.313708498984761;  // log2(e) / sqrt(128)
-    for (int e = tid; e < G * kD; e += kSAThreads) {
-      const int h = e / kD, d = e % kD, i = d & (kNFC - 1);
-      const double x = to_float(qh[h * kD + i]);
-      const double y = to_float(qh[h * kD + i + kNFC]);
-      const double c = cs[2 * i], s = cs[2 * i + 1];
-      const double r = (d < kNFC) ? (x * c - y * s) : (y * c + x * s);
-      qs[h * kD + d] = (float)(r * qscale);
-    }
-    for (int e = G * kD + tid; e < MAXG * kD; e += kSAThreads) qs[e] = 0.0f;
   }
   __syncthreads();
-  if (C > 1) cluster.sync();  // all CTAs started; leader histograms zeroed
+  if (C > 1) cluster_arrive();  // "all CTAs started": waited for before the first DSMEM access
+  bool start_waited = (C == 1);
 
   int n_mine = 0;      // rows this CTA attends over
-  int row_start = 0;   // first row (dense) / first slice position (kept lists)
+  int row_start = 0;   // first slice position (kept lists) or first row (dense)
 
   // ------------------------------------------------------------ select
   if constexpr (kSel) {
     const int start = rank * p.chunk;
     const int n_loc = max(0, min(p.chunk, p.len - start));
-    const float* srow = p.scores + (int64_t)row * p.len + start;
-    for (int i = tid; i < n_loc; i += kSAThreads) keys[i] = score_key(srow[i]);
+    const float* srow = p.scores + (int64_t)row * p.len;
+    load_keys(keys, srow + start, n_loc);
+    const int s_str = p.sample_stride;
+    const int m = (p.len + s_str - 1) / s_str;
+    const bool use_samples = p.sample_rank < m;
+    if (use_samples)
+      for (int i = tid; i < m; i += kSAThreads) samples[i] = score_key(__ldcg(srow + (int64_t)i * s_str));
     __syncthreads();
 
-    uint32_t prefix = 0u, pmask = 0u;
-    int krem = p.n_keep;
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int nb = pass == 2 ? 1024 : 2048;
-      for (int i = tid; i < kBins; i += kSAThreads) hist[i] = 0u;
-      __syncthreads();
-      for (int base = warp * 32; base < n_loc; base += kSAThreads) {
-        const int i = base + lane;
-        bool ok = false;
-        uint32_t bin = 0u;
-        if (i < n_loc) {
-          const uint32_t x = keys[i];
-          ok = (x & pmask) == prefix;
-          bin = (x >> shift) & (uint32_t)(nb - 1);
-        }
-        const unsigned act = __ballot_sync(0xFFFFFFFFu, ok);
-        if (ok) {
-          const unsigned peers = __match_any_sync(act, bin);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-        }
-      }
-      __syncthreads();
-      uint32_t* gh = cluster.map_shared_rank(ghist + pass * kBins, 0);
-      for (int i = tid; i < nb; i += kSAThreads) {
-        const uint32_t h = hist[i];
-        if (h) atomicAdd(gh + i, h);
-      }
-      if (C > 1) cluster.sync(); else __syncthreads();
-      // find the bin holding the krem-th largest key, scanning from the top
-      const int per = nb / kSAThreads;  // 4 or 2 bins per thread
-      uint32_t c[4] = {0u, 0u, 0u, 0u};
-      uint32_t sum = 0u;
-      for (int j = 0; j < per; ++j) {
-        c[j] = gh[nb - 1 - (tid * per + j)];
-        sum += c[j];
-      }
-      const uint32_t incl = block_incl_scan(sum, misc + kMiscScan);
-      const uint32_t excl = incl - sum;
-      if (excl < (uint32_t)krem && (uint32_t)krem <= incl) {
-        uint32_t acc = excl;
-        for (int j = 0; j < per; ++j) {
-          if (acc + c[j] >= (uint32_t)krem) {
-            misc[kMiscBin] = (uint32_t)(nb - 1 - (tid * per + j));
-            misc[kMiscAbove] = acc;
-            break;
-          }
-          acc += c[j];
-        }
-      }
-      __syncthreads();
-      const uint32_t bin = misc[kMiscBin];
-      krem -= (int)misc[kMiscAbove];
-      prefix |= bin << shift;
-      pmask |= (uint32_t)(nb - 1) << shift;
-      __syncthreads();
+    // 1. threshold from the sample: the top 16 bits of its j-th largest key
+    uint32_t t_lo = 0u;
+    if (use_samples) {
+      uint32_t pre;
+      int kr;
+      ballot_radix<false>(samples, m, p.sample_rank, 2, rscr, chist, cluster, pre, kr);
+      t_lo = pre;
     }
-    const uint32_t thr = prefix;  // the k_eff-th largest key; take krem of the keys equal to it
 
-    // count keys above / at the threshold per warp (warp segments in index order)
+    // 2. count local keys >= t_lo by warp segments (index order)
     const int seg = ((n_loc + kSAWarps * 32 - 1) / (kSAWarps * 32)) * 32;
     const int ws = min(n_loc, warp * seg), we = min(n_loc, ws + seg);
-    uint32_t cgt = 0u, ceq = 0u;
+    uint32_t cnt = 0u;
     for (int base = ws; base < we; base += 32) {
       const int i = base + lane;
-      const bool valid = i < we;
-      const uint32_t x = valid ? keys[i] : 0u;
-      cgt += __popc(__ballot_sync(0xFFFFFFFFu, valid && x > thr));
-      ceq += __popc(__ballot_sync(0xFFFFFFFFu, valid && x == thr));
+      cnt += __popc(__ballot_sync(0xFFFFFFFFu, i < we && keys[i] >= t_lo));
     }
-    if (lane == 0) {
-      misc[kMiscWarpGt + warp] = cgt;
-      misc[kMiscWarpEq + warp] = ceq;
-    }
+    if (lane == 0) misc[kMiscWarpA + warp] = cnt;
     __syncthreads();
-    if (tid == 0) {
-      uint32_t tg = 0u, te = 0u;
-      for (int w = 0; w < kSAWarps; ++w) {
-        const uint32_t a = misc[kMiscWarpGt + w], e = misc[kMiscWarpEq + w];
-        misc[kMiscWarpGt + w] = tg;  // exclusive offsets
-        misc[kMiscWarpEq + w] = te;
-        tg += a;
-        te += e;
-      }
-      uint32_t* lead = cluster.map_shared_rank(misc, 0);
-      lead[kMiscCtaGt + rank] = tg;
-      lead[kMiscCtaEq + rank] = te;
+    if (tid == 0) misc[kMiscBcast] = warp_offsets_serial(misc, kMiscWarpA);
+    __syncthreads();
+    if (!start_waited) {
+      cluster_wait();
+      start_waited = true;
     }
-    if (C > 1) cluster.sync(); else __syncthreads();
-    if (tid == 0) {
-      const uint32_t* lead = cluster.map_shared_rank(misc, 0);
+    if (tid < C) cluster.map_shared_rank(misc, tid)[kMiscCtaA + rank] = misc[kMiscBcast];
+    if (C > 1) {
+      cluster_arrive();
+      cluster_wait();
+    } else {
+      __syncthreads();
+    }
+    uint32_t total = 0u, before = 0u;
+    for (int r = 0; r < C; ++r) {
+      const uint32_t c = misc[kMiscCtaA + r];
+      total += c;
+      if (r < rank) before += c;
+    }
+    const bool fast = total >= (uint32_t)p.n_keep && total <= (uint32_t)p.cap;  // same in every CTA
+
+    uint32_t thr = 0u;
+    int quota = 0;
+    if (fast) {
+      // 3. candidates, in index order, into the leader
+      uint32_t* lkey = cluster.map_shared_rank(cand_key, 0);
+      int32_t* lidx = cluster.map_shared_rank(cand_idx, 0);
+      uint32_t pos = before + misc[kMiscWarpA + warp];
+      for (int base = ws; base < we; base += 32) {
+        const int i = base + lane;
+        const bool sel = i < we && keys[i] >= t_lo;
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+          const uint32_t at = pos + __popc(b & lt);
+          lkey[at] = keys[i];
+          lidx[at] = start + i;
+        }
+        pos += __popc(b);
+      }
+      if (C > 1) {
+        cluster_arrive();
+        cluster_wait();
+      } else {
+        __syncthreads();
+      }
+      if (rank == 0) {
+        // exact k_eff-th key among the candidates; the kept list is the
+        // candidates above it and the first `quota` equal to it
+        ballot_radix<false>(cand_key, (int)total, p.n_keep, 4, rscr, chist, cluster, thr, quota);
+        const int n = (int)total;
+        const int cseg = ((n + kSAWarps * 32 - 1) / (kSAWarps * 32)) * 32;
+        const int cs = min(n, warp * cseg), ce = min(n, cs + cseg);
+        uint32_t cg_ = 0u, ce_ = 0u;
+        for (int base = cs; base < ce; base += 32) {
+          const int i = base + lane;
+          const bool v = i < ce;
+          const uint32_t x = v ? cand_key[i] : 0u;
+          cg_ += __popc(__ballot_sync(0xFFFFFFFFu, v && x > thr));
+          ce_ += __popc(__ballot_sync(0xFFFFFFFFu, v && x == thr));
+        }
+        if (lane == 0) {
+          misc[kMiscWarpA + warp] = cg_;
+          misc[kMiscWarpB + warp] = ce_;
+        }
+        __syncthreads();
+        if (tid == 0) {
+          warp_offsets_serial(misc, kMiscWarpA);
+          warp_offsets_serial(misc, kMiscWarpB);
+        }
+        __syncthreads();
+        int gr = (int)misc[kMiscWarpA + warp], er = (int)misc[kMiscWarpB + warp];
+        for (int base = cs; base < ce; base += 32) {
+          const int i = base + lane;
+          const bool v = i < ce;
+          const uint32_t x = v ? cand_key[i] : 0u;
+          const bool is_gt = v && x > thr, is_eq = v && x == thr;
+          const unsigned bg = __ballot_sync(0xFFFFFFFFu, is_gt);
+          const unsigned be = __ballot_sync(0xFFFFFFFFu, is_eq);
+          const int my_gr = gr + __popc(bg & lt), my_er = er + __popc(be & lt);
+          const int at = my_gr + min(my_er, quota);
+          if ((is_gt || (is_eq && my_er < quota)) && at < p.n_keep) {
+            const int token = cand_idx[i];
+            const int owner = at / p.slice;
+            if (MODE == kDecode) cluster.map_shared_rank(idx_s, owner)[at - owner * p.slice] = token;
+            if (p.idx_out) p.idx_out[(int64_t)row * p.n_keep + at] = token;
+          }
+          gr += __popc(bg);
+          er += __popc(be);
+        }
+      }
+      if (C > 1) {
+        cluster_arrive();
+        cluster_wait();
+      } else {
+        __syncthreads();
+      }
+    } else {
+      // exact fallback over all keys, histograms summed across the cluster
+      ballot_radix<true>(keys, n_loc, p.n_keep, 4, rscr, chist, cluster, thr, quota);
+      uint32_t cgt = 0u, ceq = 0u;
+      for (int base = ws; base < we; base += 32) {
+        const int i = base + lane;
+        const bool v = i < we;
+        const uint32_t x = v ? keys[i] : 0u;
+        cgt += __popc(__ballot_sync(0xFFFFFFFFu, v && x > thr));
+        ceq += __popc(__ballot_sync(0xFFFFFFFFu, v && x == thr));
+      }
+      if (lane == 0) {
+        misc[kMiscWarpA + warp] = cgt;
+        misc[kMiscWarpB + warp] = ceq;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        misc[kMiscBcast + 1] = warp_offsets_serial(misc, kMiscWarpA);
+        misc[kMiscBcast + 2] = warp_offsets_serial(misc, kMiscWarpB);
+      }
+      __syncthreads();
+      if (tid < C) {
+        uint32_t* dst = cluster.map_shared_rank(misc, tid);
+        dst[kMiscCtaA + rank] = misc[kMiscBcast + 1];
+        dst[kMiscCtaB + rank] = misc[kMiscBcast + 2];
+      }
+      if (C > 1) {
+        cluster_arrive();
+        cluster_wait();
+      } else {
+        __syncthreads();
+      }
       uint32_t gb = 0u, eb = 0u;
       for (int r = 0; r < rank; ++r) {
-        gb += lead[kMiscCtaGt + r];
-        eb += lead[kMiscCtaEq + r];
+        gb += misc[kMiscCtaA + r];
+        eb += misc[kMiscCtaB + r];
       }
-      misc[kMiscGtBefore] = gb;
-      misc[kMiscEqBefore] = eb;
-    }
-    __syncthreads();
-
-    // emit the kept indices in ascending order
-    int gr = (int)(misc[kMiscGtBefore] + misc[kMiscWarpGt + warp]);
-    int er = (int)(misc[kMiscEqBefore] + misc[kMiscWarpEq + warp]);
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = ws; base < we; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < we;
-      const uint32_t x = valid ? keys[i] : 0u;
-      const bool is_gt = valid && x > thr, is_eq = valid && x == thr;
-      const unsigned bg = __ballot_sync(0xFFFFFFFFu, is_gt);
-      const unsigned be = __ballot_sync(0xFFFFFFFFu, is_eq);
-      const int my_gr = gr + __popc(bg & lt), my_er = er + __popc(be & lt);
-      const int pos = my_gr + min(my_er, krem);
-      if ((is_gt || (is_eq && my_er < krem)) && pos >= p.n_keep) flag_status(FASA_ERR_BAD_INDEX);
-      if ((is_gt || (is_eq && my_er < krem)) && pos < p.n_keep) {
-        const int token = start + i;
-        if (MODE == kDecode) {
-          const int owner = pos / p.slice;
-          int32_t* dst = cluster.map_shared_rank(idx_s, owner);
-          dst[pos - owner * p.slice] = token;
+      int gr = (int)(gb + misc[kMiscWarpA + warp]);
+      int er = (int)(eb + misc[kMiscWarpB + warp]);
+      for (int base = ws; base < we; base += 32) {
+        const int i = base + lane;
+        const bool v = i < we;
+        const uint32_t x = v ? keys[i] : 0u;
+        const bool is_gt = v && x > thr, is_eq = v && x == thr;
+        const unsigned bg = __ballot_sync(0xFFFFFFFFu, is_gt);
+        const unsigned be = __ballot_sync(0xFFFFFFFFu, is_eq);
+        const int my_gr = gr + __popc(bg & lt), my_er = er + __popc(be & lt);
+        const int at = my_gr + min(my_er, quota);
+        if (is_gt || (is_eq && my_er < quota)) {
+          if (at < p.n_keep) {
+            const int owner = at / p.slice;
+            if (MODE == kDecode) cluster.map_shared_rank(idx_s, owner)[at - owner * p.slice] = start + i;
+            if (p.idx_out) p.idx_out[(int64_t)row * p.n_keep + at] = start + i;
+          } else {
+            flag_status(FASA_ERR_BAD_INDEX);
+          }
         }
-        if (p.idx_out) p.idx_out[(int64_t)row * p.n_keep + pos] = token;
+        gr += __popc(bg);
+        er += __popc(be);
       }
-      gr += __popc(bg);
-      er += __popc(be);
+      if (C > 1) {
+        cluster_arrive();
+        cluster_wait();
+      } else {
+        __syncthreads();
+      }
     }
-    fence_proxy_async_smem();  // key region is reused by bulk copies below
-    if (C > 1) cluster.sync(); else __syncthreads();
     if (MODE == kDecode) {
       row_start = rank * p.slice;
       n_mine = max(0, min(p.slice, p.n_keep - row_start));
@@ -362,7 +543,9 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
   }
 
   if constexpr (!kAtt) {
-    return;  // the last cluster barrier above keeps the leader alive while read
+    // no DSMEM access follows the last cluster barrier
+    if (!start_waited) cluster_wait();
+    return;
   } else {
     if (MODE == kAttendIdx) {
       row_start = rank * p.slice;
@@ -376,106 +559,174 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
         }
         idx_s[j] = t;
       }
-      __syncthreads();
     } else if (MODE == kDense) {
       row_start = rank * p.chunk;
       n_mine = max(0, min(p.chunk, p.len - row_start));
     }
+    __syncthreads();
+
+    // rotated, pre-scaled queries: q'_h * log2(e) / sqrt(128), float32
+    cp_async_wait<0>();
+    __syncthreads();
+    {
+      const T* qh = reinterpret_cast<const T*>(qraw);
+      const double qscale = 1.4426950408889634 / 11.313708498984761;  // log2(e) / sqrt(128)
+      for (int e = tid; e < MAXG * kD; e += kSAThreads) {
+        const int h = e / kD, d = e % kD, i = d & (kNFC - 1);
+        float val = 0.0f;
+        if (h < G) {
+          const double x = to_float(qh[h * kD + i]);
+          const double y = to_float(qh[h * kD + i + kNFC]);
+          const double c = p.cosv[i], s = p.sinv[i];
+          const double r = (d < kNFC) ? (x * c - y * s) : (y * c + x * s);
+          val = (float)(r * qscale);
+        }
+        qs[e] = val;
+      }
+    }
+    __syncthreads();
 
     const T* kbase = static_cast<const T*>(p.k) + (int64_t)row * p.max_len * kD;
     const T* vbase = static_cast<const T*>(p.v) + (int64_t)row * p.max_len * kD;
     const int nbatch = (n_mine + RB - 1) / RB;
+    const int NST = p.n_stages;
+    constexpr int CPR = kD * ES / 16;  // 16-byte chunks per row
 
+    // load batch bi into stage bi % NST (gather: cp.async; dense: bulk copies)
     auto issue = [&](int bi) {
-      const int s = bi & 1;
-      const int j0 = bi * RB;
-      const int nr = min(RB, n_mine - j0);
-      T* ks = stage + (size_t)s * 2 * RB * kD;
-      T* vs = ks + RB * kD;
-      if (lane == 0) mbar_arrive_expect_tx(&bars[s], (uint32_t)(nr * 2 * kD * ES));
-      __syncwarp();
-      if (MODE == kDense) {
-        if (lane == 0) {
-          bulk_g2s(ks, kbase + (int64_t)(row_start + j0) * kD, (uint32_t)(nr * kD * ES), &bars[s]);
-          bulk_g2s(vs, vbase + (int64_t)(row_start + j0) * kD, (uint32_t)(nr * kD * ES), &bars[s]);
-        }
-      } else {
-        for (int r = lane; r < nr; r += 32) {
-          int t = idx_s[j0 + r];  // this CTA's slice of the kept list
-          if (t < 0 || t >= p.len) t = 0;  // skipped index: copy a valid row, masked below
-          bulk_g2s(ks + r * kD, kbase + (int64_t)t * kD, kD * ES, &bars[s]);
-          bulk_g2s(vs + r * kD, vbase + (int64_t)t * kD, kD * ES, &bars[s]);
+      if (bi < nbatch) {
+        const int s = bi % NST;
+        const int j0 = bi * RB;
+        const int nr = min(RB, n_mine - j0);
+        unsigned char* ks = stage + (size_t)s * kStageBytes;
+        unsigned char* vs = ks + RB * kD * ES;
+        if (MODE == kDense) {
+          if (tid == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&bars[s], (uint32_t)(nr * 2 * kD * ES));
+            bulk_g2s(ks, kbase + (int64_t)(row_start + j0) * kD, (uint32_t)(nr * kD * ES), &bars[s]);
+            bulk_g2s(vs, vbase + (int64_t)(row_start + j0) * kD, (uint32_t)(nr * kD * ES), &bars[s]);
+          }
+        } else {
+          const int tot = nr * CPR;
+          for (int c = tid; c < 2 * tot; c += kSAThreads) {
+            const int which = c >= tot;
+            const int rem = c - which * tot;
+            const int r = rem / CPR, part = rem % CPR;
+            int t = idx_s[j0 + r];
+            if (t < 0 || t >= p.len) t = 0;  // masked below
+            const T* src = (which ? vbase : kbase) + (int64_t)t * kD;
+            cp_async16((which ? vs : ks) + r * kD * ES + part * 16,
+                       reinterpret_cast<const unsigned char*>(src) + part * 16);
+          }
         }
       }
+      if (MODE != kDense) cp_async_commit();
     };
 
-    if (warp == 0) {
-      if (nbatch > 0) issue(0);
-      if (nbatch > 1) issue(1);
+    // per-lane query slice: dims 4*lane .. 4*lane+3 of every head
+    float qreg[kQReg ? MAXG : 1][4];
+    if (kQReg) {
+#pragma unroll
+      for (int h = 0; h < (kQReg ? MAXG : 1); ++h) {
+        const float4 qq = *reinterpret_cast<const float4*>(qs + h * kD + 4 * lane);
+        qreg[h][0] = qq.x;
+        qreg[h][1] = qq.y;
+        qreg[h][2] = qq.z;
+        qreg[h][3] = qq.w;
+      }
     }
 
-    // per-thread P.V accumulators: quad of dims 4*lq .. 4*lq+3, row group warp
     float acc[MAXG][4];
 #pragma unroll
     for (int h = 0; h < MAXG; ++h)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[h][e] = 0.0f;
 
+    for (int s = 0; s < NST; ++s) issue(s);
+
     for (int bi = 0; bi < nbatch; ++bi) {
-      const int s = bi & 1;
+      const int s = bi % NST;
       const int j0 = bi * RB;
       const int nr = min(RB, n_mine - j0);
-      const T* ks = stage + (size_t)s * 2 * RB * kD;
-      const T* vs = ks + RB * kD;
-      mbar_wait(&bars[s], (uint32_t)((bi >> 1) & 1));
+      const unsigned char* ks = stage + (size_t)s * kStageBytes;
+      const unsigned char* vs = ks + RB * kD * ES;
+      if (MODE == kDense) {
+        mbar_wait(&bars[s], (uint32_t)((bi / NST) & 1));
+      } else {
+        if (NST == 2) cp_async_wait<1>();
+        else if (NST == 3) cp_async_wait<2>();
+        else cp_async_wait<3>();
+        __syncthreads();
+      }
 
-      // logits: 8 lanes per row, 16 dims per lane
-      for (int r = warp * 4 + (lane >> 3); r < RB; r += kSAWarps * 4) {
-        const int sub = lane & 7;
-        float kf[16];
-        const uint4* src = reinterpret_cast<const uint4*>(ks + r * kD + sub * 16);
-        if (ES == 2) {
-          float f8[8];
-          unpack16(src[0], f8, T());
+      // logits: RPW rows per warp; lane owns 4 dims; butterfly reduce
+      for (int rg = warp; rg * RPW < RB; rg += kSAWarps) {
+        float v[NV];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) kf[e] = f8[e];
-          unpack16(src[1], f8, T());
-#pragma unroll
-          for (int e = 0; e < 8; ++e) kf[8 + e] = f8[e];
-        } else {
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 u = src[c4];
-            kf[4 * c4 + 0] = __uint_as_float(u.x);
-            kf[4 * c4 + 1] = __uint_as_float(u.y);
-            kf[4 * c4 + 2] = __uint_as_float(u.z);
-            kf[4 * c4 + 3] = __uint_as_float(u.w);
+        for (int r = 0; r < RPW; ++r) {
+          const int rr = rg * RPW + r;
+          float kf[4];
+          if (ES == 2) {
+            const uint2 u = *reinterpret_cast<const uint2*>(ks + (rr * kD + 4 * lane) * ES);
+            kf[0] = __uint_as_float(u.x << 16);
+            kf[1] = __uint_as_float(u.x & 0xFFFF0000u);
+            kf[2] = __uint_as_float(u.y << 16);
+            kf[3] = __uint_as_float(u.y & 0xFFFF0000u);
+          } else {
+            const float4 u = *reinterpret_cast<const float4*>(ks + (rr * kD + 4 * lane) * ES);
+            kf[0] = u.x;
+            kf[1] = u.y;
+            kf[2] = u.z;
+            kf[3] = u.w;
           }
-        }
-        bool valid = r < nr;
-        if (MODE != kDense && valid) {
-          const int t = idx_s[j0 + r];
-          valid = t >= 0 && t < p.len;
-          if (MODE == kDecode && !valid) flag_status(FASA_ERR_BAD_INDEX);
-        }
 #pragma unroll
-        for (int h = 0; h < MAXG; ++h) {
-          if (h < G) {
-            const float4* qv = reinterpret_cast<const float4*>(qs + h * kD + sub * 16);
-            float a = 0.0f;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const float4 qq = qv[c4];
-              a = fmaf(qq.x, kf[4 * c4 + 0], a);
-              a = fmaf(qq.y, kf[4 * c4 + 1], a);
-              a = fmaf(qq.z, kf[4 * c4 + 2], a);
-              a = fmaf(qq.w, kf[4 * c4 + 3], a);
+          for (int h = 0; h < MAXG; ++h) {
+            float q0, q1, q2, q3;
+            if (kQReg) {
+              q0 = qreg[kQReg ? h : 0][0];
+              q1 = qreg[kQReg ? h : 0][1];
+              q2 = qreg[kQReg ? h : 0][2];
+              q3 = qreg[kQReg ? h : 0][3];
+            } else {
+              const float4 qq = *reinterpret_cast<const float4*>(qs + h * kD + 4 * lane);
+              q0 = qq.x;
+              q1 = qq.y;
+              q2 = qq.z;
+              q3 = qq.w;
             }
-            a += __shfl_xor_sync(0xFFFFFFFFu, a, 1);
-            a += __shfl_xor_sync(0xFFFFFFFFu, a, 2);
-            a += __shfl_xor_sync(0xFFFFFFFFu, a, 4);
-            if (sub == 0) zs[h * RB + r] = valid ? a : -INFINITY;
+            float a = q0 * kf[0];
+            a = fmaf(q1, kf[1], a);
+            a = fmaf(q2, kf[2], a);
+            v[h * RPW + r] = fmaf(q3, kf[3], a);
           }
+        }
+        // butterfly transpose-reduce: after it, lane l holds the full sum of
+        // item l mod NV (with NV = 16 the lane-bit-4 pairs are summed first)
+        if (NV == 16) {
+#pragma unroll
+          for (int j = 0; j < NV; ++j) v[j] += __shfl_xor_sync(0xFFFFFFFFu, v[j], 16);
+        }
+#pragma unroll
+        for (int w = NV / 2; w >= 1; w >>= 1) {
+          const bool upper = (lane & w) != 0;
+#pragma unroll
+          for (int j = 0; j < w; ++j) {
+            const float send = upper ? v[j] : v[j + w];
+            const float keep = upper ? v[j + w] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, w);
+          }
+        }
+        const int item = lane & (NV - 1);
+        const int h = item / RPW, rr = rg * RPW + item % RPW;
+        if (lane < NV && h < G) {
+          bool valid = rr < nr;
+          if (MODE != kDense && valid) {
+            const int t = idx_s[j0 + rr];
+            valid = t >= 0 && t < p.len;
+            if (MODE == kDecode && !valid) flag_status(FASA_ERR_BAD_INDEX);
+          }
+          zs[h * RB + rr] = valid ? v[0] : -INFINITY;
         }
       }
       __syncthreads();
@@ -505,7 +756,7 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
         }
       }
       __syncthreads();
-      // P.V: thread = (quad lane, row group warp)
+      // P.V: thread = (quad of dims = lane, row group = warp)
 #pragma unroll
       for (int h = 0; h < MAXG; ++h) {
         if (h < G) {
@@ -517,17 +768,17 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
       for (int r = warp; r < nr; r += kSAWarps) {
         float vf[4];
         if (ES == 2) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vs + r * kD + lane * 4);
+          const uint2 u = *reinterpret_cast<const uint2*>(vs + (r * kD + lane * 4) * ES);
           vf[0] = __uint_as_float(u.x << 16);
           vf[1] = __uint_as_float(u.x & 0xFFFF0000u);
           vf[2] = __uint_as_float(u.y << 16);
           vf[3] = __uint_as_float(u.y & 0xFFFF0000u);
         } else {
-          const uint4 u = *reinterpret_cast<const uint4*>(vs + r * kD + lane * 4);
-          vf[0] = __uint_as_float(u.x);
-          vf[1] = __uint_as_float(u.y);
-          vf[2] = __uint_as_float(u.z);
-          vf[3] = __uint_as_float(u.w);
+          const float4 u = *reinterpret_cast<const float4*>(vs + (r * kD + lane * 4) * ES);
+          vf[0] = u.x;
+          vf[1] = u.y;
+          vf[2] = u.z;
+          vf[3] = u.w;
         }
 #pragma unroll
         for (int h = 0; h < MAXG; ++h) {
@@ -538,41 +789,88 @@ __global__ void __launch_bounds__(kSAThreads, (MAXG <= 4 ? 2 : 1)) select_attend
           }
         }
       }
-      fence_proxy_async_smem();
-      __syncthreads();  // stage s fully consumed
-      if (warp == 0 && bi + 2 < nbatch) issue(bi + 2);
+      __syncthreads();  // stage s and zs fully consumed
+      issue(bi + NST);
     }
+    if (MODE != kDense) cp_async_wait<0>();
 
-    // reduce the 16 row groups into this CTA's partial o
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-      if (h < G) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) atomicAdd(&os[h * kD + lane * 4 + e], acc[h][e]);
-      }
-    }
+    // reduce the 16 row groups: per-warp partials through shared memory (the
+    // stage area is free now), heads in chunks that fit
+    float* part = reinterpret_cast<float*>(stage);
+    const int hc = min(MAXG, (NST * kStageBytes) / (kSAWarps * kD * 4));
     __syncthreads();
-    if (C > 1) cluster.sync();
-
-    // merge the cluster's partials; each CTA finishes a share of the outputs
-    T* out = static_cast<T*>(p.out) + ((int64_t)row * G) * kD;
-    for (int e = rank * kSAThreads + tid; e < G * kD; e += C * kSAThreads) {
-      const int h = e / kD, d = e % kD;
-      float M = -INFINITY;
-      for (int r = 0; r < C; ++r) M = fmaxf(M, cluster.map_shared_rank(ml, r)[h]);
-      float num = 0.0f, den = 0.0f;
-      if (M != -INFINITY) {
-        for (int r = 0; r < C; ++r) {
-          const float* mlr = cluster.map_shared_rank(ml, r);
-          const float mr = mlr[h];
-          const float w = (mr == -INFINITY) ? 0.0f : exp2f(mr - M);
-          den = fmaf(w, mlr[MAXG + h], den);
-          num = fmaf(w, cluster.map_shared_rank(os, r)[h * kD + d], num);
+    for (int h0 = 0; h0 < G; h0 += hc) {
+#pragma unroll
+      for (int h = 0; h < MAXG; ++h)
+        if (h >= h0 && h < h0 + hc && h < G)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) part[((h - h0) * kSAWarps + warp) * kD + lane * 4 + e] = acc[h][e];
+      __syncthreads();
+      for (int e = tid; e < hc * kD; e += kSAThreads) {
+        const int hh = e / kD, d = e % kD;
+        if (h0 + hh < G) {
+          float s = 0.0f;
+#pragma unroll
+          for (int w = 0; w < kSAWarps; ++w) s += part[(hh * kSAWarps + w) * kD + d];
+          acc_s[(h0 + hh) * kD + d] = s;
         }
       }
-      store_f(out + h * kD + d, den > 0.0f ? num / den : 0.0f);
+      __syncthreads();
     }
-    if (C > 1) cluster.sync();  // partials stay readable until everyone is done
+
+    T* out = static_cast<T*>(p.out) + ((int64_t)row * G) * kD;
+    if (C == 1) {
+      for (int e = tid; e < G * kD; e += kSAThreads) {
+        const float l = ml[MAXG + e / kD];
+        store_f(out + e, l > 0.0f ? acc_s[e] / l : 0.0f);
+      }
+      return;
+    }
+    if (!start_waited) {
+      cluster_wait();
+      start_waited = true;
+    }
+    // merge: (m, l) of every CTA to every CTA ...
+    if (tid < C * G) {
+      const int r = tid / G, h = tid % G;
+      float* dst = cluster.map_shared_rank(mlall, r);
+      dst[(rank * MAXG + h) * 2] = ml[h];
+      dst[(rank * MAXG + h) * 2 + 1] = ml[MAXG + h];
+    }
+    cluster_arrive();
+    cluster_wait();
+    // ... then each CTA adds its rescaled o into the owner of each output
+    if (tid < G) {
+      float M = -INFINITY;
+      for (int r = 0; r < C; ++r) M = fmaxf(M, mlall[(r * MAXG + tid) * 2]);
+      float lsum = 0.0f;
+      if (M != -INFINITY)
+        for (int r = 0; r < C; ++r) {
+          const float mr = mlall[(r * MAXG + tid) * 2];
+          if (mr != -INFINITY) lsum += exp2f(mr - M) * mlall[(r * MAXG + tid) * 2 + 1];
+        }
+      ml[3 * MAXG + tid] = (ml[tid] == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ml[tid] - M);
+      ml[2 * MAXG + tid] = lsum;
+    }
+    __syncthreads();
+    // each source CTA has its own slot in the owner, summed in rank order
+    // below, so the result does not depend on arrival order
+    const int per_owner = (G * kD + C - 1) / C;
+    for (int e = tid; e < G * kD; e += kSAThreads) {
+      const int owner = e / per_owner;
+      cluster.map_shared_rank(red, owner)[rank * per_owner + (e - owner * per_owner)] =
+          ml[3 * MAXG + e / kD] * acc_s[e];
+    }
+    cluster_arrive();
+    cluster_wait();
+    const int e0 = rank * per_owner, e1 = min(G * kD, e0 + per_owner);
+    for (int e = e0 + tid; e < e1; e += kSAThreads) {
+      float s = 0.0f;
+      for (int r = 0; r < C; ++r) s += red[r * per_owner + (e - e0)];
+      const float l = ml[2 * MAXG + e / kD];
+      store_f(out + e, l > 0.0f ? s / l : 0.0f);
+    }
+    // no DSMEM access follows the last cluster barrier
   }
 }
 

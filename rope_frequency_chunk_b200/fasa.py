@@ -47,6 +47,7 @@ _CP = ctypes.POINTER(fasa_cache)
 _SIGS = {
     "fasa_abi_version": (_I, []),
     "fasa_status_string": (ctypes.c_char_p, [_I]),
+    "fasa_last_cuda_error": (ctypes.c_char_p, []),
     "fasa_sketch_stride": (_I, [_I, _I]),
     "fasa_check_dom_idx": (_I, [_P, _I, _I]),
     "fasa_append_kv": (_I, [_CP, _P, _P, _I, _I, _P]),
@@ -78,7 +79,10 @@ def lib() -> ctypes.CDLL:
 
 def _check(status: int, call: str):
     if status != 0:
-        raise FasaError(status, call)
+        detail = ""
+        if status == 5:
+            detail = " (" + lib().fasa_last_cuda_error().decode() + ")"
+        raise FasaError(status, call + detail)
 
 
 def _stream(stream) -> int | None:
