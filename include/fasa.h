@@ -209,6 +209,38 @@ fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int
                         int32_t k, void* out, int32_t* idx_out, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream);
 
+/* Size of the library's own device scratch used by
+ * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the
+ * library until the process exits. */
+#define FASA_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * fasa_decode for callers that cannot allocate device memory. (The paper has
+ * no counterpart; this is a deployment convenience.) Some callers have no
+ * way to obtain a workspace: a plugin running inside a host framework that
+ * owns the whole device memory pool and hands its extensions no scratch, or
+ * a latency-critical path that must not call cudaMalloc (it may synchronize
+ * the device) and keeps no allocator of its own. This entry point computes
+ * exactly what fasa_decode computes, but its scratch is a fixed array inside
+ * the library (FASA_STATIC_SCRATCH_BYTES per device) instead of a caller
+ * workspace. It allocates nothing. The caller still passes all inputs and
+ * outputs.
+ *
+ *  - The first call on a device looks up that device's copy of the array
+ *    (with that device current); make that first call before any stream
+ *    capture. Later calls reuse the cached address.
+ *  - Every call on a device shares the one array and leaves its last
+ *    contents behind; calls whose kernels overlap on the GPU (different
+ *    streams, or different host threads) race on it and give wrong results.
+ *    Serialize them, e.g. on one stream.
+ *  - Rejects a call needing more than FASA_STATIC_SCRATCH_BYTES of scratch
+ *    (fasa_decode_workspace_bytes(cache, len)) with FASA_ERR_WORKSPACE,
+ *    before launching anything.
+ *  Other arguments and errors: as fasa_decode.
+ */
+fasa_status fasa_decode_static_scratch(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
+                                       int32_t k, void* out, int32_t* idx_out, cudaStream_t stream);
+
 /*
  * Dense full-KV decode, the comparison path: the same attention as
  * fasa_sparse_attend over all len cached rows (the upper bound in

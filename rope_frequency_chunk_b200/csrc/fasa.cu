@@ -15,6 +15,12 @@
 
 using namespace fasa;
 
+// Fixed scratch of fasa_decode_static_scratch: one copy per device, living as
+// long as the library is loaded. Host code must not use its address directly
+// (the host-side symbol is only a stand-in); the device address comes from
+// cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_scratch[FASA_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kMaxChunkKeys = 32768;  // keys per CTA held in shared memory
@@ -301,6 +307,24 @@ fasa_status launch_sa(const fasa_cache* c, SAParams p, int rows, bool pdl, cudaS
   }
 }
 
+// Device address of this device's g_static_scratch, looked up once per
+// device with that device current.
+void* g_static_scratch_addr[kMaxDevices] = {nullptr};
+
+fasa_status static_scratch_addr(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FASA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_status(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return FASA_OK;
+}
+
 size_t decode_ws(const fasa_cache* c, int32_t len) {
   const size_t b = (size_t)c->batch * c->n_kv_heads * (size_t)std::max(len, 0) * sizeof(float);
   return (b + 255) / 256 * 256 + 256;
@@ -465,6 +489,18 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
   return launch_sa<kDecode>(c, p, c->batch * c->n_kv_heads, true, stream, c->dtype, q_pos);
+}
+
+fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,
+                                       void* out, int32_t* idx_out, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (decode_ws(c, len) > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if ((s = static_scratch_addr(&ws)) != FASA_OK) return s;
+  return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);
 }
 
 fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, void* out,

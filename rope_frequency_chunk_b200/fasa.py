@@ -56,6 +56,7 @@ _SIGS = {
     "fasa_sparse_attend": (_I, [_CP, _I, _P, _I, _P, _I, _P, _P]),
     "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
     "fasa_device_status": (_I, [_I]),
 }
