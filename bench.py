@@ -272,7 +272,7 @@ def run_fasa(args, wl):
     n_layers = args.layers or default_layers(wl)
     caches, qs = build_stack(wl, n_layers, device)
     outs = [torch.empty_like(q) for q in qs]
-    ws = torch.empty(max(F.fasa_decode_workspace_bytes(c, wl.ctx_len) for c in caches), dtype=torch.uint8,
+    ws = torch.empty(max(F.fasa_decode_workspace_bytes(c, wl.ctx_len, k) for c in caches), dtype=torch.uint8,
                      device=device)
     stream = torch.cuda.Stream(device=device)
     L = wl.ctx_len

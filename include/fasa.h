@@ -188,19 +188,25 @@ fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, i
 fasa_status fasa_sparse_attend(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
                                const int32_t* idx, int32_t n_idx, void* out, cudaStream_t stream);
 
-/* Workspace bytes fasa_decode needs for this cache at cached length len. */
-size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len);
+/* Workspace bytes fasa_decode needs for this cache at cached length len and
+ * budget k (0 for invalid arguments). */
+size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t k);
 
 /*
  * One FASA decode step over a layer: TIP (fasa_score) -> T_t
- * (fasa_select_topk with k) -> FAC (fasa_sparse_attend), fused into two
- * launches; scores stay in the workspace and the kept indices stay on chip.
+ * (fasa_select_topk with k) -> FAC (fasa_sparse_attend). Four launches
+ * chained with programmatic dependent launch: the score stream, which also
+ * builds a per-row histogram of the score keys; a filter that marks the
+ * certainly-kept tokens and collects the tokens of the threshold bin; a
+ * per-row exact resolution of that bin that emits the kept indices in
+ * ascending order; and the focused attention. Scores, histogram and index
+ * lists live in the workspace.
  *
  *  out     : [B][Hq][128] dtype.
  *  idx_out : nullable; [B][Hkv][min(k, len)] int32, the kept tokens in
  *            ascending order.
  *  workspace : caller-owned device memory of at least
- *            fasa_decode_workspace_bytes(cache, len) bytes, 256-byte aligned;
+ *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned;
  *            its contents need no initialisation and are scratch.
  *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;
  *  FASA_ERR_WORKSPACE if the workspace is missing or too small.
@@ -234,7 +240,7 @@ fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int
  *    streams, or different host threads) race on it and give wrong results.
  *    Serialize them, e.g. on one stream.
  *  - Rejects a call needing more than FASA_STATIC_SCRATCH_BYTES of scratch
- *    (fasa_decode_workspace_bytes(cache, len)) with FASA_ERR_WORKSPACE,
+ *    (fasa_decode_workspace_bytes(cache, len, k)) with FASA_ERR_WORKSPACE,
  *    before launching anything.
  *  Other arguments and errors: as fasa_decode.
  */

@@ -12,6 +12,8 @@
 #include "fasa_device.cuh"
 #include "score.cuh"
 #include "select_attend.cuh"
+#include "select_hist.cuh"
+#include "attend_mma.cuh"
 
 using namespace fasa;
 
@@ -126,10 +128,10 @@ fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
 
 // ------------------------------------------------------------ score
 
-template <typename T, int LPT>
+template <typename T, int LPT, bool kHist>
 fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
-  auto kern = score_kernel<T, LPT>;
-  const int smem = kScoreStages * kScoreStageBytes;
+  auto kern = score_kernel<T, LPT, kHist>;
+  const int smem = kScoreStages * kScoreStageBytes + kHistBins * 4;
   int set = 0;
   fasa_status s = cached_int((const void*)kern, 0, &set, [&](int* v) {
     *v = 1;
@@ -142,22 +144,25 @@ fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t 
   return cuda_status(cudaGetLastError());
 }
 
-template <typename T>
+template <typename T, bool kHist>
 fasa_status launch_score_lpt(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
   const int lpt = p.stride * (int)sizeof(T) / 16;
   switch (lpt) {
-    case 1: return launch_score_t<T, 1>(p, d, st);
-    case 2: return launch_score_t<T, 2>(p, d, st);
-    case 4: return launch_score_t<T, 4>(p, d, st);
-    case 8: return launch_score_t<T, 8>(p, d, st);
-    case 16: return launch_score_t<T, 16>(p, d, st);
-    case 32: return launch_score_t<T, 32>(p, d, st);
+    case 1: return launch_score_t<T, 1, kHist>(p, d, st);
+    case 2: return launch_score_t<T, 2, kHist>(p, d, st);
+    case 4: return launch_score_t<T, 4, kHist>(p, d, st);
+    case 8: return launch_score_t<T, 8, kHist>(p, d, st);
+    case 16: return launch_score_t<T, 16, kHist>(p, d, st);
+    case 32: return launch_score_t<T, 32, kHist>(p, d, st);
     default: return FASA_ERR_UNSUPPORTED;
   }
 }
 
+// TIP scores for every (b, g, t < len); with `hist` also the per-row
+// histogram of the top 12 bits of each score's order-preserving key (added
+// into `hist`, which must be zero).
 fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
-                         cudaStream_t st) {
+                         uint32_t* hist, cudaStream_t st) {
   DevInfo d;
   fasa_status s = device_info(&d);
   if (s != FASA_OK) return s;
@@ -166,6 +171,7 @@ fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_
   p.q = q;
   p.dom_idx = c->dom_idx;
   p.scores = scores;
+  p.hist = hist;
   p.max_len = c->max_len;
   p.total = (int64_t)c->batch * c->n_kv_heads * len;
   p.len = len;
@@ -174,7 +180,9 @@ fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_
   p.group = c->n_q_heads / c->n_kv_heads;
   p.n_dom = c->n_dom;
   fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
-  return c->dtype == FASA_F32 ? launch_score_lpt<float>(p, d, st) : launch_score_lpt<__nv_bfloat16>(p, d, st);
+  if (c->dtype == FASA_F32)
+    return hist ? launch_score_lpt<float, true>(p, d, st) : launch_score_lpt<float, false>(p, d, st);
+  return hist ? launch_score_lpt<__nv_bfloat16, true>(p, d, st) : launch_score_lpt<__nv_bfloat16, false>(p, d, st);
 }
 
 // ---------------------------------------------------- select / attend
@@ -283,7 +291,7 @@ fasa_status launch_sa(const fasa_cache* c, SAParams p, int rows, bool pdl, cudaS
   if (C > kMaxCluster) return FASA_ERR_UNSUPPORTED;
   if (c) fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   if (MODE == kSelect || MODE == kDecode) choose_sampling(p);
-  p.n_stages = 4;
+  p.n_stages = (MODE == kDense) ? 4 : 2;
   for (;;) {
     p.chunk = (int)ceil_div(p.len, C);
     p.slice = (int)ceil_div(p.n_keep, C);
@@ -325,9 +333,58 @@ fasa_status static_scratch_addr(void** out) {
   return FASA_OK;
 }
 
-size_t decode_ws(const fasa_cache* c, int32_t len) {
-  const size_t b = (size_t)c->batch * c->n_kv_heads * (size_t)std::max(len, 0) * sizeof(float);
-  return (b + 255) / 256 * 256 + 256;
+// Decode workspace, each part 256-byte aligned:
+//   scores [rows][len] f32 | hist [rows][4096] u32 | cand_cnt [rows] u32 |
+//   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
+//   cand_idx [rows][cap] i32 | idx [rows][k_eff] i32 |
+//   part [rows][splits_max][kAttPartStride] f32
+// hist, cand_cnt and att_cnt are cleared at the start of every call.
+constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
+struct DecodeWs {
+  size_t scores, hist, cnt, att_cnt, bitmap, cand, idx, part, total;
+  int cap, words, splits_max;
+};
+inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+inline int att_chunks(int keff) { return (keff + kAttChunk - 1) / kAttChunk; }
+inline int att_splits(int rows, int keff, int sms) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(att_chunks(keff), ceil_div(2LL * sms, rows)));
+}
+DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
+  DecodeWs w;
+  const size_t rows = (size_t)c->batch * c->n_kv_heads;
+  const size_t L = (size_t)std::max(len, 0);
+  const int keff = std::max(0, std::min(k, len));
+  w.words = (int)((L + 31) / 32);
+  w.cap = (int)std::min<size_t>(std::max<size_t>(L, 1), 8192);
+  w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms);
+  w.scores = 0;
+  w.hist = al256(rows * L * 4);
+  w.cnt = w.hist + rows * kHistBins * 4;
+  w.att_cnt = w.cnt + rows * 4;
+  w.bitmap = al256(w.att_cnt + rows * 4);
+  w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
+  w.idx = al256(w.cand + rows * (size_t)w.cap * 4);
+  w.part = al256(w.idx + rows * (size_t)keff * 4);
+  w.total = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4) + 256;
+  return w;
+}
+size_t decode_ws(const fasa_cache* c, int32_t len, int32_t k) { return decode_layout(c, len, k).total; }
+
+// Plain launch with programmatic stream serialization (the kernel waits
+// for its predecessor with griddepcontrol.wait).
+template <typename K, typename P>
+fasa_status launch_pdl(K kern, dim3 grid, int threads, size_t smem, cudaStream_t st, const P& p) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
 }  // namespace
@@ -419,7 +476,7 @@ fasa_status fasa_score(const fasa_cache* c, int32_t len, const void* q, int32_t 
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (len == 0) return FASA_OK;
   if (!aligned(q, 16) || !aligned(scores, 4)) return FASA_ERR_INVALID_ARG;
-  return launch_score(c, len, q, q_pos, scores, stream);
+  return launch_score(c, len, q, q_pos, scores, nullptr, stream);
 }
 
 fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, int32_t k, int32_t* idx,
@@ -458,9 +515,9 @@ fasa_status fasa_sparse_attend(const fasa_cache* c, int32_t len, const void* q, 
   return launch_sa<kAttendIdx>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype, q_pos);
 }
 
-size_t fasa_decode_workspace_bytes(const fasa_cache* c, int32_t len) {
-  if (check_cache(c) != FASA_OK || len < 0) return 0;
-  return decode_ws(c, len);
+size_t fasa_decode_workspace_bytes(const fasa_cache* c, int32_t len, int32_t k) {
+  if (check_cache(c) != FASA_OK || len < 0 || k < 0) return 0;
+  return decode_ws(c, len, k);
 }
 
 fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k, void* out,
@@ -472,23 +529,110 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   if (len > FASA_MAX_LEN || k > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
   if (idx_out != nullptr && !aligned(idx_out, 4)) return FASA_ERR_INVALID_ARG;
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < decode_ws(c, len))
-    return FASA_ERR_WORKSPACE;
-  float* scores = static_cast<float*>(workspace);
-  if ((s = launch_score(c, len, q, q_pos, scores, stream)) != FASA_OK) return s;
+  const DecodeWs w = decode_layout(c, len, k);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return FASA_ERR_WORKSPACE;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return s;
+  char* base = static_cast<char*>(workspace);
+  float* scores = reinterpret_cast<float*>(base + w.scores);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + w.hist);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(base + w.cnt);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
+  int32_t* cand = reinterpret_cast<int32_t*>(base + w.cand);
+  int32_t* idx = reinterpret_cast<int32_t*>(base + w.idx);
+  const int rows = c->batch * c->n_kv_heads;
+  const int keff = std::min(k, len);
+
+  // 1. TIP scores and the per-row key histogram
+  uint32_t* att_cnt = reinterpret_cast<uint32_t*>(base + w.att_cnt);
+  float* part = reinterpret_cast<float*>(base + w.part);
+  if ((s = cuda_status(cudaMemsetAsync(hist, 0, w.bitmap - w.hist, stream))) != FASA_OK) return s;
+  if ((s = launch_score(c, len, q, q_pos, scores, hist, stream)) != FASA_OK) return s;
+
+  // 2. filter: certain tokens into the bitmap, threshold-bin tokens into the candidate list
+  FilterParams fp{};
+  fp.scores = scores;
+  fp.hist = hist;
+  fp.cand_cnt = cnt;
+  fp.cand_idx = cand;
+  fp.bitmap = bitmap;
+  fp.len = len;
+  fp.n_keep = keff;
+  fp.cap = w.cap;
+  const int64_t tiles_per_row = std::max<int64_t>(1, ceil_div(4LL * d.sms, rows));
+  fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 32) * 32);
+  fp.words = w.words;
+  if ((s = launch_pdl(filter_kernel, dim3((unsigned)ceil_div(len, fp.tile), (unsigned)rows, 1), kFilterThreads, 0,
+                      stream, fp)) != FASA_OK)
+    return s;
+
+  // 3. finalize: exact threshold among the candidates, kept indices in ascending order
+  FinalParams np{};
+  np.scores = scores;
+  np.hist = hist;
+  np.cand_cnt = cnt;
+  np.cand_idx = cand;
+  np.bitmap = bitmap;
+  np.idx = idx;
+  np.idx_out = idx_out;
+  np.len = len;
+  np.n_keep = keff;
+  np.cap = w.cap;
+  np.words = w.words;
+  np.scap = w.cap;
+  while (np.scap > 256 && final_smem_bytes(np.words, np.scap) > d.smem_optin) np.scap /= 2;
+  const int fsmem = final_smem_bytes(np.words, np.scap);
+  if (fsmem > d.smem_optin) return FASA_ERR_UNSUPPORTED;
+  int set = 0;
+  if ((s = cached_int((const void*)finalize_kernel, 0, &set, [&](int* v) {
+         *v = 1;
+         return cuda_status(
+             cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin));
+       })) != FASA_OK)
+    return s;
+  if ((s = launch_pdl(finalize_kernel, dim3((unsigned)rows, 1, 1), kSAThreads, (size_t)fsmem, stream, np)) !=
+      FASA_OK)
+    return s;
+
+  // 4. focused attention over the kept rows
+  if (c->dtype == FASA_BF16) {
+    AttParams ap{};
+    ap.k = static_cast<const __nv_bfloat16*>(c->k);
+    ap.v = static_cast<const __nv_bfloat16*>(c->v);
+    ap.idx = idx;
+    ap.q = static_cast<const __nv_bfloat16*>(q);
+    ap.out = static_cast<__nv_bfloat16*>(out);
+    ap.part = part;
+    ap.counter = att_cnt;
+    ap.max_len = c->max_len;
+    ap.len = len;
+    ap.n_keep = keff;
+    ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms));
+    ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
+    ap.splits = (int)ceil_div(keff, ap.slice);
+    ap.group = c->n_q_heads / c->n_kv_heads;
+    fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
+    if ((s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
+           *v = 1;
+           return cuda_status(
+               cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes()));
+         })) != FASA_OK)
+      return s;
+    return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
+                      (size_t)att_smem_bytes(), stream, ap);
+  }
   SAParams p{};
-  p.scores = scores;
-  p.idx_out = idx_out;
+  p.idx_in = idx;
   p.k = c->k;
   p.v = c->v;
   p.q = q;
   p.out = out;
   p.max_len = c->max_len;
   p.len = len;
-  p.n_keep = std::min(k, len);
+  p.n_keep = keff;
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
-  return launch_sa<kDecode>(c, p, c->batch * c->n_kv_heads, true, stream, c->dtype, q_pos);
+  return launch_sa<kAttendIdx>(c, p, rows, true, stream, c->dtype, q_pos);
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,
@@ -497,7 +641,7 @@ fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const v
   if (s != FASA_OK) return s;
   if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
-  if (decode_ws(c, len) > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
+  if (decode_ws(c, len, k) > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
   void* ws = nullptr;
   if ((s = static_scratch_addr(&ws)) != FASA_OK) return s;
   return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);

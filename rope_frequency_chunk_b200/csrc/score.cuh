@@ -11,9 +11,9 @@
 // power-of-two number of 16-byte chunks. The grid is persistent (one CTA per
 // SM) and splits the flattened (row, token) range evenly. A producer warp
 // streams the CTA's contiguous range through a ring of shared-memory stages
-// with 1-D bulk copies (TMA engine, full/empty mbarriers, no multicast); 16
-// consumer warps score the tokens, each token read from shared memory by LPT
-// lanes, one 16-byte chunk each. The first stages are in flight before the
+// with 1-D bulk copies (TMA engine, full/empty mbarriers, no multicast); 12
+// consumer warps score the tokens, one token per lane (two or four lanes for
+// rows wider than 32 elements). The first stages are in flight before the
 // query coefficients are computed.
 //
 // Arithmetic: float64. Each stored element e is widened exactly to the double
@@ -28,7 +28,7 @@
 
 namespace fasa {
 
-constexpr int kScoreConsumerWarps = 16;
+constexpr int kScoreConsumerWarps = 12;
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kScoreStages = 8;
 constexpr int kScoreStageBytes = 24576;
@@ -38,6 +38,7 @@ struct ScoreParams {
   const void* q;         // [B][Hq][128]
   const int32_t* dom_idx;
   float* scores;         // [rows][len]
+  uint32_t* hist;        // [rows][4096] key-histogram counts (added to), or null
   int64_t max_len;
   int64_t total;         // rows * len
   int32_t len;
@@ -63,10 +64,10 @@ __device__ __forceinline__ double widen_scaled_f32(uint32_t w) {
 }
 
 template <typename T>
-__device__ __forceinline__ double chunk_dot(const uint4& u, const double (&qr)[Elem<T>::kPer16]);
+__device__ __forceinline__ double chunk_dot(const uint4& u, const double* qr);
 
 template <>
-__device__ __forceinline__ double chunk_dot<__nv_bfloat16>(const uint4& u, const double (&qr)[8]) {
+__device__ __forceinline__ double chunk_dot<__nv_bfloat16>(const uint4& u, const double* qr) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
   double acc = 0.0;
 #pragma unroll
@@ -79,7 +80,7 @@ __device__ __forceinline__ double chunk_dot<__nv_bfloat16>(const uint4& u, const
   return acc;
 }
 template <>
-__device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double (&qr)[4]) {
+__device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double* qr) {
   double acc = 0.0;
   acc = fma(widen_scaled_f32(u.x), qr[0], acc);
   acc = fma(widen_scaled_f32(u.y), qr[1], acc);
@@ -88,15 +89,25 @@ __device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double 
   return acc;
 }
 
-template <typename T, int LPT>
+constexpr int kHistBits = 12;                 // key bits of the per-row score histogram
+constexpr int kHistBins = 1 << kHistBits;
+
+template <typename T, int LPT, bool kHist>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScoreParams p) {
-  constexpr int EPC = Elem<T>::kPer16;
-  constexpr int TPW = 32 / LPT;                 // tokens per warp load
+  constexpr int EPC = Elem<T>::kPer16;          // elements per 16-byte chunk
+  constexpr int ROWE = LPT * EPC;               // elements per sketch row
   constexpr int ROWB = LPT * 16;                // sketch row bytes
+  constexpr int LPT2 = ROWE > 32 ? ROWE / 32 : 1;  // lanes per token
+  constexpr int EPL = ROWE / LPT2;              // elements per lane (<= 32)
+  constexpr int CPL = EPL / EPC;                // chunks per lane
+  constexpr int TPW = 32 / LPT2;                // tokens per warp step
   constexpr int TPS = kScoreStageBytes / ROWB;  // tokens per stage
   constexpr int NCW = kScoreConsumerWarps;
-  extern __shared__ __align__(128) unsigned char ring[];  // kScoreStages x kScoreStageBytes
+  extern __shared__ __align__(128) unsigned char ring[];  // stages, then the histogram
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + (size_t)kScoreStages * kScoreStageBytes);
   __shared__ double s_q[kD];
+  __shared__ __align__(16) T s_qraw[FASA_MAX_GROUP * kD];  // the group's raw queries
+  __shared__ int s_dom[kNFC];
   __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
   __shared__ int st_row[kScoreStages], st_t0[kScoreStages], st_n[kScoreStages];
   grid_dependency_wait();
@@ -115,6 +126,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     }
     fence_mbar_init();
   }
+  if (kHist)
+    for (int i = tid; i < kHistBins; i += kScoreThreads) s_hist[i] = 0u;
   __syncthreads();
 
   if (warp == NCW) {
@@ -144,12 +157,27 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     return;
   }
 
-  // ---------------- consumers
-  const int sub = lane % LPT, tl = lane / LPT;
+  // ---------------- consumers: one token per lane (LPT2 lanes for wide rows)
+  const int sub = lane % LPT2;
+  // chunk rotation per lane so that a quarter-warp's 16-byte reads hit
+  // distinct banks; the lane's coefficients are rotated the same way
+  const int rot = (LPT2 == 1) ? ((lane * CPL / 8) % CPL) : (LPT2 == 2 ? ((lane / 2) % CPL) : 0);
   const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
-  double qr[EPC];
+  double qr[EPL];
   int cur_row = -1;
   float* out = p.scores;
+
+  auto flush_hist = [&](int row) {
+    // all consumer warps are between the two named barriers around this call
+    for (int i = tid; i < kHistBins; i += NCW * 32) {
+      const uint32_t v = s_hist[i];
+      if (v) {
+        atomicAdd(p.hist + (int64_t)row * kHistBins + i, v);
+        s_hist[i] = 0u;
+      }
+    }
+  };
+
   int64_t done = 0;
   for (int j = 0; done < n_tok; ++j) {
     const int b = j % kScoreStages;
@@ -158,15 +186,25 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     if (row != cur_row) {
       // new row: the group's rotated queries summed per sketch column (float64)
       named_barrier_sync(1, NCW * 32);
-      if (tid < p.stride) {
+      if (kHist && cur_row >= 0) flush_hist(cur_row);
+      {
+        // the group's queries and the head's dominant FCs, loaded in parallel
         const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
+        const uint4* qsrc =
+            reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD);
+        for (int c = tid; c < p.group * kD * (int)sizeof(T) / 16; c += NCW * 32)
+          reinterpret_cast<uint4*>(s_qraw)[c] = __ldg(qsrc + c);
+        if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
+      }
+      named_barrier_sync(1, NCW * 32);
+      if (tid < p.stride) {
         double acc = 0.0;
         const int jj = tid >> 1;
         if (jj < p.n_dom) {
-          const int i = p.dom_idx[g * p.n_dom + jj];
+          const int i = s_dom[jj];
           if (i >= 0 && i < kNFC) {
             const double c = p.cosv[i], s = p.sinv[i];
-            const T* qh = static_cast<const T*>(p.q) + ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD;
+            const T* qh = s_qraw;
             for (int h = 0; h < p.group; ++h) {
               const double x = to_float(qh[h * kD + i]);
               const double y = to_float(qh[h * kD + i + kNFC]);
@@ -182,24 +220,48 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
       }
       named_barrier_sync(1, NCW * 32);
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) qr[e] = s_q[sub * EPC + e];
+      for (int c = 0; c < CPL; ++c)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) qr[c * EPC + e] = s_q[(sub * CPL + (c + rot) % CPL) * EPC + e];
       cur_row = row;
-      out = p.scores + (int64_t)row * p.len + 0;
+      out = p.scores + (int64_t)row * p.len;
     }
     const unsigned char* buf = ring + (size_t)b * kScoreStageBytes;
-    const int ngroups = (n + TPW - 1) / TPW;
-    for (int gi = warp; gi < ngroups; gi += NCW) {
-      const int t = gi * TPW + tl;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < n) v = *reinterpret_cast<const uint4*>(buf + t * ROWB + sub * 16);
-      double acc = chunk_dot<T>(v, qr);
+    for (int gi = warp; gi * TPW < n; gi += NCW) {
+      const int t = gi * TPW + lane / LPT2;
+      const bool valid = t < n;
+      uint4 v[CPL];
 #pragma unroll
-      for (int off = LPT / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-      if (sub == 0 && t < n) out[t0 + t] = (float)acc;
+      for (int c = 0; c < CPL; ++c)
+        v[c] = valid ? *reinterpret_cast<const uint4*>(buf + t * ROWB + (sub * CPL + (c + rot) % CPL) * 16)
+                     : make_uint4(0, 0, 0, 0);
+      double part[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) part[c] = chunk_dot<T>(v[c], qr + c * EPC);
+      double acc = part[0];
+#pragma unroll
+      for (int c = 1; c < CPL; ++c) acc += part[c];
+#pragma unroll
+      for (int off = LPT2 / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+      const float sc = (float)acc;
+      const bool writer = valid && sub == 0;
+      if (writer) out[t0 + t] = sc;
+      if (kHist) {
+        const uint32_t bin = score_key(sc) >> (32 - kHistBits);
+        const unsigned act = __ballot_sync(0xFFFFFFFFu, writer);
+        if (writer) {
+          const unsigned peers = __match_any_sync(act, bin);
+          if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
+        }
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[b]);
     done += n;
+  }
+  if (kHist && cur_row >= 0) {
+    named_barrier_sync(1, NCW * 32);
+    flush_hist(cur_row);
   }
 }
 

@@ -51,6 +51,7 @@ enum SAMode { kSelect = 0, kDecode = 1, kAttendIdx = 2, kDense = 3 };
 
 struct SAParams {
   const float* scores;       // [rows][len]
+  const uint32_t* hist;      // [rows][4096] histogram of the top 12 key bits, or null
   int32_t* idx_out;          // [rows][n_keep] or null
   const int32_t* idx_in;     // [rows][n_keep] (kAttendIdx)
   const void* k;             // [rows][max_len][128]
@@ -161,25 +162,27 @@ __device__ __forceinline__ uint32_t warp_offsets_serial(uint32_t* misc, int base
 // prefix must still be taken (ties to the lower position). With kCluster the
 // per-pass histograms are summed over the cluster in the leader's shared
 // memory.
-template <bool kCluster>
-__device__ void ballot_radix(const uint32_t* keys, int n, int k, int passes, uint32_t* rscr, uint32_t* chist,
-                             cg::cluster_group& cluster, uint32_t& out_prefix, int& out_krem) {
+template <bool kCluster, typename KeyAt>
+__device__ void ballot_radix_fn(KeyAt key_at, int n, int k, uint32_t prefix, int known, int stop, uint32_t* rscr,
+                                uint32_t* chist, cg::cluster_group& cluster, uint32_t& out_prefix, int& out_krem) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t* tot = rscr + kSAWarps * 256;
   uint32_t* bc = tot + 256;
-  uint32_t prefix = 0u, pmask = 0u;
+  uint32_t pmask = known ? ~0u << (32 - known) : 0u;
   int krem = k;
-  for (int pass = 0; pass < passes; ++pass) {
-    const int shift = 24 - 8 * pass;
+  for (int pass = 0; known < stop; ++pass) {
+    const int width = min(8, stop - known);
+    const int shift = 32 - known - width;
+    known += width;
     uint32_t cnt[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     for (int base = warp * 32; base < n; base += kSAThreads) {
       const int i = base + lane;
       bool act = false;
       uint32_t d = 0u;
       if (i < n) {
-        const uint32_t x = keys[i];
+        const uint32_t x = key_at(i);
         act = (x & pmask) == prefix;
-        d = (x >> shift) & 255u;
+        d = (x >> shift) & ((1u << width) - 1u);
       }
       unsigned b[8];
       const unsigned a = __ballot_sync(0xFFFFFFFFu, act);
@@ -247,11 +250,69 @@ __device__ void ballot_radix(const uint32_t* keys, int n, int k, int passes, uin
     }
     __syncthreads();
     prefix |= bc[0] << shift;
-    pmask |= 255u << shift;
+    pmask |= ((1u << width) - 1u) << shift;
     krem -= (int)bc[1];
   }
   out_prefix = prefix;
   out_krem = krem;
+}
+
+// From a row's 4096-bin histogram of the top 12 key bits, the bin holding
+// the k-th largest key and the number of keys in higher bins. Block-wide
+// suffix scan: thread t owns bins 4095-8t .. 4088-8t.
+__device__ __forceinline__ void hist_threshold(const uint32_t* h, int k, uint32_t* scan, uint32_t& bin,
+                                               uint32_t& above) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t c[8], sum = 0u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    c[u] = __ldcg(h + 4095 - (8 * tid + u));
+    sum += c[u];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < kSAWarps ? scan[lane] : 0u;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, w, off);
+      if (lane >= off) w += v;
+    }
+    if (lane < kSAWarps) scan[16 + lane] = w;
+  }
+  __syncthreads();
+  incl += warp > 0 ? scan[16 + warp - 1] : 0u;
+  const uint32_t excl = incl - sum;
+  if (excl < (uint32_t)k && (uint32_t)k <= incl) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (acc + c[u] >= (uint32_t)k) {
+        scan[32] = 4095u - (uint32_t)(8 * tid + u);
+        scan[33] = acc;
+        break;
+      }
+      acc += c[u];
+    }
+  }
+  __syncthreads();
+  bin = scan[32];
+  above = scan[33];
+  __syncthreads();
+}
+
+template <bool kCluster>
+__device__ __forceinline__ void ballot_radix(const uint32_t* keys, int n, int k, uint32_t prefix, int known, int stop,
+                                             uint32_t* rscr, uint32_t* chist, cg::cluster_group& cluster,
+                                             uint32_t& out_prefix, int& out_krem) {
+  ballot_radix_fn<kCluster>([keys](int i) { return keys[i]; }, n, k, prefix, known, stop, rscr, chist, cluster,
+                            out_prefix, out_krem);
 }
 
 // Unrolled coalesced load of n score keys (global float -> order-preserving key).
@@ -347,21 +408,35 @@ __global__ void __launch_bounds__(kSAThreads, 1) select_attend_kernel(const SAPa
     const int n_loc = max(0, min(p.chunk, p.len - start));
     const float* srow = p.scores + (int64_t)row * p.len;
     load_keys(keys, srow + start, n_loc);
-    const int s_str = p.sample_stride;
-    const int m = (p.len + s_str - 1) / s_str;
-    const bool use_samples = p.sample_rank < m;
-    if (use_samples)
-      for (int i = tid; i < m; i += kSAThreads) samples[i] = score_key(__ldcg(srow + (int64_t)i * s_str));
-    __syncthreads();
-
-    // 1. threshold from the sample: the top 16 bits of its j-th largest key
-    uint32_t t_lo = 0u;
-    if (use_samples) {
-      uint32_t pre;
-      int kr;
-      ballot_radix<false>(samples, m, p.sample_rank, 2, rscr, chist, cluster, pre, kr);
-      t_lo = pre;
+    // 1. threshold t_lo <= the k_eff-th key. With the score kernel's key
+    //    histogram it is the lower edge of the bin holding that key (exact:
+    //    the leader then only resolves the low 20 bits); otherwise the top 16
+    //    bits of the j-th largest of a strided sample of the row.
+    uint32_t t_lo = 0u, lead_prefix = 0u;
+    int lead_known = 0, lead_k = p.n_keep;
+    if (p.hist != nullptr) {
+      __syncthreads();
+      uint32_t bin, above;
+      hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, misc + kMiscScan, bin, above);
+      t_lo = bin << 20;
+      lead_prefix = t_lo;
+      lead_known = 12;
+      lead_k = p.n_keep - (int)above;
+    } else {
+      const int s_str = p.sample_stride;
+      const int m = (p.len + s_str - 1) / s_str;
+      const bool use_samples = p.sample_rank < m;
+      if (use_samples)
+        for (int i = tid; i < m; i += kSAThreads) samples[i] = score_key(__ldcg(srow + (int64_t)i * s_str));
+      __syncthreads();
+      if (use_samples) {
+        uint32_t pre;
+        int kr;
+        ballot_radix<false>(samples, m, p.sample_rank, 0u, 0, 16, rscr, chist, cluster, pre, kr);
+        t_lo = pre;
+      }
     }
+    __syncthreads();
 
     // 2. count local keys >= t_lo by warp segments (index order)
     const int seg = ((n_loc + kSAWarps * 32 - 1) / (kSAWarps * 32)) * 32;
@@ -421,7 +496,8 @@ __global__ void __launch_bounds__(kSAThreads, 1) select_attend_kernel(const SAPa
       if (rank == 0) {
         // exact k_eff-th key among the candidates; the kept list is the
         // candidates above it and the first `quota` equal to it
-        ballot_radix<false>(cand_key, (int)total, p.n_keep, 4, rscr, chist, cluster, thr, quota);
+        ballot_radix<false>(cand_key, (int)total, lead_k, lead_prefix, lead_known, 32, rscr, chist, cluster, thr,
+                            quota);
         const int n = (int)total;
         const int cseg = ((n + kSAWarps * 32 - 1) / (kSAWarps * 32)) * 32;
         const int cs = min(n, warp * cseg), ce = min(n, cs + cseg);
@@ -471,7 +547,7 @@ __global__ void __launch_bounds__(kSAThreads, 1) select_attend_kernel(const SAPa
       }
     } else {
       // exact fallback over all keys, histograms summed across the cluster
-      ballot_radix<true>(keys, n_loc, p.n_keep, 4, rscr, chist, cluster, thr, quota);
+      ballot_radix<true>(keys, n_loc, p.n_keep, 0u, 0, 32, rscr, chist, cluster, thr, quota);
       uint32_t cgt = 0u, ceq = 0u;
       for (int base = ws; base < we; base += 32) {
         const int i = base + lane;

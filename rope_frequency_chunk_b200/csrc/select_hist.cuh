@@ -1,0 +1,243 @@
+// Critical-set selection for the fused decode, from the score kernel's
+// per-row key histogram.
+//
+// "FASA: Frequency-aware Sparse Attention" (gist.science technical summary,
+// §2, FAC first bullet): T_t is the set of the k highest-scoring tokens
+// (ties to the lower index; k_eff = min(k, L)). Two kernels:
+//
+//  filter   (grid: token tiles x rows) The row's 4096-bin histogram of the
+//           top 12 bits of the order-preserving score keys gives the bin b1
+//           holding the k_eff-th key and the count of keys above it. Keys in
+//           higher bins are certainly kept: each warp writes the bitmap word
+//           of its 32 consecutive tokens (every word of [0, len) is written
+//           exactly once, so the bitmap needs no clearing). Keys in bin b1
+//           are appended to the row's candidate list.
+//  finalize (grid: rows) Exact k_eff-th key among the candidates (radix
+//           select on the low 20 bits, digit histograms counted with warp
+//           ballots); ties at it go to the lower token index. Their bits
+//           are added to the bitmap, and the kept indices are emitted in
+//           ascending order by a popcount scan of the bitmap. If the
+//           candidate list overflowed, the row is resolved exactly from all
+//           its scores instead (slow, rare).
+#pragma once
+
+#include "select_attend.cuh"
+
+namespace fasa {
+
+constexpr int kFilterThreads = kSAThreads;  // hist_threshold assumes 512 threads
+
+struct FilterParams {
+  const float* scores;      // [rows][len]
+  const uint32_t* hist;     // [rows][4096]
+  uint32_t* cand_cnt;       // [rows], zero before the launch
+  int32_t* cand_idx;        // [rows][cap]
+  uint32_t* bitmap;         // [rows][words]
+  int32_t len;
+  int32_t n_keep;           // k_eff
+  int32_t cap;
+  int32_t tile;             // tokens per CTA, a multiple of 32
+  int32_t words;            // ceil(len / 32)
+};
+
+__global__ void __launch_bounds__(kFilterThreads) filter_kernel(const FilterParams p) {
+  __shared__ uint32_t scan[64];
+  grid_dependency_wait();
+  const int row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t bin, above;
+  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);
+  const int t0 = blockIdx.x * p.tile;
+  const int t1 = min(p.len, t0 + p.tile);
+  const float* s = p.scores + (int64_t)row * p.len;
+  uint32_t* bm = p.bitmap + (int64_t)row * p.words;
+  int32_t* cidx = p.cand_idx + (int64_t)row * p.cap;
+  constexpr int U = 8;  // loads in flight per lane
+  for (int base0 = t0 + warp * 32; base0 < t1; base0 += kFilterThreads * U) {
+    float f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base0 + u * kFilterThreads + lane;
+      f[u] = i < t1 ? __ldcg(s + i) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int base = base0 + u * kFilterThreads;
+      if (base >= t1) break;  // warp-uniform
+      const int i = base + lane;
+      const bool v = i < t1;
+      const uint32_t b = score_key(f[u]) >> 20;
+      const unsigned def = __ballot_sync(0xFFFFFFFFu, v && b > bin);
+      const unsigned cnd = __ballot_sync(0xFFFFFFFFu, v && b == bin);
+      if (lane == 0) bm[base >> 5] = def;
+      if (cnd) {
+        uint32_t at = 0u;
+        if (lane == 0) at = atomicAdd(p.cand_cnt + row, (uint32_t)__popc(cnd));
+        at = __shfl_sync(0xFFFFFFFFu, at, 0) + __popc(cnd & lt);
+        if (((cnd >> lane) & 1u) && at < (uint32_t)p.cap) cidx[at] = i;
+      }
+    }
+  }
+}
+
+struct FinalParams {
+  float* scores;            // [rows][len]; the slow path turns a row into keys in place
+  const uint32_t* hist;
+  const uint32_t* cand_cnt;
+  const int32_t* cand_idx;  // [rows][cap]
+  const uint32_t* bitmap;   // [rows][words]
+  int32_t* idx;             // [rows][n_keep]
+  int32_t* idx_out;         // [rows][n_keep] or null
+  int32_t len;
+  int32_t n_keep;
+  int32_t cap;              // candidate list capacity
+  int32_t scap;             // candidates held in shared memory
+  int32_t words;
+};
+
+__host__ __device__ inline int final_smem_bytes(int words, int scap) {
+  return sa_align(words * 4, 128) + (kSAWarps * 256 + 264) * 4 + 64 * 4 + 2 * scap * 4;
+}
+
+__global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  grid_dependency_wait();
+  cg::cluster_group cluster = cg::this_cluster();  // a cluster of one; radix helpers take it
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + sa_align(p.words * 4, 128));
+  uint32_t* scan = rscr + kSAWarps * 256 + 264;
+  uint32_t* ckey = scan + 64;                           // [scap]
+  int32_t* cidx = reinterpret_cast<int32_t*>(ckey + p.scap);  // [scap]
+
+  uint32_t bin, above;
+  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);
+  const int krem = p.n_keep - (int)above;
+  const uint32_t n_c = __ldcg(p.cand_cnt + row);
+  const uint32_t* gbm = p.bitmap + (int64_t)row * p.words;
+
+  if (n_c <= (uint32_t)p.cap && n_c <= (uint32_t)p.scap) {
+    for (int w = tid; w < p.words; w += kSAThreads) bm[w] = __ldcg(gbm + w);
+    const float* s = p.scores + (int64_t)row * p.len;
+    const int32_t* gc0 = p.cand_idx + (int64_t)row * p.cap;
+    constexpr int U = 4;
+    for (int j0 = tid; j0 < (int)n_c; j0 += kSAThreads * U) {
+      int t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) t[u] = j0 + u * kSAThreads < (int)n_c ? __ldcg(gc0 + j0 + u * kSAThreads) : 0;
+      float f[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) f[u] = j0 + u * kSAThreads < (int)n_c ? __ldcg(s + t[u]) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (j0 + u * kSAThreads < (int)n_c) {
+          cidx[j0 + u * kSAThreads] = t[u];
+          ckey[j0 + u * kSAThreads] = score_key(f[u]);
+        }
+    }
+    const int32_t* gc = cidx;
+    auto key_of = [ckey](int j) { return ckey[j]; };
+    __syncthreads();
+    uint32_t thr;
+    int quota;
+    ballot_radix_fn<false>(key_of, (int)n_c, krem, bin << 20, 12, 32, rscr, nullptr, cluster, thr, quota);
+    // how many candidates tie at thr: keep all of them, or the `quota` with
+    // the lowest indices
+    uint32_t neq = 0u;
+    for (int base = warp * 32; base < (int)n_c; base += kSAThreads) {
+      const int j = base + lane;
+      neq += __popc(__ballot_sync(0xFFFFFFFFu, j < (int)n_c && key_of(j) == thr));
+    }
+    if (lane == 0) scan[warp] = neq;
+    __syncthreads();
+    uint32_t eq_total = 0u;
+#pragma unroll
+    for (int w = 0; w < kSAWarps; ++w) eq_total += scan[w];
+    __syncthreads();
+    uint32_t thr2 = 0u;
+    if ((int)eq_total > quota) {
+      // the tied candidates with the lowest indices: the largest ~index
+      auto tie_key = [key_of, gc, thr](int j) { return key_of(j) == thr ? ~(uint32_t)gc[j] : 0u; };
+      int q2;
+      ballot_radix_fn<false>(tie_key, (int)n_c, quota, 0u, 0, 32, rscr, nullptr, cluster, thr2, q2);
+    }
+    for (int j = tid; j < (int)n_c; j += kSAThreads) {
+      const uint32_t x = key_of(j);
+      const int t = gc[j];
+      const bool keep = x > thr || (x == thr && ((int)eq_total <= quota || ~(uint32_t)t >= thr2));
+      if (keep) atomicOr(&bm[t >> 5], 1u << (t & 31));
+    }
+  } else {
+    // slow exact path: this row's scores become keys in place, then a radix
+    // select over all of them, then the bitmap from scratch in index order
+    uint32_t* keys = reinterpret_cast<uint32_t*>(p.scores + (int64_t)row * p.len);
+    for (int i = tid; i < p.len; i += kSAThreads) keys[i] = score_key(__ldcg(p.scores + (int64_t)row * p.len + i));
+    __threadfence_block();
+    __syncthreads();
+    uint32_t thr;
+    int quota;
+    ballot_radix<false>(keys, p.len, p.n_keep, 0u, 0, 32, rscr, nullptr, cluster, thr, quota);
+    // equal keys per warp range of words, in index order
+    const int wseg = (p.words + kSAWarps - 1) / kSAWarps;
+    const int w0 = min(p.words, warp * wseg), w1 = min(p.words, w0 + wseg);
+    uint32_t neq = 0u;
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      neq += __popc(__ballot_sync(0xFFFFFFFFu, i < p.len && keys[i] == thr));
+    }
+    if (lane == 0) scan[warp] = neq;
+    __syncthreads();
+    uint32_t er = 0u;
+    for (int w = 0; w < warp; ++w) er += scan[w];
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      const bool v = i < p.len;
+      const uint32_t x = v ? keys[i] : 0u;
+      const unsigned gt = __ballot_sync(0xFFFFFFFFu, v && x > thr);
+      const unsigned eq = __ballot_sync(0xFFFFFFFFu, v && x == thr);
+      const bool take_eq = ((eq >> lane) & 1u) && (int)(er + __popc(eq & lt)) < quota;
+      const unsigned te = __ballot_sync(0xFFFFFFFFu, take_eq);
+      if (lane == 0) bm[w] = gt | te;
+      er += __popc(eq);
+    }
+  }
+  __syncthreads();
+
+  // emit the kept indices in ascending order: popcount scan of the bitmap
+  const int per = (p.words + kSAThreads - 1) / kSAThreads;
+  const int wb = min(p.words, tid * per), we_ = min(p.words, wb + per);
+  uint32_t cnt = 0u;
+  for (int w = wb; w < we_; ++w) cnt += __popc(bm[w]);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) scan[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0u;
+  for (int w = 0; w < warp; ++w) before += scan[w];
+  uint32_t pos = before + incl - cnt;
+  int32_t* out = p.idx + (int64_t)row * p.n_keep;
+  int32_t* out2 = p.idx_out ? p.idx_out + (int64_t)row * p.n_keep : nullptr;
+  for (int w = wb; w < we_; ++w) {
+    uint32_t m = bm[w];
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1;
+      if (pos < (uint32_t)p.n_keep) {
+        out[pos] = w * 32 + bit;
+        if (out2) out2[pos] = w * 32 + bit;
+      } else {
+        flag_status(FASA_ERR_BAD_INDEX);
+      }
+      ++pos;
+    }
+  }
+}
+
+}  // namespace fasa

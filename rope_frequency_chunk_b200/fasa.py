@@ -54,7 +54,7 @@ _SIGS = {
     "fasa_score": (_I, [_CP, _I, _P, _I, _P, _P]),
     "fasa_select_topk": (_I, [_P, _I, _I, _I, _P, _P]),
     "fasa_sparse_attend": (_I, [_CP, _I, _P, _I, _P, _I, _P, _P]),
-    "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
+    "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I]),
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
@@ -201,8 +201,8 @@ def fasa_sparse_attend(cache: KVCache, length: int, q, q_pos: int, idx, out=None
     return out
 
 
-def fasa_decode_workspace_bytes(cache: KVCache, length: int) -> int:
-    return int(lib().fasa_decode_workspace_bytes(cache.ref(), length))
+def fasa_decode_workspace_bytes(cache: KVCache, length: int, k: int) -> int:
+    return int(lib().fasa_decode_workspace_bytes(cache.ref(), length, k))
 
 
 def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, idx_out=None,
@@ -214,7 +214,7 @@ def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, id
     _dev(out, "out", cache.dtype)
     if idx_out is not None:
         _dev(idx_out, "idx_out", torch.int32)
-    need = fasa_decode_workspace_bytes(cache, length)
+    need = fasa_decode_workspace_bytes(cache, length, k)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _dev(workspace, "workspace", torch.uint8)

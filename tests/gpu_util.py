@@ -133,6 +133,18 @@ def check_out(wl, gpu_out, ref_out):
     return max(excess, 0.0)
 
 
+def check_gpu_pair(wl, a_stored, b_stored):
+    """Two GPU outputs of the same attention (different kernels or orders):
+    each holds one final rounding, so they may differ by two half-ulps plus
+    float32 accumulation error, which is bounded by 1e-3 of the row's rms."""
+    a = W.stored_to_f64(a_stored)
+    b = W.stored_to_f64(b_stored)
+    hu = half_ulp(np.maximum(np.abs(a), np.abs(b)), wl.dtype)
+    row = np.sqrt(np.mean(b ** 2, axis=-1, keepdims=True))
+    excess = np.max((np.abs(a - b) - 2 * hu) / (row + 1e-30))
+    assert excess <= 1e-3, f"outputs differ by {excess} of the row rms beyond rounding"
+
+
 def check_decode_heads(wl, inp, cache, q, k, heads, out, idx_out, scores_gpu=None, length=None):
     """Fused decode vs oracle on the given heads; returns worst output error."""
     L = length or wl.ctx_len

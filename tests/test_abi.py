@@ -90,7 +90,7 @@ def test_call_validation_without_launch(L):
     assert L.fasa_sparse_attend(c, 10, 0x50000, 10, 0x60000, 0, 0x70000, None) == 1   # n_idx < 1
     assert L.fasa_decode(c, 0, 0x50000, 0, 8, 0x70000, None, 0x80000, 1 << 20, None) == 1
     assert L.fasa_decode(c, 100, 0x50000, 100, 8, 0x70000, None, None, 1 << 20, None) == 4
-    need = L.fasa_decode_workspace_bytes(c, 100)
+    need = L.fasa_decode_workspace_bytes(c, 100, 8)
     assert need >= 2 * 100 * 4
     assert L.fasa_decode(c, 100, 0x50000, 100, 8, 0x70000, None, 0x80000, need - 1, None) == 4
     assert L.fasa_dense_decode(c, 0, 0x50000, 0, 0x70000, None) == 1

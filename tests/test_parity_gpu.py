@@ -161,7 +161,7 @@ def test_decode_budget_edges(k_of_L):
     U.check_decode_heads(wl, inp, cache, q, k, U.all_heads(wl), out, idx)
     if k >= L:  # keeping every token is dense attention
         dense = F.fasa_dense_decode(cache, L, q, L)
-        assert U.ulp_diff_bf16(U.stored(out), U.stored(dense)).max() <= 1
+        U.check_gpu_pair(wl, U.stored(out), U.stored(dense))
 
 
 def test_decode_single_token_cache():
@@ -178,7 +178,7 @@ def test_decode_all_fc_full_budget_is_dense():
     inp, cache, q = U.build(wl)
     out, idx = _decode(wl, cache, q, wl.k)
     dense = F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos)
-    assert U.ulp_diff_bf16(U.stored(out), U.stored(dense)).max() <= 1
+    U.check_gpu_pair(wl, U.stored(out), U.stored(dense))
 
 
 def test_decode_with_tied_tokens():
@@ -204,7 +204,7 @@ def test_decode_with_tied_tokens():
 def test_decode_is_deterministic_and_capturable():
     wl = SMALL["c2_ragged"]
     inp, cache, q = U.build(wl)
-    ws = torch.empty(F.fasa_decode_workspace_bytes(cache, wl.ctx_len), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(F.fasa_decode_workspace_bytes(cache, wl.ctx_len, wl.k), dtype=torch.uint8, device="cuda")
     out1 = torch.empty_like(q)
     F.fasa_decode(cache, wl.ctx_len, q, wl.q_pos, wl.k, out=out1, workspace=ws)
     s = torch.cuda.Stream()

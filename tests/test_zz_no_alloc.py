@@ -35,7 +35,7 @@ def test_static_scratch_decode_matches_workspace_decode():
     F.fasa_append_kv(cache, W.to_torch(inp.k, "cuda"), W.to_torch(inp.v, "cuda"), 0)
     L = wl.ctx_len
     lib = F.lib()
-    assert lib.fasa_decode_workspace_bytes(cache.ref(), L) <= (64 << 20)
+    assert lib.fasa_decode_workspace_bytes(cache.ref(), L, wl.k) <= (64 << 20)
     for step in range(2):  # two calls in a row share the library's scratch
         q = W.to_torch(np.stack([np.concatenate([W.head_q(wl, inp.params, 0, b, g, step=step)
                                                  for g in range(wl.n_kv_heads)]) for b in range(wl.batch)]),
