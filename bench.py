@@ -291,6 +291,7 @@ def run_fasa(args, wl):
         for c, q, o in zip(caches, qs, outs):
             F.fasa_dense_decode(c, L, q, wl.q_pos, out=o)
 
+    plan = F.fasa_decode_path(caches[0], L, k)
     hbm_peak, peak_kind = peaks()
     with ClockSampler(local) as clk:
         ms = time_graph(decode_step, args.steps, args.warmup, stream, dist)
@@ -305,9 +306,21 @@ def run_fasa(args, wl):
     us_layer = 1e3 * ms_step / n_layers
     gbs = world * step_bytes / (ms_step * 1e-3) / 1e9
 
-    # dominant kernel (TIP score stream), timed alone on the same stack
-    ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
-    score_gbs = sketch_bytes(wl) * n_layers / (ms_score * 1e-3) / 1e9
+    # dominant kernel: the single-launch decode is the whole step; the staged
+    # plan's is the TIP score stream, timed alone on the same stack
+    fused = plan == F.DECODE_FUSED
+    if fused:
+        roof = {"bound": "hbm", "kernel": "decode_fused_kernel (score + select + attend, one launch per layer)",
+                "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / world / hbm_peak,
+                "traffic": None, "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind,
+                "us_per_launch": us_layer}
+    else:
+        ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
+        score_gbs = sketch_bytes(wl) * n_layers / (ms_score * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "score_kernel (TIP sketch stream)", "achieved": score_gbs,
+                "peak": hbm_peak, "unit": "GB/s", "frac": score_gbs / hbm_peak,
+                "traffic": None, "bytes_per_launch": sketch_bytes(wl), "peak_kind": peak_kind,
+                "us_per_launch": 1e3 * ms_score / n_layers}
 
     extra = {}
     if not args.no_dense:
@@ -351,12 +364,11 @@ def run_fasa(args, wl):
         "decode_roofline": {"achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
                             "frac": gbs / world / hbm_peak, "bytes_per_layer_step": per_layer_bytes,
                             "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "score_kernel (TIP sketch stream)", "achieved": score_gbs,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": score_gbs / hbm_peak,
-                     "traffic": None, "bytes_per_launch": sketch_bytes(wl), "peak_kind": peak_kind,
-                     "us_per_launch": 1e3 * ms_score / n_layers},
+        "roofline": roof,
+        "decode_plan": "fused" if fused else "staged",
         "clocks": clocks,
-        "gpu_launches": 2 * n_layers * args.steps,
+        # kernels of this library per layer: fused 1; staged 4 (score, filter, finalize, attend)
+        "gpu_launches": (1 if fused else 4) * n_layers * args.steps,
         "e2e": e2e,
     }
     line.update(extra)

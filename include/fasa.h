@@ -194,26 +194,52 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
 
 /*
  * One FASA decode step over a layer: TIP (fasa_score) -> T_t
- * (fasa_select_topk with k) -> FAC (fasa_sparse_attend). Four launches
- * chained with programmatic dependent launch: the score stream, which also
- * builds a per-row histogram of the score keys; a filter that marks the
- * certainly-kept tokens and collects the tokens of the threshold bin; a
- * per-row exact resolution of that bin that emits the kept indices in
- * ascending order; and the focused attention. Scores, histogram and index
- * lists live in the workspace.
+ * (fasa_select_topk with k) -> FAC (fasa_sparse_attend), with results equal
+ * to those three calls in sequence. Two launch plans compute it:
+ *
+ *  FASA_DECODE_FUSED  (bf16 caches whose rows fit; chosen when
+ *    B * Hkv * C stays within about two CTAs per SM) one launch, one
+ *    thread-block cluster of C <= 16 CTAs per (batch, KV head) row: each CTA
+ *    scores its share of the row into shared memory, the cluster runs an
+ *    exact radix select of the k-th key over distributed shared memory, each
+ *    CTA attends its kept rows, and the partials are merged in the cluster.
+ *    The workspace is not touched.
+ *  FASA_DECODE_STAGED  four launches chained with programmatic dependent
+ *    launch: the score stream, which also builds a per-row histogram of the
+ *    score keys; a filter that marks the certainly-kept tokens and collects
+ *    the tokens of the threshold bin; a per-row exact resolution of that bin
+ *    that emits the kept indices in ascending order; and the focused
+ *    attention. Scores, histogram and index lists live in the workspace.
  *
  *  out     : [B][Hq][128] dtype.
  *  idx_out : nullable; [B][Hkv][min(k, len)] int32, the kept tokens in
  *            ascending order.
  *  workspace : caller-owned device memory of at least
- *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned;
- *            its contents need no initialisation and are scratch.
+ *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned
+ *            (required whichever plan runs); its contents need no
+ *            initialisation and are scratch.
  *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;
- *  FASA_ERR_WORKSPACE if the workspace is missing or too small.
+ *  FASA_ERR_WORKSPACE if the workspace is missing or too small;
+ *  FASA_ERR_UNSUPPORTED if fasa_set_decode_path forced FASA_DECODE_FUSED on a
+ *  shape it cannot take.
  */
 fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
                         int32_t k, void* out, int32_t* idx_out, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream);
+
+/* Launch plan of fasa_decode (library code, no counterpart in the paper). */
+#define FASA_DECODE_AUTO 0   /* chosen from the shape (default) */
+#define FASA_DECODE_FUSED 1  /* single-launch cluster decode */
+#define FASA_DECODE_STAGED 2 /* four-launch decode */
+
+/* Sets the plan every later fasa_decode call of this process uses (a
+ * process-wide setting; FASA_ERR_INVALID_ARG for an unknown value). */
+fasa_status fasa_set_decode_path(int32_t path);
+
+/* The plan fasa_decode would run for this cache, len and k under the current
+ * setting and on the current device: FASA_DECODE_FUSED or FASA_DECODE_STAGED,
+ * or a negative fasa_status for invalid arguments. */
+int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
 
 /* Size of the library's own device scratch used by
  * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the

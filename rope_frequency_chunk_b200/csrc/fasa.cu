@@ -3,6 +3,7 @@
 // Host side only: argument validation (before any launch), launch-shape
 // choice, and dispatch to the kernels in append.cuh, score.cuh and
 // select_attend.cuh. Nothing here allocates device memory.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -14,6 +15,7 @@
 #include "select_attend.cuh"
 #include "select_hist.cuh"
 #include "attend_mma.cuh"
+#include "decode_fused.cuh"
 
 using namespace fasa;
 
@@ -333,6 +335,172 @@ fasa_status static_scratch_addr(void** out) {
   return FASA_OK;
 }
 
+// ------------------------------------------------- single-launch decode
+
+std::atomic<int> g_decode_path{FASA_DECODE_AUTO};
+
+// Launch plan of the single-launch decode.
+struct FusedPlan {
+  int C = 0, n_loc = 0, ring = 0, n_stages = 0, ucap = 0, smem = 0, waves = 0;
+};
+
+template <int LPT>
+fasa_status fused_attrs(const DevInfo& d) {
+  auto kern = decode_fused_kernel<LPT>;
+  int set = 0;
+  return cached_int((const void*)kern, 0, &set, [&](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    *v = 1;
+    return cuda_status(e);
+  });
+}
+
+// Clusters of size C with `smem` bytes per CTA that fit on the GPU at once.
+template <int LPT>
+fasa_status fused_max_clusters(int C, int smem, const DevInfo& d, int* out) {
+  auto kern = decode_fused_kernel<LPT>;
+  fasa_status s = fused_attrs<LPT>(d);
+  if (s != FASA_OK) return s;
+  return cached_int((const void*)kern, 3000ull + (uint64_t)C * 1000003ull + (uint64_t)smem, out, [&](int* v) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)C, 1, 1);
+    cfg.blockDim = dim3(kFuThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    *v = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(v, kern, &cfg);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      *v = 0;  // this cluster size is not available
+    }
+    return FASA_OK;
+  });
+}
+
+// Shape of the single-launch decode for cluster size C: tokens per CTA and
+// the ring (every score stage in flight when shared memory allows; at least
+// one K+V chunk per warp), which after scoring holds the boundary bin's union.
+template <int LPT>
+bool fused_shape(int C, int32_t len, const DevInfo& d, FusedPlan* pl) {
+  constexpr int kStage = fu_stage_bytes<LPT>();
+  constexpr int TPS = kStage / (LPT * 16);
+  pl->C = C;
+  pl->n_loc = (int)(ceil_div(ceil_div(len, C), 32) * 32);
+  if (pl->n_loc > kFuMaxLoc) return false;
+  const int ring_max = (d.smem_optin - fu_layout(pl->n_loc, 0).total) / 128 * 128;
+  if (ring_max < kFuMinRing) return false;
+  pl->n_stages = (int)std::min<int64_t>(std::min<int64_t>(kFuMaxStages, ring_max / kStage), ceil_div(pl->n_loc, TPS));
+  if (pl->n_stages < 1) return false;
+  pl->ring = std::max(kFuMinRing, (pl->n_stages * kStage + 127) / 128 * 128);
+  pl->ucap = (pl->ring - kFuRadixBytes) / 8;
+  pl->smem = fu_layout(pl->n_loc, pl->ring).total;
+  return pl->smem <= d.smem_optin;
+}
+
+// Picks the cluster size: fewest waves of clusters first, then the least
+// per-CTA streaming (a wave costs about a 4096-token CTA of fixed latency).
+// Not eligible (false) for rows too long or, unless forced, more than two
+// waves.
+template <int LPT>
+fasa_status fused_plan_t(int rows, int32_t len, int keff, const DevInfo& d, bool forced, FusedPlan* out, bool* ok) {
+  static const int kSizes[] = {16, 15, 14, 13, 12, 10, 8, 6, 4, 3, 2, 1};
+  *ok = false;
+  int64_t best = -1;
+  for (int C : kSizes) {
+    FusedPlan pl;
+    if (!fused_shape<LPT>(C, len, d, &pl)) continue;
+    int maxc = 0;
+    fasa_status s = fused_max_clusters<LPT>(C, pl.smem, d, &maxc);
+    if (s != FASA_OK) return s;
+    if (maxc < 1) continue;
+    pl.waves = (int)ceil_div(rows, maxc);
+    const int64_t cost = (int64_t)pl.waves * (pl.n_loc + 4096);
+    if (best < 0 || cost < best) {
+      best = cost;
+      *out = pl;
+    }
+  }
+  *ok = best >= 0 && (forced || out->waves <= 2);
+  return FASA_OK;
+}
+
+fasa_status fused_plan(const fasa_cache* c, int32_t len, int keff, const DevInfo& d, bool forced, FusedPlan* out,
+                       bool* ok) {
+  *ok = false;
+  if (c->dtype != FASA_BF16) return FASA_OK;
+  const int rows = c->batch * c->n_kv_heads;
+  switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
+    case 1: return fused_plan_t<1>(rows, len, keff, d, forced, out, ok);
+    case 2: return fused_plan_t<2>(rows, len, keff, d, forced, out, ok);
+    case 4: return fused_plan_t<4>(rows, len, keff, d, forced, out, ok);
+    case 8: return fused_plan_t<8>(rows, len, keff, d, forced, out, ok);
+    case 16: return fused_plan_t<16>(rows, len, keff, d, forced, out, ok);
+    default: return FASA_OK;
+  }
+}
+
+template <int LPT>
+fasa_status launch_fused_t(const FusedParams& p, int rows, const FusedPlan& pl, cudaStream_t st, const DevInfo& d) {
+  auto kern = decode_fused_kernel<LPT>;
+  fasa_status s = fused_attrs<LPT>(d);
+  if (s != FASA_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[2];
+  cfg.gridDim = dim3((unsigned)pl.C, (unsigned)rows, 1);
+  cfg.blockDim = dim3(kFuThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)pl.smem;
+  cfg.stream = st;
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = (unsigned)pl.C;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
+}
+
+fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t keff, void* out,
+                         int32_t* idx_out, const FusedPlan& pl, cudaStream_t st, const DevInfo& d) {
+  FusedParams p{};
+  p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
+  p.k = static_cast<const __nv_bfloat16*>(c->k);
+  p.v = static_cast<const __nv_bfloat16*>(c->v);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.dom_idx = c->dom_idx;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.idx_out = idx_out;
+  p.max_len = c->max_len;
+  p.len = len;
+  p.stride = c->sketch_stride;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.n_dom = c->n_dom;
+  p.n_keep = keff;
+  p.n_loc = pl.n_loc;
+  p.ring = pl.ring;
+  p.n_stages = pl.n_stages;
+  p.ucap = pl.ucap;
+  fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
+  const int rows = c->batch * c->n_kv_heads;
+  switch (c->sketch_stride / 8) {
+    case 1: return launch_fused_t<1>(p, rows, pl, st, d);
+    case 2: return launch_fused_t<2>(p, rows, pl, st, d);
+    case 4: return launch_fused_t<4>(p, rows, pl, st, d);
+    case 8: return launch_fused_t<8>(p, rows, pl, st, d);
+    case 16: return launch_fused_t<16>(p, rows, pl, st, d);
+    default: return FASA_ERR_UNSUPPORTED;
+  }
+}
+
 // Decode workspace, each part 256-byte aligned:
 //   scores [rows][len] f32 | hist [rows][4096] u32 | cand_cnt [rows] u32 |
 //   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
@@ -533,6 +701,16 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return FASA_ERR_WORKSPACE;
   DevInfo d;
   if ((s = device_info(&d)) != FASA_OK) return s;
+  const int rows = c->batch * c->n_kv_heads;
+  const int keff = std::min(k, len);
+  const int path = g_decode_path.load();
+  if (path != FASA_DECODE_STAGED) {
+    FusedPlan pl;
+    bool ok = false;
+    if ((s = fused_plan(c, len, keff, d, path == FASA_DECODE_FUSED, &pl, &ok)) != FASA_OK) return s;
+    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, pl, stream, d);
+    if (path == FASA_DECODE_FUSED) return FASA_ERR_UNSUPPORTED;
+  }
   char* base = static_cast<char*>(workspace);
   float* scores = reinterpret_cast<float*>(base + w.scores);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + w.hist);
@@ -540,8 +718,6 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
   int32_t* cand = reinterpret_cast<int32_t*>(base + w.cand);
   int32_t* idx = reinterpret_cast<int32_t*>(base + w.idx);
-  const int rows = c->batch * c->n_kv_heads;
-  const int keff = std::min(k, len);
 
   // 1. TIP scores and the per-row key histogram
   uint32_t* att_cnt = reinterpret_cast<uint32_t*>(base + w.att_cnt);
@@ -633,6 +809,27 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
   return launch_sa<kAttendIdx>(c, p, rows, true, stream, c->dtype, q_pos);
+}
+
+fasa_status fasa_set_decode_path(int32_t path) {
+  if (path != FASA_DECODE_AUTO && path != FASA_DECODE_FUSED && path != FASA_DECODE_STAGED)
+    return FASA_ERR_INVALID_ARG;
+  g_decode_path.store(path);
+  return FASA_OK;
+}
+
+int32_t fasa_decode_path(const fasa_cache* c, int32_t len, int32_t k) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return -s;
+  if (len < 1 || k < 1 || len > c->max_len) return -FASA_ERR_INVALID_ARG;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return -s;
+  const int path = g_decode_path.load();
+  if (path != FASA_DECODE_AUTO) return path;
+  FusedPlan pl;
+  bool ok = false;
+  if ((s = fused_plan(c, len, std::min(k, len), d, false, &pl, &ok)) != FASA_OK) return -s;
+  return ok ? FASA_DECODE_FUSED : FASA_DECODE_STAGED;
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,

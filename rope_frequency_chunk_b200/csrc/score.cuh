@@ -92,16 +92,94 @@ __device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double*
 constexpr int kHistBits = 12;                 // key bits of the per-row score histogram
 constexpr int kHistBins = 1 << kHistBits;
 
+// Shape of the per-token work for sketch rows of LPT 16-byte chunks.
+template <typename T, int LPT>
+struct ScoreShape {
+  static constexpr int EPC = Elem<T>::kPer16;                   // elements per 16-byte chunk
+  static constexpr int ROWE = LPT * EPC;                        // elements per sketch row
+  static constexpr int ROWB = LPT * 16;                         // sketch row bytes
+  static constexpr int LPT2 = ROWE > 32 ? ROWE / 32 : 1;        // lanes per token
+  static constexpr int EPL = ROWE / LPT2;                       // elements per lane (<= 32)
+  static constexpr int CPL = EPL / EPC;                         // chunks per lane
+  static constexpr int TPW = 32 / LPT2;                         // tokens per warp step
+  // chunk rotation per lane so that a quarter-warp's 16-byte reads hit
+  // distinct banks; the lane's coefficients are rotated the same way
+  __device__ static int rot(int lane) {
+    return (LPT2 == 1) ? ((lane * CPL / 8) % CPL) : (LPT2 == 2 ? ((lane / 2) % CPL) : 0);
+  }
+};
+
+// Sketch-column coefficients of one row, scaled by 2^896: column 2j (2j+1)
+// is the first (second) dim of dominant FC dom[j], summed over the group's
+// rotated query heads; padding columns are zero. Thread `tid` < stride
+// writes column tid.
+template <typename T>
+__device__ __forceinline__ void query_coefs(const T* qraw, const int* dom, int group, int n_dom, int stride,
+                                            const double* cosv, const double* sinv, int tid, double* s_q) {
+  if (tid >= stride) return;
+  const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
+  double acc = 0.0;
+  const int jj = tid >> 1;
+  if (jj < n_dom) {
+    const int i = dom[jj];
+    if (i >= 0 && i < kNFC) {
+      const double c = cosv[i], s = sinv[i];
+      for (int h = 0; h < group; ++h) {
+        const double x = to_float(qraw[h * kD + i]);
+        const double y = to_float(qraw[h * kD + i + kNFC]);
+        // rotated query, first (x) or second (y) dim of FC i
+        acc += (tid & 1) ? __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s)) : __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
+      }
+    } else {
+      flag_status(FASA_ERR_BAD_INDEX);
+    }
+  }
+  s_q[tid] = acc * two896;
+}
+
+// The lane's share of the coefficients, in its rotated chunk order.
+template <typename T, int LPT>
+__device__ __forceinline__ void load_coefs(double (&qr)[ScoreShape<T, LPT>::EPL], const double* s_q, int lane) {
+  using S = ScoreShape<T, LPT>;
+  const int sub = lane % S::LPT2, rot = S::rot(lane);
+#pragma unroll
+  for (int c = 0; c < S::CPL; ++c)
+#pragma unroll
+    for (int e = 0; e < S::EPC; ++e) qr[c * S::EPC + e] = s_q[(sub * S::CPL + (c + rot) % S::CPL) * S::EPC + e];
+}
+
+// Scores of the n tokens of one staged block of sketch rows, warps
+// 0..NCW-1 in turn. sink(t, writer, score) is called by every lane of the
+// warp (warp-uniform), writer set on the one lane that owns token t.
+template <typename T, int LPT, int NCW, typename Sink>
+__device__ __forceinline__ void score_block(const unsigned char* buf, int n, const double (&qr)[ScoreShape<T, LPT>::EPL],
+                                            int warp, int lane, Sink&& sink) {
+  using S = ScoreShape<T, LPT>;
+  const int sub = lane % S::LPT2, rot = S::rot(lane);
+  for (int gi = warp; gi * S::TPW < n; gi += NCW) {
+    const int t = gi * S::TPW + lane / S::LPT2;
+    const bool valid = t < n;
+    uint4 v[S::CPL];
+#pragma unroll
+    for (int c = 0; c < S::CPL; ++c)
+      v[c] = valid ? *reinterpret_cast<const uint4*>(buf + t * S::ROWB + (sub * S::CPL + (c + rot) % S::CPL) * 16)
+                   : make_uint4(0, 0, 0, 0);
+    double part[S::CPL];
+#pragma unroll
+    for (int c = 0; c < S::CPL; ++c) part[c] = chunk_dot<T>(v[c], qr + c * S::EPC);
+    double acc = part[0];
+#pragma unroll
+    for (int c = 1; c < S::CPL; ++c) acc += part[c];
+#pragma unroll
+    for (int off = S::LPT2 / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+    sink(t, valid && sub == 0, (float)acc);
+  }
+}
+
 template <typename T, int LPT, bool kHist>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScoreParams p) {
-  constexpr int EPC = Elem<T>::kPer16;          // elements per 16-byte chunk
-  constexpr int ROWE = LPT * EPC;               // elements per sketch row
-  constexpr int ROWB = LPT * 16;                // sketch row bytes
-  constexpr int LPT2 = ROWE > 32 ? ROWE / 32 : 1;  // lanes per token
-  constexpr int EPL = ROWE / LPT2;              // elements per lane (<= 32)
-  constexpr int CPL = EPL / EPC;                // chunks per lane
-  constexpr int TPW = 32 / LPT2;                // tokens per warp step
-  constexpr int TPS = kScoreStageBytes / ROWB;  // tokens per stage
+  using S = ScoreShape<T, LPT>;
+  constexpr int TPS = kScoreStageBytes / S::ROWB;  // tokens per stage
   constexpr int NCW = kScoreConsumerWarps;
   extern __shared__ __align__(128) unsigned char ring[];  // stages, then the histogram
   uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + (size_t)kScoreStages * kScoreStageBytes);
@@ -142,10 +220,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
         st_row[b] = row;
         st_t0[b] = t;
         st_n[b] = n;
-        mbar_arrive_expect_tx(&full[b], (uint32_t)(n * ROWB));
+        mbar_arrive_expect_tx(&full[b], (uint32_t)(n * S::ROWB));
         bulk_g2s(ring + (size_t)b * kScoreStageBytes,
-                 static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t) * ROWB, (uint32_t)(n * ROWB),
-                 &full[b]);
+                 static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t) * S::ROWB,
+                 (uint32_t)(n * S::ROWB), &full[b]);
         left -= n;
         t += n;
         if (t == p.len) {
@@ -158,12 +236,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
   }
 
   // ---------------- consumers: one token per lane (LPT2 lanes for wide rows)
-  const int sub = lane % LPT2;
-  // chunk rotation per lane so that a quarter-warp's 16-byte reads hit
-  // distinct banks; the lane's coefficients are rotated the same way
-  const int rot = (LPT2 == 1) ? ((lane * CPL / 8) % CPL) : (LPT2 == 2 ? ((lane / 2) % CPL) : 0);
-  const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
-  double qr[EPL];
+  double qr[S::EPL];
   int cur_row = -1;
   float* out = p.scores;
 
@@ -190,71 +263,31 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
       {
         // the group's queries and the head's dominant FCs, loaded in parallel
         const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
-        const uint4* qsrc =
-            reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD);
+        const uint4* qsrc = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
+                                                           ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD);
         for (int c = tid; c < p.group * kD * (int)sizeof(T) / 16; c += NCW * 32)
           reinterpret_cast<uint4*>(s_qraw)[c] = __ldg(qsrc + c);
         if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
       }
       named_barrier_sync(1, NCW * 32);
-      if (tid < p.stride) {
-        double acc = 0.0;
-        const int jj = tid >> 1;
-        if (jj < p.n_dom) {
-          const int i = s_dom[jj];
-          if (i >= 0 && i < kNFC) {
-            const double c = p.cosv[i], s = p.sinv[i];
-            const T* qh = s_qraw;
-            for (int h = 0; h < p.group; ++h) {
-              const double x = to_float(qh[h * kD + i]);
-              const double y = to_float(qh[h * kD + i + kNFC]);
-              // rotated query, first (x) or second (y) dim of FC i
-              acc += (tid & 1) ? __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s))
-                               : __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
-            }
-          } else {
-            flag_status(FASA_ERR_BAD_INDEX);
-          }
-        }
-        s_q[tid] = acc * two896;
-      }
+      query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
       named_barrier_sync(1, NCW * 32);
-#pragma unroll
-      for (int c = 0; c < CPL; ++c)
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) qr[c * EPC + e] = s_q[(sub * CPL + (c + rot) % CPL) * EPC + e];
+      load_coefs<T, LPT>(qr, s_q, lane);
       cur_row = row;
       out = p.scores + (int64_t)row * p.len;
     }
-    const unsigned char* buf = ring + (size_t)b * kScoreStageBytes;
-    for (int gi = warp; gi * TPW < n; gi += NCW) {
-      const int t = gi * TPW + lane / LPT2;
-      const bool valid = t < n;
-      uint4 v[CPL];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c)
-        v[c] = valid ? *reinterpret_cast<const uint4*>(buf + t * ROWB + (sub * CPL + (c + rot) % CPL) * 16)
-                     : make_uint4(0, 0, 0, 0);
-      double part[CPL];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) part[c] = chunk_dot<T>(v[c], qr + c * EPC);
-      double acc = part[0];
-#pragma unroll
-      for (int c = 1; c < CPL; ++c) acc += part[c];
-#pragma unroll
-      for (int off = LPT2 / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-      const float sc = (float)acc;
-      const bool writer = valid && sub == 0;
-      if (writer) out[t0 + t] = sc;
-      if (kHist) {
-        const uint32_t bin = score_key(sc) >> (32 - kHistBits);
-        const unsigned act = __ballot_sync(0xFFFFFFFFu, writer);
-        if (writer) {
-          const unsigned peers = __match_any_sync(act, bin);
-          if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
-        }
-      }
-    }
+    score_block<T, LPT, NCW>(ring + (size_t)b * kScoreStageBytes, n, qr, warp, lane,
+                             [&](int t, bool writer, float sc) {
+                               if (writer) out[t0 + t] = sc;
+                               if (kHist) {
+                                 const uint32_t bin = score_key(sc) >> (32 - kHistBits);
+                                 const unsigned act = __ballot_sync(0xFFFFFFFFu, writer);
+                                 if (writer) {
+                                   const unsigned peers = __match_any_sync(act, bin);
+                                   if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
+                                 }
+                               }
+                             });
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[b]);
     done += n;

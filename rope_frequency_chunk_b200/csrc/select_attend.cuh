@@ -260,13 +260,14 @@ __device__ void ballot_radix_fn(KeyAt key_at, int n, int k, uint32_t prefix, int
 // From a row's 4096-bin histogram of the top 12 key bits, the bin holding
 // the k-th largest key and the number of keys in higher bins. Block-wide
 // suffix scan: thread t owns bins 4095-8t .. 4088-8t.
-__device__ __forceinline__ void hist_threshold(const uint32_t* h, int k, uint32_t* scan, uint32_t& bin,
-                                               uint32_t& above) {
+// (hist_threshold_fn takes the bin loader; hist_threshold reads global memory.)
+template <typename Ld>
+__device__ __forceinline__ void hist_threshold_fn(Ld ld, int k, uint32_t* scan, uint32_t& bin, uint32_t& above) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t c[8], sum = 0u;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    c[u] = __ldcg(h + 4095 - (8 * tid + u));
+    c[u] = ld(4095 - (8 * tid + u));
     sum += c[u];
   }
   uint32_t incl = sum;
@@ -305,6 +306,10 @@ __device__ __forceinline__ void hist_threshold(const uint32_t* h, int k, uint32_
   bin = scan[32];
   above = scan[33];
   __syncthreads();
+}
+__device__ __forceinline__ void hist_threshold(const uint32_t* h, int k, uint32_t* scan, uint32_t& bin,
+                                               uint32_t& above) {
+  hist_threshold_fn([h](int i) { return __ldcg(h + i); }, k, scan, bin, above);
 }
 
 template <bool kCluster>

@@ -59,6 +59,8 @@ _SIGS = {
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
     "fasa_device_status": (_I, [_I]),
+    "fasa_set_decode_path": (_I, [_I]),
+    "fasa_decode_path": (_I, [_CP, _I, _I]),
 }
 
 
@@ -221,6 +223,22 @@ def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, id
     _check(lib().fasa_decode(cache.ref(), length, q.data_ptr(), q_pos, k, out.data_ptr(), _ptr(idx_out),
                              workspace.data_ptr(), workspace.numel(), _stream(stream)), "fasa_decode")
     return out
+
+
+DECODE_AUTO, DECODE_FUSED, DECODE_STAGED = 0, 1, 2
+
+
+def fasa_set_decode_path(path: int) -> None:
+    """Launch plan of later fasa_decode calls (process-wide)."""
+    _check(lib().fasa_set_decode_path(int(path)), "fasa_set_decode_path")
+
+
+def fasa_decode_path(cache: KVCache, length: int, k: int) -> int:
+    """The plan fasa_decode would run for this shape (DECODE_FUSED or DECODE_STAGED)."""
+    r = int(lib().fasa_decode_path(cache.ref(), length, k))
+    if r < 0:
+        _check(-r, "fasa_decode_path")
+    return r
 
 
 def fasa_dense_decode(cache: KVCache, length: int, q, q_pos: int, out=None, stream=None):

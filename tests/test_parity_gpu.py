@@ -135,6 +135,22 @@ def test_dense_matches_oracle(name):
         U.check_out(wl, out[b, g * G:(g + 1) * G], ref)
 
 
+PATHS = {"fused": F.DECODE_FUSED, "staged": F.DECODE_STAGED}
+
+
+@pytest.fixture(params=list(PATHS))
+def path(request):
+    """Runs a decode test under each launch plan of fasa_decode."""
+    F.fasa_set_decode_path(PATHS[request.param])
+    yield request.param
+    F.fasa_set_decode_path(F.DECODE_AUTO)
+
+
+def _skip_unless_plan(wl, path):
+    if path == "fused" and wl.dtype != "bf16":
+        pytest.skip("the single-launch decode takes bf16 caches only")
+
+
 def _decode(wl, cache, q, k, length=None):
     L = length or wl.ctx_len
     idx = torch.empty(wl.batch, wl.n_kv_heads, min(k, L), dtype=torch.int32, device="cuda")
@@ -143,8 +159,9 @@ def _decode(wl, cache, q, k, length=None):
 
 
 @pytest.mark.parametrize("name", list(SMALL))
-def test_decode_matches_oracle(name):
+def test_decode_matches_oracle(name, path):
     wl = SMALL[name]
+    _skip_unless_plan(wl, path)
     inp, cache, q = U.build(wl)
     out, idx = _decode(wl, cache, q, wl.k)
     s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
@@ -152,7 +169,7 @@ def test_decode_matches_oracle(name):
 
 
 @pytest.mark.parametrize("k_of_L", ["one", "equal", "more", "half"])
-def test_decode_budget_edges(k_of_L):
+def test_decode_budget_edges(k_of_L, path):
     wl = SMALL["c2_ragged"].replace(ctx_len=1999)
     L = wl.ctx_len
     k = {"one": 1, "equal": L, "more": L + 500, "half": L // 2}[k_of_L]
@@ -164,7 +181,7 @@ def test_decode_budget_edges(k_of_L):
         U.check_gpu_pair(wl, U.stored(out), U.stored(dense))
 
 
-def test_decode_single_token_cache():
+def test_decode_single_token_cache(path):
     wl = C["c2"].replace(ctx_len=1, batch=2)
     inp, cache, q = U.build(wl)
     out, idx = _decode(wl, cache, q, 256)
@@ -172,7 +189,7 @@ def test_decode_single_token_cache():
     U.check_decode_heads(wl, inp, cache, q, 256, U.all_heads(wl), out, idx)
 
 
-def test_decode_all_fc_full_budget_is_dense():
+def test_decode_all_fc_full_budget_is_dense(path):
     """With every FC dominant and k = L, FASA is dense attention."""
     wl = C["c2"].replace(ctx_len=3000, n_dom=64, k=3000)
     inp, cache, q = U.build(wl)
@@ -181,7 +198,7 @@ def test_decode_all_fc_full_budget_is_dense():
     U.check_gpu_pair(wl, U.stored(out), U.stored(dense))
 
 
-def test_decode_with_tied_tokens():
+def test_decode_with_tied_tokens(path):
     """Tokens whose dominant dims are zero all score exactly 0; the budget is
     placed inside that tie, so ties must go to the lower index."""
     wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=4000)
@@ -201,7 +218,28 @@ def test_decode_with_tied_tokens():
     assert kept_zero == list(range(1000, 1037))
 
 
-def test_decode_is_deterministic_and_capturable():
+@pytest.mark.parametrize("case", ["all_tied", "k_beyond_union"])
+def test_decode_exact_fallbacks(case, path):
+    """Shapes where the single-launch decode's candidate union cannot prove
+    exactness (every CTA cuts inside one big tie; k above what the union
+    holds) and it falls back to the exact distributed radix select."""
+    if case == "all_tied":
+        wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=8192, k=100)
+        inp = W.layer_inputs(wl)
+        dom = inp.params.dom_idx[0]
+        inp.k[0, 0][:, np.concatenate([dom, dom + 64])] = 0
+    else:
+        wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=40000, k=20000)
+        inp = W.layer_inputs(wl)
+    _, cache, q = U.build(wl, inp=inp)
+    out, idx = _decode(wl, cache, q, wl.k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, wl.k, [(0, 0)], out, idx, scores_gpu=s)
+    if case == "all_tied":
+        assert idx.cpu().numpy()[0, 0].tolist() == list(range(wl.k))
+
+
+def test_decode_is_deterministic_and_capturable(path):
     wl = SMALL["c2_ragged"]
     inp, cache, q = U.build(wl)
     ws = torch.empty(F.fasa_decode_workspace_bytes(cache, wl.ctx_len, wl.k), dtype=torch.uint8, device="cuda")
@@ -216,6 +254,50 @@ def test_decode_is_deterministic_and_capturable():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out1, out2)
+
+
+def _both_paths(wl, cache, q, k):
+    res = {}
+    for name, pth in PATHS.items():
+        F.fasa_set_decode_path(pth)
+        try:
+            res[name] = _decode(wl, cache, q, k)
+        finally:
+            F.fasa_set_decode_path(F.DECODE_AUTO)
+    return res
+
+
+def _check_paths_agree(wl, res):
+    """Both plans score bit-identically and select exactly: same kept sets;
+    outputs differ only by float32 summation order."""
+    (o_f, i_f), (o_s, i_s) = res["fused"], res["staged"]
+    assert torch.equal(i_f, i_s)
+    U.check_gpu_pair(wl, U.stored(o_f), U.stored(o_s))
+
+
+def test_decode_path_setting_and_choice():
+    wl = C["c2"].replace(ctx_len=4096)
+    _, cache, _ = U.build(wl)
+    assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_FUSED
+    F.fasa_set_decode_path(F.DECODE_STAGED)
+    try:
+        assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_STAGED
+    finally:
+        F.fasa_set_decode_path(F.DECODE_AUTO)
+    with pytest.raises(F.FasaError):
+        F.fasa_set_decode_path(7)
+
+
+def test_fused_decode_rejects_f32_when_forced():
+    wl = SMALL["c1"]
+    _, cache, q = U.build(wl)
+    F.fasa_set_decode_path(F.DECODE_FUSED)
+    try:
+        with pytest.raises(F.FasaError) as e:
+            _decode(wl, cache, q, wl.k)
+        assert e.value.status == 2
+    finally:
+        F.fasa_set_decode_path(F.DECODE_AUTO)
 
 
 # ------------------------------------------------------------ full sizes
@@ -236,6 +318,8 @@ def test_full_c2():
     out, idx = _decode(wl, cache, q, wl.k)
     s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
     U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
+    assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_FUSED
+    _check_paths_agree(wl, _both_paths(wl, cache, q, wl.k))
     dense = U.stored(F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos))
     G = wl.group
     for (b, g) in U.sample_heads(wl, 2, seed=1):
@@ -251,6 +335,7 @@ def test_full_c3_sampled():
     U.check_append(wl, inp, cache, heads[:1])
     out, idx = _decode(wl, cache, q, wl.k)
     U.check_decode_heads(wl, inp, cache, q, wl.k, heads, out, idx)
+    _check_paths_agree(wl, _both_paths(wl, cache, q, wl.k))
 
 
 @pytest.fixture(scope="module")
@@ -267,6 +352,8 @@ def test_full_c5_sampled(k, c5_state):
     inp, cache, q = c5_state
     out, idx = _decode(wl, cache, q, k)
     U.check_decode_heads(wl, inp, cache, q, k, U.sample_heads(wl, 3, seed=k), out, idx)
+    if k == W.C5_KS[0]:
+        _check_paths_agree(wl, _both_paths(wl, cache, q, k))
     if k == W.C5_KS[-1]:
         dense = U.stored(F.fasa_dense_decode(cache, wl.ctx_len, q, wl.q_pos))
         G = wl.group
