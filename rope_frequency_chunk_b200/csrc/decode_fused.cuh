@@ -17,14 +17,15 @@
 //     key bits in a 4096-bin histogram.
 //  2. select: each CTA counts the top 8 bits of its keys (256 bins) while
 //     scoring and writes that histogram into every CTA of the cluster
-//     (distributed shared memory). After one cluster barrier every CTA knows
-//     the row's histogram, hence the bin B holding the k_eff-th key, the
-//     count above it, and every CTA's count inside B: the CTAs write their
-//     tokens of bin B, compacted in rank order, into every CTA, and after a
-//     second barrier each CTA resolves the exact k_eff-th key of the row and
-//     its ties (lower token index first) from that union alone. A union too
-//     large for shared memory (heavy ties) sends all CTAs to an exact
-//     distributed radix select over the keys of bin B instead.
+//     (distributed shared memory). After a cluster barrier every CTA knows
+//     the row's histogram, hence the bin B holding the k_eff-th key; the same
+//     exchange for B's 16 sub-bins (key bits 20..23) gives the 12-bit bin
+//     b12 holding it, the count above, and every CTA's count inside b12. The
+//     CTAs write their tokens of b12, compacted in rank order, into every
+//     CTA, and after a third barrier each CTA resolves the exact k_eff-th
+//     key of the row and its ties (lower token index first) from that union
+//     alone. A union too large for shared memory (heavy ties) sends all CTAs
+//     to an exact distributed radix select over the keys of b12 instead.
 //  3. attend: each CTA attends its own kept rows on tensor cores
 //     (mma.sync m16n8k16, Q split into three bf16 terms and P into two, as in
 //     the split-K attention kernel) and merges its warps pairwise; the CTAs
@@ -89,7 +90,7 @@ struct FusedParams {
 };
 
 struct FuLayout {
-  int ring, keys, bm, hloc, hall, qt, sq, qraw, dom, bars, chist, xch, scan, rml, ro, total;
+  int ring, keys, bm, hloc, hall, hfine, qt, sq, qraw, dom, bars, chist, xch, scan, rml, ro, total;
 };
 __host__ __device__ inline FuLayout fu_layout(int n_loc, int ring) {
   FuLayout L;
@@ -104,6 +105,8 @@ __host__ __device__ inline FuLayout fu_layout(int n_loc, int ring) {
   o += 256 * 4;
   L.hall = o;  // every rank's histogram [kFuMaxCluster][256]
   o += kFuMaxCluster * 256 * 4;
+  L.hfine = o;  // every rank's 16 sub-bins of the boundary bin [kFuMaxCluster][16], then this CTA's own
+  o += (kFuMaxCluster + 1) * 16 * 4;
   L.qt = o;  // attention Q: 3 bf16 terms x 16 heads x 128, rows of 256 B, 16-B chunks swizzled
   o += 3 * 16 * kD * 2;
   L.sq = o;
@@ -159,6 +162,66 @@ __device__ __forceinline__ void coarse_threshold(const uint32_t* h, int k, uint3
   bin = min(scan[8], 255u);
   above = scan[9];
   __syncthreads();
+}
+
+// The bin of a 1024-bin histogram holding the k-th largest entry (counting
+// from bin 1023 down) and the count in higher bins (k <= total). All
+// threads; thread t owns bins 1023 - 2t and 1022 - 2t; uses sc[0, 20).
+__device__ __forceinline__ void bins1024_threshold(const uint32_t* h, int k, uint32_t* sc, uint32_t& bin,
+                                                   uint32_t& above) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t ca = h[1023 - 2 * tid], cb = h[1022 - 2 * tid];
+  const uint32_t sum = ca + cb;
+  uint32_t incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) sc[warp] = incl;
+  if (tid == 0) sc[16] = sc[17] = 0u;  // (only reached when k exceeds the total)
+  __syncthreads();
+  uint32_t before = 0u;
+  for (int w = 0; w < warp; ++w) before += sc[w];
+  incl += before;
+  const uint32_t excl = incl - sum;
+  if (excl < (uint32_t)k && (uint32_t)k <= excl + ca) {
+    sc[16] = 1023u - 2u * (uint32_t)tid;
+    sc[17] = excl;
+  } else if (excl + ca < (uint32_t)k && (uint32_t)k <= incl) {
+    sc[16] = 1022u - 2u * (uint32_t)tid;
+    sc[17] = excl + ca;
+  }
+  __syncthreads();
+  bin = sc[16] & 1023u;
+  above = sc[17];
+  __syncthreads();
+}
+
+// Exact k-th largest of n keys that share their top 12 bits (`prefix`):
+// two passes over the remaining 20 bits, 10-bit digits counted with shared
+// memory atomics into cnt[1024]. Returns the key and how many keys equal to
+// it must still be taken. All threads.
+__device__ __forceinline__ void select_low20(const uint32_t* key, int n, int k, uint32_t prefix, uint32_t* cnt,
+                                             uint32_t* sc, uint32_t& thr, int& quota) {
+  const int tid = threadIdx.x;
+  uint32_t d1, d2, above;
+  for (int i = tid; i < 1024; i += kFuThreads) cnt[i] = 0u;
+  __syncthreads();
+  for (int e = tid; e < n; e += kFuThreads) atomicAdd(&cnt[(key[e] >> 10) & 1023u], 1u);
+  __syncthreads();
+  bins1024_threshold(cnt, k, sc, d1, above);
+  k -= (int)above;
+  for (int i = tid; i < 1024; i += kFuThreads) cnt[i] = 0u;
+  __syncthreads();
+  for (int e = tid; e < n; e += kFuThreads) {
+    const uint32_t x = key[e];
+    if (((x >> 10) & 1023u) == d1) atomicAdd(&cnt[x & 1023u], 1u);
+  }
+  __syncthreads();
+  bins1024_threshold(cnt, k, sc, d2, above);
+  thr = prefix | (d1 << 10) | d2;
+  quota = k - (int)above;
 }
 
 // Per-warp contiguous ranges of 32-token words of n tokens.
@@ -229,6 +292,8 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   uint32_t* bm = reinterpret_cast<uint32_t*>(smem + Ly.bm);
   uint32_t* hloc = reinterpret_cast<uint32_t*>(smem + Ly.hloc);
   uint32_t* hall = reinterpret_cast<uint32_t*>(smem + Ly.hall);
+  uint32_t* hfine = reinterpret_cast<uint32_t*>(smem + Ly.hfine);
+  uint32_t* hf_own = hfine + kFuMaxCluster * 16;
   unsigned char* qt = smem + Ly.qt;
   double* s_q = reinterpret_cast<double*>(smem + Ly.sq);
   T* qraw = reinterpret_cast<T*>(smem + Ly.qraw);
@@ -263,6 +328,15 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   }
   for (int i = tid; i < 4 * 256; i += kFuThreads) chist[i] = 0u;
   if (tid < 256) hloc[tid] = 0u;
+  // the sketch rows do not change between decode steps except for appended
+  // tokens: warm L2 with this CTA's range while the previous kernel in the
+  // stream may still run (the reads proper wait for it), and let the next
+  // kernel's CTAs start on free SMs to do the same
+  if (warp == kFuScoreWarps && lane == 0 && n > 0) {
+    const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
+    for (int t = 0; t < n; t += TPS) prefetch_l2(src + (int64_t)t * S::ROWB, (uint32_t)(min(TPS, n - t) * S::ROWB));
+  }
+  grid_dependents_launch();
   __syncthreads();
   cluster_arrive();  // every CTA of the cluster runs: waited for before the first remote access
   grid_dependency_wait();
@@ -353,27 +427,73 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   __syncthreads();
   uint32_t bin8, above8;
   coarse_threshold(hloc, p.n_keep, scan, bin8, above8);
-  const int krem8 = p.n_keep - (int)above8;  // keys of bin B still to take (>= 1)
-  uint32_t off = 0u, n_b = 0u;               // this CTA's offset in the union, the union's size
+  // second level: the 16 sub-bins (key bits 20..23) of bin B, counted here
+  // and written into every CTA
+  if (tid < 16) hf_own[tid] = 0u;
+  __syncthreads();
+  for (int i = tid; i < n; i += kFuThreads) {
+    const uint32_t x = keys[i];
+    if ((x >> 24) == bin8) atomicAdd(&hf_own[(x >> 20) & 15u], 1u);
+  }
+  __syncthreads();
+  if (tid < C * 16) cluster.map_shared_rank(hfine, tid >> 4)[cr * 16 + (tid & 15)] = hf_own[tid & 15];
+  cluster_arrive();
+  cluster_wait();
+  // the boundary sub-bin: the 12-bit bin b12 holding the k_eff-th key
+  uint32_t above12 = above8, b12 = bin8 << 4;
+  {
+    uint32_t cum = above8;
+    for (int f = 15; f >= 0; --f) {
+      uint32_t c = 0u;
+      for (int r = 0; r < C; ++r) c += hfine[r * 16 + f];
+      if (cum + c >= (uint32_t)p.n_keep) {
+        b12 = (bin8 << 4) | (uint32_t)f;
+        above12 = cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  const int krem12 = p.n_keep - (int)above12;  // keys of bin b12 still to take (>= 1)
+  uint32_t off = 0u, n_b = 0u;                 // this CTA's offset in the union, the union's size
   for (int r = 0; r < C; ++r) {
-    const uint32_t c = hall[r * 256 + bin8];
+    const uint32_t c = hfine[r * 16 + (b12 & 15u)];
     off += (r < cr) ? c : 0u;
     n_b += c;
   }
   const bool exact = n_b <= (uint32_t)p.ucap;  // the same in every CTA
-  auto in_bin = [keys, bin8](int i) { return (keys[i] >> 24) == bin8; };
+  auto in_bin = [keys, b12](int i) { return (keys[i] >> 20) == b12; };
   if (exact) {
+    // this CTA's tokens of b12, compacted locally (in the radix scratch,
+    // unused until the union is complete), then copied into every CTA with
+    // consecutive threads on consecutive entries
     const uint2 cp = fu_count(n, scan, in_bin);
-    fu_visit(n, cp.x, in_bin, [&](int pos, int i) {
-      const uint32_t key = keys[i];
-      const uint32_t at = off + (uint32_t)pos;
-      if (at >= n_b) return;  // keys and histogram disagree only after a recorded timeout
-#pragma unroll 1
-      for (int r = 0; r < C; ++r) {
-        cluster.map_shared_rank(ukey_s, r)[at] = key;
-        cluster.map_shared_rank(uidx_s, r)[at] = t0 + i;
+    const int mine = (int)min(cp.y, n_b - off);  // they agree unless a timeout was recorded
+    uint32_t* lk = rscr;
+    int32_t* li = reinterpret_cast<int32_t*>(rscr + kFuRadixBytes / 8);
+    if (mine <= kFuRadixBytes / 8) {
+      fu_visit(n, cp.x, in_bin, [&](int pos, int i) {
+        if (pos < mine) {
+          lk[pos] = keys[i];
+          li[pos] = t0 + i;
+        }
+      });
+      __syncthreads();
+      for (int e = tid; e < C * mine; e += kFuThreads) {
+        const int r = e / mine, j = e - r * mine;
+        cluster.map_shared_rank(ukey_s, r)[off + j] = lk[j];
+        cluster.map_shared_rank(uidx_s, r)[off + j] = li[j];
       }
-    });
+    } else {
+      fu_visit(n, cp.x, in_bin, [&](int pos, int i) {
+        if (pos >= mine) return;
+#pragma unroll 1
+        for (int r = 0; r < C; ++r) {
+          cluster.map_shared_rank(ukey_s, r)[off + pos] = keys[i];
+          cluster.map_shared_rank(uidx_s, r)[off + pos] = t0 + i;
+        }
+      });
+    }
   }
   cluster_arrive();
   cluster_wait();
@@ -383,8 +503,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
     // the exact krem8-th key of the union, and its ties (lower index first)
     const int n_u = (int)n_b;
     int quota;
-    ballot_radix_fn<false>([ukey_s](int i) { return ukey_s[i]; }, n_u, krem8, bin8 << 24, 8, 32, rscr, nullptr, cluster,
-                           thr, quota);
+    select_low20(ukey_s, n_u, krem12, b12 << 20, rscr, scan, thr, quota);
     uint32_t neq = 0u;
     for (int base = warp * 32; base < n_u; base += kFuThreads)
       neq += __popc(__ballot_sync(0xFFFFFFFFu, base + lane < n_u && ukey_s[base + lane] == thr));
@@ -411,10 +530,10 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
       if (lane == 0) bm[w] = kb;
     }
   } else {
-    // exact distributed radix select over the keys of bin B; the CTAs' tie
+    // exact distributed radix select over the keys of bin b12; the CTAs' tie
     // counts are exchanged once and CTA r keeps what the lower ranks left
     int krem;
-    ballot_radix_fn<true>([keys](int i) { return keys[i]; }, n, krem8, bin8 << 24, 8, 32, rscr, chist, cluster, thr,
+    ballot_radix_fn<true>([keys](int i) { return keys[i]; }, n, krem12, b12 << 20, 12, 32, rscr, chist, cluster, thr,
                           krem);
     const uint2 eq = fu_count(n, scan, [keys, thr](int i) { return keys[i] == thr; });
     if (tid < C) cluster.map_shared_rank(xch, tid)[kXTies * kFuMaxCluster + cr] = eq.y;

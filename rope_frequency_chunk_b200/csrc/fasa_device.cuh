@@ -158,6 +158,11 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
 
 // Programmatic dependent launch: wait until the preceding kernel in the
 // stream has completed and its memory is visible (no-op without PDL).
+// Hint: bring [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
+// Safe before griddepcontrol.wait: later loads still see the latest data.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
