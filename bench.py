@@ -238,15 +238,28 @@ def time_graph(fn, steps, warmup, stream, dist=None):
             g.replay()
         e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        dist.barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     torch.cuda.synchronize()
     del g
     return ms
+
+
+def max_over_ranks(value: float, dist=None, device: str = "cuda") -> float:
+    """The largest of every rank's value (every rank gets it); the value itself
+    on one process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.barrier()
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job GB/s: every rank moved bytes_per_rank_step per step, and a step
+    took ms_per_step (the slowest rank's time)."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
 
 
 def run_fasa(args, wl):
@@ -304,7 +317,7 @@ def run_fasa(args, wl):
     step_bytes = per_layer_bytes * n_layers
     ms_step = ms / args.steps
     us_layer = 1e3 * ms_step / n_layers
-    gbs = world * step_bytes / (ms_step * 1e-3) / 1e9
+    gbs = job_gbs(step_bytes, ms_step, world)
 
     # dominant kernel: the single-launch decode is the whole step; the staged
     # plan's is the TIP score stream, timed alone on the same stack
@@ -347,7 +360,7 @@ def run_fasa(args, wl):
         esteps = max(3, args.steps // 4)
         ms_e2e = time_graph(e2e_step, esteps, args.warmup, stream, dist) / esteps
         h2d = sum(q.numel() * q.element_size() for q in qs)
-        e2e = {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_gbs(step_bytes, ms_e2e, world), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d, "ms_per_step": ms_e2e}
 
     line = {
@@ -387,7 +400,7 @@ def run_fasa(args, wl):
     return 0
 
 
-def main(argv=None):
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -402,7 +415,11 @@ def main(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    args = ap.parse_args(argv)
+    return ap
+
+
+def main(argv=None):
+    args = build_parser().parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     wl = W.CONFIGS[args.config]
