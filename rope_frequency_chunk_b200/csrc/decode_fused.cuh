@@ -132,36 +132,40 @@ __host__ __device__ inline FuLayout fu_layout(int n_loc, int ring) {
   return L;
 }
 
-// The bin b of a 256-bin histogram (bin = key >> 24) holding the k-th
-// largest key, and the count in bins above it (k <= total). All threads;
-// thread t < 256 owns bin 255 - t; uses scan[0, 12).
-__device__ __forceinline__ void coarse_threshold(const uint32_t* h, int k, uint32_t* scan, uint32_t& bin,
-                                                 uint32_t& above) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t c = tid < 256 ? h[255 - tid] : 0u;
-  uint32_t incl = c;
+// One warp: the bin of a 256-bin histogram (bin = key >> 24) holding the
+// k-th largest key, and the count in higher bins (k <= total); lane l owns
+// bins 255 - 8l .. 248 - 8l. Every lane gets the result.
+__device__ __forceinline__ uint2 warp_bin256(const uint32_t* h, int k, int lane) {
+  uint32_t c[8], sum = 0u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    c[u] = h[255 - 8 * lane - u];
+    sum += c[u];
+  }
+  uint32_t incl = sum;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
     if (lane >= off) incl += v;
   }
-  if (lane == 31 && warp < 8) scan[warp] = incl;
-  if (tid == 0) scan[8] = scan[9] = 0u;  // (only reached when k exceeds the total)
-  __syncthreads();
-  if (tid < 256) {
-    uint32_t before = 0u;
-    for (int w = 0; w < warp; ++w) before += scan[w];
-    incl += before;
-    const uint32_t excl = incl - c;
-    if (excl < (uint32_t)k && (uint32_t)k <= incl) {
-      scan[8] = 255u - (uint32_t)tid;
-      scan[9] = excl;
+  const uint32_t excl = incl - sum;
+  const bool here = excl < (uint32_t)k && (uint32_t)k <= incl;
+  uint32_t bin = 0u, above = 0u;
+  if (here) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (acc + c[u] >= (uint32_t)k) {
+        bin = 255u - (uint32_t)(8 * lane + u);
+        above = acc;
+        break;
+      }
+      acc += c[u];
     }
   }
-  __syncthreads();
-  bin = min(scan[8], 255u);
-  above = scan[9];
-  __syncthreads();
+  const unsigned who = __ballot_sync(0xFFFFFFFFu, here);
+  const int src = who ? __ffs(who) - 1 : 0;
+  return make_uint2(__shfl_sync(0xFFFFFFFFu, bin, src), __shfl_sync(0xFFFFFFFFu, above, src));
 }
 
 // The bin of a 1024-bin histogram holding the k-th largest entry (counting
@@ -418,19 +422,25 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   for (int i = tid; i < C * 256; i += kFuThreads) cluster.map_shared_rank(hall, i >> 8)[cr * 256 + (i & 255)] = hloc[i & 255];
   cluster_arrive();  // histograms delivered; this CTA's ring is free for the union
   cluster_wait();
-  // the row's histogram, the boundary bin B and what lies above it
+  // the row's histogram (one bin per thread), then the boundary bin B by one warp
   if (tid < 256) {
     uint32_t t = 0u;
     for (int r = 0; r < C; ++r) t += hall[r * 256 + tid];
     hloc[tid] = t;
   }
-  __syncthreads();
-  uint32_t bin8, above8;
-  coarse_threshold(hloc, p.n_keep, scan, bin8, above8);
-  // second level: the 16 sub-bins (key bits 20..23) of bin B, counted here
-  // and written into every CTA
   if (tid < 16) hf_own[tid] = 0u;
   __syncthreads();
+  if (warp == 0) {
+    const uint2 b = warp_bin256(hloc, p.n_keep, lane);
+    if (lane == 0) {
+      scan[61] = b.x;
+      scan[62] = b.y;
+    }
+  }
+  __syncthreads();
+  const uint32_t bin8 = scan[61], above8 = scan[62];
+  // second level: the 16 sub-bins (key bits 20..23) of bin B, counted here
+  // and written into every CTA
   for (int i = tid; i < n; i += kFuThreads) {
     const uint32_t x = keys[i];
     if ((x >> 24) == bin8) atomicAdd(&hf_own[(x >> 20) & 15u], 1u);
@@ -439,28 +449,43 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   if (tid < C * 16) cluster.map_shared_rank(hfine, tid >> 4)[cr * 16 + (tid & 15)] = hf_own[tid & 15];
   cluster_arrive();
   cluster_wait();
-  // the boundary sub-bin: the 12-bit bin b12 holding the k_eff-th key
-  uint32_t above12 = above8, b12 = bin8 << 4;
-  {
-    uint32_t cum = above8;
-    for (int f = 15; f >= 0; --f) {
-      uint32_t c = 0u;
-      for (int r = 0; r < C; ++r) c += hfine[r * 16 + f];
-      if (cum + c >= (uint32_t)p.n_keep) {
-        b12 = (bin8 << 4) | (uint32_t)f;
-        above12 = cum;
-        break;
-      }
-      cum += c;
+  // one warp: the 12-bit bin b12 holding the k_eff-th key, the count above
+  // it, every rank's count inside it and their offsets in the union
+  uint32_t* uoff = hloc;  // [16] (the row histogram is no longer needed)
+  if (warp == 0) {
+    uint32_t cf = 0u;  // lane l < 16: sub-bin 15 - l of the row
+    if (lane < 16)
+      for (int r = 0; r < C; ++r) cf += hfine[r * 16 + (15 - lane)];
+    uint32_t incl = cf;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o2);
+      if (lane >= o2) incl += v;
+    }
+    const uint32_t excl = incl - cf;
+    const unsigned hit = __ballot_sync(0xFFFFFFFFu, lane < 16 && above8 + excl < (uint32_t)p.n_keep &&
+                                                        (uint32_t)p.n_keep <= above8 + incl);
+    const int fl = hit ? __ffs(hit) - 1 : 0;
+    const uint32_t f12 = 15u - (uint32_t)fl;
+    const uint32_t ab = above8 + __shfl_sync(0xFFFFFFFFu, excl, fl);
+    const uint32_t nr = lane < C ? hfine[lane * 16 + f12] : 0u;
+    uint32_t inr = nr;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, inr, o2);
+      if (lane >= o2) inr += v;
+    }
+    if (lane < C) uoff[lane] = inr - nr;
+    if (lane == 31) {
+      scan[56] = (bin8 << 4) | f12;
+      scan[57] = ab;
+      scan[58] = inr;
     }
   }
+  __syncthreads();
+  const uint32_t b12 = scan[56], above12 = scan[57], n_b = scan[58];
   const int krem12 = p.n_keep - (int)above12;  // keys of bin b12 still to take (>= 1)
-  uint32_t off = 0u, n_b = 0u;                 // this CTA's offset in the union, the union's size
-  for (int r = 0; r < C; ++r) {
-    const uint32_t c = hfine[r * 16 + (b12 & 15u)];
-    off += (r < cr) ? c : 0u;
-    n_b += c;
-  }
+  const uint32_t off = uoff[cr];               // this CTA's offset in the union
   const bool exact = n_b <= (uint32_t)p.ucap;  // the same in every CTA
   auto in_bin = [keys, b12](int i) { return (keys[i] >> 20) == b12; };
   if (exact) {
