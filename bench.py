@@ -378,10 +378,11 @@ def run_fasa(args, wl):
                             "frac": gbs / world / hbm_peak, "bytes_per_layer_step": per_layer_bytes,
                             "peak_kind": peak_kind},
         "roofline": roof,
-        "decode_plan": "fused" if fused else "staged",
+        "decode_plan": {F.DECODE_FUSED: "fused", F.DECODE_SCORED: "scored"}.get(plan, "staged"),
         "clocks": clocks,
-        # kernels of this library per layer: fused 1; staged 4 (score, filter, finalize, attend)
-        "gpu_launches": (1 if fused else 4) * n_layers * args.steps,
+        # kernels of this library per layer: fused 1; scored 2 (score stream, cluster select + attend);
+        # staged 4 (score, filter, finalize, attend)
+        "gpu_launches": {F.DECODE_FUSED: 1, F.DECODE_SCORED: 2}.get(plan, 4) * n_layers * args.steps,
         "e2e": e2e,
     }
     line.update(extra)
@@ -411,6 +412,7 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--k", type=int, default=0)
     ap.add_argument("--ctx-len", type=int, default=0)
     ap.add_argument("--n-dom", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -427,6 +429,8 @@ def main(argv=None):
         wl = wl.replace(ctx_len=args.ctx_len, k=W.c4_budget(args.ctx_len) if wl.name == "c4" else wl.k)
     if args.n_dom:
         wl = wl.replace(n_dom=args.n_dom)
+    if args.batch:
+        wl = wl.replace(batch=args.batch)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_fasa(args, wl)

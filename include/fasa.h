@@ -204,6 +204,11 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *    exact radix select of the k-th key over distributed shared memory, each
  *    CTA attends its kept rows, and the partials are merged in the cluster.
  *    The workspace is not touched.
+ *  FASA_DECODE_SCORED  (bf16 caches whose rows fit 16 CTAs of 16384 tokens,
+ *    within about two waves of clusters when not forced) two launches: the
+ *    score stream writes the TIP scores to the workspace, then the same
+ *    cluster kernel as FASA_DECODE_FUSED reads them (from L2) instead of the
+ *    sketch and selects and attends.
  *  FASA_DECODE_STAGED  four launches chained with programmatic dependent
  *    launch: the score stream, which also builds a per-row histogram of the
  *    score keys; a filter that marks the certainly-kept tokens and collects
@@ -231,14 +236,15 @@ fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int
 #define FASA_DECODE_AUTO 0   /* chosen from the shape (default) */
 #define FASA_DECODE_FUSED 1  /* single-launch cluster decode */
 #define FASA_DECODE_STAGED 2 /* four-launch decode */
+#define FASA_DECODE_SCORED 3 /* two launches: the score stream, then the cluster select + attend */
 
 /* Sets the plan every later fasa_decode call of this process uses (a
  * process-wide setting; FASA_ERR_INVALID_ARG for an unknown value). */
 fasa_status fasa_set_decode_path(int32_t path);
 
 /* The plan fasa_decode would run for this cache, len and k under the current
- * setting and on the current device: FASA_DECODE_FUSED or FASA_DECODE_STAGED,
- * or a negative fasa_status for invalid arguments. */
+ * setting and on the current device: FASA_DECODE_FUSED, FASA_DECODE_SCORED or
+ * FASA_DECODE_STAGED, or a negative fasa_status for invalid arguments. */
 int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
 
 /* Size of the library's own device scratch used by

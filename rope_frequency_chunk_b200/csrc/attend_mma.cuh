@@ -1,4 +1,4 @@
-// Focused attention of the fused decode on tensor cores (bf16 caches).
+// Focused attention of the staged decode on tensor cores (bf16 caches).
 //
 // "FASA: Frequency-aware Sparse Attention" (gist.science technical summary,
 // §2, FAC bullets): full softmax attention of each query head over exactly
@@ -16,9 +16,11 @@
 //   O[16 x 128] += P[16 x 16] V     (K = 16 rows, N = head dim)
 // with an online base-2 softmax in registers (the 1/sqrt(128) and log2(e)
 // scale folded into Q). Q is split into three bf16 terms (about 24 bits, as
-// float32) and P into two (P is in [0, 1] and only weights V); K and V are
-// bf16 already and enter exactly. The warps
-// of a CTA are merged in shared memory; the CTA writes its partial
+// float32), prepared once per row by the selection kernel and read here with
+// ldmatrix; each term accumulates in its own registers so the three MMA
+// chains run side by side. P is split into two terms (P is in [0, 1] and only
+// weights V); K and V are bf16 already and enter exactly. The warps of a CTA
+// are merged pairwise through shared memory; the CTA writes its partial
 // (m, l, o) to the workspace and the row's last CTA (atomic counter) merges
 // the splits and writes the bf16 output.
 #pragma once
@@ -34,12 +36,14 @@ constexpr int kAttStages = 3;                          // per-warp ring depth
 constexpr int kAttHalf = kAttChunk * kD * 2;           // bytes of 16 bf16 rows (K or V)
 constexpr int kAttStageBytes = 2 * kAttHalf;           // K + V
 constexpr int kAttPartStride = 16 * kD + 32;           // floats: m[16], l[16], o[16][128]
+constexpr int kQTermBytes = 3 * 16 * kD * 2;           // the three bf16 terms of 16 query rows
+constexpr int kAttSlot = 68 * 32;                      // floats of one warp's (o, m, l) fragments
 
 struct AttParams {
   const __nv_bfloat16* k;   // [rows][max_len][128]
   const __nv_bfloat16* v;
   const int32_t* idx;       // [rows][n_keep] kept rows; null: rows 0 .. n_keep-1
-  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
+  const unsigned char* qterms;  // [rows][kQTermBytes] query terms (see query_terms)
   __nv_bfloat16* out;       // [B][Hq][128]
   float* part;              // [rows][splits][kAttPartStride]
   uint32_t* counter;        // [rows], zero before the launch; the last CTA resets it
@@ -49,11 +53,10 @@ struct AttParams {
   int32_t slice;            // rows per CTA, a multiple of kAttChunk
   int32_t splits;
   int32_t group;
-  double cosv[kNFC];        // cos / sin of q_pos * theta_i (host, float64)
-  double sinv[kNFC];
 };
 
-__host__ __device__ constexpr int att_smem_bytes() { return kAttWarps * kAttStages * kAttStageBytes + 16 * kD * 4; }
+__host__ __device__ constexpr int att_smem_bytes() { return kAttWarps * kAttStages * kAttStageBytes + kQTermBytes; }
+static_assert(kAttSlot * 4 * (kAttWarps / 2) <= kAttWarps * kAttStages * kAttStageBytes, "merge slots exceed the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -84,50 +87,80 @@ __device__ __forceinline__ float2 split_pack(float x, float y, uint32_t& hi, uin
   return r;
 }
 
+// Attention queries of the group: rotated, scaled by log2(e)/sqrt(128),
+// rounded to float32, then split into three bf16 terms (low, middle, high)
+// stored as rows of 256 B with 16-byte chunks XOR-swizzled by row for
+// ldmatrix; heads >= G are zero. Threads tid < nthreads share the work.
+__device__ __forceinline__ void query_terms(const __nv_bfloat16* qraw, int G, const double* cosv, const double* sinv,
+                                            unsigned char* qt, int tid, int nthreads) {
+  const double qscale = 1.4426950408889634 / 11.313708498984761;
+  for (int e = tid; e < 16 * kD / 2; e += nthreads) {
+    const int h = e / (kD / 2), d = 2 * (e % (kD / 2));
+    float v2[2] = {0.0f, 0.0f};
+    if (h < G) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int dd = d + u, i = dd & (kNFC - 1);
+        const double x = __bfloat162float(qraw[h * kD + i]);
+        const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
+        const double c = cosv[i], sn = sinv[i];
+        v2[u] = (float)(((dd < kNFC) ? (x * c - y * sn) : (y * c + x * sn)) * qscale);
+      }
+    }
+    uint32_t hi, mid, lo;
+    const float2 r = split_pack(v2[0], v2[1], hi, mid);
+    const float2 mf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&mid));
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(r.x - mf.x, r.y - mf.y);
+    lo = *reinterpret_cast<const uint32_t*>(&ll);
+    const int off = h * 256 + (((d / 8) ^ (h & 7)) * 16) + (d % 8) * 2;
+    *reinterpret_cast<uint32_t*>(qt + 0 * 4096 + off) = lo;
+    *reinterpret_cast<uint32_t*>(qt + 1 * 4096 + off) = mid;
+    *reinterpret_cast<uint32_t*>(qt + 2 * 4096 + off) = hi;
+  }
+}
+
+// S = Q K^T for one 16-row chunk staged at Ks: s0 rows 0-7, s1 rows 8-15 of
+// the chunk (fragment layout of m16n8k16), each Q term in its own chain.
+__device__ __forceinline__ void chunk_logits(const unsigned char* qt, const unsigned char* Ks, int lane, float (&s0)[4],
+                                             float (&s1)[4]) {
+  float a0[3][4], a1[3][4];
+#pragma unroll
+  for (int t = 0; t < 3; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a0[t][e] = a1[t][e] = 0.0f;
+  const int arow = (lane % 8) + ((lane / 8) % 2) * 8;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t b[4];
+    ldsm_x4(b, Ks + ((lane / 16) * 8 + lane % 8) * 256 + (((ks * 2 + (lane / 8) % 2) ^ (lane % 8)) * 16));
+    const int aoff = arow * 256 + (((ks * 2 + lane / 16) ^ (arow & 7)) * 16);
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {  // low, middle, high bf16 term of Q
+      uint32_t a[4];
+      ldsm_x4(a, qt + t * 4096 + aoff);
+      mma_16816(a0[t], a, b[0], b[1]);
+      mma_16816(a1[t], a, b[2], b[3]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    s0[e] = (a0[0][e] + a0[1][e]) + a0[2][e];
+    s1[e] = (a1[0][e] + a1[1][e]) + a1[2][e];
+  }
+}
+
 __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   grid_dependency_wait();
   const int split = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.group;
-  float* qs = reinterpret_cast<float*>(smem + kAttWarps * kAttStages * kAttStageBytes);  // [16][128]
-
-  // rotated, pre-scaled queries: q'_h * log2(e) / sqrt(128); rows >= G are
-  // zero. The raw rows are first brought into shared memory in one go.
+  unsigned char* qt = smem + kAttWarps * kAttStages * kAttStageBytes;
   {
-    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);  // ring area, free until the gathers
-    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)row * G) * kD);
-    for (int c = tid; c < G * kD / 8; c += kAttThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
-    __syncthreads();
-    const double qscale = 1.4426950408889634 / 11.313708498984761;
-    for (int e = tid; e < 16 * kD; e += kAttThreads) {
-      const int h = e / kD, d = e % kD, i = d & (kNFC - 1);
-      float val = 0.0f;
-      if (h < G) {
-        const double x = __bfloat162float(qraw[h * kD + i]);
-        const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
-        const double c = p.cosv[i], s = p.sinv[i];
-        val = (float)(((d < kNFC) ? (x * c - y * s) : (y * c + x * s)) * qscale);
-      }
-      qs[e] = val;
-    }
+    const unsigned char* src = p.qterms + (int64_t)row * kQTermBytes;
+    for (int c = tid; c < kQTermBytes / 16; c += kAttThreads) cp_async16(qt + c * 16, src + c * 16);
+    cp_async_commit();
   }
-  __syncthreads();
-  // A fragments of Q for the 8 k-steps as three bf16 terms (about 24 bits,
-  // so large logits keep float32 accuracy)
-  uint32_t ah[8][4], am[8][4], al[8][4];
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = lane / 4 + (j & 1) * 8;
-      const int c = ks * 16 + (lane % 4) * 2 + (j >> 1) * 8;
-      const float2 res = split_pack(qs[r * kD + c], qs[r * kD + c + 1], ah[ks][j], am[ks][j]);
-      const __nv_bfloat162 mm = *reinterpret_cast<const __nv_bfloat162*>(&am[ks][j]);
-      const float2 mf = __bfloat1622float2(mm);
-      const __nv_bfloat162 ll = __floats2bfloat162_rn(res.x - mf.x, res.y - mf.y);
-      al[ks][j] = *reinterpret_cast<const uint32_t*>(&ll);
-    }
 
   const int r_beg = split * p.slice;
   const int r_end = min(p.n_keep, r_beg + p.slice);
@@ -148,14 +181,17 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
     if (ci < mine) {
       const int j0 = r_beg + (warp + ci * kAttWarps) * kAttChunk;
       unsigned char* st = ring + (ci % kAttStages) * kAttStageBytes;
+      int tr = lane < kAttChunk ? row_of(j0 + lane) : 0;
+      if (tr < 0) {
+        if (lane < kAttChunk && j0 + lane < r_end) flag_status(FASA_ERR_BAD_INDEX);
+        tr = 0;  // masked below
+      }
 #pragma unroll
-      for (int x = lane; x < kAttChunk * 32; x += 32) {  // 16 rows x (16 K + 16 V) 16-byte parts
-        const int r = x / 32, part = x % 32;
-        int t = row_of(j0 + r);
-        if (t < 0) t = 0;  // masked below
-        const __nv_bfloat16* src = (part < 16 ? kb : vb) + (int64_t)t * kD + (part % 16) * 8;
+      for (int r = 0; r < kAttChunk; ++r) {  // 16 rows x (16 K + 16 V) 16-byte parts, one part per lane
+        const int t = __shfl_sync(0xFFFFFFFFu, tr, r);
+        const __nv_bfloat16* src = (lane < 16 ? kb : vb) + (int64_t)t * kD + (lane % 16) * 8;
         // 16-byte chunk c of row r is stored at chunk c ^ (r & 7) (bank-conflict-free ldmatrix)
-        cp_async16(st + (part < 16 ? 0 : kAttHalf) + r * 256 + (((part % 16) ^ (r & 7)) * 16), src);
+        cp_async16(st + (lane < 16 ? 0 : kAttHalf) + r * 256 + (((lane % 16) ^ (r & 7)) * 16), src);
       }
     }
     cp_async_commit();
@@ -170,23 +206,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
 
 #pragma unroll
   for (int s = 0; s < kAttStages; ++s) issue(s);
+  cp_async_wait<kAttStages>();  // the query terms (the oldest group)
+  __syncthreads();
   for (int ci = 0; ci < mine; ++ci) {
     cp_async_wait<kAttStages - 1>();
     __syncwarp();
     const unsigned char* Ks = ring + (ci % kAttStages) * kAttStageBytes;
     const unsigned char* Vs = Ks + kAttHalf;
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};  // rows 0-7, 8-15 of the chunk
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t b[4];
-      ldsm_x4(b, Ks + ((lane / 16) * 8 + lane % 8) * 256 + (((ks * 2 + (lane / 8) % 2) ^ (lane % 8)) * 16));
-      mma_16816(s0, al[ks], b[0], b[1]);
-      mma_16816(s0, am[ks], b[0], b[1]);
-      mma_16816(s0, ah[ks], b[0], b[1]);
-      mma_16816(s1, al[ks], b[2], b[3]);
-      mma_16816(s1, am[ks], b[2], b[3]);
-      mma_16816(s1, ah[ks], b[2], b[3]);
-    }
+    float s0[4], s1[4];  // rows 0-7, 8-15 of the chunk
+    chunk_logits(qt, Ks, lane, s0, s1);
     // mask the chunk's missing or invalid rows (columns of S)
     const int j0 = r_beg + (warp + ci * kAttWarps) * kAttChunk;
     const int c0 = (lane % 4) * 2;
@@ -243,55 +271,62 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
     issue(ci + kAttStages);
   }
   cp_async_wait<0>();
-  l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
-  l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
-  l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
-  l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
 
-  // merge the CTA's warps through shared memory (the rings are free now)
-  __syncthreads();
-  float* wm = reinterpret_cast<float*>(smem);   // [warp][16] running max
-  float* wl = wm + kAttWarps * 16;              // [warp][16] sums
-  float* wo = wl + kAttWarps * 16;              // [warp][16][128]
-  if (lane % 4 == 0) {
-    wm[warp * 16 + lane / 4] = m0;
-    wm[warp * 16 + lane / 4 + 8] = m1;
-    wl[warp * 16 + lane / 4] = l0;
-    wl[warp * 16 + lane / 4 + 8] = l1;
-  }
+  // warps merged pairwise through shared memory (the rings are free now):
+  // warps [h, 2h) hand their fragments to warps [0, h), lane-major slots
+  float* slots = reinterpret_cast<float*>(smem);
+#pragma unroll 1
+  for (int half = kAttWarps / 2; half >= 1; half >>= 1) {
+    __syncthreads();
+    if (warp >= half && warp < 2 * half) {
+      float* sl = slots + (warp - half) * kAttSlot;
 #pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    const int d = n * 8 + (lane % 4) * 2;
-    wo[(warp * 16 + lane / 4) * kD + d] = o[n][0];
-    wo[(warp * 16 + lane / 4) * kD + d + 1] = o[n][1];
-    wo[(warp * 16 + lane / 4 + 8) * kD + d] = o[n][2];
-    wo[(warp * 16 + lane / 4 + 8) * kD + d + 1] = o[n][3];
-  }
-  __syncthreads();
-  float* pp = p.part + ((int64_t)row * p.splits + split) * kAttPartStride;
-  for (int e = tid; e < 16 * kD; e += kAttThreads) {
-    const int h = e / kD;
-    float M = -INFINITY;
+      for (int n = 0; n < 16; ++n)
 #pragma unroll
-    for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, wm[w * 16 + h]);
-    float acc = 0.0f;
-    if (M != -INFINITY)
+        for (int e = 0; e < 4; ++e) sl[(n * 4 + e) * 32 + lane] = o[n][e];
+      sl[64 * 32 + lane] = m0;
+      sl[65 * 32 + lane] = m1;
+      sl[66 * 32 + lane] = l0;
+      sl[67 * 32 + lane] = l1;
+    }
+    __syncthreads();
+    if (warp < half) {
+      const float* sl = slots + warp * kAttSlot;
+      const float pm0 = sl[64 * 32 + lane], pm1 = sl[65 * 32 + lane];
+      const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
+      const float a0 = (m0 == -INFINITY) ? 0.0f : exp2f(m0 - n0), a1 = (m1 == -INFINITY) ? 0.0f : exp2f(m1 - n1);
+      const float b0 = (pm0 == -INFINITY) ? 0.0f : exp2f(pm0 - n0), b1 = (pm1 == -INFINITY) ? 0.0f : exp2f(pm1 - n1);
 #pragma unroll
-      for (int w = 0; w < kAttWarps; ++w) {
-        const float mw = wm[w * 16 + h];
-        if (mw != -INFINITY) acc += exp2f(mw - M) * wo[(w * 16 + h) * kD + e % kD];
+      for (int n = 0; n < 16; ++n) {
+        o[n][0] = o[n][0] * a0 + sl[(n * 4 + 0) * 32 + lane] * b0;
+        o[n][1] = o[n][1] * a0 + sl[(n * 4 + 1) * 32 + lane] * b0;
+        o[n][2] = o[n][2] * a1 + sl[(n * 4 + 2) * 32 + lane] * b1;
+        o[n][3] = o[n][3] * a1 + sl[(n * 4 + 3) * 32 + lane] * b1;
       }
-    pp[32 + e] = acc;
-    if (e % kD == 0) {
-      float L = 0.0f;
-      if (M != -INFINITY)
+      l0 = l0 * a0 + sl[66 * 32 + lane] * b0;
+      l1 = l1 * a1 + sl[67 * 32 + lane] * b1;
+      m0 = n0;
+      m1 = n1;
+    }
+  }
+  // warp 0: the CTA's partial (m, l, o) to the workspace
+  float* pp = p.part + ((int64_t)row * p.splits + split) * kAttPartStride;
+  if (warp == 0) {
+    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
+    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
+    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
+    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
+    if (lane % 4 == 0) {
+      pp[lane / 4] = m0;
+      pp[lane / 4 + 8] = m1;
+      pp[16 + lane / 4] = l0;
+      pp[16 + lane / 4 + 8] = l1;
+    }
 #pragma unroll
-        for (int w = 0; w < kAttWarps; ++w) {
-          const float mw = wm[w * 16 + h];
-          if (mw != -INFINITY) L += exp2f(mw - M) * wl[w * 16 + h];
-        }
-      pp[h] = M;
-      pp[16 + h] = L;
+    for (int n = 0; n < 16; ++n) {
+      const int d = n * 8 + (lane % 4) * 2;
+      *reinterpret_cast<float2*>(pp + 32 + (lane / 4) * kD + d) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(pp + 32 + (lane / 4 + 8) * kD + d) = make_float2(o[n][2], o[n][3]);
     }
   }
   // the row's last CTA merges all splits

@@ -46,7 +46,7 @@ constexpr int kFuWarps = kFuThreads / 32;
 constexpr int kFuScoreWarps = kFuWarps - 1;  // + one producer warp
 constexpr int kFuMaxStages = 16;
 constexpr int kFuMinRing = kFuWarps * kAttStageBytes;  // 128 KB: one K+V chunk per warp
-constexpr int kFuMaxLoc = 8192;                         // tokens per CTA
+constexpr int kFuMaxLoc = 16384;                        // tokens per CTA
 constexpr int kFuMaxCluster = 16;
 constexpr int kFuSlot = 68 * 32;  // floats of one warp's (o, m, l) fragments in the warp merge
 constexpr int kFuPartOff = 98304; // byte offset of the CTA partial inside the ring
@@ -68,6 +68,7 @@ enum FuXch { kXTies = 0, kXKept = 1, kXRows = 2 };
 
 struct FusedParams {
   const __nv_bfloat16* sketch;  // [rows][max_len][stride]
+  const float* scores;          // [rows][len] TIP scores (the from-scores variant), else unused
   const __nv_bfloat16* k;       // [rows][max_len][128], rotated
   const __nv_bfloat16* v;
   const __nv_bfloat16* q;       // [B][Hq][128], pre-RoPE
@@ -279,7 +280,9 @@ __device__ __forceinline__ void fu_visit(int n, uint32_t before, Pred&& pred, Fn
   }
 }
 
-template <int LPT>
+// kFromScores: phase 1 reads the TIP scores a score-kernel launch wrote
+// (L2-resident) instead of streaming and scoring the sketch; LPT is unused.
+template <int LPT, bool kFromScores>
 __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const FusedParams p) {
   using T = __nv_bfloat16;
   using S = ScoreShape<T, LPT>;
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   // tokens: warm L2 with this CTA's range while the previous kernel in the
   // stream may still run (the reads proper wait for it), and let the next
   // kernel's CTAs start on free SMs to do the same
-  if (warp == kFuScoreWarps && lane == 0 && n > 0) {
+  if (!kFromScores && warp == kFuScoreWarps && lane == 0 && n > 0) {
     const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
     for (int t = 0; t < n; t += TPS) prefetch_l2(src + (int64_t)t * S::ROWB, (uint32_t)(min(TPS, n - t) * S::ROWB));
   }
@@ -346,7 +349,29 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
   grid_dependency_wait();
 
   // ---------------------------------------------------------------- 1. score
-  if (warp == kFuScoreWarps) {
+  if constexpr (kFromScores) {
+    {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
+      for (int c = tid; c < G * kD / 8; c += kFuThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    }
+    __syncthreads();
+    query_terms(qraw, G, p.cosv, p.sinv, qt, tid, kFuThreads);
+    // the row's scores of this CTA's range: keys and the top-8-bit histogram
+    const float* src = p.scores + (int64_t)row * p.len + t0;
+    constexpr int U = 8;
+    for (int i0 = tid; i0 < n; i0 += kFuThreads * U) {
+      float f[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) f[u] = i0 + u * kFuThreads < n ? __ldcg(src + i0 + u * kFuThreads) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u * kFuThreads < n) {
+          const uint32_t key = score_key(f[u]);
+          keys[i0 + u * kFuThreads] = key;
+          atomicAdd(&hloc[key >> 24], 1u);
+        }
+    }
+  } else if (warp == kFuScoreWarps) {
     // the stream starts before the query work of the other warps
     if (lane == 0 && n > 0) {
       const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
@@ -369,32 +394,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
     }
     named_barrier_sync(1, kFuScoreWarps * 32);
     query_coefs<T>(qraw, s_dom, G, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
-    // attention queries: rotated, scaled by log2(e)/sqrt(128), rounded to
-    // float32, then split into three bf16 terms; heads >= G are zero
-    const double qscale = 1.4426950408889634 / 11.313708498984761;
-    for (int e = tid; e < 16 * kD / 2; e += kFuScoreWarps * 32) {
-      const int h = e / (kD / 2), d = 2 * (e % (kD / 2));
-      float v2[2] = {0.0f, 0.0f};
-      if (h < G) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int dd = d + u, i = dd & (kNFC - 1);
-          const double x = __bfloat162float(qraw[h * kD + i]);
-          const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
-          const double c = p.cosv[i], sn = p.sinv[i];
-          v2[u] = (float)(((dd < kNFC) ? (x * c - y * sn) : (y * c + x * sn)) * qscale);
-        }
-      }
-      uint32_t hi, mid, lo;
-      const float2 r = split_pack(v2[0], v2[1], hi, mid);
-      const float2 mf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&mid));
-      const __nv_bfloat162 ll = __floats2bfloat162_rn(r.x - mf.x, r.y - mf.y);
-      lo = *reinterpret_cast<const uint32_t*>(&ll);
-      const int off = h * 256 + (((d / 8) ^ (h & 7)) * 16) + (d % 8) * 2;
-      *reinterpret_cast<uint32_t*>(qt + 0 * 4096 + off) = lo;
-      *reinterpret_cast<uint32_t*>(qt + 1 * 4096 + off) = mid;
-      *reinterpret_cast<uint32_t*>(qt + 2 * 4096 + off) = hi;
-    }
+    query_terms(qraw, G, p.cosv, p.sinv, qt, tid, kFuScoreWarps * 32);
     named_barrier_sync(1, kFuScoreWarps * 32);
     double qr[S::EPL];
     load_coefs<T, LPT>(qr, s_q, lane);

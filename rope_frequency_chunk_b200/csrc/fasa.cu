@@ -344,9 +344,9 @@ struct FusedPlan {
   int C = 0, n_loc = 0, ring = 0, n_stages = 0, ucap = 0, smem = 0, waves = 0;
 };
 
-template <int LPT>
+template <int LPT, bool kSc>
 fasa_status fused_attrs(const DevInfo& d) {
-  auto kern = decode_fused_kernel<LPT>;
+  auto kern = decode_fused_kernel<LPT, kSc>;
   int set = 0;
   return cached_int((const void*)kern, 0, &set, [&](int* v) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin);
@@ -357,10 +357,10 @@ fasa_status fused_attrs(const DevInfo& d) {
 }
 
 // Clusters of size C with `smem` bytes per CTA that fit on the GPU at once.
-template <int LPT>
+template <int LPT, bool kSc>
 fasa_status fused_max_clusters(int C, int smem, const DevInfo& d, int* out) {
-  auto kern = decode_fused_kernel<LPT>;
-  fasa_status s = fused_attrs<LPT>(d);
+  auto kern = decode_fused_kernel<LPT, kSc>;
+  fasa_status s = fused_attrs<LPT, kSc>(d);
   if (s != FASA_OK) return s;
   return cached_int((const void*)kern, 3000ull + (uint64_t)C * 1000003ull + (uint64_t)smem, out, [&](int* v) {
     cudaLaunchConfig_t cfg = {};
@@ -384,10 +384,12 @@ fasa_status fused_max_clusters(int C, int smem, const DevInfo& d, int* out) {
   });
 }
 
-// Shape of the single-launch decode for cluster size C: tokens per CTA and
-// the ring (every score stage in flight when shared memory allows; at least
-// one K+V chunk per warp), which after scoring holds the boundary bin's union.
-template <int LPT>
+// Shape of the cluster decode for cluster size C: tokens per CTA and the ring,
+// which after phase 1 holds the boundary bin's union and later one K+V chunk
+// per warp. Streaming the sketch (kSc false), the ring also holds every
+// score stage in flight when shared memory allows; reading scores (kSc
+// true) it has no stages.
+template <int LPT, bool kSc>
 bool fused_shape(int C, int32_t len, const DevInfo& d, FusedPlan* pl) {
   constexpr int kStage = fu_stage_bytes<LPT>();
   constexpr int TPS = kStage / (LPT * 16);
@@ -396,32 +398,39 @@ bool fused_shape(int C, int32_t len, const DevInfo& d, FusedPlan* pl) {
   if (pl->n_loc > kFuMaxLoc) return false;
   const int ring_max = (d.smem_optin - fu_layout(pl->n_loc, 0).total) / 128 * 128;
   if (ring_max < kFuMinRing) return false;
-  pl->n_stages = (int)std::min<int64_t>(std::min<int64_t>(kFuMaxStages, ring_max / kStage), ceil_div(pl->n_loc, TPS));
-  if (pl->n_stages < 1) return false;
-  pl->ring = std::max(kFuMinRing, (pl->n_stages * kStage + 127) / 128 * 128);
+  if (kSc) {
+    pl->n_stages = 0;
+    pl->ring = kFuMinRing;
+  } else {
+    pl->n_stages =
+        (int)std::min<int64_t>(std::min<int64_t>(kFuMaxStages, ring_max / kStage), ceil_div(pl->n_loc, TPS));
+    if (pl->n_stages < 1) return false;
+    pl->ring = std::max(kFuMinRing, (pl->n_stages * kStage + 127) / 128 * 128);
+  }
   pl->ucap = (pl->ring - kFuRadixBytes) / 8;
   pl->smem = fu_layout(pl->n_loc, pl->ring).total;
   return pl->smem <= d.smem_optin;
 }
 
 // Picks the cluster size: fewest waves of clusters first, then the least
-// per-CTA streaming (a wave costs about a 4096-token CTA of fixed latency).
-// Not eligible (false) for rows too long or, unless forced, more than two
-// waves.
-template <int LPT>
-fasa_status fused_plan_t(int rows, int32_t len, int keff, const DevInfo& d, bool forced, FusedPlan* out, bool* ok) {
+// per-CTA work (a wave costs about a 4096-token CTA of fixed latency; a
+// token read as a score costs an eighth of one streamed as a sketch row).
+// Neither is eligible (false), unless forced, beyond two waves: each wave
+// repeats the kernel's serial select-and-attend chain.
+template <int LPT, bool kSc>
+fasa_status fused_plan_t(int rows, int32_t len, const DevInfo& d, bool forced, FusedPlan* out, bool* ok) {
   static const int kSizes[] = {16, 15, 14, 13, 12, 10, 8, 6, 4, 3, 2, 1};
   *ok = false;
   int64_t best = -1;
   for (int C : kSizes) {
     FusedPlan pl;
-    if (!fused_shape<LPT>(C, len, d, &pl)) continue;
+    if (!fused_shape<LPT, kSc>(C, len, d, &pl)) continue;
     int maxc = 0;
-    fasa_status s = fused_max_clusters<LPT>(C, pl.smem, d, &maxc);
+    fasa_status s = fused_max_clusters<LPT, kSc>(C, pl.smem, d, &maxc);
     if (s != FASA_OK) return s;
     if (maxc < 1) continue;
     pl.waves = (int)ceil_div(rows, maxc);
-    const int64_t cost = (int64_t)pl.waves * (pl.n_loc + 4096);
+    const int64_t cost = (int64_t)pl.waves * ((kSc ? pl.n_loc / 8 : pl.n_loc) + 4096);
     if (best < 0 || cost < best) {
       best = cost;
       *out = pl;
@@ -431,25 +440,28 @@ fasa_status fused_plan_t(int rows, int32_t len, int keff, const DevInfo& d, bool
   return FASA_OK;
 }
 
-fasa_status fused_plan(const fasa_cache* c, int32_t len, int keff, const DevInfo& d, bool forced, FusedPlan* out,
+// Plan of the single-launch decode (scored false) or of the cluster decode
+// that reads a score-kernel launch's scores (scored true); bf16 caches only.
+fasa_status fused_plan(const fasa_cache* c, int32_t len, const DevInfo& d, bool forced, bool scored, FusedPlan* out,
                        bool* ok) {
   *ok = false;
   if (c->dtype != FASA_BF16) return FASA_OK;
   const int rows = c->batch * c->n_kv_heads;
+  if (scored) return fused_plan_t<1, true>(rows, len, d, forced, out, ok);
   switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
-    case 1: return fused_plan_t<1>(rows, len, keff, d, forced, out, ok);
-    case 2: return fused_plan_t<2>(rows, len, keff, d, forced, out, ok);
-    case 4: return fused_plan_t<4>(rows, len, keff, d, forced, out, ok);
-    case 8: return fused_plan_t<8>(rows, len, keff, d, forced, out, ok);
-    case 16: return fused_plan_t<16>(rows, len, keff, d, forced, out, ok);
+    case 1: return fused_plan_t<1, false>(rows, len, d, forced, out, ok);
+    case 2: return fused_plan_t<2, false>(rows, len, d, forced, out, ok);
+    case 4: return fused_plan_t<4, false>(rows, len, d, forced, out, ok);
+    case 8: return fused_plan_t<8, false>(rows, len, d, forced, out, ok);
+    case 16: return fused_plan_t<16, false>(rows, len, d, forced, out, ok);
     default: return FASA_OK;
   }
 }
 
-template <int LPT>
+template <int LPT, bool kSc>
 fasa_status launch_fused_t(const FusedParams& p, int rows, const FusedPlan& pl, cudaStream_t st, const DevInfo& d) {
-  auto kern = decode_fused_kernel<LPT>;
-  fasa_status s = fused_attrs<LPT>(d);
+  auto kern = decode_fused_kernel<LPT, kSc>;
+  fasa_status s = fused_attrs<LPT, kSc>(d);
   if (s != FASA_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attrs[2];
@@ -468,10 +480,14 @@ fasa_status launch_fused_t(const FusedParams& p, int rows, const FusedPlan& pl, 
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
+// The cluster decode: streaming the sketch when scores is null, else reading
+// the scores [rows][len] a score-kernel launch wrote before it in the stream.
 fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t keff, void* out,
-                         int32_t* idx_out, const FusedPlan& pl, cudaStream_t st, const DevInfo& d) {
+                         int32_t* idx_out, const float* scores, const FusedPlan& pl, cudaStream_t st,
+                         const DevInfo& d) {
   FusedParams p{};
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
+  p.scores = scores;
   p.k = static_cast<const __nv_bfloat16*>(c->k);
   p.v = static_cast<const __nv_bfloat16*>(c->v);
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -491,12 +507,13 @@ fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_
   p.ucap = pl.ucap;
   fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   const int rows = c->batch * c->n_kv_heads;
+  if (scores != nullptr) return launch_fused_t<1, true>(p, rows, pl, st, d);
   switch (c->sketch_stride / 8) {
-    case 1: return launch_fused_t<1>(p, rows, pl, st, d);
-    case 2: return launch_fused_t<2>(p, rows, pl, st, d);
-    case 4: return launch_fused_t<4>(p, rows, pl, st, d);
-    case 8: return launch_fused_t<8>(p, rows, pl, st, d);
-    case 16: return launch_fused_t<16>(p, rows, pl, st, d);
+    case 1: return launch_fused_t<1, false>(p, rows, pl, st, d);
+    case 2: return launch_fused_t<2, false>(p, rows, pl, st, d);
+    case 4: return launch_fused_t<4, false>(p, rows, pl, st, d);
+    case 8: return launch_fused_t<8, false>(p, rows, pl, st, d);
+    case 16: return launch_fused_t<16, false>(p, rows, pl, st, d);
     default: return FASA_ERR_UNSUPPORTED;
   }
 }
@@ -505,11 +522,11 @@ fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_
 //   scores [rows][len] f32 | hist [rows][4096] u32 | cand_cnt [rows] u32 |
 //   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | idx [rows][k_eff] i32 |
-//   part [rows][splits_max][kAttPartStride] f32
+//   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
 // hist, cand_cnt and att_cnt are cleared at the start of every call.
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 struct DecodeWs {
-  size_t scores, hist, cnt, att_cnt, bitmap, cand, idx, part, total;
+  size_t scores, hist, cnt, att_cnt, bitmap, cand, idx, part, qterm, total;
   int cap, words, splits_max;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -533,7 +550,8 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
   w.idx = al256(w.cand + rows * (size_t)w.cap * 4);
   w.part = al256(w.idx + rows * (size_t)keff * 4);
-  w.total = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4) + 256;
+  w.qterm = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4);
+  w.total = al256(w.qterm + rows * (size_t)kQTermBytes) + 256;
   return w;
 }
 size_t decode_ws(const fasa_cache* c, int32_t len, int32_t k) { return decode_layout(c, len, k).total; }
@@ -704,14 +722,25 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   const int rows = c->batch * c->n_kv_heads;
   const int keff = std::min(k, len);
   const int path = g_decode_path.load();
-  if (path != FASA_DECODE_STAGED) {
+  char* base = static_cast<char*>(workspace);
+  if (path == FASA_DECODE_AUTO || path == FASA_DECODE_FUSED) {
     FusedPlan pl;
     bool ok = false;
-    if ((s = fused_plan(c, len, keff, d, path == FASA_DECODE_FUSED, &pl, &ok)) != FASA_OK) return s;
-    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, pl, stream, d);
+    if ((s = fused_plan(c, len, d, path == FASA_DECODE_FUSED, false, &pl, &ok)) != FASA_OK) return s;
+    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, nullptr, pl, stream, d);
     if (path == FASA_DECODE_FUSED) return FASA_ERR_UNSUPPORTED;
   }
-  char* base = static_cast<char*>(workspace);
+  if (path == FASA_DECODE_AUTO || path == FASA_DECODE_SCORED) {
+    FusedPlan pl;
+    bool ok = false;
+    if ((s = fused_plan(c, len, d, path == FASA_DECODE_SCORED, true, &pl, &ok)) != FASA_OK) return s;
+    if (ok) {
+      float* sc = reinterpret_cast<float*>(base + w.scores);
+      if ((s = launch_score(c, len, q, q_pos, sc, nullptr, stream)) != FASA_OK) return s;
+      return launch_fused(c, len, q, q_pos, keff, out, idx_out, sc, pl, stream, d);
+    }
+    if (path == FASA_DECODE_SCORED) return FASA_ERR_UNSUPPORTED;
+  }
   float* scores = reinterpret_cast<float*>(base + w.scores);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + w.hist);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(base + w.cnt);
@@ -756,6 +785,10 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   np.cap = w.cap;
   np.words = w.words;
   np.scap = w.cap;
+  np.q = static_cast<const __nv_bfloat16*>(q);
+  np.qterms = reinterpret_cast<unsigned char*>(base + w.qterm);
+  np.group = c->n_q_heads / c->n_kv_heads;
+  fill_query_angle(np.cosv, np.sinv, c->rope_base, q_pos);
   while (np.scap > 256 && final_smem_bytes(np.words, np.scap) > d.smem_optin) np.scap /= 2;
   const int fsmem = final_smem_bytes(np.words, np.scap);
   if (fsmem > d.smem_optin) return FASA_ERR_UNSUPPORTED;
@@ -776,7 +809,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     ap.k = static_cast<const __nv_bfloat16*>(c->k);
     ap.v = static_cast<const __nv_bfloat16*>(c->v);
     ap.idx = idx;
-    ap.q = static_cast<const __nv_bfloat16*>(q);
+    ap.qterms = reinterpret_cast<const unsigned char*>(base + w.qterm);
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.part = part;
     ap.counter = att_cnt;
@@ -787,7 +820,6 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
     ap.splits = (int)ceil_div(keff, ap.slice);
     ap.group = c->n_q_heads / c->n_kv_heads;
-    fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
     if ((s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
            *v = 1;
            return cuda_status(
@@ -812,7 +844,8 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
 }
 
 fasa_status fasa_set_decode_path(int32_t path) {
-  if (path != FASA_DECODE_AUTO && path != FASA_DECODE_FUSED && path != FASA_DECODE_STAGED)
+  if (path != FASA_DECODE_AUTO && path != FASA_DECODE_FUSED && path != FASA_DECODE_STAGED &&
+      path != FASA_DECODE_SCORED)
     return FASA_ERR_INVALID_ARG;
   g_decode_path.store(path);
   return FASA_OK;
@@ -828,8 +861,10 @@ int32_t fasa_decode_path(const fasa_cache* c, int32_t len, int32_t k) {
   if (path != FASA_DECODE_AUTO) return path;
   FusedPlan pl;
   bool ok = false;
-  if ((s = fused_plan(c, len, std::min(k, len), d, false, &pl, &ok)) != FASA_OK) return -s;
-  return ok ? FASA_DECODE_FUSED : FASA_DECODE_STAGED;
+  if ((s = fused_plan(c, len, d, false, false, &pl, &ok)) != FASA_OK) return -s;
+  if (ok) return FASA_DECODE_FUSED;
+  if ((s = fused_plan(c, len, d, false, true, &pl, &ok)) != FASA_OK) return -s;
+  return ok ? FASA_DECODE_SCORED : FASA_DECODE_STAGED;
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,

@@ -279,14 +279,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     score_block<T, LPT, NCW>(ring + (size_t)b * kScoreStageBytes, n, qr, warp, lane,
                              [&](int t, bool writer, float sc) {
                                if (writer) out[t0 + t] = sc;
-                               if (kHist) {
-                                 const uint32_t bin = score_key(sc) >> (32 - kHistBits);
-                                 const unsigned act = __ballot_sync(0xFFFFFFFFu, writer);
-                                 if (writer) {
-                                   const unsigned peers = __match_any_sync(act, bin);
-                                   if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (uint32_t)__popc(peers));
-                                 }
-                               }
+                               if (kHist && writer) atomicAdd(&s_hist[score_key(sc) >> (32 - kHistBits)], 1u);
                              });
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[b]);

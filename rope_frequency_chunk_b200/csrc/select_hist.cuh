@@ -21,6 +21,7 @@
 //           its scores instead (slow, rare).
 #pragma once
 
+#include "attend_mma.cuh"
 #include "select_attend.cuh"
 
 namespace fasa {
@@ -94,10 +95,17 @@ struct FinalParams {
   int32_t cap;              // candidate list capacity
   int32_t scap;             // candidates held in shared memory
   int32_t words;
+  // the attention kernel's query terms, prepared here once per row
+  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
+  unsigned char* qterms;    // [rows][kQTermBytes]
+  int32_t group;
+  double cosv[kNFC];        // cos / sin of q_pos * theta_i (host, float64)
+  double sinv[kNFC];
 };
 
 __host__ __device__ inline int final_smem_bytes(int words, int scap) {
-  return sa_align(words * 4, 128) + (kSAWarps * 256 + 264) * 4 + 64 * 4 + 2 * scap * 4;
+  return sa_align(words * 4, 128) + (kSAWarps * 256 + 264) * 4 + 64 * 4 + sa_align(2 * scap * 4, 16) +
+         FASA_MAX_GROUP * kD * 2;
 }
 
 __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalParams p) {
@@ -112,6 +120,17 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
   uint32_t* scan = rscr + kSAWarps * 256 + 264;
   uint32_t* ckey = scan + 64;                           // [scap]
   int32_t* cidx = reinterpret_cast<int32_t*>(ckey + p.scap);  // [scap]
+  // [G][128], 16-byte aligned for the vector stores below (scap may be odd)
+  __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(
+      reinterpret_cast<unsigned char*>(ckey) + sa_align(2 * p.scap * 4, 16));
+
+  // the group's rotated query terms for the attention kernel
+  {
+    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)row * p.group) * kD);
+    for (int c = tid; c < p.group * kD / 8; c += kSAThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    __syncthreads();
+    query_terms(qraw, p.group, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes, tid, kSAThreads);
+  }
 
   uint32_t bin, above;
   hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);

@@ -225,7 +225,7 @@ def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, id
     return out
 
 
-DECODE_AUTO, DECODE_FUSED, DECODE_STAGED = 0, 1, 2
+DECODE_AUTO, DECODE_FUSED, DECODE_STAGED, DECODE_SCORED = 0, 1, 2, 3
 
 
 def fasa_set_decode_path(path: int) -> None:
@@ -234,7 +234,7 @@ def fasa_set_decode_path(path: int) -> None:
 
 
 def fasa_decode_path(cache: KVCache, length: int, k: int) -> int:
-    """The plan fasa_decode would run for this shape (DECODE_FUSED or DECODE_STAGED)."""
+    """The plan fasa_decode would run for this shape (DECODE_FUSED, DECODE_SCORED or DECODE_STAGED)."""
     r = int(lib().fasa_decode_path(cache.ref(), length, k))
     if r < 0:
         _check(-r, "fasa_decode_path")

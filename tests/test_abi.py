@@ -104,7 +104,7 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 
 
 def test_decode_path_setting_is_validated_on_the_host(L):
-    assert L.fasa_set_decode_path(3) == 1 and L.fasa_set_decode_path(-1) == 1
-    for p in (1, 2, 0):
+    assert L.fasa_set_decode_path(4) == 1 and L.fasa_set_decode_path(-1) == 1
+    for p in (1, 2, 3, 0):
         assert L.fasa_set_decode_path(p) == 0
     assert L.fasa_decode_path(None, 10, 10) < 0

@@ -135,7 +135,7 @@ def test_dense_matches_oracle(name):
         U.check_out(wl, out[b, g * G:(g + 1) * G], ref)
 
 
-PATHS = {"fused": F.DECODE_FUSED, "staged": F.DECODE_STAGED}
+PATHS = {"fused": F.DECODE_FUSED, "scored": F.DECODE_SCORED, "staged": F.DECODE_STAGED}
 
 
 @pytest.fixture(params=list(PATHS))
@@ -147,8 +147,8 @@ def path(request):
 
 
 def _skip_unless_plan(wl, path):
-    if path == "fused" and wl.dtype != "bf16":
-        pytest.skip("the single-launch decode takes bf16 caches only")
+    if path in ("fused", "scored") and wl.dtype != "bf16":
+        pytest.skip("the cluster decode takes bf16 caches only")
 
 
 def _decode(wl, cache, q, k, length=None):
@@ -268,11 +268,13 @@ def _both_paths(wl, cache, q, k):
 
 
 def _check_paths_agree(wl, res):
-    """Both plans score bit-identically and select exactly: same kept sets;
-    outputs differ only by float32 summation order."""
-    (o_f, i_f), (o_s, i_s) = res["fused"], res["staged"]
-    assert torch.equal(i_f, i_s)
-    U.check_gpu_pair(wl, U.stored(o_f), U.stored(o_s))
+    """Every plan scores bit-identically and selects exactly: the same kept
+    sets; outputs differ only by float32 summation order."""
+    o_s, i_s = res["staged"]
+    for name in ("fused", "scored"):
+        o_x, i_x = res[name]
+        assert torch.equal(i_x, i_s), name
+        U.check_gpu_pair(wl, U.stored(o_x), U.stored(o_s))
 
 
 def test_decode_path_setting_and_choice():
@@ -288,10 +290,11 @@ def test_decode_path_setting_and_choice():
         F.fasa_set_decode_path(7)
 
 
-def test_fused_decode_rejects_f32_when_forced():
+@pytest.mark.parametrize("plan", [F.DECODE_FUSED, F.DECODE_SCORED])
+def test_cluster_decode_rejects_f32_when_forced(plan):
     wl = SMALL["c1"]
     _, cache, q = U.build(wl)
-    F.fasa_set_decode_path(F.DECODE_FUSED)
+    F.fasa_set_decode_path(plan)
     try:
         with pytest.raises(F.FasaError) as e:
             _decode(wl, cache, q, wl.k)
@@ -333,6 +336,7 @@ def test_full_c3_sampled():
     inp, cache, q = U.build(wl)
     heads = U.sample_heads(wl, 3)
     U.check_append(wl, inp, cache, heads[:1])
+    assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_STAGED
     out, idx = _decode(wl, cache, q, wl.k)
     U.check_decode_heads(wl, inp, cache, q, wl.k, heads, out, idx)
     _check_paths_agree(wl, _both_paths(wl, cache, q, wl.k))
