@@ -133,7 +133,7 @@ fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
 template <typename T, int LPT, bool kHist>
 fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t st) {
   auto kern = score_kernel<T, LPT, kHist>;
-  const int smem = kScoreStages * kScoreStageBytes + kHistBins * 4;
+  const int smem = score_smem_bytes();
   int set = 0;
   fasa_status s = cached_int((const void*)kern, 0, &set, [&](int* v) {
     *v = 1;

@@ -9,12 +9,12 @@
 //
 // Data path: the sketch holds 2*n_dom values per token, stride padded to a
 // power-of-two number of 16-byte chunks. The grid is persistent (one CTA per
-// SM) and splits the flattened (row, token) range evenly. A producer warp
-// streams the CTA's contiguous range through a ring of shared-memory stages
-// with 1-D bulk copies (TMA engine, full/empty mbarriers, no multicast); 12
-// consumer warps score the tokens, one token per lane (two or four lanes for
-// rows wider than 32 elements). The first stages are in flight before the
-// query coefficients are computed.
+// SM) and splits the flattened (row, token) range evenly; a CTA takes its
+// range row segment by row segment. Each warp streams its own 32-lane steps
+// of consecutive tokens through a private ring of shared-memory slots with
+// 16-byte cp.async copies (no block barrier inside a segment, many requests
+// in flight per SM) and scores them, one token per lane (two or four lanes
+// for rows wider than 32 elements).
 //
 // Arithmetic: float64. Each stored element e is widened exactly to the double
 // e * 2^-896 by placing its sign, exponent and mantissa bits in the double's
@@ -28,10 +28,9 @@
 
 namespace fasa {
 
-constexpr int kScoreConsumerWarps = 12;
-constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kScoreStages = 8;
-constexpr int kScoreStageBytes = 24576;
+constexpr int kScoreWarps = 12;
+constexpr int kScoreThreads = kScoreWarps * 32;
+constexpr int kScoreWarpBytes = 12288;  // each warp's ring of copy slots
 
 struct ScoreParams {
   const void* sketch;    // [rows][max_len][stride]
@@ -176,118 +175,101 @@ __device__ __forceinline__ void score_block(const unsigned char* buf, int n, con
   }
 }
 
+// Slots of a warp's ring: one warp step (32 lanes x their chunks) each.
+template <typename T, int LPT>
+struct ScoreRing {
+  static constexpr int kSlot = 32 * ScoreShape<T, LPT>::CPL * 16;
+  static constexpr int kRaw = kScoreWarpBytes / kSlot;
+  static constexpr int kDepth = kRaw < 2 ? 2 : (kRaw > 16 ? 16 : kRaw);
+  static_assert(kDepth * kSlot <= kScoreWarpBytes, "ring slots exceed the warp's ring");
+};
+
+__host__ __device__ constexpr int score_smem_bytes() { return kScoreWarps * kScoreWarpBytes + kHistBins * 4; }
+
 template <typename T, int LPT, bool kHist>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScoreParams p) {
   using S = ScoreShape<T, LPT>;
-  constexpr int TPS = kScoreStageBytes / S::ROWB;  // tokens per stage
-  constexpr int NCW = kScoreConsumerWarps;
-  extern __shared__ __align__(128) unsigned char ring[];  // stages, then the histogram
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + (size_t)kScoreStages * kScoreStageBytes);
+  using R = ScoreRing<T, LPT>;
+  constexpr int D = R::kDepth;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + kScoreWarps * kScoreWarpBytes);
   __shared__ double s_q[kD];
   __shared__ __align__(16) T s_qraw[FASA_MAX_GROUP * kD];  // the group's raw queries
   __shared__ int s_dom[kNFC];
-  __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
-  __shared__ int st_row[kScoreStages], st_t0[kScoreStages], st_n[kScoreStages];
   grid_dependency_wait();
   grid_dependents_launch();  // the selection kernel may be scheduled now; it waits for our results
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned char* ring = smem + warp * kScoreWarpBytes;
+  const int sub = lane % S::LPT2, tl = lane / S::LPT2;  // the lane's chunk group and token in a step
   const int64_t per = (p.total + gridDim.x - 1) / gridDim.x;
   const int64_t f_beg = min(p.total, (int64_t)blockIdx.x * per);
   const int64_t f_end = min(p.total, f_beg + per);
-  const int64_t n_tok = f_end - f_beg;
-
-  if (tid == 0) {
-    for (int b = 0; b < kScoreStages; ++b) {
-      mbar_init(&full[b], 1);
-      mbar_init(&empty[b], NCW);
-    }
-    fence_mbar_init();
-  }
   if (kHist)
     for (int i = tid; i < kHistBins; i += kScoreThreads) s_hist[i] = 0u;
-  __syncthreads();
 
-  if (warp == NCW) {
-    // ---------------- producer: one lane walks the range, stage by stage
-    if (lane == 0 && n_tok > 0) {
-      int row = (int)(f_beg / p.len), t = (int)(f_beg % p.len);
-      int64_t left = n_tok;
-      for (int j = 0; left > 0; ++j) {
-        const int b = j % kScoreStages;
-        if (j >= kScoreStages && !mbar_wait(&empty[b], (uint32_t)(((j / kScoreStages) - 1) & 1))) break;
-        const int n = (int)min((int64_t)min(TPS, p.len - t), left);
-        st_row[b] = row;
-        st_t0[b] = t;
-        st_n[b] = n;
-        mbar_arrive_expect_tx(&full[b], (uint32_t)(n * S::ROWB));
-        bulk_g2s(ring + (size_t)b * kScoreStageBytes,
-                 static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t) * S::ROWB,
-                 (uint32_t)(n * S::ROWB), &full[b]);
-        left -= n;
-        t += n;
-        if (t == p.len) {
-          t = 0;
-          ++row;
+  for (int64_t seg = f_beg; seg < f_end;) {
+    const int row = (int)(seg / p.len), t0 = (int)(seg % p.len);
+    const int n = (int)min((int64_t)(p.len - t0), f_end - seg);
+    // the row's query coefficients (float64), every thread taking part
+    __syncthreads();
+    {
+      const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
+                                                         ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD);
+      for (int c = tid; c < p.group * kD * (int)sizeof(T) / 16; c += kScoreThreads)
+        reinterpret_cast<uint4*>(s_qraw)[c] = __ldg(qsrc + c);
+      if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
+    }
+    __syncthreads();
+    query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
+    __syncthreads();
+    double qr[S::EPL];
+    load_coefs<T, LPT>(qr, s_q, lane);
+
+    // warp w takes the steps w, w + kScoreWarps, ... of TPW consecutive tokens
+    const char* src = static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
+    float* out = p.scores + (int64_t)row * p.len + t0;
+    const int nblk = (n + S::TPW - 1) / S::TPW;
+    const int mine = nblk > warp ? (nblk - warp + kScoreWarps - 1) / kScoreWarps : 0;
+    auto issue = [&](int j) {
+      if (j < mine) {
+        const int tok = (j * kScoreWarps + warp) * S::TPW + tl;
+        if (tok < n) {
+          unsigned char* slot = ring + (j % D) * R::kSlot + tl * S::ROWB;
+#pragma unroll
+          for (int c = 0; c < S::CPL; ++c)
+            cp_async16(slot + (sub * S::CPL + c) * 16, src + (int64_t)tok * S::ROWB + (sub * S::CPL + c) * 16);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int j = 0; j < D; ++j) issue(j);
+    for (int j = 0; j < mine; ++j) {
+      cp_async_wait<D - 1>();
+      __syncwarp();
+      const int b0 = (j * kScoreWarps + warp) * S::TPW;
+      score_block<T, LPT, 1>(ring + (j % D) * R::kSlot, min(S::TPW, n - b0), qr, 0, lane,
+                             [&](int t, bool writer, float sc) {
+                               if (writer) out[b0 + t] = sc;
+                               if (kHist && writer) atomicAdd(&s_hist[score_key(sc) >> (32 - kHistBits)], 1u);
+                             });
+      __syncwarp();
+      issue(j + D);
+    }
+    cp_async_wait<0>();
+    if (kHist) {
+      __syncthreads();
+      for (int i = tid; i < kHistBins; i += kScoreThreads) {
+        const uint32_t v = s_hist[i];
+        if (v) {
+          atomicAdd(p.hist + (int64_t)row * kHistBins + i, v);
+          s_hist[i] = 0u;
         }
       }
     }
-    return;
-  }
-
-  // ---------------- consumers: one token per lane (LPT2 lanes for wide rows)
-  double qr[S::EPL];
-  int cur_row = -1;
-  float* out = p.scores;
-
-  auto flush_hist = [&](int row) {
-    // all consumer warps are between the two named barriers around this call
-    for (int i = tid; i < kHistBins; i += NCW * 32) {
-      const uint32_t v = s_hist[i];
-      if (v) {
-        atomicAdd(p.hist + (int64_t)row * kHistBins + i, v);
-        s_hist[i] = 0u;
-      }
-    }
-  };
-
-  int64_t done = 0;
-  for (int j = 0; done < n_tok; ++j) {
-    const int b = j % kScoreStages;
-    if (!mbar_wait(&full[b], (uint32_t)((j / kScoreStages) & 1))) break;  // status already recorded
-    const int row = st_row[b], t0 = st_t0[b], n = st_n[b];
-    if (row != cur_row) {
-      // new row: the group's rotated queries summed per sketch column (float64)
-      named_barrier_sync(1, NCW * 32);
-      if (kHist && cur_row >= 0) flush_hist(cur_row);
-      {
-        // the group's queries and the head's dominant FCs, loaded in parallel
-        const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
-        const uint4* qsrc = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
-                                                           ((int64_t)(bb * p.n_kv_heads + g) * p.group) * kD);
-        for (int c = tid; c < p.group * kD * (int)sizeof(T) / 16; c += NCW * 32)
-          reinterpret_cast<uint4*>(s_qraw)[c] = __ldg(qsrc + c);
-        if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
-      }
-      named_barrier_sync(1, NCW * 32);
-      query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
-      named_barrier_sync(1, NCW * 32);
-      load_coefs<T, LPT>(qr, s_q, lane);
-      cur_row = row;
-      out = p.scores + (int64_t)row * p.len;
-    }
-    score_block<T, LPT, NCW>(ring + (size_t)b * kScoreStageBytes, n, qr, warp, lane,
-                             [&](int t, bool writer, float sc) {
-                               if (writer) out[t0 + t] = sc;
-                               if (kHist && writer) atomicAdd(&s_hist[score_key(sc) >> (32 - kHistBits)], 1u);
-                             });
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[b]);
-    done += n;
-  }
-  if (kHist && cur_row >= 0) {
-    named_barrier_sync(1, NCW * 32);
-    flush_hist(cur_row);
+    seg += n;
   }
 }
 
