@@ -32,7 +32,7 @@ namespace fasa {
 constexpr int kAttWarps = 4;
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttChunk = 16;                          // rows per warp step
-constexpr int kAttStages = 3;                          // per-warp ring depth
+constexpr int kAttStages = 2;                          // per-warp ring depth
 constexpr int kAttHalf = kAttChunk * kD * 2;           // bytes of 16 bf16 rows (K or V)
 constexpr int kAttStageBytes = 2 * kAttHalf;           // K + V
 constexpr int kAttPartStride = 16 * kD + 32;           // floats: m[16], l[16], o[16][128]
@@ -55,8 +55,15 @@ struct AttParams {
   int32_t group;
 };
 
-__host__ __device__ constexpr int att_smem_bytes() { return kAttWarps * kAttStages * kAttStageBytes + kQTermBytes; }
+// The ring, then the G query rows of each term (256 B each) and one zero row
+// that stands in for the padding heads G..15.
+__host__ __device__ constexpr int att_smem_bytes(int G) { return kAttWarps * kAttStages * kAttStageBytes + (3 * G + 1) * 256; }
 static_assert(kAttSlot * 4 * (kAttWarps / 2) <= kAttWarps * kAttStages * kAttStageBytes, "merge slots exceed the ring");
+// The last CTA of a row merges the splits in the ring's space: (m, l, weight)
+// of 16 heads per split, then 16 denominators.
+__host__ __device__ constexpr int att_merge_bytes(int splits) { return splits * 3 * 16 * 4 + 16 * 4; }
+constexpr int kAttMaxSplits = (kAttWarps * kAttStages * kAttStageBytes - 16 * 4) / (3 * 16 * 4);
+static_assert(att_merge_bytes(kAttMaxSplits) <= kAttWarps * kAttStages * kAttStageBytes, "split merge exceeds the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -121,8 +128,10 @@ __device__ __forceinline__ void query_terms(const __nv_bfloat16* qraw, int G, co
 
 // S = Q K^T for one 16-row chunk staged at Ks: s0 rows 0-7, s1 rows 8-15 of
 // the chunk (fragment layout of m16n8k16), each Q term in its own chain.
-__device__ __forceinline__ void chunk_logits(const unsigned char* qt, const unsigned char* Ks, int lane, float (&s0)[4],
-                                             float (&s1)[4]) {
+// Query row r of term t is at qt + (t * G + r) * 256 for r < G, the zero
+// row (qt + 3 * G * 256) otherwise.
+__device__ __forceinline__ void chunk_logits(const unsigned char* qt, int G, const unsigned char* Ks, int lane,
+                                             float (&s0)[4], float (&s1)[4]) {
   float a0[3][4], a1[3][4];
 #pragma unroll
   for (int t = 0; t < 3; ++t)
@@ -133,11 +142,11 @@ __device__ __forceinline__ void chunk_logits(const unsigned char* qt, const unsi
   for (int ks = 0; ks < 8; ++ks) {
     uint32_t b[4];
     ldsm_x4(b, Ks + ((lane / 16) * 8 + lane % 8) * 256 + (((ks * 2 + (lane / 8) % 2) ^ (lane % 8)) * 16));
-    const int aoff = arow * 256 + (((ks * 2 + lane / 16) ^ (arow & 7)) * 16);
+    const int aoff = (((ks * 2 + lane / 16) ^ (arow & 7)) * 16);
 #pragma unroll
     for (int t = 0; t < 3; ++t) {  // low, middle, high bf16 term of Q
       uint32_t a[4];
-      ldsm_x4(a, qt + t * 4096 + aoff);
+      ldsm_x4(a, qt + (arow < G ? (t * G + arow) : 3 * G) * 256 + aoff);
       mma_16816(a0[t], a, b[0], b[1]);
       mma_16816(a1[t], a, b[2], b[3]);
     }
@@ -157,8 +166,14 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
   const int G = p.group;
   unsigned char* qt = smem + kAttWarps * kAttStages * kAttStageBytes;
   {
+    // the G real rows of each term (rows of the staged terms keep their
+    // swizzle, which depends on the row index only), then a zero row
     const unsigned char* src = p.qterms + (int64_t)row * kQTermBytes;
-    for (int c = tid; c < kQTermBytes / 16; c += kAttThreads) cp_async16(qt + c * 16, src + c * 16);
+    for (int c = tid; c < 3 * G * 16; c += kAttThreads) {
+      const int t = c / (G * 16), r = (c / 16) % G, part = c % 16;
+      cp_async16(qt + (t * G + r) * 256 + part * 16, src + t * 4096 + r * 256 + part * 16);
+    }
+    if (tid < 16) reinterpret_cast<uint4*>(qt + 3 * G * 256)[tid] = make_uint4(0u, 0u, 0u, 0u);
     cp_async_commit();
   }
 
@@ -214,7 +229,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
     const unsigned char* Ks = ring + (ci % kAttStages) * kAttStageBytes;
     const unsigned char* Vs = Ks + kAttHalf;
     float s0[4], s1[4];  // rows 0-7, 8-15 of the chunk
-    chunk_logits(qt, Ks, lane, s0, s1);
+    chunk_logits(qt, G, Ks, lane, s0, s1);
     // mask the chunk's missing or invalid rows (columns of S)
     const int j0 = r_beg + (warp + ci * kAttWarps) * kAttChunk;
     const int c0 = (lane % 4) * 2;

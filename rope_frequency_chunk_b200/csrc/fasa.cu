@@ -525,14 +525,19 @@ fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_
 //   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
 // hist, cand_cnt and att_cnt are cleared at the start of every call.
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
+constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 struct DecodeWs {
   size_t scores, hist, cnt, att_cnt, bitmap, cand, idx, part, qterm, total;
   int cap, words, splits_max;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 inline int att_chunks(int keff) { return (keff + kAttChunk - 1) / kAttChunk; }
-inline int att_splits(int rows, int keff, int sms) {
-  return (int)std::max<int64_t>(1, std::min<int64_t>(att_chunks(keff), ceil_div(2LL * sms, rows)));
+// Splits per row so that the attention grid fills, without exceeding, one
+// wave of resident CTAs; at most kAttMaxSplits, whose merge state fits in
+// the kernel's shared memory.
+inline int att_splits(int rows, int keff, int sms, int per_sm) {
+  const int64_t s = std::min<int64_t>(att_chunks(keff), (int64_t)per_sm * sms / rows);
+  return (int)std::max<int64_t>(1, std::min<int64_t>(s, kAttMaxSplits));
 }
 DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   DecodeWs w;
@@ -541,7 +546,7 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   const int keff = std::max(0, std::min(k, len));
   w.words = (int)((L + 31) / 32);
   w.cap = (int)std::min<size_t>(std::max<size_t>(L, 1), 8192);
-  w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms);
+  w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms, kAttMaxPerSm);
   w.scores = 0;
   w.hist = al256(rows * L * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
@@ -764,7 +769,8 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   fp.len = len;
   fp.n_keep = keff;
   fp.cap = w.cap;
-  const int64_t tiles_per_row = std::max<int64_t>(1, ceil_div(4LL * d.sms, rows));
+  // one wave of four resident filter CTAs per SM
+  const int64_t tiles_per_row = std::max<int64_t>(1, 4LL * d.sms / rows);
   fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 32) * 32);
   fp.words = w.words;
   if ((s = launch_pdl(filter_kernel, dim3((unsigned)ceil_div(len, fp.tile), (unsigned)rows, 1), kFilterThreads, 0,
@@ -816,18 +822,26 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     ap.max_len = c->max_len;
     ap.len = len;
     ap.n_keep = keff;
-    ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms));
-    ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
-    ap.splits = (int)ceil_div(keff, ap.slice);
     ap.group = c->n_q_heads / c->n_kv_heads;
     if ((s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
            *v = 1;
-           return cuda_status(
-               cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, att_smem_bytes()));
+           return cuda_status(cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   att_smem_bytes(FASA_MAX_GROUP)));
          })) != FASA_OK)
       return s;
+    int per_sm = 0;  // resident attention CTAs per SM at this group size
+    if ((s = cached_int((const void*)attend_mma_kernel, 1 + (uint64_t)ap.group, &per_sm, [&](int* v) {
+           return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, attend_mma_kernel, kAttThreads,
+                                                                             (size_t)att_smem_bytes(ap.group)));
+         })) != FASA_OK)
+      return s;
+    per_sm = std::max(1, std::min(per_sm, kAttMaxPerSm));
+    ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms, per_sm));
+    ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
+    ap.splits = (int)ceil_div(keff, ap.slice);
+    if (ap.splits > kAttMaxSplits) return FASA_ERR_UNSUPPORTED;  // cannot happen: splits only shrank
     return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
-                      (size_t)att_smem_bytes(), stream, ap);
+                      (size_t)att_smem_bytes(ap.group), stream, ap);
   }
   SAParams p{};
   p.idx_in = idx;
