@@ -521,13 +521,13 @@ fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_
 // Decode workspace, each part 256-byte aligned:
 //   scores [rows][len] f32 | hist [rows][4096] u32 | cand_cnt [rows] u32 |
 //   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
-//   cand_idx [rows][cap] i32 | idx [rows][k_eff] i32 |
+//   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
 // hist, cand_cnt and att_cnt are cleared at the start of every call.
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 struct DecodeWs {
-  size_t scores, hist, cnt, att_cnt, bitmap, cand, idx, part, qterm, total;
+  size_t scores, hist, cnt, att_cnt, bitmap, cand, ckey, idx, part, qterm, total;
   int cap, words, splits_max;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -553,7 +553,8 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.att_cnt = w.cnt + rows * 4;
   w.bitmap = al256(w.att_cnt + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
-  w.idx = al256(w.cand + rows * (size_t)w.cap * 4);
+  w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
+  w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
   w.part = al256(w.idx + rows * (size_t)keff * 4);
   w.qterm = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4);
   w.total = al256(w.qterm + rows * (size_t)kQTermBytes) + 256;
@@ -751,6 +752,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   uint32_t* cnt = reinterpret_cast<uint32_t*>(base + w.cnt);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
   int32_t* cand = reinterpret_cast<int32_t*>(base + w.cand);
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(base + w.ckey);
   int32_t* idx = reinterpret_cast<int32_t*>(base + w.idx);
 
   // 1. TIP scores and the per-row key histogram
@@ -765,6 +767,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   fp.hist = hist;
   fp.cand_cnt = cnt;
   fp.cand_idx = cand;
+  fp.cand_key = ckey;
   fp.bitmap = bitmap;
   fp.len = len;
   fp.n_keep = keff;
@@ -773,6 +776,10 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   const int64_t tiles_per_row = std::max<int64_t>(1, 4LL * d.sms / rows);
   fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 32) * 32);
   fp.words = w.words;
+  fp.q = static_cast<const __nv_bfloat16*>(q);
+  fp.qterms = c->dtype == FASA_BF16 ? reinterpret_cast<unsigned char*>(base + w.qterm) : nullptr;
+  fp.group = c->n_q_heads / c->n_kv_heads;
+  fill_query_angle(fp.cosv, fp.sinv, c->rope_base, q_pos);
   if ((s = launch_pdl(filter_kernel, dim3((unsigned)ceil_div(len, fp.tile), (unsigned)rows, 1), kFilterThreads, 0,
                       stream, fp)) != FASA_OK)
     return s;
@@ -783,6 +790,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   np.hist = hist;
   np.cand_cnt = cnt;
   np.cand_idx = cand;
+  np.cand_key = ckey;
   np.bitmap = bitmap;
   np.idx = idx;
   np.idx_out = idx_out;
@@ -791,10 +799,6 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   np.cap = w.cap;
   np.words = w.words;
   np.scap = w.cap;
-  np.q = static_cast<const __nv_bfloat16*>(q);
-  np.qterms = reinterpret_cast<unsigned char*>(base + w.qterm);
-  np.group = c->n_q_heads / c->n_kv_heads;
-  fill_query_angle(np.cosv, np.sinv, c->rope_base, q_pos);
   while (np.scap > 256 && final_smem_bytes(np.words, np.scap) > d.smem_optin) np.scap /= 2;
   const int fsmem = final_smem_bytes(np.words, np.scap);
   if (fsmem > d.smem_optin) return FASA_ERR_UNSUPPORTED;

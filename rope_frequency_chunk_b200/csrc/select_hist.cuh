@@ -11,7 +11,11 @@
 //           higher bins are certainly kept: each warp writes the bitmap word
 //           of its 32 consecutive tokens (every word of [0, len) is written
 //           exactly once, so the bitmap needs no clearing). Keys in bin b1
-//           are appended to the row's candidate list.
+//           are gathered in shared memory and appended, (index, key) pairs,
+//           to the row's candidate list with one global atomic per CTA (a
+//           per-warp atomic on the row's counter serialises thousands of
+//           warps on one cache line). Tile 0 of each row also prepares the
+//           attention kernel's query terms, before waiting for the scores.
 //  finalize (grid: rows) Exact k_eff-th key among the candidates (radix
 //           select on the low 20 bits, digit histograms counted with warp
 //           ballots); ties at it go to the lower token index. Their bits
@@ -28,27 +32,46 @@ namespace fasa {
 
 constexpr int kFilterThreads = kSAThreads;  // hist_threshold assumes 512 threads
 
+constexpr int kFilterCands = 2048;  // candidates a CTA gathers in shared memory
+
 struct FilterParams {
   const float* scores;      // [rows][len]
   const uint32_t* hist;     // [rows][4096]
   uint32_t* cand_cnt;       // [rows], zero before the launch
   int32_t* cand_idx;        // [rows][cap]
+  uint32_t* cand_key;       // [rows][cap], the candidates' score keys
   uint32_t* bitmap;         // [rows][words]
   int32_t len;
   int32_t n_keep;           // k_eff
   int32_t cap;
   int32_t tile;             // tokens per CTA, a multiple of 32
   int32_t words;            // ceil(len / 32)
+  // the attention kernel's query terms, prepared by tile 0 of each row
+  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
+  unsigned char* qterms;    // [rows][kQTermBytes], or null (no attention follows)
+  int32_t group;
+  double cosv[kNFC];        // cos / sin of q_pos * theta_i (host, float64)
+  double sinv[kNFC];
 };
 
-__global__ void __launch_bounds__(kFilterThreads) filter_kernel(const FilterParams p) {
+__global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterParams p) {
   __shared__ uint32_t scan[64];
-  grid_dependency_wait();
+  __shared__ int32_t s_cidx[kFilterCands];
+  __shared__ uint32_t s_ckey[kFilterCands];
+  __shared__ uint32_t s_n, s_base;
   const int row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  // The query is an input of the whole decode, complete before the score
+  // kernel started, so tile 0 can turn it into query terms before waiting;
+  // the attention kernel reads them two launches later.
+  if (blockIdx.x == 0 && p.qterms)
+    query_terms(p.q + (int64_t)row * p.group * kD, p.group, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes,
+                tid, kFilterThreads);
+  if (tid == 0) s_n = 0u;
+  grid_dependency_wait();
   uint32_t bin, above;
-  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);
+  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);  // its barriers publish s_n
   const int t0 = blockIdx.x * p.tile;
   const int t1 = min(p.len, t0 + p.tile);
   const float* s = p.scores + (int64_t)row * p.len;
@@ -68,16 +91,40 @@ __global__ void __launch_bounds__(kFilterThreads) filter_kernel(const FilterPara
       if (base >= t1) break;  // warp-uniform
       const int i = base + lane;
       const bool v = i < t1;
-      const uint32_t b = score_key(f[u]) >> 20;
+      const uint32_t key = score_key(f[u]);
+      const uint32_t b = key >> 20;
       const unsigned def = __ballot_sync(0xFFFFFFFFu, v && b > bin);
       const unsigned cnd = __ballot_sync(0xFFFFFFFFu, v && b == bin);
       if (lane == 0) bm[base >> 5] = def;
       if (cnd) {
         uint32_t at = 0u;
-        if (lane == 0) at = atomicAdd(p.cand_cnt + row, (uint32_t)__popc(cnd));
+        if (lane == 0) at = atomicAdd(&s_n, (uint32_t)__popc(cnd));
         at = __shfl_sync(0xFFFFFFFFu, at, 0) + __popc(cnd & lt);
-        if (((cnd >> lane) & 1u) && at < (uint32_t)p.cap) cidx[at] = i;
+        if ((cnd >> lane) & 1u) {
+          if (at < (uint32_t)kFilterCands) {
+            s_cidx[at] = i;
+            s_ckey[at] = key;
+          } else {  // this CTA's buffer is full (heavy ties): straight to the global list
+            const uint32_t g = atomicAdd(p.cand_cnt + row, 1u);
+            if (g < (uint32_t)p.cap) {
+              cidx[g] = i;
+              p.cand_key[(int64_t)row * p.cap + g] = key;
+            }
+          }
+        }
       }
+    }
+  }
+  __syncthreads();
+  const uint32_t n = min(s_n, (uint32_t)kFilterCands);
+  if (tid == 0) s_base = n ? atomicAdd(p.cand_cnt + row, n) : 0u;
+  __syncthreads();
+  uint32_t* ckey = p.cand_key + (int64_t)row * p.cap;
+  for (uint32_t j = tid; j < n; j += kFilterThreads) {
+    const uint32_t g = s_base + j;
+    if (g < (uint32_t)p.cap) {
+      cidx[g] = s_cidx[j];
+      ckey[g] = s_ckey[j];
     }
   }
 }
@@ -87,6 +134,7 @@ struct FinalParams {
   const uint32_t* hist;
   const uint32_t* cand_cnt;
   const int32_t* cand_idx;  // [rows][cap]
+  const uint32_t* cand_key; // [rows][cap]
   const uint32_t* bitmap;   // [rows][words]
   int32_t* idx;             // [rows][n_keep]
   int32_t* idx_out;         // [rows][n_keep] or null
@@ -95,17 +143,10 @@ struct FinalParams {
   int32_t cap;              // candidate list capacity
   int32_t scap;             // candidates held in shared memory
   int32_t words;
-  // the attention kernel's query terms, prepared here once per row
-  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
-  unsigned char* qterms;    // [rows][kQTermBytes]
-  int32_t group;
-  double cosv[kNFC];        // cos / sin of q_pos * theta_i (host, float64)
-  double sinv[kNFC];
 };
 
 __host__ __device__ inline int final_smem_bytes(int words, int scap) {
-  return sa_align(words * 4, 128) + (kSAWarps * 256 + 264) * 4 + 64 * 4 + sa_align(2 * scap * 4, 16) +
-         FASA_MAX_GROUP * kD * 2;
+  return sa_align(words * 4, 128) + (kSAWarps * 256 + 264) * 4 + 64 * 4 + 2 * scap * 4;
 }
 
 __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalParams p) {
@@ -120,43 +161,30 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
   uint32_t* scan = rscr + kSAWarps * 256 + 264;
   uint32_t* ckey = scan + 64;                           // [scap]
   int32_t* cidx = reinterpret_cast<int32_t*>(ckey + p.scap);  // [scap]
-  // [G][128], 16-byte aligned for the vector stores below (scap may be odd)
-  __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(
-      reinterpret_cast<unsigned char*>(ckey) + sa_align(2 * p.scap * 4, 16));
 
-  // the group's rotated query terms for the attention kernel
-  {
-    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)row * p.group) * kD);
-    for (int c = tid; c < p.group * kD / 8; c += kSAThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
-    __syncthreads();
-    query_terms(qraw, p.group, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes, tid, kSAThreads);
+  // the candidate count and, asynchronously, the filter's bitmap, while
+  // the threshold bin is found again from the histogram
+  const uint32_t n_c = __ldcg(p.cand_cnt + row);
+  const uint32_t* gbm = p.bitmap + (int64_t)row * p.words;
+  for (int w = tid; w < p.words; w += kSAThreads) cp_async4(bm + w, gbm + w);
+  cp_async_commit();
+  const bool fast = n_c <= (uint32_t)p.cap && n_c <= (uint32_t)p.scap;
+  if (fast) {  // the (index, key) candidates, also in flight during the scan
+    const int32_t* gi = p.cand_idx + (int64_t)row * p.cap;
+    const uint32_t* gk = p.cand_key + (int64_t)row * p.cap;
+    for (int j = tid; j < (int)n_c; j += kSAThreads) {
+      cp_async4(cidx + j, gi + j);
+      cp_async4(ckey + j, gk + j);
+    }
   }
-
+  cp_async_commit();
   uint32_t bin, above;
   hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);
   const int krem = p.n_keep - (int)above;
-  const uint32_t n_c = __ldcg(p.cand_cnt + row);
-  const uint32_t* gbm = p.bitmap + (int64_t)row * p.words;
+  cp_async_wait<0>();
+  __syncthreads();
 
-  if (n_c <= (uint32_t)p.cap && n_c <= (uint32_t)p.scap) {
-    for (int w = tid; w < p.words; w += kSAThreads) bm[w] = __ldcg(gbm + w);
-    const float* s = p.scores + (int64_t)row * p.len;
-    const int32_t* gc0 = p.cand_idx + (int64_t)row * p.cap;
-    constexpr int U = 4;
-    for (int j0 = tid; j0 < (int)n_c; j0 += kSAThreads * U) {
-      int t[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) t[u] = j0 + u * kSAThreads < (int)n_c ? __ldcg(gc0 + j0 + u * kSAThreads) : 0;
-      float f[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) f[u] = j0 + u * kSAThreads < (int)n_c ? __ldcg(s + t[u]) : 0.0f;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (j0 + u * kSAThreads < (int)n_c) {
-          cidx[j0 + u * kSAThreads] = t[u];
-          ckey[j0 + u * kSAThreads] = score_key(f[u]);
-        }
-    }
+  if (fast) {
     const int32_t* gc = cidx;
     auto key_of = [ckey](int j) { return ckey[j]; };
     __syncthreads();
@@ -192,6 +220,7 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
   } else {
     // slow exact path: this row's scores become keys in place, then a radix
     // select over all of them, then the bitmap from scratch in index order
+    // (overwriting the copied filter bitmap)
     uint32_t* keys = reinterpret_cast<uint32_t*>(p.scores + (int64_t)row * p.len);
     for (int i = tid; i < p.len; i += kSAThreads) keys[i] = score_key(__ldcg(p.scores + (int64_t)row * p.len + i));
     __threadfence_block();
