@@ -68,7 +68,8 @@ enum FuXch { kXTies = 0, kXKept = 1, kXRows = 2 };
 
 struct FusedParams {
   const __nv_bfloat16* sketch;  // [rows][max_len][stride]
-  const float* scores;          // [rows][len] TIP scores (the from-scores variant), else unused
+  const float* scores;          // [rows][sld] TIP scores (the from-scores variant), else unused
+  int64_t sld;                  // their row stride
   const __nv_bfloat16* k;       // [rows][max_len][128], rotated
   const __nv_bfloat16* v;
   const __nv_bfloat16* q;       // [B][Hq][128], pre-RoPE
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) decode_fused_kernel(const Fused
     __syncthreads();
     query_terms(qraw, G, p.cosv, p.sinv, qt, tid, kFuThreads);
     // the row's scores of this CTA's range: keys and the top-8-bit histogram
-    const float* src = p.scores + (int64_t)row * p.len + t0;
+    const float* src = p.scores + (int64_t)row * p.sld + t0;
     constexpr int U = 8;
     for (int i0 = tid; i0 < n; i0 += kFuThreads * U) {
       float f[U];

@@ -164,7 +164,7 @@ fasa_status launch_score_lpt(const ScoreParams& p, const DevInfo& d, cudaStream_
 // histogram of the top 12 bits of each score's order-preserving key (added
 // into `hist`, which must be zero).
 fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
-                         uint32_t* hist, cudaStream_t st) {
+                         int64_t ld, uint32_t* hist, cudaStream_t st) {
   DevInfo d;
   fasa_status s = device_info(&d);
   if (s != FASA_OK) return s;
@@ -173,6 +173,7 @@ fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_
   p.q = q;
   p.dom_idx = c->dom_idx;
   p.scores = scores;
+  p.ld = ld;
   p.hist = hist;
   p.max_len = c->max_len;
   p.total = (int64_t)c->batch * c->n_kv_heads * len;
@@ -483,11 +484,12 @@ fasa_status launch_fused_t(const FusedParams& p, int rows, const FusedPlan& pl, 
 // The cluster decode: streaming the sketch when scores is null, else reading
 // the scores [rows][len] a score-kernel launch wrote before it in the stream.
 fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t keff, void* out,
-                         int32_t* idx_out, const float* scores, const FusedPlan& pl, cudaStream_t st,
+                         int32_t* idx_out, const float* scores, int64_t sld, const FusedPlan& pl, cudaStream_t st,
                          const DevInfo& d) {
   FusedParams p{};
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
   p.scores = scores;
+  p.sld = sld;
   p.k = static_cast<const __nv_bfloat16*>(c->k);
   p.v = static_cast<const __nv_bfloat16*>(c->v);
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -519,7 +521,7 @@ fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_
 }
 
 // Decode workspace, each part 256-byte aligned:
-//   scores [rows][len] f32 | hist [rows][4096] u32 | cand_cnt [rows] u32 |
+//   scores [rows][ld] f32 (ld = len rounded up to 32) | hist [rows][4096] u32 | cand_cnt [rows] u32 |
 //   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
@@ -528,6 +530,7 @@ constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 struct DecodeWs {
   size_t scores, hist, cnt, att_cnt, bitmap, cand, ckey, idx, part, qterm, total;
+  int64_t ld;
   int cap, words, splits_max;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -547,8 +550,9 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.words = (int)((L + 31) / 32);
   w.cap = (int)std::min<size_t>(std::max<size_t>(L, 1), 8192);
   w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms, kAttMaxPerSm);
+  w.ld = (int64_t)((L + 31) / 32 * 32);
   w.scores = 0;
-  w.hist = al256(rows * L * 4);
+  w.hist = al256(rows * (size_t)w.ld * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
   w.att_cnt = w.cnt + rows * 4;
   w.bitmap = al256(w.att_cnt + rows * 4);
@@ -668,7 +672,7 @@ fasa_status fasa_score(const fasa_cache* c, int32_t len, const void* q, int32_t 
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (len == 0) return FASA_OK;
   if (!aligned(q, 16) || !aligned(scores, 4)) return FASA_ERR_INVALID_ARG;
-  return launch_score(c, len, q, q_pos, scores, nullptr, stream);
+  return launch_score(c, len, q, q_pos, scores, len, nullptr, stream);
 }
 
 fasa_status fasa_select_topk(const float* scores, int32_t n_rows, int32_t len, int32_t k, int32_t* idx,
@@ -733,7 +737,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     FusedPlan pl;
     bool ok = false;
     if ((s = fused_plan(c, len, d, path == FASA_DECODE_FUSED, false, &pl, &ok)) != FASA_OK) return s;
-    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, nullptr, pl, stream, d);
+    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, nullptr, 0, pl, stream, d);
     if (path == FASA_DECODE_FUSED) return FASA_ERR_UNSUPPORTED;
   }
   if (path == FASA_DECODE_AUTO || path == FASA_DECODE_SCORED) {
@@ -742,8 +746,8 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     if ((s = fused_plan(c, len, d, path == FASA_DECODE_SCORED, true, &pl, &ok)) != FASA_OK) return s;
     if (ok) {
       float* sc = reinterpret_cast<float*>(base + w.scores);
-      if ((s = launch_score(c, len, q, q_pos, sc, nullptr, stream)) != FASA_OK) return s;
-      return launch_fused(c, len, q, q_pos, keff, out, idx_out, sc, pl, stream, d);
+      if ((s = launch_score(c, len, q, q_pos, sc, w.ld, nullptr, stream)) != FASA_OK) return s;
+      return launch_fused(c, len, q, q_pos, keff, out, idx_out, sc, w.ld, pl, stream, d);
     }
     if (path == FASA_DECODE_SCORED) return FASA_ERR_UNSUPPORTED;
   }
@@ -759,11 +763,12 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   uint32_t* att_cnt = reinterpret_cast<uint32_t*>(base + w.att_cnt);
   float* part = reinterpret_cast<float*>(base + w.part);
   if ((s = cuda_status(cudaMemsetAsync(hist, 0, w.bitmap - w.hist, stream))) != FASA_OK) return s;
-  if ((s = launch_score(c, len, q, q_pos, scores, hist, stream)) != FASA_OK) return s;
+  if ((s = launch_score(c, len, q, q_pos, scores, w.ld, hist, stream)) != FASA_OK) return s;
 
   // 2. filter: certain tokens into the bitmap, threshold-bin tokens into the candidate list
   FilterParams fp{};
   fp.scores = scores;
+  fp.ld = w.ld;
   fp.hist = hist;
   fp.cand_cnt = cnt;
   fp.cand_idx = cand;
@@ -774,7 +779,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   fp.cap = w.cap;
   // one wave of four resident filter CTAs per SM
   const int64_t tiles_per_row = std::max<int64_t>(1, 4LL * d.sms / rows);
-  fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 32) * 32);
+  fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 128) * 128);
   fp.words = w.words;
   fp.q = static_cast<const __nv_bfloat16*>(q);
   fp.qterms = c->dtype == FASA_BF16 ? reinterpret_cast<unsigned char*>(base + w.qterm) : nullptr;
@@ -787,6 +792,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   // 3. finalize: exact threshold among the candidates, kept indices in ascending order
   FinalParams np{};
   np.scores = scores;
+  np.ld = w.ld;
   np.hist = hist;
   np.cand_cnt = cnt;
   np.cand_idx = cand;

@@ -36,7 +36,8 @@ struct ScoreParams {
   const void* sketch;    // [rows][max_len][stride]
   const void* q;         // [B][Hq][128]
   const int32_t* dom_idx;
-  float* scores;         // [rows][len]
+  float* scores;         // [rows][ld]
+  int64_t ld;            // row stride of scores, >= len
   uint32_t* hist;        // [rows][4096] key-histogram counts (added to), or null
   int64_t max_len;
   int64_t total;         // rows * len
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
 
     // warp w takes the steps w, w + kScoreWarps, ... of TPW consecutive tokens
     const char* src = static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
-    float* out = p.scores + (int64_t)row * p.len + t0;
+    float* out = p.scores + (int64_t)row * p.ld + t0;
     const int nblk = (n + S::TPW - 1) / S::TPW;
     const int mine = nblk > warp ? (nblk - warp + kScoreWarps - 1) / kScoreWarps : 0;
     auto issue = [&](int j) {

@@ -35,7 +35,8 @@ constexpr int kFilterThreads = kSAThreads;  // hist_threshold assumes 512 thread
 constexpr int kFilterCands = 2048;  // candidates a CTA gathers in shared memory
 
 struct FilterParams {
-  const float* scores;      // [rows][len]
+  const float* scores;      // [rows][ld], 16-byte aligned
+  int64_t ld;               // row stride of scores, a multiple of 32
   const uint32_t* hist;     // [rows][4096]
   uint32_t* cand_cnt;       // [rows], zero before the launch
   int32_t* cand_idx;        // [rows][cap]
@@ -44,7 +45,7 @@ struct FilterParams {
   int32_t len;
   int32_t n_keep;           // k_eff
   int32_t cap;
-  int32_t tile;             // tokens per CTA, a multiple of 32
+  int32_t tile;             // tokens per CTA, a multiple of 128
   int32_t words;            // ceil(len / 32)
   // the attention kernel's query terms, prepared by tile 0 of each row
   const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
@@ -61,7 +62,6 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
   __shared__ uint32_t s_n, s_base;
   const int row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned lt = (1u << lane) - 1u;
   // The query is an input of the whole decode, complete before the score
   // kernel started, so tile 0 can turn it into query terms before waiting;
   // the attention kernel reads them two launches later.
@@ -74,44 +74,58 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
   hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);  // its barriers publish s_n
   const int t0 = blockIdx.x * p.tile;
   const int t1 = min(p.len, t0 + p.tile);
-  const float* s = p.scores + (int64_t)row * p.len;
+  const float4* s4 = reinterpret_cast<const float4*>(p.scores + (int64_t)row * p.ld);
   uint32_t* bm = p.bitmap + (int64_t)row * p.words;
   int32_t* cidx = p.cand_idx + (int64_t)row * p.cap;
-  constexpr int U = 8;  // loads in flight per lane
-  for (int base0 = t0 + warp * 32; base0 < t1; base0 += kFilterThreads * U) {
-    float f[U];
+  // Lane l of a warp holds tokens base + 4l .. base + 4l + 3 of a 128-token
+  // step, so lanes 8j .. 8j+7 hold the 32 tokens of bitmap word j of the
+  // step (the row stride and the tile are multiples of 32 and 128, so every
+  // float4 is aligned and inside the row's padded stride).
+  constexpr int U = 2;  // 16-byte loads in flight per lane
+  constexpr int kStep = 128, kPass = kFilterThreads / 32 * kStep;
+  for (int base0 = t0 + warp * kStep; base0 < t1; base0 += kPass * U) {
+    float4 f[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int i = base0 + u * kFilterThreads + lane;
-      f[u] = i < t1 ? __ldcg(s + i) : 0.0f;
+      const int i = base0 + u * kPass + lane * 4;
+      f[u] = i < t1 ? __ldcg(s4 + i / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int base = base0 + u * kFilterThreads;
+      const int base = base0 + u * kPass;
       if (base >= t1) break;  // warp-uniform
-      const int i = base + lane;
-      const bool v = i < t1;
-      const uint32_t key = score_key(f[u]);
-      const uint32_t b = key >> 20;
-      const unsigned def = __ballot_sync(0xFFFFFFFFu, v && b > bin);
-      const unsigned cnd = __ballot_sync(0xFFFFFFFFu, v && b == bin);
-      if (lane == 0) bm[base >> 5] = def;
-      if (cnd) {
-        uint32_t at = 0u;
-        if (lane == 0) at = atomicAdd(&s_n, (uint32_t)__popc(cnd));
-        at = __shfl_sync(0xFFFFFFFFu, at, 0) + __popc(cnd & lt);
-        if ((cnd >> lane) & 1u) {
-          if (at < (uint32_t)kFilterCands) {
-            s_cidx[at] = i;
-            s_ckey[at] = key;
-          } else {  // this CTA's buffer is full (heavy ties): straight to the global list
-            const uint32_t g = atomicAdd(p.cand_cnt + row, 1u);
-            if (g < (uint32_t)p.cap) {
-              cidx[g] = i;
-              p.cand_key[(int64_t)row * p.cap + g] = key;
+      const int i = base + lane * 4;
+      const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+      uint32_t dn = 0u, cn = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool v = i + e < t1;
+        const uint32_t b = score_key(fv[e]) >> 20;
+        dn |= (uint32_t)(v && b > bin) << e;
+        cn |= (uint32_t)(v && b == bin) << e;
+      }
+      uint32_t dw = dn << (4 * (lane & 7));
+      dw |= __shfl_xor_sync(0xFFFFFFFFu, dw, 1);
+      dw |= __shfl_xor_sync(0xFFFFFFFFu, dw, 2);
+      dw |= __shfl_xor_sync(0xFFFFFFFFu, dw, 4);
+      if ((lane & 7) == 0 && i < t1) bm[i >> 5] = dw;
+      if (cn) {  // rare: this lane's threshold-bin tokens into the CTA's list
+        uint32_t at = atomicAdd(&s_n, (uint32_t)__popc(cn));
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((cn >> e) & 1u) {
+            if (at < (uint32_t)kFilterCands) {
+              s_cidx[at] = i + e;
+              s_ckey[at] = score_key(fv[e]);
+            } else {  // this CTA's buffer is full (heavy ties): straight to the global list
+              const uint32_t g = atomicAdd(p.cand_cnt + row, 1u);
+              if (g < (uint32_t)p.cap) {
+                cidx[g] = i + e;
+                p.cand_key[(int64_t)row * p.cap + g] = score_key(fv[e]);
+              }
             }
+            ++at;
           }
-        }
       }
     }
   }
@@ -130,7 +144,8 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
 }
 
 struct FinalParams {
-  float* scores;            // [rows][len]; the slow path turns a row into keys in place
+  float* scores;            // [rows][ld]; the slow path turns a row into keys in place
+  int64_t ld;
   const uint32_t* hist;
   const uint32_t* cand_cnt;
   const int32_t* cand_idx;  // [rows][cap]
@@ -221,8 +236,8 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
     // slow exact path: this row's scores become keys in place, then a radix
     // select over all of them, then the bitmap from scratch in index order
     // (overwriting the copied filter bitmap)
-    uint32_t* keys = reinterpret_cast<uint32_t*>(p.scores + (int64_t)row * p.len);
-    for (int i = tid; i < p.len; i += kSAThreads) keys[i] = score_key(__ldcg(p.scores + (int64_t)row * p.len + i));
+    uint32_t* keys = reinterpret_cast<uint32_t*>(p.scores + (int64_t)row * p.ld);
+    for (int i = tid; i < p.len; i += kSAThreads) keys[i] = score_key(__ldcg(p.scores + (int64_t)row * p.ld + i));
     __threadfence_block();
     __syncthreads();
     uint32_t thr;
