@@ -218,6 +218,27 @@ def test_decode_with_tied_tokens(path):
     assert kept_zero == list(range(1000, 1037))
 
 
+def test_decode_with_small_tie_at_budget_edge(path):
+    """Six scattered tokens score exactly 0 and the budget ends inside them:
+    the threshold bin holds only the tie (a small union, resolved by
+    ranking), and the three lowest indices of it are kept."""
+    wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=4000)
+    inp = W.layer_inputs(wl)
+    dom = inp.params.dom_idx[0]
+    tied = [17, 400, 401, 1999, 2500, 3999]
+    for t in tied:
+        inp.k[0, 0, t, np.concatenate([dom, dom + 64])] = 0   # +0.0
+    _, cache, q = U.build(wl, inp=inp)
+    _, s_ref, _ = U.oracle_scores(wl, inp, cache, 0, 0)
+    assert np.sum(s_ref == 0) == len(tied)
+    k = int(np.sum(s_ref > 0)) + 3
+    out, idx = _decode(wl, cache, q, k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, k, [(0, 0)], out, idx, scores_gpu=s)
+    kept_zero = [t for t in idx.cpu().numpy()[0, 0] if s_ref[t] == 0]
+    assert kept_zero == tied[:3]
+
+
 @pytest.mark.parametrize("case", ["all_tied", "k_beyond_union"])
 def test_decode_exact_fallbacks(case, path):
     """Shapes where the single-launch decode's candidate union cannot prove
