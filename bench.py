@@ -70,6 +70,39 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def csrc_sha256() -> str:
+    """Digest of every kernel and host source of the library, in name order."""
+    import hashlib
+    d = os.path.join(ROOT, "rope_frequency_chunk_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read() + b"\0")
+    return h.hexdigest()
+
+
+def workload_sig(wl: W.Workload, k: int) -> str:
+    """The shape a launch processes: config, batch, heads, context, FCs, budget."""
+    return f"{wl.name}-B{wl.batch}-H{wl.n_q_heads}/{wl.n_kv_heads}-L{wl.ctx_len}-n{wl.n_dom}-k{k}-{wl.dtype}"
+
+
+def profiled_traffic(summary: str, workload: str):
+    """DRAM bytes per launch (read + write) that an ncu capture recorded for
+    the dominant kernel on this workload, or None: the summary under profiles/
+    carries one machine-readable line, and its figure holds only while the
+    library's sources are byte-identical to those captured."""
+    import re
+    try:
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m = re.search(r"<!-- traffic workload=(\S+) bytes_per_launch=(\d+) csrc_sha256=([0-9a-f]{64}) -->", text)
+    if not m or m.group(1) != workload or m.group(3) != csrc_sha256():
+        return None
+    return int(m.group(2))
+
+
 # ------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -325,7 +358,8 @@ def run_fasa(args, wl):
     if fused:
         roof = {"bound": "hbm", "kernel": "decode_fused_kernel (score + select + attend, one launch per layer)",
                 "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / world / hbm_peak,
-                "traffic": None, "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind,
+                "traffic": profiled_traffic("decode_fused_kernel_c2.md", workload_sig(wl, k)),
+                "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind,
                 "us_per_launch": us_layer}
     else:
         ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
