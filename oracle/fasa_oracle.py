@@ -21,6 +21,10 @@ Attention" computes at decode time (gist.science technical summary, §2
    attention over exactly those rows, each kept at its original absolute
    position (its key was rotated at that position when it was cached).
 4. Dense full-KV attention (the comparison): the same attention over all rows.
+5. Offline calibration (§2, TIP first bullet): the agreement of each single
+   FC's token selection with the full head's over calibration queries picks
+   the dominant FCs (the reading of "Contextual Agreement" is stated at the
+   calibration functions).
 
 Stored values (the KV cache, the dominant-FC key sketch) are rounded once to
 the cache dtype, as the cache stores them. Every function takes and returns
@@ -218,3 +222,66 @@ def decode_head(q_pre: np.ndarray, q_pos: int, k_rot: np.ndarray, v: np.ndarray,
     out = focused_attention(q_rot, k_rot, v, idx)
     return idx, out, s
 
+
+
+# ------------------------------------------------------- calibration
+#
+# Offline calibration of the dominant FCs (gist.science technical summary,
+# §2, TIP first bullet): per attention head, the "Contextual Agreement" (CA)
+# between the attention scores of a single FC and those of the full head,
+# over a small calibration set, picks I_dom. The pages give no formula for
+# CA. Reading taken here: the agreement of the token sets each one selects
+# at the decode budget K, i.e. |Top_K(P_i) ∩ Top_K(full)| summed over the
+# calibration queries, with scores and selection exactly as the decode does
+# them (group-summed, rounded to float32, ties to the lower index).
+
+
+def calibration_scores(q_pre_win: np.ndarray, pos_win, k_rot: np.ndarray, base: float) -> np.ndarray:
+    """Score planes of one (sequence, KV head) for W calibration queries.
+
+    q_pre_win: [W, G, d] stored pre-RoPE queries; pos_win: [W] positions;
+    k_rot: [L, d] stored rotated keys. Returns float32 [W, 65, L]: plane i < 64
+    is the single-FC score P_i(t) = qs[i] k[t][i] + qs[i+64] k[t][i+64] with
+    qs the group's rotated queries added head by head (head 0 first), and
+    plane 64 the full-head score, the 64 planes added in FC order. Every
+    product and sum is one float64 operation, rounded to float32 at the end.
+    """
+    q = to_f64(q_pre_win)
+    W, G, d = q.shape
+    h = d // 2
+    k = to_f64(k_rot)
+    out = np.empty((W, NFC + 1, k.shape[0]), np.float32)
+    for w in range(W):
+        qr = rope_rotate(q[w], int(pos_win[w]), base)           # [G, d]
+        qs = qr[0].copy()
+        for g in range(1, G):
+            qs = qs + qr[g]
+        acc = None
+        for i in range(h):
+            p = qs[i] * k[:, i] + qs[i + h] * k[:, i + h]
+            out[w, i] = p.astype(np.float32)
+            acc = p if acc is None else acc + p
+        out[w, NFC] = acc.astype(np.float32)
+    return out
+
+
+def calibration_counts(planes: np.ndarray, budget: int) -> np.ndarray:
+    """Agreement counts of one (sequence, KV head): for each FC i, the number
+    of tokens its top-K set shares with the full head's, summed over the W
+    calibration queries (K_eff = min(K, L); selection as select_critical_set
+    on the float32 planes). planes: [W, 65, L]. Returns int64 [64]."""
+    W = planes.shape[0]
+    counts = np.zeros(NFC, np.int64)
+    for w in range(W):
+        full = select_critical_set(planes[w, NFC], budget)
+        for i in range(NFC):
+            counts[i] += np.intersect1d(select_critical_set(planes[w, i], budget), full).size
+    return counts
+
+
+def dominant_from_counts(counts: np.ndarray, n_dom: int) -> np.ndarray:
+    """I_dom: the n_dom FCs of largest agreement, ties to the lower FC index,
+    listed in that order (int32)."""
+    c = np.asarray(counts, dtype=np.int64)
+    order = np.lexsort((np.arange(c.shape[0]), -c))
+    return order[:n_dom].astype(np.int32)

@@ -301,12 +301,105 @@ def check_append_positions(m):
     return bool(ok)
 
 
+# ------------------------------------------------------------ calibration
+
+def _calib_case(L=40, G=3, W=3, seed=21, dtype="f32", base=1e4):
+    r = np.random.default_rng(seed)
+    q = (r.standard_normal((W, G, 128)) * np.exp(r.standard_normal(128))).astype(np.float32)
+    kpre = (r.standard_normal((L, 128)) * np.exp(r.standard_normal(128))).astype(np.float32)
+    q = O.store(q, dtype)
+    k_rot = O.store(O.rope_rotate(O.to_f64(O.store(kpre, dtype)), np.arange(L), base), dtype)
+    pos = L + np.arange(W) * 7
+    return q, pos, k_rot, base
+
+
+def _complex_planes(q, pos, k_rot, base):
+    """Group-summed FC shares by complex rotation: z = (x_i + j x_{i+64}) e^{j p theta_i}."""
+    qq = O.to_f64(q)
+    kk = O.to_f64(k_rot)
+    theta = np.power(float(base), -np.arange(64) / 64.0)
+    kz = kk[:, :64] + 1j * kk[:, 64:]
+    out = []
+    for w in range(qq.shape[0]):
+        z = (qq[w, :, :64] + 1j * qq[w, :, 64:]) * np.exp(1j * pos[w] * theta)   # [G, 64]
+        share = np.real(z.sum(0)[None, :] * np.conj(kz))                           # [L, 64]
+        out.append(np.concatenate([share.T, share.sum(1)[None, :]], axis=0))      # [65, L]
+    return np.stack(out)
+
+
+def check_calib_planes_closed_form(m):
+    q, pos, k_rot, base = _calib_case(dtype="bf16")
+    got = m.calibration_scores(q, pos, k_rot, base).astype(np.float64)
+    want = _complex_planes(q, pos, k_rot, base)
+    scale = np.abs(want).max()
+    return got.shape == (3, 65, 40) and np.abs(got - want).max() <= 1e-6 * scale
+
+
+def check_calib_planes_match_tip(m):
+    q, pos, k_rot, base = _calib_case(L=33, G=2, W=2, seed=22)
+    planes = m.calibration_scores(q, pos, k_rot, base)
+    ok = True
+    for w in range(2):
+        qr = m.rotate_queries(q[w], int(pos[w]), base)
+        full = m.tip_scores(qr, m.sketch_rows(k_rot, np.arange(64)), np.arange(64))
+        ok &= np.allclose(planes[w, 64], full, rtol=2e-7, atol=1e-6 * np.abs(full).max())
+        for i in (0, 17, 63):
+            one = m.tip_scores(qr, m.sketch_rows(k_rot, np.array([i])), np.array([i]))
+            ok &= np.allclose(planes[w, i], one, rtol=2e-7, atol=1e-6 * np.abs(one).max() + 1e-30)
+    return bool(ok)
+
+
+def check_calib_counts_brute_force(m):
+    r = np.random.default_rng(23)
+    W, L, K = 3, 24, 5
+    planes = r.standard_normal((W, 65, L)).astype(np.float32)
+    planes[0, 3, 7] = planes[0, 3, 11] = np.sort(planes[0, 3])[-5]   # a tie at the boundary
+    planes[1, 64, 2] = planes[1, 64, 20] = np.sort(planes[1, 64])[-5]
+    want = np.zeros(64, np.int64)
+    for w in range(W):
+        rank = lambda row: {t for _, t in sorted((-float(row[t]), t) for t in range(L))[:K]}
+        full = rank(planes[w, 64])
+        for i in range(64):
+            want[i] += len(rank(planes[w, i]) & full)
+    return np.array_equal(m.calibration_counts(planes, K), want)
+
+
+def check_calib_single_fc_query(m):
+    q, pos, k_rot, base = _calib_case(L=60, G=2, W=2, seed=24)
+    j = 37
+    mask = np.zeros(128, bool)
+    mask[[j, j + 64]] = True
+    q = np.where(mask, q, np.float32(0))
+    planes = m.calibration_scores(q, pos, k_rot, base)
+    c = m.calibration_counts(planes, 8)
+    others = np.delete(c, j)
+    return (np.array_equal(planes[:, j], planes[:, 64]) and c[j] == 2 * 8 and others.max() < c[j]
+            and m.dominant_from_counts(c, 1)[0] == j)
+
+
+def check_calib_budget_covers_all(m):
+    q, pos, k_rot, base = _calib_case(L=12, G=1, W=2, seed=25)
+    c = m.calibration_counts(m.calibration_scores(q, pos, k_rot, base), 50)
+    return np.array_equal(c, np.full(64, 2 * 12)) and list(m.dominant_from_counts(c, 4)) == [0, 1, 2, 3]
+
+
+def check_dominant_ties(m):
+    c = np.zeros(64, np.int64)
+    c[[1, 2, 4]] = 7
+    c[0] = 5
+    c[3] = 1
+    return (list(m.dominant_from_counts(c, 3)) == [1, 2, 4]
+            and list(m.dominant_from_counts(c, 6)) == [1, 2, 4, 0, 3, 5])
+
+
 PINS = [check_bf16_vs_torch, check_bf16_halfway_exact, check_rope_vs_complex,
         check_rope_vs_transformers, check_rope_invariants, check_fc_partials_sum_to_dot,
         check_fc_partial_closed_form, check_tip_all_fcs_is_dot, check_tip_subset_is_partial_sum,
         check_tip_gqa_linear, check_tip_brute_force, check_select_brute_force,
         check_select_permutation, check_dense_vs_sdpa, check_focused_special_cases,
-        check_e2e_all_fc_full_k_is_dense, check_e2e_all_fc_topk_exact, check_append_positions]
+        check_e2e_all_fc_full_k_is_dense, check_e2e_all_fc_topk_exact, check_append_positions,
+        check_calib_planes_closed_form, check_calib_planes_match_tip, check_calib_counts_brute_force,
+        check_calib_single_fc_query, check_calib_budget_covers_all, check_dominant_ties]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -391,6 +484,29 @@ def _mut_bf16_trunc(x):
     return (x.view(np.uint32) >> 16).astype(np.uint16)
 
 
+def _mut_calib_adjacent(q_pre_win, pos_win, k_rot, base):
+    perm = np.empty(128, np.int64)
+    perm[0::2], perm[1::2] = np.arange(64), np.arange(64, 128)
+    return _orig_calib_scores(q_pre_win[..., perm], pos_win, k_rot[..., perm], base)
+
+
+def _mut_calib_head0(q_pre_win, pos_win, k_rot, base):
+    return _orig_calib_scores(q_pre_win[:, :1], pos_win, k_rot, base)
+
+
+def _mut_calib_abs(planes, budget):
+    return _orig_calib_counts(np.abs(planes), budget)
+
+
+def _mut_dominant_high_tie(counts, n_dom):
+    c = np.asarray(counts, dtype=np.int64)
+    return np.lexsort((-np.arange(c.shape[0]), -c))[:n_dom].astype(np.int32)
+
+
+_orig_calib_scores = O.calibration_scores
+_orig_calib_counts = O.calibration_counts
+
+
 _orig_append = O.append_kv
 _orig_tip = O.tip_scores
 
@@ -405,6 +521,10 @@ MUTANTS = {
     "sketch_wrong_pair": ("sketch_rows", _mut_sketch),
     "append_position_off_by_one": ("append_kv", _mut_append_pos),
     "bf16_truncates": ("f64_to_bf16_bits", _mut_bf16_trunc),
+    "calib_adjacent_pairs": ("calibration_scores", _mut_calib_adjacent),
+    "calib_drops_group_heads": ("calibration_scores", _mut_calib_head0),
+    "calib_selects_magnitude": ("calibration_counts", _mut_calib_abs),
+    "calib_dominant_ties_to_higher_fc": ("dominant_from_counts", _mut_dominant_high_tie),
 }
 
 
