@@ -435,6 +435,80 @@ def run_fasa(args, wl):
     return 0
 
 
+def run_calibrate(args, wl):
+    """Offline FC calibration of one layer: its 65 score planes per calibration
+    query, the agreement counts and the dominant sets, each stage timed from
+    a CUDA graph with events. Algorithmic bytes: the layer's K cache and the
+    calibration queries; the score planes are the implementation's own
+    intermediate (written once, read once by the selection)."""
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+    torch.cuda.set_device(0)
+    k = args.k or wl.k
+    n_win = args.cal_win
+    inp = W.layer_inputs(wl, layer=0)
+    lp = inp.params
+    cache = F.KVCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, lp.dom_idx.shape[1], wl.ctx_len, wl.dtype,
+                      wl.rope_base, lp.dom_idx)
+    F.fasa_append_kv(cache, W.to_torch(inp.k, "cuda"), W.to_torch(inp.v, "cuda"), 0)
+    G = wl.group
+    sdt = np.float32 if wl.dtype == "f32" else np.uint16
+    qw = np.empty((wl.batch, n_win, wl.n_q_heads, W.HEAD_DIM), sdt)
+    for b in range(wl.batch):
+        for w in range(n_win):
+            for g in range(wl.n_kv_heads):
+                qw[b, w, g * G:(g + 1) * G] = W.head_q(wl, lp, 0, b, g, step=100 + w)
+    q_t = W.to_torch(qw, "cuda")
+    L = wl.ctx_len
+    rows = wl.batch * wl.n_kv_heads
+    planes = torch.empty(wl.batch, wl.n_kv_heads, n_win, F.CAL_PLANES, L, dtype=torch.float32, device="cuda")
+    counts = torch.empty(wl.n_kv_heads, 64, dtype=torch.int32, device="cuda")
+    dom = torch.empty(wl.n_kv_heads, wl.n_dom, dtype=torch.int32, device="cuda")
+    sel_ws = torch.empty(rows * n_win * F.CAL_PLANES * min(k, L) * 4, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(F.fasa_calibrate_workspace_bytes(cache, L, n_win, k), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    stages = {
+        "scores": lambda: F.fasa_calibrate_scores(cache, L, q_t, L, planes=planes, stream=stream),
+        "counts": lambda: F.fasa_calibrate_counts(planes, wl.n_kv_heads, k, counts=counts, workspace=sel_ws,
+                                                  stream=stream),
+        "dominant": lambda: F.fasa_calibrate_dominant(counts, wl.n_dom, dom_idx=dom, stream=stream),
+        "whole": lambda: F.fasa_calibrate(cache, L, q_t, L, k, wl.n_dom, counts=counts, dom_idx=dom,
+                                          workspace=ws, stream=stream),
+    }
+    hbm_peak, peak_kind = peaks()
+    with ClockSampler(0) as clk:
+        ms = {name: time_graph(fn, args.steps, args.warmup, stream) / args.steps for name, fn in stages.items()}
+    status = F.fasa_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed calibration")
+    es = wl.elem_bytes
+    alg = rows * L * W.HEAD_DIM * es + wl.batch * n_win * wl.n_q_heads * W.HEAD_DIM * es
+    plane_bytes = rows * n_win * F.CAL_PLANES * L * 4
+    scores_gbs = (rows * L * W.HEAD_DIM * es + plane_bytes) / (ms["scores"] * 1e-3) / 1e9
+    line = {
+        "metric": "fasa_calibrate ms per layer calibration (calibration queries x budget), algorithmic GB/s",
+        "value": alg / (ms["whole"] * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms["whole"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name} calibration", "batch": wl.batch,
+                   "heads": f"{wl.n_q_heads}/{wl.n_kv_heads}", "ctx_len": L, "budget": k, "n_win": n_win,
+                   "n_dom": wl.n_dom, "parallelism": "single",
+                   "l2": f"score planes of {plane_bytes / 2**20:.0f} MiB per step (larger than L2)"},
+        "stage_ms": ms,
+        "roofline": {"bound": "hbm", "kernel": "calib_score_kernel (65 score planes per query)",
+                     "achieved": scores_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": scores_gbs / hbm_peak,
+                     "traffic": None, "bytes_per_launch": rows * L * W.HEAD_DIM * es + plane_bytes,
+                     "peak_kind": peak_kind, "us_per_launch": 1e3 * ms["scores"]},
+        "algorithmic_bytes": alg, "plane_bytes": plane_bytes,
+        "clocks": clk.summary(),
+        # per whole calibration: the score kernel, the selection launches, overlap, rank
+        "gpu_launches": (3 + -(-rows * n_win * F.CAL_PLANES // 65535)) * args.steps,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,6 +525,9 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--calibrate", action="store_true",
+                    help="time the offline FC calibration on one layer of the workload instead of the decode")
+    ap.add_argument("--cal-win", type=int, default=8, help="calibration queries per sequence (--calibrate)")
     return ap
 
 
@@ -467,6 +544,8 @@ def main(argv=None):
         wl = wl.replace(batch=args.batch)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.calibrate:
+        return run_calibrate(args, wl)
     return run_fasa(args, wl)
 
 

@@ -54,6 +54,7 @@ extern "C" {
 #define FASA_MAX_GROUP 16          /* largest G = Hq / Hkv */
 #define FASA_MAX_LEN (1 << 19)     /* largest cached length a decode call accepts */
 #define FASA_MAX_K (1 << 17)       /* largest kept-token budget */
+#define FASA_CAL_MAX_WIN 8         /* calibration queries per calibration call */
 
 typedef enum fasa_status {
   FASA_OK = 0,
@@ -294,6 +295,73 @@ fasa_status fasa_dense_decode(const fasa_cache* cache, int32_t len, const void* 
  * Returns FASA_ERR_CUDA if the synchronization itself fails.
  */
 fasa_status fasa_device_status(int32_t clear);
+
+/*
+ * Offline calibration of the dominant FCs ([tech §2] TIP, first bullet: once,
+ * before decoding, each head's I_dom is found from the "Contextual Agreement"
+ * between the attention scores of a single FC and of the full head over a
+ * small calibration set). The pages give no formula for the agreement; these
+ * calls measure it as the overlap of the token sets the two scores select
+ * at the decode budget, exactly as the decode selects them.
+ *
+ * Calibration query w of sequence b sits at position q_pos0 + w and attends
+ * to the len cached rows of the cache (its keys, not its sketch). For KV
+ * head g, with qs = the group's G rotated queries added head by head:
+ *   plane i < 64 : P_i(t)  = qs[i] k[t][i] + qs[i+64] k[t][i+64]
+ *   plane 64     : full(t) = P_0(t) + P_1(t) + ... + P_63(t)   (FC order)
+ * each product and sum one float64 operation, the result rounded once to
+ * float32. Then, with K_eff = min(budget, len) and Top_K the selection of
+ * fasa_select_topk (ties to the lower index):
+ *   counts[g][i] = sum over b and w of |Top_K(plane i) ∩ Top_K(plane 64)|
+ *   dom_idx[g]   = the n_dom FCs with the largest counts, ties to the lower
+ *                  FC index, in that order (a valid cache dom_idx row).
+ */
+
+/* Workspace bytes fasa_calibrate needs (0 for invalid arguments). */
+size_t fasa_calibrate_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t n_win, int32_t budget);
+
+/*
+ * The 65 score planes of every calibration query.
+ *  q_win  : [B][n_win][Hq][128] dtype, pre-RoPE calibration queries.
+ *  planes : [B][Hkv][n_win][65][len] float32 (row stride len).
+ *  Errors: n_win outside 1..FASA_CAL_MAX_WIN, len < 1, q_pos0 < 0 or
+ *  q_pos0 + n_win > 2^31 - 1 -> FASA_ERR_INVALID_ARG; len > max_len ->
+ *  FASA_ERR_CAPACITY.
+ */
+fasa_status fasa_calibrate_scores(const fasa_cache* cache, int32_t len, const void* q_win, int32_t q_pos0,
+                                  int32_t n_win, float* planes, cudaStream_t stream);
+
+/*
+ * Agreement counts from score planes laid out as fasa_calibrate_scores
+ * writes them ([n_rows][n_win][65][len], n_rows = B * Hkv, row r belonging
+ * to KV head r % n_kv_heads).
+ *  counts    : [n_kv_heads][64] uint32, overwritten.
+ *  workspace : at least n_rows * n_win * 65 * min(budget, len) * 4 bytes
+ *              (the selections), 4-byte aligned.
+ *  Errors: n_rows not a positive multiple of n_kv_heads, budget < 1,
+ *  n_win outside 1..FASA_CAL_MAX_WIN or len < 1 -> FASA_ERR_INVALID_ARG;
+ *  len > FASA_MAX_LEN or budget > FASA_MAX_K -> FASA_ERR_UNSUPPORTED;
+ *  a short workspace -> FASA_ERR_WORKSPACE.
+ */
+fasa_status fasa_calibrate_counts(const float* planes, int32_t n_rows, int32_t n_kv_heads, int32_t n_win,
+                                  int32_t len, int32_t budget, uint32_t* counts, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * I_dom from counts: dom_idx [n_kv_heads][n_dom] int32 (device).
+ *  Errors: n_kv_heads < 1 or n_dom outside 1..64 -> FASA_ERR_INVALID_ARG.
+ */
+fasa_status fasa_calibrate_dominant(const uint32_t* counts, int32_t n_kv_heads, int32_t n_dom, int32_t* dom_idx,
+                                    cudaStream_t stream);
+
+/*
+ * The whole calibration: fasa_calibrate_scores into the workspace, then
+ * fasa_calibrate_counts and fasa_calibrate_dominant. counts and dom_idx as
+ * above; workspace of fasa_calibrate_workspace_bytes, 256-byte aligned.
+ */
+fasa_status fasa_calibrate(const fasa_cache* cache, int32_t len, const void* q_win, int32_t q_pos0, int32_t n_win,
+                           int32_t budget, int32_t n_dom, uint32_t* counts, int32_t* dom_idx, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -16,6 +16,7 @@
 #include "select_hist.cuh"
 #include "attend_mma.cuh"
 #include "decode_fused.cuh"
+#include "calibrate.cuh"
 
 using namespace fasa;
 
@@ -583,6 +584,38 @@ fasa_status launch_pdl(K kern, dim3 grid, int threads, size_t smem, cudaStream_t
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
+// Calibration workspace: score planes [rows][n_win][65][len] f32, then the
+// selections [rows][n_win][65][k_eff] i32.
+struct CalWs {
+  size_t planes, idx, total;
+};
+CalWs cal_layout(int64_t rows, int32_t len, int32_t n_win, int32_t budget) {
+  CalWs w;
+  const int64_t keff = std::min<int64_t>(budget, len);
+  w.planes = 0;
+  w.idx = al256((size_t)rows * n_win * kCalPlanes * (size_t)len * 4);
+  w.total = al256(w.idx + (size_t)rows * n_win * kCalPlanes * (size_t)keff * 4);
+  return w;
+}
+
+template <typename T>
+fasa_status launch_cal_scores(const fasa_cache* c, int32_t len, const void* q_win, int32_t q_pos0, int32_t n_win,
+                              float* planes, cudaStream_t st) {
+  CalScoreParams p{};
+  p.k = c->k;
+  p.q = q_win;
+  p.planes = planes;
+  p.max_len = c->max_len;
+  p.len = len;
+  p.n_win = n_win;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  for (int w = 0; w < n_win; ++w) fill_query_angle(p.cosv[w], p.sinv[w], c->rope_base, q_pos0 + w);
+  const dim3 grid((unsigned)ceil_div(len, kCalThreads), (unsigned)(c->batch * c->n_kv_heads), 1);
+  calib_score_kernel<T><<<grid, kCalThreads, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 // =================================================================== ABI
@@ -921,6 +954,96 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
   p.n_kv_heads = c->n_kv_heads;
   p.group = c->n_q_heads / c->n_kv_heads;
   return launch_sa<kDense>(c, p, c->batch * c->n_kv_heads, false, stream, c->dtype, q_pos);
+}
+
+size_t fasa_calibrate_workspace_bytes(const fasa_cache* c, int32_t len, int32_t n_win, int32_t budget) {
+  if (check_cache(c) != FASA_OK || len < 1 || len > c->max_len || n_win < 1 || n_win > kCalMaxWin || budget < 1)
+    return 0;
+  return cal_layout((int64_t)c->batch * c->n_kv_heads, len, n_win, budget).total;
+}
+
+fasa_status fasa_calibrate_scores(const fasa_cache* c, int32_t len, const void* q_win, int32_t q_pos0,
+                                  int32_t n_win, float* planes, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || n_win < 1 || n_win > kCalMaxWin || q_pos0 < 0 || (int64_t)q_pos0 + n_win > INT32_MAX)
+    return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (!aligned(q_win, 16) || !aligned(planes, 4)) return FASA_ERR_INVALID_ARG;
+  return c->dtype == FASA_F32 ? launch_cal_scores<float>(c, len, q_win, q_pos0, n_win, planes, stream)
+                              : launch_cal_scores<__nv_bfloat16>(c, len, q_win, q_pos0, n_win, planes, stream);
+}
+
+fasa_status fasa_calibrate_counts(const float* planes, int32_t n_rows, int32_t n_kv_heads, int32_t n_win,
+                                  int32_t len, int32_t budget, uint32_t* counts, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+  if (!aligned(planes, 4) || !aligned(counts, 4)) return FASA_ERR_INVALID_ARG;
+  if (n_kv_heads < 1 || n_rows < 1 || n_rows % n_kv_heads != 0 || n_win < 1 || n_win > kCalMaxWin || len < 1 ||
+      budget < 1)
+    return FASA_ERR_INVALID_ARG;
+  if (len > FASA_MAX_LEN || budget > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
+  const int64_t keff = std::min<int64_t>(budget, len);
+  const int64_t sel_rows = (int64_t)n_rows * n_win * kCalPlanes;
+  if (sel_rows > INT32_MAX) return FASA_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 4) || workspace_bytes < (size_t)(sel_rows * keff * 4))
+    return FASA_ERR_WORKSPACE;
+  DevInfo d;
+  fasa_status s = device_info(&d);
+  if (s != FASA_OK) return s;
+  int32_t* idx = static_cast<int32_t*>(workspace);
+  if ((s = cuda_status(cudaMemsetAsync(counts, 0, (size_t)n_kv_heads * kNFC * 4, stream))) != FASA_OK) return s;
+  // every plane's selection, in launches of at most 65535 rows
+  for (int64_t r0 = 0; r0 < sel_rows; r0 += 65535) {
+    SAParams p{};
+    p.scores = planes + r0 * len;
+    p.idx_out = idx + r0 * keff;
+    p.len = len;
+    p.n_keep = (int32_t)keff;
+    p.group = 1;
+    if ((s = launch_sa<kSelect>(nullptr, p, (int)std::min<int64_t>(65535, sel_rows - r0), false, stream, FASA_F32,
+                                0)) != FASA_OK)
+      return s;
+  }
+  const size_t bm_bytes = (size_t)(len + 31) / 32 * 4;
+  if (bm_bytes > (size_t)d.smem_optin) return FASA_ERR_UNSUPPORTED;
+  int set = 0;
+  if ((s = cached_int((const void*)calib_overlap_kernel, 0, &set, [&](int* v) {
+         *v = 1;
+         return cuda_status(
+             cudaFuncSetAttribute(calib_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin));
+       })) != FASA_OK)
+    return s;
+  calib_overlap_kernel<<<(unsigned)((int64_t)n_rows * n_win), kCalThreads, bm_bytes, stream>>>(
+      idx, (int32_t)keff, len, n_kv_heads, n_win, counts);
+  return cuda_status(cudaGetLastError());
+}
+
+fasa_status fasa_calibrate_dominant(const uint32_t* counts, int32_t n_kv_heads, int32_t n_dom, int32_t* dom_idx,
+                                    cudaStream_t stream) {
+  if (!aligned(counts, 4) || !aligned(dom_idx, 4) || n_kv_heads < 1 || n_dom < 1 || n_dom > kNFC)
+    return FASA_ERR_INVALID_ARG;
+  calib_rank_kernel<<<(unsigned)n_kv_heads, kNFC, 0, stream>>>(counts, n_dom, dom_idx);
+  return cuda_status(cudaGetLastError());
+}
+
+fasa_status fasa_calibrate(const fasa_cache* c, int32_t len, const void* q_win, int32_t q_pos0, int32_t n_win,
+                           int32_t budget, int32_t n_dom, uint32_t* counts, int32_t* dom_idx, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (budget < 1 || n_dom < 1 || n_dom > kNFC || n_win < 1 || n_win > kCalMaxWin || len < 1)
+    return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  const int64_t rows = (int64_t)c->batch * c->n_kv_heads;
+  const CalWs w = cal_layout(rows, len, n_win, budget);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return FASA_ERR_WORKSPACE;
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  float* planes = reinterpret_cast<float*>(base + w.planes);
+  if ((s = fasa_calibrate_scores(c, len, q_win, q_pos0, n_win, planes, stream)) != FASA_OK) return s;
+  if ((s = fasa_calibrate_counts(planes, (int32_t)rows, c->n_kv_heads, n_win, len, budget, counts, base + w.idx,
+                                 w.total - w.idx, stream)) != FASA_OK)
+    return s;
+  return fasa_calibrate_dominant(counts, c->n_kv_heads, n_dom, dom_idx, stream);
 }
 
 fasa_status fasa_device_status(int32_t clear) {

@@ -61,6 +61,11 @@ _SIGS = {
     "fasa_device_status": (_I, [_I]),
     "fasa_set_decode_path": (_I, [_I]),
     "fasa_decode_path": (_I, [_CP, _I, _I]),
+    "fasa_calibrate_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I, _I]),
+    "fasa_calibrate_scores": (_I, [_CP, _I, _P, _I, _I, _P, _P]),
+    "fasa_calibrate_counts": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
+    "fasa_calibrate_dominant": (_I, [_P, _I, _I, _P, _P]),
+    "fasa_calibrate": (_I, [_CP, _I, _P, _I, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -254,3 +259,85 @@ def fasa_dense_decode(cache: KVCache, length: int, q, q_pos: int, out=None, stre
 def fasa_device_status(clear: bool = True) -> int:
     """Synchronizes; returns the device status word (0 = OK)."""
     return int(lib().fasa_device_status(1 if clear else 0))
+
+
+# ------------------------------------------------------------ calibration
+
+CAL_MAX_WIN = 8
+CAL_PLANES = 65
+
+
+def _q_win(cache, q_win):
+    _dev(q_win, "q_win", cache.dtype)
+    if q_win.dim() != 4 or q_win.shape[0] != cache.batch or q_win.shape[2] != cache.n_q_heads \
+            or q_win.shape[3] != HEAD_DIM:
+        raise ValueError("q_win must be [B, n_win, Hq, 128]")
+    return q_win.shape[1]
+
+
+def fasa_calibrate_workspace_bytes(cache: KVCache, length: int, n_win: int, budget: int) -> int:
+    return int(lib().fasa_calibrate_workspace_bytes(cache.ref(), length, n_win, budget))
+
+
+def fasa_calibrate_scores(cache: KVCache, length: int, q_win, q_pos0: int, planes=None, stream=None):
+    """Score planes [B, Hkv, n_win, 65, len] float32 of the calibration queries."""
+    n_win = _q_win(cache, q_win)
+    if planes is None:
+        planes = torch.empty(cache.batch, cache.n_kv_heads, n_win, CAL_PLANES, length, dtype=torch.float32,
+                             device=q_win.device)
+    _dev(planes, "planes", torch.float32)
+    _check(lib().fasa_calibrate_scores(cache.ref(), length, q_win.data_ptr(), q_pos0, n_win, planes.data_ptr(),
+                                       _stream(stream)), "fasa_calibrate_scores")
+    return planes
+
+
+def fasa_calibrate_counts(planes, n_kv_heads: int, budget: int, counts=None, workspace=None, stream=None):
+    """Agreement counts [Hkv, 64] uint32 (as int32 storage) from planes [..., n_win, 65, len]."""
+    _dev(planes, "planes", torch.float32)
+    n_win, length = planes.shape[-3], planes.shape[-1]
+    if planes.shape[-2] != CAL_PLANES:
+        raise ValueError("planes must be [..., n_win, 65, len]")
+    rows = planes.numel() // (n_win * CAL_PLANES * length)
+    if counts is None:
+        counts = torch.empty(n_kv_heads, 64, dtype=torch.int32, device=planes.device)
+    _dev(counts, "counts", torch.int32)
+    need = rows * n_win * CAL_PLANES * min(budget, length) * 4
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=planes.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_calibrate_counts(planes.data_ptr(), rows, n_kv_heads, n_win, length, budget,
+                                       counts.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                       _stream(stream)), "fasa_calibrate_counts")
+    return counts
+
+
+def fasa_calibrate_dominant(counts, n_dom: int, dom_idx=None, stream=None):
+    """I_dom [Hkv, n_dom] int32 from counts [Hkv, 64]."""
+    _dev(counts, "counts", torch.int32)
+    if dom_idx is None:
+        dom_idx = torch.empty(counts.shape[0], n_dom, dtype=torch.int32, device=counts.device)
+    _dev(dom_idx, "dom_idx", torch.int32)
+    _check(lib().fasa_calibrate_dominant(counts.data_ptr(), counts.shape[0], n_dom, dom_idx.data_ptr(),
+                                         _stream(stream)), "fasa_calibrate_dominant")
+    return dom_idx
+
+
+def fasa_calibrate(cache: KVCache, length: int, q_win, q_pos0: int, budget: int, n_dom: int,
+                   counts=None, dom_idx=None, workspace=None, stream=None):
+    """Offline calibration; returns (counts [Hkv, 64], dom_idx [Hkv, n_dom])."""
+    n_win = _q_win(cache, q_win)
+    dev = q_win.device
+    if counts is None:
+        counts = torch.empty(cache.n_kv_heads, 64, dtype=torch.int32, device=dev)
+    if dom_idx is None:
+        dom_idx = torch.empty(cache.n_kv_heads, n_dom, dtype=torch.int32, device=dev)
+    _dev(counts, "counts", torch.int32)
+    _dev(dom_idx, "dom_idx", torch.int32)
+    need = fasa_calibrate_workspace_bytes(cache, length, n_win, budget)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_calibrate(cache.ref(), length, q_win.data_ptr(), q_pos0, n_win, budget, n_dom,
+                                counts.data_ptr(), dom_idx.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                _stream(stream)), "fasa_calibrate")
+    return counts, dom_idx

@@ -108,3 +108,29 @@ def test_decode_path_setting_is_validated_on_the_host(L):
     for p in (1, 2, 3, 0):
         assert L.fasa_set_decode_path(p) == 0
     assert L.fasa_decode_path(None, 10, 10) < 0
+
+
+def test_calibration_validation_without_launch(L):
+    c = ctypes.byref(_fake_cache())
+    ws = L.fasa_calibrate_workspace_bytes
+    assert ws(c, 100, 0, 8) == 0 and ws(c, 100, 9, 8) == 0 and ws(c, 0, 2, 8) == 0 and ws(c, 100, 2, 0) == 0
+    rows = 2
+    need = ws(c, 100, 2, 8)
+    assert need >= rows * 2 * 65 * (100 + 8) * 4 and need % 256 == 0
+    assert L.fasa_calibrate_scores(c, 100, 0x50000, 0, 0, 0x60000, None) == 1       # n_win 0
+    assert L.fasa_calibrate_scores(c, 100, 0x50000, 0, 9, 0x60000, None) == 1       # n_win > 8
+    assert L.fasa_calibrate_scores(c, 100, 0x50000, -1, 2, 0x60000, None) == 1      # q_pos0 < 0
+    assert L.fasa_calibrate_scores(c, 2000, 0x50000, 0, 2, 0x60000, None) == 3      # len > max_len
+    assert L.fasa_calibrate_scores(c, 100, 0x50008, 0, 2, 0x60000, None) == 1       # misaligned q
+    cnt = L.fasa_calibrate_counts
+    assert cnt(0x50000, 3, 2, 2, 100, 8, 0x60000, 0x70000, 1 << 20, None) == 1      # rows % Hkv
+    assert cnt(0x50000, 2, 2, 2, 100, 0, 0x60000, 0x70000, 1 << 20, None) == 1      # budget 0
+    assert cnt(0x50000, 2, 2, 2, (1 << 19) + 1, 8, 0x60000, 0x70000, 1 << 30, None) == 2
+    assert cnt(0x50000, 2, 2, 2, 100, 8, 0x60000, 0x70000, 2 * 2 * 65 * 8 * 4 - 1, None) == 4
+    assert cnt(0x50000, 2, 2, 2, 100, 8, 0x60000, None, 1 << 20, None) == 4
+    assert L.fasa_calibrate_dominant(0x60000, 2, 0, 0x70000, None) == 1
+    assert L.fasa_calibrate_dominant(0x60000, 2, 65, 0x70000, None) == 1
+    assert L.fasa_calibrate_dominant(0x60000, 0, 4, 0x70000, None) == 1
+    assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 4, 0x60000, 0x70000, None, need, None) == 4
+    assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 4, 0x60000, 0x70000, 0x80000, need - 1, None) == 4
+    assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 0, 0x60000, 0x70000, 0x80000, need, None) == 1
