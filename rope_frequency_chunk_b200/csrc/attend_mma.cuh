@@ -29,7 +29,7 @@
 
 namespace fasa {
 
-constexpr int kAttWarps = 4;
+constexpr int kAttWarps = 3;  // four CTAs (12 warps) per SM at G <= 8
 constexpr int kAttThreads = kAttWarps * 32;
 constexpr int kAttChunk = 16;                          // rows per warp step
 constexpr int kAttStages = 2;                          // per-warp ring depth
@@ -287,14 +287,16 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
   }
   cp_async_wait<0>();
 
-  // warps merged pairwise through shared memory (the rings are free now):
-  // warps [h, 2h) hand their fragments to warps [0, h), lane-major slots
+  // warps merged as a tree through shared memory (the rings are free now):
+  // of the cnt warps still holding a partial, warps [h, cnt) hand their
+  // fragments to warps [0, cnt - h), h = ceil(cnt / 2); lane-major slots
   float* slots = reinterpret_cast<float*>(smem);
 #pragma unroll 1
-  for (int half = kAttWarps / 2; half >= 1; half >>= 1) {
+  for (int cnt = kAttWarps; cnt > 1;) {
+    const int h = (cnt + 1) / 2;
     __syncthreads();
-    if (warp >= half && warp < 2 * half) {
-      float* sl = slots + (warp - half) * kAttSlot;
+    if (warp >= h && warp < cnt) {
+      float* sl = slots + (warp - h) * kAttSlot;
 #pragma unroll
       for (int n = 0; n < 16; ++n)
 #pragma unroll
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
       sl[67 * 32 + lane] = l1;
     }
     __syncthreads();
-    if (warp < half) {
+    if (warp < cnt - h) {
       const float* sl = slots + warp * kAttSlot;
       const float pm0 = sl[64 * 32 + lane], pm1 = sl[65 * 32 + lane];
       const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
       m0 = n0;
       m1 = n1;
     }
+    cnt = h;
   }
   // warp 0: the CTA's partial (m, l, o) to the workspace
   float* pp = p.part + ((int64_t)row * p.splits + split) * kAttPartStride;
