@@ -224,6 +224,12 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned
  *            (required whichever plan runs); its contents need no
  *            initialisation and are scratch.
+ *  Ordering: the kernels of a plan follow one another with programmatic
+ *  dependent launch, but every read of q, the cache and the workspace
+ *  happens after all work issued earlier on the stream has completed (the
+ *  staged plan starts with a memset; the other plans wait on the preceding
+ *  grid before reading); only L2 prefetch hints of the sketch may run
+ *  earlier.
  *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;
  *  FASA_ERR_WORKSPACE if the workspace is missing or too small;
  *  FASA_ERR_UNSUPPORTED if fasa_set_decode_path forced FASA_DECODE_FUSED on a
