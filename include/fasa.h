@@ -196,10 +196,10 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
 /*
  * One FASA decode step over a layer: TIP (fasa_score) -> T_t
  * (fasa_select_topk with k) -> FAC (fasa_sparse_attend), with results equal
- * to those three calls in sequence. Two launch plans compute it:
+ * to those three calls in sequence. Three launch plans compute it:
  *
- *  FASA_DECODE_FUSED  (bf16 caches whose rows fit; chosen when
- *    B * Hkv * C stays within about two CTAs per SM) one launch, one
+ *  FASA_DECODE_FUSED  (bf16 caches whose rows fit; chosen when the
+ *    clusters of all B * Hkv rows fit in at most two waves) one launch, one
  *    thread-block cluster of C <= 16 CTAs per (batch, KV head) row: each CTA
  *    scores its share of the row into shared memory, the cluster runs an
  *    exact radix select of the k-th key over distributed shared memory, each

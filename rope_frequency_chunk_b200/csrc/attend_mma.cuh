@@ -6,9 +6,10 @@
 // rotated at append).
 //
 // Layout of the work: grid = (splits, rows); a CTA takes a contiguous slice
-// of the row's kept list and its 4 warps take 16-row chunks of it in turn.
-// Each warp gathers its chunks' K and V rows with 16-byte cp.async into its
-// own 3-stage ring (no block barriers in the main loop; 16-byte chunks
+// of the row's kept list and its 3 warps take 16-row chunks of it in turn
+// (four CTAs per SM at G <= 8). Each warp gathers its chunks' K and V rows
+// with 16-byte cp.async into its own 2-stage ring (no block barriers in the
+// main loop; 16-byte chunks
 // XOR-swizzled by row so ldmatrix reads are bank-conflict-free) and runs
 // mma.sync.m16n8k16 (bf16 in, float32 accumulate):
 //   S[16 x 16] = Q[16 x 128] K^T   (M = the group's query heads padded to 16,
@@ -16,11 +17,11 @@
 //   O[16 x 128] += P[16 x 16] V     (K = 16 rows, N = head dim)
 // with an online base-2 softmax in registers (the 1/sqrt(128) and log2(e)
 // scale folded into Q). Q is split into three bf16 terms (about 24 bits, as
-// float32), prepared once per row by the selection kernel and read here with
+// float32), prepared once per row by the filter kernel and read here with
 // ldmatrix; each term accumulates in its own registers so the three MMA
 // chains run side by side. P is split into two terms (P is in [0, 1] and only
 // weights V); K and V are bf16 already and enter exactly. The warps of a CTA
-// are merged pairwise through shared memory; the CTA writes its partial
+// are merged as a tree through shared memory; the CTA writes its partial
 // (m, l, o) to the workspace and the row's last CTA (atomic counter) merges
 // the splits and writes the bf16 output.
 #pragma once
