@@ -516,6 +516,86 @@ def run_calibrate(args, wl):
     return 0
 
 
+def run_sweep(args, wl):
+    """The long-CoT sweep: for each dominant-set size, contexts grow from
+    1K to 32K tokens in 1K appends (fasa_append_kv); after each append one
+    decode at the new length with the 18.9% budget. Both are timed with
+    events per step (median of `--sweep-reps` repetitions, L2 flushed before
+    each by writing a buffer larger than L2; re-appending a chunk rewrites the
+    same slots with the same values)."""
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+    torch.cuda.set_device(0)
+    chunk, steps = W.C4_APPEND_CHUNK, W.C4_STEPS
+    L_max = chunk * steps
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    reps = max(3, args.sweep_reps)
+    result = {}
+    hbm_peak, peak_kind = peaks()
+    with ClockSampler(0) as clk:
+        for n_dom in W.C4_NDOMS:
+            w = wl.replace(ctx_len=L_max, n_dom=n_dom)
+            inp = W.layer_inputs(w, layer=0, n_dom=n_dom)
+            cache = F.KVCache(w.batch, w.n_q_heads, w.n_kv_heads, n_dom, L_max, w.dtype, w.rope_base,
+                              inp.params.dom_idx)
+            k_all = W.to_torch(inp.k, "cuda")
+            v_all = W.to_torch(inp.v, "cuda")
+            q = W.to_torch(inp.q, "cuda")
+            out = torch.empty_like(q)
+            ws = torch.empty(F.fasa_decode_workspace_bytes(cache, L_max, W.c4_budget(L_max)), dtype=torch.uint8,
+                             device="cuda")
+            rows = []
+            for st in range(steps):
+                pos0, L = st * chunk, (st + 1) * chunk
+                kn = k_all[:, :, pos0:L].contiguous()
+                vn = v_all[:, :, pos0:L].contiguous()
+                k = W.c4_budget(L)
+
+                def timed(fn):
+                    ts = []
+                    for _ in range(reps):
+                        flush.fill_(1.0)
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        fn()
+                        e1.record()
+                        torch.cuda.synchronize()
+                        ts.append(e0.elapsed_time(e1) * 1e3)
+                    return float(np.median(ts))
+
+                t_app = timed(lambda: F.fasa_append_kv(cache, kn, vn, pos0))
+                for _ in range(args.warmup):
+                    F.fasa_decode(cache, L, q, L, k, out=out, workspace=ws)
+                t_dec = timed(lambda: F.fasa_decode(cache, L, q, L, k, out=out, workspace=ws))
+                alg = roofline_bytes(w.replace(ctx_len=L, k=k), k)
+                rows.append({"L": L, "k": k, "append_us": t_app, "decode_us": t_dec,
+                             "decode_gbs": alg / (t_dec * 1e-6) / 1e9,
+                             "plan": int(F.fasa_decode_path(cache, L, k))})
+            status = F.fasa_device_status(clear=True)
+            if status != 0:
+                raise RuntimeError(f"device status {status} in the sweep")
+            result[str(n_dom)] = rows
+            del cache, k_all, v_all, ws
+    per_step = {nd: float(np.mean([r["append_us"] + r["decode_us"] for r in rows])) for nd, rows in result.items()}
+    last = {nd: rows[-1] for nd, rows in result.items()}
+    line = {
+        "metric": "c4 long-CoT sweep: append + decode us per step (1K..32K in 1K appends), mean over steps",
+        "value": per_step["16"], "unit": "us", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "c4 sweep", "batch": wl.batch, "heads": f"{wl.n_q_heads}/{wl.n_kv_heads}",
+                   "n_dom": list(W.C4_NDOMS), "budget": "18.9% of L", "reps": reps,
+                   "l2": "flushed before every timed call (a write of twice the L2 size)"},
+        "mean_us_per_step": per_step,
+        "at_32k": {nd: {"decode_us": r["decode_us"], "decode_gbs": r["decode_gbs"],
+                        "frac": r["decode_gbs"] / hbm_peak, "append_us": r["append_us"], "plan": r["plan"]}
+                   for nd, r in last.items()},
+        "peak": hbm_peak, "peak_kind": peak_kind, "steps_detail": result, "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -535,6 +615,9 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--calibrate", action="store_true",
                     help="time the offline FC calibration on one layer of the workload instead of the decode")
     ap.add_argument("--cal-win", type=int, default=8, help="calibration queries per sequence (--calibrate)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the c4 long-CoT sweep: append + decode timed per step for every dominant-set size")
+    ap.add_argument("--sweep-reps", type=int, default=5)
     return ap
 
 
@@ -553,6 +636,8 @@ def main(argv=None):
         return run_reference(args, wl)
     if args.calibrate:
         return run_calibrate(args, wl)
+    if args.sweep:
+        return run_sweep(args, W.CONFIGS["c4"])
     return run_fasa(args, wl)
 
 
