@@ -93,21 +93,22 @@ def workload_sig(wl: W.Workload, k: int) -> str:
     return f"{wl.name}-B{wl.batch}-H{wl.n_q_heads}/{wl.n_kv_heads}-L{wl.ctx_len}-n{wl.n_dom}-k{k}-{wl.dtype}"
 
 
-def profiled_traffic(summary: str, workload: str):
-    """DRAM bytes per launch (read + write) that an ncu capture recorded for
-    the dominant kernel on this workload, or None: the summary under profiles/
-    carries one machine-readable line, and its figure holds only while the
-    library's sources are byte-identical to those captured."""
-    import re
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) of `kernel` on this workload from
+    the ncu record in profiles/traffic.json, or None: a figure holds only
+    while the library's sources hash to the digest it was captured under."""
     try:
-        with open(os.path.join(ROOT, "profiles", summary)) as f:
-            text = f.read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    m = re.search(r"<!-- traffic workload=(\S+) bytes_per_launch=(\d+) csrc_sha256=([0-9a-f]{64}) -->", text)
-    if not m or m.group(1) != workload or m.group(3) != csrc_sha256():
+    e = rec.get(f"{kernel}@{workload}")
+    if not e or e.get("csrc_sha256") != csrc_sha256():
         return None
-    return int(m.group(2))
+    return int(e["bytes_per_launch"])
 
 
 # ------------------------------------------------------------- clocks
@@ -253,9 +254,11 @@ def build_stack(wl, n_layers, device):
     return caches, qs
 
 
-def time_graph(fn, steps, warmup, stream, dist=None):
+def time_graph(fn, steps, warmup, stream, dist=None, per_step=None):
     """Capture fn() (one step) in a CUDA graph; replay warmup + steps; return
-    device ms for the steps (events on the replay stream), max over ranks."""
+    device ms for the steps (events on the replay stream), max over ranks.
+    With a list `per_step`, also appends each step's device ms (an event
+    between consecutive replays)."""
     import torch
     with torch.cuda.stream(stream):
         for _ in range(max(1, warmup)):
@@ -270,15 +273,16 @@ def time_graph(fn, steps, warmup, stream, dist=None):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps):
+        ev[0].record(stream)
+        for i in range(steps):
             g.replay()
-        e1.record(stream)
+            ev[i + 1].record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, "cuda")
+    if per_step is not None:
+        per_step.extend(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
     torch.cuda.synchronize()
     del g
     return ms
@@ -325,7 +329,7 @@ def run_fasa(args, wl):
     n_layers = args.layers or default_layers(wl)
     caches, qs = build_stack(wl, n_layers, device)
     outs = [torch.empty_like(q) for q in qs]
-    ws = torch.empty(max(F.fasa_decode_workspace_bytes(c, wl.ctx_len, k) for c in caches), dtype=torch.uint8,
+    ws = torch.zeros(max(F.fasa_decode_workspace_bytes(c, wl.ctx_len, k) for c in caches), dtype=torch.uint8,
                      device=device)
     stream = torch.cuda.Stream(device=device)
     L = wl.ctx_len
@@ -345,9 +349,11 @@ def run_fasa(args, wl):
             F.fasa_dense_decode(c, L, q, wl.q_pos, out=o)
 
     plan = F.fasa_decode_path(caches[0], L, k)
+    launches = F.fasa_decode_launches(caches[0], L, k)
     hbm_peak, peak_kind = peaks()
+    step_ms = []
     with ClockSampler(local) as clk:
-        ms = time_graph(decode_step, args.steps, args.warmup, stream, dist)
+        ms = time_graph(decode_step, args.steps, args.warmup, stream, dist, per_step=step_ms)
     clocks = clk.summary()
     status = F.fasa_device_status(clear=True)
     if status != 0:
@@ -358,23 +364,25 @@ def run_fasa(args, wl):
     ms_step = ms / args.steps
     us_layer = 1e3 * ms_step / n_layers
     gbs = job_gbs(step_bytes, ms_step, world)
+    us_dist = {f"p{q}": float(np.percentile(step_ms, q)) * 1e3 / n_layers for q in (10, 50, 90)}
 
-    # dominant kernel: the single-launch decode is the whole step; the staged
-    # plan's is the TIP score stream, timed alone on the same stack
+    # the roofline is the whole decode of a layer (all of its launches,
+    # back to back in the replayed graph); for the fused plan with one
+    # launch per layer that is the fused kernel itself
     fused = plan == F.DECODE_FUSED
-    if fused:
-        roof = {"bound": "hbm", "kernel": "decode_fused_kernel (score + select + attend, one launch per layer)",
-                "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / world / hbm_peak,
-                "traffic": profiled_traffic("decode_fused_kernel_c2.md", workload_sig(wl, k)),
-                "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind,
-                "us_per_launch": us_layer}
-    else:
+    kern = {1: "decode_wide_kernel (score + select + attend, one launch per layer)",
+            2: "decode_wide_kernel + attend_mma_kernel (two launches per layer)",
+            4: "score_kernel + filter_kernel + finalize_kernel + attend (four launches per layer)"}[launches]
+    roof = {"bound": "hbm", "kernel": kern, "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
+            "frac": gbs / world / hbm_peak,
+            "traffic": profiled_traffic("decode_wide_kernel", workload_sig(wl, k)) if launches == 1 else None,
+            "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind, "us_per_launch": us_layer,
+            "us_per_layer_percentiles": us_dist}
+    if not fused:
         ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
         score_gbs = sketch_bytes(wl) * n_layers / (ms_score * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "score_kernel (TIP sketch stream)", "achieved": score_gbs,
-                "peak": hbm_peak, "unit": "GB/s", "frac": score_gbs / hbm_peak,
-                "traffic": None, "bytes_per_launch": sketch_bytes(wl), "peak_kind": peak_kind,
-                "us_per_launch": 1e3 * ms_score / n_layers}
+        roof["score_kernel"] = {"achieved": score_gbs, "frac": score_gbs / hbm_peak,
+                                "bytes_per_launch": sketch_bytes(wl), "us_per_launch": 1e3 * ms_score / n_layers}
 
     extra = {}
     if not args.no_dense:
@@ -414,16 +422,17 @@ def run_fasa(args, wl):
                    "l2": f"inputs larger than L2: {n_layers} layer caches "
                          f"({step_bytes / 2**20:.0f} MiB of roofline bytes per step) stepped in order"},
         "us_per_layer_step": us_layer,
+        "us_per_layer_step_percentiles": us_dist,
         "tokens_per_s": world * wl.batch / (us_layer * 1e-6),
         "decode_roofline": {"achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
                             "frac": gbs / world / hbm_peak, "bytes_per_layer_step": per_layer_bytes,
                             "peak_kind": peak_kind},
         "roofline": roof,
-        "decode_plan": {F.DECODE_FUSED: "fused", F.DECODE_SCORED: "scored"}.get(plan, "staged"),
+        "decode_plan": "fused" if fused else "staged",
         "clocks": clocks,
-        # kernels of this library per layer: fused 1; scored 2 (score stream, cluster select + attend);
-        # staged 4 (score, filter, finalize, attend)
-        "gpu_launches": {F.DECODE_FUSED: 1, F.DECODE_SCORED: 2}.get(plan, 4) * n_layers * args.steps,
+        # kernels of this library per layer (fasa_decode_launches): fused 1, or 2 with the split-K
+        # attention; staged 4 (score, filter, finalize, attend)
+        "gpu_launches": launches * n_layers * args.steps,
         "e2e": e2e,
     }
     line.update(extra)
@@ -542,7 +551,7 @@ def run_sweep(args, wl):
             v_all = W.to_torch(inp.v, "cuda")
             q = W.to_torch(inp.q, "cuda")
             out = torch.empty_like(q)
-            ws = torch.empty(F.fasa_decode_workspace_bytes(cache, L_max, W.c4_budget(L_max)), dtype=torch.uint8,
+            ws = torch.zeros(F.fasa_decode_workspace_bytes(cache, L_max, W.c4_budget(L_max)), dtype=torch.uint8,
                              device="cuda")
             rows = []
             for st in range(steps):

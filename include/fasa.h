@@ -151,7 +151,10 @@ fasa_status fasa_append_kv(const fasa_cache* cache, const void* k_new, const voi
  *
  *  q      : [B][Hq][128] dtype, pre-RoPE queries.
  *  scores : [B][Hkv][len] float32 (row stride len).
- *  Arithmetic: query rotation and the sum in float64, rounded once to float32.
+ *  Arithmetic: the query rotation and the group sum of each sketch column's
+ *  coefficient c_j in float64, rounded once to float32; the score is then a
+ *  float32 sum of products in a fixed order (the same in every plan of
+ *  fasa_decode), with |error| < 13.01 * 2^-24 * sum_j |c_j| |sketch_j|.
  *  len may be 0 (nothing is written). Errors: FASA_ERR_CAPACITY if
  *  len > max_len.
  */
@@ -196,20 +199,16 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
 /*
  * One FASA decode step over a layer: TIP (fasa_score) -> T_t
  * (fasa_select_topk with k) -> FAC (fasa_sparse_attend), with results equal
- * to those three calls in sequence. Three launch plans compute it:
+ * to those three calls in sequence (the same float32 scores, hence the same
+ * kept set). Two launch plans compute it:
  *
- *  FASA_DECODE_FUSED  (bf16 caches whose rows fit; chosen when the
- *    clusters of all B * Hkv rows fit in at most two waves) one launch, one
- *    thread-block cluster of C <= 16 CTAs per (batch, KV head) row: each CTA
- *    scores its share of the row into shared memory, the cluster runs an
- *    exact radix select of the k-th key over distributed shared memory, each
- *    CTA attends its kept rows, and the partials are merged in the cluster.
- *    The workspace is not touched.
- *  FASA_DECODE_SCORED  (bf16 caches whose rows fit 16 CTAs of 16384 tokens,
- *    within about two waves of clusters when not forced) two launches: the
- *    score stream writes the TIP scores to the workspace, then the same
- *    cluster kernel as FASA_DECODE_FUSED reads them (from L2) instead of the
- *    sketch and selects and attends.
+ *  FASA_DECODE_FUSED  (bf16 caches) each (batch, KV head) row is spread over
+ *    about (SM count / rows) independent CTAs. Each scores its share of the
+ *    sketch in registers, keeps its own top-k candidates and publishes them
+ *    to the workspace; the row's last CTA to finish (an atomic ticket, no
+ *    waiting) selects the exact top-k of the union and, for k_eff <= 512,
+ *    attends those rows itself: one launch. Larger budgets add a split-K
+ *    attention launch over the kept list.
  *  FASA_DECODE_STAGED  four launches chained with programmatic dependent
  *    launch: the score stream, which also builds a per-row histogram of the
  *    score keys; a filter that marks the certainly-kept tokens and collects
@@ -222,14 +221,22 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *            ascending order.
  *  workspace : caller-owned device memory of at least
  *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned
- *            (required whichever plan runs); its contents need no
- *            initialisation and are scratch.
+ *            (required whichever plan runs). Zero it once after allocating it
+ *            (e.g. cudaMemsetAsync): its first 12 * B * Hkv bytes hold
+ *            per-row semaphores that must be zero when a call starts, and
+ *            every call leaves them zero again. The rest is scratch. After a
+ *            call that ended in an error (a CUDA error, FASA_ERR_TIMEOUT),
+ *            zero it again. A semaphore found non-zero is reported as
+ *            FASA_ERR_WORKSPACE in the device status word; no access then
+ *            leaves the workspace.
  *  Ordering: the kernels of a plan follow one another with programmatic
  *  dependent launch, but every read of q, the cache and the workspace
  *  happens after all work issued earlier on the stream has completed (the
- *  staged plan starts with a memset; the other plans wait on the preceding
+ *  staged plan starts with a memset; the fused plan waits on the preceding
  *  grid before reading); only L2 prefetch hints of the sketch may run
  *  earlier.
+ *  Calls that overlap on the GPU (different streams) must not share a
+ *  workspace.
  *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;
  *  FASA_ERR_WORKSPACE if the workspace is missing or too small;
  *  FASA_ERR_UNSUPPORTED if fasa_set_decode_path forced FASA_DECODE_FUSED on a
@@ -241,18 +248,23 @@ fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int
 
 /* Launch plan of fasa_decode (library code, no counterpart in the paper). */
 #define FASA_DECODE_AUTO 0   /* chosen from the shape (default) */
-#define FASA_DECODE_FUSED 1  /* single-launch cluster decode */
+#define FASA_DECODE_FUSED 1  /* row-split decode: one launch (two for k_eff > 512) */
 #define FASA_DECODE_STAGED 2 /* four-launch decode */
-#define FASA_DECODE_SCORED 3 /* two launches: the score stream, then the cluster select + attend */
 
 /* Sets the plan every later fasa_decode call of this process uses (a
  * process-wide setting; FASA_ERR_INVALID_ARG for an unknown value). */
 fasa_status fasa_set_decode_path(int32_t path);
 
 /* The plan fasa_decode would run for this cache, len and k under the current
- * setting and on the current device: FASA_DECODE_FUSED, FASA_DECODE_SCORED or
- * FASA_DECODE_STAGED, or a negative fasa_status for invalid arguments. */
+ * setting and on the current device: FASA_DECODE_FUSED or FASA_DECODE_STAGED,
+ * or a negative fasa_status for invalid arguments. */
 int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
+
+/* Kernels of this library one fasa_decode call launches for this cache, len
+ * and k under the current setting (the fused plan: 1, or 2 when the budget
+ * needs the split-K attention; the staged plan: 4), or a negative
+ * fasa_status for invalid arguments. */
+int32_t fasa_decode_launches(const fasa_cache* cache, int32_t len, int32_t k);
 
 /* Size of the library's own device scratch used by
  * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the
@@ -278,6 +290,9 @@ int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
  *    contents behind; calls whose kernels overlap on the GPU (different
  *    streams, or different host threads) race on it and give wrong results.
  *    Serialize them, e.g. on one stream.
+ *  - Each call clears the array's per-row semaphores (a cudaMemsetAsync of
+ *    12 * B * Hkv bytes on `stream`) before its kernels, so a call that
+ *    ended in an error does not affect the next one.
  *  - Rejects a call needing more than FASA_STATIC_SCRATCH_BYTES of scratch
  *    (fasa_decode_workspace_bytes(cache, len, k)) with FASA_ERR_WORKSPACE,
  *    before launching anything.

@@ -1,0 +1,599 @@
+// Fused decode for bf16 caches: each (batch, KV head) row is spread over
+// n_split independent CTAs, so a layer fills the GPU whatever its row count.
+//
+// "FASA: Frequency-aware Sparse Attention" (gist.science technical summary,
+// §2): TIP scores from the dominant FCs only ("online prediction", a proxy at
+// no significant compute cost), the critical set T_t = the k highest-scoring
+// tokens (ties to the lower index, k_eff = min(k, L)), then full softmax
+// attention of every query head of the group over exactly those rows at
+// their original positions (FAC).
+//
+// Grid n_split x rows, 512 threads, no clusters. CTA s of a row owns the
+// tokens [s*n_loc, (s+1)*n_loc). Every CTA:
+//  1. prefetches its sketch range into L2 (a hint, issued before the wait on
+//     the preceding grid, so a layer's stream overlaps the previous layer's
+//     tail), waits, then forms the float32 TIP coefficients of its group
+//     (tip.cuh);
+//  2. streams its sketch rows straight into registers with 16-byte loads
+//     (one token per lane, 2 or 4 lanes for wide rows), scores them in
+//     float32 and keeps each score's order-preserving key in shared memory,
+//     with a 4096-bin histogram of the top 12 key bits;
+//  3. finds the bin b_loc holding its own k_eff-th key and publishes every
+//     token in bins >= b_loc as a (key, token) pair: a token of the row's top
+//     k_eff is in its CTA's top k_eff, so the published union holds the row's
+//     whole critical set, and every token of the row in a bin at or above the
+//     row's boundary bin (which is >= every b_loc);
+//  4. takes a ticket on the row's semaphore word; the last CTA of the row to
+//     arrive (no CTA ever waits on another) resolves the row:
+//      - a histogram of the union gives the boundary bin B and the count
+//        above it (exact: the union holds every token of bins >= B);
+//      - tokens above B are kept; among the tokens of B the need largest keys
+//        are kept, ties to the lower token index (rank counting for a few,
+//        else an exact radix select);
+//      - a bitmap of the kept tokens emits them in ascending order;
+//      - with `direct` the same CTA attends them on tensor cores (mma.sync,
+//        the split-K kernel's per-warp chunk step, one chunk per warp at a
+//        time) and merges its warps; otherwise it writes the kept list and
+//        the query terms for attend_mma_kernel, launched next.
+//
+// Semaphore: sem[row] = (tickets << 32) | entries reserved. It must be zero
+// when a call starts; the last CTA of the row writes it back to zero, so a
+// workspace zeroed once stays valid. A ticket or reservation beyond its
+// range (a workspace that was not zero) is flagged FASA_ERR_WORKSPACE and
+// never written out of bounds.
+#pragma once
+
+#include "attend_mma.cuh"
+#include "select_attend.cuh"
+#include "tip.cuh"
+
+namespace fasa {
+
+constexpr int kWdThreads = kSAThreads;  // 512 (the histogram and radix helpers' block size)
+constexpr int kWdWarps = kWdThreads / 32;
+constexpr int kWdMaxLoc = 16384;        // tokens per CTA (their keys live in shared memory)
+constexpr int kWdTieCap = 2048;         // boundary-bin entries held in shared memory
+constexpr int kWdRankMax = 512;         // boundary-bin entries resolved by rank counting
+constexpr int kWdMaxDirect = 512;       // kept rows the resolving CTA attends itself
+constexpr int kWdRadixWords = kSAWarps * 256 + 256 + 8;
+constexpr int kWdMisc = 128;            // words of scan and flag scratch
+
+struct WideParams {
+  const __nv_bfloat16* sketch;  // [rows][max_len][stride]
+  const __nv_bfloat16* k;       // [rows][max_len][128], rotated
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* q;       // [B][Hq][128], pre-RoPE
+  const int32_t* dom_idx;       // [Hkv][n_dom]
+  __nv_bfloat16* out;           // [B][Hq][128]
+  int32_t* idx_out;             // [rows][n_keep] kept tokens, ascending, or null
+  int32_t* idx_ws;              // [rows][n_keep] for the attention launch, or null (direct)
+  unsigned char* qterms;        // [rows][kQTermBytes] for the attention launch, or null (direct)
+  uint2* cand;                  // [rows][len] published (key, token) pairs
+  unsigned long long* sem;      // [rows], zero between calls
+  int64_t max_len;
+  int32_t len;
+  int32_t stride;
+  int32_t n_kv_heads;
+  int32_t group;
+  int32_t n_dom;
+  int32_t n_keep;   // k_eff, 1 .. len
+  int32_t n_loc;    // tokens per CTA, <= kWdMaxLoc
+  int32_t n_split;  // CTAs per row
+  int32_t ucache;   // union entries the resolving CTA caches in shared memory
+  int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect)
+  double cosv[kNFC];
+  double sinv[kNFC];
+};
+
+__host__ __device__ constexpr int wd_al(int x, int a) { return (x + a - 1) / a * a; }
+
+// Shared-memory layout. r1 is reused: the CTA's keys (steps 1-3); then, in
+// the resolving CTA, the bitmap, boundary-bin entries, radix scratch and the
+// cached union; then the attention's query terms and K/V ring.
+struct WdLayout {
+  int hist, misc, coef, qraw, dom, kept, r1, bitmap, ties, rscr, ucache, qt, ring, total;
+};
+__host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, int direct, int group, int ucache) {
+  WdLayout L;
+  int o = 0;
+  L.hist = o;
+  o += 4096 * 4;
+  L.misc = o;
+  o += kWdMisc * 4;
+  L.coef = o;
+  o += kD * 4;
+  L.qraw = o;
+  o += FASA_MAX_GROUP * kD * 2;
+  L.dom = o;
+  o += kNFC * 4;
+  L.kept = o;
+  o += wd_al(direct ? n_keep * 4 : 0, 128);
+  L.r1 = o;
+  const int a = n_loc * 4;
+  L.bitmap = o;
+  int b = wd_al((len + 31) / 32 * 4, 16);
+  L.ties = o + b;
+  b += kWdTieCap * 8;
+  L.rscr = o + b;
+  b += wd_al(kWdRadixWords * 4, 16);
+  L.ucache = o + b;
+  b += ucache * 8;
+  L.qt = o;
+  int c = 0;
+  if (direct) {
+    c = wd_al((3 * group + 1) * 256, 128);
+    L.ring = o + c;
+    c += kWdWarps * kAttStageBytes;
+  } else {
+    L.ring = o;
+  }
+  L.total = o + (a > b ? (a > c ? a : c) : (b > c ? b : c));
+  return L;
+}
+
+// Exclusive scan of one value per thread over the 512 threads; returns the
+// thread's offset and, in *total, the sum. scr: 17 words. Ends synchronized.
+__device__ __forceinline__ uint32_t wd_block_scan(uint32_t v, uint32_t* scr, uint32_t* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  if (lane == 31) scr[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < kWdWarps ? scr[lane] : 0u;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, w, off);
+      if (lane >= off) w += x;
+    }
+    if (lane < kWdWarps) scr[lane] = w;  // inclusive warp sums
+  }
+  __syncthreads();
+  const uint32_t before = warp > 0 ? scr[warp - 1] : 0u;
+  *total = scr[kWdWarps - 1];
+  __syncthreads();
+  return before + incl - v;
+}
+
+__device__ __forceinline__ void wd_keep(uint32_t* bm, uint32_t t, int len) {
+  if (t < (uint32_t)len) atomicOr(bm + (t >> 5), 1u << (t & 31));
+}
+
+// Exact choice of the `need` largest keys among the entries of bin B (ties to
+// the lower token index), by two radix selects: the need-th key K, then, if
+// only some of the keys equal to K fit, the lowest token indices among them.
+// entry_at(i) gives entry i of n (any entries; only bin B's take part).
+template <typename At>
+__device__ void wd_resolve_radix(At entry_at, int n, int need, uint32_t B, uint32_t* rscr, uint32_t* misc,
+                                 uint32_t* bm, int len) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int tid = threadIdx.x;
+  uint32_t K = 0;
+  int krem = 0;
+  ballot_radix_fn<false>([&](int i) { return entry_at(i).x; }, n, need, B << 20, 12, 32, rscr, nullptr, cl, K, krem);
+  // keys above K in bin B are kept; count the keys equal to K
+  if (tid == 0) misc[0] = 0u;
+  __syncthreads();
+  for (int i = tid; i < n; i += kWdThreads) {
+    const uint2 e = entry_at(i);
+    if ((e.x >> 20) == B && e.x > K) wd_keep(bm, e.y, len);
+    if (e.x == K) atomicAdd(misc, 1u);
+  }
+  __syncthreads();
+  const int n_eq = (int)misc[0];
+  __syncthreads();
+  if (krem >= n_eq) {
+    for (int i = tid; i < n; i += kWdThreads) {
+      const uint2 e = entry_at(i);
+      if (e.x == K) wd_keep(bm, e.y, len);
+    }
+    return;
+  }
+  // the krem lowest indices among the keys equal to K: select the largest ~t
+  // (token indices are below 2^19, so ~t has its top 13 bits set)
+  uint32_t T = 0;
+  int trem = 0;
+  ballot_radix_fn<false>([&](int i) {
+    const uint2 e = entry_at(i);
+    return e.x == K ? ~e.y : 0u;
+  }, n, krem, 0xFFF80000u, 13, 32, rscr, nullptr, cl, T, trem);
+  for (int i = tid; i < n; i += kWdThreads) {
+    const uint2 e = entry_at(i);
+    if (e.x == K && ~e.y >= T) wd_keep(bm, e.y, len);
+  }
+}
+
+// Softmax attention of the group's query heads over the n kept rows in
+// `kept` (shared memory, ascending), one 16-row chunk per warp at a time,
+// the warps merged as a tree; writes out[h][d] for the G heads.
+__device__ void wd_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, const int* kept, int n,
+                          const unsigned char* qt, int G, unsigned char* ring, __nv_bfloat16* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned char* st = ring + warp * kAttStageBytes;
+  const int nchunks = (n + kAttChunk - 1) / kAttChunk;
+  float o[16][4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[j][e] = 0.0f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // heads lane/4 and lane/4 + 8
+  for (int ci = warp; ci < nchunks; ci += kWdWarps) {
+    const int j0 = ci * kAttChunk;
+    const int tr = (lane < kAttChunk && j0 + lane < n) ? kept[j0 + lane] : 0;
+#pragma unroll
+    for (int r = 0; r < kAttChunk; ++r) {  // 16 rows x (16 K + 16 V) 16-byte parts, one part per lane
+      const int t = __shfl_sync(0xFFFFFFFFu, tr, r);
+      const __nv_bfloat16* src = (lane < 16 ? kb : vb) + (int64_t)t * kD + (lane % 16) * 8;
+      cp_async16(st + (lane < 16 ? 0 : kAttHalf) + r * 256 + (((lane % 16) ^ (r & 7)) * 16), src);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+    const unsigned char* Ks = st;
+    const unsigned char* Vs = st + kAttHalf;
+    float s0[4], s1[4];
+    chunk_logits(qt, G, Ks, lane, s0, s1);
+    const int c0 = (lane % 4) * 2;
+    if (j0 + c0 >= n) s0[0] = s0[2] = -INFINITY;
+    if (j0 + c0 + 1 >= n) s0[1] = s0[3] = -INFINITY;
+    if (j0 + 8 + c0 >= n) s1[0] = s1[2] = -INFINITY;
+    if (j0 + 8 + c0 + 1 >= n) s1[1] = s1[3] = -INFINITY;
+    float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
+    float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float sc0 = (m0 == -INFINITY) ? 0.0f : exp2f(m0 - n0);
+    const float sc1 = (m1 == -INFINITY) ? 0.0f : exp2f(m1 - n1);
+    float pr[8];
+    pr[0] = s0[0] == -INFINITY ? 0.f : exp2f(s0[0] - n0);
+    pr[1] = s0[1] == -INFINITY ? 0.f : exp2f(s0[1] - n0);
+    pr[2] = s0[2] == -INFINITY ? 0.f : exp2f(s0[2] - n1);
+    pr[3] = s0[3] == -INFINITY ? 0.f : exp2f(s0[3] - n1);
+    pr[4] = s1[0] == -INFINITY ? 0.f : exp2f(s1[0] - n0);
+    pr[5] = s1[1] == -INFINITY ? 0.f : exp2f(s1[1] - n0);
+    pr[6] = s1[2] == -INFINITY ? 0.f : exp2f(s1[2] - n1);
+    pr[7] = s1[3] == -INFINITY ? 0.f : exp2f(s1[3] - n1);
+    l0 = l0 * sc0 + (pr[0] + pr[1] + pr[4] + pr[5]);
+    l1 = l1 * sc1 + (pr[2] + pr[3] + pr[6] + pr[7]);
+    m0 = n0;
+    m1 = n1;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      o[j][0] *= sc0;
+      o[j][1] *= sc0;
+      o[j][2] *= sc1;
+      o[j][3] *= sc1;
+    }
+    uint32_t ph[4], pl[4];
+    split_pack(pr[0], pr[1], ph[0], pl[0]);
+    split_pack(pr[2], pr[3], ph[1], pl[1]);
+    split_pack(pr[4], pr[5], ph[2], pl[2]);
+    split_pack(pr[6], pr[7], ph[3], pl[3]);
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      uint32_t b[4];
+      ldsm_x4_t(b, Vs + (((lane / 8) % 2) * 8 + lane % 8) * 256 + (((j + lane / 16) ^ (lane % 8)) * 16));
+      mma_16816(o[j], ph, b[0], b[1]);
+      mma_16816(o[j], pl, b[0], b[1]);
+      mma_16816(o[j + 1], ph, b[2], b[3]);
+      mma_16816(o[j + 1], pl, b[2], b[3]);
+    }
+    __syncwarp();
+  }
+  // warps merged as a tree in the ring (of the cnt warps still holding a
+  // partial, warps [h, cnt) hand theirs to warps [0, cnt - h))
+  float* slots = reinterpret_cast<float*>(ring);
+#pragma unroll 1
+  for (int cnt = kWdWarps; cnt > 1;) {
+    const int h = (cnt + 1) / 2;
+    __syncthreads();
+    if (warp >= h && warp < cnt) {
+      float* sl = slots + (warp - h) * kAttSlot;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sl[(j * 4 + e) * 32 + lane] = o[j][e];
+      sl[64 * 32 + lane] = m0;
+      sl[65 * 32 + lane] = m1;
+      sl[66 * 32 + lane] = l0;
+      sl[67 * 32 + lane] = l1;
+    }
+    __syncthreads();
+    if (warp < cnt - h) {
+      const float* sl = slots + warp * kAttSlot;
+      const float pm0 = sl[64 * 32 + lane], pm1 = sl[65 * 32 + lane];
+      const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
+      const float a0 = (m0 == -INFINITY) ? 0.0f : exp2f(m0 - n0), a1 = (m1 == -INFINITY) ? 0.0f : exp2f(m1 - n1);
+      const float b0 = (pm0 == -INFINITY) ? 0.0f : exp2f(pm0 - n0), b1 = (pm1 == -INFINITY) ? 0.0f : exp2f(pm1 - n1);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        o[j][0] = o[j][0] * a0 + sl[(j * 4 + 0) * 32 + lane] * b0;
+        o[j][1] = o[j][1] * a0 + sl[(j * 4 + 1) * 32 + lane] * b0;
+        o[j][2] = o[j][2] * a1 + sl[(j * 4 + 2) * 32 + lane] * b1;
+        o[j][3] = o[j][3] * a1 + sl[(j * 4 + 3) * 32 + lane] * b1;
+      }
+      l0 = l0 * a0 + sl[66 * 32 + lane] * b0;
+      l1 = l1 * a1 + sl[67 * 32 + lane] * b1;
+      m0 = n0;
+      m1 = n1;
+    }
+    cnt = h;
+  }
+  if (warp == 0) {
+    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
+    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
+    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
+    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
+    const int h0 = lane / 4, h1 = lane / 4 + 8;
+    const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int d = j * 8 + (lane % 4) * 2;
+      if (h0 < G)
+        *reinterpret_cast<__nv_bfloat162*>(out + h0 * kD + d) = __floats2bfloat162_rn(o[j][0] * i0, o[j][1] * i0);
+      if (h1 < G)
+        *reinterpret_cast<__nv_bfloat162*>(out + h1 * kD + d) = __floats2bfloat162_rn(o[j][2] * i1, o[j][3] * i1);
+    }
+  }
+}
+
+// The attention query terms in the compact shared-memory layout chunk_logits
+// reads: term t (low, middle, high) of head r at row t*G + r, then a zero
+// row at 3G; the values are query_terms' bit for bit.
+__device__ __forceinline__ void wd_query_terms(const __nv_bfloat16* qraw, int G, const double* cosv,
+                                               const double* sinv, unsigned char* qt) {
+  const int tid = threadIdx.x;
+  const double qscale = 1.4426950408889634 / 11.313708498984761;
+  for (int e = tid; e < G * (kD / 2); e += kWdThreads) {
+    const int h = e / (kD / 2), d = 2 * (e % (kD / 2));
+    float v2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int dd = d + u, i = dd & (kNFC - 1);
+      const double x = __bfloat162float(qraw[h * kD + i]);
+      const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
+      const double c = cosv[i], sn = sinv[i];
+      v2[u] = (float)(((dd < kNFC) ? (x * c - y * sn) : (y * c + x * sn)) * qscale);
+    }
+    uint32_t hi, mid, lo;
+    const float2 r = split_pack(v2[0], v2[1], hi, mid);
+    const float2 mf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&mid));
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(r.x - mf.x, r.y - mf.y);
+    lo = *reinterpret_cast<const uint32_t*>(&ll);
+    const int off = (((d / 8) ^ (h & 7)) * 16) + (d % 8) * 2;
+    *reinterpret_cast<uint32_t*>(qt + (0 * G + h) * 256 + off) = lo;
+    *reinterpret_cast<uint32_t*>(qt + (1 * G + h) * 256 + off) = mid;
+    *reinterpret_cast<uint32_t*>(qt + (2 * G + h) * 256 + off) = hi;
+  }
+  if (tid < 16) reinterpret_cast<uint4*>(qt + 3 * G * 256)[tid] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int LPT>
+__global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WideParams p) {
+  using S = TipShape<__nv_bfloat16, LPT>;
+  constexpr int U = S::LPT2 == 1 ? 4 : 2;  // tokens in flight per lane
+  extern __shared__ __align__(128) unsigned char smem[];
+  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.ucache);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + Lo.hist);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lo.misc);
+  float* coef = reinterpret_cast<float*>(smem + Lo.coef);
+  __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem + Lo.qraw);
+  int* s_dom = reinterpret_cast<int*>(smem + Lo.dom);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + Lo.r1);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, row = blockIdx.y;
+  const int t_beg = split * p.n_loc;
+  const int n_tok = max(0, min(p.len - t_beg, p.n_loc));
+  const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t_beg) * S::ROWB;
+  {  // L2 prefetch of this CTA's sketch range: a hint, safe before the wait
+    const int64_t bytes = (int64_t)n_tok * S::ROWB;
+    constexpr int kPf = 8192;
+    for (int64_t o = (int64_t)tid * kPf; o < bytes; o += (int64_t)kWdThreads * kPf)
+      prefetch_l2(src + o, (uint32_t)(bytes - o < kPf ? bytes - o : kPf));
+  }
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  // 1. the group's queries and dominant FCs, the coefficients
+  const int G = p.group;
+  const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
+  {
+    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
+    for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
+    for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+  }
+  __syncthreads();
+  if (tid < p.stride) coef[tid] = tip_coef<__nv_bfloat16>(qraw, s_dom, G, p.n_dom, tid, p.cosv, p.sinv);
+  __syncthreads();
+  const int sub = tid % S::LPT2;  // the lane's chunk group; a token's lanes are adjacent
+  float cr[S::EPL];
+#pragma unroll
+  for (int e = 0; e < S::EPL; ++e) cr[e] = coef[sub * S::EPL + e];
+
+  // 2. score the CTA's tokens straight from global memory
+  constexpr int kTokPass = kWdThreads / S::LPT2;
+  const int my_tok = tid / S::LPT2;
+  for (int base = 0; base < n_tok; base += kTokPass * U) {  // block-uniform trip count
+    uint4 v[U][S::CPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = base + u * kTokPass + my_tok;
+#pragma unroll
+      for (int c = 0; c < S::CPL; ++c)
+        v[u][c] = t < n_tok ? __ldg(reinterpret_cast<const uint4*>(src + (int64_t)t * S::ROWB) + sub * S::CPL + c)
+                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = base + u * kTokPass + my_tok;
+      float part[S::CPL];
+#pragma unroll
+      for (int c = 0; c < S::CPL; ++c) part[c] = tip_chunk(v[u][c], cr + c * 8, __nv_bfloat16());
+      const float sc = tip_lanes_sum<S::LPT2>(tip_lane_sum<S::CPL>(part));
+      if (t < n_tok && sub == 0) {
+        const uint32_t key = score_key(sc);
+        keys[t] = key;
+        atomicAdd(hist + (key >> 20), 1u);
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. the bin holding this CTA's k_eff-th key; publish the tokens at or above it
+  uint32_t b_loc = 0u;
+  if (n_tok > p.n_keep) {
+    uint32_t above = 0u;
+    hist_threshold_fn([&](int i) { return hist[i]; }, p.n_keep, misc, b_loc, above);
+  }
+  uint32_t wc = 0u;
+  for (int i0 = warp * 32; i0 < n_tok; i0 += kWdThreads) {
+    const int i = i0 + lane;
+    wc += __popc(__ballot_sync(0xFFFFFFFFu, i < n_tok && (keys[i] >> 20) >= b_loc));
+  }
+  if (lane == 0) misc[64 + warp] = wc;
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t tot = warp_offsets_serial(misc, 64);
+    uint32_t base = 0u;
+    if (tot) base = (uint32_t)atomicAdd(p.sem + row, (unsigned long long)tot);
+    const bool ok = (uint64_t)base + tot <= (uint64_t)p.len;
+    if (!ok) flag_status(FASA_ERR_WORKSPACE);
+    misc[96] = base;
+    misc[97] = ok ? 1u : 0u;
+  }
+  __syncthreads();
+  uint2* crow = p.cand + (int64_t)row * p.len;
+  if (misc[97]) {
+    uint32_t pos = misc[96] + misc[64 + warp];
+    for (int i0 = warp * 32; i0 < n_tok; i0 += kWdThreads) {
+      const int i = i0 + lane;
+      const uint32_t key = i < n_tok ? keys[i] : 0u;
+      const bool q = i < n_tok && (key >> 20) >= b_loc;
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, q);
+      if (q) crow[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
+      pos += __popc(m);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned long long old = atomicAdd(p.sem + row, 1ull << 32);
+    const uint32_t tk = (uint32_t)(old >> 32);
+    if (tk >= (uint32_t)p.n_split) flag_status(FASA_ERR_WORKSPACE);
+    misc[98] = (tk == (uint32_t)p.n_split - 1) ? 1u : 0u;
+    misc[99] = (uint32_t)old;  // entries reserved by the row's CTAs (all of them, in the last CTA)
+  }
+  __syncthreads();
+  if (!misc[98]) return;
+
+  // 4. the row's last CTA: exact selection over the published union
+  __threadfence();
+  const int nu = (int)min(misc[99], (uint32_t)p.len);
+  const bool cached = nu <= p.ucache;
+  uint2* uc = reinterpret_cast<uint2*>(smem + Lo.ucache);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + Lo.bitmap);
+  uint2* ties = reinterpret_cast<uint2*>(smem + Lo.ties);
+  uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + Lo.rscr);
+  const int words = (p.len + 31) / 32;
+  if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
+  for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+  for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
+  if (tid == 0) misc[100] = 0u;
+  __syncthreads();
+  for (int i = tid; i < nu; i += kWdThreads) {
+    const uint2 e = __ldcg(crow + i);
+    if (cached) uc[i] = e;
+    atomicAdd(hist + (e.x >> 20), 1u);
+  }
+  __syncthreads();
+  int n_keep = p.n_keep;
+  if (nu < n_keep) {  // only a workspace that was not zero gets here
+    if (tid == 0) flag_status(FASA_ERR_WORKSPACE);
+    n_keep = nu;
+  }
+  uint32_t B = 0u, above = 0u;
+  if (n_keep > 0) hist_threshold_fn([&](int i) { return hist[i]; }, n_keep, misc, B, above);
+  for (int i = tid; i < nu; i += kWdThreads) {
+    const uint2 e = cached ? uc[i] : __ldcg(crow + i);
+    const uint32_t b = e.x >> 20;
+    if (b > B) {
+      wd_keep(bm, e.y, p.len);
+    } else if (b == B) {
+      const uint32_t at = atomicAdd(misc + 100, 1u);
+      if (at < (uint32_t)kWdTieCap) ties[at] = e;
+    }
+  }
+  __syncthreads();
+  const int n_b = (int)misc[100];
+  const int need = n_keep - (int)above;
+  __syncthreads();
+  if (need > 0 && n_keep > 0) {
+    if (n_b == need && n_b <= kWdTieCap) {
+      for (int i = tid; i < n_b; i += kWdThreads) wd_keep(bm, ties[i].y, p.len);
+    } else if (n_b <= kWdRankMax) {
+      for (int i = tid; i < n_b; i += kWdThreads) {
+        const uint2 a = ties[i];
+        int r = 0;
+        for (int j = 0; j < n_b; ++j) {
+          const uint2 c = ties[j];
+          r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
+        }
+        if (r < need) wd_keep(bm, a.y, p.len);
+      }
+    } else if (n_b <= kWdTieCap) {
+      wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need, B, rscr, misc, bm, p.len);
+    } else if (cached) {
+      wd_resolve_radix([&](int i) { return uc[i]; }, nu, need, B, rscr, misc, bm, p.len);
+    } else {
+      wd_resolve_radix([&](int i) { return __ldcg(crow + i); }, nu, need, B, rscr, misc, bm, p.len);
+    }
+  }
+  __syncthreads();
+
+  // ascending emission from the bitmap
+  int* kept = reinterpret_cast<int*>(smem + Lo.kept);
+  const int wpt = (words + kWdThreads - 1) / kWdThreads;
+  const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+  uint32_t cnt = 0u;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  uint32_t total = 0u;
+  uint32_t pos = wd_block_scan(cnt, misc, &total);
+  if (tid == 0 && total != (uint32_t)n_keep) flag_status(FASA_ERR_WORKSPACE);
+  int32_t* io = p.idx_out ? p.idx_out + (int64_t)row * p.n_keep : nullptr;
+  int32_t* iw = p.idx_ws ? p.idx_ws + (int64_t)row * p.n_keep : nullptr;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int t = w * 32 + __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < (uint32_t)p.n_keep) {
+        if (p.direct) kept[pos] = t;
+        if (io) io[pos] = t;
+        if (iw) iw[pos] = t;
+      }
+      ++pos;
+    }
+  }
+  __syncthreads();
+  const int n_att = min((int)total, p.n_keep);
+  if (!p.direct) {  // attend_mma_kernel follows: its query terms
+    query_terms(qraw, G, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes, tid, kWdThreads);
+    return;
+  }
+  unsigned char* qt = smem + Lo.qt;
+  wd_query_terms(qraw, G, p.cosv, p.sinv, qt);
+  __syncthreads();
+  wd_attend(p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD, kept, n_att, qt, G,
+            smem + Lo.ring, p.out + (int64_t)row * G * kD);
+}
+
+}  // namespace fasa

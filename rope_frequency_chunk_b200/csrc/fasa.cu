@@ -15,7 +15,7 @@
 #include "select_attend.cuh"
 #include "select_hist.cuh"
 #include "attend_mma.cuh"
-#include "decode_fused.cuh"
+#include "decode_wide.cuh"
 #include "calibrate.cuh"
 
 using namespace fasa;
@@ -337,200 +337,84 @@ fasa_status static_scratch_addr(void** out) {
   return FASA_OK;
 }
 
-// ------------------------------------------------- single-launch decode
+// ------------------------------------------------- wide fused decode
 
 std::atomic<int> g_decode_path{FASA_DECODE_AUTO};
 
-// Launch plan of the single-launch decode.
-struct FusedPlan {
-  int C = 0, n_loc = 0, ring = 0, n_stages = 0, ucap = 0, smem = 0, waves = 0;
+// Launch plan of the wide fused decode (decode_wide.cuh).
+struct WidePlan {
+  int n_split = 0, n_loc = 0, direct = 0, ucache = 0, smem = 0;
 };
 
-template <int LPT, bool kSc>
-fasa_status fused_attrs(const DevInfo& d) {
-  auto kern = decode_fused_kernel<LPT, kSc>;
+template <int LPT>
+fasa_status wide_attrs(const DevInfo& d) {
+  auto kern = decode_wide_kernel<LPT>;
   int set = 0;
   return cached_int((const void*)kern, 0, &set, [&](int* v) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     *v = 1;
-    return cuda_status(e);
+    return cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin));
   });
 }
 
-// Clusters of size C with `smem` bytes per CTA that fit on the GPU at once.
-template <int LPT, bool kSc>
-fasa_status fused_max_clusters(int C, int smem, const DevInfo& d, int* out) {
-  auto kern = decode_fused_kernel<LPT, kSc>;
-  fasa_status s = fused_attrs<LPT, kSc>(d);
-  if (s != FASA_OK) return s;
-  return cached_int((const void*)kern, 3000ull + (uint64_t)C * 1000003ull + (uint64_t)smem, out, [&](int* v) {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)C, 1, 1);
-    cfg.blockDim = dim3(kFuThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    *v = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveClusters(v, kern, &cfg);
-    if (e != cudaSuccess) {
-      (void)cudaGetLastError();
-      *v = 0;  // this cluster size is not available
-    }
-    return FASA_OK;
-  });
-}
-
-// Shape of the cluster decode for cluster size C: tokens per CTA and the ring,
-// which after phase 1 holds the boundary bin's union and later one K+V chunk
-// per warp. Streaming the sketch (kSc false), the ring also holds every
-// score stage in flight when shared memory allows; reading scores (kSc
-// true) it has no stages.
-template <int LPT, bool kSc>
-bool fused_shape(int C, int32_t len, const DevInfo& d, FusedPlan* pl) {
-  constexpr int kStage = fu_stage_bytes<LPT>();
-  constexpr int TPS = kStage / (LPT * 16);
-  pl->C = C;
-  pl->n_loc = (int)(ceil_div(ceil_div(len, C), 32) * 32);
-  if (pl->n_loc > kFuMaxLoc) return false;
-  const int ring_max = (d.smem_optin - fu_layout(pl->n_loc, 0).total) / 128 * 128;
-  if (ring_max < kFuMinRing) return false;
-  if (kSc) {
-    pl->n_stages = 0;
-    pl->ring = kFuMinRing;
-  } else {
-    pl->n_stages =
-        (int)std::min<int64_t>(std::min<int64_t>(kFuMaxStages, ring_max / kStage), ceil_div(pl->n_loc, TPS));
-    if (pl->n_stages < 1) return false;
-    pl->ring = std::max(kFuMinRing, (pl->n_stages * kStage + 127) / 128 * 128);
+// CTAs per row: about one per SM over all rows (never fewer than the
+// shared-memory limit on keys per CTA allows); tokens per CTA. The
+// resolving CTA attends itself for budgets up to kWdMaxDirect when its ring
+// fits, and caches as much of the published union as shared memory allows.
+bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl) {
+  if (c->dtype != FASA_BF16) return false;
+  const int64_t rows = (int64_t)c->batch * c->n_kv_heads;
+  int64_t S = std::max<int64_t>(1, (d.sms + rows / 2) / rows);
+  S = std::max<int64_t>(S, ceil_div(len, kWdMaxLoc));
+  S = std::min<int64_t>(S, std::max<int64_t>(1, ceil_div(len, 256)));
+  pl->n_split = (int)S;
+  pl->n_loc = (int)ceil_div(len, S);
+  if (pl->n_loc > kWdMaxLoc || S > 65535) return false;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  for (int direct = keff <= kWdMaxDirect ? 1 : 0; direct >= 0; --direct) {
+    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, 0);
+    if (base.total > d.smem_optin) continue;
+    // the union cache is the last part of its region: whatever shared memory is left
+    const int64_t uc = std::min<int64_t>(len, std::max<int64_t>(0, (d.smem_optin - base.ucache) / 8));
+    pl->direct = direct;
+    pl->ucache = (int)uc;
+    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->ucache).total;
+    return true;
   }
-  pl->ucap = (pl->ring - kFuRadixBytes) / 8;
-  pl->smem = fu_layout(pl->n_loc, pl->ring).total;
-  return pl->smem <= d.smem_optin;
+  return false;
 }
 
-// Picks the cluster size: fewest waves of clusters first, then the least
-// per-CTA work (a wave costs about a 4096-token CTA of fixed latency; a
-// token read as a score costs an eighth of one streamed as a sketch row).
-// Neither is eligible (false), unless forced, beyond two waves: each wave
-// repeats the kernel's serial select-and-attend chain.
-template <int LPT, bool kSc>
-fasa_status fused_plan_t(int rows, int32_t len, const DevInfo& d, bool forced, FusedPlan* out, bool* ok) {
-  static const int kSizes[] = {16, 15, 14, 13, 12, 10, 8, 6, 4, 3, 2, 1};
-  *ok = false;
-  int64_t best = -1;
-  for (int C : kSizes) {
-    FusedPlan pl;
-    if (!fused_shape<LPT, kSc>(C, len, d, &pl)) continue;
-    int maxc = 0;
-    fasa_status s = fused_max_clusters<LPT, kSc>(C, pl.smem, d, &maxc);
-    if (s != FASA_OK) return s;
-    if (maxc < 1) continue;
-    pl.waves = (int)ceil_div(rows, maxc);
-    const int64_t cost = (int64_t)pl.waves * ((kSc ? pl.n_loc / 8 : pl.n_loc) + 4096);
-    if (best < 0 || cost < best) {
-      best = cost;
-      *out = pl;
-    }
-  }
-  *ok = best >= 0 && (forced || out->waves <= 2);
-  return FASA_OK;
-}
-
-// Plan of the single-launch decode (scored false) or of the cluster decode
-// that reads a score-kernel launch's scores (scored true); bf16 caches only.
-fasa_status fused_plan(const fasa_cache* c, int32_t len, const DevInfo& d, bool forced, bool scored, FusedPlan* out,
-                       bool* ok) {
-  *ok = false;
-  if (c->dtype != FASA_BF16) return FASA_OK;
-  const int rows = c->batch * c->n_kv_heads;
-  if (scored) return fused_plan_t<1, true>(rows, len, d, forced, out, ok);
-  switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
-    case 1: return fused_plan_t<1, false>(rows, len, d, forced, out, ok);
-    case 2: return fused_plan_t<2, false>(rows, len, d, forced, out, ok);
-    case 4: return fused_plan_t<4, false>(rows, len, d, forced, out, ok);
-    case 8: return fused_plan_t<8, false>(rows, len, d, forced, out, ok);
-    case 16: return fused_plan_t<16, false>(rows, len, d, forced, out, ok);
-    default: return FASA_OK;
-  }
-}
-
-template <int LPT, bool kSc>
-fasa_status launch_fused_t(const FusedParams& p, int rows, const FusedPlan& pl, cudaStream_t st, const DevInfo& d) {
-  auto kern = decode_fused_kernel<LPT, kSc>;
-  fasa_status s = fused_attrs<LPT, kSc>(d);
+template <int LPT>
+fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cudaStream_t st, const DevInfo& d) {
+  auto kern = decode_wide_kernel<LPT>;
+  fasa_status s = wide_attrs<LPT>(d);
   if (s != FASA_OK) return s;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attrs[2];
-  cfg.gridDim = dim3((unsigned)pl.C, (unsigned)rows, 1);
-  cfg.blockDim = dim3(kFuThreads, 1, 1);
+  cudaLaunchAttribute attrs[1];
+  cfg.gridDim = dim3((unsigned)pl.n_split, (unsigned)rows, 1);
+  cfg.blockDim = dim3(kWdThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)pl.smem;
   cfg.stream = st;
-  attrs[0].id = cudaLaunchAttributeClusterDimension;
-  attrs[0].val.clusterDim.x = (unsigned)pl.C;
-  attrs[0].val.clusterDim.y = 1;
-  attrs[0].val.clusterDim.z = 1;
-  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
-// The cluster decode: streaming the sketch when scores is null, else reading
-// the scores [rows][len] a score-kernel launch wrote before it in the stream.
-fasa_status launch_fused(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t keff, void* out,
-                         int32_t* idx_out, const float* scores, int64_t sld, const FusedPlan& pl, cudaStream_t st,
-                         const DevInfo& d) {
-  FusedParams p{};
-  p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
-  p.scores = scores;
-  p.sld = sld;
-  p.k = static_cast<const __nv_bfloat16*>(c->k);
-  p.v = static_cast<const __nv_bfloat16*>(c->v);
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.dom_idx = c->dom_idx;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.idx_out = idx_out;
-  p.max_len = c->max_len;
-  p.len = len;
-  p.stride = c->sketch_stride;
-  p.n_kv_heads = c->n_kv_heads;
-  p.group = c->n_q_heads / c->n_kv_heads;
-  p.n_dom = c->n_dom;
-  p.n_keep = keff;
-  p.n_loc = pl.n_loc;
-  p.ring = pl.ring;
-  p.n_stages = pl.n_stages;
-  p.ucap = pl.ucap;
-  fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
-  const int rows = c->batch * c->n_kv_heads;
-  if (scores != nullptr) return launch_fused_t<1, true>(p, rows, pl, st, d);
-  switch (c->sketch_stride / 8) {
-    case 1: return launch_fused_t<1, false>(p, rows, pl, st, d);
-    case 2: return launch_fused_t<2, false>(p, rows, pl, st, d);
-    case 4: return launch_fused_t<4, false>(p, rows, pl, st, d);
-    case 8: return launch_fused_t<8, false>(p, rows, pl, st, d);
-    case 16: return launch_fused_t<16, false>(p, rows, pl, st, d);
-    default: return FASA_ERR_UNSUPPORTED;
-  }
-}
-
 // Decode workspace, each part 256-byte aligned:
-//   scores [rows][ld] f32 (ld = len rounded up to 32) | hist [rows][4096] u32 | cand_cnt [rows] u32 |
-//   att_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
+//   sem [rows] u64 | att_cnt [rows] u32          (zero between calls: every
+//                                                 call leaves them zero)
+//   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the wide plan,
+//     the published (key, token) pairs [rows][len] u32x2 |
+//   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
-// hist, cand_cnt and att_cnt are cleared at the start of every call.
+// The staged plan clears the first two parts and hist, cand_cnt at the start
+// of every call; the wide plan relies on them being zero.
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 struct DecodeWs {
-  size_t scores, hist, cnt, att_cnt, bitmap, cand, ckey, idx, part, qterm, total;
+  size_t sem, att_cnt, scores, hist, cnt, bitmap, cand, ckey, idx, part, qterm, total;
   int64_t ld;
   int cap, words, splits_max;
 };
@@ -552,11 +436,12 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.cap = (int)std::min<size_t>(std::max<size_t>(L, 1), 8192);
   w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms, kAttMaxPerSm);
   w.ld = (int64_t)((L + 31) / 32 * 32);
-  w.scores = 0;
-  w.hist = al256(rows * (size_t)w.ld * 4);
+  w.sem = 0;
+  w.att_cnt = rows * 8;
+  w.scores = al256(w.att_cnt + rows * 4);
+  w.hist = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, L * 8));
   w.cnt = w.hist + rows * kHistBins * 4;
-  w.att_cnt = w.cnt + rows * 4;
-  w.bitmap = al256(w.att_cnt + rows * 4);
+  w.bitmap = al256(w.cnt + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
   w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
   w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
@@ -614,6 +499,89 @@ fasa_status launch_cal_scores(const fasa_cache* c, int32_t len, const void* q_wi
   const dim3 grid((unsigned)ceil_div(len, kCalThreads), (unsigned)(c->batch * c->n_kv_heads), 1);
   calib_score_kernel<T><<<grid, kCalThreads, 0, st>>>(p);
   return cuda_status(cudaGetLastError());
+}
+
+// Split-K focused attention (attend_mma_kernel) over the kept lists idx
+// [rows][keff] and query terms of the workspace; its per-row counters are
+// the workspace's att_cnt (zero between calls).
+fasa_status launch_attend(const fasa_cache* c, int32_t len, int keff, void* out, const DecodeWs& w, char* base,
+                          const DevInfo& d, cudaStream_t st) {
+  const int rows = c->batch * c->n_kv_heads;
+  AttParams ap{};
+  ap.k = static_cast<const __nv_bfloat16*>(c->k);
+  ap.v = static_cast<const __nv_bfloat16*>(c->v);
+  ap.idx = reinterpret_cast<const int32_t*>(base + w.idx);
+  ap.qterms = reinterpret_cast<const unsigned char*>(base + w.qterm);
+  ap.out = static_cast<__nv_bfloat16*>(out);
+  ap.part = reinterpret_cast<float*>(base + w.part);
+  ap.counter = reinterpret_cast<uint32_t*>(base + w.att_cnt);
+  ap.max_len = c->max_len;
+  ap.len = len;
+  ap.n_keep = keff;
+  ap.group = c->n_q_heads / c->n_kv_heads;
+  int set = 0;
+  fasa_status s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
+    *v = 1;
+    return cuda_status(cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            att_smem_bytes(FASA_MAX_GROUP)));
+  });
+  if (s != FASA_OK) return s;
+  int per_sm = 0;  // resident attention CTAs per SM at this group size
+  if ((s = cached_int((const void*)attend_mma_kernel, 1 + (uint64_t)ap.group, &per_sm, [&](int* v) {
+         return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, attend_mma_kernel, kAttThreads,
+                                                                           (size_t)att_smem_bytes(ap.group)));
+       })) != FASA_OK)
+    return s;
+  per_sm = std::max(1, std::min(per_sm, kAttMaxPerSm));
+  ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms, per_sm));
+  ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
+  ap.splits = (int)ceil_div(keff, ap.slice);
+  if (ap.splits > kAttMaxSplits) return FASA_ERR_UNSUPPORTED;  // cannot happen: splits only shrank
+  return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
+                    (size_t)att_smem_bytes(ap.group), st, ap);
+}
+
+// The wide fused decode: one launch, plus the split-K attention when the
+// budget is beyond what the resolving CTA attends itself.
+fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int keff, void* out,
+                        int32_t* idx_out, const DecodeWs& w, char* base, const WidePlan& pl, const DevInfo& d,
+                        cudaStream_t st) {
+  WideParams p{};
+  p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
+  p.k = static_cast<const __nv_bfloat16*>(c->k);
+  p.v = static_cast<const __nv_bfloat16*>(c->v);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.dom_idx = c->dom_idx;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.idx_out = idx_out;
+  p.idx_ws = pl.direct ? nullptr : reinterpret_cast<int32_t*>(base + w.idx);
+  p.qterms = pl.direct ? nullptr : reinterpret_cast<unsigned char*>(base + w.qterm);
+  p.cand = reinterpret_cast<uint2*>(base + w.scores);
+  p.sem = reinterpret_cast<unsigned long long*>(base + w.sem);
+  p.max_len = c->max_len;
+  p.len = len;
+  p.stride = c->sketch_stride;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.n_dom = c->n_dom;
+  p.n_keep = keff;
+  p.n_loc = pl.n_loc;
+  p.n_split = pl.n_split;
+  p.ucache = pl.ucache;
+  p.direct = pl.direct;
+  fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
+  const int rows = c->batch * c->n_kv_heads;
+  fasa_status s;
+  switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
+    case 1: s = launch_wide_t<1>(p, rows, pl, st, d); break;
+    case 2: s = launch_wide_t<2>(p, rows, pl, st, d); break;
+    case 4: s = launch_wide_t<4>(p, rows, pl, st, d); break;
+    case 8: s = launch_wide_t<8>(p, rows, pl, st, d); break;
+    case 16: s = launch_wide_t<16>(p, rows, pl, st, d); break;
+    default: return FASA_ERR_UNSUPPORTED;
+  }
+  if (s != FASA_OK || pl.direct) return s;
+  return launch_attend(c, len, keff, out, w, base, d, st);
 }
 
 }  // namespace
@@ -767,22 +735,9 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   const int path = g_decode_path.load();
   char* base = static_cast<char*>(workspace);
   if (path == FASA_DECODE_AUTO || path == FASA_DECODE_FUSED) {
-    FusedPlan pl;
-    bool ok = false;
-    if ((s = fused_plan(c, len, d, path == FASA_DECODE_FUSED, false, &pl, &ok)) != FASA_OK) return s;
-    if (ok) return launch_fused(c, len, q, q_pos, keff, out, idx_out, nullptr, 0, pl, stream, d);
+    WidePlan pl;
+    if (wide_plan(c, len, keff, d, &pl)) return launch_wide(c, len, q, q_pos, keff, out, idx_out, w, base, pl, d, stream);
     if (path == FASA_DECODE_FUSED) return FASA_ERR_UNSUPPORTED;
-  }
-  if (path == FASA_DECODE_AUTO || path == FASA_DECODE_SCORED) {
-    FusedPlan pl;
-    bool ok = false;
-    if ((s = fused_plan(c, len, d, path == FASA_DECODE_SCORED, true, &pl, &ok)) != FASA_OK) return s;
-    if (ok) {
-      float* sc = reinterpret_cast<float*>(base + w.scores);
-      if ((s = launch_score(c, len, q, q_pos, sc, w.ld, nullptr, stream)) != FASA_OK) return s;
-      return launch_fused(c, len, q, q_pos, keff, out, idx_out, sc, w.ld, pl, stream, d);
-    }
-    if (path == FASA_DECODE_SCORED) return FASA_ERR_UNSUPPORTED;
   }
   float* scores = reinterpret_cast<float*>(base + w.scores);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + w.hist);
@@ -793,8 +748,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   int32_t* idx = reinterpret_cast<int32_t*>(base + w.idx);
 
   // 1. TIP scores and the per-row key histogram
-  uint32_t* att_cnt = reinterpret_cast<uint32_t*>(base + w.att_cnt);
-  float* part = reinterpret_cast<float*>(base + w.part);
+  if ((s = cuda_status(cudaMemsetAsync(base + w.sem, 0, w.scores - w.sem, stream))) != FASA_OK) return s;
   if ((s = cuda_status(cudaMemsetAsync(hist, 0, w.bitmap - w.hist, stream))) != FASA_OK) return s;
   if ((s = launch_score(c, len, q, q_pos, scores, w.ld, hist, stream)) != FASA_OK) return s;
 
@@ -853,39 +807,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     return s;
 
   // 4. focused attention over the kept rows
-  if (c->dtype == FASA_BF16) {
-    AttParams ap{};
-    ap.k = static_cast<const __nv_bfloat16*>(c->k);
-    ap.v = static_cast<const __nv_bfloat16*>(c->v);
-    ap.idx = idx;
-    ap.qterms = reinterpret_cast<const unsigned char*>(base + w.qterm);
-    ap.out = static_cast<__nv_bfloat16*>(out);
-    ap.part = part;
-    ap.counter = att_cnt;
-    ap.max_len = c->max_len;
-    ap.len = len;
-    ap.n_keep = keff;
-    ap.group = c->n_q_heads / c->n_kv_heads;
-    if ((s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
-           *v = 1;
-           return cuda_status(cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   att_smem_bytes(FASA_MAX_GROUP)));
-         })) != FASA_OK)
-      return s;
-    int per_sm = 0;  // resident attention CTAs per SM at this group size
-    if ((s = cached_int((const void*)attend_mma_kernel, 1 + (uint64_t)ap.group, &per_sm, [&](int* v) {
-           return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, attend_mma_kernel, kAttThreads,
-                                                                             (size_t)att_smem_bytes(ap.group)));
-         })) != FASA_OK)
-      return s;
-    per_sm = std::max(1, std::min(per_sm, kAttMaxPerSm));
-    ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms, per_sm));
-    ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
-    ap.splits = (int)ceil_div(keff, ap.slice);
-    if (ap.splits > kAttMaxSplits) return FASA_ERR_UNSUPPORTED;  // cannot happen: splits only shrank
-    return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
-                      (size_t)att_smem_bytes(ap.group), stream, ap);
-  }
+  if (c->dtype == FASA_BF16) return launch_attend(c, len, keff, out, w, base, d, stream);
   SAParams p{};
   p.idx_in = idx;
   p.k = c->k;
@@ -901,8 +823,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
 }
 
 fasa_status fasa_set_decode_path(int32_t path) {
-  if (path != FASA_DECODE_AUTO && path != FASA_DECODE_FUSED && path != FASA_DECODE_STAGED &&
-      path != FASA_DECODE_SCORED)
+  if (path != FASA_DECODE_AUTO && path != FASA_DECODE_FUSED && path != FASA_DECODE_STAGED)
     return FASA_ERR_INVALID_ARG;
   g_decode_path.store(path);
   return FASA_OK;
@@ -916,23 +837,39 @@ int32_t fasa_decode_path(const fasa_cache* c, int32_t len, int32_t k) {
   if ((s = device_info(&d)) != FASA_OK) return -s;
   const int path = g_decode_path.load();
   if (path != FASA_DECODE_AUTO) return path;
-  FusedPlan pl;
-  bool ok = false;
-  if ((s = fused_plan(c, len, d, false, false, &pl, &ok)) != FASA_OK) return -s;
-  if (ok) return FASA_DECODE_FUSED;
-  if ((s = fused_plan(c, len, d, false, true, &pl, &ok)) != FASA_OK) return -s;
-  return ok ? FASA_DECODE_SCORED : FASA_DECODE_STAGED;
+  WidePlan pl;
+  return wide_plan(c, len, std::min(k, len), d, &pl) ? FASA_DECODE_FUSED : FASA_DECODE_STAGED;
+}
+
+int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
+  const int32_t path = fasa_decode_path(c, len, k);
+  if (path < 0) return path;
+  if (path == FASA_DECODE_STAGED) return 4;
+  DevInfo d;
+  if (device_info(&d) != FASA_OK) return -FASA_ERR_CUDA;
+  WidePlan pl;
+  if (!wide_plan(c, len, std::min(k, len), d, &pl)) return -FASA_ERR_UNSUPPORTED;
+  return pl.direct ? 1 : 2;
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,
                                        void* out, int32_t* idx_out, cudaStream_t stream) {
+  // fasa_decode's own checks first, so a call both unsupported and too large
+  // gets the same status as from fasa_decode; then the scratch limit
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
   if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
-  if (decode_ws(c, len, k) > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
+  if (len > FASA_MAX_LEN || k > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  if (idx_out != nullptr && !aligned(idx_out, 4)) return FASA_ERR_INVALID_ARG;
+  const DecodeWs w = decode_layout(c, len, k);
+  if (w.total > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
   void* ws = nullptr;
   if ((s = static_scratch_addr(&ws)) != FASA_OK) return s;
+  // the semaphores start zero at load and every call leaves them zero; clear
+  // them anyway, so that a call that ended in an error cannot poison the next
+  if ((s = cuda_status(cudaMemsetAsync(ws, 0, w.scores, stream))) != FASA_OK) return s;
   return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);
 }
 

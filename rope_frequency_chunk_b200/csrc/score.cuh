@@ -16,15 +16,11 @@
 // in flight per SM) and scores them, one token per lane (two or four lanes
 // for rows wider than 32 elements).
 //
-// Arithmetic: float64. Each stored element e is widened exactly to the double
-// e * 2^-896 by placing its sign, exponent and mantissa bits in the double's
-// high word (bf16: 7 mantissa bits; f32: 23); the coefficients carry the
-// compensating 2^896, so each product equals Q[c]*e rounded once. This avoids
-// the float->double conversion unit in the hot loop. The sum is rounded to
-// float32 once at the end.
+// Arithmetic: float32, in the fixed order and with the error bound stated in
+// tip.cuh (coefficients from a float64 rotation and group sum, rounded once).
 #pragma once
 
-#include "fasa_device.cuh"
+#include "tip.cuh"
 
 namespace fasa {
 
@@ -50,96 +46,32 @@ struct ScoreParams {
   double sinv[kNFC];
 };
 
-// Widen the two bf16 halves of w to (value * 2^-896) doubles, exactly.
-__device__ __forceinline__ void widen_scaled(uint32_t w, double& lo, double& hi, __nv_bfloat16) {
-  const uint32_t lo_hi = ((w << 16) & 0x80000000u) | ((w << 13) & 0x0FFFE000u);
-  const uint32_t hi_hi = (w & 0x80000000u) | ((w >> 3) & 0x0FFFE000u);
-  lo = __hiloint2double((int)lo_hi, 0);
-  hi = __hiloint2double((int)hi_hi, 0);
-}
-// Widen one float32 to (value * 2^-896) double, exactly.
-__device__ __forceinline__ double widen_scaled_f32(uint32_t w) {
-  const uint32_t h = (w & 0x80000000u) | ((w & 0x7FFFFFFFu) >> 3);
-  return __hiloint2double((int)h, (int)(w << 29));
-}
-
-template <typename T>
-__device__ __forceinline__ double chunk_dot(const uint4& u, const double* qr);
-
-template <>
-__device__ __forceinline__ double chunk_dot<__nv_bfloat16>(const uint4& u, const double* qr) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  double acc = 0.0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    double a, b;
-    widen_scaled(w[i], a, b, __nv_bfloat16());
-    acc = fma(a, qr[2 * i], acc);
-    acc = fma(b, qr[2 * i + 1], acc);
-  }
-  return acc;
-}
-template <>
-__device__ __forceinline__ double chunk_dot<float>(const uint4& u, const double* qr) {
-  double acc = 0.0;
-  acc = fma(widen_scaled_f32(u.x), qr[0], acc);
-  acc = fma(widen_scaled_f32(u.y), qr[1], acc);
-  acc = fma(widen_scaled_f32(u.z), qr[2], acc);
-  acc = fma(widen_scaled_f32(u.w), qr[3], acc);
-  return acc;
-}
-
 constexpr int kHistBits = 12;                 // key bits of the per-row score histogram
 constexpr int kHistBins = 1 << kHistBits;
 
-// Shape of the per-token work for sketch rows of LPT 16-byte chunks.
+// Shape of the per-token work for sketch rows of LPT 16-byte chunks, with a
+// chunk rotation per lane so that a quarter-warp's 16-byte shared-memory
+// reads hit distinct banks (the lane's coefficients are rotated the same way).
 template <typename T, int LPT>
-struct ScoreShape {
-  static constexpr int EPC = Elem<T>::kPer16;                   // elements per 16-byte chunk
-  static constexpr int ROWE = LPT * EPC;                        // elements per sketch row
-  static constexpr int ROWB = LPT * 16;                         // sketch row bytes
-  static constexpr int LPT2 = ROWE > 32 ? ROWE / 32 : 1;        // lanes per token
-  static constexpr int EPL = ROWE / LPT2;                       // elements per lane (<= 32)
-  static constexpr int CPL = EPL / EPC;                         // chunks per lane
-  static constexpr int TPW = 32 / LPT2;                         // tokens per warp step
-  // chunk rotation per lane so that a quarter-warp's 16-byte reads hit
-  // distinct banks; the lane's coefficients are rotated the same way
+struct ScoreShape : TipShape<T, LPT> {
+  using B = TipShape<T, LPT>;
+  static constexpr int TPW = 32 / B::LPT2;  // tokens per warp step
   __device__ static int rot(int lane) {
-    return (LPT2 == 1) ? ((lane * CPL / 8) % CPL) : (LPT2 == 2 ? ((lane / 2) % CPL) : 0);
+    return (B::LPT2 == 1) ? ((lane * B::CPL / 8) % B::CPL) : (B::LPT2 == 2 ? ((lane / 2) % B::CPL) : 0);
   }
 };
 
-// Sketch-column coefficients of one row, scaled by 2^896: column 2j (2j+1)
-// is the first (second) dim of dominant FC dom[j], summed over the group's
-// rotated query heads; padding columns are zero. Thread `tid` < stride
+// Sketch-column coefficients of one row (tip_coef): thread `tid` < stride
 // writes column tid.
 template <typename T>
 __device__ __forceinline__ void query_coefs(const T* qraw, const int* dom, int group, int n_dom, int stride,
-                                            const double* cosv, const double* sinv, int tid, double* s_q) {
-  if (tid >= stride) return;
-  const double two896 = __hiloint2double(0x77F00000, 0);  // 2^896: exponent field 1919
-  double acc = 0.0;
-  const int jj = tid >> 1;
-  if (jj < n_dom) {
-    const int i = dom[jj];
-    if (i >= 0 && i < kNFC) {
-      const double c = cosv[i], s = sinv[i];
-      for (int h = 0; h < group; ++h) {
-        const double x = to_float(qraw[h * kD + i]);
-        const double y = to_float(qraw[h * kD + i + kNFC]);
-        // rotated query, first (x) or second (y) dim of FC i
-        acc += (tid & 1) ? __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s)) : __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
-      }
-    } else {
-      flag_status(FASA_ERR_BAD_INDEX);
-    }
-  }
-  s_q[tid] = acc * two896;
+                                            const double* cosv, const double* sinv, int tid, float* s_q) {
+  if (tid < stride) s_q[tid] = tip_coef<T>(qraw, dom, group, n_dom, tid, cosv, sinv);
 }
 
 // The lane's share of the coefficients, in its rotated chunk order.
 template <typename T, int LPT>
-__device__ __forceinline__ void load_coefs(double (&qr)[ScoreShape<T, LPT>::EPL], const double* s_q, int lane) {
+__device__ __forceinline__ void load_coefs(float (&qr)[ScoreShape<T, LPT>::EPL], const float* s_q, int lane) {
   using S = ScoreShape<T, LPT>;
   const int sub = lane % S::LPT2, rot = S::rot(lane);
 #pragma unroll
@@ -152,7 +84,7 @@ __device__ __forceinline__ void load_coefs(double (&qr)[ScoreShape<T, LPT>::EPL]
 // 0..NCW-1 in turn. sink(t, writer, score) is called by every lane of the
 // warp (warp-uniform), writer set on the one lane that owns token t.
 template <typename T, int LPT, int NCW, typename Sink>
-__device__ __forceinline__ void score_block(const unsigned char* buf, int n, const double (&qr)[ScoreShape<T, LPT>::EPL],
+__device__ __forceinline__ void score_block(const unsigned char* buf, int n, const float (&qr)[ScoreShape<T, LPT>::EPL],
                                             int warp, int lane, Sink&& sink) {
   using S = ScoreShape<T, LPT>;
   const int sub = lane % S::LPT2, rot = S::rot(lane);
@@ -164,15 +96,13 @@ __device__ __forceinline__ void score_block(const unsigned char* buf, int n, con
     for (int c = 0; c < S::CPL; ++c)
       v[c] = valid ? *reinterpret_cast<const uint4*>(buf + t * S::ROWB + (sub * S::CPL + (c + rot) % S::CPL) * 16)
                    : make_uint4(0, 0, 0, 0);
-    double part[S::CPL];
+    // chunk partials in the lane's rotated order; the halving tree does not
+    // depend on the rotation
+    float part[S::CPL];
 #pragma unroll
-    for (int c = 0; c < S::CPL; ++c) part[c] = chunk_dot<T>(v[c], qr + c * S::EPC);
-    double acc = part[0];
-#pragma unroll
-    for (int c = 1; c < S::CPL; ++c) acc += part[c];
-#pragma unroll
-    for (int off = S::LPT2 / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-    sink(t, valid && sub == 0, (float)acc);
+    for (int c = 0; c < S::CPL; ++c) part[c] = tip_chunk(v[c], qr + c * S::EPC, T());
+    const float acc = tip_lanes_sum<S::LPT2>(tip_lane_sum<S::CPL>(part));
+    sink(t, valid && sub == 0, acc);
   }
 }
 
@@ -194,7 +124,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
   constexpr int D = R::kDepth;
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + kScoreWarps * kScoreWarpBytes);
-  __shared__ double s_q[kD];
+  __shared__ float s_q[kD];
   __shared__ __align__(16) T s_qraw[FASA_MAX_GROUP * kD];  // the group's raw queries
   __shared__ int s_dom[kNFC];
   grid_dependency_wait();
@@ -225,7 +155,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     __syncthreads();
     query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
     __syncthreads();
-    double qr[S::EPL];
+    float qr[S::EPL];
     load_coefs<T, LPT>(qr, s_q, lane);
 
     // warp w takes the steps w, w + kScoreWarps, ... of TPW consecutive tokens

@@ -55,6 +55,7 @@ _SIGS = {
     "fasa_select_topk": (_I, [_P, _I, _I, _I, _P, _P]),
     "fasa_sparse_attend": (_I, [_CP, _I, _P, _I, _P, _I, _P, _P]),
     "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I]),
+    "fasa_decode_launches": (_I, [_CP, _I, _I]),
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
@@ -212,9 +213,17 @@ def fasa_decode_workspace_bytes(cache: KVCache, length: int, k: int) -> int:
     return int(lib().fasa_decode_workspace_bytes(cache.ref(), length, k))
 
 
+def fasa_decode_workspace(cache: KVCache, length: int, k: int, device=None):
+    """A decode workspace for this shape, zeroed as fasa_decode requires
+    before its first use (every call leaves its semaphores zero again)."""
+    dev = device if device is not None else cache.k.device
+    return torch.zeros(max(fasa_decode_workspace_bytes(cache, length, k), 1), dtype=torch.uint8, device=dev)
+
+
 def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, idx_out=None,
                 workspace=None, stream=None):
-    """One FASA decode step; returns out (and fills idx_out when given)."""
+    """One FASA decode step; returns out (and fills idx_out when given). A
+    given workspace must have been zeroed once (fasa_decode_workspace)."""
     _q(cache, q)
     if out is None:
         out = torch.empty_like(q)
@@ -223,14 +232,14 @@ def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, id
         _dev(idx_out, "idx_out", torch.int32)
     need = fasa_decode_workspace_bytes(cache, length, k)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     _dev(workspace, "workspace", torch.uint8)
     _check(lib().fasa_decode(cache.ref(), length, q.data_ptr(), q_pos, k, out.data_ptr(), _ptr(idx_out),
                              workspace.data_ptr(), workspace.numel(), _stream(stream)), "fasa_decode")
     return out
 
 
-DECODE_AUTO, DECODE_FUSED, DECODE_STAGED, DECODE_SCORED = 0, 1, 2, 3
+DECODE_AUTO, DECODE_FUSED, DECODE_STAGED = 0, 1, 2
 
 
 def fasa_set_decode_path(path: int) -> None:
@@ -239,10 +248,18 @@ def fasa_set_decode_path(path: int) -> None:
 
 
 def fasa_decode_path(cache: KVCache, length: int, k: int) -> int:
-    """The plan fasa_decode would run for this shape (DECODE_FUSED, DECODE_SCORED or DECODE_STAGED)."""
+    """The plan fasa_decode would run for this shape (DECODE_FUSED or DECODE_STAGED)."""
     r = int(lib().fasa_decode_path(cache.ref(), length, k))
     if r < 0:
         _check(-r, "fasa_decode_path")
+    return r
+
+
+def fasa_decode_launches(cache: KVCache, length: int, k: int) -> int:
+    """Kernels of this library one fasa_decode call launches for this shape."""
+    r = int(lib().fasa_decode_launches(cache.ref(), length, k))
+    if r < 0:
+        _check(-r, "fasa_decode_launches")
     return r
 
 

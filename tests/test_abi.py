@@ -104,10 +104,12 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 
 
 def test_decode_path_setting_is_validated_on_the_host(L):
-    assert L.fasa_set_decode_path(4) == 1 and L.fasa_set_decode_path(-1) == 1
-    for p in (1, 2, 3, 0):
+    for bad in (3, 4, -1):
+        assert L.fasa_set_decode_path(bad) == 1
+    for p in (1, 2, 0):
         assert L.fasa_set_decode_path(p) == 0
     assert L.fasa_decode_path(None, 10, 10) < 0
+    assert L.fasa_decode_launches(None, 10, 10) < 0
 
 
 def test_calibration_validation_without_launch(L):

@@ -135,7 +135,7 @@ def test_dense_matches_oracle(name):
         U.check_out(wl, out[b, g * G:(g + 1) * G], ref)
 
 
-PATHS = {"fused": F.DECODE_FUSED, "scored": F.DECODE_SCORED, "staged": F.DECODE_STAGED}
+PATHS = {"fused": F.DECODE_FUSED, "staged": F.DECODE_STAGED}
 
 
 @pytest.fixture(params=list(PATHS))
@@ -147,8 +147,8 @@ def path(request):
 
 
 def _skip_unless_plan(wl, path):
-    if path in ("fused", "scored") and wl.dtype != "bf16":
-        pytest.skip("the cluster decode takes bf16 caches only")
+    if path == "fused" and wl.dtype != "bf16":
+        pytest.skip("the fused decode takes bf16 caches only")
 
 
 def _decode(wl, cache, q, k, length=None):
@@ -241,9 +241,10 @@ def test_decode_with_small_tie_at_budget_edge(path):
 
 @pytest.mark.parametrize("case", ["all_tied", "k_beyond_union"])
 def test_decode_exact_fallbacks(case, path):
-    """Shapes where the single-launch decode's candidate union cannot prove
-    exactness (every CTA cuts inside one big tie; k above what the union
-    holds) and it falls back to the exact distributed radix select."""
+    """Shapes that take the exact radix selects: every token tied (the
+    boundary bin holds the whole row, far beyond the shared-memory tie list)
+    and a budget of half a 40000-token row (every CTA publishes all of its
+    tokens; the kept list goes to the split-K attention)."""
     if case == "all_tied":
         wl = C["c2"].replace(n_q_heads=4, n_kv_heads=1, ctx_len=8192, k=100)
         inp = W.layer_inputs(wl)
@@ -263,7 +264,7 @@ def test_decode_exact_fallbacks(case, path):
 def test_decode_is_deterministic_and_capturable(path):
     wl = SMALL["c2_ragged"]
     inp, cache, q = U.build(wl)
-    ws = torch.empty(F.fasa_decode_workspace_bytes(cache, wl.ctx_len, wl.k), dtype=torch.uint8, device="cuda")
+    ws = F.fasa_decode_workspace(cache, wl.ctx_len, wl.k)
     out1 = torch.empty_like(q)
     F.fasa_decode(cache, wl.ctx_len, q, wl.q_pos, wl.k, out=out1, workspace=ws)
     s = torch.cuda.Stream()
@@ -292,7 +293,7 @@ def _check_paths_agree(wl, res):
     """Every plan scores bit-identically and selects exactly: the same kept
     sets; outputs differ only by float32 summation order."""
     o_s, i_s = res["staged"]
-    for name in ("fused", "scored"):
+    for name in ("fused",):
         o_x, i_x = res[name]
         assert torch.equal(i_x, i_s), name
         U.check_gpu_pair(wl, U.stored(o_x), U.stored(o_s))
@@ -311,11 +312,10 @@ def test_decode_path_setting_and_choice():
         F.fasa_set_decode_path(7)
 
 
-@pytest.mark.parametrize("plan", [F.DECODE_FUSED, F.DECODE_SCORED])
-def test_cluster_decode_rejects_f32_when_forced(plan):
+def test_fused_decode_rejects_f32_when_forced():
     wl = SMALL["c1"]
     _, cache, q = U.build(wl)
-    F.fasa_set_decode_path(plan)
+    F.fasa_set_decode_path(F.DECODE_FUSED)
     try:
         with pytest.raises(F.FasaError) as e:
             _decode(wl, cache, q, wl.k)
@@ -352,14 +352,13 @@ def test_full_c2():
         U.check_out(wl, dense[b, g * G:(g + 1) * G], ref)
 
 
-def test_full_c3_sampled():
+def test_full_c3():
+    """Every (sequence, KV head) row of c3 against the oracle."""
     wl = C["c3"]
     inp, cache, q = U.build(wl)
-    heads = U.sample_heads(wl, 3)
-    U.check_append(wl, inp, cache, heads[:1])
-    assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_STAGED
+    U.check_append(wl, inp, cache, U.sample_heads(wl, 1))
     out, idx = _decode(wl, cache, q, wl.k)
-    U.check_decode_heads(wl, inp, cache, q, wl.k, heads, out, idx)
+    U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx)
     _check_paths_agree(wl, _both_paths(wl, cache, q, wl.k))
 
 
@@ -372,11 +371,12 @@ def c5_state():
 
 
 @pytest.mark.parametrize("k", W.C5_KS)
-def test_full_c5_sampled(k, c5_state):
+def test_full_c5(k, c5_state):
+    """Every row of c5 at each budget against the oracle."""
     wl = C["c5"]
     inp, cache, q = c5_state
     out, idx = _decode(wl, cache, q, k)
-    U.check_decode_heads(wl, inp, cache, q, k, U.sample_heads(wl, 3, seed=k), out, idx)
+    U.check_decode_heads(wl, inp, cache, q, k, U.all_heads(wl), out, idx)
     if k == W.C5_KS[0]:
         _check_paths_agree(wl, _both_paths(wl, cache, q, k))
     if k == W.C5_KS[-1]:
@@ -389,8 +389,9 @@ def test_full_c5_sampled(k, c5_state):
 
 
 @pytest.mark.parametrize("n_dom", W.C4_NDOMS)
-def test_full_c4_sweep_sampled(n_dom):
-    """Long-CoT sweep: 1K appends up to 32K; decode with k = 18.9% of L at several steps."""
+def test_full_c4_sweep(n_dom):
+    """Long-CoT sweep: 1K appends up to 32K; decode with k = 18.9% of L at
+    several steps, every row against the oracle."""
     wl = C["c4"]
     inp = W.layer_inputs(wl, n_dom=n_dom)
     lp = inp.params
@@ -398,7 +399,7 @@ def test_full_c4_sweep_sampled(n_dom):
                       lp.dom_idx)
     k_all = W.to_torch(inp.k, "cuda")
     v_all = W.to_torch(inp.v, "cuda")
-    heads = U.sample_heads(wl, 2, seed=n_dom)
+    heads = U.all_heads(wl)
     for step in range(W.C4_STEPS):
         c0 = step * W.C4_APPEND_CHUNK
         c1 = c0 + W.C4_APPEND_CHUNK
@@ -412,4 +413,4 @@ def test_full_c4_sweep_sampled(n_dom):
             sub = W.LayerInputs(lp, q_np, inp.k, inp.v)
             out, idx = _decode(wl, cache, q, k, length=L)
             U.check_decode_heads(wl, sub, cache, q, k, heads, out, idx, length=L)
-    U.check_append(wl, inp, cache, heads[:1])
+    U.check_append(wl, inp, cache, U.sample_heads(wl, 1, seed=n_dom))
