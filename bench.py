@@ -344,9 +344,11 @@ def run_fasa(args, wl):
         for c, q in zip(caches, qs):
             F.fasa_score(c, L, q, wl.q_pos, scores=scores)
 
+    dws = F.fasa_dense_workspace(caches[0], L, device)
+
     def dense_step():
         for c, q, o in zip(caches, qs, outs):
-            F.fasa_dense_decode(c, L, q, wl.q_pos, out=o)
+            F.fasa_dense_decode(c, L, q, wl.q_pos, out=o, workspace=dws)
 
     plan = F.fasa_decode_path(caches[0], L, k)
     launches = F.fasa_decode_launches(caches[0], L, k)

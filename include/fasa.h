@@ -301,13 +301,26 @@ int32_t fasa_decode_launches(const fasa_cache* cache, int32_t len, int32_t k);
 fasa_status fasa_decode_static_scratch(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
                                        int32_t k, void* out, int32_t* idx_out, cudaStream_t stream);
 
+/* Workspace bytes fasa_dense_decode needs for this cache and len (0 for
+ * invalid arguments). */
+size_t fasa_dense_workspace_bytes(const fasa_cache* cache, int32_t len);
+
 /*
  * Dense full-KV decode, the comparison path: the same attention as
  * fasa_sparse_attend over all len cached rows (the upper bound in
- * [tech §4] "Resultados Experimentais", full KV "FKV").
+ * [tech §4] "Resultados Experimentais", full KV "FKV"). bf16 caches run the
+ * decode's split-K tensor-core attention over every row (a one-wave grid of
+ * splits, merged by each row's last CTA); f32 caches a cluster kernel.
+ *
+ *  workspace : at least fasa_dense_workspace_bytes(cache, len) bytes,
+ *            256-byte aligned, zeroed once after allocation: its first
+ *            4 * B * Hkv bytes are per-row counters that must be zero when a
+ *            call starts and that every call leaves zero; the rest is scratch.
+ *  Errors: as fasa_sparse_attend; FASA_ERR_WORKSPACE for a missing or short
+ *  workspace.
  */
 fasa_status fasa_dense_decode(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos,
-                              void* out, cudaStream_t stream);
+                              void* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Synchronizes the current device, then returns FASA_OK or the first

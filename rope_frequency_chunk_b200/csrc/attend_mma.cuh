@@ -44,7 +44,10 @@ struct AttParams {
   const __nv_bfloat16* k;   // [rows][max_len][128]
   const __nv_bfloat16* v;
   const int32_t* idx;       // [rows][n_keep] kept rows; null: rows 0 .. n_keep-1
-  const unsigned char* qterms;  // [rows][kQTermBytes] query terms (see query_terms)
+  const unsigned char* qterms;  // [rows][kQTermBytes] query terms (see query_terms), or null:
+                                // each CTA forms its row's terms from q (query_terms_compact)
+  const __nv_bfloat16* q;   // [B][Hq][128] pre-RoPE (with qterms null)
+  int32_t n_kv_heads;       // (with qterms null)
   __nv_bfloat16* out;       // [B][Hq][128]
   float* part;              // [rows][splits][kAttPartStride]
   uint32_t* counter;        // [rows], zero before the launch; the last CTA resets it
@@ -54,6 +57,8 @@ struct AttParams {
   int32_t slice;            // rows per CTA, a multiple of kAttChunk
   int32_t splits;
   int32_t group;
+  double cosv[kNFC];        // cos / sin of q_pos * theta_i (with qterms null)
+  double sinv[kNFC];
 };
 
 // The ring, then the G query rows of each term (256 B each) and one zero row
@@ -127,6 +132,36 @@ __device__ __forceinline__ void query_terms(const __nv_bfloat16* qraw, int G, co
   }
 }
 
+// The same terms in the compact layout chunk_logits reads: term t (low,
+// middle, high) of head r at row t*G + r, then a zero row at 3G; the values
+// are query_terms' bit for bit. qraw: the group's G pre-RoPE query rows.
+__device__ __forceinline__ void query_terms_compact(const __nv_bfloat16* qraw, int G, const double* cosv,
+                                                    const double* sinv, unsigned char* qt, int tid, int nthreads) {
+  const double qscale = 1.4426950408889634 / 11.313708498984761;
+  for (int e = tid; e < G * (kD / 2); e += nthreads) {
+    const int h = e / (kD / 2), d = 2 * (e % (kD / 2));
+    float v2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int dd = d + u, i = dd & (kNFC - 1);
+      const double x = __bfloat162float(qraw[h * kD + i]);
+      const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
+      const double c = cosv[i], sn = sinv[i];
+      v2[u] = (float)(((dd < kNFC) ? (x * c - y * sn) : (y * c + x * sn)) * qscale);
+    }
+    uint32_t hi, mid, lo;
+    const float2 r = split_pack(v2[0], v2[1], hi, mid);
+    const float2 mf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&mid));
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(r.x - mf.x, r.y - mf.y);
+    lo = *reinterpret_cast<const uint32_t*>(&ll);
+    const int off = (((d / 8) ^ (h & 7)) * 16) + (d % 8) * 2;
+    *reinterpret_cast<uint32_t*>(qt + (0 * G + h) * 256 + off) = lo;
+    *reinterpret_cast<uint32_t*>(qt + (1 * G + h) * 256 + off) = mid;
+    *reinterpret_cast<uint32_t*>(qt + (2 * G + h) * 256 + off) = hi;
+  }
+  for (int c = tid; c < 16; c += nthreads) reinterpret_cast<uint4*>(qt + 3 * G * 256)[c] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // S = Q K^T for one 16-row chunk staged at Ks: s0 rows 0-7, s1 rows 8-15 of
 // the chunk (fragment layout of m16n8k16), each Q term in its own chain.
 // Query row r of term t is at qt + (t * G + r) * 256 for r < G, the zero
@@ -166,7 +201,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.group;
   unsigned char* qt = smem + kAttWarps * kAttStages * kAttStageBytes;
-  {
+  if (p.qterms) {
     // the G real rows of each term (rows of the staged terms keep their
     // swizzle, which depends on the row index only), then a zero row
     const unsigned char* src = p.qterms + (int64_t)row * kQTermBytes;
@@ -176,6 +211,15 @@ __global__ void __launch_bounds__(kAttThreads) attend_mma_kernel(const AttParams
     }
     if (tid < 16) reinterpret_cast<uint4*>(qt + 3 * G * 256)[tid] = make_uint4(0u, 0u, 0u, 0u);
     cp_async_commit();
+  } else {
+    // the row's query terms from q, staged through the (not yet used) ring
+    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
+    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
+    for (int c = tid; c < G * kD / 8; c += kAttThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    __syncthreads();
+    query_terms_compact(qraw, G, p.cosv, p.sinv, qt, tid, kAttThreads);
+    __syncthreads();
+    cp_async_commit();  // an empty group: the pipeline below counts one group for the terms
   }
 
   const int r_beg = split * p.slice;

@@ -501,24 +501,30 @@ fasa_status launch_cal_scores(const fasa_cache* c, int32_t len, const void* q_wi
   return cuda_status(cudaGetLastError());
 }
 
-// Split-K focused attention (attend_mma_kernel) over the kept lists idx
-// [rows][keff] and query terms of the workspace; its per-row counters are
-// the workspace's att_cnt (zero between calls).
-fasa_status launch_attend(const fasa_cache* c, int32_t len, int keff, void* out, const DecodeWs& w, char* base,
-                          const DevInfo& d, cudaStream_t st) {
+// Split-K attention (attend_mma_kernel) of every row over its kept list
+// idx [rows][n_keep], or over rows 0 .. n_keep-1 when idx is null (the dense
+// decode); the query terms come from qterms [rows][kQTermBytes], or, when it
+// is null, each CTA forms them from q. part [rows][splits_max][...] holds
+// the split partials; counter [rows] must be zero (the kernel leaves it zero).
+fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
+                          const unsigned char* qterms, const void* q, int32_t q_pos, float* part, uint32_t* counter,
+                          int splits_max, const DevInfo& d, cudaStream_t st) {
   const int rows = c->batch * c->n_kv_heads;
   AttParams ap{};
   ap.k = static_cast<const __nv_bfloat16*>(c->k);
   ap.v = static_cast<const __nv_bfloat16*>(c->v);
-  ap.idx = reinterpret_cast<const int32_t*>(base + w.idx);
-  ap.qterms = reinterpret_cast<const unsigned char*>(base + w.qterm);
+  ap.idx = idx;
+  ap.qterms = qterms;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.n_kv_heads = c->n_kv_heads;
   ap.out = static_cast<__nv_bfloat16*>(out);
-  ap.part = reinterpret_cast<float*>(base + w.part);
-  ap.counter = reinterpret_cast<uint32_t*>(base + w.att_cnt);
+  ap.part = part;
+  ap.counter = counter;
   ap.max_len = c->max_len;
   ap.len = len;
-  ap.n_keep = keff;
+  ap.n_keep = n_keep;
   ap.group = c->n_q_heads / c->n_kv_heads;
+  if (qterms == nullptr) fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
   int set = 0;
   fasa_status s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
     *v = 1;
@@ -533,12 +539,37 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int keff, void* out,
        })) != FASA_OK)
     return s;
   per_sm = std::max(1, std::min(per_sm, kAttMaxPerSm));
-  ap.splits = std::min(w.splits_max, att_splits(rows, keff, d.sms, per_sm));
-  ap.slice = (int)ceil_div(att_chunks(keff), ap.splits) * kAttChunk;
-  ap.splits = (int)ceil_div(keff, ap.slice);
+  ap.splits = std::min(splits_max, att_splits(rows, n_keep, d.sms, per_sm));
+  ap.slice = (int)ceil_div(att_chunks(n_keep), ap.splits) * kAttChunk;
+  ap.splits = (int)ceil_div(n_keep, ap.slice);
   if (ap.splits > kAttMaxSplits) return FASA_ERR_UNSUPPORTED;  // cannot happen: splits only shrank
   return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
                     (size_t)att_smem_bytes(ap.group), st, ap);
+}
+
+// The decode's attention over the kept lists and query terms in the workspace.
+fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, void* out, const DecodeWs& w, char* base,
+                             const DevInfo& d, cudaStream_t st) {
+  return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx),
+                       reinterpret_cast<const unsigned char*>(base + w.qterm), nullptr, 0,
+                       reinterpret_cast<float*>(base + w.part), reinterpret_cast<uint32_t*>(base + w.att_cnt),
+                       w.splits_max, d, st);
+}
+
+// Dense decode workspace: att_cnt [rows] u32 (zero between calls) | part
+// [rows][splits_max][kAttPartStride] f32.
+struct DenseWs {
+  size_t att_cnt, part, total;
+  int splits_max;
+};
+DenseWs dense_layout(const fasa_cache* c, int32_t len) {
+  DenseWs w;
+  const size_t rows = (size_t)c->batch * c->n_kv_heads;
+  w.splits_max = att_splits((int)rows, std::max(len, 1), kAssumedMaxSms, kAttMaxPerSm);
+  w.att_cnt = 0;
+  w.part = al256(rows * 4);
+  w.total = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4) + 256;
+  return w;
 }
 
 // The wide fused decode: one launch, plus the split-K attention when the
@@ -581,7 +612,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
     default: return FASA_ERR_UNSUPPORTED;
   }
   if (s != FASA_OK || pl.direct) return s;
-  return launch_attend(c, len, keff, out, w, base, d, st);
+  return launch_attend_ws(c, len, keff, out, w, base, d, st);
 }
 
 }  // namespace
@@ -807,7 +838,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     return s;
 
   // 4. focused attention over the kept rows
-  if (c->dtype == FASA_BF16) return launch_attend(c, len, keff, out, w, base, d, stream);
+  if (c->dtype == FASA_BF16) return launch_attend_ws(c, len, keff, out, w, base, d, stream);
   SAParams p{};
   p.idx_in = idx;
   p.k = c->k;
@@ -873,13 +904,27 @@ fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const v
   return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);
 }
 
+size_t fasa_dense_workspace_bytes(const fasa_cache* c, int32_t len) {
+  if (check_cache(c) != FASA_OK || len < 0) return 0;
+  return dense_layout(c, len).total;
+}
+
 fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, void* out,
-                              cudaStream_t stream) {
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
   if (len < 1 || q_pos < 0) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  const DenseWs w = dense_layout(c, len);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return FASA_ERR_WORKSPACE;
+  if (c->dtype == FASA_BF16) {
+    DevInfo d;
+    if ((s = device_info(&d)) != FASA_OK) return s;
+    char* base = static_cast<char*>(workspace);
+    return launch_attend(c, len, len, out, nullptr, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part),
+                         reinterpret_cast<uint32_t*>(base + w.att_cnt), w.splits_max, d, stream);
+  }
   SAParams p{};
   p.k = c->k;
   p.v = c->v;

@@ -58,7 +58,8 @@ _SIGS = {
     "fasa_decode_launches": (_I, [_CP, _I, _I]),
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
-    "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P]),
+    "fasa_dense_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
+    "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]),
     "fasa_device_status": (_I, [_I]),
     "fasa_set_decode_path": (_I, [_I]),
     "fasa_decode_path": (_I, [_CP, _I, _I]),
@@ -263,13 +264,25 @@ def fasa_decode_launches(cache: KVCache, length: int, k: int) -> int:
     return r
 
 
-def fasa_dense_decode(cache: KVCache, length: int, q, q_pos: int, out=None, stream=None):
+def fasa_dense_workspace(cache: KVCache, length: int, device=None):
+    """A zeroed workspace for fasa_dense_decode at this length."""
+    dev = device if device is not None else cache.k.device
+    need = int(lib().fasa_dense_workspace_bytes(cache.ref(), length))
+    return torch.zeros(max(need, 1), dtype=torch.uint8, device=dev)
+
+
+def fasa_dense_decode(cache: KVCache, length: int, q, q_pos: int, out=None, workspace=None, stream=None):
+    """Dense attention over all `length` cached rows (the comparison path). A
+    given workspace must have been zeroed once (fasa_dense_workspace)."""
     _q(cache, q)
     if out is None:
         out = torch.empty_like(q)
     _dev(out, "out", cache.dtype)
-    _check(lib().fasa_dense_decode(cache.ref(), length, q.data_ptr(), q_pos, out.data_ptr(), _stream(stream)),
-           "fasa_dense_decode")
+    if workspace is None:
+        workspace = fasa_dense_workspace(cache, length, q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_dense_decode(cache.ref(), length, q.data_ptr(), q_pos, out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel(), _stream(stream)), "fasa_dense_decode")
     return out
 
 

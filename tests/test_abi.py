@@ -93,7 +93,11 @@ def test_call_validation_without_launch(L):
     need = L.fasa_decode_workspace_bytes(c, 100, 8)
     assert need >= 2 * 100 * 4
     assert L.fasa_decode(c, 100, 0x50000, 100, 8, 0x70000, None, 0x80000, need - 1, None) == 4
-    assert L.fasa_dense_decode(c, 0, 0x50000, 0, 0x70000, None) == 1
+    assert L.fasa_dense_decode(c, 0, 0x50000, 0, 0x70000, 0x80000, 1 << 20, None) == 1
+    dneed = L.fasa_dense_workspace_bytes(c, 100)
+    assert dneed > 0
+    assert L.fasa_dense_decode(c, 100, 0x50000, 100, 0x70000, 0x80000, dneed - 1, None) == 4
+    assert L.fasa_dense_decode(c, 100, 0x50000, 100, 0x70000, None, dneed, None) == 4
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
