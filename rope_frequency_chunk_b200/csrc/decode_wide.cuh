@@ -53,9 +53,11 @@ constexpr int kWdThreads = kSAThreads;  // 512 (the histogram and radix helpers'
 constexpr int kWdWarps = kWdThreads / 32;
 constexpr int kWdMaxLoc = 16384;        // tokens per CTA (their keys live in shared memory)
 constexpr int kWdTieCap = 2048;         // boundary-bin entries held in shared memory
-constexpr int kWdRankMax = 512;         // boundary-bin entries resolved by rank counting
+constexpr int kWdRankMax = 128;         // entries of the finest bin resolved by rank counting
+constexpr int kWdUnionUnroll = 8;       // union entries in flight per thread
 constexpr int kWdMaxDirect = 512;       // kept rows the resolving CTA attends itself
-constexpr int kWdRadixWords = kSAWarps * 256 + 256 + 8;
+// radix scratch: the sub-bin histogram and entries, then ballot_radix_fn's
+constexpr int kWdRadixWords = 256 + 2 * 128 + kSAWarps * 256 + 264;
 constexpr int kWdMisc = 128;            // words of scan and flag scratch
 
 struct WideParams {
@@ -163,24 +165,28 @@ __device__ __forceinline__ void wd_keep(uint32_t* bm, uint32_t t, int len) {
   if (t < (uint32_t)len) atomicOr(bm + (t >> 5), 1u << (t & 31));
 }
 
-// Exact choice of the `need` largest keys among the entries of bin B (ties to
-// the lower token index), by two radix selects: the need-th key K, then, if
-// only some of the keys equal to K fit, the lowest token indices among them.
-// entry_at(i) gives entry i of n (any entries; only bin B's take part).
+// Exact choice of the `need` largest keys among the entries whose top
+// `known` key bits equal those of `prefix` (ties to the lower token index), by
+// two radix selects: the need-th key K, then, if only some of the keys equal
+// to K fit, the lowest token indices among them. entry_at(i) gives entry i
+// of n (any entries; only the prefix's take part). rscr: kSAWarps * 256 +
+// 258 words.
 template <typename At>
-__device__ void wd_resolve_radix(At entry_at, int n, int need, uint32_t B, uint32_t* rscr, uint32_t* misc,
-                                 uint32_t* bm, int len) {
+__device__ void wd_resolve_radix(At entry_at, int n, int need, uint32_t prefix, int known, uint32_t* rscr,
+                                 uint32_t* misc, uint32_t* bm, int len) {
   cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x;
   uint32_t K = 0;
   int krem = 0;
-  ballot_radix_fn<false>([&](int i) { return entry_at(i).x; }, n, need, B << 20, 12, 32, rscr, nullptr, cl, K, krem);
-  // keys above K in bin B are kept; count the keys equal to K
+  ballot_radix_fn<false>([&](int i) { return entry_at(i).x; }, n, need, prefix, known, 32, rscr, nullptr, cl, K,
+                         krem);
+  // keys above K with the prefix are kept; count the keys equal to K
+  const uint32_t pmask = ~0u << (32 - known);
   if (tid == 0) misc[0] = 0u;
   __syncthreads();
   for (int i = tid; i < n; i += kWdThreads) {
     const uint2 e = entry_at(i);
-    if ((e.x >> 20) == B && e.x > K) wd_keep(bm, e.y, len);
+    if ((e.x & pmask) == prefix && e.x > K) wd_keep(bm, e.y, len);
     if (e.x == K) atomicAdd(misc, 1u);
   }
   __syncthreads();
@@ -204,6 +210,38 @@ __device__ void wd_resolve_radix(At entry_at, int n, int need, uint32_t B, uint3
   for (int i = tid; i < n; i += kWdThreads) {
     const uint2 e = entry_at(i);
     if (e.x == K && ~e.y >= T) wd_keep(bm, e.y, len);
+  }
+}
+
+// One warp: in the 256-bin histogram h, the bin holding the k-th largest
+// (k <= total) and the count in higher bins, written to out[0], out[1].
+// Lane l owns bins 255 - 8l .. 248 - 8l.
+__device__ __forceinline__ void wd_warp_bin256(const uint32_t* h, int k, uint32_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t c[8], sum = 0u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    c[u] = h[255 - (8 * lane + u)];
+    sum += c[u];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  const uint32_t excl = incl - sum;
+  if (excl < (uint32_t)k && (uint32_t)k <= incl) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (acc + c[u] >= (uint32_t)k) {
+        out[0] = 255u - (uint32_t)(8 * lane + u);
+        out[1] = acc;
+        break;
+      }
+      acc += c[u];
+    }
   }
 }
 
@@ -509,11 +547,30 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
   if (tid == 0) misc[100] = 0u;
   __syncthreads();
-  for (int i = tid; i < nu; i += kWdThreads) {
-    const uint2 e = __ldcg(crow + i);
+  // union entries: global loads batched so that many are in flight
+  auto for_union = [&](auto&& fn, bool from_cache) {
+    if (from_cache) {
+      for (int i = tid; i < nu; i += kWdThreads) fn(i, uc[i]);
+      return;
+    }
+    for (int base = 0; base < nu; base += kWdThreads * kWdUnionUnroll) {
+      uint2 e[kWdUnionUnroll];
+#pragma unroll
+      for (int u = 0; u < kWdUnionUnroll; ++u) {
+        const int i = base + u * kWdThreads + tid;
+        e[u] = i < nu ? __ldcg(crow + i) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kWdUnionUnroll; ++u) {
+        const int i = base + u * kWdThreads + tid;
+        if (i < nu) fn(i, e[u]);
+      }
+    }
+  };
+  for_union([&](int i, const uint2& e) {
     if (cached) uc[i] = e;
     atomicAdd(hist + (e.x >> 20), 1u);
-  }
+  }, false);
   __syncthreads();
   int n_keep = p.n_keep;
   if (nu < n_keep) {  // only a workspace that was not zero gets here
@@ -522,8 +579,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   uint32_t B = 0u, above = 0u;
   if (n_keep > 0) hist_threshold_fn([&](int i) { return hist[i]; }, n_keep, misc, B, above);
-  for (int i = tid; i < nu; i += kWdThreads) {
-    const uint2 e = cached ? uc[i] : __ldcg(crow + i);
+  for_union([&](int, const uint2& e) {
     const uint32_t b = e.x >> 20;
     if (b > B) {
       wd_keep(bm, e.y, p.len);
@@ -531,7 +587,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       const uint32_t at = atomicAdd(misc + 100, 1u);
       if (at < (uint32_t)kWdTieCap) ties[at] = e;
     }
-  }
+  }, cached);
   __syncthreads();
   const int n_b = (int)misc[100];
   const int need = n_keep - (int)above;
@@ -539,22 +595,56 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   if (need > 0 && n_keep > 0) {
     if (n_b == need && n_b <= kWdTieCap) {
       for (int i = tid; i < n_b; i += kWdThreads) wd_keep(bm, ties[i].y, p.len);
-    } else if (n_b <= kWdRankMax) {
-      for (int i = tid; i < n_b; i += kWdThreads) {
-        const uint2 a = ties[i];
-        int r = 0;
-        for (int j = 0; j < n_b; ++j) {
-          const uint2 c = ties[j];
-          r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
-        }
-        if (r < need) wd_keep(bm, a.y, p.len);
-      }
     } else if (n_b <= kWdTieCap) {
-      wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need, B, rscr, misc, bm, p.len);
+      // next 8 key bits of the boundary bin's entries, then ranks (or a
+      // radix select) among the entries of the boundary sub-bin
+      uint32_t* h2 = rscr;             // 256 counts
+      uint2* t2 = reinterpret_cast<uint2*>(rscr + 256);  // the sub-bin's entries
+      for (int i = tid; i < 256; i += kWdThreads) h2[i] = 0u;
+      if (tid == 0) misc[101] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n_b; i += kWdThreads) atomicAdd(h2 + ((ties[i].x >> 12) & 255u), 1u);
+      __syncthreads();
+      if (warp == 0) wd_warp_bin256(h2, need, misc + 102);
+      __syncthreads();
+      const uint32_t B2 = misc[102];
+      const int need2 = need - (int)misc[103];
+      for (int i = tid; i < n_b; i += kWdThreads) {
+        const uint2 e = ties[i];
+        const uint32_t sb = (e.x >> 12) & 255u;
+        if (sb > B2) {
+          wd_keep(bm, e.y, p.len);
+        } else if (sb == B2) {
+          const uint32_t at = atomicAdd(misc + 101, 1u);
+          if (at < (uint32_t)kWdRankMax) t2[at] = e;
+        }
+      }
+      __syncthreads();
+      const int n_b2 = (int)misc[101];
+      __syncthreads();
+      if (n_b2 == need2 && n_b2 <= kWdRankMax) {
+        for (int i = tid; i < n_b2; i += kWdThreads) wd_keep(bm, t2[i].y, p.len);
+      } else if (n_b2 <= kWdRankMax) {
+        for (int i = tid; i < n_b2; i += kWdThreads) {
+          const uint2 a = t2[i];
+          int r = 0;
+          for (int j = 0; j < n_b2; ++j) {
+            const uint2 c = t2[j];
+            r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
+          }
+          if (r < need2) wd_keep(bm, a.y, p.len);
+        }
+      } else {
+        // a crowded sub-bin (ties): exact radix select over the boundary
+        // bin's entries, restricted to the sub-bin by its 20-bit prefix
+        const uint32_t pre = (B << 20) | (B2 << 12);
+        wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need2, pre, 20, rscr + 256 + 2 * kWdRankMax, misc,
+                         bm, p.len);
+      }
     } else if (cached) {
-      wd_resolve_radix([&](int i) { return uc[i]; }, nu, need, B, rscr, misc, bm, p.len);
+      wd_resolve_radix([&](int i) { return uc[i]; }, nu, need, B << 20, 12, rscr, misc, bm, p.len);
     } else {
-      wd_resolve_radix([&](int i) { return __ldcg(crow + i); }, nu, need, B, rscr, misc, bm, p.len);
+      wd_resolve_radix([&](int i) { return __ldcg(crow + i); }, nu, need, B << 20, 12, rscr, misc, bm, p.len);
     }
   }
   __syncthreads();

@@ -363,7 +363,9 @@ fasa_status wide_attrs(const DevInfo& d) {
 bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl) {
   if (c->dtype != FASA_BF16) return false;
   const int64_t rows = (int64_t)c->batch * c->n_kv_heads;
-  int64_t S = std::max<int64_t>(1, (d.sms + rows / 2) / rows);
+  // about one CTA per SM, leaving one SM per row free: the rows' resolving
+  // CTAs then never hold back a CTA of the next launch
+  int64_t S = std::max<int64_t>(1, (d.sms - std::min<int64_t>(rows, d.sms / 2)) / rows);
   S = std::max<int64_t>(S, ceil_div(len, kWdMaxLoc));
   S = std::min<int64_t>(S, std::max<int64_t>(1, ceil_div(len, 256)));
   pl->n_split = (int)S;
