@@ -1,0 +1,389 @@
+// Focused attention on CUDA cores (bf16 caches): flash decode in float32.
+//
+// "FASA: Frequency-aware Sparse Attention" (gist.science technical summary,
+// §2, FAC bullets): full softmax attention of each query head of a KV-head
+// group over exactly the kept rows, each row at its original position (keys
+// were rotated at append time). The dense comparison decode is the same
+// attention over every row ([tech §4] "Resultados Experimentais", FKV).
+//
+// Decode attention has G (<= 16) query rows per KV head, so QK^T and PV are
+// matrix-vector products at about G flops per byte: the path is bound by
+// HBM, and float32 fma on CUDA cores keeps up with it at these group sizes.
+//
+// Warp step: 8 rows. Lane l owns head dims 4l .. 4l+3: it loads those 8
+// bytes of each K and V row (a warp reads whole 256-byte rows, coalesced),
+// forms the partial dot products of its 4 dims with every head's query (an
+// fma chain), and a reduce-scatter butterfly over the 32 lanes (5 rounds of
+// shuffles, each halving the values a lane holds) leaves lane l with the
+// full logit of (row l/4, head 4g + l%4) for head group g. Online softmax in
+// base 2 (the 1/sqrt(128) and log2(e) scale is folded into the queries):
+// per-head chunk maxima and sums by shuffles among the lanes of one head,
+// running (m, l) in the warp's shared-memory scratch, probabilities
+// broadcast through it; o[h][4l..4l+3] += p * v in registers.
+//
+// Error: a logit is a float32 sum of 128 products (query rounded once from
+// float64; keys exact) along a 4-fma chain and a 5-level tree, so its error
+// is below 10 * 2^-24 * sum_d |q_d k_d|; probabilities and the output
+// accumulate in float32.
+#pragma once
+
+#include "fasa_device.cuh"
+
+namespace fasa {
+
+constexpr int kCcStep = 8;  // rows per warp step
+
+// Per-warp shared-memory scratch (floats): p[8][MG], then running max, sum
+// and the last rescale factor per head.
+__host__ __device__ constexpr int cc_warp_scratch(int MG) { return (kCcStep + 3) * MG; }
+
+// Attention queries of one KV-head group, [MG][128] floats: query h rotated
+// at the query position and scaled by log2(e)/sqrt(128), in float64, rounded
+// to float32; rows h >= G are zero. qraw: the group's G pre-RoPE rows.
+template <typename T>
+__device__ __forceinline__ void cc_queries(const T* qraw, int G, int MG, const double* cosv, const double* sinv,
+                                           float* qs, int tid, int nthreads) {
+  const double qscale = 1.4426950408889634 / 11.313708498984761;
+  for (int e = tid; e < MG * kD; e += nthreads) {
+    const int h = e / kD, dd = e % kD, i = dd & (kNFC - 1);
+    float v = 0.0f;
+    if (h < G) {
+      const double x = to_float(qraw[h * kD + i]);
+      const double y = to_float(qraw[h * kD + i + kNFC]);
+      const double c = cosv[i], s = sinv[i];
+      const double r = (dd < kNFC) ? __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s))
+                                   : __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s));
+      v = (float)(r * qscale);
+    }
+    qs[e] = v;
+  }
+}
+
+// A warp's running attention state: o for the lane's 4 dims of every head
+// (the running max and sum live in the warp's scratch).
+template <int MG>
+struct CcAcc {
+  float o[MG][4];
+};
+
+template <int MG>
+__device__ __forceinline__ void cc_init(CcAcc<MG>& a, float* ws, int lane) {
+#pragma unroll
+  for (int h = 0; h < MG; ++h)
+#pragma unroll
+    for (int d = 0; d < 4; ++d) a.o[h][d] = 0.0f;
+  float* wm = ws + kCcStep * MG;
+  for (int h = lane; h < MG; h += 32) {
+    wm[h] = -INFINITY;
+    wm[MG + h] = 0.0f;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void cc_bf16x4(const uint2& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x << 16);
+  f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+
+// One step of 8 rows: kk[r], vv[r] are the lane's 8 bytes of K and V row r;
+// bit r of `valid` says whether row r takes part. qs: [MG][128] queries;
+// ws: the warp's scratch (cc_warp_scratch floats).
+template <int MG>
+__device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep], const uint2 (&vv)[kCcStep],
+                                         unsigned valid, const float* qs, float* ws, int lane) {
+  constexpr int NG = MG / 4;
+  float* wp = ws;                    // p[8][MG]
+  float* wm = ws + kCcStep * MG;     // running max [MG]
+  float* wl = wm + MG;               // running sum [MG]
+  float* wsc = wl + MG;              // rescale of this step [MG]
+  float kf[kCcStep][4];
+#pragma unroll
+  for (int r = 0; r < kCcStep; ++r) cc_bf16x4(kk[r], kf[r]);
+  const int r_me = lane >> 2;           // the row and head (within a group) whose logit this lane ends with
+  const bool row_ok = (valid >> r_me) & 1u;
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    float v[32];  // index r * 4 + hh
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + hh) * kD + 4 * lane);
+#pragma unroll
+      for (int r = 0; r < kCcStep; ++r)
+        v[r * 4 + hh] = __fmaf_rn(q4.w, kf[r][3], __fmaf_rn(q4.z, kf[r][2], __fmaf_rn(q4.y, kf[r][1],
+                                                                                    __fmul_rn(q4.x, kf[r][0]))));
+    }
+    // reduce-scatter: after the round with offset o the lane keeps the half
+    // of its values whose index bit matches its own lane bit o
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+      const int off = 16 >> s, half = 16 >> s;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = __fadd_rn(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
+      }
+    }
+    const int h = g * 4 + (lane & 3);
+    const float z = row_ok ? v[0] : -INFINITY;
+    float cm = z;
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 4));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 8));
+    cm = fmaxf(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 16));
+    const float mold = wm[h];
+    const float mnew = fmaxf(mold, cm);
+    const float p = (z == -INFINITY) ? 0.0f : exp2f(z - mnew);
+    float cs = p;
+    cs += __shfl_xor_sync(0xFFFFFFFFu, cs, 4);
+    cs += __shfl_xor_sync(0xFFFFFFFFu, cs, 8);
+    cs += __shfl_xor_sync(0xFFFFFFFFu, cs, 16);
+    const float sc = (mold == -INFINITY) ? 0.0f : exp2f(mold - mnew);
+    wp[r_me * MG + h] = p;
+    __syncwarp();
+    if (lane < 4) {
+      wm[h] = mnew;
+      wl[h] = wl[h] * sc + cs;
+      wsc[h] = sc;
+    }
+  }
+  __syncwarp();
+  // rescale, then o += p v
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const float4 s4 = *reinterpret_cast<const float4*>(wsc + g * 4);
+    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh)
+#pragma unroll
+      for (int d = 0; d < 4; ++d) a.o[g * 4 + hh][d] *= sv[hh];
+  }
+#pragma unroll
+  for (int r = 0; r < kCcStep; ++r) {
+    float vf[4];
+    cc_bf16x4(vv[r], vf);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const float4 p4 = *reinterpret_cast<const float4*>(wp + r * MG + g * 4);
+      const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh)
+#pragma unroll
+        for (int d = 0; d < 4; ++d) a.o[g * 4 + hh][d] = __fmaf_rn(pv[hh], vf[d], a.o[g * 4 + hh][d]);
+    }
+  }
+  __syncwarp();
+}
+
+// A warp attends rows j0 .. j1-1 of a list: token(j) gives the cache slot
+// of list position j, or -1 for a position to skip. kb, vb: the row's K and
+// V planes [max_len][128]. With kPipe the next step's rows are loaded before
+// the current step is computed (two register buffers).
+template <int MG, bool kPipe, typename Tok>
+__device__ __forceinline__ void cc_warp_rows(CcAcc<MG>& a, const __nv_bfloat16* kb, const __nv_bfloat16* vb,
+                                             Tok token, int j0, int j1, const float* qs, float* ws, int lane) {
+  auto load = [&](uint2 (&kk)[kCcStep], uint2 (&vv)[kCcStep], unsigned& valid, int jb) {
+    const int mine = (lane < kCcStep && jb + lane < j1) ? token(jb + lane) : -1;
+    valid = __ballot_sync(0xFFFFFFFFu, mine >= 0) & 0xFFu;
+#pragma unroll
+    for (int r = 0; r < kCcStep; ++r) {
+      int t = __shfl_sync(0xFFFFFFFFu, mine, r);
+      if (t < 0) t = 0;  // masked out; row 0 is a valid address
+      kk[r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t * kD) + lane);
+      vv[r] = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t * kD) + lane);
+    }
+  };
+  if (j0 >= j1) return;
+  uint2 k0[kCcStep], v0[kCcStep];
+  unsigned m0;
+  if constexpr (kPipe) {
+    uint2 k1[kCcStep], v1[kCcStep];
+    unsigned m1;
+    load(k0, v0, m0, j0);
+    for (int jb = j0; jb < j1; jb += 2 * kCcStep) {
+      if (jb + kCcStep < j1) load(k1, v1, m1, jb + kCcStep);
+      cc_step8<MG>(a, k0, v0, m0, qs, ws, lane);
+      if (jb + kCcStep >= j1) break;
+      if (jb + 2 * kCcStep < j1) load(k0, v0, m0, jb + 2 * kCcStep);
+      cc_step8<MG>(a, k1, v1, m1, qs, ws, lane);
+    }
+  } else {
+    for (int jb = j0; jb < j1; jb += kCcStep) {
+      load(k0, v0, m0, jb);
+      cc_step8<MG>(a, k0, v0, m0, qs, ws, lane);
+    }
+  }
+}
+
+// Merges the nw warps' states of a CTA in shared memory. Warp w writes its
+// o to mo[w][MG][128] and its (m, l) are in its scratch ws0 + w * stride;
+// afterwards thread tid < MG*128 ... handles output element e = tid (and
+// e + nthreads ...): returns nothing, calls emit(h, d, m, l, o) once per
+// element (head h, dim d) with the merged state. Must be called by every
+// thread of the CTA.
+template <int MG, typename Emit>
+__device__ __forceinline__ void cc_block_merge(const CcAcc<MG>& a, float* mo, const float* ws0, int ws_stride, int nw,
+                                               Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = nw * 32;
+#pragma unroll
+  for (int h = 0; h < MG; ++h)
+    *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) =
+        make_float4(a.o[h][0], a.o[h][1], a.o[h][2], a.o[h][3]);
+  __syncthreads();
+  for (int e = tid; e < MG * kD; e += nthreads) {
+    const int h = e / kD, d = e % kD;
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, ws0[w * ws_stride + kCcStep * MG + h]);
+    float L = 0.0f, O = 0.0f;
+    for (int w = 0; w < nw; ++w) {
+      const float mw = ws0[w * ws_stride + kCcStep * MG + h];
+      const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+      L += f * ws0[w * ws_stride + kCcStep * MG + MG + h];
+      O += f * mo[(w * MG + h) * kD + d];
+    }
+    emit(h, d, M, L, O);
+  }
+}
+
+}  // namespace fasa
+
+namespace fasa {
+
+constexpr int kCcWarps = 8;
+constexpr int kCcThreads = kCcWarps * 32;
+constexpr int kCcPartStride = 16 * kD + 32;  // floats per split partial: m[16], l[16], o[16][128]
+
+struct CcParams {
+  const __nv_bfloat16* k;   // [rows][max_len][128]
+  const __nv_bfloat16* v;
+  const int32_t* idx;       // [rows][n_keep] kept rows, or null: rows 0 .. n_keep-1 (dense)
+  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
+  __nv_bfloat16* out;       // [B][Hq][128]
+  float* part;              // [rows][splits][kCcPartStride]
+  uint32_t* counter;        // [rows], zero before the launch; the last CTA of a row leaves it zero
+  int64_t max_len;
+  int32_t len;              // kept indices must lie in [0, len)
+  int32_t n_keep;
+  int32_t slice;            // list positions per CTA, a multiple of 8 * kCcWarps
+  int32_t splits;
+  int32_t group;
+  double cosv[kNFC];        // cos / sin of q_pos * theta_i
+  double sinv[kNFC];
+};
+
+// Shared memory of attend_cc_kernel: group queries (raw), queries (scaled
+// float32), warp scratch, warp partials; the split merge reuses the partials.
+__host__ __device__ constexpr int cc_smem_bytes(int MG) {
+  return FASA_MAX_GROUP * kD * 2 + MG * kD * 4 + kCcWarps * cc_warp_scratch(MG) * 4 + kCcWarps * MG * kD * 4;
+}
+constexpr int kCcMaxSplits = (kCcWarps * 4 * kD * 4) / (3 * 16 * 4);  // the merge state fits the MG = 4 partials
+
+// Split-K attention over a row's kept list (or all its rows): grid
+// (splits, rows); CTA `split` takes list positions [split*slice, ...), its
+// 8 warps contiguous eighths of them; the warps merge in shared memory, the
+// CTA writes its partial (m, l, o) and the row's last CTA (atomic ticket, no
+// waiting) merges the splits in a fixed order and writes the output.
+template <int MG>
+__global__ void __launch_bounds__(kCcThreads) attend_cc_kernel(const CcParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
+  float* qs = reinterpret_cast<float*>(smem + FASA_MAX_GROUP * kD * 2);
+  float* wsall = qs + MG * kD;
+  float* mo = wsall + kCcWarps * cc_warp_scratch(MG);
+  grid_dependency_wait();
+  const int split = blockIdx.x, row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.group;
+  {
+    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
+    for (int c = tid; c < G * kD / 8; c += kCcThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+  }
+  __syncthreads();
+  cc_queries(qraw, G, MG, p.cosv, p.sinv, qs, tid, kCcThreads);
+  __syncthreads();
+  float* ws = wsall + warp * cc_warp_scratch(MG);
+  CcAcc<MG> acc;
+  cc_init<MG>(acc, ws, lane);
+  const int r_beg = split * p.slice, r_end = min(p.n_keep, r_beg + p.slice);
+  const int per_warp = ((max(0, r_end - r_beg) + kCcWarps * kCcStep - 1) / (kCcWarps * kCcStep)) * kCcStep;
+  const int j0 = min(r_end, r_beg + warp * per_warp), j1 = min(r_end, j0 + per_warp);
+  const __nv_bfloat16* kb = p.k + (int64_t)row * p.max_len * kD;
+  const __nv_bfloat16* vb = p.v + (int64_t)row * p.max_len * kD;
+  const int32_t* idx = p.idx ? p.idx + (int64_t)row * p.n_keep : nullptr;
+  cc_warp_rows<MG, true>(acc, kb, vb, [&](int j) -> int {
+    const int t = idx ? __ldg(idx + j) : j;
+    if (t < 0 || t >= p.len) {
+      flag_status(FASA_ERR_BAD_INDEX);
+      return -1;
+    }
+    return t;
+  }, j0, j1, qs, ws, lane);
+  __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
+  float* pp = p.part + ((int64_t)row * p.splits + split) * kCcPartStride;
+  const bool single = p.splits == 1;
+  cc_block_merge<MG>(acc, mo, wsall, cc_warp_scratch(MG), kCcWarps, [&](int h, int d, float M, float L, float O) {
+    if (single) {
+      if (h < G) out[h * kD + d] = __float2bfloat16_rn(L > 0.0f ? O / L : 0.0f);
+    } else {
+      pp[32 + h * kD + d] = O;
+      if (d == 0) {
+        pp[h] = M;
+        pp[16 + h] = L;
+      }
+    }
+  });
+  if (single) return;
+  // the row's last CTA merges all splits
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(p.counter + row, 1u) == (uint32_t)(p.splits - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* rp = p.part + (int64_t)row * p.splits * kCcPartStride;
+  float* sm_m = mo;                        // [splits][16]
+  float* sm_l = sm_m + p.splits * 16;      // [splits][16]
+  float* sm_w = sm_l + p.splits * 16;      // [splits][16] weights
+  float* sm_den = sm_w + p.splits * 16;    // [16]
+  for (int i = tid; i < p.splits * 16; i += kCcThreads) {
+    sm_m[i] = __ldcg(rp + (i / 16) * kCcPartStride + i % 16);
+    sm_l[i] = __ldcg(rp + (i / 16) * kCcPartStride + 16 + i % 16);
+  }
+  __syncthreads();
+  if (tid < 16) {
+    float M = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, sm_m[s * 16 + tid]);
+    float den = 0.0f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float ms = sm_m[s * 16 + tid];
+      const float w = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
+      sm_w[s * 16 + tid] = w;
+      den += w * sm_l[s * 16 + tid];
+    }
+    sm_den[tid] = den;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * kD; e += kCcThreads) {
+    const int h = e / kD;
+    float num = 0.0f;
+    int s = 0;
+    for (; s + 4 <= p.splits; s += 4) {
+      const float v0 = __ldcg(rp + (s + 0) * kCcPartStride + 32 + e);
+      const float v1 = __ldcg(rp + (s + 1) * kCcPartStride + 32 + e);
+      const float v2 = __ldcg(rp + (s + 2) * kCcPartStride + 32 + e);
+      const float v3 = __ldcg(rp + (s + 3) * kCcPartStride + 32 + e);
+      num += sm_w[(s + 0) * 16 + h] * v0 + sm_w[(s + 1) * 16 + h] * v1 + sm_w[(s + 2) * 16 + h] * v2 +
+             sm_w[(s + 3) * 16 + h] * v3;
+    }
+    for (; s < p.splits; ++s) num += sm_w[s * 16 + h] * __ldcg(rp + s * kCcPartStride + 32 + e);
+    const float den = sm_den[h];
+    out[e] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
+  }
+  if (tid == 0) p.counter[row] = 0u;
+}
+
+}  // namespace fasa

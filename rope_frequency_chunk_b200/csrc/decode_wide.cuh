@@ -31,10 +31,10 @@
 //        are kept, ties to the lower token index (rank counting for a few,
 //        else an exact radix select);
 //      - a bitmap of the kept tokens emits them in ascending order;
-//      - with `direct` the same CTA attends them on tensor cores (mma.sync,
-//        the split-K kernel's per-warp chunk step, one chunk per warp at a
-//        time) and merges its warps; otherwise it writes the kept list and
-//        the query terms for attend_mma_kernel, launched next.
+//      - with `direct` (k_eff <= 512, G <= 8) the same CTA attends them on
+//        CUDA cores (attend_cc.cuh: each warp a contiguous part of the kept
+//        list, then the warps merged); otherwise it writes the kept list for
+//        attend_cc_kernel, launched next.
 //
 // Semaphore: sem[row] = (tickets << 32) | entries reserved. It must be zero
 // when a call starts; the last CTA of the row writes it back to zero, so a
@@ -43,7 +43,7 @@
 // never written out of bounds.
 #pragma once
 
-#include "attend_mma.cuh"
+#include "attend_cc.cuh"
 #include "select_attend.cuh"
 #include "tip.cuh"
 
@@ -69,7 +69,6 @@ struct WideParams {
   __nv_bfloat16* out;           // [B][Hq][128]
   int32_t* idx_out;             // [rows][n_keep] kept tokens, ascending, or null
   int32_t* idx_ws;              // [rows][n_keep] for the attention launch, or null (direct)
-  unsigned char* qterms;        // [rows][kQTermBytes] for the attention launch, or null (direct)
   uint2* cand;                  // [rows][len] published (key, token) pairs
   unsigned long long* sem;      // [rows], zero between calls
   int64_t max_len;
@@ -82,7 +81,7 @@ struct WideParams {
   int32_t n_loc;    // tokens per CTA, <= kWdMaxLoc
   int32_t n_split;  // CTAs per row
   int32_t ucache;   // union entries the resolving CTA caches in shared memory
-  int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect)
+  int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect, G <= 8)
   double cosv[kNFC];
   double sinv[kNFC];
 };
@@ -120,12 +119,14 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   b += wd_al(kWdRadixWords * 4, 16);
   L.ucache = o + b;
   b += ucache * 8;
+  // the attention: queries [MG][128] f32, warp scratch, warp partials [16][MG][128] f32
+  const int MG = group <= 4 ? 4 : 8;
   L.qt = o;
   int c = 0;
   if (direct) {
-    c = wd_al((3 * group + 1) * 256, 128);
+    c = MG * kD * 4 + kWdWarps * cc_warp_scratch(MG) * 4;
     L.ring = o + c;
-    c += kWdWarps * kAttStageBytes;
+    c += kWdWarps * MG * kD * 4;
   } else {
     L.ring = o;
   }
@@ -245,175 +246,7 @@ __device__ __forceinline__ void wd_warp_bin256(const uint32_t* h, int k, uint32_
   }
 }
 
-// Softmax attention of the group's query heads over the n kept rows in
-// `kept` (shared memory, ascending), one 16-row chunk per warp at a time,
-// the warps merged as a tree; writes out[h][d] for the G heads.
-__device__ void wd_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, const int* kept, int n,
-                          const unsigned char* qt, int G, unsigned char* ring, __nv_bfloat16* out) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  unsigned char* st = ring + warp * kAttStageBytes;
-  const int nchunks = (n + kAttChunk - 1) / kAttChunk;
-  float o[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[j][e] = 0.0f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // heads lane/4 and lane/4 + 8
-  for (int ci = warp; ci < nchunks; ci += kWdWarps) {
-    const int j0 = ci * kAttChunk;
-    const int tr = (lane < kAttChunk && j0 + lane < n) ? kept[j0 + lane] : 0;
-#pragma unroll
-    for (int r = 0; r < kAttChunk; ++r) {  // 16 rows x (16 K + 16 V) 16-byte parts, one part per lane
-      const int t = __shfl_sync(0xFFFFFFFFu, tr, r);
-      const __nv_bfloat16* src = (lane < 16 ? kb : vb) + (int64_t)t * kD + (lane % 16) * 8;
-      cp_async16(st + (lane < 16 ? 0 : kAttHalf) + r * 256 + (((lane % 16) ^ (r & 7)) * 16), src);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
-    const unsigned char* Ks = st;
-    const unsigned char* Vs = st + kAttHalf;
-    float s0[4], s1[4];
-    chunk_logits(qt, G, Ks, lane, s0, s1);
-    const int c0 = (lane % 4) * 2;
-    if (j0 + c0 >= n) s0[0] = s0[2] = -INFINITY;
-    if (j0 + c0 + 1 >= n) s0[1] = s0[3] = -INFINITY;
-    if (j0 + 8 + c0 >= n) s1[0] = s1[2] = -INFINITY;
-    if (j0 + 8 + c0 + 1 >= n) s1[1] = s1[3] = -INFINITY;
-    float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
-    float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float sc0 = (m0 == -INFINITY) ? 0.0f : exp2f(m0 - n0);
-    const float sc1 = (m1 == -INFINITY) ? 0.0f : exp2f(m1 - n1);
-    float pr[8];
-    pr[0] = s0[0] == -INFINITY ? 0.f : exp2f(s0[0] - n0);
-    pr[1] = s0[1] == -INFINITY ? 0.f : exp2f(s0[1] - n0);
-    pr[2] = s0[2] == -INFINITY ? 0.f : exp2f(s0[2] - n1);
-    pr[3] = s0[3] == -INFINITY ? 0.f : exp2f(s0[3] - n1);
-    pr[4] = s1[0] == -INFINITY ? 0.f : exp2f(s1[0] - n0);
-    pr[5] = s1[1] == -INFINITY ? 0.f : exp2f(s1[1] - n0);
-    pr[6] = s1[2] == -INFINITY ? 0.f : exp2f(s1[2] - n1);
-    pr[7] = s1[3] == -INFINITY ? 0.f : exp2f(s1[3] - n1);
-    l0 = l0 * sc0 + (pr[0] + pr[1] + pr[4] + pr[5]);
-    l1 = l1 * sc1 + (pr[2] + pr[3] + pr[6] + pr[7]);
-    m0 = n0;
-    m1 = n1;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      o[j][0] *= sc0;
-      o[j][1] *= sc0;
-      o[j][2] *= sc1;
-      o[j][3] *= sc1;
-    }
-    uint32_t ph[4], pl[4];
-    split_pack(pr[0], pr[1], ph[0], pl[0]);
-    split_pack(pr[2], pr[3], ph[1], pl[1]);
-    split_pack(pr[4], pr[5], ph[2], pl[2]);
-    split_pack(pr[6], pr[7], ph[3], pl[3]);
-#pragma unroll
-    for (int j = 0; j < 16; j += 2) {
-      uint32_t b[4];
-      ldsm_x4_t(b, Vs + (((lane / 8) % 2) * 8 + lane % 8) * 256 + (((j + lane / 16) ^ (lane % 8)) * 16));
-      mma_16816(o[j], ph, b[0], b[1]);
-      mma_16816(o[j], pl, b[0], b[1]);
-      mma_16816(o[j + 1], ph, b[2], b[3]);
-      mma_16816(o[j + 1], pl, b[2], b[3]);
-    }
-    __syncwarp();
-  }
-  // warps merged as a tree in the ring (of the cnt warps still holding a
-  // partial, warps [h, cnt) hand theirs to warps [0, cnt - h))
-  float* slots = reinterpret_cast<float*>(ring);
-#pragma unroll 1
-  for (int cnt = kWdWarps; cnt > 1;) {
-    const int h = (cnt + 1) / 2;
-    __syncthreads();
-    if (warp >= h && warp < cnt) {
-      float* sl = slots + (warp - h) * kAttSlot;
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sl[(j * 4 + e) * 32 + lane] = o[j][e];
-      sl[64 * 32 + lane] = m0;
-      sl[65 * 32 + lane] = m1;
-      sl[66 * 32 + lane] = l0;
-      sl[67 * 32 + lane] = l1;
-    }
-    __syncthreads();
-    if (warp < cnt - h) {
-      const float* sl = slots + warp * kAttSlot;
-      const float pm0 = sl[64 * 32 + lane], pm1 = sl[65 * 32 + lane];
-      const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
-      const float a0 = (m0 == -INFINITY) ? 0.0f : exp2f(m0 - n0), a1 = (m1 == -INFINITY) ? 0.0f : exp2f(m1 - n1);
-      const float b0 = (pm0 == -INFINITY) ? 0.0f : exp2f(pm0 - n0), b1 = (pm1 == -INFINITY) ? 0.0f : exp2f(pm1 - n1);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        o[j][0] = o[j][0] * a0 + sl[(j * 4 + 0) * 32 + lane] * b0;
-        o[j][1] = o[j][1] * a0 + sl[(j * 4 + 1) * 32 + lane] * b0;
-        o[j][2] = o[j][2] * a1 + sl[(j * 4 + 2) * 32 + lane] * b1;
-        o[j][3] = o[j][3] * a1 + sl[(j * 4 + 3) * 32 + lane] * b1;
-      }
-      l0 = l0 * a0 + sl[66 * 32 + lane] * b0;
-      l1 = l1 * a1 + sl[67 * 32 + lane] * b1;
-      m0 = n0;
-      m1 = n1;
-    }
-    cnt = h;
-  }
-  if (warp == 0) {
-    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
-    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
-    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
-    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
-    const int h0 = lane / 4, h1 = lane / 4 + 8;
-    const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int d = j * 8 + (lane % 4) * 2;
-      if (h0 < G)
-        *reinterpret_cast<__nv_bfloat162*>(out + h0 * kD + d) = __floats2bfloat162_rn(o[j][0] * i0, o[j][1] * i0);
-      if (h1 < G)
-        *reinterpret_cast<__nv_bfloat162*>(out + h1 * kD + d) = __floats2bfloat162_rn(o[j][2] * i1, o[j][3] * i1);
-    }
-  }
-}
-
-// The attention query terms in the compact shared-memory layout chunk_logits
-// reads: term t (low, middle, high) of head r at row t*G + r, then a zero
-// row at 3G; the values are query_terms' bit for bit.
-__device__ __forceinline__ void wd_query_terms(const __nv_bfloat16* qraw, int G, const double* cosv,
-                                               const double* sinv, unsigned char* qt) {
-  const int tid = threadIdx.x;
-  const double qscale = 1.4426950408889634 / 11.313708498984761;
-  for (int e = tid; e < G * (kD / 2); e += kWdThreads) {
-    const int h = e / (kD / 2), d = 2 * (e % (kD / 2));
-    float v2[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int dd = d + u, i = dd & (kNFC - 1);
-      const double x = __bfloat162float(qraw[h * kD + i]);
-      const double y = __bfloat162float(qraw[h * kD + i + kNFC]);
-      const double c = cosv[i], sn = sinv[i];
-      v2[u] = (float)(((dd < kNFC) ? (x * c - y * sn) : (y * c + x * sn)) * qscale);
-    }
-    uint32_t hi, mid, lo;
-    const float2 r = split_pack(v2[0], v2[1], hi, mid);
-    const float2 mf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&mid));
-    const __nv_bfloat162 ll = __floats2bfloat162_rn(r.x - mf.x, r.y - mf.y);
-    lo = *reinterpret_cast<const uint32_t*>(&ll);
-    const int off = (((d / 8) ^ (h & 7)) * 16) + (d % 8) * 2;
-    *reinterpret_cast<uint32_t*>(qt + (0 * G + h) * 256 + off) = lo;
-    *reinterpret_cast<uint32_t*>(qt + (1 * G + h) * 256 + off) = mid;
-    *reinterpret_cast<uint32_t*>(qt + (2 * G + h) * 256 + off) = hi;
-  }
-  if (tid < 16) reinterpret_cast<uint4*>(qt + 3 * G * 256)[tid] = make_uint4(0u, 0u, 0u, 0u);
-}
-
-template <int LPT>
+template <int LPT, int MG>
 __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WideParams p) {
   using S = TipShape<__nv_bfloat16, LPT>;
   constexpr int U = S::LPT2 == 1 ? 4 : 2;  // tokens in flight per lane
@@ -675,15 +508,25 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   __syncthreads();
   const int n_att = min((int)total, p.n_keep);
-  if (!p.direct) {  // attend_mma_kernel follows: its query terms
-    query_terms(qraw, G, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes, tid, kWdThreads);
-    return;
-  }
-  unsigned char* qt = smem + Lo.qt;
-  wd_query_terms(qraw, G, p.cosv, p.sinv, qt);
+  if (!p.direct) return;  // the split-K attention launch follows
+  // the group's attention over the kept rows: each warp a contiguous part
+  // of the kept list, then the warps merged
+  float* qs = reinterpret_cast<float*>(smem + Lo.qt);
+  float* wsall = qs + MG * kD;
+  float* mo = reinterpret_cast<float*>(smem + Lo.ring);
+  cc_queries(qraw, G, MG, p.cosv, p.sinv, qs, tid, kWdThreads);
   __syncthreads();
-  wd_attend(p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD, kept, n_att, qt, G,
-            smem + Lo.ring, p.out + (int64_t)row * G * kD);
+  float* ws = wsall + warp * cc_warp_scratch(MG);
+  CcAcc<MG> acc;
+  cc_init<MG>(acc, ws, lane);
+  const int per_warp = ((n_att + kWdWarps * kCcStep - 1) / (kWdWarps * kCcStep)) * kCcStep;
+  const int j0 = min(n_att, warp * per_warp), j1 = min(n_att, j0 + per_warp);
+  cc_warp_rows<MG, false>(acc, p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD,
+                          [&](int j) -> int { return kept[j]; }, j0, j1, qs, ws, lane);
+  __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
+  cc_block_merge<MG>(acc, mo, wsall, cc_warp_scratch(MG), kWdWarps, [&](int h, int d, float, float L, float O) {
+    if (h < G) out[h * kD + d] = __float2bfloat16_rn(L > 0.0f ? O / L : 0.0f);
+  });
 }
 
 }  // namespace fasa

@@ -14,7 +14,7 @@
 #include "score.cuh"
 #include "select_attend.cuh"
 #include "select_hist.cuh"
-#include "attend_mma.cuh"
+#include "attend_cc.cuh"
 #include "decode_wide.cuh"
 #include "calibrate.cuh"
 
@@ -346,9 +346,9 @@ struct WidePlan {
   int n_split = 0, n_loc = 0, direct = 0, ucache = 0, smem = 0;
 };
 
-template <int LPT>
+template <int LPT, int MG>
 fasa_status wide_attrs(const DevInfo& d) {
-  auto kern = decode_wide_kernel<LPT>;
+  auto kern = decode_wide_kernel<LPT, MG>;
   int set = 0;
   return cached_int((const void*)kern, 0, &set, [&](int* v) {
     *v = 1;
@@ -372,7 +372,7 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   pl->n_loc = (int)ceil_div(len, S);
   if (pl->n_loc > kWdMaxLoc || S > 65535) return false;
   const int G = c->n_q_heads / c->n_kv_heads;
-  for (int direct = keff <= kWdMaxDirect ? 1 : 0; direct >= 0; --direct) {
+  for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
     const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, 0);
     if (base.total > d.smem_optin) continue;
     // the union cache is the last part of its region: whatever shared memory is left
@@ -385,10 +385,10 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   return false;
 }
 
-template <int LPT>
+template <int LPT, int MG>
 fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cudaStream_t st, const DevInfo& d) {
-  auto kern = decode_wide_kernel<LPT>;
-  fasa_status s = wide_attrs<LPT>(d);
+  auto kern = decode_wide_kernel<LPT, MG>;
+  fasa_status s = wide_attrs<LPT, MG>(d);
   if (s != FASA_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attrs[1];
@@ -410,24 +410,25 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 //     the published (key, token) pairs [rows][len] u32x2 |
 //   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
-//   part [rows][splits_max][kAttPartStride] f32 | qterm [rows][kQTermBytes]
+//   part [rows][splits_max][kCcPartStride] f32
 // The staged plan clears the first two parts and hist, cand_cnt at the start
 // of every call; the wide plan relies on them being zero.
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
+constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
 struct DecodeWs {
-  size_t sem, att_cnt, scores, hist, cnt, bitmap, cand, ckey, idx, part, qterm, total;
+  size_t sem, att_cnt, scores, hist, cnt, bitmap, cand, ckey, idx, part, total;
   int64_t ld;
   int cap, words, splits_max;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
-inline int att_chunks(int keff) { return (keff + kAttChunk - 1) / kAttChunk; }
+inline int att_chunks(int keff) { return (keff + kAttUnit - 1) / kAttUnit; }
 // Splits per row so that the attention grid fills, without exceeding, one
-// wave of resident CTAs; at most kAttMaxSplits, whose merge state fits in
+// wave of resident CTAs; at most kCcMaxSplits, whose merge state fits in
 // the kernel's shared memory.
 inline int att_splits(int rows, int keff, int sms, int per_sm) {
   const int64_t s = std::min<int64_t>(att_chunks(keff), (int64_t)per_sm * sms / rows);
-  return (int)std::max<int64_t>(1, std::min<int64_t>(s, kAttMaxSplits));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(s, kCcMaxSplits));
 }
 DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   DecodeWs w;
@@ -448,8 +449,7 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
   w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
   w.part = al256(w.idx + rows * (size_t)keff * 4);
-  w.qterm = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4);
-  w.total = al256(w.qterm + rows * (size_t)kQTermBytes) + 256;
+  w.total = al256(w.part + rows * (size_t)w.splits_max * kCcPartStride * 4) + 256;
   return w;
 }
 size_t decode_ws(const fasa_cache* c, int32_t len, int32_t k) { return decode_layout(c, len, k).total; }
@@ -503,22 +503,42 @@ fasa_status launch_cal_scores(const fasa_cache* c, int32_t len, const void* q_wi
   return cuda_status(cudaGetLastError());
 }
 
-// Split-K attention (attend_mma_kernel) of every row over its kept list
-// idx [rows][n_keep], or over rows 0 .. n_keep-1 when idx is null (the dense
-// decode); the query terms come from qterms [rows][kQTermBytes], or, when it
-// is null, each CTA forms them from q. part [rows][splits_max][...] holds
-// the split partials; counter [rows] must be zero (the kernel leaves it zero).
+// Split-K attention (attend_cc_kernel) of every row over its kept list idx
+// [rows][n_keep], or over rows 0 .. n_keep-1 when idx is null (the dense
+// decode); every CTA forms its group's queries from q. part [rows][splits_max]
+// [kCcPartStride] holds the split partials; counter [rows] must be zero (the
+// kernel leaves it zero).
+template <int MG>
+fasa_status launch_attend_t(CcParams& ap, int rows, int splits_max, const DevInfo& d, cudaStream_t st) {
+  auto kern = attend_cc_kernel<MG>;
+  const int smem = cc_smem_bytes(MG);
+  int per_sm = 0;
+  fasa_status s = cached_int((const void*)kern, 7, &per_sm, [&](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kern, kCcThreads, (size_t)smem);
+    return cuda_status(e);
+  });
+  if (s != FASA_OK) return s;
+  per_sm = std::max(1, per_sm);
+  // one wave of resident CTAs at most, each with at least one step per warp
+  constexpr int kUnit = kCcWarps * kCcStep;
+  const int64_t units = ceil_div(ap.n_keep, kUnit);
+  int64_t splits = std::min<int64_t>(units, std::max<int64_t>(1, (int64_t)per_sm * d.sms / rows));
+  splits = std::min<int64_t>(splits, std::min<int64_t>(splits_max, kCcMaxSplits));
+  ap.slice = (int)(ceil_div(units, splits) * kUnit);
+  ap.splits = (int)ceil_div(ap.n_keep, ap.slice);
+  return launch_pdl(kern, dim3((unsigned)ap.splits, (unsigned)rows, 1), kCcThreads, (size_t)smem, st, ap);
+}
+
 fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
-                          const unsigned char* qterms, const void* q, int32_t q_pos, float* part, uint32_t* counter,
-                          int splits_max, const DevInfo& d, cudaStream_t st) {
+                          const void* q, int32_t q_pos, float* part, uint32_t* counter, int splits_max,
+                          const DevInfo& d, cudaStream_t st) {
   const int rows = c->batch * c->n_kv_heads;
-  AttParams ap{};
+  CcParams ap{};
   ap.k = static_cast<const __nv_bfloat16*>(c->k);
   ap.v = static_cast<const __nv_bfloat16*>(c->v);
   ap.idx = idx;
-  ap.qterms = qterms;
   ap.q = static_cast<const __nv_bfloat16*>(q);
-  ap.n_kv_heads = c->n_kv_heads;
   ap.out = static_cast<__nv_bfloat16*>(out);
   ap.part = part;
   ap.counter = counter;
@@ -526,40 +546,22 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
   ap.len = len;
   ap.n_keep = n_keep;
   ap.group = c->n_q_heads / c->n_kv_heads;
-  if (qterms == nullptr) fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
-  int set = 0;
-  fasa_status s = cached_int((const void*)attend_mma_kernel, 0, &set, [&](int* v) {
-    *v = 1;
-    return cuda_status(cudaFuncSetAttribute(attend_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            att_smem_bytes(FASA_MAX_GROUP)));
-  });
-  if (s != FASA_OK) return s;
-  int per_sm = 0;  // resident attention CTAs per SM at this group size
-  if ((s = cached_int((const void*)attend_mma_kernel, 1 + (uint64_t)ap.group, &per_sm, [&](int* v) {
-         return cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, attend_mma_kernel, kAttThreads,
-                                                                           (size_t)att_smem_bytes(ap.group)));
-       })) != FASA_OK)
-    return s;
-  per_sm = std::max(1, std::min(per_sm, kAttMaxPerSm));
-  ap.splits = std::min(splits_max, att_splits(rows, n_keep, d.sms, per_sm));
-  ap.slice = (int)ceil_div(att_chunks(n_keep), ap.splits) * kAttChunk;
-  ap.splits = (int)ceil_div(n_keep, ap.slice);
-  if (ap.splits > kAttMaxSplits) return FASA_ERR_UNSUPPORTED;  // cannot happen: splits only shrank
-  return launch_pdl(attend_mma_kernel, dim3((unsigned)ap.splits, (unsigned)rows, 1), kAttThreads,
-                    (size_t)att_smem_bytes(ap.group), st, ap);
+  fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
+  if (ap.group <= 4) return launch_attend_t<4>(ap, rows, splits_max, d, st);
+  if (ap.group <= 8) return launch_attend_t<8>(ap, rows, splits_max, d, st);
+  return launch_attend_t<16>(ap, rows, splits_max, d, st);
 }
 
-// The decode's attention over the kept lists and query terms in the workspace.
-fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, void* out, const DecodeWs& w, char* base,
-                             const DevInfo& d, cudaStream_t st) {
-  return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx),
-                       reinterpret_cast<const unsigned char*>(base + w.qterm), nullptr, 0,
+// The decode's attention over the kept lists in the workspace.
+fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, const void* q, int32_t q_pos, void* out,
+                             const DecodeWs& w, char* base, const DevInfo& d, cudaStream_t st) {
+  return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx), q, q_pos,
                        reinterpret_cast<float*>(base + w.part), reinterpret_cast<uint32_t*>(base + w.att_cnt),
                        w.splits_max, d, st);
 }
 
 // Dense decode workspace: att_cnt [rows] u32 (zero between calls) | part
-// [rows][splits_max][kAttPartStride] f32.
+// [rows][splits_max][kCcPartStride] f32.
 struct DenseWs {
   size_t att_cnt, part, total;
   int splits_max;
@@ -570,7 +572,7 @@ DenseWs dense_layout(const fasa_cache* c, int32_t len) {
   w.splits_max = att_splits((int)rows, std::max(len, 1), kAssumedMaxSms, kAttMaxPerSm);
   w.att_cnt = 0;
   w.part = al256(rows * 4);
-  w.total = al256(w.part + rows * (size_t)w.splits_max * kAttPartStride * 4) + 256;
+  w.total = al256(w.part + rows * (size_t)w.splits_max * kCcPartStride * 4) + 256;
   return w;
 }
 
@@ -588,7 +590,6 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.out = static_cast<__nv_bfloat16*>(out);
   p.idx_out = idx_out;
   p.idx_ws = pl.direct ? nullptr : reinterpret_cast<int32_t*>(base + w.idx);
-  p.qterms = pl.direct ? nullptr : reinterpret_cast<unsigned char*>(base + w.qterm);
   p.cand = reinterpret_cast<uint2*>(base + w.scores);
   p.sem = reinterpret_cast<unsigned long long*>(base + w.sem);
   p.max_len = c->max_len;
@@ -605,16 +606,17 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   const int rows = c->batch * c->n_kv_heads;
   fasa_status s;
+  const bool g4 = p.group <= 4;  // padded heads of the in-CTA attention: 4 or 8
   switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
-    case 1: s = launch_wide_t<1>(p, rows, pl, st, d); break;
-    case 2: s = launch_wide_t<2>(p, rows, pl, st, d); break;
-    case 4: s = launch_wide_t<4>(p, rows, pl, st, d); break;
-    case 8: s = launch_wide_t<8>(p, rows, pl, st, d); break;
-    case 16: s = launch_wide_t<16>(p, rows, pl, st, d); break;
+    case 1: s = g4 ? launch_wide_t<1, 4>(p, rows, pl, st, d) : launch_wide_t<1, 8>(p, rows, pl, st, d); break;
+    case 2: s = g4 ? launch_wide_t<2, 4>(p, rows, pl, st, d) : launch_wide_t<2, 8>(p, rows, pl, st, d); break;
+    case 4: s = g4 ? launch_wide_t<4, 4>(p, rows, pl, st, d) : launch_wide_t<4, 8>(p, rows, pl, st, d); break;
+    case 8: s = g4 ? launch_wide_t<8, 4>(p, rows, pl, st, d) : launch_wide_t<8, 8>(p, rows, pl, st, d); break;
+    case 16: s = g4 ? launch_wide_t<16, 4>(p, rows, pl, st, d) : launch_wide_t<16, 8>(p, rows, pl, st, d); break;
     default: return FASA_ERR_UNSUPPORTED;
   }
   if (s != FASA_OK || pl.direct) return s;
-  return launch_attend_ws(c, len, keff, out, w, base, d, st);
+  return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st);
 }
 
 }  // namespace
@@ -801,10 +803,6 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   const int64_t tiles_per_row = std::max<int64_t>(1, 4LL * d.sms / rows);
   fp.tile = (int)std::max<int64_t>(2048, ceil_div(ceil_div(len, tiles_per_row), 128) * 128);
   fp.words = w.words;
-  fp.q = static_cast<const __nv_bfloat16*>(q);
-  fp.qterms = c->dtype == FASA_BF16 ? reinterpret_cast<unsigned char*>(base + w.qterm) : nullptr;
-  fp.group = c->n_q_heads / c->n_kv_heads;
-  fill_query_angle(fp.cosv, fp.sinv, c->rope_base, q_pos);
   if ((s = launch_pdl(filter_kernel, dim3((unsigned)ceil_div(len, fp.tile), (unsigned)rows, 1), kFilterThreads, 0,
                       stream, fp)) != FASA_OK)
     return s;
@@ -840,7 +838,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
     return s;
 
   // 4. focused attention over the kept rows
-  if (c->dtype == FASA_BF16) return launch_attend_ws(c, len, keff, out, w, base, d, stream);
+  if (c->dtype == FASA_BF16) return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, stream);
   SAParams p{};
   p.idx_in = idx;
   p.k = c->k;
@@ -924,7 +922,7 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
     DevInfo d;
     if ((s = device_info(&d)) != FASA_OK) return s;
     char* base = static_cast<char*>(workspace);
-    return launch_attend(c, len, len, out, nullptr, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part),
+    return launch_attend(c, len, len, out, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part),
                          reinterpret_cast<uint32_t*>(base + w.att_cnt), w.splits_max, d, stream);
   }
   SAParams p{};

@@ -25,7 +25,7 @@
 //           its scores instead (slow, rare).
 #pragma once
 
-#include "attend_mma.cuh"
+#include "score.cuh"
 #include "select_attend.cuh"
 
 namespace fasa {
@@ -47,12 +47,6 @@ struct FilterParams {
   int32_t cap;
   int32_t tile;             // tokens per CTA, a multiple of 128
   int32_t words;            // ceil(len / 32)
-  // the attention kernel's query terms, prepared by tile 0 of each row
-  const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
-  unsigned char* qterms;    // [rows][kQTermBytes], or null (no attention follows)
-  int32_t group;
-  double cosv[kNFC];        // cos / sin of q_pos * theta_i (host, float64)
-  double sinv[kNFC];
 };
 
 __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterParams p) {
@@ -62,12 +56,6 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
   __shared__ uint32_t s_n, s_base;
   const int row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // The query is an input of the whole decode, complete before the score
-  // kernel started, so tile 0 can turn it into query terms before waiting;
-  // the attention kernel reads them two launches later.
-  if (blockIdx.x == 0 && p.qterms)
-    query_terms(p.q + (int64_t)row * p.group * kD, p.group, p.cosv, p.sinv, p.qterms + (int64_t)row * kQTermBytes,
-                tid, kFilterThreads);
   if (tid == 0) s_n = 0u;
   grid_dependency_wait();
   uint32_t bin, above;
