@@ -87,11 +87,12 @@ __device__ __forceinline__ void cc_bf16x4(const uint2& u, float (&f)[4]) {
   f[3] = __uint_as_float(u.y & 0xFFFF0000u);
 }
 
-// One step of 8 rows: kk[r], vv[r] are the lane's 8 bytes of K and V row r;
-// bit r of `valid` says whether row r takes part. qs: [MG][128] queries;
-// ws: the warp's scratch (cc_warp_scratch floats).
+// One step of 8 rows: kk[r] is the lane's 8 bytes of K row r, and vs the
+// 8 V rows in shared memory ([8][128] bf16, the lane reads its own 8 bytes
+// of each); bit r of `valid` says whether row r takes part. qs: [MG][128]
+// queries; ws: the warp's scratch (cc_warp_scratch floats).
 template <int MG>
-__device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep], const uint2 (&vv)[kCcStep],
+__device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep], const __nv_bfloat16* vs,
                                          unsigned valid, const float* qs, float* ws, int lane) {
   constexpr int NG = MG / 4;
   float* wp = ws;                    // p[8][MG]
@@ -163,7 +164,7 @@ __device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep
 #pragma unroll
   for (int r = 0; r < kCcStep; ++r) {
     float vf[4];
-    cc_bf16x4(vv[r], vf);
+    cc_bf16x4(*reinterpret_cast<const uint2*>(vs + r * kD + 4 * lane), vf);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const float4 p4 = *reinterpret_cast<const float4*>(wp + r * MG + g * 4);
@@ -179,12 +180,14 @@ __device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep
 
 // A warp attends rows j0 .. j1-1 of a list: token(j) gives the cache slot
 // of list position j, or -1 for a position to skip. kb, vb: the row's K and
-// V planes [max_len][128]. With kPipe the next step's rows are loaded before
-// the current step is computed (two register buffers).
-template <int MG, bool kPipe, typename Tok>
+// V planes [max_len][128]. K rows go to registers, V rows to the warp's
+// shared-memory buffer vbuf ([2][8][128] bf16) with 8-byte cp.async; the
+// next step's rows are loaded before the current step is computed.
+template <int MG, typename Tok>
 __device__ __forceinline__ void cc_warp_rows(CcAcc<MG>& a, const __nv_bfloat16* kb, const __nv_bfloat16* vb,
-                                             Tok token, int j0, int j1, const float* qs, float* ws, int lane) {
-  auto load = [&](uint2 (&kk)[kCcStep], uint2 (&vv)[kCcStep], unsigned& valid, int jb) {
+                                             Tok token, int j0, int j1, const float* qs, float* ws,
+                                             __nv_bfloat16* vbuf, int lane) {
+  auto load = [&](uint2 (&kk)[kCcStep], __nv_bfloat16* vs, unsigned& valid, int jb) {
     const int mine = (lane < kCcStep && jb + lane < j1) ? token(jb + lane) : -1;
     valid = __ballot_sync(0xFFFFFFFFu, mine >= 0) & 0xFFu;
 #pragma unroll
@@ -192,28 +195,36 @@ __device__ __forceinline__ void cc_warp_rows(CcAcc<MG>& a, const __nv_bfloat16* 
       int t = __shfl_sync(0xFFFFFFFFu, mine, r);
       if (t < 0) t = 0;  // masked out; row 0 is a valid address
       kk[r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t * kD) + lane);
-      vv[r] = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t * kD) + lane);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(vs + r * kD + 4 * lane)),
+                   "l"(vb + (int64_t)t * kD + 4 * lane)
+                   : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
   if (j0 >= j1) return;
-  uint2 k0[kCcStep], v0[kCcStep];
-  unsigned m0;
-  if constexpr (kPipe) {
-    uint2 k1[kCcStep], v1[kCcStep];
-    unsigned m1;
-    load(k0, v0, m0, j0);
-    for (int jb = j0; jb < j1; jb += 2 * kCcStep) {
-      if (jb + kCcStep < j1) load(k1, v1, m1, jb + kCcStep);
-      cc_step8<MG>(a, k0, v0, m0, qs, ws, lane);
-      if (jb + kCcStep >= j1) break;
-      if (jb + 2 * kCcStep < j1) load(k0, v0, m0, jb + 2 * kCcStep);
-      cc_step8<MG>(a, k1, v1, m1, qs, ws, lane);
+  uint2 k0[kCcStep], k1[kCcStep];
+  unsigned m0, m1;
+  __nv_bfloat16* vs0 = vbuf;
+  __nv_bfloat16* vs1 = vbuf + kCcStep * kD;
+  load(k0, vs0, m0, j0);
+  for (int jb = j0; jb < j1; jb += 2 * kCcStep) {
+    const bool more = jb + kCcStep < j1;
+    if (more) {
+      load(k1, vs1, m1, jb + kCcStep);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
-  } else {
-    for (int jb = j0; jb < j1; jb += kCcStep) {
-      load(k0, v0, m0, jb);
-      cc_step8<MG>(a, k0, v0, m0, qs, ws, lane);
+    cc_step8<MG>(a, k0, vs0, m0, qs, ws, lane);
+    if (!more) break;
+    const bool more2 = jb + 2 * kCcStep < j1;
+    if (more2) {
+      load(k0, vs0, m0, jb + 2 * kCcStep);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
+    cc_step8<MG>(a, k1, vs1, m1, qs, ws, lane);
   }
 }
 
@@ -277,7 +288,8 @@ struct CcParams {
 // Shared memory of attend_cc_kernel: group queries (raw), queries (scaled
 // float32), warp scratch, warp partials; the split merge reuses the partials.
 __host__ __device__ constexpr int cc_smem_bytes(int MG) {
-  return FASA_MAX_GROUP * kD * 2 + MG * kD * 4 + kCcWarps * cc_warp_scratch(MG) * 4 + kCcWarps * MG * kD * 4;
+  return FASA_MAX_GROUP * kD * 2 + MG * kD * 4 + kCcWarps * cc_warp_scratch(MG) * 4 + kCcWarps * MG * kD * 4 +
+         kCcWarps * 2 * kCcStep * kD * 2;
 }
 constexpr int kCcMaxSplits = (kCcWarps * 4 * kD * 4) / (3 * 16 * 4);  // the merge state fits the MG = 4 partials
 
@@ -287,12 +299,13 @@ constexpr int kCcMaxSplits = (kCcWarps * 4 * kD * 4) / (3 * 16 * 4);  // the mer
 // CTA writes its partial (m, l, o) and the row's last CTA (atomic ticket, no
 // waiting) merges the splits in a fixed order and writes the output.
 template <int MG>
-__global__ void __launch_bounds__(kCcThreads) attend_cc_kernel(const CcParams p) {
+__global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(const CcParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
   float* qs = reinterpret_cast<float*>(smem + FASA_MAX_GROUP * kD * 2);
   float* wsall = qs + MG * kD;
   float* mo = wsall + kCcWarps * cc_warp_scratch(MG);
+  __nv_bfloat16* vball = reinterpret_cast<__nv_bfloat16*>(mo + kCcWarps * MG * kD);
   grid_dependency_wait();
   const int split = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -313,14 +326,14 @@ __global__ void __launch_bounds__(kCcThreads) attend_cc_kernel(const CcParams p)
   const __nv_bfloat16* kb = p.k + (int64_t)row * p.max_len * kD;
   const __nv_bfloat16* vb = p.v + (int64_t)row * p.max_len * kD;
   const int32_t* idx = p.idx ? p.idx + (int64_t)row * p.n_keep : nullptr;
-  cc_warp_rows<MG, true>(acc, kb, vb, [&](int j) -> int {
+  cc_warp_rows<MG>(acc, kb, vb, [&](int j) -> int {
     const int t = idx ? __ldg(idx + j) : j;
     if (t < 0 || t >= p.len) {
       flag_status(FASA_ERR_BAD_INDEX);
       return -1;
     }
     return t;
-  }, j0, j1, qs, ws, lane);
+  }, j0, j1, qs, ws, vball + warp * 2 * kCcStep * kD, lane);
   __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
   float* pp = p.part + ((int64_t)row * p.splits + split) * kCcPartStride;
   const bool single = p.splits == 1;
@@ -384,6 +397,133 @@ __global__ void __launch_bounds__(kCcThreads) attend_cc_kernel(const CcParams p)
     out[e] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
   }
   if (tid == 0) p.counter[row] = 0u;
+}
+
+}  // namespace fasa
+
+namespace fasa {
+
+// One CTA of NW warps attends a short kept list (n <= 16 * NW rows) in
+// phases, with every load in flight at once: (1) warp w loads the K and V
+// rows of its list positions [16w, 16w + 16) into registers (the lane's 8
+// bytes of each) and forms their logits (cc_step8's dot products and
+// reduce-scatter), stored to zs[j][h]; (2) warp h < G takes the softmax of
+// head h over all n logits (max, exp2, sum; zs becomes the probabilities);
+// (3) each warp adds p * v over its rows for the lane's 4 dims; (4) the warp
+// sums are added in a fixed order and divided by the head's sum.
+// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [MG],
+// vst [16 * NW][128] bf16 (the V rows, staged with cp.async).
+template <int MG, int NW, typename Tok>
+__device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
+                                                int G, const float* qs, float* zs, float* mo, float* lsum,
+                                                __nv_bfloat16* vst, __nv_bfloat16* out) {
+  constexpr int NG = MG / 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int jb = warp * 16;
+  uint2 kk[2][kCcStep];
+  const int mine = (lane < 16 && jb + lane < n) ? token(jb + lane) : -1;
+  const unsigned valid = __ballot_sync(0xFFFFFFFFu, mine >= 0) & 0xFFFFu;
+#pragma unroll
+  for (int s = 0; s < 2; ++s)
+#pragma unroll
+    for (int r = 0; r < kCcStep; ++r) {
+      int t = __shfl_sync(0xFFFFFFFFu, mine, s * kCcStep + r);
+      if (t < 0) t = 0;  // masked out; row 0 is a valid address
+      kk[s][r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t * kD) + lane);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(vst + (jb + s * kCcStep + r) * kD + 4 * lane)),
+                   "l"(vb + (int64_t)t * kD + 4 * lane)
+                   : "memory");
+    }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  // (1) logits
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    float kf[kCcStep][4];
+#pragma unroll
+    for (int r = 0; r < kCcStep; ++r) cc_bf16x4(kk[s][r], kf[r]);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      float v[32];
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + hh) * kD + 4 * lane);
+#pragma unroll
+        for (int r = 0; r < kCcStep; ++r)
+          v[r * 4 + hh] = __fmaf_rn(q4.w, kf[r][3], __fmaf_rn(q4.z, kf[r][2], __fmaf_rn(q4.y, kf[r][1],
+                                                                                      __fmul_rn(q4.x, kf[r][0]))));
+      }
+#pragma unroll
+      for (int st = 0; st < 5; ++st) {
+        const int off = 16 >> st, half = 16 >> st;
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = up ? v[i] : v[i + half];
+          const float keep = up ? v[i + half] : v[i];
+          v[i] = __fadd_rn(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
+        }
+      }
+      const int r = s * kCcStep + (lane >> 2);
+      zs[(jb + r) * MG + g * 4 + (lane & 3)] = ((valid >> r) & 1u) ? v[0] : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // (2) softmax of head `warp` over the n rows
+  const int nr = (n + 15) / 16 * 16;  // rows written in (1), padding rows at -inf
+  if (warp < G) {
+    float m = -INFINITY;
+    for (int j = lane; j < nr; j += 32) m = fmaxf(m, zs[j * MG + warp]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    float l = 0.0f;
+    for (int j = lane; j < nr; j += 32) {
+      const float z = zs[j * MG + warp];
+      const float pz = (z == -INFINITY) ? 0.0f : exp2f(z - m);
+      zs[j * MG + warp] = pz;
+      l += pz;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
+    if (lane == 0) lsum[warp] = l;
+  }
+  __syncthreads();
+  // (3) p * v over the warp's rows
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+  float o[MG][4];
+#pragma unroll
+  for (int h = 0; h < MG; ++h)
+#pragma unroll
+    for (int d = 0; d < 4; ++d) o[h][d] = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 2; ++s)
+#pragma unroll
+    for (int r = 0; r < kCcStep; ++r) {
+      const int j = jb + s * kCcStep + r;
+      float vf[4];
+      cc_bf16x4(*reinterpret_cast<const uint2*>(vst + j * kD + 4 * lane), vf);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const float4 p4 = *reinterpret_cast<const float4*>(zs + j * MG + g * 4);
+        const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh)
+#pragma unroll
+          for (int d = 0; d < 4; ++d) o[g * 4 + hh][d] = __fmaf_rn(pv[hh], vf[d], o[g * 4 + hh][d]);
+      }
+    }
+#pragma unroll
+  for (int h = 0; h < MG; ++h)
+    *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+  __syncthreads();
+  // (4) warp sums in warp order, divided by the head's sum
+  for (int e = tid; e < G * kD; e += NW * 32) {
+    const int h = e / kD, d = e % kD;
+    float acc = 0.0f;
+    for (int w = 0; w < NW; ++w) acc += mo[(w * MG + h) * kD + d];
+    const float l = lsum[h];
+    out[e] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
+  }
 }
 
 }  // namespace fasa

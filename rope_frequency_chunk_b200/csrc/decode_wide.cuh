@@ -55,7 +55,7 @@ constexpr int kWdMaxLoc = 16384;        // tokens per CTA (their keys live in sh
 constexpr int kWdTieCap = 2048;         // boundary-bin entries held in shared memory
 constexpr int kWdRankMax = 128;         // entries of the finest bin resolved by rank counting
 constexpr int kWdUnionUnroll = 8;       // union entries in flight per thread
-constexpr int kWdMaxDirect = 512;       // kept rows the resolving CTA attends itself
+constexpr int kWdMaxDirect = 16 * kWdWarps;  // kept rows the resolving CTA attends itself (16 per warp)
 // radix scratch: the sub-bin histogram and entries, then ballot_radix_fn's
 constexpr int kWdRadixWords = 256 + 2 * 128 + kSAWarps * 256 + 264;
 constexpr int kWdMisc = 128;            // words of scan and flag scratch
@@ -119,14 +119,15 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   b += wd_al(kWdRadixWords * 4, 16);
   L.ucache = o + b;
   b += ucache * 8;
-  // the attention: queries [MG][128] f32, warp scratch, warp partials [16][MG][128] f32
+  // the attention (cc_block_attend): queries [MG][128] f32, logits [256][MG]
+  // f32, warp sums [16][MG][128] f32, head sums [MG] (64 B), V rows [256][128] bf16
   const int MG = group <= 4 ? 4 : 8;
   L.qt = o;
   int c = 0;
   if (direct) {
-    c = MG * kD * 4 + kWdWarps * cc_warp_scratch(MG) * 4;
+    c = MG * kD * 4 + kWdMaxDirect * MG * 4;
     L.ring = o + c;
-    c += kWdWarps * MG * kD * 4;
+    c += kWdWarps * MG * kD * 4 + 64 + kWdMaxDirect * kD * 2;
   } else {
     L.ring = o;
   }
@@ -509,24 +510,17 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   __syncthreads();
   const int n_att = min((int)total, p.n_keep);
   if (!p.direct) return;  // the split-K attention launch follows
-  // the group's attention over the kept rows: each warp a contiguous part
-  // of the kept list, then the warps merged
+  // the group's attention over the kept rows (at most 16 per warp)
   float* qs = reinterpret_cast<float*>(smem + Lo.qt);
-  float* wsall = qs + MG * kD;
+  float* zs = qs + MG * kD;
   float* mo = reinterpret_cast<float*>(smem + Lo.ring);
+  float* lsum = mo + kWdWarps * MG * kD;
+  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
   cc_queries(qraw, G, MG, p.cosv, p.sinv, qs, tid, kWdThreads);
   __syncthreads();
-  float* ws = wsall + warp * cc_warp_scratch(MG);
-  CcAcc<MG> acc;
-  cc_init<MG>(acc, ws, lane);
-  const int per_warp = ((n_att + kWdWarps * kCcStep - 1) / (kWdWarps * kCcStep)) * kCcStep;
-  const int j0 = min(n_att, warp * per_warp), j1 = min(n_att, j0 + per_warp);
-  cc_warp_rows<MG, false>(acc, p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD,
-                          [&](int j) -> int { return kept[j]; }, j0, j1, qs, ws, lane);
-  __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
-  cc_block_merge<MG>(acc, mo, wsall, cc_warp_scratch(MG), kWdWarps, [&](int h, int d, float, float L, float O) {
-    if (h < G) out[h * kD + d] = __float2bfloat16_rn(L > 0.0f ? O / L : 0.0f);
-  });
+  cc_block_attend<MG, kWdWarps>(p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD,
+                                [&](int j) -> int { return kept[j]; }, n_att, G, qs, zs, mo, lsum, vst,
+                                p.out + (int64_t)row * G * kD);
 }
 
 }  // namespace fasa
