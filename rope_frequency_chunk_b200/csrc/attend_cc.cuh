@@ -469,7 +469,7 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
   }
   __syncthreads();
   // (2) softmax of head `warp` over the n rows
-  const int nr = (n + 15) / 16 * 16;  // rows written in (1), padding rows at -inf
+  const int nr = 16 * NW;  // every row written in (1); padding rows are -inf and become 0
   if (warp < G) {
     float m = -INFINITY;
     for (int j = lane; j < nr; j += 32) m = fmaxf(m, zs[j * MG + warp]);
