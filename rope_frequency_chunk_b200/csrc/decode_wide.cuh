@@ -36,11 +36,11 @@
 //        list, then the warps merged); otherwise it writes the kept list for
 //        attend_cc_kernel, launched next.
 //
-// Semaphore: sem[row] = (tickets << 32) | entries reserved. It must be zero
-// when a call starts; the last CTA of the row writes it back to zero, so a
-// workspace zeroed once stays valid. A ticket or reservation beyond its
-// range (a workspace that was not zero) is flagged FASA_ERR_WORKSPACE and
-// never written out of bounds.
+// Semaphore: sem[row] counts the row's CTAs that have published. It must be
+// zero when a call starts; the last CTA of the row writes it back to zero,
+// so a workspace zeroed once stays valid. A ticket beyond its range (a
+// workspace that was not zero) is flagged FASA_ERR_WORKSPACE; region counts
+// are clamped to the region size, so nothing is read out of bounds.
 #pragma once
 
 #include "attend_cc.cuh"
@@ -69,7 +69,7 @@ struct WideParams {
   __nv_bfloat16* out;           // [B][Hq][128]
   int32_t* idx_out;             // [rows][n_keep] kept tokens, ascending, or null
   int32_t* idx_ws;              // [rows][n_keep] for the attention launch, or null (direct)
-  uint2* cand;                  // [rows][len] published (key, token) pairs
+  uint2* cand;                  // [rows][n_split][n_loc + 1] regions: count, then (key, token) pairs
   unsigned long long* sem;      // [rows], zero between calls
   int64_t max_len;
   int32_t len;
@@ -80,7 +80,7 @@ struct WideParams {
   int32_t n_keep;   // k_eff, 1 .. len
   int32_t n_loc;    // tokens per CTA, <= kWdMaxLoc
   int32_t n_split;  // CTAs per row
-  int32_t ucache;   // union entries the resolving CTA caches in shared memory
+  int32_t ucache;   // entries of each CTA's region the resolving CTA stages in shared memory (P)
   int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect, G <= 8)
   double cosv[kNFC];
   double sinv[kNFC];
@@ -90,12 +90,15 @@ __host__ __device__ constexpr int wd_al(int x, int a) { return (x + a - 1) / a *
 
 // Shared-memory layout. r1 is reused: the CTA's keys (steps 1-3); then, in
 // the resolving CTA, the bitmap, boundary-bin entries, radix scratch and the
-// cached union; then the attention's query terms and K/V ring.
+// staged union ([n_split][P] entries); then the attention's logits, warp
+// sums and V rows.
 struct WdLayout {
-  int hist, misc, coef, qraw, dom, kept, r1, bitmap, ties, rscr, ucache, qt, ring, total;
+  int hist, misc, coef, qraw, dom, cs, qs, cnt, kept, r1, bitmap, ties, rscr, ucache, zs, ring, total;
 };
-__host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, int direct, int group, int ucache) {
+__host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, int direct, int group, int n_split,
+                                              int P) {
   WdLayout L;
+  const int MG = group <= 4 ? 4 : 8;
   int o = 0;
   L.hist = o;
   o += 4096 * 4;
@@ -107,6 +110,12 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   o += FASA_MAX_GROUP * kD * 2;
   L.dom = o;
   o += kNFC * 4;
+  L.cs = o;  // cos, sin of the query angle (float64)
+  o += 2 * kNFC * 8;
+  L.qs = o;  // attention queries [MG][128] f32
+  o += direct ? MG * kD * 4 : 0;
+  L.cnt = o;  // region counts, then their prefix sums
+  o += wd_al((2 * n_split + 2) * 4, 16);
   L.kept = o;
   o += wd_al(direct ? n_keep * 4 : 0, 128);
   L.r1 = o;
@@ -118,14 +127,13 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   L.rscr = o + b;
   b += wd_al(kWdRadixWords * 4, 16);
   L.ucache = o + b;
-  b += ucache * 8;
-  // the attention (cc_block_attend): queries [MG][128] f32, logits [256][MG]
-  // f32, warp sums [16][MG][128] f32, head sums [MG] (64 B), V rows [256][128] bf16
-  const int MG = group <= 4 ? 4 : 8;
-  L.qt = o;
+  b += n_split * P * 8;
+  // the attention (cc_block_attend): logits [256][MG] f32, warp sums
+  // [16][MG][128] f32, head sums [MG] (64 B), V rows [256][128] bf16
+  L.zs = o;
   int c = 0;
   if (direct) {
-    c = MG * kD * 4 + kWdMaxDirect * MG * 4;
+    c = kWdMaxDirect * MG * 4;
     L.ring = o + c;
     c += kWdWarps * MG * kD * 4 + 64 + kWdMaxDirect * kD * 2;
   } else {
@@ -252,7 +260,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   using S = TipShape<__nv_bfloat16, LPT>;
   constexpr int U = S::LPT2 == 1 ? 4 : 2;  // tokens in flight per lane
   extern __shared__ __align__(128) unsigned char smem[];
-  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.ucache);
+  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.n_split, p.ucache);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + Lo.hist);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lo.misc);
   float* coef = reinterpret_cast<float*>(smem + Lo.coef);
@@ -274,28 +282,24 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   grid_dependency_wait();
   grid_dependents_launch();
 
-  // 1. the group's queries and dominant FCs, the coefficients
+  // 1. the group's queries, dominant FCs and rotation table; the CTA's first
+  // sketch rows are requested before the coefficients are formed, so the
+  // query's round trip and the float64 work overlap the stream
   const int G = p.group;
   const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
+  double* cs_sm = reinterpret_cast<double*>(smem + Lo.cs);
   {
     const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
     for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
     if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
-    for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+    if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
+    else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
   }
-  __syncthreads();
-  if (tid < p.stride) coef[tid] = tip_coef<__nv_bfloat16>(qraw, s_dom, G, p.n_dom, tid, p.cosv, p.sinv);
-  __syncthreads();
-  const int sub = tid % S::LPT2;  // the lane's chunk group; a token's lanes are adjacent
-  float cr[S::EPL];
-#pragma unroll
-  for (int e = 0; e < S::EPL; ++e) cr[e] = coef[sub * S::EPL + e];
-
-  // 2. score the CTA's tokens straight from global memory
   constexpr int kTokPass = kWdThreads / S::LPT2;
   const int my_tok = tid / S::LPT2;
-  for (int base = 0; base < n_tok; base += kTokPass * U) {  // block-uniform trip count
-    uint4 v[U][S::CPL];
+  const int sub = tid % S::LPT2;  // the lane's chunk group; a token's lanes are adjacent
+  uint4 v[U][S::CPL];
+  auto load_rows = [&](int base) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int t = base + u * kTokPass + my_tok;
@@ -304,6 +308,21 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
         v[u][c] = t < n_tok ? __ldg(reinterpret_cast<const uint4*>(src + (int64_t)t * S::ROWB) + sub * S::CPL + c)
                             : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  load_rows(0);
+  for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+  __syncthreads();
+  if (tid < p.stride) coef[tid] = tip_coef<__nv_bfloat16>(qraw, s_dom, G, p.n_dom, tid, cs_sm, cs_sm + kNFC);
+  // the attention queries, used by the row's resolving CTA
+  if (p.direct) cc_queries(qraw, G, MG, cs_sm, cs_sm + kNFC, reinterpret_cast<float*>(smem + Lo.qs), tid, kWdThreads);
+  __syncthreads();
+  float cr[S::EPL];
+#pragma unroll
+  for (int e = 0; e < S::EPL; ++e) cr[e] = coef[sub * S::EPL + e];
+
+  // 2. score the CTA's tokens straight from global memory
+  for (int base = 0; base < n_tok; base += kTokPass * U) {  // block-uniform trip count
+    if (base > 0) load_rows(base);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int t = base + u * kTokPass + my_tok;
@@ -320,7 +339,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   __syncthreads();
 
-  // 3. the bin holding this CTA's k_eff-th key; publish the tokens at or above it
+  // 3. the bin holding this CTA's k_eff-th key; publish the tokens at or
+  // above it into the CTA's own region: [count][(key, token) ...]
   uint32_t b_loc = 0u;
   if (n_tok > p.n_keep) {
     uint32_t above = 0u;
@@ -333,78 +353,120 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   if (lane == 0) misc[64 + warp] = wc;
   __syncthreads();
-  if (tid == 0) {
-    const uint32_t tot = warp_offsets_serial(misc, 64);
-    uint32_t base = 0u;
-    if (tot) base = (uint32_t)atomicAdd(p.sem + row, (unsigned long long)tot);
-    const bool ok = (uint64_t)base + tot <= (uint64_t)p.len;
-    if (!ok) flag_status(FASA_ERR_WORKSPACE);
-    misc[96] = base;
-    misc[97] = ok ? 1u : 0u;
+  if (warp == 0) {  // exclusive offsets of the warps, and the total
+    const uint32_t c = lane < kWdWarps ? misc[64 + lane] : 0u;
+    uint32_t incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += x;
+    }
+    if (lane < kWdWarps) misc[64 + lane] = incl - c;
+    if (lane == kWdWarps - 1) misc[96] = incl;
   }
   __syncthreads();
-  uint2* crow = p.cand + (int64_t)row * p.len;
-  if (misc[97]) {
-    uint32_t pos = misc[96] + misc[64 + warp];
+  const int64_t rstride = (int64_t)p.n_loc + 1;  // entries per region, with its header
+  uint2* region = p.cand + ((int64_t)row * p.n_split + split) * rstride;
+  {
+    uint32_t pos = 1u + misc[64 + warp];
     for (int i0 = warp * 32; i0 < n_tok; i0 += kWdThreads) {
       const int i = i0 + lane;
       const uint32_t key = i < n_tok ? keys[i] : 0u;
       const bool q = i < n_tok && (key >> 20) >= b_loc;
       const unsigned m = __ballot_sync(0xFFFFFFFFu, q);
-      if (q) crow[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
+      if (q) region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
       pos += __popc(m);
     }
+    if (tid == 0) region[0] = make_uint2(misc[96], 0u);
   }
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned long long old = atomicAdd(p.sem + row, 1ull << 32);
-    const uint32_t tk = (uint32_t)(old >> 32);
-    if (tk >= (uint32_t)p.n_split) flag_status(FASA_ERR_WORKSPACE);
-    misc[98] = (tk == (uint32_t)p.n_split - 1) ? 1u : 0u;
-    misc[99] = (uint32_t)old;  // entries reserved by the row's CTAs (all of them, in the last CTA)
+    const unsigned long long old = atomicAdd(p.sem + row, 1ull);
+    if (old >= (unsigned long long)p.n_split) flag_status(FASA_ERR_WORKSPACE);
+    misc[98] = (old == (unsigned long long)p.n_split - 1) ? 1u : 0u;
   }
   __syncthreads();
   if (!misc[98]) return;
 
-  // 4. the row's last CTA: exact selection over the published union
+  // 4. the row's last CTA: exact selection over the published union. One
+  // batched read brings every region's count and first P entries into
+  // shared memory (entries beyond P, rare, are read from global memory).
   __threadfence();
-  const int nu = (int)min(misc[99], (uint32_t)p.len);
-  const bool cached = nu <= p.ucache;
-  uint2* uc = reinterpret_cast<uint2*>(smem + Lo.ucache);
+  const int S_ = p.n_split, P = p.ucache;
+  uint2* stage = reinterpret_cast<uint2*>(smem + Lo.ucache);  // [S][P]
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + Lo.cnt);  // [S] counts, then [S + 1] prefix sums
   uint32_t* bm = reinterpret_cast<uint32_t*>(smem + Lo.bitmap);
   uint2* ties = reinterpret_cast<uint2*>(smem + Lo.ties);
   uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + Lo.rscr);
   const int words = (p.len + 31) / 32;
+  const uint2* rows0 = p.cand + (int64_t)row * p.n_split * rstride;
   if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
+  {
+    const int nslots = S_ * (P + 1);
+    for (int base = 0; base < nslots; base += kWdThreads * kWdUnionUnroll) {
+      uint2 e[kWdUnionUnroll];
+#pragma unroll
+      for (int u = 0; u < kWdUnionUnroll; ++u) {
+        const int f = base + u * kWdThreads + tid;
+        e[u] = f < nslots ? __ldcg(rows0 + (int64_t)(f / (P + 1)) * rstride + f % (P + 1)) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kWdUnionUnroll; ++u) {
+        const int f = base + u * kWdThreads + tid;
+        if (f < nslots) {
+          const int sr = f / (P + 1), j = f % (P + 1);
+          if (j == 0) cnt[sr] = min(e[u].x, (uint32_t)p.n_loc);
+          else stage[sr * P + j - 1] = e[u];
+        }
+      }
+    }
+  }
   for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
   for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
   if (tid == 0) misc[100] = 0u;
   __syncthreads();
-  // union entries: global loads batched so that many are in flight
-  auto for_union = [&](auto&& fn, bool from_cache) {
-    if (from_cache) {
-      for (int i = tid; i < nu; i += kWdThreads) fn(i, uc[i]);
-      return;
-    }
-    for (int base = 0; base < nu; base += kWdThreads * kWdUnionUnroll) {
-      uint2 e[kWdUnionUnroll];
+  if (warp == 0) {  // prefix sums of the counts (S <= 32 per pass of the warp)
+    uint32_t run = 0u;
+    for (int s0 = 0; s0 < S_; s0 += 32) {
+      const uint32_t c = s0 + lane < S_ ? cnt[s0 + lane] : 0u;
+      uint32_t incl = c;
 #pragma unroll
-      for (int u = 0; u < kWdUnionUnroll; ++u) {
-        const int i = base + u * kWdThreads + tid;
-        e[u] = i < nu ? __ldcg(crow + i) : make_uint2(0u, 0u);
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += x;
       }
-#pragma unroll
-      for (int u = 0; u < kWdUnionUnroll; ++u) {
-        const int i = base + u * kWdThreads + tid;
-        if (i < nu) fn(i, e[u]);
-      }
+      if (s0 + lane < S_) cnt[S_ + 1 + s0 + lane] = run + incl;
+      run += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
+    if (lane == 0) cnt[S_] = 0u;
+  }
+  __syncthreads();
+  const uint32_t* pre = cnt + S_;  // pre[s] = entries of regions before s; pre[S] = all
+  const int nu = (int)min(pre[S_], (uint32_t)p.len);
+  bool overflow = false;
+  for (int sr = 0; sr < S_; ++sr) overflow |= cnt[sr] > (uint32_t)P;
+  // every union entry once: the staged ones, then (rare) the rest from global memory
+  auto for_union = [&](auto&& fn) {
+    for (int f = tid; f < S_ * P; f += kWdThreads) {
+      const int sr = f / P, j = f % P;
+      if (j < (int)cnt[sr]) fn(stage[f]);
+    }
+    if (overflow)
+      for (int sr = 0; sr < S_; ++sr)
+        for (int j = P + tid; j < (int)cnt[sr]; j += kWdThreads) fn(__ldcg(rows0 + sr * rstride + 1 + j));
   };
-  for_union([&](int i, const uint2& e) {
-    if (cached) uc[i] = e;
-    atomicAdd(hist + (e.x >> 20), 1u);
-  }, false);
+  // entry i of the union in region order (binary search over the prefix sums)
+  auto union_at = [&](int i) -> uint2 {
+    int lo = 0, hi = S_;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int)pre[mid] <= i) lo = mid; else hi = mid;
+    }
+    const int j = i - (int)pre[lo];
+    return j < P ? stage[lo * P + j] : __ldcg(rows0 + lo * rstride + 1 + j);
+  };
+  for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
   __syncthreads();
   int n_keep = p.n_keep;
   if (nu < n_keep) {  // only a workspace that was not zero gets here
@@ -413,7 +475,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   uint32_t B = 0u, above = 0u;
   if (n_keep > 0) hist_threshold_fn([&](int i) { return hist[i]; }, n_keep, misc, B, above);
-  for_union([&](int, const uint2& e) {
+  for_union([&](const uint2& e) {
     const uint32_t b = e.x >> 20;
     if (b > B) {
       wd_keep(bm, e.y, p.len);
@@ -421,7 +483,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       const uint32_t at = atomicAdd(misc + 100, 1u);
       if (at < (uint32_t)kWdTieCap) ties[at] = e;
     }
-  }, cached);
+  });
   __syncthreads();
   const int n_b = (int)misc[100];
   const int need = n_keep - (int)above;
@@ -475,10 +537,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
         wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need2, pre, 20, rscr + 256 + 2 * kWdRankMax, misc,
                          bm, p.len);
       }
-    } else if (cached) {
-      wd_resolve_radix([&](int i) { return uc[i]; }, nu, need, B << 20, 12, rscr, misc, bm, p.len);
     } else {
-      wd_resolve_radix([&](int i) { return __ldcg(crow + i); }, nu, need, B << 20, 12, rscr, misc, bm, p.len);
+      wd_resolve_radix(union_at, nu, need, B << 20, 12, rscr, misc, bm, p.len);
     }
   }
   __syncthreads();
@@ -487,10 +547,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   int* kept = reinterpret_cast<int*>(smem + Lo.kept);
   const int wpt = (words + kWdThreads - 1) / kWdThreads;
   const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
-  uint32_t cnt = 0u;
-  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  uint32_t nbits = 0u;
+  for (int w = w0; w < w1; ++w) nbits += __popc(bm[w]);
   uint32_t total = 0u;
-  uint32_t pos = wd_block_scan(cnt, misc, &total);
+  uint32_t pos = wd_block_scan(nbits, misc, &total);
   if (tid == 0 && total != (uint32_t)n_keep) flag_status(FASA_ERR_WORKSPACE);
   int32_t* io = p.idx_out ? p.idx_out + (int64_t)row * p.n_keep : nullptr;
   int32_t* iw = p.idx_ws ? p.idx_ws + (int64_t)row * p.n_keep : nullptr;
@@ -511,13 +571,11 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int n_att = min((int)total, p.n_keep);
   if (!p.direct) return;  // the split-K attention launch follows
   // the group's attention over the kept rows (at most 16 per warp)
-  float* qs = reinterpret_cast<float*>(smem + Lo.qt);
-  float* zs = qs + MG * kD;
+  const float* qs = reinterpret_cast<const float*>(smem + Lo.qs);
+  float* zs = reinterpret_cast<float*>(smem + Lo.zs);
   float* mo = reinterpret_cast<float*>(smem + Lo.ring);
   float* lsum = mo + kWdWarps * MG * kD;
   __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
-  cc_queries(qraw, G, MG, p.cosv, p.sinv, qs, tid, kWdThreads);
-  __syncthreads();
   cc_block_attend<MG, kWdWarps>(p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD,
                                 [&](int j) -> int { return kept[j]; }, n_att, G, qs, zs, mo, lsum, vst,
                                 p.out + (int64_t)row * G * kD);

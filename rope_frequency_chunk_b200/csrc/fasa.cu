@@ -356,6 +356,10 @@ fasa_status wide_attrs(const DevInfo& d) {
   });
 }
 
+// Published-candidate slots per row in the decode workspace: the CTAs'
+// regions (n_split * (n_loc + 1) entries) stay within len + len/64 + 64.
+inline int64_t wide_region_slots(int64_t len) { return len + len / 64 + 64; }
+
 // CTAs per row: about one per SM over all rows (never fewer than the
 // shared-memory limit on keys per CTA allows); tokens per CTA. The
 // resolving CTA attends itself for budgets up to kWdMaxDirect when its ring
@@ -371,15 +375,17 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   pl->n_split = (int)S;
   pl->n_loc = (int)ceil_div(len, S);
   if (pl->n_loc > kWdMaxLoc || S > 65535) return false;
+  if ((int64_t)pl->n_split * (pl->n_loc + 1) > wide_region_slots(len)) return false;
   const int G = c->n_q_heads / c->n_kv_heads;
   for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
-    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, 0);
+    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0);
     if (base.total > d.smem_optin) continue;
-    // the union cache is the last part of its region: whatever shared memory is left
-    const int64_t uc = std::min<int64_t>(len, std::max<int64_t>(0, (d.smem_optin - base.ucache) / 8));
+    // entries of each CTA's region the resolving CTA stages in shared memory
+    const int64_t room = std::max<int64_t>(0, (int64_t)(d.smem_optin - base.ucache) / (8 * pl->n_split));
     pl->direct = direct;
-    pl->ucache = (int)uc;
-    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->ucache).total;
+    pl->ucache = (int)std::min<int64_t>(pl->n_loc, room);
+    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache).total;
+    if (pl->smem > d.smem_optin) continue;
     return true;
   }
   return false;
@@ -406,8 +412,8 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 // Decode workspace, each part 256-byte aligned:
 //   sem [rows] u64 | att_cnt [rows] u32          (zero between calls: every
 //                                                 call leaves them zero)
-//   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the wide plan,
-//     the published (key, token) pairs [rows][len] u32x2 |
+//   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the fused plan,
+//     the CTAs' published candidates [rows][len + len/64 + 64] u32x2 |
 //   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kCcPartStride] f32
@@ -442,7 +448,7 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.sem = 0;
   w.att_cnt = rows * 8;
   w.scores = al256(w.att_cnt + rows * 4);
-  w.hist = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, L * 8));
+  w.hist = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
   w.cnt = w.hist + rows * kHistBins * 4;
   w.bitmap = al256(w.cnt + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
