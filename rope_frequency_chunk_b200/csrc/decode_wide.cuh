@@ -80,7 +80,8 @@ struct WideParams {
   int32_t n_keep;   // k_eff, 1 .. len
   int32_t n_loc;    // tokens per CTA, <= kWdMaxLoc
   int32_t n_split;  // CTAs per row
-  int32_t ucache;   // entries of each CTA's region the resolving CTA stages in shared memory (P)
+  int32_t ucache;   // entries of each CTA's region the resolving CTA stages in shared memory (P, a power of two)
+  int32_t ushift;   // log2(P)
   int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect, G <= 8)
   double cosv[kNFC];
   double sinv[kNFC];
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   // batched read brings every region's count and first P entries into
   // shared memory (entries beyond P, rare, are read from global memory).
   __threadfence();
-  const int S_ = p.n_split, P = p.ucache;
+  const int S_ = p.n_split, P = p.ucache;  // P: a power of two
   uint2* stage = reinterpret_cast<uint2*>(smem + Lo.ucache);  // [S][P]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + Lo.cnt);  // [S] counts, then [S + 1] prefix sums
   uint32_t* bm = reinterpret_cast<uint32_t*>(smem + Lo.bitmap);
@@ -402,23 +403,22 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int words = (p.len + 31) / 32;
   const uint2* rows0 = p.cand + (int64_t)row * p.n_split * rstride;
   if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
-  {
-    const int nslots = S_ * (P + 1);
+  {  // slots [0, S): the regions' counts; then entry j < P of region s at S + s*P + j
+    const int nslots = S_ + (S_ << p.ushift);
     for (int base = 0; base < nslots; base += kWdThreads * kWdUnionUnroll) {
       uint2 e[kWdUnionUnroll];
 #pragma unroll
       for (int u = 0; u < kWdUnionUnroll; ++u) {
         const int f = base + u * kWdThreads + tid;
-        e[u] = f < nslots ? __ldcg(rows0 + (int64_t)(f / (P + 1)) * rstride + f % (P + 1)) : make_uint2(0u, 0u);
+        const int g = f - S_;
+        const int64_t at = f < S_ ? (int64_t)f * rstride : (int64_t)(g >> p.ushift) * rstride + 1 + (g & (P - 1));
+        e[u] = f < nslots ? __ldcg(rows0 + at) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < kWdUnionUnroll; ++u) {
         const int f = base + u * kWdThreads + tid;
-        if (f < nslots) {
-          const int sr = f / (P + 1), j = f % (P + 1);
-          if (j == 0) cnt[sr] = min(e[u].x, (uint32_t)p.n_loc);
-          else stage[sr * P + j - 1] = e[u];
-        }
+        if (f < S_) cnt[f] = min(e[u].x, (uint32_t)p.n_loc);
+        else if (f < nslots) stage[f - S_] = e[u];
       }
     }
   }
@@ -448,10 +448,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   for (int sr = 0; sr < S_; ++sr) overflow |= cnt[sr] > (uint32_t)P;
   // every union entry once: the staged ones, then (rare) the rest from global memory
   auto for_union = [&](auto&& fn) {
-    for (int f = tid; f < S_ * P; f += kWdThreads) {
-      const int sr = f / P, j = f % P;
-      if (j < (int)cnt[sr]) fn(stage[f]);
-    }
+    for (int f = tid; f < (S_ << p.ushift); f += kWdThreads)
+      if ((f & (P - 1)) < (int)cnt[f >> p.ushift]) fn(stage[f]);
     if (overflow)
       for (int sr = 0; sr < S_; ++sr)
         for (int j = P + tid; j < (int)cnt[sr]; j += kWdThreads) fn(__ldcg(rows0 + sr * rstride + 1 + j));

@@ -343,7 +343,7 @@ std::atomic<int> g_decode_path{FASA_DECODE_AUTO};
 
 // Launch plan of the wide fused decode (decode_wide.cuh).
 struct WidePlan {
-  int n_split = 0, n_loc = 0, direct = 0, ucache = 0, smem = 0;
+  int n_split = 0, n_loc = 0, direct = 0, ucache = 0, ushift = 0, smem = 0;
 };
 
 template <int LPT, int MG>
@@ -380,10 +380,17 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
     const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0);
     if (base.total > d.smem_optin) continue;
-    // entries of each CTA's region the resolving CTA stages in shared memory
-    const int64_t room = std::max<int64_t>(0, (int64_t)(d.smem_optin - base.ucache) / (8 * pl->n_split));
+    // entries of each CTA's region the resolving CTA stages in shared memory:
+    // a power of two covering what a CTA usually publishes (its k_eff best
+    // and the rest of their bin), as far as shared memory allows
+    const int64_t room = std::max<int64_t>(1, (int64_t)(d.smem_optin - base.ucache) / (8 * pl->n_split));
+    const int64_t want = std::min<int64_t>(pl->n_loc, (int64_t)keff + keff / 4 + 64);
+    int64_t P = 1;
+    while (P < want && 2 * P <= room) P *= 2;
     pl->direct = direct;
-    pl->ucache = (int)std::min<int64_t>(pl->n_loc, room);
+    pl->ucache = (int)P;
+    pl->ushift = 0;
+    while ((1 << pl->ushift) < P) ++pl->ushift;
     pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache).total;
     if (pl->smem > d.smem_optin) continue;
     return true;
@@ -608,6 +615,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.n_loc = pl.n_loc;
   p.n_split = pl.n_split;
   p.ucache = pl.ucache;
+  p.ushift = pl.ushift;
   p.direct = pl.direct;
   fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   const int rows = c->batch * c->n_kv_heads;
