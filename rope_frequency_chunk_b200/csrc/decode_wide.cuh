@@ -69,7 +69,8 @@ struct WideParams {
   __nv_bfloat16* out;           // [B][Hq][128]
   int32_t* idx_out;             // [rows][n_keep] kept tokens, ascending, or null
   int32_t* idx_ws;              // [rows][n_keep] for the attention launch, or null (direct)
-  uint2* cand;                  // [rows][n_split][n_loc + 1] regions: count, then (key, token) pairs
+  uint2* cand;                  // [rows][n_split][n_loc + 1] regions: (count, b_loc), then (key, token) pairs
+  uint32_t* keys;               // [rows][len] every token's score key
   unsigned long long* sem;      // [rows], zero between calls
   int64_t max_len;
   int32_t len;
@@ -78,6 +79,7 @@ struct WideParams {
   int32_t group;
   int32_t n_dom;
   int32_t n_keep;   // k_eff, 1 .. len
+  int32_t n_pub;    // each CTA publishes its n_pub best tokens (with the rest of their bin), <= n_keep
   int32_t n_loc;    // tokens per CTA, <= kWdMaxLoc
   int32_t n_split;  // CTAs per row
   int32_t ucache;   // entries of each CTA's region the resolving CTA stages in shared memory (P, a power of two)
@@ -115,8 +117,8 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   o += 2 * kNFC * 8;
   L.qs = o;  // attention queries [MG][128] f32
   o += direct ? MG * kD * 4 : 0;
-  L.cnt = o;  // region counts, then their prefix sums
-  o += wd_al((2 * n_split + 2) * 4, 16);
+  L.cnt = o;  // region counts, their prefix sums, the regions' b_loc
+  o += wd_al((3 * n_split + 2) * 4, 16);
   L.kept = o;
   o += wd_al(direct ? n_keep * 4 : 0, 128);
   L.r1 = o;
@@ -256,6 +258,90 @@ __device__ __forceinline__ void wd_warp_bin256(const uint32_t* h, int k, uint32_
   }
 }
 
+// Exact choice of the n_keep largest keys (ties to the lower token index)
+// among n_src (key, token) entries, given their 4096-bin histogram of the
+// top 12 key bits in hist: sets the kept tokens' bits in bm (zero before).
+// for_src(fn) calls fn(entry) once per entry, spread over the CTA's threads;
+// src_at(i) is entry i (for the rare radix path). *B_out: the boundary bin.
+template <typename ForSrc, typename SrcAt>
+__device__ void wd_select(ForSrc&& for_src, SrcAt&& src_at, int n_src, int n_keep, uint32_t* hist, uint32_t* misc,
+                          uint32_t* bm, uint2* ties, uint32_t* rscr, int len, uint32_t* B_out) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  uint32_t B = 0u, above = 0u;
+  if (n_keep > 0) hist_threshold_fn([&](int i) { return hist[i]; }, n_keep, misc, B, above);
+  if (tid == 0) misc[100] = 0u;
+  __syncthreads();
+  for_src([&](const uint2& e) {
+    const uint32_t b = e.x >> 20;
+    if (b > B) {
+      wd_keep(bm, e.y, len);
+    } else if (b == B) {
+      const uint32_t at = atomicAdd(misc + 100, 1u);
+      if (at < (uint32_t)kWdTieCap) ties[at] = e;
+    }
+  });
+  __syncthreads();
+  const int n_b = (int)misc[100];
+  const int need = n_keep - (int)above;
+  __syncthreads();
+  if (need > 0 && n_keep > 0) {
+    if (n_b == need && n_b <= kWdTieCap) {
+      for (int i = tid; i < n_b; i += kWdThreads) wd_keep(bm, ties[i].y, len);
+    } else if (n_b <= kWdTieCap) {
+      // next 8 key bits of the boundary bin's entries, then ranks (or a
+      // radix select) among the entries of the boundary sub-bin
+      uint32_t* h2 = rscr;             // 256 counts
+      uint2* t2 = reinterpret_cast<uint2*>(rscr + 256);  // the sub-bin's entries
+      for (int i = tid; i < 256; i += kWdThreads) h2[i] = 0u;
+      if (tid == 0) misc[101] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n_b; i += kWdThreads) atomicAdd(h2 + ((ties[i].x >> 12) & 255u), 1u);
+      __syncthreads();
+      if (warp == 0) wd_warp_bin256(h2, need, misc + 102);
+      __syncthreads();
+      const uint32_t B2 = misc[102];
+      const int need2 = need - (int)misc[103];
+      for (int i = tid; i < n_b; i += kWdThreads) {
+        const uint2 e = ties[i];
+        const uint32_t sb = (e.x >> 12) & 255u;
+        if (sb > B2) {
+          wd_keep(bm, e.y, len);
+        } else if (sb == B2) {
+          const uint32_t at = atomicAdd(misc + 101, 1u);
+          if (at < (uint32_t)kWdRankMax) t2[at] = e;
+        }
+      }
+      __syncthreads();
+      const int n_b2 = (int)misc[101];
+      __syncthreads();
+      if (n_b2 == need2 && n_b2 <= kWdRankMax) {
+        for (int i = tid; i < n_b2; i += kWdThreads) wd_keep(bm, t2[i].y, len);
+      } else if (n_b2 <= kWdRankMax) {
+        for (int i = tid; i < n_b2; i += kWdThreads) {
+          const uint2 a = t2[i];
+          int r = 0;
+          for (int j = 0; j < n_b2; ++j) {
+            const uint2 c = t2[j];
+            r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
+          }
+          if (r < need2) wd_keep(bm, a.y, len);
+        }
+      } else {
+        // a crowded sub-bin (ties): exact radix select over the boundary
+        // bin's entries, restricted to the sub-bin by its 20-bit prefix
+        const uint32_t pre = (B << 20) | (B2 << 12);
+        wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need2, pre, 20, rscr + 256 + 2 * kWdRankMax, misc,
+                         bm, len);
+      }
+    } else {
+      wd_resolve_radix(src_at, n_src, need, B << 20, 12, rscr, misc, bm, len);
+    }
+  }
+  __syncthreads();
+
+  *B_out = B;
+}
+
 template <int LPT, int MG>
 __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WideParams p) {
   using S = TipShape<__nv_bfloat16, LPT>;
@@ -340,12 +426,13 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   __syncthreads();
 
-  // 3. the bin holding this CTA's k_eff-th key; publish the tokens at or
-  // above it into the CTA's own region: [count][(key, token) ...]
+  // 3. the bin b_loc holding this CTA's n_pub-th key; publish the tokens at
+  // or above it into the CTA's own region: [(count, b_loc)][(key, token) ...],
+  // and every key to the row's key array
   uint32_t b_loc = 0u;
-  if (n_tok > p.n_keep) {
+  if (n_tok > p.n_pub) {
     uint32_t above = 0u;
-    hist_threshold_fn([&](int i) { return hist[i]; }, p.n_keep, misc, b_loc, above);
+    hist_threshold_fn([&](int i) { return hist[i]; }, p.n_pub, misc, b_loc, above);
   }
   uint32_t wc = 0u;
   for (int i0 = warp * 32; i0 < n_tok; i0 += kWdThreads) {
@@ -378,7 +465,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       if (q) region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
       pos += __popc(m);
     }
-    if (tid == 0) region[0] = make_uint2(misc[96], 0u);
+    if (tid == 0) region[0] = make_uint2(misc[96], b_loc);
+    // every key, for the exact fallback
+    uint32_t* kdst = p.keys + (int64_t)row * p.len + t_beg;
+    for (int i = tid; i < n_tok; i += kWdThreads) kdst[i] = keys[i];
   }
   __threadfence();
   __syncthreads();
@@ -417,7 +507,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
 #pragma unroll
       for (int u = 0; u < kWdUnionUnroll; ++u) {
         const int f = base + u * kWdThreads + tid;
-        if (f < S_) cnt[f] = min(e[u].x, (uint32_t)p.n_loc);
+        if (f < S_) {
+          cnt[f] = min(e[u].x, (uint32_t)p.n_loc);
+          cnt[2 * S_ + 1 + f] = e[u].y;  // the region's b_loc
+        }
         else if (f < nslots) stage[f - S_] = e[u];
       }
     }
@@ -443,6 +536,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   __syncthreads();
   const uint32_t* pre = cnt + S_;  // pre[s] = entries of regions before s; pre[S] = all
+  uint32_t b_max = 0u;  // the highest b_loc: a row boundary bin below it cannot be trusted
+  for (int sr = 0; sr < S_; ++sr) b_max = max(b_max, cnt[2 * S_ + 1 + sr]);
   const int nu = (int)min(pre[S_], (uint32_t)p.len);
   bool overflow = false;
   for (int sr = 0; sr < S_; ++sr) overflow |= cnt[sr] > (uint32_t)P;
@@ -466,80 +561,36 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   };
   for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
   __syncthreads();
-  int n_keep = p.n_keep;
-  if (nu < n_keep) {  // only a workspace that was not zero gets here
-    if (tid == 0) flag_status(FASA_ERR_WORKSPACE);
-    n_keep = nu;
-  }
-  uint32_t B = 0u, above = 0u;
-  if (n_keep > 0) hist_threshold_fn([&](int i) { return hist[i]; }, n_keep, misc, B, above);
-  for_union([&](const uint2& e) {
-    const uint32_t b = e.x >> 20;
-    if (b > B) {
-      wd_keep(bm, e.y, p.len);
-    } else if (b == B) {
-      const uint32_t at = atomicAdd(misc + 100, 1u);
-      if (at < (uint32_t)kWdTieCap) ties[at] = e;
-    }
-  });
-  __syncthreads();
-  const int n_b = (int)misc[100];
-  const int need = n_keep - (int)above;
-  __syncthreads();
-  if (need > 0 && n_keep > 0) {
-    if (n_b == need && n_b <= kWdTieCap) {
-      for (int i = tid; i < n_b; i += kWdThreads) wd_keep(bm, ties[i].y, p.len);
-    } else if (n_b <= kWdTieCap) {
-      // next 8 key bits of the boundary bin's entries, then ranks (or a
-      // radix select) among the entries of the boundary sub-bin
-      uint32_t* h2 = rscr;             // 256 counts
-      uint2* t2 = reinterpret_cast<uint2*>(rscr + 256);  // the sub-bin's entries
-      for (int i = tid; i < 256; i += kWdThreads) h2[i] = 0u;
-      if (tid == 0) misc[101] = 0u;
-      __syncthreads();
-      for (int i = tid; i < n_b; i += kWdThreads) atomicAdd(h2 + ((ties[i].x >> 12) & 255u), 1u);
-      __syncthreads();
-      if (warp == 0) wd_warp_bin256(h2, need, misc + 102);
-      __syncthreads();
-      const uint32_t B2 = misc[102];
-      const int need2 = need - (int)misc[103];
-      for (int i = tid; i < n_b; i += kWdThreads) {
-        const uint2 e = ties[i];
-        const uint32_t sb = (e.x >> 12) & 255u;
-        if (sb > B2) {
-          wd_keep(bm, e.y, p.len);
-        } else if (sb == B2) {
-          const uint32_t at = atomicAdd(misc + 101, 1u);
-          if (at < (uint32_t)kWdRankMax) t2[at] = e;
+  const int n_keep = min(p.n_keep, nu);
+  uint32_t B = 0u;
+  wd_select(for_union, union_at, nu, n_keep, hist, misc, bm, ties, rscr, p.len, &B);
+  if (nu < n_keep || B < b_max) {
+    // some CTA may hold unpublished tokens at or above the boundary: the exact
+    // selection again, over every key of the row
+    const uint32_t* krow = p.keys + (int64_t)row * p.len;
+    auto for_keys = [&](auto&& fn) {
+      for (int base = 0; base < p.len; base += kWdThreads * kWdUnionUnroll) {
+        uint32_t kx[kWdUnionUnroll];
+#pragma unroll
+        for (int u = 0; u < kWdUnionUnroll; ++u) {
+          const int i = base + u * kWdThreads + tid;
+          kx[u] = i < p.len ? __ldcg(krow + i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kWdUnionUnroll; ++u) {
+          const int i = base + u * kWdThreads + tid;
+          if (i < p.len) fn(make_uint2(kx[u], (uint32_t)i));
         }
       }
-      __syncthreads();
-      const int n_b2 = (int)misc[101];
-      __syncthreads();
-      if (n_b2 == need2 && n_b2 <= kWdRankMax) {
-        for (int i = tid; i < n_b2; i += kWdThreads) wd_keep(bm, t2[i].y, p.len);
-      } else if (n_b2 <= kWdRankMax) {
-        for (int i = tid; i < n_b2; i += kWdThreads) {
-          const uint2 a = t2[i];
-          int r = 0;
-          for (int j = 0; j < n_b2; ++j) {
-            const uint2 c = t2[j];
-            r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
-          }
-          if (r < need2) wd_keep(bm, a.y, p.len);
-        }
-      } else {
-        // a crowded sub-bin (ties): exact radix select over the boundary
-        // bin's entries, restricted to the sub-bin by its 20-bit prefix
-        const uint32_t pre = (B << 20) | (B2 << 12);
-        wd_resolve_radix([&](int i) { return ties[i]; }, n_b, need2, pre, 20, rscr + 256 + 2 * kWdRankMax, misc,
-                         bm, p.len);
-      }
-    } else {
-      wd_resolve_radix(union_at, nu, need, B << 20, 12, rscr, misc, bm, p.len);
-    }
+    };
+    auto keys_at = [&](int i) -> uint2 { return make_uint2(__ldcg(krow + i), (uint32_t)i); };
+    for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
+    for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+    __syncthreads();
+    for_keys([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
+    __syncthreads();
+    wd_select(for_keys, keys_at, p.len, p.n_keep, hist, misc, bm, ties, rscr, p.len, &B);
   }
-  __syncthreads();
 
   // ascending emission from the bitmap
   int* kept = reinterpret_cast<int*>(smem + Lo.kept);

@@ -343,7 +343,7 @@ std::atomic<int> g_decode_path{FASA_DECODE_AUTO};
 
 // Launch plan of the wide fused decode (decode_wide.cuh).
 struct WidePlan {
-  int n_split = 0, n_loc = 0, direct = 0, ucache = 0, ushift = 0, smem = 0;
+  int n_split = 0, n_loc = 0, n_pub = 0, direct = 0, ucache = 0, ushift = 0, smem = 0;
 };
 
 template <int LPT, int MG>
@@ -376,6 +376,11 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   pl->n_loc = (int)ceil_div(len, S);
   if (pl->n_loc > kWdMaxLoc || S > 65535) return false;
   if ((int64_t)pl->n_split * (pl->n_loc + 1) > wide_region_slots(len)) return false;
+  // each CTA publishes about twice its expected share of the kept set (and
+  // the rest of its boundary bin); the resolving CTA falls back to every key
+  // of the row when a CTA turns out to hold more of the kept set than that
+  pl->n_pub = pl->n_split == 1 ? keff
+                                : (int)std::min<int64_t>(keff, (2 * ceil_div(keff, pl->n_split) + 32 + 31) / 32 * 32);
   const int G = c->n_q_heads / c->n_kv_heads;
   for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
     const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0);
@@ -384,7 +389,7 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
     // a power of two covering what a CTA usually publishes (its k_eff best
     // and the rest of their bin), as far as shared memory allows
     const int64_t room = std::max<int64_t>(1, (int64_t)(d.smem_optin - base.ucache) / (8 * pl->n_split));
-    const int64_t want = std::min<int64_t>(pl->n_loc, (int64_t)keff + keff / 4 + 64);
+    const int64_t want = std::min<int64_t>(pl->n_loc, (int64_t)pl->n_pub + pl->n_pub / 4 + 32);
     int64_t P = 1;
     while (P < want && 2 * P <= room) P *= 2;
     pl->direct = direct;
@@ -421,6 +426,7 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 //                                                 call leaves them zero)
 //   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the fused plan,
 //     the CTAs' published candidates [rows][len + len/64 + 64] u32x2 |
+//   keys [rows][len] u32 (fused plan: every token's score key) |
 //   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kCcPartStride] f32
@@ -430,7 +436,7 @@ constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
 struct DecodeWs {
-  size_t sem, att_cnt, scores, hist, cnt, bitmap, cand, ckey, idx, part, total;
+  size_t sem, att_cnt, scores, keys, hist, cnt, bitmap, cand, ckey, idx, part, total;
   int64_t ld;
   int cap, words, splits_max;
 };
@@ -455,7 +461,8 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.sem = 0;
   w.att_cnt = rows * 8;
   w.scores = al256(w.att_cnt + rows * 4);
-  w.hist = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
+  w.keys = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
+  w.hist = al256(w.keys + rows * L * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
   w.bitmap = al256(w.cnt + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
@@ -612,6 +619,8 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.group = c->n_q_heads / c->n_kv_heads;
   p.n_dom = c->n_dom;
   p.n_keep = keff;
+  p.n_pub = pl.n_pub;
+  p.keys = reinterpret_cast<uint32_t*>(base + w.keys);
   p.n_loc = pl.n_loc;
   p.n_split = pl.n_split;
   p.ucache = pl.ucache;

@@ -261,6 +261,26 @@ def test_decode_exact_fallbacks(case, path):
         assert idx.cpu().numpy()[0, 0].tolist() == list(range(wl.k))
 
 
+def test_decode_with_clustered_top_scores(path):
+    """The highest scores sit in a few hundred consecutive tokens, inside one
+    or two of the fused plan's CTA slices: such a CTA holds far more of the
+    kept set than it publishes, and the selection must still be exact (the
+    fused plan falls back to every key of the row)."""
+    wl = C["c2"].replace(ctx_len=8192, k=256)
+    inp = W.layer_inputs(wl)
+    for g in range(wl.n_kv_heads):
+        dom = inp.params.dom_idx[g]
+        cols = np.concatenate([dom, dom + 64])
+        blk = W.stored_to_f64(inp.k[0, g, 100:700][:, cols]) * 16.0  # exact: a power of two
+        inp.k[0, g, 100:700][:, cols] = W.round_to_dtype(blk.astype(np.float32), wl.dtype)
+    _, cache, q = U.build(wl, inp=inp)
+    out, idx = _decode(wl, cache, q, wl.k)
+    s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
+    U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
+    kept = idx.cpu().numpy()
+    assert (kept >= 100).all() and (kept < 700).mean() > 0.5  # the cluster dominates the kept sets
+
+
 def test_decode_is_deterministic_and_capturable(path):
     wl = SMALL["c2_ragged"]
     inp, cache, q = U.build(wl)
