@@ -278,7 +278,9 @@ def test_decode_with_clustered_top_scores(path):
     s = F.fasa_score(cache, wl.ctx_len, q, wl.q_pos).cpu().numpy()
     U.check_decode_heads(wl, inp, cache, q, wl.k, U.all_heads(wl), out, idx, scores_gpu=s)
     kept = idx.cpu().numpy()
-    assert (kept >= 100).all() and (kept < 700).mean() > 0.5  # the cluster dominates the kept sets
+    # the cluster holds most of each kept set, so at least one CTA slice
+    # (about 480 tokens at this shape) holds far more than it publishes
+    assert ((kept >= 100) & (kept < 700)).mean() > 0.5
 
 
 def test_decode_is_deterministic_and_capturable(path):
