@@ -380,6 +380,7 @@ def run_fasa(args, wl):
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
     F.lib()
+    F.fasa_set_decode_path({"auto": F.DECODE_AUTO, "fused": F.DECODE_FUSED, "staged": F.DECODE_STAGED}[args.plan])
 
     k = args.k or wl.k
     n_layers = args.layers or default_layers(wl)
@@ -679,6 +680,8 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--ctx-len", type=int, default=0)
     ap.add_argument("--n-dom", type=int, default=0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
+    ap.add_argument("--plan", default="auto", choices=["auto", "fused", "staged"],
+                    help="launch plan of fasa_decode (default: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
