@@ -11,11 +11,13 @@
 // HBM, and float32 fma on CUDA cores keeps up with it at these group sizes.
 //
 // Warp step: 8 rows. Lane l owns head dims 4l .. 4l+3: it loads those 8
-// bytes of each K and V row (a warp reads whole 256-byte rows, coalesced),
-// forms the partial dot products of its 4 dims with every head's query (an
-// fma chain), and a reduce-scatter butterfly over the 32 lanes (5 rounds of
-// shuffles, each halving the values a lane holds) leaves lane l with the
-// full logit of (row l/4, head 4g + l%4) for head group g. Online softmax in
+// bytes of each K and V row, forms the partial dot products of its 4 dims
+// with every head's query (an fma chain), and a reduce-scatter butterfly
+// over the 32 lanes (5 rounds of shuffles, each halving the values a lane
+// holds) leaves lane l with the full logit of (row l/4, head 4g + l%4) for
+// head group g. Each lane takes the rows and heads in an order permuted by
+// its own lane bits, so every round keeps the lower half of the registers
+// and sends the upper half (no selects). Online softmax in
 // base 2 (the 1/sqrt(128) and log2(e) scale is folded into the queries):
 // per-head chunk maxima and sums by shuffles among the lanes of one head,
 // running (m, l) in the warp's shared-memory scratch, probabilities
@@ -99,6 +101,11 @@ __device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep
   float* wm = ws + kCcStep * MG;     // running max [MG]
   float* wl = wm + MG;               // running sum [MG]
   float* wsc = wl + MG;              // rescale of this step [MG]
+  // kk[r'] holds row r' ^ (lane >> 2) (cc_warp_rows loads the rows in that
+  // lane-permuted order), and register r'*4 + h' takes head h' ^ (lane & 3):
+  // register p then holds the partial of logical (row, head) index p ^ lane,
+  // so each butterfly round keeps the lower half of the registers and sends
+  // the upper half, with no selects
   float kf[kCcStep][4];
 #pragma unroll
   for (int r = 0; r < kCcStep; ++r) cc_bf16x4(kk[r], kf[r]);
@@ -106,27 +113,23 @@ __device__ __forceinline__ void cc_step8(CcAcc<MG>& a, const uint2 (&kk)[kCcStep
   const bool row_ok = (valid >> r_me) & 1u;
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
-    float v[32];  // index r * 4 + hh
+    float v[32];  // register p: logical index (p ^ lane) = row * 4 + head
 #pragma unroll
     for (int hh = 0; hh < 4; ++hh) {
-      const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + hh) * kD + 4 * lane);
+      const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + (hh ^ (lane & 3))) * kD + 4 * lane);
 #pragma unroll
       for (int r = 0; r < kCcStep; ++r)
         v[r * 4 + hh] = __fmaf_rn(q4.w, kf[r][3], __fmaf_rn(q4.z, kf[r][2], __fmaf_rn(q4.y, kf[r][1],
                                                                                     __fmul_rn(q4.x, kf[r][0]))));
     }
-    // reduce-scatter: after the round with offset o the lane keeps the half
-    // of its values whose index bit matches its own lane bit o
+    // reduce-scatter: the round with offset o adds the partner's upper half
+    // onto the lower half (the partner's registers i + o hold the logical
+    // indices this lane keeps at registers i)
 #pragma unroll
     for (int s = 0; s < 5; ++s) {
-      const int off = 16 >> s, half = 16 >> s;
-      const bool up = (lane & off) != 0;
+      const int off = 16 >> s;
 #pragma unroll
-      for (int i = 0; i < half; ++i) {
-        const float send = up ? v[i] : v[i + half];
-        const float keep = up ? v[i + half] : v[i];
-        v[i] = __fadd_rn(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
-      }
+      for (int i = 0; i < off; ++i) v[i] = __fadd_rn(v[i], __shfl_xor_sync(0xFFFFFFFFu, v[i + off], off));
     }
     const int h = g * 4 + (lane & 3);
     const float z = row_ok ? v[0] : -INFINITY;
@@ -193,8 +196,10 @@ __device__ __forceinline__ void cc_warp_rows(CcAcc<MG>& a, const __nv_bfloat16* 
 #pragma unroll
     for (int r = 0; r < kCcStep; ++r) {
       int t = __shfl_sync(0xFFFFFFFFu, mine, r);
+      int tk = __shfl_sync(0xFFFFFFFFu, mine, r ^ (lane >> 2));  // K rows in the lane-permuted order
       if (t < 0) t = 0;  // masked out; row 0 is a valid address
-      kk[r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t * kD) + lane);
+      if (tk < 0) tk = 0;
+      kk[r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)tk * kD) + lane);
       asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(vs + r * kD + 4 * lane)),
                    "l"(vb + (int64_t)t * kD + 4 * lane)
                    : "memory");
@@ -428,8 +433,10 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
 #pragma unroll
     for (int r = 0; r < kCcStep; ++r) {
       int t = __shfl_sync(0xFFFFFFFFu, mine, s * kCcStep + r);
+      int tk = __shfl_sync(0xFFFFFFFFu, mine, s * kCcStep + (r ^ (lane >> 2)));  // lane-permuted K rows
       if (t < 0) t = 0;  // masked out; row 0 is a valid address
-      kk[s][r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t * kD) + lane);
+      if (tk < 0) tk = 0;
+      kk[s][r] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)tk * kD) + lane);
       asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(vst + (jb + s * kCcStep + r) * kD + 4 * lane)),
                    "l"(vb + (int64_t)t * kD + 4 * lane)
                    : "memory");
@@ -446,7 +453,7 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
       float v[32];
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + hh) * kD + 4 * lane);
+        const float4 q4 = *reinterpret_cast<const float4*>(qs + (g * 4 + (hh ^ (lane & 3))) * kD + 4 * lane);
 #pragma unroll
         for (int r = 0; r < kCcStep; ++r)
           v[r * 4 + hh] = __fmaf_rn(q4.w, kf[r][3], __fmaf_rn(q4.z, kf[r][2], __fmaf_rn(q4.y, kf[r][1],
@@ -454,14 +461,9 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
       }
 #pragma unroll
       for (int st = 0; st < 5; ++st) {
-        const int off = 16 >> st, half = 16 >> st;
-        const bool up = (lane & off) != 0;
+        const int off = 16 >> st;
 #pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = up ? v[i] : v[i + half];
-          const float keep = up ? v[i + half] : v[i];
-          v[i] = __fadd_rn(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
-        }
+        for (int i = 0; i < off; ++i) v[i] = __fadd_rn(v[i], __shfl_xor_sync(0xFFFFFFFFu, v[i + off], off));
       }
       const int r = s * kCcStep + (lane >> 2);
       zs[(jb + r) * MG + g * 4 + (lane & 3)] = ((valid >> r) & 1u) ? v[0] : -INFINITY;
