@@ -36,6 +36,8 @@
  *    fasa_device_status. The offending element is skipped, never accessed.
  *  - Thread safety: calls may be made from several host threads; the only
  *    library state is the per-device status word and cached device attributes.
+ *  - q_pos, where a call takes it, is the query's absolute position (>= 0) or
+ *    FASA_Q_PREROTATED for queries the caller has rotated already.
  */
 #ifndef FASA_H_
 #define FASA_H_
@@ -55,6 +57,11 @@ extern "C" {
 #define FASA_MAX_LEN (1 << 19)     /* largest cached length a decode call accepts */
 #define FASA_MAX_K (1 << 17)       /* largest kept-token budget */
 #define FASA_CAL_MAX_WIN 8         /* calibration queries per calibration call */
+/* A query position meaning "q is already rotated" (RoPE applied by the
+ * caller): the library applies no rotation. Accepted wherever a call takes
+ * q_pos (not by the calibration calls). Rotation at angle 0 is the identity,
+ * so this equals rotating by position 0. */
+#define FASA_Q_PREROTATED (-1)
 
 typedef enum fasa_status {
   FASA_OK = 0,
@@ -265,6 +272,57 @@ int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
  * needs the split-K attention; the staged plan: 4), or a negative
  * fasa_status for invalid arguments. */
 int32_t fasa_decode_launches(const fasa_cache* cache, int32_t len, int32_t k);
+
+/*
+ * Batches of sequences at different lengths, and per-KV-head budgets
+ * ([tech §3] "Contribuições Principais", versatility: FASA works with
+ * budgets allocated per layer and per head). The lengths live on the device
+ * (a serving loop updates them without a host round trip); the host gives
+ * upper bounds that size the launch and the workspace.
+ *
+ *  seq_len    : device [B] int32: sequence b holds cache slots 0 ..
+ *               seq_len[b]-1 and its query sits at position seq_len[b]
+ *               (or, with q_prerotated, is already rotated). Each value must
+ *               lie in 1 .. max_seq_len; a value outside is clamped into that
+ *               range and flagged FASA_ERR_BAD_INDEX in the status word.
+ *  budget     : device [Hkv] int32, kept tokens for every sequence's KV head
+ *               g, in 1 .. max_budget (clamped and flagged likewise), or
+ *               NULL: max_budget for every head. A layer's call takes that
+ *               layer's budgets, so budgets can differ per layer and per head.
+ *  max_seq_len: host bound, 1 .. cache max_len and <= FASA_MAX_LEN.
+ *  max_budget : host bound, 1 .. FASA_MAX_K.
+ *  q_prerotated: 0: queries are pre-RoPE; 1: already rotated.
+ */
+typedef struct fasa_varlen {
+  const int32_t* seq_len;
+  const int32_t* budget;
+  int32_t max_seq_len;
+  int32_t max_budget;
+  int32_t q_prerotated;
+  int32_t reserved;
+} fasa_varlen;
+
+/* Workspace bytes fasa_decode_varlen needs (0 for invalid arguments). */
+size_t fasa_decode_varlen_workspace_bytes(const fasa_cache* cache, const fasa_varlen* vl);
+
+/*
+ * fasa_decode over sequences of their own lengths with per-head budgets:
+ * for every (b, g), the critical set of the k_eff = min(budget[g],
+ * seq_len[b]) best-scoring tokens of slots 0 .. seq_len[b]-1 and the focused
+ * attention of the group's query heads over it (results equal to fasa_decode
+ * run on that sequence alone at its length and budget). Runs the fused plan
+ * (bf16 caches): the kernels size their work from the device lengths.
+ *
+ *  q       : [B][Hq][128] dtype.
+ *  out     : [B][Hq][128] dtype.
+ *  idx_out : nullable; [B][Hkv][max_budget] int32: the kept tokens of (b, g)
+ *            in ascending order, then -1 up to max_budget.
+ *  workspace: as fasa_decode (zeroed once; at least
+ *            fasa_decode_varlen_workspace_bytes bytes, 256-byte aligned).
+ *  Errors: as fasa_decode; FASA_ERR_UNSUPPORTED for f32 caches.
+ */
+fasa_status fasa_decode_varlen(const fasa_cache* cache, const fasa_varlen* vl, const void* q, void* out,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Size of the library's own device scratch used by
  * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the

@@ -286,7 +286,13 @@ struct CcParams {
   int32_t slice;            // list positions per CTA, a multiple of 8 * kCcWarps
   int32_t splits;
   int32_t group;
-  double cosv[kNFC];        // cos / sin of q_pos * theta_i
+  // per-sequence lengths (fasa_decode_varlen), or null: len and n_keep for
+  // every row (then the upper bounds, n_keep the kept lists' row stride)
+  const int32_t* seq_len;   // [B]
+  const int32_t* row_keep;  // [rows] each row's kept count
+  int32_t n_kv_heads;
+  int32_t q_prerot;         // varlen: 1 if the queries are already rotated
+  double cosv[kNFC];        // cos / sin of q_pos * theta_i; varlen: theta_i in cosv
   double sinv[kNFC];
 };
 
@@ -294,7 +300,7 @@ struct CcParams {
 // float32), warp scratch, warp partials; the split merge reuses the partials.
 __host__ __device__ constexpr int cc_smem_bytes(int MG) {
   return FASA_MAX_GROUP * kD * 2 + MG * kD * 4 + kCcWarps * cc_warp_scratch(MG) * 4 + kCcWarps * MG * kD * 4 +
-         kCcWarps * 2 * kCcStep * kD * 2;
+         kCcWarps * 2 * kCcStep * kD * 2 + 2 * kNFC * 8;
 }
 constexpr int kCcMaxSplits = (kCcWarps * 4 * kD * 4) / (3 * 16 * 4);  // the merge state fits the MG = 4 partials
 
@@ -311,21 +317,37 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   float* wsall = qs + MG * kD;
   float* mo = wsall + kCcWarps * cc_warp_scratch(MG);
   __nv_bfloat16* vball = reinterpret_cast<__nv_bfloat16*>(mo + kCcWarps * MG * kD);
+  double* cs = reinterpret_cast<double*>(vball + kCcWarps * 2 * kCcStep * kD);
   grid_dependency_wait();
   const int split = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.group;
+  int len = p.len, n_keep = p.n_keep;  // the row's length and kept count
+  if (p.seq_len) {
+    len = min(max(__ldg(p.seq_len + row / p.n_kv_heads), 1), p.len);  // range flagged by the fused kernel
+    n_keep = min(max(p.row_keep[row], 0), p.n_keep);
+  }
   {
     const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
     for (int c = tid; c < G * kD / 8; c += kCcThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    if (tid < kNFC) {
+      double sn = p.sinv[tid], cn = p.cosv[tid];
+      if (p.seq_len) {  // the query of sequence b sits at position len
+        sn = 0.0;
+        cn = 1.0;
+        if (!p.q_prerot) sincos((double)len * p.cosv[tid], &sn, &cn);
+      }
+      cs[tid] = cn;
+      cs[kNFC + tid] = sn;
+    }
   }
   __syncthreads();
-  cc_queries(qraw, G, MG, p.cosv, p.sinv, qs, tid, kCcThreads);
+  cc_queries(qraw, G, MG, cs, cs + kNFC, qs, tid, kCcThreads);
   __syncthreads();
   float* ws = wsall + warp * cc_warp_scratch(MG);
   CcAcc<MG> acc;
   cc_init<MG>(acc, ws, lane);
-  const int r_beg = split * p.slice, r_end = min(p.n_keep, r_beg + p.slice);
+  const int r_beg = split * p.slice, r_end = min(n_keep, r_beg + p.slice);
   const int per_warp = ((max(0, r_end - r_beg) + kCcWarps * kCcStep - 1) / (kCcWarps * kCcStep)) * kCcStep;
   const int j0 = min(r_end, r_beg + warp * per_warp), j1 = min(r_end, j0 + per_warp);
   const __nv_bfloat16* kb = p.k + (int64_t)row * p.max_len * kD;
@@ -333,7 +355,7 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   const int32_t* idx = p.idx ? p.idx + (int64_t)row * p.n_keep : nullptr;
   cc_warp_rows<MG>(acc, kb, vb, [&](int j) -> int {
     const int t = idx ? __ldg(idx + j) : j;
-    if (t < 0 || t >= p.len) {
+    if (t < 0 || t >= len) {
       flag_status(FASA_ERR_BAD_INDEX);
       return -1;
     }

@@ -85,9 +85,38 @@ struct WideParams {
   int32_t ucache;   // entries of each CTA's region the resolving CTA stages in shared memory (P, a power of two)
   int32_t ushift;   // log2(P)
   int32_t direct;   // 1: the resolving CTA attends (n_keep <= kWdMaxDirect, G <= 8)
-  double cosv[kNFC];
-  double sinv[kNFC];
+  // per-sequence lengths and per-head budgets (fasa_decode_varlen), or null:
+  // len and n_keep for every row; len and n_keep are then upper bounds and
+  // the row strides of keys and the kept lists
+  const int32_t* seq_len;  // [B]
+  const int32_t* budget;   // [Hkv]
+  int32_t* row_keep;       // [rows] each row's k_eff, for the attention launch (varlen), or null
+  int32_t q_prerot;        // varlen: 1 if the queries are already rotated
+  double cosv[kNFC];       // cos / sin of the query angle (uniform length), or
+  double sinv[kNFC];       // theta_i in cosv (varlen: the angle is seq_len[b] * theta_i)
 };
+
+// The row's length and k_eff: uniform, or from the device arrays (clamped
+// into range, a value outside flagged).
+__device__ __forceinline__ int2 wd_row_shape(const WideParams& p, int row) {
+  int L = p.len, k = p.n_keep;
+  if (p.seq_len) {
+    const int b = row / p.n_kv_heads, g = row % p.n_kv_heads;
+    L = __ldg(p.seq_len + b);
+    if (L < 1 || L > p.len) {
+      if (threadIdx.x == 0) flag_status(FASA_ERR_BAD_INDEX);
+      L = min(max(L, 1), p.len);
+    }
+    if (p.budget) {
+      k = __ldg(p.budget + g);
+      if (k < 1 || k > p.n_keep) {
+        if (threadIdx.x == 0) flag_status(FASA_ERR_BAD_INDEX);
+        k = min(max(k, 1), p.n_keep);
+      }
+    }
+  }
+  return make_int2(L, min(k, L));
+}
 
 __host__ __device__ constexpr int wd_al(int x, int a) { return (x + a - 1) / a * a; }
 
@@ -358,7 +387,12 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, row = blockIdx.y;
   const int t_beg = split * p.n_loc;
-  const int n_tok = max(0, min(p.len - t_beg, p.n_loc));
+  const int2 shp = wd_row_shape(p, row);
+  const int Lr = shp.x, kr = shp.y;  // the row's length and k_eff
+  // each CTA publishes its n_pub best (about twice its share of the kept set)
+  const int n_pub = p.seq_len ? (p.n_split == 1 ? kr : min(kr, (2 * ((kr + p.n_split - 1) / p.n_split) + 63) / 32 * 32))
+                              : p.n_pub;
+  const int n_tok = max(0, min(Lr - t_beg, p.n_loc));
   const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t_beg) * S::ROWB;
   {  // L2 prefetch of this CTA's sketch range: a hint, safe before the wait
     const int64_t bytes = (int64_t)n_tok * S::ROWB;
@@ -379,8 +413,15 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
     for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
     if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
-    if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
-    else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
+    if (!p.seq_len) {
+      if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
+      else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
+    } else if (tid < kNFC) {  // the query of sequence b sits at position Lr
+      double sn = 0.0, cn = 1.0;
+      if (!p.q_prerot) sincos((double)Lr * p.cosv[tid], &sn, &cn);
+      cs_sm[tid] = cn;
+      cs_sm[kNFC + tid] = sn;
+    }
   }
   constexpr int kTokPass = kWdThreads / S::LPT2;
   const int my_tok = tid / S::LPT2;
@@ -430,9 +471,9 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   // or above it into the CTA's own region: [(count, b_loc)][(key, token) ...],
   // and every key to the row's key array
   uint32_t b_loc = 0u;
-  if (n_tok > p.n_pub) {
+  if (n_tok > n_pub) {
     uint32_t above = 0u;
-    hist_threshold_fn([&](int i) { return hist[i]; }, p.n_pub, misc, b_loc, above);
+    hist_threshold_fn([&](int i) { return hist[i]; }, n_pub, misc, b_loc, above);
   }
   uint32_t wc = 0u;
   for (int i0 = warp * 32; i0 < n_tok; i0 += kWdThreads) {
@@ -490,7 +531,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   uint32_t* bm = reinterpret_cast<uint32_t*>(smem + Lo.bitmap);
   uint2* ties = reinterpret_cast<uint2*>(smem + Lo.ties);
   uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + Lo.rscr);
-  const int words = (p.len + 31) / 32;
+  const int words = (Lr + 31) / 32;
   const uint2* rows0 = p.cand + (int64_t)row * p.n_split * rstride;
   if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
   {  // slots [0, S): the regions' counts; then entry j < P of region s at S + s*P + j
@@ -561,25 +602,25 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   };
   for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
   __syncthreads();
-  const int n_keep = min(p.n_keep, nu);
+  const int n_keep = min(kr, nu);
   uint32_t B = 0u;
-  wd_select(for_union, union_at, nu, n_keep, hist, misc, bm, ties, rscr, p.len, &B);
-  if (nu < n_keep || B < b_max) {
+  wd_select(for_union, union_at, nu, n_keep, hist, misc, bm, ties, rscr, Lr, &B);
+  if (nu < kr || B < b_max) {
     // some CTA may hold unpublished tokens at or above the boundary: the exact
     // selection again, over every key of the row
     const uint32_t* krow = p.keys + (int64_t)row * p.len;
     auto for_keys = [&](auto&& fn) {
-      for (int base = 0; base < p.len; base += kWdThreads * kWdUnionUnroll) {
+      for (int base = 0; base < Lr; base += kWdThreads * kWdUnionUnroll) {
         uint32_t kx[kWdUnionUnroll];
 #pragma unroll
         for (int u = 0; u < kWdUnionUnroll; ++u) {
           const int i = base + u * kWdThreads + tid;
-          kx[u] = i < p.len ? __ldcg(krow + i) : 0u;
+          kx[u] = i < Lr ? __ldcg(krow + i) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < kWdUnionUnroll; ++u) {
           const int i = base + u * kWdThreads + tid;
-          if (i < p.len) fn(make_uint2(kx[u], (uint32_t)i));
+          if (i < Lr) fn(make_uint2(kx[u], (uint32_t)i));
         }
       }
     };
@@ -589,7 +630,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     __syncthreads();
     for_keys([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
     __syncthreads();
-    wd_select(for_keys, keys_at, p.len, p.n_keep, hist, misc, bm, ties, rscr, p.len, &B);
+    wd_select(for_keys, keys_at, Lr, kr, hist, misc, bm, ties, rscr, Lr, &B);
   }
 
   // ascending emission from the bitmap
@@ -600,7 +641,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   for (int w = w0; w < w1; ++w) nbits += __popc(bm[w]);
   uint32_t total = 0u;
   uint32_t pos = wd_block_scan(nbits, misc, &total);
-  if (tid == 0 && total != (uint32_t)n_keep) flag_status(FASA_ERR_WORKSPACE);
+  if (tid == 0 && total != (uint32_t)kr) flag_status(FASA_ERR_WORKSPACE);
   int32_t* io = p.idx_out ? p.idx_out + (int64_t)row * p.n_keep : nullptr;
   int32_t* iw = p.idx_ws ? p.idx_ws + (int64_t)row * p.n_keep : nullptr;
   for (int w = w0; w < w1; ++w) {
@@ -608,7 +649,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     while (bits) {
       const int t = w * 32 + __ffs(bits) - 1;
       bits &= bits - 1u;
-      if (pos < (uint32_t)p.n_keep) {
+      if (pos < (uint32_t)kr) {
         if (p.direct) kept[pos] = t;
         if (io) io[pos] = t;
         if (iw) iw[pos] = t;
@@ -616,8 +657,14 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       ++pos;
     }
   }
+  if (kr < p.n_keep)  // a shorter row: pad its kept lists
+    for (int j = kr + tid; j < p.n_keep; j += kWdThreads) {
+      if (io) io[j] = -1;
+      if (iw) iw[j] = -1;
+    }
+  if (p.row_keep && tid == 0) p.row_keep[row] = kr;
   __syncthreads();
-  const int n_att = min((int)total, p.n_keep);
+  const int n_att = min((int)total, kr);
   if (!p.direct) return;  // the split-K attention launch follows
   // the group's attention over the kept rows (at most 16 per warp)
   const float* qs = reinterpret_cast<const float*>(smem + Lo.qs);

@@ -56,6 +56,8 @@ fasa_status device_info(DevInfo* out) {
   return FASA_OK;
 }
 
+// A query position: >= 0, or FASA_Q_PREROTATED.
+inline bool bad_qpos(int32_t q_pos) { return q_pos < 0 && q_pos != FASA_Q_PREROTATED; }
 inline bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int pow2ceil(int64_t x) {
@@ -71,6 +73,13 @@ void fill_theta(double* th, double base) {
 
 // cos / sin of the query's rotation angle pos * theta_i, float64 on the host.
 void fill_query_angle(double* cosv, double* sinv, double base, int32_t pos) {
+  if (pos == FASA_Q_PREROTATED) {  // q is already rotated: the identity
+    for (int i = 0; i < kNFC; ++i) {
+      cosv[i] = 1.0;
+      sinv[i] = 0.0;
+    }
+    return;
+  }
   double th[kNFC];
   fill_theta(th, base);
   for (int i = 0; i < kNFC; ++i) {
@@ -434,7 +443,7 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 //                                                 call leaves them zero)
 //   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the fused plan,
 //     the CTAs' published candidates [rows][len + len/64 + 64] u32x2 |
-//   keys [rows][len] u32 (fused plan: every token's score key) |
+//   keys [rows][len] u32 (fused plan: every token's score key) | rowk [rows] i32 (varlen: each row's k_eff) |
 //   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kCcPartStride] f32
@@ -444,7 +453,7 @@ constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
 struct DecodeWs {
-  size_t sem, att_cnt, scores, keys, hist, cnt, bitmap, cand, ckey, idx, part, total;
+  size_t sem, att_cnt, scores, keys, rowk, hist, cnt, bitmap, cand, ckey, idx, part, total;
   int64_t ld;
   int cap, words, splits_max;
 };
@@ -470,7 +479,8 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.att_cnt = rows * 8;
   w.scores = al256(w.att_cnt + rows * 4);
   w.keys = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
-  w.hist = al256(w.keys + rows * L * 4);
+  w.rowk = al256(w.keys + rows * L * 4);
+  w.hist = al256(w.rowk + rows * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
   w.bitmap = al256(w.cnt + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
@@ -560,7 +570,8 @@ fasa_status launch_attend_t(CcParams& ap, int rows, int splits_max, const DevInf
 
 fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
                           const void* q, int32_t q_pos, float* part, uint32_t* counter, int splits_max,
-                          const DevInfo& d, cudaStream_t st) {
+                          const DevInfo& d, cudaStream_t st, const fasa_varlen* vl = nullptr,
+                          const int32_t* row_keep = nullptr) {
   const int rows = c->batch * c->n_kv_heads;
   CcParams ap{};
   ap.k = static_cast<const __nv_bfloat16*>(c->k);
@@ -574,7 +585,15 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
   ap.len = len;
   ap.n_keep = n_keep;
   ap.group = c->n_q_heads / c->n_kv_heads;
-  fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
+  ap.n_kv_heads = c->n_kv_heads;
+  if (vl) {  // per-row lengths and kept counts; the angles from the lengths on the device
+    ap.seq_len = vl->seq_len;
+    ap.row_keep = row_keep;
+    ap.q_prerot = vl->q_prerotated;
+    fill_theta(ap.cosv, c->rope_base);
+  } else {
+    fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
+  }
   if (ap.group <= 4) return launch_attend_t<4>(ap, rows, splits_max, d, st);
   if (ap.group <= 8) return launch_attend_t<8>(ap, rows, splits_max, d, st);
   return launch_attend_t<16>(ap, rows, splits_max, d, st);
@@ -582,10 +601,11 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
 
 // The decode's attention over the kept lists in the workspace.
 fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, const void* q, int32_t q_pos, void* out,
-                             const DecodeWs& w, char* base, const DevInfo& d, cudaStream_t st) {
+                             const DecodeWs& w, char* base, const DevInfo& d, cudaStream_t st,
+                             const fasa_varlen* vl = nullptr) {
   return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx), q, q_pos,
                        reinterpret_cast<float*>(base + w.part), reinterpret_cast<uint32_t*>(base + w.att_cnt),
-                       w.splits_max, d, st);
+                       w.splits_max, d, st, vl, reinterpret_cast<const int32_t*>(base + w.rowk));
 }
 
 // Dense decode workspace: att_cnt [rows] u32 (zero between calls) | part
@@ -608,7 +628,7 @@ DenseWs dense_layout(const fasa_cache* c, int32_t len) {
 // budget is beyond what the resolving CTA attends itself.
 fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int keff, void* out,
                         int32_t* idx_out, const DecodeWs& w, char* base, const WidePlan& pl, const DevInfo& d,
-                        cudaStream_t st) {
+                        cudaStream_t st, const fasa_varlen* vl = nullptr) {
   WideParams p{};
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
@@ -634,7 +654,15 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   p.ucache = pl.ucache;
   p.ushift = pl.ushift;
   p.direct = pl.direct;
-  fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
+  if (vl) {  // per-sequence lengths and per-head budgets; len and keff are their bounds
+    p.seq_len = vl->seq_len;
+    p.budget = vl->budget;
+    p.row_keep = pl.direct ? nullptr : reinterpret_cast<int32_t*>(base + w.rowk);
+    p.q_prerot = vl->q_prerotated;
+    fill_theta(p.cosv, c->rope_base);
+  } else {
+    fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
+  }
   const int rows = c->batch * c->n_kv_heads;
   fasa_status s;
   const bool g4 = p.group <= 4;  // padded heads of the in-CTA attention: 4 or 8
@@ -647,7 +675,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
     default: return FASA_ERR_UNSUPPORTED;
   }
   if (s != FASA_OK || pl.direct) return s;
-  return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st);
+  return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st, vl);
 }
 
 }  // namespace
@@ -735,7 +763,7 @@ fasa_status fasa_score(const fasa_cache* c, int32_t len, const void* q, int32_t 
                        cudaStream_t stream) {
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
-  if (len < 0 || q_pos < 0) return FASA_ERR_INVALID_ARG;
+  if (len < 0 || bad_qpos(q_pos)) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (len == 0) return FASA_OK;
   if (!aligned(q, 16) || !aligned(scores, 4)) return FASA_ERR_INVALID_ARG;
@@ -760,7 +788,7 @@ fasa_status fasa_sparse_attend(const fasa_cache* c, int32_t len, const void* q, 
                                const int32_t* idx, int32_t n_idx, void* out, cudaStream_t stream) {
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
-  if (len < 1 || q_pos < 0 || n_idx < 1) return FASA_ERR_INVALID_ARG;
+  if (len < 1 || bad_qpos(q_pos) || n_idx < 1) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (n_idx > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(idx, 4)) return FASA_ERR_INVALID_ARG;
@@ -787,7 +815,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
                         int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
-  if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
+  if (len < 1 || bad_qpos(q_pos) || k < 1) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (len > FASA_MAX_LEN || k > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
@@ -914,13 +942,47 @@ int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
   return pl.direct ? 1 : 2;
 }
 
+// Host checks of a varlen description against the cache.
+fasa_status check_varlen(const fasa_cache* c, const fasa_varlen* vl) {
+  if (vl == nullptr || !aligned(vl->seq_len, 4)) return FASA_ERR_INVALID_ARG;
+  if (vl->budget != nullptr && !aligned(vl->budget, 4)) return FASA_ERR_INVALID_ARG;
+  if (vl->max_seq_len < 1 || vl->max_budget < 1 || (vl->q_prerotated != 0 && vl->q_prerotated != 1))
+    return FASA_ERR_INVALID_ARG;
+  if (vl->max_seq_len > c->max_len) return FASA_ERR_CAPACITY;
+  if (vl->max_seq_len > FASA_MAX_LEN || vl->max_budget > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
+  return FASA_OK;
+}
+
+size_t fasa_decode_varlen_workspace_bytes(const fasa_cache* c, const fasa_varlen* vl) {
+  if (check_cache(c) != FASA_OK || check_varlen(c, vl) != FASA_OK) return 0;
+  return decode_ws(c, vl->max_seq_len, vl->max_budget);
+}
+
+fasa_status fasa_decode_varlen(const fasa_cache* c, const fasa_varlen* vl, const void* q, void* out,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if ((s = check_varlen(c, vl)) != FASA_OK) return s;
+  if (c->dtype != FASA_BF16) return FASA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  if (idx_out != nullptr && !aligned(idx_out, 4)) return FASA_ERR_INVALID_ARG;
+  const int32_t len = vl->max_seq_len, keff = std::min(vl->max_budget, vl->max_seq_len);
+  const DecodeWs w = decode_layout(c, len, vl->max_budget);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return FASA_ERR_WORKSPACE;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return s;
+  WidePlan pl;
+  if (!wide_plan(c, len, keff, d, &pl)) return FASA_ERR_UNSUPPORTED;
+  return launch_wide(c, len, q, 0, keff, out, idx_out, w, static_cast<char*>(workspace), pl, d, stream, vl);
+}
+
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,
                                        void* out, int32_t* idx_out, cudaStream_t stream) {
   // fasa_decode's own checks first, so a call both unsupported and too large
   // gets the same status as from fasa_decode; then the scratch limit
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
-  if (len < 1 || q_pos < 0 || k < 1) return FASA_ERR_INVALID_ARG;
+  if (len < 1 || bad_qpos(q_pos) || k < 1) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (len > FASA_MAX_LEN || k > FASA_MAX_K) return FASA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
@@ -944,7 +1006,7 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fasa_status s = check_cache(c);
   if (s != FASA_OK) return s;
-  if (len < 1 || q_pos < 0) return FASA_ERR_INVALID_ARG;
+  if (len < 1 || bad_qpos(q_pos)) return FASA_ERR_INVALID_ARG;
   if (len > c->max_len) return FASA_ERR_CAPACITY;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
   const DenseWs w = dense_layout(c, len);

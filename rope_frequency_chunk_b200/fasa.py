@@ -39,6 +39,11 @@ class fasa_cache(ctypes.Structure):
                 ("dom_idx", ctypes.c_void_p)]
 
 
+class fasa_varlen(ctypes.Structure):
+    _fields_ = [("seq_len", ctypes.c_void_p), ("budget", ctypes.c_void_p), ("max_seq_len", ctypes.c_int32),
+                ("max_budget", ctypes.c_int32), ("q_prerotated", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -57,6 +62,8 @@ _SIGS = {
     "fasa_decode_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I]),
     "fasa_decode_launches": (_I, [_CP, _I, _I]),
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fasa_decode_varlen_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.POINTER(fasa_varlen)]),
+    "fasa_decode_varlen": (_I, [_CP, ctypes.POINTER(fasa_varlen), _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]),
@@ -237,6 +244,53 @@ def fasa_decode(cache: KVCache, length: int, q, q_pos: int, k: int, out=None, id
     _dev(workspace, "workspace", torch.uint8)
     _check(lib().fasa_decode(cache.ref(), length, q.data_ptr(), q_pos, k, out.data_ptr(), _ptr(idx_out),
                              workspace.data_ptr(), workspace.numel(), _stream(stream)), "fasa_decode")
+    return out
+
+
+def _varlen(seq_len, budget, max_seq_len: int, max_budget: int, q_prerotated: bool):
+    """The C description of a varlen call; seq_len [B] and budget [Hkv]
+    (or None) are int32 device tensors."""
+    if seq_len is not None:
+        _dev(seq_len, "seq_len", torch.int32)
+    if budget is not None:
+        _dev(budget, "budget", torch.int32)
+    return fasa_varlen(_ptr(seq_len), _ptr(budget), int(max_seq_len), int(max_budget),
+                       1 if q_prerotated else 0, 0)
+
+
+def fasa_decode_varlen_workspace_bytes(cache: KVCache, max_seq_len: int, max_budget: int) -> int:
+    d = fasa_varlen(None, None, int(max_seq_len), int(max_budget), 0, 0)
+    d.seq_len = 16  # any aligned non-null value: only the bounds size the workspace
+    return int(lib().fasa_decode_varlen_workspace_bytes(cache.ref(), ctypes.byref(d)))
+
+
+def fasa_decode_varlen_workspace(cache: KVCache, max_seq_len: int, max_budget: int, device=None):
+    """A zeroed workspace for fasa_decode_varlen with these bounds."""
+    dev = device if device is not None else cache.k.device
+    need = fasa_decode_varlen_workspace_bytes(cache, max_seq_len, max_budget)
+    return torch.zeros(max(need, 1), dtype=torch.uint8, device=dev)
+
+
+def fasa_decode_varlen(cache: KVCache, seq_len, q, max_seq_len: int, max_budget: int, budget=None,
+                       q_prerotated: bool = False, out=None, idx_out=None, workspace=None, stream=None):
+    """One decode step over sequences of their own lengths (seq_len, int32
+    [B] on the device; the query of sequence b sits at position seq_len[b])
+    with per-KV-head budgets (budget, int32 [Hkv] on the device, or None for
+    max_budget everywhere). idx_out, when given, is int32 [B][Hkv][max_budget]:
+    each row's kept tokens ascending, then -1."""
+    _q(cache, q)
+    vl = _varlen(seq_len, budget, max_seq_len, max_budget, q_prerotated)
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    if idx_out is not None:
+        _dev(idx_out, "idx_out", torch.int32)
+    if workspace is None:
+        workspace = fasa_decode_varlen_workspace(cache, max_seq_len, max_budget, q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_decode_varlen(cache.ref(), ctypes.byref(vl), q.data_ptr(), out.data_ptr(), _ptr(idx_out),
+                                    workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "fasa_decode_varlen")
     return out
 
 

@@ -81,11 +81,16 @@ def check_append(wl, inp, cache, heads, length=None):
     return worst
 
 
-def oracle_scores(wl, inp, cache, b, g, length=None):
+def oracle_scores(wl, inp, cache, b, g, length=None, q_rot=None):
+    """The oracle's rotated group queries, TIP scores and sum_j |c_j| |x_j| of
+    (b, g) over the first `length` slots; the query sits at position
+    `length` (default: the workload's), or q_rot gives it already rotated."""
     L = length or wl.ctx_len
     dom = inp.params.dom_idx[g]
     G = wl.group
-    q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos if length is None else length, wl.rope_base)
+    if q_rot is None:
+        q_rot = O.rotate_queries(inp.q[b, g * G:(g + 1) * G], wl.q_pos if length is None else length,
+                                 wl.rope_base)
     sk = stored(cache.sketch[b, g, :L])[:, :2 * len(dom)]
     s = O.tip_scores(q_rot, sk, dom)
     qd = O.sketch_rows(q_rot, dom)

@@ -140,3 +140,36 @@ def test_calibration_validation_without_launch(L):
     assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 4, 0x60000, 0x70000, None, need, None) == 4
     assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 4, 0x60000, 0x70000, 0x80000, need - 1, None) == 4
     assert L.fasa_calibrate(c, 100, 0x50000, 0, 2, 8, 0, 0x60000, 0x70000, 0x80000, need, None) == 1
+
+
+def test_varlen_validation_without_launch(L):
+    c = ctypes.byref(_fake_cache())
+
+    def vl(**kw):
+        d = dict(seq_len=0x90000, budget=None, max_seq_len=100, max_budget=8, q_prerotated=0, reserved=0)
+        d.update(kw)
+        return ctypes.byref(F.fasa_varlen(**d))
+
+    ws = L.fasa_decode_varlen_workspace_bytes
+    need = ws(c, vl())
+    assert need > 0 and need % 256 == 0
+    # the bounds size the workspace like a uniform call at those bounds
+    assert need == L.fasa_decode_workspace_bytes(c, 100, 8)
+    assert ws(c, None) == 0 and ws(c, vl(seq_len=None)) == 0 and ws(c, vl(max_seq_len=0)) == 0
+    run = L.fasa_decode_varlen
+    args = (0x50000, 0x70000, None, 0x80000, need, None)
+    assert run(c, None, *args) == 1                                  # no description
+    assert run(c, vl(seq_len=None), *args) == 1                      # no lengths
+    assert run(c, vl(seq_len=0x90002), *args) == 1                   # misaligned lengths
+    assert run(c, vl(budget=0x90001), *args) == 1                    # misaligned budgets
+    assert run(c, vl(max_seq_len=0), *args) == 1
+    assert run(c, vl(max_budget=0), *args) == 1
+    assert run(c, vl(q_prerotated=2), *args) == 1
+    assert run(c, vl(max_seq_len=2000), *args) == 3                  # beyond the cache
+    assert run(c, vl(max_budget=(1 << 17) + 1), *args) == 2
+    assert run(ctypes.byref(_fake_cache(dtype=0)), vl(), *args) == 2  # f32 caches: fused plan only
+    assert run(c, vl(), 0x50008, 0x70000, None, 0x80000, need, None) == 1   # misaligned q
+    assert run(c, vl(), 0x50000, 0x70000, 0x60002, 0x80000, need, None) == 1
+    assert run(c, vl(), 0x50000, 0x70000, None, None, need, None) == 4
+    assert run(c, vl(), 0x50000, 0x70000, None, 0x80000, need - 1, None) == 4
+    assert run(c, vl(), 0x50000, 0x70000, None, 0x80010, need, None) == 4  # workspace alignment
