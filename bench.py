@@ -291,14 +291,14 @@ def run_reference(args, wl):
 
 # ---------------------------------------------------------------- GPU leg
 
-def build_stack(wl, n_layers, device):
+def build_stack(wl, n_layers, device, kv_on_host=False):
     import torch
     from rope_frequency_chunk_b200 import fasa as F
     caches, qs = [], []
     for layer in range(n_layers):
         inp = W.layer_inputs(wl, layer=layer)
         c = F.KVCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.n_dom, wl.ctx_len, wl.dtype, wl.rope_base,
-                      inp.params.dom_idx, device=device)
+                      inp.params.dom_idx, device=device, kv_on_host=kv_on_host)
         k = W.to_torch(inp.k, device)
         v = W.to_torch(inp.v, device)
         F.fasa_append_kv(c, k, v, 0)
@@ -360,6 +360,66 @@ def job_gbs(bytes_per_rank_step: float, ms_per_step: float, world: int) -> float
     """Whole-job GB/s: every rank moved bytes_per_rank_step per step, and a step
     took ms_per_step (the slowest rank's time)."""
     return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
+FASA_M_MAX_HOST_BYTES = 16 << 30
+
+
+def link_copy_gbs(device, nbytes=256 << 20, reps=5):
+    """Pinned host -> device copy bandwidth (the host link as the copy engine
+    sees it), CUDA events on the copying stream."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    st = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(st):
+        dst.copy_(src, non_blocking=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(reps):
+            dst.copy_(src, non_blocking=True)
+        e1.record(st)
+    torch.cuda.synchronize()
+    return reps * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+
+def run_fasa_m(args, wl, k, n_layers, qs, outs, ws, stream, fasa_c_bytes):
+    """FASA-M: the same decode on caches whose K and V sit in pinned host
+    memory (only the sketch on the device); kept rows cross the host link."""
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+    hcaches, _ = build_stack(wl, n_layers, qs[0].device, kv_on_host=True)
+    L = wl.ctx_len
+
+    def m_step():
+        for c, q, o in zip(hcaches, qs, outs):
+            F.fasa_decode(c, L, q, wl.q_pos, k, out=o, workspace=ws)
+
+    msteps = max(3, args.steps // 4)
+    per = []
+    ms = time_graph(m_step, msteps, args.warmup, stream, None, per_step=per) / msteps
+    status = F.fasa_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the FASA-M decode")
+    link_bytes = wl.batch * wl.n_kv_heads * min(k, L) * 2 * W.HEAD_DIM * wl.elem_bytes
+    copy_gbs = link_copy_gbs(qs[0].device)
+    us = 1e3 * ms / n_layers
+    res = {"us_per_layer_step": us,
+           "us_per_layer_step_percentiles": {f"p{p}": float(np.percentile(per, p)) * 1e3 / n_layers
+                                             for p in (10, 50, 90)},
+           "gpu_resident_bytes_per_layer": hcaches[0].device_bytes(),
+           "fasa_c_resident_bytes_per_layer": fasa_c_bytes,
+           "gpu_memory_compression": fasa_c_bytes / hcaches[0].device_bytes(),
+           "link_bytes_per_layer_step": link_bytes,
+           "link_gbs": link_bytes / (us * 1e-6) / 1e9,
+           "link_copy_gbs": copy_gbs,
+           "link_frac_of_copy": link_bytes / (us * 1e-6) / 1e9 / copy_gbs,
+           "hbm_bytes_per_layer_step": roofline_bytes(wl, k) - link_bytes,
+           "note": "K and V in pinned host memory read by the kernels across the host link; the sketch, "
+                   "queries and outputs in HBM; link_copy_gbs is a pinned host-to-device copy for scale"}
+    del hcaches
+    torch.cuda.synchronize()
+    return res
 
 
 def run_fasa(args, wl):
@@ -450,6 +510,14 @@ def run_fasa(args, wl):
         extra["dense_us_per_layer_step"] = 1e3 * ms_dense / n_layers
         extra["dense_gbs"] = dense_bytes(wl) * n_layers / (ms_dense * 1e-3) / 1e9
         extra["speedup_vs_dense"] = ms_dense / ms_step
+
+    kv_host_bytes = 2 * wl.batch * wl.n_kv_heads * L * W.HEAD_DIM * wl.elem_bytes * n_layers
+    if not args.no_fasa_m and world == 1 and kv_host_bytes <= FASA_M_MAX_HOST_BYTES:
+        extra["fasa_m"] = run_fasa_m(args, wl, k, n_layers, qs, outs, ws, stream, caches[0].device_bytes())
+    elif not args.no_fasa_m:
+        extra["fasa_m"] = {"skipped": f"host K/V of {kv_host_bytes / 2**30:.1f} GiB for {n_layers} layers "
+                                      f"exceeds the {FASA_M_MAX_HOST_BYTES / 2**30:.0f} GiB bound"
+                           if world == 1 else "one GPU only"}
 
     e2e = None
     if not args.no_e2e:
@@ -684,6 +752,7 @@ def build_parser() -> argparse.ArgumentParser:
                     help="launch plan of fasa_decode (default: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-fasa-m", action="store_true", help="skip the FASA-M (host-resident K/V) leg")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--calibrate", action="store_true",

@@ -133,6 +133,36 @@ int32_t fasa_sketch_stride(int32_t n_dom, int32_t dtype);
 fasa_status fasa_check_dom_idx(const int32_t* dom_idx_host, int32_t n_kv_heads, int32_t n_dom);
 
 /*
+ * FASA-M, the memory-optimised variant ([tech §2] "Variantes de
+ * Implementação": the value cache and the non-dominant key parts are moved
+ * to CPU memory, only what scoring needs stays on the GPU; [tech §4]
+ * Eficiência/Compressão: 8x smaller KV cache on the GPU).
+ *
+ * A cache is FASA-M when its k and v point into pinned host memory that the
+ * device can address, while sketch and dom_idx stay in device memory. Then
+ * the GPU holds 2*n_dom of the 256 K and V values of a token (8x less at
+ * n_dom = 16). The keys are kept whole on the host (their dominant dims are
+ * also in the sketch), so the attention reads a kept row in one piece. Every
+ * call works on such a cache unchanged:
+ *  - fasa_append_kv writes K_rot and V through the host link and the sketch
+ *    to device memory.
+ *  - A decode streams the sketch from HBM, selects, and then reads only the
+ *    k_eff kept K and V rows of each (b, g) across the host link, 2 * 128 *
+ *    es bytes per kept token.
+ *  - fasa_dense_decode reads all of K and V across the link (correct, slow;
+ *    bf16 caches only: FASA_ERR_UNSUPPORTED for an f32 FASA-M cache).
+ *
+ * fasa_host_kv_pointer returns in *device_ptr the address under which the
+ * device reads the pinned host range starting at host_ptr, for use as
+ * fasa_cache.k or .v. The range must lie in an allocation pinned with
+ * cudaHostAlloc / cudaMallocHost (mapped; with unified addressing every such
+ * allocation is) or registered with cudaHostRegister(cudaHostRegisterMapped).
+ * Errors: NULL arguments or memory the device cannot address ->
+ * FASA_ERR_INVALID_ARG (no CUDA error is left pending).
+ */
+fasa_status fasa_host_kv_pointer(void* host_ptr, void** device_ptr);
+
+/*
  * Append n_new tokens at positions pos0 .. pos0+n_new-1 of every sequence.
  * [tech §2] "A Descoberta" (RoPE rotates each FC at its own frequency) and
  * FAC (positions are kept absolute): each key is rotated at its own position

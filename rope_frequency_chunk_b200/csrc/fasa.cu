@@ -106,6 +106,16 @@ fasa_status check_cache(const fasa_cache* c) {
   return FASA_OK;
 }
 
+// True when p lies in host memory (a FASA-M cache's K or V).
+bool host_resident(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
 thread_local const char* t_last_cuda_error = "no error";
 
 fasa_status cuda_status(cudaError_t e) {
@@ -723,6 +733,18 @@ fasa_status fasa_check_dom_idx(const int32_t* dom, int32_t n_kv_heads, int32_t n
   return FASA_OK;
 }
 
+fasa_status fasa_host_kv_pointer(void* host, void** dev) {
+  if (host == nullptr || dev == nullptr) return FASA_ERR_INVALID_ARG;
+  void* d = nullptr;
+  const cudaError_t e = cudaHostGetDevicePointer(&d, host, 0);
+  if (e != cudaSuccess || d == nullptr) {
+    (void)cudaGetLastError();
+    return FASA_ERR_INVALID_ARG;
+  }
+  *dev = d;
+  return FASA_OK;
+}
+
 fasa_status fasa_append_kv(const fasa_cache* c, const void* k_new, const void* v_new, int32_t n_new,
                            int32_t pos0, cudaStream_t stream) {
   fasa_status s = check_cache(c);
@@ -1018,6 +1040,9 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
     return launch_attend(c, len, len, out, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part),
                          reinterpret_cast<uint32_t*>(base + w.att_cnt), w.splits_max, d, stream);
   }
+  // the f32 dense kernel stages K and V with bulk copies, which are kept to
+  // device memory: a FASA-M cache (host-resident K/V) is refused here
+  if (host_resident(c->k) || host_resident(c->v)) return FASA_ERR_UNSUPPORTED;
   SAParams p{};
   p.k = c->k;
   p.v = c->v;

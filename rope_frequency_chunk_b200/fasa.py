@@ -68,6 +68,7 @@ _SIGS = {
     "fasa_dense_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]),
     "fasa_device_status": (_I, [_I]),
+    "fasa_host_kv_pointer": (_I, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "fasa_set_decode_path": (_I, [_I]),
     "fasa_decode_path": (_I, [_CP, _I, _I]),
     "fasa_calibrate_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I, _I]),
@@ -135,10 +136,13 @@ def fasa_check_dom_idx(dom_idx_host) -> None:
 
 
 class KVCache:
-    """A layer's KV cache and dominant-FC key sketch, in caller-owned device memory."""
+    """A layer's KV cache and dominant-FC key sketch, in caller-owned memory:
+    all on the device (FASA-C), or, with kv_on_host, K and V in pinned host
+    memory that the device reads across the host link and only the sketch on
+    the device (FASA-M)."""
 
     def __init__(self, batch, n_q_heads, n_kv_heads, n_dom, max_len, dtype, rope_base, dom_idx,
-                 device="cuda"):
+                 device="cuda", kv_on_host=False):
         code = _DTYPE_CODE[dtype]
         tdt = _TORCH_DTYPE[code]
         stride = fasa_sketch_stride(n_dom, code)
@@ -147,21 +151,44 @@ class KVCache:
         fasa_check_dom_idx(dom_idx)
         self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
         self.n_dom, self.max_len, self.dtype, self.rope_base = n_dom, max_len, tdt, float(rope_base)
-        self.k = torch.empty(batch, n_kv_heads, max_len, HEAD_DIM, dtype=tdt, device=device)
-        self.v = torch.empty_like(self.k)
+        shape = (batch, n_kv_heads, max_len, HEAD_DIM)
+        self.kv_on_host = bool(kv_on_host)
+        if self.kv_on_host:
+            self.k = torch.empty(shape, dtype=tdt, pin_memory=True)
+            self.v = torch.empty(shape, dtype=tdt, pin_memory=True)
+            kp, vp = fasa_host_kv_pointer(self.k), fasa_host_kv_pointer(self.v)
+        else:
+            self.k = torch.empty(shape, dtype=tdt, device=device)
+            self.v = torch.empty_like(self.k)
+            kp, vp = self.k.data_ptr(), self.v.data_ptr()
         self.sketch = torch.empty(batch, n_kv_heads, max_len, stride, dtype=tdt, device=device)
         self.dom_idx = torch.as_tensor(dom_idx, dtype=torch.int32).to(device).contiguous()
         self.struct = fasa_cache(batch, n_q_heads, n_kv_heads, HEAD_DIM, n_dom, max_len, code, stride,
-                                 float(rope_base), self.k.data_ptr(), self.v.data_ptr(),
-                                 self.sketch.data_ptr(), self.dom_idx.data_ptr())
+                                 float(rope_base), kp, vp, self.sketch.data_ptr(), self.dom_idx.data_ptr())
         self.sketch_stride = stride
 
     @property
     def group(self):
         return self.n_q_heads // self.n_kv_heads
 
+    def device_bytes(self) -> int:
+        """Bytes of this cache held in device memory."""
+        n = self.sketch.numel() * self.sketch.element_size() + self.dom_idx.numel() * 4
+        if not self.kv_on_host:
+            n += (self.k.numel() + self.v.numel()) * self.k.element_size()
+        return n
+
     def ref(self):
         return ctypes.byref(self.struct)
+
+
+def fasa_host_kv_pointer(t: torch.Tensor) -> int:
+    """Device address of a pinned host tensor's data (FASA-M K and V)."""
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+        raise TypeError("expected a pinned host tensor")
+    out = ctypes.c_void_p()
+    _check(lib().fasa_host_kv_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(out)), "fasa_host_kv_pointer")
+    return int(out.value)
 
 
 # ------------------------------------------------------------------ calls

@@ -19,12 +19,13 @@ TIP_REL = 13.01 * 2.0 ** -24
 ABS_SLACK = 1e-12
 
 
-def build(wl, layer=0, n_dom=None, max_len=None, chunks=None, inp=None):
-    """Generate a layer's inputs and append them to a fresh cache on the GPU."""
+def build(wl, layer=0, n_dom=None, max_len=None, chunks=None, inp=None, kv_on_host=False):
+    """Generate a layer's inputs and append them to a fresh cache on the GPU
+    (K and V in pinned host memory with kv_on_host)."""
     inp = inp or W.layer_inputs(wl, layer=layer, n_dom=n_dom)
     lp = inp.params
     cache = F.KVCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, lp.dom_idx.shape[1],
-                      max_len or wl.ctx_len, wl.dtype, wl.rope_base, lp.dom_idx)
+                      max_len or wl.ctx_len, wl.dtype, wl.rope_base, lp.dom_idx, kv_on_host=kv_on_host)
     k = W.to_torch(inp.k, "cuda")
     v = W.to_torch(inp.v, "cuda")
     if chunks is None:
