@@ -354,6 +354,61 @@ size_t fasa_decode_varlen_workspace_bytes(const fasa_cache* cache, const fasa_va
 fasa_status fasa_decode_varlen(const fasa_cache* cache, const fasa_varlen* vl, const void* q, void* out,
                                int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Paged caches (serving realism, [tech §3] "Contribuições Principais",
+ * Versatilidade: sequences of their own lengths sharing one pool). The
+ * cache's k, v and sketch then point to page pools,
+ *   k, v   : [n_pages][Hkv][block_size][128] dtype,
+ *   sketch : [n_pages][Hkv][block_size][sketch_stride] dtype,
+ * and slot t of sequence b, KV head g is row t % block_size of page
+ * block_table[b][t / block_size], head g. fasa_cache.batch is the number of
+ * sequences and fasa_cache.max_len must equal max_blocks * block_size (the
+ * capacity of one sequence). Pages are owned and assigned by the caller.
+ *
+ *  block_table: device [B][max_blocks] int32. Every entry a call reaches
+ *               (blocks 0 .. (slot)/block_size of the slots it reads or
+ *               writes) must lie in 0 .. n_pages-1; an entry outside is
+ *               flagged FASA_ERR_BAD_INDEX in the status word and its rows
+ *               are skipped (not read, not written). The table is read on
+ *               the device after the call's launch dependencies, so a kernel
+ *               earlier in the stream may fill it.
+ *  block_size : tokens per page, a power of two in 16 .. 65536.
+ *  max_blocks : table row length (>= 1).
+ *  n_pages    : pages in each pool; n_pages * Hkv * block_size < 2^31.
+ */
+typedef struct fasa_paged {
+  const int32_t* block_table;
+  int32_t block_size;
+  int32_t max_blocks;
+  int32_t n_pages;
+  int32_t reserved;
+} fasa_paged;
+
+/*
+ * fasa_append_kv into a paged (or, with pages NULL, contiguous) cache, each
+ * sequence at its own position: the n_new tokens of sequence b go to slots
+ * pos0[b] .. pos0[b]+n_new-1, rotated at those positions.
+ *  pos0  : device [B] int32. A sequence whose range leaves 0 .. max_len-1 is
+ *          skipped and flagged FASA_ERR_BAD_INDEX in the status word.
+ *  k_new, v_new: [B][Hkv][n_new][128] dtype, device.
+ *  Errors: as fasa_append_kv (host checks), invalid pages -> INVALID_ARG.
+ */
+fasa_status fasa_append_kv_paged(const fasa_cache* cache, const fasa_paged* pages, const void* k_new,
+                                 const void* v_new, int32_t n_new, const int32_t* pos0, cudaStream_t stream);
+
+/* Workspace bytes fasa_decode_paged needs (0 for invalid arguments). */
+size_t fasa_decode_paged_workspace_bytes(const fasa_cache* cache, const fasa_paged* pages, const fasa_varlen* vl);
+
+/*
+ * fasa_decode_varlen over a paged cache: the same results as
+ * fasa_decode_varlen on a contiguous cache holding the same slots (bf16
+ * caches; kept indices are logical slots). Errors: as fasa_decode_varlen;
+ * invalid pages -> FASA_ERR_INVALID_ARG.
+ */
+fasa_status fasa_decode_paged(const fasa_cache* cache, const fasa_paged* pages, const fasa_varlen* vl,
+                              const void* q, void* out, int32_t* idx_out, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
 /* Size of the library's own device scratch used by
  * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the
  * library until the process exits. */

@@ -9,7 +9,9 @@
 //
 // Grid: x = blocks of kAppendTok tokens, y = groups of `heads_per_cta`
 // consecutive (b, g) rows. cos/sin of a token block are computed once in
-// float64 and reused across the CTA's heads.
+// float64 and reused across the CTA's heads (recomputed per sequence when
+// every sequence appends at its own position). Slots are addressed through
+// a PageMap, so the same kernel fills contiguous and paged caches.
 #pragma once
 
 #include "fasa_device.cuh"
@@ -34,6 +36,8 @@ struct AppendParams {
   int32_t n_dom;
   int32_t stride;
   int32_t heads_per_cta;
+  const int32_t* pos0v;  // [B] each sequence's first new position, or null: pos0 for all
+  PageMap pm;            // paged pools, or pm.table null: [B*Hkv][max_len] planes
   double theta[kNFC];    // base^(-2i/128), computed on the host in float64
 };
 
@@ -43,6 +47,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
   __shared__ double s_sin[kAppendTok][kNFC];
   __shared__ T s_row[kAppendTok][kD];
   __shared__ int s_dom[kNFC];
+  __shared__ int64_t s_dst[kAppendTok];  // each token's row in the K / V / sketch planes, or -1
 
   const int tid = threadIdx.x;
   const int tok0 = blockIdx.x * kAppendTok;
@@ -50,18 +55,39 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
   const int row0 = blockIdx.y * p.heads_per_cta;
   const int row1 = min(p.n_rows, row0 + p.heads_per_cta);
 
-  for (int e = tid; e < ntok * kNFC; e += kAppendThreads) {
-    const int t = e / kNFC, i = e % kNFC;
-    const double ang = (double)(p.pos0 + tok0 + t) * p.theta[i];
-    double s, c;
-    sincos(ang, &s, &c);
-    s_cos[t][i] = c;
-    s_sin[t][i] = s;
-  }
+  auto angles = [&](int pos) {
+    for (int e = tid; e < ntok * kNFC; e += kAppendThreads) {
+      const int t = e / kNFC, i = e % kNFC;
+      const double ang = (double)(pos + tok0 + t) * p.theta[i];
+      double s, c;
+      sincos(ang, &s, &c);
+      s_cos[t][i] = c;
+      s_sin[t][i] = s;
+    }
+  };
+  int cur = p.pos0;
+  if (!p.pos0v) angles(cur);
 
   for (int row = row0; row < row1; ++row) {
-    const int g = row % p.n_kv_heads;
-    __syncthreads();  // s_cos ready; previous row done with s_row / s_dom
+    const int b = row / p.n_kv_heads, g = row % p.n_kv_heads;
+    int pos = p.pos0;
+    if (p.pos0v) {
+      pos = __ldg(p.pos0v + b);
+      if (pos < 0 || (int64_t)pos + p.n_new > p.max_len) {  // block-uniform: skip the row
+        if (tid == 0 && blockIdx.x == 0) flag_status(FASA_ERR_BAD_INDEX);
+        continue;
+      }
+      if (row == row0 || pos != cur) {
+        __syncthreads();  // the previous row is done with the angles
+        angles(pos);
+        cur = pos;
+      }
+    }
+    __syncthreads();  // s_cos ready; previous row done with s_row / s_dom / s_dst
+    if (tid < ntok) {
+      const int t = pos + tok0 + tid;
+      s_dst[tid] = p.pm.table ? (int64_t)paged_row(p.pm, b, g, t) : (int64_t)row * p.max_len + t;
+    }
     if (tid < p.n_dom) {
       int d = p.dom_idx[g * p.n_dom + tid];
       if (d < 0 || d >= kNFC) {
@@ -72,9 +98,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
     }
     const T* kin = static_cast<const T*>(p.k_new) + ((int64_t)row * p.n_new + tok0) * kD;
     const T* vin = static_cast<const T*>(p.v_new) + ((int64_t)row * p.n_new + tok0) * kD;
-    T* kc = static_cast<T*>(p.k) + ((int64_t)row * p.max_len + p.pos0 + tok0) * kD;
-    T* vc = static_cast<T*>(p.v) + ((int64_t)row * p.max_len + p.pos0 + tok0) * kD;
-    T* sk = static_cast<T*>(p.sketch) + ((int64_t)row * p.max_len + p.pos0 + tok0) * p.stride;
+    T* kc = static_cast<T*>(p.k);
+    T* vc = static_cast<T*>(p.v);
+    T* sk = static_cast<T*>(p.sketch);
+    __syncthreads();  // s_dst ready
 
     // RoPE of FC i: (x, y) -> (x cos - y sin, y cos + x sin), float64, no
     // contraction, one rounding to the cache dtype.
@@ -88,15 +115,21 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
       T xs, ys;
       round_store(&xs, xr);
       round_store(&ys, yr);
-      kc[t * kD + i] = xs;
-      kc[t * kD + i + kNFC] = ys;
+      const int64_t dst = s_dst[t];
+      if (dst >= 0) {
+        kc[dst * kD + i] = xs;
+        kc[dst * kD + i + kNFC] = ys;
+      }
       s_row[t][i] = xs;
       s_row[t][i + kNFC] = ys;
     }
     // values are stored as given (16-byte vectors)
-    const int nvec = ntok * kD * (int)sizeof(T) / 16;
-    for (int e = tid; e < nvec; e += kAppendThreads)
-      reinterpret_cast<uint4*>(vc)[e] = reinterpret_cast<const uint4*>(vin)[e];
+    constexpr int kVecRow = kD * (int)sizeof(T) / 16;  // 16-byte vectors per row
+    for (int e = tid; e < ntok * kVecRow; e += kAppendThreads) {
+      const int64_t dst = s_dst[e / kVecRow];
+      if (dst >= 0)
+        reinterpret_cast<uint4*>(vc + dst * kD)[e % kVecRow] = reinterpret_cast<const uint4*>(vin)[e];
+    }
     __syncthreads();
     // sketch row: dims (dom[j], dom[j]+64) at 2j, 2j+1, zero padding
     for (int e = tid; e < ntok * p.stride; e += kAppendThreads) {
@@ -106,7 +139,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
         const int d = s_dom[j];
         if (d >= 0) val = s_row[t][d + (c & 1) * kNFC];
       }
-      sk[(int64_t)t * p.stride + c] = val;
+      const int64_t dst = s_dst[t];
+      if (dst >= 0) sk[dst * p.stride + c] = val;
     }
   }
 }

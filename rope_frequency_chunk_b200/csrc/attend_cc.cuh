@@ -292,6 +292,7 @@ struct CcParams {
   const int32_t* row_keep;  // [rows] each row's kept count
   int32_t n_kv_heads;
   int32_t q_prerot;         // varlen: 1 if the queries are already rotated
+  PageMap pm;               // paged pools (pm.table set), else [rows][max_len] planes
   double cosv[kNFC];        // cos / sin of q_pos * theta_i; varlen: theta_i in cosv
   double sinv[kNFC];
 };
@@ -350,8 +351,10 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   const int r_beg = split * p.slice, r_end = min(n_keep, r_beg + p.slice);
   const int per_warp = ((max(0, r_end - r_beg) + kCcWarps * kCcStep - 1) / (kCcWarps * kCcStep)) * kCcStep;
   const int j0 = min(r_end, r_beg + warp * per_warp), j1 = min(r_end, j0 + per_warp);
-  const __nv_bfloat16* kb = p.k + (int64_t)row * p.max_len * kD;
-  const __nv_bfloat16* vb = p.v + (int64_t)row * p.max_len * kD;
+  const bool paged = p.pm.table != nullptr;
+  const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
+  const __nv_bfloat16* kb = p.k + plane;
+  const __nv_bfloat16* vb = p.v + plane;
   const int32_t* idx = p.idx ? p.idx + (int64_t)row * p.n_keep : nullptr;
   cc_warp_rows<MG>(acc, kb, vb, [&](int j) -> int {
     const int t = idx ? __ldg(idx + j) : j;
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
       flag_status(FASA_ERR_BAD_INDEX);
       return -1;
     }
-    return t;
+    return paged ? paged_row(p.pm, row / p.n_kv_heads, row % p.n_kv_heads, t) : t;
   }, j0, j1, qs, ws, vball + warp * 2 * kCcStep * kD, lane);
   __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
   float* pp = p.part + ((int64_t)row * p.splits + split) * kCcPartStride;

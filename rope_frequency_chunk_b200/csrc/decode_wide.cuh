@@ -92,6 +92,7 @@ struct WideParams {
   const int32_t* budget;   // [Hkv]
   int32_t* row_keep;       // [rows] each row's k_eff, for the attention launch (varlen), or null
   int32_t q_prerot;        // varlen: 1 if the queries are already rotated
+  PageMap pm;              // paged pools (pm.table set), else [rows][max_len] planes
   double cosv[kNFC];       // cos / sin of the query angle (uniform length), or
   double sinv[kNFC];       // theta_i in cosv (varlen: the angle is seq_len[b] * theta_i)
 };
@@ -125,10 +126,10 @@ __host__ __device__ constexpr int wd_al(int x, int a) { return (x + a - 1) / a *
 // staged union ([n_split][P] entries); then the attention's logits, warp
 // sums and V rows.
 struct WdLayout {
-  int hist, misc, coef, qraw, dom, cs, qs, cnt, kept, r1, bitmap, ties, rscr, ucache, zs, ring, total;
+  int hist, misc, coef, qraw, dom, cs, qs, pgs, cnt, kept, r1, bitmap, ties, rscr, ucache, zs, ring, total;
 };
 __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, int direct, int group, int n_split,
-                                              int P) {
+                                              int P, int paged) {
   WdLayout L;
   const int MG = group <= 4 ? 4 : 8;
   int o = 0;
@@ -146,6 +147,8 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   o += 2 * kNFC * 8;
   L.qs = o;  // attention queries [MG][128] f32
   o += direct ? MG * kD * 4 : 0;
+  L.pgs = o;  // paged: the CTA's pages (block size >= 16)
+  o += paged ? wd_al((n_loc / 16 + 2) * 4, 16) : 0;
   L.cnt = o;  // region counts, their prefix sums, the regions' b_loc
   o += wd_al((3 * n_split + 2) * 4, 16);
   L.kept = o;
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   using S = TipShape<__nv_bfloat16, LPT>;
   constexpr int U = S::LPT2 == 1 ? 4 : 2;  // tokens in flight per lane
   extern __shared__ __align__(128) unsigned char smem[];
-  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.n_split, p.ucache);
+  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.n_split, p.ucache, p.pm.table != nullptr);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + Lo.hist);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lo.misc);
   float* coef = reinterpret_cast<float*>(smem + Lo.coef);
@@ -393,8 +396,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int n_pub = p.seq_len ? (p.n_split == 1 ? kr : min(kr, (2 * ((kr + p.n_split - 1) / p.n_split) + 63) / 32 * 32))
                               : p.n_pub;
   const int n_tok = max(0, min(Lr - t_beg, p.n_loc));
+  const bool paged = p.pm.table != nullptr;
+  const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
   const char* src = reinterpret_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t_beg) * S::ROWB;
-  {  // L2 prefetch of this CTA's sketch range: a hint, safe before the wait
+  if (!paged) {  // L2 prefetch of this CTA's sketch range: a hint, safe before the wait
     const int64_t bytes = (int64_t)n_tok * S::ROWB;
     constexpr int kPf = 8192;
     for (int64_t o = (int64_t)tid * kPf; o < bytes; o += (int64_t)kWdThreads * kPf)
@@ -402,12 +407,39 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   grid_dependency_wait();
   grid_dependents_launch();
+  // paged: the CTA's pages (read after the wait: an earlier launch may have
+  // written the table), each prefetched to L2 whole
+  int* s_pg = reinterpret_cast<int*>(smem + Lo.pgs);
+  const int pg0 = paged ? t_beg >> p.pm.log2bs : 0;
+  if (paged) {
+    const int n_pg = n_tok > 0 ? ((t_beg + n_tok - 1) >> p.pm.log2bs) - pg0 + 1 : 0;
+    for (int i = tid; i < n_pg; i += kWdThreads) {
+      int pg = __ldg(p.pm.table + (int64_t)bb * p.pm.max_blocks + pg0 + i);
+      if ((unsigned)pg >= (unsigned)p.pm.n_pages) {
+        flag_status(FASA_ERR_BAD_INDEX);
+        pg = -1;
+      } else {
+        prefetch_l2(reinterpret_cast<const char*>(p.sketch) +
+                        ((int64_t)(pg * p.pm.n_kv_heads + g) << p.pm.log2bs) * S::ROWB,
+                    (uint32_t)(S::ROWB << p.pm.log2bs));
+      }
+      s_pg[i] = pg;
+    }
+    __syncthreads();
+  }
+  // sketch row of the CTA's token t (< n_tok), or null for a page outside the pool
+  auto sk_row = [&](int t) -> const char* {
+    if (!paged) return src + (int64_t)t * S::ROWB;
+    const int tt = t_beg + t, pg = s_pg[(tt >> p.pm.log2bs) - pg0];
+    if (pg < 0) return nullptr;
+    return reinterpret_cast<const char*>(p.sketch) +
+           (int64_t)(((pg * p.pm.n_kv_heads + g) << p.pm.log2bs) | (tt & ((1 << p.pm.log2bs) - 1))) * S::ROWB;
+  };
 
   // 1. the group's queries, dominant FCs and rotation table; the CTA's first
   // sketch rows are requested before the coefficients are formed, so the
   // query's round trip and the float64 work overlap the stream
   const int G = p.group;
-  const int bb = row / p.n_kv_heads, g = row % p.n_kv_heads;
   double* cs_sm = reinterpret_cast<double*>(smem + Lo.cs);
   {
     const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
@@ -431,10 +463,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int t = base + u * kTokPass + my_tok;
+      const char* rp = t < n_tok ? sk_row(t) : nullptr;
 #pragma unroll
       for (int c = 0; c < S::CPL; ++c)
-        v[u][c] = t < n_tok ? __ldg(reinterpret_cast<const uint4*>(src + (int64_t)t * S::ROWB) + sub * S::CPL + c)
-                            : make_uint4(0u, 0u, 0u, 0u);
+        v[u][c] = rp ? __ldg(reinterpret_cast<const uint4*>(rp) + sub * S::CPL + c) : make_uint4(0u, 0u, 0u, 0u);
     }
   };
   load_rows(0);
@@ -672,9 +704,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   float* mo = reinterpret_cast<float*>(smem + Lo.ring);
   float* lsum = mo + kWdWarps * MG * kD;
   __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
-  cc_block_attend<MG, kWdWarps>(p.k + (int64_t)row * p.max_len * kD, p.v + (int64_t)row * p.max_len * kD,
-                                [&](int j) -> int { return kept[j]; }, n_att, G, qs, zs, mo, lsum, vst,
-                                p.out + (int64_t)row * G * kD);
+  const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
+  cc_block_attend<MG, kWdWarps>(p.k + plane, p.v + plane,
+                                [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
+                                n_att, G, qs, zs, mo, lsum, vst, p.out + (int64_t)row * G * kD);
 }
 
 }  // namespace fasa

@@ -379,11 +379,37 @@ fasa_status wide_attrs(const DevInfo& d) {
 // regions (n_split * (n_loc + 1) entries) stay within len + len/64 + 64.
 inline int64_t wide_region_slots(int64_t len) { return len + len / 64 + 64; }
 
+// Device view of a paged cache's block table (table null: contiguous).
+PageMap page_map(const fasa_cache* c, const fasa_paged* pg) {
+  PageMap m{};
+  m.n_kv_heads = c->n_kv_heads;
+  if (pg == nullptr) return m;
+  m.table = pg->block_table;
+  m.max_blocks = pg->max_blocks;
+  m.n_pages = pg->n_pages;
+  int l = 0;
+  while ((1 << l) < pg->block_size) ++l;
+  m.log2bs = l;
+  return m;
+}
+
+// Host checks of a paged description against the cache.
+fasa_status check_paged(const fasa_cache* c, const fasa_paged* pg) {
+  if (pg == nullptr || !aligned(pg->block_table, 4)) return FASA_ERR_INVALID_ARG;
+  const int32_t bs = pg->block_size;
+  if (bs < 16 || bs > (1 << 16) || (bs & (bs - 1)) != 0) return FASA_ERR_INVALID_ARG;
+  if (pg->max_blocks < 1 || pg->n_pages < 1) return FASA_ERR_INVALID_ARG;
+  if ((int64_t)pg->max_blocks * bs != c->max_len) return FASA_ERR_INVALID_ARG;
+  // pool rows are addressed with 32-bit indices
+  if ((int64_t)pg->n_pages * c->n_kv_heads * bs > INT32_MAX) return FASA_ERR_UNSUPPORTED;
+  return FASA_OK;
+}
+
 // CTAs per row: about one per SM over all rows (never fewer than the
 // shared-memory limit on keys per CTA allows); tokens per CTA. The
 // resolving CTA attends itself for budgets up to kWdMaxDirect when its ring
 // fits, and caches as much of the published union as shared memory allows.
-bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl) {
+bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl, int paged = 0) {
   if (c->dtype != FASA_BF16) return false;
   const int64_t rows = (int64_t)c->batch * c->n_kv_heads;
   // about one CTA per SM, leaving one SM per row free: the rows' resolving
@@ -402,7 +428,7 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
                                 : (int)std::min<int64_t>(keff, (2 * ceil_div(keff, pl->n_split) + 32 + 31) / 32 * 32);
   const int G = c->n_q_heads / c->n_kv_heads;
   for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
-    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0);
+    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0, paged);
     if (base.total > d.smem_optin) continue;
     // entries of each CTA's region the resolving CTA stages in shared memory:
     // a power of two covering what a CTA usually publishes (its k_eff best
@@ -415,7 +441,7 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
     pl->ucache = (int)P;
     pl->ushift = 0;
     while ((1 << pl->ushift) < P) ++pl->ushift;
-    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache).total;
+    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache, paged).total;
     if (pl->smem > d.smem_optin) continue;
     return true;
   }
@@ -581,7 +607,7 @@ fasa_status launch_attend_t(CcParams& ap, int rows, int splits_max, const DevInf
 fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
                           const void* q, int32_t q_pos, float* part, uint32_t* counter, int splits_max,
                           const DevInfo& d, cudaStream_t st, const fasa_varlen* vl = nullptr,
-                          const int32_t* row_keep = nullptr) {
+                          const int32_t* row_keep = nullptr, const fasa_paged* pg = nullptr) {
   const int rows = c->batch * c->n_kv_heads;
   CcParams ap{};
   ap.k = static_cast<const __nv_bfloat16*>(c->k);
@@ -596,6 +622,7 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
   ap.n_keep = n_keep;
   ap.group = c->n_q_heads / c->n_kv_heads;
   ap.n_kv_heads = c->n_kv_heads;
+  ap.pm = page_map(c, pg);
   if (vl) {  // per-row lengths and kept counts; the angles from the lengths on the device
     ap.seq_len = vl->seq_len;
     ap.row_keep = row_keep;
@@ -612,10 +639,10 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
 // The decode's attention over the kept lists in the workspace.
 fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, const void* q, int32_t q_pos, void* out,
                              const DecodeWs& w, char* base, const DevInfo& d, cudaStream_t st,
-                             const fasa_varlen* vl = nullptr) {
+                             const fasa_varlen* vl = nullptr, const fasa_paged* pg = nullptr) {
   return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx), q, q_pos,
                        reinterpret_cast<float*>(base + w.part), reinterpret_cast<uint32_t*>(base + w.att_cnt),
-                       w.splits_max, d, st, vl, reinterpret_cast<const int32_t*>(base + w.rowk));
+                       w.splits_max, d, st, vl, reinterpret_cast<const int32_t*>(base + w.rowk), pg);
 }
 
 // Dense decode workspace: att_cnt [rows] u32 (zero between calls) | part
@@ -634,12 +661,44 @@ DenseWs dense_layout(const fasa_cache* c, int32_t len) {
   return w;
 }
 
+// The append kernel's launch: every sequence at pos0, or at pos0v[b].
+fasa_status launch_append(const fasa_cache* c, const void* k_new, const void* v_new, int32_t n_new, int32_t pos0,
+                          const int32_t* pos0v, const fasa_paged* pg, const DevInfo& d, cudaStream_t stream) {
+  AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k = c->k;
+  p.v = c->v;
+  p.sketch = c->sketch;
+  p.dom_idx = c->dom_idx;
+  p.max_len = c->max_len;
+  p.n_rows = c->batch * c->n_kv_heads;
+  p.n_kv_heads = c->n_kv_heads;
+  p.n_new = n_new;
+  p.pos0 = pos0;
+  p.pos0v = pos0v;
+  p.pm = page_map(c, pg);
+  p.n_dom = c->n_dom;
+  p.stride = c->sketch_stride;
+  fill_theta(p.theta, c->rope_base);
+  const int64_t tok_blocks = ceil_div(n_new, kAppendTok);
+  const int64_t groups = std::max<int64_t>(1, std::min<int64_t>(p.n_rows, ceil_div(4LL * d.sms, tok_blocks)));
+  p.heads_per_cta = (int)ceil_div(p.n_rows, groups);
+  const dim3 grid((unsigned)tok_blocks, (unsigned)ceil_div(p.n_rows, p.heads_per_cta), 1);
+  if (c->dtype == FASA_F32)
+    append_kernel<float><<<grid, kAppendThreads, 0, stream>>>(p);
+  else
+    append_kernel<__nv_bfloat16><<<grid, kAppendThreads, 0, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
 // The wide fused decode: one launch, plus the split-K attention when the
 // budget is beyond what the resolving CTA attends itself.
 fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int keff, void* out,
                         int32_t* idx_out, const DecodeWs& w, char* base, const WidePlan& pl, const DevInfo& d,
-                        cudaStream_t st, const fasa_varlen* vl = nullptr) {
+                        cudaStream_t st, const fasa_varlen* vl = nullptr, const fasa_paged* pg = nullptr) {
   WideParams p{};
+  p.pm = page_map(c, pg);
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
   p.v = static_cast<const __nv_bfloat16*>(c->v);
@@ -685,7 +744,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
     default: return FASA_ERR_UNSUPPORTED;
   }
   if (s != FASA_OK || pl.direct) return s;
-  return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st, vl);
+  return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st, vl, pg);
 }
 
 }  // namespace
@@ -755,30 +814,7 @@ fasa_status fasa_append_kv(const fasa_cache* c, const void* k_new, const void* v
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return FASA_ERR_INVALID_ARG;
   DevInfo d;
   if ((s = device_info(&d)) != FASA_OK) return s;
-  AppendParams p{};
-  p.k_new = k_new;
-  p.v_new = v_new;
-  p.k = c->k;
-  p.v = c->v;
-  p.sketch = c->sketch;
-  p.dom_idx = c->dom_idx;
-  p.max_len = c->max_len;
-  p.n_rows = c->batch * c->n_kv_heads;
-  p.n_kv_heads = c->n_kv_heads;
-  p.n_new = n_new;
-  p.pos0 = pos0;
-  p.n_dom = c->n_dom;
-  p.stride = c->sketch_stride;
-  fill_theta(p.theta, c->rope_base);
-  const int64_t tok_blocks = ceil_div(n_new, kAppendTok);
-  const int64_t groups = std::max<int64_t>(1, std::min<int64_t>(p.n_rows, ceil_div(4LL * d.sms, tok_blocks)));
-  p.heads_per_cta = (int)ceil_div(p.n_rows, groups);
-  const dim3 grid((unsigned)tok_blocks, (unsigned)ceil_div(p.n_rows, p.heads_per_cta), 1);
-  if (c->dtype == FASA_F32)
-    append_kernel<float><<<grid, kAppendThreads, 0, stream>>>(p);
-  else
-    append_kernel<__nv_bfloat16><<<grid, kAppendThreads, 0, stream>>>(p);
-  return cuda_status(cudaGetLastError());
+  return launch_append(c, k_new, v_new, n_new, pos0, nullptr, nullptr, d, stream);
 }
 
 fasa_status fasa_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
@@ -964,6 +1000,9 @@ int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
   return pl.direct ? 1 : 2;
 }
 
+}  // extern "C"
+
+namespace {
 // Host checks of a varlen description against the cache.
 fasa_status check_varlen(const fasa_cache* c, const fasa_varlen* vl) {
   if (vl == nullptr || !aligned(vl->seq_len, 4)) return FASA_ERR_INVALID_ARG;
@@ -975,15 +1014,10 @@ fasa_status check_varlen(const fasa_cache* c, const fasa_varlen* vl) {
   return FASA_OK;
 }
 
-size_t fasa_decode_varlen_workspace_bytes(const fasa_cache* c, const fasa_varlen* vl) {
-  if (check_cache(c) != FASA_OK || check_varlen(c, vl) != FASA_OK) return 0;
-  return decode_ws(c, vl->max_seq_len, vl->max_budget);
-}
-
-fasa_status fasa_decode_varlen(const fasa_cache* c, const fasa_varlen* vl, const void* q, void* out,
-                               int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  fasa_status s = check_cache(c);
-  if (s != FASA_OK) return s;
+// fasa_decode_varlen / fasa_decode_paged after the cache checks.
+fasa_status decode_varlen(const fasa_cache* c, const fasa_varlen* vl, const void* q, void* out, int32_t* idx_out,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream, const fasa_paged* pg) {
+  fasa_status s;
   if ((s = check_varlen(c, vl)) != FASA_OK) return s;
   if (c->dtype != FASA_BF16) return FASA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
@@ -994,8 +1028,52 @@ fasa_status fasa_decode_varlen(const fasa_cache* c, const fasa_varlen* vl, const
   DevInfo d;
   if ((s = device_info(&d)) != FASA_OK) return s;
   WidePlan pl;
-  if (!wide_plan(c, len, keff, d, &pl)) return FASA_ERR_UNSUPPORTED;
-  return launch_wide(c, len, q, 0, keff, out, idx_out, w, static_cast<char*>(workspace), pl, d, stream, vl);
+  if (!wide_plan(c, len, keff, d, &pl, pg != nullptr)) return FASA_ERR_UNSUPPORTED;
+  return launch_wide(c, len, q, 0, keff, out, idx_out, w, static_cast<char*>(workspace), pl, d, stream, vl, pg);
+}
+}  // namespace
+
+extern "C" {
+
+size_t fasa_decode_varlen_workspace_bytes(const fasa_cache* c, const fasa_varlen* vl) {
+  if (check_cache(c) != FASA_OK || check_varlen(c, vl) != FASA_OK) return 0;
+  return decode_ws(c, vl->max_seq_len, vl->max_budget);
+}
+
+fasa_status fasa_decode_varlen(const fasa_cache* c, const fasa_varlen* vl, const void* q, void* out,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  return decode_varlen(c, vl, q, out, idx_out, workspace, workspace_bytes, stream, nullptr);
+}
+
+
+fasa_status fasa_append_kv_paged(const fasa_cache* c, const fasa_paged* pg, const void* k_new, const void* v_new,
+                                 int32_t n_new, const int32_t* pos0, cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (pg != nullptr && (s = check_paged(c, pg)) != FASA_OK) return s;
+  if (n_new < 0 || !aligned(pos0, 4)) return FASA_ERR_INVALID_ARG;
+  if (n_new > c->max_len) return FASA_ERR_CAPACITY;
+  if (n_new == 0) return FASA_OK;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return FASA_ERR_INVALID_ARG;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return s;
+  return launch_append(c, k_new, v_new, n_new, 0, pos0, pg, d, stream);
+}
+
+size_t fasa_decode_paged_workspace_bytes(const fasa_cache* c, const fasa_paged* pg, const fasa_varlen* vl) {
+  if (check_cache(c) != FASA_OK || check_paged(c, pg) != FASA_OK || check_varlen(c, vl) != FASA_OK) return 0;
+  return decode_ws(c, vl->max_seq_len, vl->max_budget);
+}
+
+fasa_status fasa_decode_paged(const fasa_cache* c, const fasa_paged* pg, const fasa_varlen* vl, const void* q,
+                              void* out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if ((s = check_paged(c, pg)) != FASA_OK) return s;
+  return decode_varlen(c, vl, q, out, idx_out, workspace, workspace_bytes, stream, pg);
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,

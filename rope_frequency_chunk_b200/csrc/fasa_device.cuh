@@ -20,6 +20,32 @@ __device__ unsigned int g_status;
 
 __device__ __forceinline__ void flag_status(unsigned int code) { atomicCAS(&g_status, 0u, code); }
 
+// Where slot t of row (b, g) lives. Contiguous caches: row t of the (b, g)
+// plane [max_len][W]. Paged caches: the pools are [n_pages][Hkv][bs][W]
+// and logical block t / bs of sequence b is page table[b][t / bs]; the row
+// index below counts W-element rows from the pool's start.
+struct PageMap {
+  const int32_t* table;  // [B][max_blocks], or null for a contiguous cache
+  int32_t max_blocks;
+  int32_t n_pages;
+  int32_t log2bs;        // log2 of the block size
+  int32_t n_kv_heads;
+};
+
+// Pool row of slot t of (b, g) given the page, or -1 for a page outside the
+// pool (flagged FASA_ERR_BAD_INDEX).
+__device__ __forceinline__ int page_row(const PageMap& m, int pg, int g, int t) {
+  if ((unsigned)pg >= (unsigned)m.n_pages) {
+    flag_status(FASA_ERR_BAD_INDEX);
+    return -1;
+  }
+  return ((pg * m.n_kv_heads + g) << m.log2bs) | (t & ((1 << m.log2bs) - 1));
+}
+// The same, looking the page up in the table.
+__device__ __forceinline__ int paged_row(const PageMap& m, int b, int g, int t) {
+  return page_row(m, __ldg(m.table + (int64_t)b * m.max_blocks + (t >> m.log2bs)), g, t);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

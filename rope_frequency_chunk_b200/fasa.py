@@ -44,6 +44,11 @@ class fasa_varlen(ctypes.Structure):
                 ("max_budget", ctypes.c_int32), ("q_prerotated", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class fasa_paged(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("block_size", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("n_pages", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -64,6 +69,11 @@ _SIGS = {
     "fasa_decode": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_varlen_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.POINTER(fasa_varlen)]),
     "fasa_decode_varlen": (_I, [_CP, ctypes.POINTER(fasa_varlen), _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fasa_append_kv_paged": (_I, [_CP, ctypes.POINTER(fasa_paged), _P, _P, _I, _P, _P]),
+    "fasa_decode_paged_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.POINTER(fasa_paged),
+                                                            ctypes.POINTER(fasa_varlen)]),
+    "fasa_decode_paged": (_I, [_CP, ctypes.POINTER(fasa_paged), ctypes.POINTER(fasa_varlen), _P, _P, _P, _P,
+                               ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]),
@@ -189,6 +199,84 @@ def fasa_host_kv_pointer(t: torch.Tensor) -> int:
     out = ctypes.c_void_p()
     _check(lib().fasa_host_kv_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(out)), "fasa_host_kv_pointer")
     return int(out.value)
+
+
+class PagedKVCache:
+    """A layer's paged KV cache: K, V and sketch page pools [n_pages][Hkv]
+    [block_size][...] on the device and a block table [B][max_blocks] (int32,
+    device) mapping each sequence's logical blocks to pages. The caller
+    assigns pages by writing block_table."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, n_dom, n_pages, block_size, max_blocks, dtype, rope_base,
+                 dom_idx, device="cuda"):
+        code = _DTYPE_CODE[dtype]
+        tdt = _TORCH_DTYPE[code]
+        stride = fasa_sketch_stride(n_dom, code)
+        if stride < 0:
+            raise FasaError(1, "fasa_sketch_stride")
+        fasa_check_dom_idx(dom_idx)
+        self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
+        self.n_dom, self.dtype, self.rope_base = n_dom, tdt, float(rope_base)
+        self.n_pages, self.block_size, self.max_blocks = n_pages, block_size, max_blocks
+        self.max_len = max_blocks * block_size
+        self.k = torch.zeros(n_pages, n_kv_heads, block_size, HEAD_DIM, dtype=tdt, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.sketch = torch.zeros(n_pages, n_kv_heads, block_size, stride, dtype=tdt, device=device)
+        self.block_table = torch.zeros(batch, max_blocks, dtype=torch.int32, device=device)
+        self.dom_idx = torch.as_tensor(dom_idx, dtype=torch.int32).to(device).contiguous()
+        self.struct = fasa_cache(batch, n_q_heads, n_kv_heads, HEAD_DIM, n_dom, self.max_len, code, stride,
+                                 float(rope_base), self.k.data_ptr(), self.v.data_ptr(), self.sketch.data_ptr(),
+                                 self.dom_idx.data_ptr())
+        self.pages = fasa_paged(self.block_table.data_ptr(), block_size, max_blocks, n_pages, 0)
+        self.sketch_stride = stride
+
+    @property
+    def group(self):
+        return self.n_q_heads // self.n_kv_heads
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    def pref(self):
+        return ctypes.byref(self.pages)
+
+    def logical(self, pool, b: int, g: int, length: int):
+        """Rows 0 .. length-1 of (b, g) gathered from a pool (k, v or sketch)."""
+        t = torch.arange(length, device=pool.device)
+        pg = self.block_table[b, (t // self.block_size)].long()
+        return pool[pg, g, t % self.block_size]
+
+
+def fasa_append_kv_paged(cache: PagedKVCache, k_new, v_new, pos0, stream=None) -> None:
+    """Append n_new tokens to every sequence b at slots pos0[b] .. (pos0: int32 [B] on the device)."""
+    _dev(k_new, "k_new", cache.dtype)
+    _dev(v_new, "v_new", cache.dtype)
+    _dev(pos0, "pos0", torch.int32)
+    n_new = k_new.shape[2]
+    if tuple(k_new.shape) != (cache.batch, cache.n_kv_heads, n_new, HEAD_DIM) or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new must be [B, Hkv, n_new, 128]")
+    _check(lib().fasa_append_kv_paged(cache.ref(), cache.pref(), k_new.data_ptr(), v_new.data_ptr(), n_new,
+                                      pos0.data_ptr(), _stream(stream)), "fasa_append_kv_paged")
+
+
+def fasa_decode_paged(cache: PagedKVCache, seq_len, q, max_seq_len: int, max_budget: int, budget=None,
+                      q_prerotated: bool = False, out=None, idx_out=None, workspace=None, stream=None):
+    """fasa_decode_varlen over a paged cache."""
+    _q(cache, q)
+    vl = _varlen(seq_len, budget, max_seq_len, max_budget, q_prerotated)
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    if idx_out is not None:
+        _dev(idx_out, "idx_out", torch.int32)
+    if workspace is None:
+        need = int(lib().fasa_decode_paged_workspace_bytes(cache.ref(), cache.pref(), ctypes.byref(vl)))
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_decode_paged(cache.ref(), cache.pref(), ctypes.byref(vl), q.data_ptr(), out.data_ptr(),
+                                   _ptr(idx_out), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "fasa_decode_paged")
+    return out
 
 
 # ------------------------------------------------------------------ calls

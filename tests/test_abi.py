@@ -173,3 +173,40 @@ def test_varlen_validation_without_launch(L):
     assert run(c, vl(), 0x50000, 0x70000, None, None, need, None) == 4
     assert run(c, vl(), 0x50000, 0x70000, None, 0x80000, need - 1, None) == 4
     assert run(c, vl(), 0x50000, 0x70000, None, 0x80010, need, None) == 4  # workspace alignment
+
+
+def test_paged_validation_without_launch(L):
+    # a paged cache: max_len = max_blocks * block_size
+    c = ctypes.byref(_fake_cache(max_len=64 * 16))
+
+    def pg(**kw):
+        d = dict(block_table=0xA0000, block_size=16, max_blocks=64, n_pages=100, reserved=0)
+        d.update(kw)
+        return ctypes.byref(F.fasa_paged(**d))
+
+    vl = ctypes.byref(F.fasa_varlen(seq_len=0x90000, budget=None, max_seq_len=1000, max_budget=8,
+                                    q_prerotated=0, reserved=0))
+    ws = L.fasa_decode_paged_workspace_bytes
+    need = ws(c, pg(), vl)
+    assert need > 0 and need == L.fasa_decode_varlen_workspace_bytes(c, vl)
+    for bad in (dict(block_table=None), dict(block_table=0xA0002), dict(block_size=8), dict(block_size=48),
+                dict(block_size=1 << 17), dict(max_blocks=0), dict(n_pages=0), dict(max_blocks=63)):
+        assert ws(c, pg(**bad), vl) == 0, bad
+        assert L.fasa_decode_paged(c, pg(**bad), vl, 0x50000, 0x70000, None, 0x80000, need, None) == 1, bad
+    assert ws(c, None, vl) == 0
+    big = ctypes.byref(_fake_cache(max_len=64 * 65536))
+    assert L.fasa_decode_paged(big, pg(block_size=65536, n_pages=20000), vl, 0x50000, 0x70000, None, 0x80000,
+                               1 << 40, None) == 2                      # pool rows beyond 32-bit indices
+    run = L.fasa_decode_paged
+    assert run(c, pg(), None, 0x50000, 0x70000, None, 0x80000, need, None) == 1
+    assert run(c, pg(), vl, 0x50000, 0x70000, None, 0x80000, need - 1, None) == 4
+    assert run(ctypes.byref(_fake_cache(max_len=64 * 16, dtype=0)), pg(), vl, 0x50000, 0x70000, None, 0x80000,
+               need, None) == 2
+    app = L.fasa_append_kv_paged
+    assert app(c, pg(), 0x50000, 0x60000, 4, None, None) == 1                  # no positions
+    assert app(c, pg(), 0x50000, 0x60000, 4, 0x90002, None) == 1               # misaligned positions
+    assert app(c, pg(), 0x50000, 0x60000, -1, 0x90000, None) == 1
+    assert app(c, pg(), 0x50000, 0x60000, 2000, 0x90000, None) == 3           # more than a sequence holds
+    assert app(c, pg(), 0x50000, 0x60000, 0, 0x90000, None) == 0              # no-op
+    assert app(c, pg(), 0x50008, 0x60000, 4, 0x90000, None) == 1              # misaligned input
+    assert app(c, pg(block_size=24), 0x50000, 0x60000, 4, 0x90000, None) == 1
