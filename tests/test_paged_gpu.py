@@ -47,7 +47,9 @@ def paged_cache(wl, inp, bs, seq_len, spare=7, seed=0, chunks=None):
     # every sequence receives chunks of the same size at its own position,
     # until its length is reached (sequences that are full take a position
     # whose range leaves the cache: the kernel skips them and flags it)
-    chunks = chunks or [max(seq_len)]
+    if chunks is None:  # the gaps between the distinct lengths: every sequence ends exactly full
+        ends = sorted(set(seq_len))
+        chunks = [e - s for s, e in zip([0] + ends[:-1], ends)]
     pos = np.zeros(B, np.int64)
     for n in chunks:
         p0 = torch.tensor([int(x) if x + n <= seq_len[b] else -1 for b, x in enumerate(pos)], dtype=torch.int32,
