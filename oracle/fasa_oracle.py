@@ -21,7 +21,11 @@ Attention" computes at decode time (gist.science technical summary, §2
    attention over exactly those rows, each kept at its original absolute
    position (its key was rotated at that position when it was cached).
 4. Dense full-KV attention (the comparison): the same attention over all rows.
-5. Offline calibration (§2, TIP first bullet): the agreement of each single
+5. Multi-query decode (several query tokens per sequence in one step): the
+   group sum of step 2 taken over every query row, one shared critical set,
+   each row attending over the kept slots not after its position (the
+   reading is stated at decode_multi_head).
+6. Offline calibration (§2, TIP first bullet): the agreement of each single
    FC's token selection with the full head's over calibration queries picks
    the dominant FCs (the reading of "Contextual Agreement" is stated at the
    calibration functions).
@@ -222,6 +226,35 @@ def decode_head(q_pre: np.ndarray, q_pos: int, k_rot: np.ndarray, v: np.ndarray,
     out = focused_attention(q_rot, k_rot, v, idx)
     return idx, out, s
 
+
+
+def decode_multi_head(q_pre: np.ndarray, q_pos0: int, k_rot: np.ndarray, v: np.ndarray,
+                      sketch: np.ndarray, dom, k: int, base: float):
+    """One (sequence, KV head) of a multi-query decode step: n_q query tokens
+    (speculative drafts or batched rows), token j at position q_pos0 + j,
+    each with the group's G query heads.
+
+    Reading (the pages treat one query at a time): TIP's group sum extends
+    over every query row of the KV head, so the n_q * G rows share one
+    critical set, T = top-k of s_t = sum_j sum_h sum_{i in D_g} P_i(q'_{j,h},
+    k'_t). Each row then attends over the kept slots that are not after its
+    own position (t <= q_pos0 + j; every slot when the cache ends before the
+    queries, the usual decode). A row left with no slot gets a zero output.
+
+    q_pre: [n_q, G, d] pre-RoPE queries. Returns (idx, out [n_q, G, d]
+    float64, scores [L]).
+    """
+    q_pre = to_f64(q_pre)
+    n_q = q_pre.shape[0]
+    q_rot = np.stack([rotate_queries(q_pre[j], q_pos0 + j, base) for j in range(n_q)])
+    s = tip_scores(q_rot.reshape(-1, q_rot.shape[-1]), sketch, dom)
+    idx = select_critical_set(s, k)
+    out = np.zeros(q_rot.shape)
+    for j in range(n_q):
+        seen = idx[idx <= q_pos0 + j]
+        if len(seen):
+            out[j] = focused_attention(q_rot[j], k_rot, v, seen)
+    return idx, out, s
 
 
 # ------------------------------------------------------- calibration

@@ -288,6 +288,80 @@ def check_e2e_all_fc_topk_exact(m):
     return list(idx) == list(top) and _close(out, want, rtol=1e-9, atol=1e-12)
 
 
+def _multi_case(L=40, n_q=4, G=2, seed=30, base=1e4):
+    r = np.random.default_rng(seed)
+    qpre = r.standard_normal((n_q, G, 128)).astype(np.float32)
+    kpre = r.standard_normal((L, 128)).astype(np.float32)
+    v = r.standard_normal((L, 128)).astype(np.float32)
+    return qpre, kpre, v
+
+
+def check_multi_one_query_is_decode(m):
+    qpre, kpre, v = _multi_case(n_q=1, seed=31)
+    dom = np.array([4, 17, 60])
+    k_rot, v_st, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    a = m.decode_multi_head(qpre, 40, k_rot, v_st, sk, dom, 9, 1e4)
+    b = m.decode_head(qpre[0], 40, k_rot, v_st, sk, dom, 9, 1e4)
+    return list(a[0]) == list(b[0]) and np.array_equal(a[1][0], b[1]) and np.array_equal(a[2], b[2])
+
+
+def check_multi_scores_add_over_positions(m):
+    # the shared score is the sum of the per-token group scores, each token
+    # rotated at its own position (dominant dims by brute force)
+    qpre, kpre, v = _multi_case(L=30, n_q=3, G=2, seed=32)
+    dom = [9, 2, 33]
+    k_rot, v_st, sk = m.append_kv(kpre, v, 0, 1e4, np.array(dom), "f32")
+    _, _, s = m.decode_multi_head(qpre, 30, k_rot, v_st, sk, np.array(dom), 5, 1e4)
+    kr = m.to_f64(k_rot)
+    want = np.zeros(30)
+    for j in range(3):
+        ang = (30 + j) * 1e4 ** (-2.0 * np.arange(64) / 128)
+        for h in range(2):
+            z = (qpre[j, h, :64] + 1j * qpre[j, h, 64:]).astype(np.complex128) * np.exp(1j * ang)
+            for i in dom:
+                want += z[i].real * kr[:, i] + z[i].imag * kr[:, i + 64]
+    return _close(s, want, rtol=1e-10, atol=1e-10)
+
+
+def check_multi_causal_vs_sdpa(m):
+    # drafts already in the cache: query j at position 36 + j sees slots
+    # 0 .. 36 + j; all FCs and k = L reduce it to masked dense attention
+    qpre, kpre, v = _multi_case(L=40, n_q=4, G=2, seed=33)
+    dom = np.arange(64)
+    k_rot, v_st, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+    idx, out, _ = m.decode_multi_head(qpre, 36, k_rot, v_st, sk, dom, 40, 1e4)
+    ok = list(idx) == list(range(40))
+    for j in range(4):
+        qr = m.rope_rotate(m.to_f64(qpre[j]), 36 + j, 1e4)
+        mask = torch.from_numpy(np.arange(40) <= 36 + j)[None].expand(2, 40)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qr)[None], torch.from_numpy(m.to_f64(k_rot))[None],
+            torch.from_numpy(m.to_f64(v_st))[None], attn_mask=mask[None])[0].numpy()
+        ok &= _close(out[j], want, rtol=1e-9, atol=1e-12)
+    return bool(ok)
+
+
+def check_multi_masked_row_without_slots_is_zero(m):
+    # one kept token after the first query's position: that row is zero, the
+    # rows that see it get its V row (the first seed where the best token is
+    # slot 10 or 11 of 12)
+    dom = np.arange(64)
+    for seed in range(34, 400):
+        qpre, kpre, v = _multi_case(L=12, n_q=3, G=1, seed=seed)
+        k_rot, v_st, sk = m.append_kv(kpre, v, 0, 1e4, dom, "f32")
+        idx, out, s = m.decode_multi_head(qpre, 9, k_rot, v_st, sk, dom, 1, 1e4)
+        if idx[0] > 9:
+            break
+    else:
+        return False
+    t = int(idx[0])
+    ok = int(np.argmax(s)) == t and np.all(out[0] == 0.0)
+    for j in (1, 2):
+        want = m.to_f64(v_st)[t][None] if t <= 9 + j else np.zeros((1, 128))
+        ok &= _close(out[j], want)
+    return bool(ok)
+
+
 def check_append_positions(m):
     qpre, kpre, v = _head(L=30, seed=10, dtype="bf16")
     dom = np.array([0, 2, 4])
@@ -399,7 +473,9 @@ PINS = [check_bf16_vs_torch, check_bf16_halfway_exact, check_rope_vs_complex,
         check_select_permutation, check_dense_vs_sdpa, check_focused_special_cases,
         check_e2e_all_fc_full_k_is_dense, check_e2e_all_fc_topk_exact, check_append_positions,
         check_calib_planes_closed_form, check_calib_planes_match_tip, check_calib_counts_brute_force,
-        check_calib_single_fc_query, check_calib_budget_covers_all, check_dominant_ties]
+        check_calib_single_fc_query, check_calib_budget_covers_all, check_dominant_ties,
+        check_multi_one_query_is_decode, check_multi_scores_add_over_positions, check_multi_causal_vs_sdpa,
+        check_multi_masked_row_without_slots_is_zero]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -510,7 +586,25 @@ _orig_calib_counts = O.calibration_counts
 _orig_append = O.append_kv
 _orig_tip = O.tip_scores
 
+def _mut_multi_one_position(q_pre, q_pos0, k_rot, v, sketch, dom, k, base):
+    q = O.to_f64(q_pre)
+    qr = np.stack([O.rotate_queries(q[j], q_pos0, base) for j in range(q.shape[0])])
+    s = O.tip_scores(qr.reshape(-1, 128), sketch, dom)
+    idx = O.select_critical_set(s, k)
+    return idx, np.stack([O.focused_attention(qr[j], k_rot, v, idx) for j in range(q.shape[0])]), s
+
+
+def _mut_multi_no_mask(q_pre, q_pos0, k_rot, v, sketch, dom, k, base):
+    q = O.to_f64(q_pre)
+    qr = np.stack([O.rotate_queries(q[j], q_pos0 + j, base) for j in range(q.shape[0])])
+    s = O.tip_scores(qr.reshape(-1, 128), sketch, dom)
+    idx = O.select_critical_set(s, k)
+    return idx, np.stack([O.focused_attention(qr[j], k_rot, v, idx) for j in range(q.shape[0])]), s
+
+
 MUTANTS = {
+    "multi_rotates_every_token_at_first_position": ("decode_multi_head", _mut_multi_one_position),
+    "multi_without_causal_mask": ("decode_multi_head", _mut_multi_no_mask),
     "rope_rotates_backwards": ("rope_rotate", _mut_rope_sign),
     "rope_adjacent_pairs": ("rope_rotate", _mut_rope_adjacent),
     "rope_theta_exponent": ("rope_frequencies", _mut_freq),
