@@ -409,6 +409,39 @@ fasa_status fasa_decode_paged(const fasa_cache* cache, const fasa_paged* pages, 
                               const void* q, void* out, int32_t* idx_out, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Multi-query decode: n_q query tokens per sequence in one step (draft
+ * tokens to verify, or several rows served together). Reading of the pages
+ * for more than one query ([tech §2] TIP's group sum, FAC): the n_q * G
+ * query rows of KV head g share one critical set, the k_eff best tokens by
+ * s_t = sum_j sum_{h in g} sum_{i in D_g} P_i(q'_{j,h}, k'_t); each row then
+ * attends over the kept slots that are not after its own position. Query
+ * token j sits at position q_pos0 + j: with q_pos0 >= len (the usual case)
+ * every kept slot is visible; with draft tokens already appended at
+ * q_pos0 .. q_pos0 + n_q - 1 the rows see only what precedes them. A row
+ * left with no visible kept slot is zero. With q_pos0 = FASA_Q_PREROTATED
+ * the queries are used as given and nothing is masked.
+ *
+ * The attention runs on the tensor cores (tcgen05, accumulators in tensor
+ * memory): Q K^T and P V over tiles of 128 kept rows, each bf16 operand
+ * that is not stored in the cache (the scaled rotated queries, the
+ * probabilities) split into two bf16 terms, float32 accumulation.
+ *
+ *  q       : [B][n_q][Hq][128] bf16.
+ *  out     : [B][n_q][Hq][128] bf16.
+ *  idx_out : nullable; [B][Hkv][k_eff] int32, ascending.
+ *  n_q     : 1 .. 16, with n_q * G <= 64.
+ *  workspace: zeroed once before first use, at least
+ *            fasa_decode_multi_workspace_bytes(cache, len, n_q, k) bytes,
+ *            256-byte aligned; every call leaves it ready for the next.
+ *  Errors: as fasa_decode; n_q out of range or f32 caches ->
+ *  FASA_ERR_UNSUPPORTED (n_q < 1 -> FASA_ERR_INVALID_ARG).
+ */
+size_t fasa_decode_multi_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t n_q, int32_t k);
+fasa_status fasa_decode_multi(const fasa_cache* cache, int32_t len, const void* q, int32_t q_pos0, int32_t n_q,
+                              int32_t k, void* out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
 /* Size of the library's own device scratch used by
  * fasa_decode_static_scratch: 64 MiB, held by every GPU that loads the
  * library until the process exits. */

@@ -93,6 +93,10 @@ struct WideParams {
   int32_t* row_keep;       // [rows] each row's k_eff, for the attention launch (varlen), or null
   int32_t q_prerot;        // varlen: 1 if the queries are already rotated
   PageMap pm;              // paged pools (pm.table set), else [rows][max_len] planes
+  // multi-query decode: n_q query tokens per sequence, q [B][n_q][Hq][128],
+  // token j at position q_pos0 + j (angles from theta_i in cosv), or 1
+  int32_t n_q;
+  int32_t q_pos0;
   double cosv[kNFC];       // cos / sin of the query angle (uniform length), or
   double sinv[kNFC];       // theta_i in cosv (varlen: the angle is seq_len[b] * theta_i)
 };
@@ -129,7 +133,7 @@ struct WdLayout {
   int hist, misc, coef, qraw, dom, cs, qs, pgs, cnt, kept, r1, bitmap, ties, rscr, ucache, zs, ring, total;
 };
 __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, int direct, int group, int n_split,
-                                              int P, int paged) {
+                                              int P, int paged, int n_q) {
   WdLayout L;
   const int MG = group <= 4 ? 4 : 8;
   int o = 0;
@@ -140,11 +144,11 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   L.coef = o;
   o += kD * 4;
   L.qraw = o;
-  o += FASA_MAX_GROUP * kD * 2;
+  o += (n_q * group > FASA_MAX_GROUP ? n_q * group : FASA_MAX_GROUP) * kD * 2;
   L.dom = o;
   o += kNFC * 4;
-  L.cs = o;  // cos, sin of the query angle (float64)
-  o += 2 * kNFC * 8;
+  L.cs = o;  // cos, sin of each query token's angle (float64)
+  o += 2 * kNFC * 8 * n_q;
   L.qs = o;  // attention queries [MG][128] f32
   o += direct ? MG * kD * 4 : 0;
   L.pgs = o;  // paged: the CTA's pages (block size >= 16)
@@ -379,7 +383,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   using S = TipShape<__nv_bfloat16, LPT>;
   constexpr int U = S::LPT2 == 1 ? 4 : 2;  // tokens in flight per lane
   extern __shared__ __align__(128) unsigned char smem[];
-  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.n_split, p.ucache, p.pm.table != nullptr);
+  const WdLayout Lo = wd_layout(p.n_loc, p.len, p.n_keep, p.direct, p.group, p.n_split, p.ucache, p.pm.table != nullptr,
+                                p.n_q);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + Lo.hist);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lo.misc);
   float* coef = reinterpret_cast<float*>(smem + Lo.coef);
@@ -442,10 +447,27 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int G = p.group;
   double* cs_sm = reinterpret_cast<double*>(smem + Lo.cs);
   {
-    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
-    for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    if (p.n_q == 1) {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
+      for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+    } else {  // rows j * G + h: token j's group queries
+      const int hq = p.n_kv_heads * G;
+      for (int c = tid; c < p.n_q * G * kD / 8; c += kWdThreads) {
+        const int r = c / (kD / 8), j = r / G, h = r % G;
+        reinterpret_cast<uint4*>(qraw)[c] = __ldg(
+            reinterpret_cast<const uint4*>(p.q + (((int64_t)bb * p.n_q + j) * hq + g * G + h) * kD) + c % (kD / 8));
+      }
+    }
     if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
-    if (!p.seq_len) {
+    if (p.n_q > 1) {  // token j at position q_pos0 + j
+      for (int e = tid; e < p.n_q * kNFC; e += kWdThreads) {
+        const int j = e / kNFC, i = e % kNFC;
+        double sn = 0.0, cn = 1.0;
+        if (!p.q_prerot) sincos((double)(p.q_pos0 + j) * p.cosv[i], &sn, &cn);
+        cs_sm[j * 2 * kNFC + i] = cn;
+        cs_sm[j * 2 * kNFC + kNFC + i] = sn;
+      }
+    } else if (!p.seq_len) {
       if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
       else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
     } else if (tid < kNFC) {  // the query of sequence b sits at position Lr
@@ -472,7 +494,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   load_rows(0);
   for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
   __syncthreads();
-  if (tid < p.stride) coef[tid] = tip_coef<__nv_bfloat16>(qraw, s_dom, G, p.n_dom, tid, cs_sm, cs_sm + kNFC);
+  if (tid < p.stride)
+    coef[tid] = tip_coef<__nv_bfloat16>(qraw, s_dom, G, p.n_dom, tid, cs_sm, cs_sm + kNFC, p.n_q, 2 * kNFC);
   // the attention queries, used by the row's resolving CTA
   if (p.direct) cc_queries(qraw, G, MG, cs_sm, cs_sm + kNFC, reinterpret_cast<float*>(smem + Lo.qs), tid, kWdThreads);
   __syncthreads();

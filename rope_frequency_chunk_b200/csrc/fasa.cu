@@ -15,6 +15,7 @@
 #include "select_attend.cuh"
 #include "select_hist.cuh"
 #include "attend_cc.cuh"
+#include "attend_tc.cuh"
 #include "decode_wide.cuh"
 #include "calibrate.cuh"
 
@@ -409,7 +410,8 @@ fasa_status check_paged(const fasa_cache* c, const fasa_paged* pg) {
 // shared-memory limit on keys per CTA allows); tokens per CTA. The
 // resolving CTA attends itself for budgets up to kWdMaxDirect when its ring
 // fits, and caches as much of the published union as shared memory allows.
-bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl, int paged = 0) {
+bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d, WidePlan* pl, int paged = 0,
+               int n_q = 0) {
   if (c->dtype != FASA_BF16) return false;
   const int64_t rows = (int64_t)c->batch * c->n_kv_heads;
   // about one CTA per SM, leaving one SM per row free: the rows' resolving
@@ -427,8 +429,10 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   pl->n_pub = pl->n_split == 1 ? keff
                                 : (int)std::min<int64_t>(keff, (2 * ceil_div(keff, pl->n_split) + 32 + 31) / 32 * 32);
   const int G = c->n_q_heads / c->n_kv_heads;
-  for (int direct = (keff <= kWdMaxDirect && G <= 8) ? 1 : 0; direct >= 0; --direct) {
-    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0, paged);
+  // n_q > 0: the multi-query decode (n_q tokens, the attention in its own launch)
+  const int nq = n_q > 0 ? n_q : 1;
+  for (int direct = (keff <= kWdMaxDirect && G <= 8 && n_q == 0) ? 1 : 0; direct >= 0; --direct) {
+    const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0, paged, nq);
     if (base.total > d.smem_optin) continue;
     // entries of each CTA's region the resolving CTA stages in shared memory:
     // a power of two covering what a CTA usually publishes (its k_eff best
@@ -441,7 +445,7 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
     pl->ucache = (int)P;
     pl->ushift = 0;
     while ((1 << pl->ushift) < P) ++pl->ushift;
-    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache, paged).total;
+    pl->smem = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, pl->ucache, paged, nq).total;
     if (pl->smem > d.smem_optin) continue;
     return true;
   }
@@ -692,6 +696,78 @@ fasa_status launch_append(const fasa_cache* c, const void* k_new, const void* v_
   return cuda_status(cudaGetLastError());
 }
 
+// Multi-query decode workspace: the decode workspace, then the tensor-core
+// attention's split partials [rows][splits][kTcPartStride] f32.
+struct MultiWs {
+  DecodeWs w;
+  size_t tpart, total;
+  int splits_max;
+};
+inline int tc_splits(int rows, int keff, int sms) {
+  const int64_t tiles = ceil_div(std::max(keff, 1), kTcTile);
+  const int64_t s = std::min<int64_t>(tiles, std::max<int64_t>(1, (int64_t)sms / rows));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(s, kTcMaxSplits));
+}
+MultiWs multi_layout(const fasa_cache* c, int32_t len, int32_t k) {
+  MultiWs m;
+  m.w = decode_layout(c, len, k);
+  const size_t rows = (size_t)c->batch * c->n_kv_heads;
+  m.splits_max = tc_splits((int)rows, std::max(0, std::min(k, len)), kAssumedMaxSms);
+  m.tpart = al256(m.w.total);
+  m.total = al256(m.tpart + rows * (size_t)m.splits_max * kTcPartStride * 4) + 256;
+  return m;
+}
+
+fasa_status launch_tc(const fasa_cache* c, int32_t len, int keff, const void* q, int32_t q_pos0, int32_t n_q,
+                      void* out, const MultiWs& m, char* base, const DevInfo& d, cudaStream_t st) {
+  const int rows = c->batch * c->n_kv_heads;
+  TcParams tp{};
+  tp.k = static_cast<const __nv_bfloat16*>(c->k);
+  tp.v = static_cast<const __nv_bfloat16*>(c->v);
+  tp.idx = reinterpret_cast<const int32_t*>(base + m.w.idx);
+  tp.q = static_cast<const __nv_bfloat16*>(q);
+  tp.out = static_cast<__nv_bfloat16*>(out);
+  tp.part = reinterpret_cast<float*>(base + m.tpart);
+  tp.counter = reinterpret_cast<uint32_t*>(base + m.w.att_cnt);
+  tp.max_len = c->max_len;
+  tp.len = len;
+  tp.n_keep = keff;
+  tp.group = c->n_q_heads / c->n_kv_heads;
+  tp.n_q = n_q;
+  tp.n_kv_heads = c->n_kv_heads;
+  tp.q_prerot = q_pos0 == FASA_Q_PREROTATED ? 1 : 0;
+  tp.q_pos0 = tp.q_prerot ? 0 : q_pos0;
+  fill_theta(tp.theta, c->rope_base);
+  const int splits = std::min(m.splits_max, tc_splits(rows, keff, d.sms));
+  const int64_t tiles = ceil_div(keff, kTcTile);
+  tp.slice = (int)(ceil_div(tiles, splits) * kTcTile);
+  tp.splits = (int)ceil_div(keff, tp.slice);
+  const int smem = tc_smem_bytes(n_q * tp.group, n_q);
+  int ok = 0;
+  fasa_status s = cached_int(reinterpret_cast<const void*>(attend_tc_kernel), 0, &ok, [&](int* r) {
+    *r = 1;
+    return cuda_status(cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            tc_smem_bytes(kTcMaxRows, kTcMaxTok)));
+  });
+  if (s != FASA_OK) return s;
+  return launch_pdl(attend_tc_kernel, dim3((unsigned)tp.splits, (unsigned)rows, 1), kTcThreads, (size_t)smem, st,
+                    tp);
+}
+
+// The fused kernel's instance for the sketch row length (16-byte chunks) and
+// the padded head count of its in-CTA attention.
+fasa_status launch_wide_sel(const WideParams& p, int rows, const WidePlan& pl, const DevInfo& d, cudaStream_t st) {
+  const bool g4 = p.group <= 4;  // padded heads of the in-CTA attention: 4 or 8
+  switch (p.stride / 8) {
+    case 1: return g4 ? launch_wide_t<1, 4>(p, rows, pl, st, d) : launch_wide_t<1, 8>(p, rows, pl, st, d);
+    case 2: return g4 ? launch_wide_t<2, 4>(p, rows, pl, st, d) : launch_wide_t<2, 8>(p, rows, pl, st, d);
+    case 4: return g4 ? launch_wide_t<4, 4>(p, rows, pl, st, d) : launch_wide_t<4, 8>(p, rows, pl, st, d);
+    case 8: return g4 ? launch_wide_t<8, 4>(p, rows, pl, st, d) : launch_wide_t<8, 8>(p, rows, pl, st, d);
+    case 16: return g4 ? launch_wide_t<16, 4>(p, rows, pl, st, d) : launch_wide_t<16, 8>(p, rows, pl, st, d);
+    default: return FASA_ERR_UNSUPPORTED;
+  }
+}
+
 // The wide fused decode: one launch, plus the split-K attention when the
 // budget is beyond what the resolving CTA attends itself.
 fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int keff, void* out,
@@ -699,6 +775,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
                         cudaStream_t st, const fasa_varlen* vl = nullptr, const fasa_paged* pg = nullptr) {
   WideParams p{};
   p.pm = page_map(c, pg);
+  p.n_q = 1;
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
   p.v = static_cast<const __nv_bfloat16*>(c->v);
@@ -732,17 +809,7 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   } else {
     fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos);
   }
-  const int rows = c->batch * c->n_kv_heads;
-  fasa_status s;
-  const bool g4 = p.group <= 4;  // padded heads of the in-CTA attention: 4 or 8
-  switch (c->sketch_stride / 8) {  // 16-byte chunks per sketch row
-    case 1: s = g4 ? launch_wide_t<1, 4>(p, rows, pl, st, d) : launch_wide_t<1, 8>(p, rows, pl, st, d); break;
-    case 2: s = g4 ? launch_wide_t<2, 4>(p, rows, pl, st, d) : launch_wide_t<2, 8>(p, rows, pl, st, d); break;
-    case 4: s = g4 ? launch_wide_t<4, 4>(p, rows, pl, st, d) : launch_wide_t<4, 8>(p, rows, pl, st, d); break;
-    case 8: s = g4 ? launch_wide_t<8, 4>(p, rows, pl, st, d) : launch_wide_t<8, 8>(p, rows, pl, st, d); break;
-    case 16: s = g4 ? launch_wide_t<16, 4>(p, rows, pl, st, d) : launch_wide_t<16, 8>(p, rows, pl, st, d); break;
-    default: return FASA_ERR_UNSUPPORTED;
-  }
+  const fasa_status s = launch_wide_sel(p, c->batch * c->n_kv_heads, pl, d, st);
   if (s != FASA_OK || pl.direct) return s;
   return launch_attend_ws(c, len, keff, q, q_pos, out, w, base, d, st, vl, pg);
 }
@@ -1074,6 +1141,66 @@ fasa_status fasa_decode_paged(const fasa_cache* c, const fasa_paged* pg, const f
   if (s != FASA_OK) return s;
   if ((s = check_paged(c, pg)) != FASA_OK) return s;
   return decode_varlen(c, vl, q, out, idx_out, workspace, workspace_bytes, stream, pg);
+}
+
+size_t fasa_decode_multi_workspace_bytes(const fasa_cache* c, int32_t len, int32_t n_q, int32_t k) {
+  if (check_cache(c) != FASA_OK || len < 1 || k < 1 || n_q < 1) return 0;
+  return multi_layout(c, len, k).total;
+}
+
+fasa_status fasa_decode_multi(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos0, int32_t n_q,
+                              int32_t k, void* out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  fasa_status s = check_cache(c);
+  if (s != FASA_OK) return s;
+  if (len < 1 || k < 1 || n_q < 1 || bad_qpos(q_pos0)) return FASA_ERR_INVALID_ARG;
+  if (q_pos0 != FASA_Q_PREROTATED && (int64_t)q_pos0 + n_q - 1 > INT32_MAX) return FASA_ERR_INVALID_ARG;
+  if (len > c->max_len) return FASA_ERR_CAPACITY;
+  if (len > FASA_MAX_LEN || k > FASA_MAX_K || c->dtype != FASA_BF16) return FASA_ERR_UNSUPPORTED;
+  if (n_q > kTcMaxTok || n_q * (c->n_q_heads / c->n_kv_heads) > kTcMaxRows) return FASA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16)) return FASA_ERR_INVALID_ARG;
+  if (idx_out != nullptr && !aligned(idx_out, 4)) return FASA_ERR_INVALID_ARG;
+  const int keff = std::min(k, len);
+  const MultiWs m = multi_layout(c, len, k);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < m.total) return FASA_ERR_WORKSPACE;
+  DevInfo d;
+  if ((s = device_info(&d)) != FASA_OK) return s;
+  WidePlan pl;
+  if (!wide_plan(c, len, keff, d, &pl, 0, n_q)) return FASA_ERR_UNSUPPORTED;
+  char* base = static_cast<char*>(workspace);
+  // scoring and selection: the fused kernel with the n_q tokens' coefficients
+  WideParams p{};
+  p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
+  p.k = static_cast<const __nv_bfloat16*>(c->k);
+  p.v = static_cast<const __nv_bfloat16*>(c->v);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.dom_idx = c->dom_idx;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.idx_out = idx_out;
+  p.idx_ws = reinterpret_cast<int32_t*>(base + m.w.idx);
+  p.cand = reinterpret_cast<uint2*>(base + m.w.scores);
+  p.sem = reinterpret_cast<unsigned long long*>(base + m.w.sem);
+  p.keys = reinterpret_cast<uint32_t*>(base + m.w.keys);
+  p.max_len = c->max_len;
+  p.len = len;
+  p.stride = c->sketch_stride;
+  p.n_kv_heads = c->n_kv_heads;
+  p.group = c->n_q_heads / c->n_kv_heads;
+  p.n_dom = c->n_dom;
+  p.n_keep = keff;
+  p.n_pub = pl.n_pub;
+  p.n_loc = pl.n_loc;
+  p.n_split = pl.n_split;
+  p.ucache = pl.ucache;
+  p.ushift = pl.ushift;
+  p.direct = 0;
+  p.pm = page_map(c, nullptr);
+  p.n_q = n_q;
+  p.q_prerot = q_pos0 == FASA_Q_PREROTATED ? 1 : 0;
+  p.q_pos0 = p.q_prerot ? 0 : q_pos0;
+  fill_theta(p.cosv, c->rope_base);
+  if ((s = launch_wide_sel(p, c->batch * c->n_kv_heads, pl, d, stream)) != FASA_OK) return s;
+  return launch_tc(c, len, keff, q, q_pos0, n_q, out, m, base, d, stream);
 }
 
 fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, int32_t k,

@@ -49,9 +49,14 @@ struct TipShape {
 // once to float32). qraw holds the group's G pre-RoPE queries [G][128];
 // cosv/sinv are cos and sin of q_pos * theta_i. Padding columns (col >=
 // 2 n_dom) are zero. An FC index outside [0, 64) is flagged and gives zero.
+// With n_tok query tokens per sequence (multi-query decode), qraw holds
+// n_tok * G rows, token-major, and the rows of token j take the angle table
+// at cosv + j * cs_stride (sinv likewise); the sum runs over every row in
+// that order.
 template <typename T>
 __device__ __forceinline__ float tip_coef(const T* qraw, const int* dom, int group, int n_dom, int col,
-                                          const double* cosv, const double* sinv) {
+                                          const double* cosv, const double* sinv, int n_tok = 1,
+                                          int cs_stride = 0) {
   const int jj = col >> 1;
   if (jj >= n_dom) return 0.0f;
   const int i = dom[jj];
@@ -59,9 +64,10 @@ __device__ __forceinline__ float tip_coef(const T* qraw, const int* dom, int gro
     flag_status(FASA_ERR_BAD_INDEX);
     return 0.0f;
   }
-  const double c = cosv[i], s = sinv[i];
   double acc = 0.0;
-  for (int h = 0; h < group; ++h) {
+  for (int h = 0; h < group * n_tok; ++h) {
+    const int j = h / group;
+    const double c = cosv[j * cs_stride + i], s = sinv[j * cs_stride + i];
     const double x = to_float(qraw[h * kD + i]);
     const double y = to_float(qraw[h * kD + i + kNFC]);
     // rotated query, first (x') or second (y') dim of FC i

@@ -74,6 +74,8 @@ _SIGS = {
                                                             ctypes.POINTER(fasa_varlen)]),
     "fasa_decode_paged": (_I, [_CP, ctypes.POINTER(fasa_paged), ctypes.POINTER(fasa_varlen), _P, _P, _P, _P,
                                ctypes.c_size_t, _P]),
+    "fasa_decode_multi_workspace_bytes": (ctypes.c_size_t, [_CP, _I, _I, _I]),
+    "fasa_decode_multi": (_I, [_CP, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "fasa_decode_static_scratch": (_I, [_CP, _I, _P, _I, _I, _P, _P, _P]),
     "fasa_dense_workspace_bytes": (ctypes.c_size_t, [_CP, _I]),
     "fasa_dense_decode": (_I, [_CP, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]),
@@ -406,6 +408,35 @@ def fasa_decode_varlen(cache: KVCache, seq_len, q, max_seq_len: int, max_budget:
     _check(lib().fasa_decode_varlen(cache.ref(), ctypes.byref(vl), q.data_ptr(), out.data_ptr(), _ptr(idx_out),
                                     workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "fasa_decode_varlen")
+    return out
+
+
+def fasa_decode_multi_workspace(cache: KVCache, length: int, n_q: int, k: int, device=None):
+    """A zeroed workspace for fasa_decode_multi at this shape."""
+    dev = device if device is not None else cache.k.device
+    need = int(lib().fasa_decode_multi_workspace_bytes(cache.ref(), length, n_q, k))
+    return torch.zeros(max(need, 1), dtype=torch.uint8, device=dev)
+
+
+def fasa_decode_multi(cache: KVCache, length: int, q, q_pos0: int, k: int, out=None, idx_out=None,
+                      workspace=None, stream=None):
+    """Multi-query decode: q [B, n_q, Hq, 128], token j at position q_pos0 + j;
+    the query rows of a KV head share one kept set (idx_out [B, Hkv, k_eff])."""
+    _dev(q, "q", cache.dtype)
+    if q.dim() != 4 or tuple(q.shape[::2]) != (cache.batch, cache.n_q_heads) or q.shape[3] != HEAD_DIM:
+        raise ValueError("q must be [B, n_q, Hq, 128]")
+    n_q = q.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", cache.dtype)
+    if idx_out is not None:
+        _dev(idx_out, "idx_out", torch.int32)
+    if workspace is None:
+        workspace = fasa_decode_multi_workspace(cache, length, n_q, k, q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    _check(lib().fasa_decode_multi(cache.ref(), length, q.data_ptr(), q_pos0, n_q, k, out.data_ptr(),
+                                   _ptr(idx_out), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "fasa_decode_multi")
     return out
 
 

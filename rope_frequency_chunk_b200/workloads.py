@@ -249,6 +249,20 @@ def layer_inputs(wl: Workload, layer: int = 0, n_dom: int | None = None,
     return LayerInputs(lp, q, k, v)
 
 
+def multi_queries(wl: Workload, n_q: int, layer: int = 0, n_dom: int | None = None) -> np.ndarray:
+    """Queries of n_q tokens per sequence, [B][n_q][Hq][128] stored: token j
+    is the layer's query of decode step j (token 0 = layer_inputs' q)."""
+    lp = layer_params(wl, layer, n_dom)
+    B, H, G = wl.batch, wl.n_kv_heads, wl.group
+    sdt = np.float32 if wl.dtype == "f32" else np.uint16
+    q = np.empty((B, n_q, H * G, HEAD_DIM), sdt)
+    for j in range(n_q):
+        for b in range(B):
+            for g in range(H):
+                q[b, j, g * G:(g + 1) * G] = head_q(wl, lp, layer, b, g, j)
+    return q
+
+
 def to_torch(a: np.ndarray, device="cpu"):
     """Stored array (float32, or uint16 bf16 bits) -> torch tensor of the cache dtype."""
     import torch

@@ -210,3 +210,23 @@ def test_paged_validation_without_launch(L):
     assert app(c, pg(), 0x50000, 0x60000, 0, 0x90000, None) == 0              # no-op
     assert app(c, pg(), 0x50008, 0x60000, 4, 0x90000, None) == 1              # misaligned input
     assert app(c, pg(block_size=24), 0x50000, 0x60000, 4, 0x90000, None) == 1
+
+
+def test_multi_validation_without_launch(L):
+    c = ctypes.byref(_fake_cache())  # G = 2
+    ws = L.fasa_decode_multi_workspace_bytes
+    need = ws(c, 100, 4, 8)
+    assert need > L.fasa_decode_workspace_bytes(c, 100, 8) and need % 256 == 0
+    assert ws(c, 0, 4, 8) == 0 and ws(c, 100, 0, 8) == 0 and ws(c, 100, 4, 0) == 0
+    run = L.fasa_decode_multi
+    tail = (0x70000, None, 0x80000, need, None)
+    assert run(c, 100, 0x50000, 100, 0, 8, *tail) == 1          # n_q < 1
+    assert run(c, 100, 0x50000, 100, 17, 8, *tail) == 2         # more than 16 tokens
+    assert run(ctypes.byref(_fake_cache(n_q_heads=32, n_kv_heads=2)), 100, 0x50000, 100, 5, 8, *tail) == 2
+    assert run(c, 100, 0x50000, -2, 4, 8, *tail) == 1           # bad position
+    assert run(c, 100, 0x50000, 2 ** 31 - 2, 4, 8, *tail) == 1  # positions overflow
+    assert run(c, 2000, 0x50000, 100, 4, 8, *tail) == 3
+    assert run(ctypes.byref(_fake_cache(dtype=0)), 100, 0x50000, 100, 4, 8, *tail) == 2
+    assert run(c, 100, 0x50008, 100, 4, 8, *tail) == 1
+    assert run(c, 100, 0x50000, 100, 4, 8, 0x70000, None, 0x80000, need - 1, None) == 4
+    assert run(c, 100, 0x50000, 100, 4, 8, 0x70000, None, None, need, None) == 4
