@@ -1198,7 +1198,10 @@ fasa_status fasa_decode_multi(const fasa_cache* c, int32_t len, const void* q, i
   p.n_q = n_q;
   p.q_prerot = q_pos0 == FASA_Q_PREROTATED ? 1 : 0;
   p.q_pos0 = p.q_prerot ? 0 : q_pos0;
-  fill_theta(p.cosv, c->rope_base);
+  if (n_q == 1)  // the single-token path takes the angle's cos / sin
+    fill_query_angle(p.cosv, p.sinv, c->rope_base, q_pos0);
+  else
+    fill_theta(p.cosv, c->rope_base);
   if ((s = launch_wide_sel(p, c->batch * c->n_kv_heads, pl, d, stream)) != FASA_OK) return s;
   return launch_tc(c, len, keff, q, q_pos0, n_q, out, m, base, d, stream);
 }
