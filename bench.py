@@ -422,6 +422,43 @@ def run_fasa_m(args, wl, k, n_layers, qs, outs, ws, stream, fasa_c_bytes):
     return res
 
 
+def run_multi_query(args, wl, k, n_layers, caches, stream, us_single):
+    """Multi-query decode legs: n_q tokens per sequence (one shared kept set
+    per KV head, attention on the tensor cores) on the same layer stack."""
+    import torch
+    from rope_frequency_chunk_b200 import fasa as F
+    G = wl.group
+    L = wl.ctx_len
+    res = {}
+    for n_q in args.multi:
+        if n_q * G > 64 or n_q > 16:
+            continue
+        qs = [W.to_torch(W.multi_queries(wl, n_q, layer=i), caches[0].k.device) for i in range(n_layers)]
+        outs = [torch.empty_like(q) for q in qs]
+        ws = F.fasa_decode_multi_workspace(caches[0], L, n_q, k)
+
+        def step():
+            for c, q, o in zip(caches, qs, outs):
+                F.fasa_decode_multi(c, L, q, wl.q_pos, k, out=o, workspace=ws)
+
+        msteps = max(3, args.steps // 4)
+        per = []
+        ms = time_graph(step, msteps, args.warmup, stream, None, per_step=per) / msteps
+        status = F.fasa_device_status(clear=True)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after the multi-query decode")
+        us = 1e3 * ms / n_layers
+        qbytes = 2 * wl.batch * n_q * wl.n_q_heads * W.HEAD_DIM * wl.elem_bytes
+        byts = roofline_bytes(wl, k) - 2 * wl.batch * wl.n_q_heads * W.HEAD_DIM * wl.elem_bytes + qbytes
+        res[str(n_q)] = {"us_per_layer_step": us,
+                         "us_per_layer_step_p50": float(np.percentile(per, 50)) * 1e3 / n_layers,
+                         "query_rows_per_kv_head": n_q * G, "bytes_per_layer_step": byts,
+                         "gbs": byts / (us * 1e-6) / 1e9, "us_per_query_token": us / n_q,
+                         "speedup_vs_single_query_decodes": n_q * us_single / us}
+        del qs, outs, ws
+    return res
+
+
 def run_fasa(args, wl):
     import torch
     from rope_frequency_chunk_b200 import fasa as F
@@ -510,6 +547,9 @@ def run_fasa(args, wl):
         extra["dense_us_per_layer_step"] = 1e3 * ms_dense / n_layers
         extra["dense_gbs"] = dense_bytes(wl) * n_layers / (ms_dense * 1e-3) / 1e9
         extra["speedup_vs_dense"] = ms_dense / ms_step
+
+    if args.multi and wl.dtype == "bf16" and world == 1:
+        extra["multi_query"] = run_multi_query(args, wl, k, n_layers, caches, stream, us_layer)
 
     kv_host_bytes = 2 * wl.batch * wl.n_kv_heads * L * W.HEAD_DIM * wl.elem_bytes * n_layers
     if not args.no_fasa_m and world == 1 and kv_host_bytes <= FASA_M_MAX_HOST_BYTES:
@@ -753,6 +793,8 @@ def build_parser() -> argparse.ArgumentParser:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-fasa-m", action="store_true", help="skip the FASA-M (host-resident K/V) leg")
+    ap.add_argument("--multi", type=lambda s: [int(x) for x in s.split(",") if x], default=[4, 8, 16],
+                    help="query tokens per sequence of the multi-query legs (comma list; empty to skip)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--calibrate", action="store_true",
