@@ -178,28 +178,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
 
   const int b = row / p.n_kv_heads, g = row % p.n_kv_heads;
   const int hq = p.n_kv_heads * G;
-  // the query rows: row r = token j, head h of the group; rotated (float64),
-  // scaled by log2(e) / sqrt(128), split into bf16 hi + lo
-  if (tid < MQ) {
-    const int j = tid / G, h = tid % G;
-    const __nv_bfloat16* qr = p.q + (((int64_t)b * p.n_q + j) * hq + g * G + h) * kD;
-    const double* c = cs + j * 2 * kNFC;
+  // the query rows: row r = token j, head h of the group; staged raw in the
+  // P hi tiles (free until the first softmax), then rotated (float64),
+  // scaled by log2(e) / sqrt(128) and split into bf16 hi + lo, 8 dims per
+  // thread and step
+  {
+    uint4* qst = reinterpret_cast<uint4*>(phi);  // [MQ][16] raw chunks
+    for (int c = tid; c < MQ * 16; c += kTcThreads) {
+      const int r = c >> 4, j = r / G, h = r % G;
+      qst[c] = __ldg(reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.n_q + j) * hq + g * G + h) * kD) +
+                     (c & 15));
+    }
+    __syncthreads();
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(phi);
     const double qscale = 1.4426950408889634 / 11.313708498984761;
-#pragma unroll 1
-    for (int ch = 0; ch < 16; ++ch) {
+    for (int c = tid; c < MQ * 16; c += kTcThreads) {
+      const int r = c >> 4, ch = c & 15;
+      const double* cz = cs + (r / G) * 2 * kNFC;
       float x[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int d = ch * 8 + e, i = d & (kNFC - 1);
-        const double a = __bfloat162float(qr[i]), bb = __bfloat162float(qr[i + kNFC]);
-        const double rr = d < kNFC ? __dsub_rn(__dmul_rn(a, c[i]), __dmul_rn(bb, c[kNFC + i]))
-                                   : __dadd_rn(__dmul_rn(bb, c[i]), __dmul_rn(a, c[kNFC + i]));
+        const double a = __bfloat162float(qs[r * kD + i]), bb = __bfloat162float(qs[r * kD + i + kNFC]);
+        const double rr = d < kNFC ? __dsub_rn(__dmul_rn(a, cz[i]), __dmul_rn(bb, cz[kNFC + i]))
+                                   : __dadd_rn(__dmul_rn(bb, cz[i]), __dmul_rn(a, cz[kNFC + i]));
         x[e] = (float)(rr * qscale);
       }
       uint4 hi, lo;
       tc_split8(x, hi, lo);
-      *reinterpret_cast<uint4*>(qhi + tc_sw(tid, ch, RQ)) = hi;
-      *reinterpret_cast<uint4*>(qlo + tc_sw(tid, ch, RQ)) = lo;
+      *reinterpret_cast<uint4*>(qhi + tc_sw(r, ch, RQ)) = hi;
+      *reinterpret_cast<uint4*>(qlo + tc_sw(r, ch, RQ)) = lo;
     }
   }
 
