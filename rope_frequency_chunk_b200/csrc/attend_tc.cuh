@@ -217,7 +217,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
   const __nv_bfloat16* vb = p.v + (int64_t)row * p.max_len * kD;
   const bool soft = warp * 32 < MQ;  // warps holding query rows (whole warps: tcgen05.ld is warp-wide)
   const int jq = tid / G;
-  const int lim = p.q_prerot ? 0x7FFFFFFF : p.q_pos0 + jq;  // slots after the row's position are masked
+  // visible columns: kept slot <= lim (masked entries hold kTcMasked)
+  constexpr int kTcMasked = 0x7FFFFFFF;
+  const int lim = p.q_prerot ? kTcMasked - 1 : min(p.q_pos0 + jq, kTcMasked - 1);
   const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
   float m_run = -INFINITY, l_run = 0.0f;
   float o[kD];
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
           t = -1;
         }
       }
-      tok_s[tid] = t;
+      tok_s[tid] = t < 0 ? kTcMasked : t;
       const uint4* kr = reinterpret_cast<const uint4*>(kb + (int64_t)(t < 0 ? 0 : t) * kD);
       const uint4* vr = reinterpret_cast<const uint4*>(vb + (int64_t)(t < 0 ? 0 : t) * kD);
 #pragma unroll
@@ -277,8 +279,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
         tc_ld32(tl + ch * 32, s);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int t = tok_s[ch * 32 + i];
-          if (t >= 0 && t <= lim) cmax = fmaxf(cmax, s[i]);
+          if (tok_s[ch * 32 + i] <= lim) cmax = fmaxf(cmax, s[i]);
         }
       }
       const float m_new = fmaxf(m_run, cmax);
@@ -290,8 +291,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
         tc_ld32(tl + ch * 32, s);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int t = tok_s[ch * 32 + i];
-          s[i] = (t >= 0 && t <= lim && m_new != -INFINITY) ? exp2f(s[i] - m_new) : 0.0f;
+          s[i] = (tok_s[ch * 32 + i] <= lim && m_new != -INFINITY) ? exp2f(s[i] - m_new) : 0.0f;
           lsum += s[i];
         }
         if (tid < MQ) {
@@ -372,14 +372,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // merge in split order: weights w[s][r] = 2^(m_s - M), denominators
+  // merge in split order: weights w[s][r] = 2^(m_s - M), denominators; then
+  // each thread sums its float4 groups of o over the splits (the loads of one
+  // split are independent of each other, so they overlap)
   const float* rp = p.part + (int64_t)row * p.splits * kTcPartStride;
   float* w = reinterpret_cast<float*>(ks);  // [splits][64]
   float* den = w + p.splits * kTcMaxRows;   // [64]
   if (tid < MQ) {
     float M = -INFINITY;
+#pragma unroll 8
     for (int s = 0; s < p.splits; ++s) M = fmaxf(M, __ldcg(rp + s * kTcPartStride + tid));
     float dn = 0.0f;
+#pragma unroll 8
     for (int s = 0; s < p.splits; ++s) {
       const float ms = __ldcg(rp + s * kTcPartStride + tid);
       const float ws = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
@@ -389,12 +393,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
     den[tid] = dn;
   }
   __syncthreads();
-  for (int e = tid; e < MQ * kD; e += kTcThreads) {
-    const int r = e / kD, d = e % kD;
-    float num = 0.0f;
-    for (int s = 0; s < p.splits; ++s)
-      num = __fmaf_rn(w[s * kTcMaxRows + r], __ldcg(rp + s * kTcPartStride + 2 * kTcMaxRows + e), num);
-    *out_at(r, d) = __float2bfloat16_rn(den[r] > 0.0f ? num / den[r] : 0.0f);
+  constexpr int kGroups = kTcMaxRows * kD / 4 / kTcThreads;  // float4 groups per thread at most
+  const int n4 = MQ * kD / 4;
+  float4 acc[kGroups];
+#pragma unroll
+  for (int i = 0; i < kGroups; ++i) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int s = 0; s < p.splits; ++s) {
+    const float4* src = reinterpret_cast<const float4*>(rp + s * kTcPartStride + 2 * kTcMaxRows);
+#pragma unroll
+    for (int i = 0; i < kGroups; ++i) {
+      const int f = tid + i * kTcThreads;
+      if (f < n4) {
+        const float4 v = __ldcg(src + f);
+        const float ws = w[s * kTcMaxRows + f / (kD / 4)];
+        acc[i].x = __fmaf_rn(ws, v.x, acc[i].x);
+        acc[i].y = __fmaf_rn(ws, v.y, acc[i].y);
+        acc[i].z = __fmaf_rn(ws, v.z, acc[i].z);
+        acc[i].w = __fmaf_rn(ws, v.w, acc[i].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kGroups; ++i) {
+    const int f = tid + i * kTcThreads;
+    if (f < n4) {
+      const int r = f / (kD / 4), d = (f % (kD / 4)) * 4;
+      const float inv = den[r] > 0.0f ? 1.0f / den[r] : 0.0f;
+      __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out_at(r, d));
+      o2[0] = __floats2bfloat162_rn(acc[i].x * inv, acc[i].y * inv);
+      o2[1] = __floats2bfloat162_rn(acc[i].z * inv, acc[i].w * inv);
+    }
   }
   if (tid == 0) p.counter[row] = 0u;
 }
