@@ -558,23 +558,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       const uint32_t key = i < n_tok ? keys[i] : 0u;
       const bool q = i < n_tok && (key >> 20) >= b_loc;
       const unsigned m = __ballot_sync(0xFFFFFFFFu, q);
-      if (q) {
-        region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
-        // the candidate's K and V rows to L2: most of the kept set is among
-        // the published candidates, and the attention gathers it soon
-        const int tt = t_beg + i;
-        int64_t kr = -1;
-        if (!paged) {
-          kr = (int64_t)row * p.max_len + tt;
-        } else {
-          const int pg = s_pg[(tt >> p.pm.log2bs) - pg0];
-          if (pg >= 0) kr = ((pg * p.pm.n_kv_heads + g) << p.pm.log2bs) | (tt & ((1 << p.pm.log2bs) - 1));
-        }
-        if (kr >= 0) {
-          prefetch_l2(p.k + kr * kD, kD * 2);
-          prefetch_l2(p.v + kr * kD, kD * 2);
-        }
-      }
+      if (q) region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
       pos += __popc(m);
     }
     if (tid == 0) region[0] = make_uint2(misc[96], b_loc);
