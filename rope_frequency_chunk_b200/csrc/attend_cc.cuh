@@ -319,10 +319,16 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   float* mo = wsall + kCcWarps * cc_warp_scratch(MG);
   __nv_bfloat16* vball = reinterpret_cast<__nv_bfloat16*>(mo + kCcWarps * MG * kD);
   double* cs = reinterpret_cast<double*>(vball + kCcWarps * 2 * kCcStep * kD);
-  grid_dependency_wait();
   const int split = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.group;
+  // the angle table from the parameters, before the wait (its constant-bank
+  // misses overlap it); varlen rows take theta_i and rotate on the device
+  if (tid < kNFC) {
+    cs[tid] = p.cosv[tid];
+    cs[kNFC + tid] = p.sinv[tid];
+  }
+  grid_dependency_wait();
   int len = p.len, n_keep = p.n_keep;  // the row's length and kept count
   if (p.seq_len) {
     len = min(max(__ldg(p.seq_len + row / p.n_kv_heads), 1), p.len);  // range flagged by the fused kernel
@@ -331,13 +337,9 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   {
     const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
     for (int c = tid; c < G * kD / 8; c += kCcThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
-    if (tid < kNFC) {
-      double sn = p.sinv[tid], cn = p.cosv[tid];
-      if (p.seq_len) {  // the query of sequence b sits at position len
-        sn = 0.0;
-        cn = 1.0;
-        if (!p.q_prerot) sincos((double)len * p.cosv[tid], &sn, &cn);
-      }
+    if (p.seq_len && tid < kNFC) {  // the query of sequence b sits at position len
+      double sn = 0.0, cn = 1.0;
+      if (!p.q_prerot) sincos((double)len * cs[tid], &sn, &cn);
       cs[tid] = cn;
       cs[kNFC + tid] = sn;
     }

@@ -410,6 +410,13 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     for (int64_t o = (int64_t)tid * kPf; o < bytes; o += (int64_t)kWdThreads * kPf)
       prefetch_l2(src + o, (uint32_t)(bytes - o < kPf ? bytes - o : kPf));
   }
+  double* cs_sm = reinterpret_cast<double*>(smem + Lo.cs);
+  // the angle table from the parameters (no dependence on the previous
+  // launch): read before the wait, so its constant-bank misses overlap it
+  if (p.n_q == 1 && !p.seq_len) {
+    if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
+    else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
+  }
   grid_dependency_wait();
   grid_dependents_launch();
   // paged: the CTA's pages (read after the wait: an earlier launch may have
@@ -445,7 +452,6 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   // sketch rows are requested before the coefficients are formed, so the
   // query's round trip and the float64 work overlap the stream
   const int G = p.group;
-  double* cs_sm = reinterpret_cast<double*>(smem + Lo.cs);
   {
     if (p.n_q == 1) {
       const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
@@ -467,10 +473,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
         cs_sm[j * 2 * kNFC + i] = cn;
         cs_sm[j * 2 * kNFC + kNFC + i] = sn;
       }
-    } else if (!p.seq_len) {
-      if (tid < kNFC) cs_sm[tid] = p.cosv[tid];
-      else if (tid < 2 * kNFC) cs_sm[tid] = p.sinv[tid - kNFC];
-    } else if (tid < kNFC) {  // the query of sequence b sits at position Lr
+    } else if (p.seq_len && tid < kNFC) {  // the query of sequence b sits at position Lr
       double sn = 0.0, cn = 1.0;
       if (!p.q_prerot) sincos((double)Lr * p.cosv[tid], &sn, &cn);
       cs_sm[tid] = cn;

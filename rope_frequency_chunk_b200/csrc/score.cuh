@@ -127,6 +127,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
   __shared__ float s_q[kD];
   __shared__ __align__(16) T s_qraw[FASA_MAX_GROUP * kD];  // the group's raw queries
   __shared__ int s_dom[kNFC];
+  __shared__ double s_cs[2 * kNFC];  // cos, sin of the query angle
+  // the angle table from the parameters (no dependence on the previous
+  // launch): read before the wait, so its constant-bank misses overlap it
+  if (threadIdx.x < kNFC) s_cs[threadIdx.x] = p.cosv[threadIdx.x];
+  else if (threadIdx.x < 2 * kNFC) s_cs[threadIdx.x] = p.sinv[threadIdx.x - kNFC];
   grid_dependency_wait();
   grid_dependents_launch();  // the selection kernel may be scheduled now; it waits for our results
 
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
       if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
     }
     __syncthreads();
-    query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, p.cosv, p.sinv, tid, s_q);
+    query_coefs<T>(s_qraw, s_dom, p.group, p.n_dom, p.stride, s_cs, s_cs + kNFC, tid, s_q);
     __syncthreads();
     float qr[S::EPL];
     load_coefs<T, LPT>(qr, s_q, lane);
