@@ -327,6 +327,8 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   if (tid < kNFC) {
     cs[tid] = p.cosv[tid];
     cs[kNFC + tid] = p.sinv[tid];
+  } else if (tid < kNFC + 2 * G) {  // the group's queries to L2 (a hint)
+    prefetch_line_l2(p.q + (int64_t)row * G * kD + (tid - kNFC) * 64);
   }
   grid_dependency_wait();
   int len = p.len, n_keep = p.n_keep;  // the row's length and kept count
@@ -443,12 +445,15 @@ namespace fasa {
 // head h over all n logits (max, exp2, sum; zs becomes the probabilities);
 // (3) each warp adds p * v over its rows for the lane's 4 dims; (4) the warp
 // sums are added in a fixed order and divided by the head's sum.
-// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [MG],
-// vst [16 * NW][128] bf16 (the V rows, staged with cp.async).
-template <int MG, int NW, typename Tok>
+// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [16]
+// (sums, then maxima at lsum + 8), vst [16 * NW][128] bf16 (the V rows,
+// staged with cp.async). With PART the state is written unnormalised to
+// part instead (m at part[h], l at part[16 + h], o at part[32 + h * 128 + d],
+// the layout of a split partial) and out is not touched.
+template <int MG, int NW, bool PART = false, typename Tok>
 __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
                                                 int G, const float* qs, float* zs, float* mo, float* lsum,
-                                                __nv_bfloat16* vst, __nv_bfloat16* out) {
+                                                __nv_bfloat16* vst, __nv_bfloat16* out, float* part = nullptr) {
   constexpr int NG = MG / 4;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int jb = warp * 16;
@@ -513,7 +518,10 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-    if (lane == 0) lsum[warp] = l;
+    if (lane == 0) {
+      lsum[warp] = l;
+      if (PART) lsum[8 + warp] = m;
+    }
   }
   __syncthreads();
   // (3) p * v over the warp's rows
@@ -545,13 +553,22 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
   for (int h = 0; h < MG; ++h)
     *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
   __syncthreads();
-  // (4) warp sums in warp order, divided by the head's sum
+  // (4) warp sums in warp order, divided by the head's sum (or, with PART,
+  // written with the head's maximum and sum)
   for (int e = tid; e < G * kD; e += NW * 32) {
     const int h = e / kD, d = e % kD;
     float acc = 0.0f;
     for (int w = 0; w < NW; ++w) acc += mo[(w * MG + h) * kD + d];
     const float l = lsum[h];
-    out[e] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
+    if (PART) {
+      part[32 + e] = acc;
+      if (d == 0) {
+        part[h] = lsum[8 + h];
+        part[16 + h] = l;
+      }
+    } else {
+      out[e] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
+    }
   }
 }
 
