@@ -425,12 +425,15 @@ __device__ void wd_select(ForSrc&& for_src, SrcAt&& src_at, int n_src, int n_kee
 // union (key descending, token ascending), attend over the ones ranked below
 // kr, write the partial (and the kept list), and let the row's last CTA
 // merge the partials in CTA order. stage holds the union ([S][P], counts in
-// cnt[0, S)); rank (>= P words), kept and misc are shared scratch.
+// cnt[0, S)); rank (>= P words), kept, bm (zeroed, >= n_loc bits) and misc
+// are shared scratch. A region lists its tokens warp by warp, not in token
+// order: the kept ones are marked in bm and emitted in ascending order.
 template <int MG>
 __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int split, int bb, int g, int kr,
                                                bool paged, const uint2* stage, const uint32_t* cnt, uint32_t* rank,
-                                               uint32_t* misc, int* kept, const float* qs, float* zs, float* mo,
-                                               float* lsum, __nv_bfloat16* vst, int64_t plane) {
+                                               uint32_t* misc, int* kept, uint32_t* bm, int t_beg, int n_tok,
+                                               const float* qs, float* zs, float* mo, float* lsum,
+                                               __nv_bfloat16* vst, int64_t plane) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S_ = p.n_split, P = p.ucache, G = p.group;
   const int c = (int)cnt[split];  // own candidates, all staged (no overflow on this path)
@@ -458,11 +461,18 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
     if (r) atomicAdd(rank + i, r);
   }
   __syncthreads();
-  // 2. the CTA's kept tokens, ascending (its region is in token order)
-  const bool keep = tid < c && rank[tid] < (uint32_t)kr;
+  // 2. the CTA's kept tokens, ascending: marked in bm, emitted word by word
+  for (int i = tid; i < c; i += kWdThreads)
+    if (rank[i] < (uint32_t)kr) {
+      const int t = (int)own[i].y - t_beg;
+      atomicOr(bm + (t >> 5), 1u << (t & 31));
+    }
+  __syncthreads();
+  const int nw = (n_tok + 31) / 32;  // <= kWdThreads (n_loc <= 32 * kWdThreads)
+  const uint32_t word = tid < nw ? bm[tid] : 0u;
   uint32_t n_own = 0u;
-  const uint32_t pos = wd_block_scan(keep ? 1u : 0u, misc, &n_own);
-  if (keep) kept[pos] = (int)own[tid].y;
+  uint32_t pos = wd_block_scan((uint32_t)__popc(word), misc, &n_own);
+  for (uint32_t bits = word; bits; bits &= bits - 1u) kept[pos++] = t_beg + tid * 32 + __ffs(bits) - 1;
   __syncthreads();
   // 3. the attention partial over them
   float* pp = p.cpart + ((int64_t)row * S_ + split) * kCcPartStride;
@@ -849,8 +859,8 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     __syncthreads();
     const bool exact = !overflow && nu >= kr && (int)misc[102] >= kr;
     if (exact) {
-      wd_coop_finish<MG>(p, row, split, bb, g, kr, paged, stage, cnt, hist, misc, kept, qs, zs, mo, lsum, vst,
-                         plane);
+      wd_coop_finish<MG>(p, row, split, bb, g, kr, paged, stage, cnt, hist, misc, kept, bm, t_beg, n_tok, qs, zs,
+                         mo, lsum, vst, plane);
       return;
     }
     // the last CTA resolves over every key as in the single-resolver plan;
