@@ -425,40 +425,39 @@ __device__ void wd_select(ForSrc&& for_src, SrcAt&& src_at, int n_src, int n_kee
 // union (key descending, token ascending), attend over the ones ranked below
 // kr, write the partial (and the kept list), and let the row's last CTA
 // merge the partials in CTA order. stage holds the union ([S][P], counts in
-// cnt[0, S)); rank (>= P words), kept, bm (zeroed, >= n_loc bits) and misc
-// are shared scratch. A region lists its tokens warp by warp, not in token
+// cnt[0, S)); misc[104..106] the boundary bin, the entries above it and the
+// number of its entries, which are listed in list; rank (>= P words), kept,
+// bm (zeroed, >= n_loc bits) and misc are shared scratch. A region lists its tokens warp by warp, not in token
 // order: the kept ones are marked in bm and emitted in ascending order.
 template <int MG>
 __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int split, int bb, int g, int kr,
                                                bool paged, const uint2* stage, const uint32_t* cnt, uint32_t* rank,
-                                               uint32_t* misc, int* kept, uint32_t* bm, int t_beg, int n_tok,
+                                               const uint2* list, uint32_t* misc, int* kept, uint32_t* bm, int t_beg,
+                                               int n_tok,
                                                const float* qs, float* zs, float* mo, float* lsum,
                                                __nv_bfloat16* vst, int64_t plane) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S_ = p.n_split, P = p.ucache, G = p.group;
   const int c = (int)cnt[split];  // own candidates, all staged (no overflow on this path)
   const uint2* own = stage + split * P;
-  // 1. ranks; the union is cut into Q slices per own entry, the lanes of a
-  // warp share a slice (broadcast reads)
-  for (int i = tid; i < c; i += kWdThreads) rank[i] = 0u;
-  __syncthreads();
-  const int Q = c > 0 ? max(1, kWdThreads / c) : 1;
-  const int nslot = S_ * P;
-  const int per = (nslot + Q - 1) / Q;
-  for (int item = tid; item < c * Q; item += kWdThreads) {
-    const int i = item % c, q = item / c;
+  (void)S_;
+  // 1. classification against the union's bin counts: hist holds, for
+  // every 12-bit bin b, the union entries in bins >= b; bin B* (suffix count
+  // >= kr > the next one's) is the boundary, its entries are listed in `list`
+  // (n_list of them) and ranked exactly (key descending, token ascending)
+  const uint32_t Bs = misc[104], above = misc[105];
+  const int n_list = (int)misc[106];
+  for (int i = tid; i < c; i += kWdThreads) {
     const uint2 e = own[i];
-    const uint64_t ve = ((uint64_t)e.x << 32) | (uint32_t)(~e.y);
-    const int f0 = q * per, f1 = min(nslot, f0 + per);
-    uint32_t r = 0u;
-    for (int sr = f0 / P; sr * P < f1; ++sr) {  // the valid part of each region in the slice
-      const int j0 = max(f0, sr * P), j1 = min(f1, sr * P + (int)cnt[sr]);
-      for (int f = j0; f < j1; ++f) {
-        const uint2 u = stage[f];
-        r += (((uint64_t)u.x << 32) | (uint32_t)(~u.y)) > ve ? 1u : 0u;
-      }
+    const uint32_t b = e.x >> 20;
+    bool keep = b > Bs;
+    if (b == Bs) {
+      const uint64_t ve = ((uint64_t)e.x << 32) | (uint32_t)(~e.y);
+      uint32_t r = above;
+      for (int j = 0; j < n_list; ++j) r += (((uint64_t)list[j].x << 32) | (uint32_t)(~list[j].y)) > ve ? 1u : 0u;
+      keep = r < (uint32_t)kr;
     }
-    if (r) atomicAdd(rank + i, r);
+    rank[i] = keep ? 0u : 0xFFFFFFFFu;
   }
   __syncthreads();
   // 2. the CTA's kept tokens, ascending: marked in bm, emitted word by word
@@ -490,18 +489,26 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
   if (!misc[103]) return;
   __threadfence();
   const float* rp = p.cpart + (int64_t)row * S_ * kCcPartStride;
-  float* w = mo;  // [S][8] weights, then [8] denominators
+  float* w = mo;                // [S][8] maxima, then weights
+  float* lw = mo + S_ * 8;      // [S][8] sums
+  float* den = lw + S_ * 8;     // [8]
+  for (int it = tid; it < S_ * G; it += kWdThreads) {  // every partial's (m, l) at once
+    const int sr = it / G, h = it % G;
+    w[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + h);
+    lw[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + 16 + h);
+  }
+  __syncthreads();
   if (tid < G) {
     float M = -INFINITY;
-    for (int sr = 0; sr < S_; ++sr) M = fmaxf(M, __ldcg(rp + sr * kCcPartStride + tid));
-    float den = 0.0f;
+    for (int sr = 0; sr < S_; ++sr) M = fmaxf(M, w[sr * 8 + tid]);
+    float dn = 0.0f;
     for (int sr = 0; sr < S_; ++sr) {
-      const float ms = __ldcg(rp + sr * kCcPartStride + tid);
+      const float ms = w[sr * 8 + tid];
       const float ws = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
       w[sr * 8 + tid] = ws;
-      den += ws * __ldcg(rp + sr * kCcPartStride + 16 + tid);
+      dn += ws * lw[sr * 8 + tid];
     }
-    w[S_ * 8 + tid] = den;
+    den[tid] = dn;
   }
   int* offs = reinterpret_cast<int*>(zs);  // [S + 1] prefix sums of the CTAs' kept counts
   if (warp == kWdWarps - 1) {
@@ -527,9 +534,16 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
   for (int e = tid; e < G * kD; e += kWdThreads) {
     const int h = e / kD;
     float num = 0.0f;
-    for (int sr = 0; sr < S_; ++sr) num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
-    const float den = w[S_ * 8 + h];
-    out[e] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
+    int sr = 0;
+    for (; sr + 8 <= S_; sr += 8) {  // eight loads in flight, added in split order
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(rp + (sr + u) * kCcPartStride + 32 + e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) num = __fmaf_rn(w[(sr + u) * 8 + h], v[u], num);
+    }
+    for (; sr < S_; ++sr) num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
+    out[e] = __float2bfloat16_rn(den[h] > 0.0f ? num / den[h] : 0.0f);
   }
   if (p.idx_out) {
     int32_t* io = p.idx_out + (int64_t)row * p.n_keep;
@@ -735,7 +749,23 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       const uint32_t key = i < n_tok ? keys[i] : 0u;
       const bool q = i < n_tok && (key >> 20) >= b_loc;
       const unsigned m = __ballot_sync(0xFFFFFFFFu, q);
-      if (q) region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
+      if (q) {
+        region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
+        if (p.coop) {  // this CTA attends over its kept candidates later: their K and V rows to L2
+          const int tt = t_beg + i;
+          int64_t kr_ = -1;
+          if (!paged) {
+            kr_ = (int64_t)row * p.max_len + tt;
+          } else {
+            const int pg = s_pg[(tt >> p.pm.log2bs) - pg0];
+            if (pg >= 0) kr_ = ((pg * p.pm.n_kv_heads + g) << p.pm.log2bs) | (tt & ((1 << p.pm.log2bs) - 1));
+          }
+          if (kr_ >= 0) {
+            prefetch_l2(p.k + kr_ * kD, kD * 2);
+            prefetch_l2(p.v + kr_ * kD, kD * 2);
+          }
+        }
+      }
       pos += __popc(m);
     }
     if (tid == 0) region[0] = make_uint2(misc[96], b_loc);
@@ -850,17 +880,47 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
   int* kept = reinterpret_cast<int*>(smem + Lo.kept);
   if (p.coop) {
+    // the union's bin counts, then suffix counts (entries in bins >= b)
+    for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
+    __syncthreads();
+    {
+      uint32_t loc[8], run = 0u;
+#pragma unroll
+      for (int u = 7; u >= 0; --u) {
+        run += hist[tid * 8 + u];
+        loc[u] = run;
+      }
+      // plus the entries in the bins of later threads
+      uint32_t tot = 0u;
+      const uint32_t earlier = wd_block_scan(run, misc, &tot);
+      const uint32_t later = tot - earlier - run;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) hist[tid * 8 + u] = loc[u] + later;
+    }
+    __syncthreads();
+    // the boundary bin B*: suffix count >= kr > the next bin's
+    for (int b = tid; b < 4096; b += kWdThreads) {
+      const uint32_t here = hist[b], next = b < 4095 ? hist[b + 1] : 0u;
+      if (here >= (uint32_t)kr && next < (uint32_t)kr) {
+        misc[104] = (uint32_t)b;
+        misc[105] = next;
+      }
+    }
+    if (tid == 0) misc[106] = 0u;
+    __syncthreads();
     // exact when at least kr union entries lie at or above the highest
     // boundary bin: every unpublished token is then below the kr-th entry
-    uint32_t hi = 0u;
-    for_union([&](const uint2& e) { hi += (e.x >> 20) >= b_max ? 1u : 0u; });
-    hi = __reduce_add_sync(0xFFFFFFFFu, hi);
-    if (lane == 0 && hi) atomicAdd(misc + 102, hi);
-    __syncthreads();
-    const bool exact = !overflow && nu >= kr && (int)misc[102] >= kr;
+    const bool exact = !overflow && nu >= kr && hist[b_max] >= (uint32_t)kr &&
+                       hist[misc[104]] - misc[105] <= (uint32_t)kWdTieCap;
     if (exact) {
-      wd_coop_finish<MG>(p, row, split, bb, g, kr, paged, stage, cnt, hist, misc, kept, bm, t_beg, n_tok, qs, zs,
-                         mo, lsum, vst, plane);
+      uint2* list = ties;  // the boundary bin's entries
+      const uint32_t Bs = misc[104];
+      for_union([&](const uint2& e) {
+        if ((e.x >> 20) == Bs) list[atomicAdd(misc + 106, 1u)] = e;
+      });
+      __syncthreads();
+      wd_coop_finish<MG>(p, row, split, bb, g, kr, paged, stage, cnt, hist, list, misc, kept, bm, t_beg, n_tok, qs,
+                         zs, mo, lsum, vst, plane);
       return;
     }
     // the last CTA resolves over every key as in the single-resolver plan;
@@ -870,6 +930,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       if (tid == 0) atomicAdd(p.cticket + row, 1u);
       return;
     }
+    for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;  // the plain histogram again
     __syncthreads();
   }
   for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
