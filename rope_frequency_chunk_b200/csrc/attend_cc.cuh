@@ -572,4 +572,102 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
   }
 }
 
+
+// A few kept rows (tens) for one CTA of NW warps, written as a split partial
+// (m at part[h], l at part[16 + h], unnormalised o at part[32 + h * 128 + d]):
+// warp w takes rows w, w + NW, ... whole (lane: 4 dims of K and V), forms
+// each head's logit with a warp all-reduce and keeps an online softmax state
+// per head in registers; the warps' states are merged in warp order through
+// shared memory. Only warps with rows issue loads. qs: scaled rotated
+// queries [MG][128]; ml: [NW][2][MG] floats; mo: [NW][MG][128] floats.
+template <int MG, int NW, typename Tok>
+__device__ __forceinline__ void cc_rows_partial(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
+                                                int G, const float* qs, float* ml, float* mo, float* part) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float q[MG][4], m[MG], l[MG], o[MG][4];
+#pragma unroll
+  for (int h = 0; h < MG; ++h) {
+    const float4 q4 = *reinterpret_cast<const float4*>(qs + h * kD + 4 * lane);
+    q[h][0] = q4.x;
+    q[h][1] = q4.y;
+    q[h][2] = q4.z;
+    q[h][3] = q4.w;
+    m[h] = -INFINITY;
+    l[h] = 0.0f;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) o[h][d] = 0.0f;
+  }
+  for (int j0 = warp; j0 < n; j0 += 2 * NW) {  // two rows of the warp in flight
+    const int j1 = j0 + NW;
+    const int t0 = token(j0), t1 = j1 < n ? token(j1) : -1;
+    uint2 k0 = make_uint2(0u, 0u), v0 = k0, k1 = k0, v1 = k0;
+    if (t0 >= 0) {
+      k0 = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t0 * kD) + lane);
+      v0 = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t0 * kD) + lane);
+    }
+    if (t1 >= 0) {
+      k1 = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t1 * kD) + lane);
+      v1 = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t1 * kD) + lane);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if ((r == 0 ? t0 : t1) < 0) continue;  // warp-uniform
+      float kf[4], vf[4];
+      cc_bf16x4(r == 0 ? k0 : k1, kf);
+      cc_bf16x4(r == 0 ? v0 : v1, vf);
+      float z[MG];
+#pragma unroll
+      for (int h = 0; h < MG; ++h)
+        z[h] = __fmaf_rn(q[h][3], kf[3], __fmaf_rn(q[h][2], kf[2], __fmaf_rn(q[h][1], kf[1], __fmul_rn(q[h][0], kf[0]))));
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int h = 0; h < MG; ++h) z[h] = __fadd_rn(z[h], __shfl_xor_sync(0xFFFFFFFFu, z[h], off));
+#pragma unroll
+      for (int h = 0; h < MG; ++h) {
+        const float mn = fmaxf(m[h], z[h]);
+        const float a = exp2f(m[h] - mn), b = exp2f(z[h] - mn);
+        l[h] = __fmaf_rn(l[h], a, b);
+#pragma unroll
+        for (int d = 0; d < 4; ++d) o[h][d] = __fmaf_rn(o[h][d], a, b * vf[d]);
+        m[h] = mn;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < MG; ++h)
+    *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+  if (lane < MG) {
+    float mv = m[0], lv = l[0];
+#pragma unroll
+    for (int h = 1; h < MG; ++h)
+      if (lane == h) {
+        mv = m[h];
+        lv = l[h];
+      }
+    ml[(warp * 2) * MG + lane] = mv;
+    ml[(warp * 2 + 1) * MG + lane] = lv;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * kD; e += NW * 32) {
+    const int h = e / kD, d = e % kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * 2) * MG + h]);
+    float L = 0.0f, O = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float mw = ml[(w * 2) * MG + h];
+      const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+      L = __fmaf_rn(f, ml[(w * 2 + 1) * MG + h], L);
+      O = __fmaf_rn(f, mo[(w * MG + h) * kD + d], O);
+    }
+    part[32 + e] = O;
+    if (d == 0) {
+      part[h] = M;
+      part[16 + h] = L;
+    }
+  }
+}
+
 }  // namespace fasa

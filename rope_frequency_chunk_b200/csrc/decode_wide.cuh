@@ -475,9 +475,9 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
   __syncthreads();
   // 3. the attention partial over them
   float* pp = p.cpart + ((int64_t)row * S_ + split) * kCcPartStride;
-  cc_block_attend<MG, kWdWarps, true>(
+  cc_rows_partial<MG, kWdWarps>(
       p.k + plane, p.v + plane, [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
-      (int)n_own, G, qs, zs, mo, lsum, vst, nullptr, pp);
+      (int)n_own, G, qs, zs, mo, pp);
   if (tid == 0) pp[kCoopCnt] = __int_as_float((int)n_own);
   if (p.idx_out)
     for (int j = tid; j < (int)n_own; j += kWdThreads) pp[kCoopList + j] = __int_as_float(kept[j]);
