@@ -492,7 +492,15 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
   float* w = mo;                // [S][8] maxima, then weights
   float* lw = mo + S_ * 8;      // [S][8] sums
   float* den = lw + S_ * 8;     // [8]
-  for (int it = tid; it < S_ * G; it += kWdThreads) {  // every partial's (m, l) at once
+  // every load of the merge in one round trip: the (m, l) pairs, and for up
+  // to kCoopHold splits the thread's output element of each partial
+  constexpr int kCoopHold = 24;
+  const int e0 = tid;  // output element of this thread (G * 128 <= 2 * kWdThreads)
+  float hv[kCoopHold];
+#pragma unroll
+  for (int u = 0; u < kCoopHold; ++u)
+    hv[u] = (u < S_ && e0 < G * kD) ? __ldcg(rp + u * kCcPartStride + 32 + e0) : 0.0f;
+  for (int it = tid; it < S_ * G; it += kWdThreads) {
     const int sr = it / G, h = it % G;
     w[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + h);
     lw[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + 16 + h);
@@ -531,18 +539,18 @@ __device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int
   }
   __syncthreads();
   __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
-  for (int e = tid; e < G * kD; e += kWdThreads) {
+  for (int e = tid; e < G * kD; e += kWdThreads) {  // added in split order
     const int h = e / kD;
     float num = 0.0f;
-    int sr = 0;
-    for (; sr + 8 <= S_; sr += 8) {  // eight loads in flight, added in split order
-      float v[8];
+    if (e == e0) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(rp + (sr + u) * kCcPartStride + 32 + e);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) num = __fmaf_rn(w[(sr + u) * 8 + h], v[u], num);
+      for (int u = 0; u < kCoopHold; ++u)
+        if (u < S_) num = __fmaf_rn(w[u * 8 + h], hv[u], num);
+      for (int sr = kCoopHold; sr < S_; ++sr)
+        num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
+    } else {
+      for (int sr = 0; sr < S_; ++sr) num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
     }
-    for (; sr < S_; ++sr) num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
     out[e] = __float2bfloat16_rn(den[h] > 0.0f ? num / den[h] : 0.0f);
   }
   if (p.idx_out) {
