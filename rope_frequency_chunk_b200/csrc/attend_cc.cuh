@@ -445,15 +445,12 @@ namespace fasa {
 // head h over all n logits (max, exp2, sum; zs becomes the probabilities);
 // (3) each warp adds p * v over its rows for the lane's 4 dims; (4) the warp
 // sums are added in a fixed order and divided by the head's sum.
-// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [16]
-// (sums, then maxima at lsum + 8), vst [16 * NW][128] bf16 (the V rows,
-// staged with cp.async). With PART the state is written unnormalised to
-// part instead (m at part[h], l at part[16 + h], o at part[32 + h * 128 + d],
-// the layout of a split partial) and out is not touched.
-template <int MG, int NW, bool PART = false, typename Tok>
+// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [MG],
+// vst [16 * NW][128] bf16 (the V rows, staged with cp.async).
+template <int MG, int NW, typename Tok>
 __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
                                                 int G, const float* qs, float* zs, float* mo, float* lsum,
-                                                __nv_bfloat16* vst, __nv_bfloat16* out, float* part = nullptr) {
+                                                __nv_bfloat16* vst, __nv_bfloat16* out) {
   constexpr int NG = MG / 4;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int jb = warp * 16;
@@ -518,10 +515,7 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-    if (lane == 0) {
-      lsum[warp] = l;
-      if (PART) lsum[8 + warp] = m;
-    }
+    if (lane == 0) lsum[warp] = l;
   }
   __syncthreads();
   // (3) p * v over the warp's rows
@@ -553,120 +547,13 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
   for (int h = 0; h < MG; ++h)
     *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
   __syncthreads();
-  // (4) warp sums in warp order, divided by the head's sum (or, with PART,
-  // written with the head's maximum and sum)
+  // (4) warp sums in warp order, divided by the head's sum
   for (int e = tid; e < G * kD; e += NW * 32) {
     const int h = e / kD, d = e % kD;
     float acc = 0.0f;
     for (int w = 0; w < NW; ++w) acc += mo[(w * MG + h) * kD + d];
     const float l = lsum[h];
-    if (PART) {
-      part[32 + e] = acc;
-      if (d == 0) {
-        part[h] = lsum[8 + h];
-        part[16 + h] = l;
-      }
-    } else {
-      out[e] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
-    }
-  }
-}
-
-
-// A few kept rows (tens) for one CTA of NW warps, written as a split partial
-// (m at part[h], l at part[16 + h], unnormalised o at part[32 + h * 128 + d]):
-// warp w takes rows w, w + NW, ... whole (lane: 4 dims of K and V), forms
-// each head's logit with a warp all-reduce and keeps an online softmax state
-// per head in registers; the warps' states are merged in warp order through
-// shared memory. Only warps with rows issue loads. qs: scaled rotated
-// queries [MG][128]; ml: [NW][2][MG] floats; mo: [NW][MG][128] floats.
-template <int MG, int NW, typename Tok>
-__device__ __forceinline__ void cc_rows_partial(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
-                                                int G, const float* qs, float* ml, float* mo, float* part) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float q[MG][4], m[MG], l[MG], o[MG][4];
-#pragma unroll
-  for (int h = 0; h < MG; ++h) {
-    const float4 q4 = *reinterpret_cast<const float4*>(qs + h * kD + 4 * lane);
-    q[h][0] = q4.x;
-    q[h][1] = q4.y;
-    q[h][2] = q4.z;
-    q[h][3] = q4.w;
-    m[h] = -INFINITY;
-    l[h] = 0.0f;
-#pragma unroll
-    for (int d = 0; d < 4; ++d) o[h][d] = 0.0f;
-  }
-  for (int j0 = warp; j0 < n; j0 += 2 * NW) {  // two rows of the warp in flight
-    const int j1 = j0 + NW;
-    const int t0 = token(j0), t1 = j1 < n ? token(j1) : -1;
-    uint2 k0 = make_uint2(0u, 0u), v0 = k0, k1 = k0, v1 = k0;
-    if (t0 >= 0) {
-      k0 = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t0 * kD) + lane);
-      v0 = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t0 * kD) + lane);
-    }
-    if (t1 >= 0) {
-      k1 = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)t1 * kD) + lane);
-      v1 = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)t1 * kD) + lane);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      if ((r == 0 ? t0 : t1) < 0) continue;  // warp-uniform
-      float kf[4], vf[4];
-      cc_bf16x4(r == 0 ? k0 : k1, kf);
-      cc_bf16x4(r == 0 ? v0 : v1, vf);
-      float z[MG];
-#pragma unroll
-      for (int h = 0; h < MG; ++h)
-        z[h] = __fmaf_rn(q[h][3], kf[3], __fmaf_rn(q[h][2], kf[2], __fmaf_rn(q[h][1], kf[1], __fmul_rn(q[h][0], kf[0]))));
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1)
-#pragma unroll
-        for (int h = 0; h < MG; ++h) z[h] = __fadd_rn(z[h], __shfl_xor_sync(0xFFFFFFFFu, z[h], off));
-#pragma unroll
-      for (int h = 0; h < MG; ++h) {
-        const float mn = fmaxf(m[h], z[h]);
-        const float a = exp2f(m[h] - mn), b = exp2f(z[h] - mn);
-        l[h] = __fmaf_rn(l[h], a, b);
-#pragma unroll
-        for (int d = 0; d < 4; ++d) o[h][d] = __fmaf_rn(o[h][d], a, b * vf[d]);
-        m[h] = mn;
-      }
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < MG; ++h)
-    *reinterpret_cast<float4*>(mo + (warp * MG + h) * kD + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
-  if (lane < MG) {
-    float mv = m[0], lv = l[0];
-#pragma unroll
-    for (int h = 1; h < MG; ++h)
-      if (lane == h) {
-        mv = m[h];
-        lv = l[h];
-      }
-    ml[(warp * 2) * MG + lane] = mv;
-    ml[(warp * 2 + 1) * MG + lane] = lv;
-  }
-  __syncthreads();
-  for (int e = tid; e < G * kD; e += NW * 32) {
-    const int h = e / kD, d = e % kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * 2) * MG + h]);
-    float L = 0.0f, O = 0.0f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float mw = ml[(w * 2) * MG + h];
-      const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
-      L = __fmaf_rn(f, ml[(w * 2 + 1) * MG + h], L);
-      O = __fmaf_rn(f, mo[(w * MG + h) * kD + d], O);
-    }
-    part[32 + e] = O;
-    if (d == 0) {
-      part[h] = M;
-      part[16 + h] = L;
-    }
+    out[e] = __float2bfloat16_rn(l > 0.0f ? acc / l : 0.0f);
   }
 }
 

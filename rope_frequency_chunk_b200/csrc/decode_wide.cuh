@@ -93,14 +93,6 @@ struct WideParams {
   int32_t* row_keep;       // [rows] each row's k_eff, for the attention launch (varlen), or null
   int32_t q_prerot;        // varlen: 1 if the queries are already rotated
   PageMap pm;              // paged pools (pm.table set), else [rows][max_len] planes
-  // cooperative resolution (direct plan, every CTA of the launch resident at
-  // once): the row's CTAs wait for each other, each ranks its own candidates
-  // against the published union and attends over its kept ones; cpart
-  // [rows][n_split][kCcPartStride] holds their partials, cticket [rows] the
-  // second ticket (zero between calls)
-  int32_t coop;
-  float* cpart;
-  uint32_t* cticket;
   // multi-query decode: n_q query tokens per sequence, q [B][n_q][Hq][128],
   // token j at position q_pos0 + j (angles from theta_i in cosv), or 1
   int32_t n_q;
@@ -132,40 +124,6 @@ __device__ __forceinline__ int2 wd_row_shape(const WideParams& p, int row) {
 }
 
 __host__ __device__ constexpr int wd_al(int x, int a) { return (x + a - 1) / a * a; }
-
-// Bounded wait until *ctr >= target (acquire). Gives up after ~1 s, records
-// FASA_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool wd_wait_ge(const unsigned long long* ctr, unsigned long long target) {
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
-    if (v >= target) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      flag_status(FASA_ERR_TIMEOUT);
-      return false;
-    }
-    __nanosleep(20);
-  }
-}
-__device__ __forceinline__ bool wd_wait_ge32(const uint32_t* ctr, uint32_t target) {
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    if (v >= target) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      flag_status(FASA_ERR_TIMEOUT);
-      return false;
-    }
-    __nanosleep(20);
-  }
-}
-
-// Slots of a cooperative partial past the attention state (G <= 8 heads):
-// the CTA's kept count, then its kept tokens in ascending order.
-constexpr int kCoopCnt = 32 + 8 * kD;
-constexpr int kCoopList = kCoopCnt + 1;
 
 // Shared-memory layout. r1 is reused: the CTA's keys (steps 1-3); then, in
 // the resolving CTA, the bitmap, boundary-bin entries, radix scratch and the
@@ -420,155 +378,6 @@ __device__ void wd_select(ForSrc&& for_src, SrcAt&& src_at, int n_src, int n_kee
   *B_out = B;
 }
 
-// Cooperative finish of one CTA of a row whose published union is exact
-// (every kept token is in it): rank the CTA's own candidates against the
-// union (key descending, token ascending), attend over the ones ranked below
-// kr, write the partial (and the kept list), and let the row's last CTA
-// merge the partials in CTA order. stage holds the union ([S][P], counts in
-// cnt[0, S)); misc[104..106] the boundary bin, the entries above it and the
-// number of its entries, which are listed in list; rank (>= P words), kept,
-// bm (zeroed, >= n_loc bits) and misc are shared scratch. A region lists its tokens warp by warp, not in token
-// order: the kept ones are marked in bm and emitted in ascending order.
-template <int MG>
-__device__ __forceinline__ void wd_coop_finish(const WideParams& p, int row, int split, int bb, int g, int kr,
-                                               bool paged, const uint2* stage, const uint32_t* cnt, uint32_t* rank,
-                                               const uint2* list, uint32_t* misc, int* kept, uint32_t* bm, int t_beg,
-                                               int n_tok,
-                                               const float* qs, float* zs, float* mo, float* lsum,
-                                               __nv_bfloat16* vst, int64_t plane) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int S_ = p.n_split, P = p.ucache, G = p.group;
-  const int c = (int)cnt[split];  // own candidates, all staged (no overflow on this path)
-  const uint2* own = stage + split * P;
-  (void)S_;
-  // 1. classification against the union's bin counts: hist holds, for
-  // every 12-bit bin b, the union entries in bins >= b; bin B* (suffix count
-  // >= kr > the next one's) is the boundary, its entries are listed in `list`
-  // (n_list of them) and ranked exactly (key descending, token ascending)
-  const uint32_t Bs = misc[104], above = misc[105];
-  const int n_list = (int)misc[106];
-  for (int i = tid; i < c; i += kWdThreads) {
-    const uint2 e = own[i];
-    const uint32_t b = e.x >> 20;
-    bool keep = b > Bs;
-    if (b == Bs) {
-      const uint64_t ve = ((uint64_t)e.x << 32) | (uint32_t)(~e.y);
-      uint32_t r = above;
-      for (int j = 0; j < n_list; ++j) r += (((uint64_t)list[j].x << 32) | (uint32_t)(~list[j].y)) > ve ? 1u : 0u;
-      keep = r < (uint32_t)kr;
-    }
-    rank[i] = keep ? 0u : 0xFFFFFFFFu;
-  }
-  __syncthreads();
-  // 2. the CTA's kept tokens, ascending: marked in bm, emitted word by word
-  for (int i = tid; i < c; i += kWdThreads)
-    if (rank[i] < (uint32_t)kr) {
-      const int t = (int)own[i].y - t_beg;
-      atomicOr(bm + (t >> 5), 1u << (t & 31));
-    }
-  __syncthreads();
-  const int nw = (n_tok + 31) / 32;  // <= kWdThreads (n_loc <= 32 * kWdThreads)
-  const uint32_t word = tid < nw ? bm[tid] : 0u;
-  uint32_t n_own = 0u;
-  uint32_t pos = wd_block_scan((uint32_t)__popc(word), misc, &n_own);
-  for (uint32_t bits = word; bits; bits &= bits - 1u) kept[pos++] = t_beg + tid * 32 + __ffs(bits) - 1;
-  __syncthreads();
-  // 3. the attention partial over them
-  float* pp = p.cpart + ((int64_t)row * S_ + split) * kCcPartStride;
-  cc_rows_partial<MG, kWdWarps>(
-      p.k + plane, p.v + plane, [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
-      (int)n_own, G, qs, zs, mo, pp);
-  if (tid == 0) pp[kCoopCnt] = __int_as_float((int)n_own);
-  if (p.idx_out)
-    for (int j = tid; j < (int)n_own; j += kWdThreads) pp[kCoopList + j] = __int_as_float(kept[j]);
-  // 4. second ticket; the last CTA merges
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) misc[103] = atomicAdd(p.cticket + row, 1u) == (uint32_t)S_ - 1u ? 1u : 0u;
-  __syncthreads();
-  if (!misc[103]) return;
-  __threadfence();
-  const float* rp = p.cpart + (int64_t)row * S_ * kCcPartStride;
-  float* w = mo;                // [S][8] maxima, then weights
-  float* lw = mo + S_ * 8;      // [S][8] sums
-  float* den = lw + S_ * 8;     // [8]
-  // every load of the merge in one round trip: the (m, l) pairs, and for up
-  // to kCoopHold splits the thread's output element of each partial
-  constexpr int kCoopHold = 24;
-  const int e0 = tid;  // output element of this thread (G * 128 <= 2 * kWdThreads)
-  float hv[kCoopHold];
-#pragma unroll
-  for (int u = 0; u < kCoopHold; ++u)
-    hv[u] = (u < S_ && e0 < G * kD) ? __ldcg(rp + u * kCcPartStride + 32 + e0) : 0.0f;
-  for (int it = tid; it < S_ * G; it += kWdThreads) {
-    const int sr = it / G, h = it % G;
-    w[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + h);
-    lw[sr * 8 + h] = __ldcg(rp + sr * kCcPartStride + 16 + h);
-  }
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int sr = 0; sr < S_; ++sr) M = fmaxf(M, w[sr * 8 + tid]);
-    float dn = 0.0f;
-    for (int sr = 0; sr < S_; ++sr) {
-      const float ms = w[sr * 8 + tid];
-      const float ws = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
-      w[sr * 8 + tid] = ws;
-      dn += ws * lw[sr * 8 + tid];
-    }
-    den[tid] = dn;
-  }
-  int* offs = reinterpret_cast<int*>(zs);  // [S + 1] prefix sums of the CTAs' kept counts
-  if (warp == kWdWarps - 1) {
-    uint32_t run = 0u;
-    for (int s0 = 0; s0 < S_; s0 += 32) {
-      const uint32_t cn = s0 + lane < S_ ? (uint32_t)__float_as_int(__ldcg(rp + (s0 + lane) * kCcPartStride + kCoopCnt)) : 0u;
-      uint32_t incl = cn;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += x;
-      }
-      if (s0 + lane < S_) offs[s0 + lane + 1] = (int)(run + incl);
-      run += __shfl_sync(0xFFFFFFFFu, incl, 31);
-    }
-    if (lane == 0) {
-      offs[0] = 0;
-      if (run != (uint32_t)kr) flag_status(FASA_ERR_WORKSPACE);
-    }
-  }
-  __syncthreads();
-  __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
-  for (int e = tid; e < G * kD; e += kWdThreads) {  // added in split order
-    const int h = e / kD;
-    float num = 0.0f;
-    if (e == e0) {
-#pragma unroll
-      for (int u = 0; u < kCoopHold; ++u)
-        if (u < S_) num = __fmaf_rn(w[u * 8 + h], hv[u], num);
-      for (int sr = kCoopHold; sr < S_; ++sr)
-        num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
-    } else {
-      for (int sr = 0; sr < S_; ++sr) num = __fmaf_rn(w[sr * 8 + h], __ldcg(rp + sr * kCcPartStride + 32 + e), num);
-    }
-    out[e] = __float2bfloat16_rn(den[h] > 0.0f ? num / den[h] : 0.0f);
-  }
-  if (p.idx_out) {
-    int32_t* io = p.idx_out + (int64_t)row * p.n_keep;
-    for (int sr = warp; sr < S_; sr += kWdWarps) {
-      const int o0 = offs[sr], n = offs[sr + 1] - o0;
-      for (int j = lane; j < n; j += 32)
-        if (o0 + j < kr) io[o0 + j] = __float_as_int(__ldcg(rp + sr * kCcPartStride + kCoopList + j));
-    }
-    for (int j = kr + tid; j < p.n_keep; j += kWdThreads) io[j] = -1;  // a shorter row's padding
-  }
-  if (tid == 0) {  // every CTA of the row is past both tickets: ready for the next call
-    p.sem[row] = 0ull;
-    p.cticket[row] = 0u;
-  }
-  if (p.row_keep && tid == 0) p.row_keep[row] = kr;
-}
-
 template <int LPT, int MG>
 __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WideParams p) {
   using S = TipShape<__nv_bfloat16, LPT>;
@@ -757,23 +566,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       const uint32_t key = i < n_tok ? keys[i] : 0u;
       const bool q = i < n_tok && (key >> 20) >= b_loc;
       const unsigned m = __ballot_sync(0xFFFFFFFFu, q);
-      if (q) {
-        region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
-        if (p.coop) {  // this CTA attends over its kept candidates later: their K and V rows to L2
-          const int tt = t_beg + i;
-          int64_t kr_ = -1;
-          if (!paged) {
-            kr_ = (int64_t)row * p.max_len + tt;
-          } else {
-            const int pg = s_pg[(tt >> p.pm.log2bs) - pg0];
-            if (pg >= 0) kr_ = ((pg * p.pm.n_kv_heads + g) << p.pm.log2bs) | (tt & ((1 << p.pm.log2bs) - 1));
-          }
-          if (kr_ >= 0) {
-            prefetch_l2(p.k + kr_ * kD, kD * 2);
-            prefetch_l2(p.v + kr_ * kD, kD * 2);
-          }
-        }
-      }
+      if (q) region[pos + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)(t_beg + i));
       pos += __popc(m);
     }
     if (tid == 0) region[0] = make_uint2(misc[96], b_loc);
@@ -789,18 +582,11 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     misc[98] = (old == (unsigned long long)p.n_split - 1) ? 1u : 0u;
   }
   __syncthreads();
-  const bool last = misc[98] != 0u;
-  if (!p.coop && !last) return;
-  if (p.coop) {  // row barrier: every CTA of the row has published (bounded wait)
-    if (tid == 0) misc[101] = (last || wd_wait_ge(p.sem + row, (unsigned long long)p.n_split)) ? 1u : 0u;
-    __syncthreads();
-    if (!misc[101]) return;
-  }
+  if (!misc[98]) return;
 
-  // 4. exact selection over the published union: by the row's last CTA, or
-  // (cooperative) by every CTA for its own candidates. One batched read
-  // brings every region's count and first P entries into shared memory
-  // (entries beyond P, rare, are read from global memory).
+  // 4. the row's last CTA: exact selection over the published union. One
+  // batched read brings every region's count and first P entries into
+  // shared memory (entries beyond P, rare, are read from global memory).
   __threadfence();
   const int S_ = p.n_split, P = p.ucache;  // P: a power of two
   uint2* stage = reinterpret_cast<uint2*>(smem + Lo.ucache);  // [S][P]
@@ -810,7 +596,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   uint32_t* rscr = reinterpret_cast<uint32_t*>(smem + Lo.rscr);
   const int words = (Lr + 31) / 32;
   const uint2* rows0 = p.cand + (int64_t)row * p.n_split * rstride;
-  if (tid == 0 && !p.coop) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
+  if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
   {  // slots [0, S): the regions' counts; then entry j < P of region s at S + s*P + j
     const int nslots = S_ + (S_ << p.ushift);
     for (int base = 0; base < nslots; base += kWdThreads * kWdUnionUnroll) {
@@ -835,10 +621,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
   for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
-  if (tid == 0) {
-    misc[100] = 0u;
-    misc[102] = 0u;
-  }
+  if (tid == 0) misc[100] = 0u;
   __syncthreads();
   if (warp == 0) {  // prefix sums of the counts (S <= 32 per pass of the warp)
     uint32_t run = 0u;
@@ -880,67 +663,6 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
     const int j = i - (int)pre[lo];
     return j < P ? stage[lo * P + j] : __ldcg(rows0 + lo * rstride + 1 + j);
   };
-  const float* qs = reinterpret_cast<const float*>(smem + Lo.qs);
-  float* zs = reinterpret_cast<float*>(smem + Lo.zs);
-  float* mo = reinterpret_cast<float*>(smem + Lo.ring);
-  float* lsum = mo + kWdWarps * MG * kD;
-  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
-  const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
-  int* kept = reinterpret_cast<int*>(smem + Lo.kept);
-  if (p.coop) {
-    // the union's bin counts, then suffix counts (entries in bins >= b)
-    for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
-    __syncthreads();
-    {
-      uint32_t loc[8], run = 0u;
-#pragma unroll
-      for (int u = 7; u >= 0; --u) {
-        run += hist[tid * 8 + u];
-        loc[u] = run;
-      }
-      // plus the entries in the bins of later threads
-      uint32_t tot = 0u;
-      const uint32_t earlier = wd_block_scan(run, misc, &tot);
-      const uint32_t later = tot - earlier - run;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) hist[tid * 8 + u] = loc[u] + later;
-    }
-    __syncthreads();
-    // the boundary bin B*: suffix count >= kr > the next bin's
-    for (int b = tid; b < 4096; b += kWdThreads) {
-      const uint32_t here = hist[b], next = b < 4095 ? hist[b + 1] : 0u;
-      if (here >= (uint32_t)kr && next < (uint32_t)kr) {
-        misc[104] = (uint32_t)b;
-        misc[105] = next;
-      }
-    }
-    if (tid == 0) misc[106] = 0u;
-    __syncthreads();
-    // exact when at least kr union entries lie at or above the highest
-    // boundary bin: every unpublished token is then below the kr-th entry
-    const bool exact = !overflow && nu >= kr && hist[b_max] >= (uint32_t)kr &&
-                       hist[misc[104]] - misc[105] <= (uint32_t)kWdTieCap;
-    if (exact) {
-      uint2* list = ties;  // the boundary bin's entries
-      const uint32_t Bs = misc[104];
-      for_union([&](const uint2& e) {
-        if ((e.x >> 20) == Bs) list[atomicAdd(misc + 106, 1u)] = e;
-      });
-      __syncthreads();
-      wd_coop_finish<MG>(p, row, split, bb, g, kr, paged, stage, cnt, hist, list, misc, kept, bm, t_beg, n_tok, qs,
-                         zs, mo, lsum, vst, plane);
-      return;
-    }
-    // the last CTA resolves over every key as in the single-resolver plan;
-    // the others leave (the last resets the counters once all have arrived)
-    if (!last) {
-      __syncthreads();
-      if (tid == 0) atomicAdd(p.cticket + row, 1u);
-      return;
-    }
-    for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;  // the plain histogram again
-    __syncthreads();
-  }
   for_union([&](const uint2& e) { atomicAdd(hist + (e.x >> 20), 1u); });
   __syncthreads();
   const int n_keep = min(kr, nu);
@@ -975,6 +697,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
 
   // ascending emission from the bitmap
+  int* kept = reinterpret_cast<int*>(smem + Lo.kept);
   const int wpt = (words + kWdThreads - 1) / kWdThreads;
   const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
   uint32_t nbits = 0u;
@@ -1005,14 +728,14 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   if (p.row_keep && tid == 0) p.row_keep[row] = kr;
   __syncthreads();
   const int n_att = min((int)total, kr);
-  if (p.coop && tid == 0) {  // every other CTA of the row has left the barrier: reset the counters
-    if (wd_wait_ge32(p.cticket + row, (uint32_t)p.n_split - 1u)) {
-      p.sem[row] = 0ull;
-      p.cticket[row] = 0u;
-    }
-  }
   if (!p.direct) return;  // the split-K attention launch follows
   // the group's attention over the kept rows (at most 16 per warp)
+  const float* qs = reinterpret_cast<const float*>(smem + Lo.qs);
+  float* zs = reinterpret_cast<float*>(smem + Lo.zs);
+  float* mo = reinterpret_cast<float*>(smem + Lo.ring);
+  float* lsum = mo + kWdWarps * MG * kD;
+  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
+  const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
   cc_block_attend<MG, kWdWarps>(p.k + plane, p.v + plane,
                                 [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
                                 n_att, G, qs, zs, mo, lsum, vst, p.out + (int64_t)row * G * kD);

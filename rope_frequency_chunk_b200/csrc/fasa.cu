@@ -493,7 +493,7 @@ constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
 struct DecodeWs {
-  size_t sem, att_cnt, scores, keys, rowk, hist, cnt, bitmap, cand, ckey, idx, part, cpart, total;
+  size_t sem, att_cnt, scores, keys, rowk, hist, cnt, bitmap, cand, ckey, idx, part, total;
   int64_t ld;
   int cap, words, splits_max;
 };
@@ -527,10 +527,7 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
   w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
   w.part = al256(w.idx + rows * (size_t)keff * 4);
-  // the cooperative plan's partials: one per CTA of the launch (at most one
-  // per SM, or one per row)
-  w.cpart = al256(w.part + rows * (size_t)w.splits_max * kCcPartStride * 4);
-  w.total = al256(w.cpart + std::max<size_t>(rows, kAssumedMaxSms) * kCcPartStride * 4) + 256;
+  w.total = al256(w.part + rows * (size_t)w.splits_max * kCcPartStride * 4) + 256;
   return w;
 }
 size_t decode_ws(const fasa_cache* c, int32_t len, int32_t k) { return decode_layout(c, len, k).total; }
@@ -779,16 +776,6 @@ fasa_status launch_wide(const fasa_cache* c, int32_t len, const void* q, int32_t
   WideParams p{};
   p.pm = page_map(c, pg);
   p.n_q = 1;
-  // cooperative resolution when the row's CTAs can wait for each other: the
-  // direct plan, every CTA of the launch resident at once (at most one per
-  // SM), and room for their partials
-  {
-    const int64_t ctas = (int64_t)c->batch * c->n_kv_heads * pl.n_split;
-    p.coop = (pl.direct && pl.ucache <= kWdThreads && ctas <= d.sms &&
-              ctas <= std::max<int64_t>((int64_t)c->batch * c->n_kv_heads, kAssumedMaxSms)) ? 1 : 0;
-    p.cpart = reinterpret_cast<float*>(base + w.cpart);
-    p.cticket = reinterpret_cast<uint32_t*>(base + w.att_cnt);
-  }
   p.sketch = static_cast<const __nv_bfloat16*>(c->sketch);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
   p.v = static_cast<const __nv_bfloat16*>(c->v);
