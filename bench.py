@@ -70,15 +70,15 @@ def peaks():
         return 6650.0, "fallback"
 
 
-def csrc_sha256() -> str:
-    """Digest of the code of every kernel and host source of the library, in
+def csrc_sha256(files=None) -> str:
+    """Digest of the code of the named library sources (default: all), in
     name order, with comments and runs of white space removed: a figure
-    captured from the code holds while the code is unchanged."""
+    captured from the code holds while that code is unchanged."""
     import hashlib
     import re
     d = os.path.join(ROOT, "rope_frequency_chunk_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
+    for name in sorted(files or os.listdir(d)):
         with open(os.path.join(d, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -106,7 +106,7 @@ def profiled_traffic(kernel: str, workload: str):
     except (OSError, ValueError):
         return None
     e = rec.get(f"{kernel}@{workload}")
-    if not e or e.get("csrc_sha256") != csrc_sha256():
+    if not e or e.get("csrc_sha256") != csrc_sha256(e.get("sources")):
         return None
     return int(e["bytes_per_launch"])
 
