@@ -109,22 +109,24 @@ def test_reference_arm_prints_on_rank_zero_only(capsys, monkeypatch):
 
 def test_profiled_traffic_is_gated_by_workload_and_sources(tmp_path, monkeypatch):
     """roofline.traffic comes from the committed ncu record (JSON) only for the
-    captured kernel and workload, and only while the library sources are the
+    captured kernel and workload, and only while the kernel's sources are the
     captured ones."""
     import json
     wl = bench.W.CONFIGS["c2"]
     sig = bench.workload_sig(wl, wl.k)
     assert sig == "c2-B1-H32/8-L32768-n16-k256-bf16"
-    digest = "ab" * 32
-    rec = {f"decode_wide_kernel@{sig}": {"bytes_per_launch": 123, "csrc_sha256": digest}}
+    srcs = ["decode_wide.cuh", "tip.cuh"]
+    rec = {f"decode_wide_kernel@{sig}": {"bytes_per_launch": 123, "sources": srcs,
+                                         "csrc_sha256": bench.csrc_sha256(srcs)}}
     path = tmp_path / "traffic.json"
     path.write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
-    monkeypatch.setattr(bench, "csrc_sha256", lambda: digest)
     assert bench.profiled_traffic("decode_wide_kernel", sig) == 123
     assert bench.profiled_traffic("decode_wide_kernel", bench.workload_sig(wl, 512)) is None
     assert bench.profiled_traffic("score_kernel", sig) is None
-    monkeypatch.setattr(bench, "csrc_sha256", lambda: "0" * 64)
+    # the digest covers the named sources only; any change there voids the figure
+    assert bench.csrc_sha256(srcs) != bench.csrc_sha256(["decode_wide.cuh"])
+    monkeypatch.setattr(bench, "csrc_sha256", lambda files=None: "0" * 64)
     assert bench.profiled_traffic("decode_wide_kernel", sig) is None
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
     assert bench.profiled_traffic("decode_wide_kernel", sig) is None
