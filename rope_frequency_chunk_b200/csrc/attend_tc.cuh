@@ -12,9 +12,10 @@
 //  - K and V rows are gathered with 16-byte cp.async into shared memory in
 //    the 128-byte-swizzled layout the tensor core reads (K-major for K, the
 //    same bytes read MN-major for V);
-//  - the scaled rotated queries and the probabilities are split into two
-//    bf16 terms (hi + lo), two MMAs each, so S and O keep about 16
-//    significant bits of each operand instead of 8;
+//  - the scaled rotated queries are split into three bf16 terms (hi + mid +
+//    lo) and the probabilities into two (hi + lo), one MMA per term, so the
+//    logits keep about 24 significant bits of the queries and O about 16 of
+//    the probabilities (bf16 alone keeps 8);
 //  - one thread issues tcgen05.mma; completion is signalled by
 //    tcgen05.commit on an mbarrier (bounded wait); each query row's thread
 //    reads its S row from TMEM (tcgen05.ld), runs the online softmax in base 2
@@ -56,12 +57,12 @@ struct TcParams {
   double theta[kNFC];
 };
 
-// Shared memory: four K-major tile pairs of RQ rows (Q hi, Q lo, P hi, P lo),
+// Shared memory: five K-major tile pairs of RQ rows (Q hi, Q mid, Q lo, P hi, P lo),
 // the K and V tiles (128 rows each), kept slots, mbarrier, TMEM address, the
 // tokens' rotation tables; plus 1 KB to align the tiles to 1024 bytes.
 __host__ __device__ constexpr int tc_rows_pad(int mq) { return (mq + 7) / 8 * 8; }
 __host__ __device__ constexpr int tc_smem_bytes(int mq, int n_q) {
-  return 4 * 2 * tc_rows_pad(mq) * 128 + 2 * 32768 + kTcTile * 4 + 16 + n_q * 2 * kNFC * 8 + 1024;
+  return 5 * 2 * tc_rows_pad(mq) * 128 + 2 * 32768 + kTcTile * 4 + 16 + n_q * 2 * kNFC * 8 + 1024;
 }
 
 // Byte offset of 16-byte chunk c (0 .. 15) of row r in a tile pair of R rows
@@ -149,6 +150,20 @@ __device__ __forceinline__ uint32_t tc_pack(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// hi + mid + lo split of 8 floats into three 16-byte bf16 chunks (each
+// difference is exact in float32): about 24 significant bits.
+__device__ __forceinline__ void tc_split8x3(const float* x, uint4& hi, uint4& mid, uint4& lo) {
+  float r[8], t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r[i] = x[i] - __bfloat162float(__float2bfloat16_rn(x[i]));
+    t[i] = r[i] - __bfloat162float(__float2bfloat16_rn(r[i]));
+  }
+  hi = make_uint4(tc_pack(x[0], x[1]), tc_pack(x[2], x[3]), tc_pack(x[4], x[5]), tc_pack(x[6], x[7]));
+  mid = make_uint4(tc_pack(r[0], r[1]), tc_pack(r[2], r[3]), tc_pack(r[4], r[5]), tc_pack(r[6], r[7]));
+  lo = make_uint4(tc_pack(t[0], t[1]), tc_pack(t[2], t[3]), tc_pack(t[4], t[5]), tc_pack(t[6], t[7]));
+}
+
 // hi + lo split of 8 floats into two 16-byte bf16 chunks.
 __device__ __forceinline__ void tc_split8(const float* x, uint4& hi, uint4& lo) {
   float r[8];
@@ -166,8 +181,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
   const int split = blockIdx.x, row = blockIdx.y;
   const int G = p.group, MQ = p.n_q * G, RQ = tc_rows_pad(MQ);
   const uint32_t pair = 2u * RQ * 128u;  // bytes of one Q / P tile pair
+  // the Q and P tile pairs come first: an MMA reads all 128 rows of a pair
+  // (rows past RQ only feed accumulator rows that are never read), so each
+  // pair's reads stay inside the allocation, within the K and V tiles
   unsigned char* qhi = smem;
-  unsigned char* qlo = qhi + pair;
+  unsigned char* qmd = qhi + pair;
+  unsigned char* qlo = qmd + pair;
   unsigned char* phi = qlo + pair;
   unsigned char* plo = phi + pair;
   unsigned char* ks = plo + pair;  // K tile pair, 128 rows (1024-aligned: pair is a multiple of 1024)
@@ -223,9 +242,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
                                    : __dadd_rn(__dmul_rn(bb, cz[i]), __dmul_rn(a, cz[kNFC + i]));
         x[e] = (float)(rr * qscale);
       }
-      uint4 hi, lo;
-      tc_split8(x, hi, lo);
+      uint4 hi, md, lo;
+      tc_split8x3(x, hi, md, lo);
       *reinterpret_cast<uint4*>(qhi + tc_sw(r, ch, RQ)) = hi;
+      *reinterpret_cast<uint4*>(qmd + tc_sw(r, ch, RQ)) = md;
       *reinterpret_cast<uint4*>(qlo + tc_sw(r, ch, RQ)) = lo;
     }
   }
@@ -272,7 +292,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // S = (Q hi + Q lo) K^T
+    // S = (Q hi + Q mid + Q lo) K^T
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -280,6 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const TcParams
         const uint32_t qo = (s8 >> 2) * RQ * 128 + (s8 & 3) * 32;
         const uint64_t bd = tc_desc(smem_u32(ks) + (s8 >> 2) * kTcTile * 128 + (s8 & 3) * 32, 16, 1024);
         tc_mma(tbase, tc_desc(smem_u32(qhi) + qo, 16, 1024), bd, tc_idesc(0), s8 > 0);
+        tc_mma(tbase, tc_desc(smem_u32(qmd) + qo, 16, 1024), bd, tc_idesc(0), 1);
         tc_mma(tbase, tc_desc(smem_u32(qlo) + qo, 16, 1024), bd, tc_idesc(0), 1);
       }
       tc_commit(bar);

@@ -14,9 +14,9 @@
 // and V rows (16-byte cp.async into the swizzled layout) bounds the kernel,
 // and two CTAs per SM overlap their chains.
 //
-// The rotated, scaled queries and the probabilities are split into two bf16
-// terms (hi + lo, two MMAs each): about 16 significant bits per operand,
-// float32 accumulation. A kept row outside [0, len) is masked (its logit is
+// The rotated, scaled queries are split into three bf16 terms (hi + mid +
+// lo) and the probabilities into two (hi + lo), one MMA per term: about 24
+// and 16 significant bits, float32 accumulation. A kept row outside [0, len) is masked (its logit is
 // -inf) and flagged; a multi-query row does not see kept slots after its
 // own position. Splits of a row write (m, l, o) partials in the layout of
 // the CUDA-core split-K kernel's; the row's last CTA merges them in order.
@@ -60,10 +60,10 @@ struct TsParams {
 };
 
 __host__ __device__ constexpr int ts_smem_bytes(int n_q) {
-  // Q hi / lo and P hi / lo tile pairs of 16 rows, K and V tiles, kept slots,
+  // Q hi / lo and P hi / lo tile pairs of 16 rows, K and V tiles, Q mid, kept slots,
   // column maxima / sums / weights, mbarrier and TMEM address, angle tables,
   // 1 KB to align the tiles
-  return 4 * 2 * kTsN * 128 + 2 * 32768 + kTsTile * 4 + (2 * 4 * kTsN + 3 * kTsN) * 4 + 16 +
+  return 5 * 2 * kTsN * 128 + 2 * 32768 + kTsTile * 4 + (2 * 4 * kTsN + 3 * kTsN) * 4 + 16 +
          n_q * 2 * kNFC * 8 + 1024;
 }
 
@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(kTsThreads, 2) attend_tcs_kernel(const TsParam
   const int G = p.group, MQ = p.n_q * G;
   constexpr uint32_t kPair = 2u * kTsN * 128u;  // one 16-row tile pair (4 KB)
   unsigned char* qhi = smem;
-  unsigned char* qlo = qhi + kPair;
+  unsigned char* qmd = qhi + kPair;
+  unsigned char* qlo = qmd + kPair;
   unsigned char* phi = qlo + kPair;
   unsigned char* plo = phi + kPair;
   unsigned char* ks = plo + kPair;  // 1024-aligned
@@ -156,9 +157,10 @@ __global__ void __launch_bounds__(kTsThreads, 2) attend_tcs_kernel(const TsParam
                                    : __dadd_rn(__dmul_rn(bb, cz[i]), __dmul_rn(a, cz[kNFC + i]));
         x[e] = (float)(rr * qscale);
       }
-      uint4 hi, lo;
-      tc_split8(x, hi, lo);
+      uint4 hi, md, lo;
+      tc_split8x3(x, hi, md, lo);
       *reinterpret_cast<uint4*>(qhi + tc_sw(r, ch, kTsN)) = hi;
+      *reinterpret_cast<uint4*>(qmd + tc_sw(r, ch, kTsN)) = md;
       *reinterpret_cast<uint4*>(qlo + tc_sw(r, ch, kTsN)) = lo;
     }
   }
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kTsThreads, 2) attend_tcs_kernel(const TsParam
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // S^T = K (Q hi + Q lo)^T: M 128 kept rows, N 16 query rows, K 128 dims
+    // S^T = K (Q hi + Q mid + Q lo)^T: M 128 kept rows, N 16 query rows, K 128 dims
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(kTsThreads, 2) attend_tcs_kernel(const TsParam
         const uint32_t qo = (s8 >> 2) * kTsN * 128 + (s8 & 3) * 32;
         const uint64_t ad = tc_desc(smem_u32(ks) + ko, 16, 1024);
         tc_mma(tbase, ad, tc_desc(smem_u32(qhi) + qo, 16, 1024), tc_idesc_n(kTsN, 0, 0), s8 > 0);
+        tc_mma(tbase, ad, tc_desc(smem_u32(qmd) + qo, 16, 1024), tc_idesc_n(kTsN, 0, 0), 1);
         tc_mma(tbase, ad, tc_desc(smem_u32(qlo) + qo, 16, 1024), tc_idesc_n(kTsN, 0, 0), 1);
       }
       tc_commit(bar);
