@@ -16,7 +16,6 @@
 #include "select_hist.cuh"
 #include "attend_cc.cuh"
 #include "attend_tc.cuh"
-#include "attend_tcs.cuh"
 #include "decode_wide.cuh"
 #include "calibrate.cuh"
 
@@ -609,27 +608,6 @@ fasa_status launch_attend_t(CcParams& ap, int rows, int splits_max, const DevInf
   return launch_pdl(kern, dim3((unsigned)ap.splits, (unsigned)rows, 1), kCcThreads, (size_t)smem, st, ap);
 }
 
-// The tensor-core attention for up to 16 query rows per KV head (kept rows
-// along the TMEM lanes): splits per row so that about two CTAs per SM run,
-// each over a multiple of 128 list positions.
-fasa_status launch_ts(TsParams& tp, int rows, int splits_max, const DevInfo& d, cudaStream_t st) {
-  const int64_t tiles = ceil_div(std::max(tp.n_keep, 1), kTsTile);
-  int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, 2LL * d.sms / rows));
-  splits = std::max<int64_t>(1, std::min<int64_t>(splits, std::min(splits_max, kTsMaxSplits)));
-  tp.slice = (int)(ceil_div(tiles, splits) * kTsTile);
-  tp.splits = (int)ceil_div(std::max(tp.n_keep, 1), tp.slice);
-  const int smem = ts_smem_bytes(tp.n_q);
-  int ok = 0;
-  fasa_status s = cached_int(reinterpret_cast<const void*>(attend_tcs_kernel), 0, &ok, [&](int* r) {
-    *r = 1;
-    return cuda_status(cudaFuncSetAttribute(attend_tcs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            ts_smem_bytes(kTcMaxTok)));
-  });
-  if (s != FASA_OK) return s;
-  return launch_pdl(attend_tcs_kernel, dim3((unsigned)tp.splits, (unsigned)rows, 1), kTsThreads, (size_t)smem, st,
-                    tp);
-}
-
 fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
                           const void* q, int32_t q_pos, float* part, uint32_t* counter, int splits_max,
                           const DevInfo& d, cudaStream_t st, const fasa_varlen* vl = nullptr,
@@ -656,32 +634,6 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
     fill_theta(ap.cosv, c->rope_base);
   } else {
     fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
-  }
-  {  // the tensor-core kernel (kept rows on the TMEM lanes), G <= 16 query rows
-    TsParams tp{};
-    tp.k = ap.k;
-    tp.v = ap.v;
-    tp.idx = idx;
-    tp.q = ap.q;
-    tp.out = ap.out;
-    tp.part = part;
-    tp.counter = counter;
-    tp.max_len = c->max_len;
-    tp.len = len;
-    tp.n_keep = n_keep;
-    tp.group = ap.group;
-    tp.n_q = 1;
-    tp.n_kv_heads = c->n_kv_heads;
-    tp.q_pos0 = q_pos;
-    tp.q_prerot = (vl && vl->q_prerotated) ? 1 : 0;
-    tp.seq_len = ap.seq_len;
-    tp.row_keep = ap.row_keep;
-    tp.pm = ap.pm;
-    for (int i = 0; i < kNFC; ++i) {
-      tp.cosv[i] = ap.cosv[i];
-      tp.sinv[i] = ap.sinv[i];
-    }
-    return launch_ts(tp, rows, splits_max, d, st);
   }
   if (ap.group <= 4) return launch_attend_t<4>(ap, rows, splits_max, d, st);
   if (ap.group <= 8) return launch_attend_t<8>(ap, rows, splits_max, d, st);
@@ -1251,30 +1203,6 @@ fasa_status fasa_decode_multi(const fasa_cache* c, int32_t len, const void* q, i
   else
     fill_theta(p.cosv, c->rope_base);
   if ((s = launch_wide_sel(p, c->batch * c->n_kv_heads, pl, d, stream)) != FASA_OK) return s;
-  if (n_q * p.group <= kTsN) {  // up to 16 query rows: kept rows along the TMEM lanes
-    TsParams tp{};
-    tp.k = p.k;
-    tp.v = p.v;
-    tp.idx = p.idx_ws;
-    tp.q = p.q;
-    tp.out = p.out;
-    tp.part = reinterpret_cast<float*>(base + m.tpart);
-    tp.counter = reinterpret_cast<uint32_t*>(base + m.w.att_cnt);
-    tp.max_len = c->max_len;
-    tp.len = len;
-    tp.n_keep = keff;
-    tp.group = p.group;
-    tp.n_q = n_q;
-    tp.n_kv_heads = c->n_kv_heads;
-    tp.q_pos0 = p.q_pos0;
-    tp.q_prerot = p.q_prerot;
-    tp.mask_after = 1;
-    for (int i = 0; i < kNFC; ++i) {
-      tp.cosv[i] = p.cosv[i];
-      tp.sinv[i] = p.sinv[i];
-    }
-    return launch_ts(tp, c->batch * c->n_kv_heads, m.splits_max, d, stream);
-  }
   return launch_tc(c, len, keff, q, q_pos0, n_q, out, m, base, d, stream);
 }
 
