@@ -174,7 +174,7 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   if (direct) {
     c = kWdMaxDirect * MG * 4;
     L.ring = o + c;
-    c += kWdWarps * MG * kD * 4 + 64 + kWdMaxDirect * kD * 2;
+    c += kWdWarps * MG * kD * 4 + (16 + 2 * kWdWarps) * 4 + kWdMaxDirect * kD * 2;
   } else {
     L.ring = o;
   }
@@ -597,6 +597,10 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   const int words = (Lr + 31) / 32;
   const uint2* rows0 = p.cand + (int64_t)row * p.n_split * rstride;
   if (tid == 0) p.sem[row] = 0ull;  // every CTA of the row has arrived: ready for the next call
+  // the histogram and the bitmap are cleared while the union's loads are in flight
+  for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
+  for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
+  if (tid == 0) misc[100] = 0u;
   {  // slots [0, S): the regions' counts; then entry j < P of region s at S + s*P + j
     const int nslots = S_ + (S_ << p.ushift);
     for (int base = 0; base < nslots; base += kWdThreads * kWdUnionUnroll) {
@@ -619,14 +623,14 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       }
     }
   }
-  for (int i = tid; i < 4096; i += kWdThreads) hist[i] = 0u;
-  for (int i = tid; i < words; i += kWdThreads) bm[i] = 0u;
-  if (tid == 0) misc[100] = 0u;
   __syncthreads();
-  if (warp == 0) {  // prefix sums of the counts (S <= 32 per pass of the warp)
-    uint32_t run = 0u;
+  if (warp == 0) {  // prefix sums of the counts (S <= 32 per pass of the warp), the highest b_loc, overflow
+    uint32_t run = 0u, bmx = 0u;
+    bool ovf = false;
     for (int s0 = 0; s0 < S_; s0 += 32) {
       const uint32_t c = s0 + lane < S_ ? cnt[s0 + lane] : 0u;
+      if (s0 + lane < S_) bmx = max(bmx, cnt[2 * S_ + 1 + s0 + lane]);
+      ovf |= c > (uint32_t)P;
       uint32_t incl = c;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -636,15 +640,19 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       if (s0 + lane < S_) cnt[S_ + 1 + s0 + lane] = run + incl;
       run += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
-    if (lane == 0) cnt[S_] = 0u;
+    bmx = __reduce_max_sync(0xFFFFFFFFu, bmx);
+    ovf = __any_sync(0xFFFFFFFFu, ovf);
+    if (lane == 0) {
+      cnt[S_] = 0u;
+      misc[110] = bmx;
+      misc[111] = ovf ? 1u : 0u;
+    }
   }
   __syncthreads();
   const uint32_t* pre = cnt + S_;  // pre[s] = entries of regions before s; pre[S] = all
-  uint32_t b_max = 0u;  // the highest b_loc: a row boundary bin below it cannot be trusted
-  for (int sr = 0; sr < S_; ++sr) b_max = max(b_max, cnt[2 * S_ + 1 + sr]);
+  const uint32_t b_max = misc[110];  // the highest b_loc: a row boundary bin below it cannot be trusted
   const int nu = (int)min(pre[S_], (uint32_t)p.len);
-  bool overflow = false;
-  for (int sr = 0; sr < S_; ++sr) overflow |= cnt[sr] > (uint32_t)P;
+  const bool overflow = misc[111] != 0u;
   // every union entry once: the staged ones, then (rare) the rest from global memory
   auto for_union = [&](auto&& fn) {
     for (int f = tid; f < (S_ << p.ushift); f += kWdThreads)
@@ -734,7 +742,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   float* zs = reinterpret_cast<float*>(smem + Lo.zs);
   float* mo = reinterpret_cast<float*>(smem + Lo.ring);
   float* lsum = mo + kWdWarps * MG * kD;
-  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
+  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16 + 2 * kWdWarps);
   const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
   cc_block_attend<MG, kWdWarps>(p.k + plane, p.v + plane,
                                 [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
