@@ -445,9 +445,8 @@ namespace fasa {
 // head h over all n logits (max, exp2, sum; zs becomes the probabilities);
 // (3) each warp adds p * v over its rows for the lane's 4 dims; (4) the warp
 // sums are added in a fixed order and divided by the head's sum.
-// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [16 +
-// 2 * NW] floats (head sums, then the softmax's partial maxima and sums),
-// vst [16 * NW][128] bf16 (the V rows, staged with cp.async).
+// Shared memory: zs [16 * NW][MG] floats, mo [NW][MG][128] floats, lsum [16]
+// floats, vst [16 * NW][128] bf16 (the V rows, staged with cp.async).
 template <int MG, int NW, typename Tok>
 __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const __nv_bfloat16* vb, Tok token, int n,
                                                 int G, const float* qs, float* zs, float* mo, float* lsum,
@@ -500,42 +499,25 @@ __device__ __forceinline__ void cc_block_attend(const __nv_bfloat16* kb, const _
     }
   }
   __syncthreads();
-  // (2) softmax of each head over the n rows: wph = NW / G warps per head,
-  // each over a strided share of the rows; partial maxima, then the head's
-  // maximum, the probabilities and partial sums (added in warp order in (3))
+  // (2) softmax of head `warp` over the n rows
   const int nr = 16 * NW;  // every row written in (1); padding rows are -inf and become 0
-  const int wph = NW / G;  // >= 2 (G <= 8)
-  const int hh = warp / wph, part = warp % wph;
-  float* pm = lsum + 16;   // [NW] partial maxima
-  float* pl = pm + NW;     // [NW] partial sums
-  if (hh < G) {
+  if (warp < G) {
     float m = -INFINITY;
-    for (int j = part * 32 + lane; j < nr; j += wph * 32) m = fmaxf(m, zs[j * MG + hh]);
+    for (int j = lane; j < nr; j += 32) m = fmaxf(m, zs[j * MG + warp]);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-    if (lane == 0) pm[warp] = m;
-  }
-  __syncthreads();
-  if (hh < G) {
-    float m = -INFINITY;
-    for (int q = 0; q < wph; ++q) m = fmaxf(m, pm[hh * wph + q]);
     float l = 0.0f;
-    for (int j = part * 32 + lane; j < nr; j += wph * 32) {
-      const float z = zs[j * MG + hh];
+    for (int j = lane; j < nr; j += 32) {
+      const float z = zs[j * MG + warp];
       const float pz = (z == -INFINITY) ? 0.0f : exp2f(z - m);
-      zs[j * MG + hh] = pz;
+      zs[j * MG + warp] = pz;
       l += pz;
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-    if (lane == 0) pl[warp] = l;
+    if (lane == 0) lsum[warp] = l;
   }
   __syncthreads();
-  if (tid < G) {  // the head's sum, its partial sums in warp order
-    float l = 0.0f;
-    for (int q = 0; q < wph; ++q) l += pl[tid * wph + q];
-    lsum[tid] = l;
-  }
   // (3) p * v over the warp's rows
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncwarp();

@@ -174,7 +174,7 @@ __host__ __device__ inline WdLayout wd_layout(int n_loc, int len, int n_keep, in
   if (direct) {
     c = kWdMaxDirect * MG * 4;
     L.ring = o + c;
-    c += kWdWarps * MG * kD * 4 + (16 + 2 * kWdWarps) * 4 + kWdMaxDirect * kD * 2;
+    c += kWdWarps * MG * kD * 4 + 64 + kWdMaxDirect * kD * 2;
   } else {
     L.ring = o;
   }
@@ -742,7 +742,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   float* zs = reinterpret_cast<float*>(smem + Lo.zs);
   float* mo = reinterpret_cast<float*>(smem + Lo.ring);
   float* lsum = mo + kWdWarps * MG * kD;
-  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16 + 2 * kWdWarps);
+  __nv_bfloat16* vst = reinterpret_cast<__nv_bfloat16*>(lsum + 16);
   const int64_t plane = paged ? 0 : (int64_t)row * p.max_len * kD;
   cc_block_attend<MG, kWdWarps>(p.k + plane, p.v + plane,
                                 [&](int j) -> int { return paged ? paged_row(p.pm, bb, g, kept[j]) : kept[j]; },
