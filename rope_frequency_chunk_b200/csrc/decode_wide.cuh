@@ -53,7 +53,6 @@ constexpr int kWdThreads = kSAThreads;  // 512 (the histogram and radix helpers'
 constexpr int kWdWarps = kWdThreads / 32;
 constexpr int kWdMaxLoc = 16384;        // tokens per CTA (their keys live in shared memory)
 constexpr int kWdTieCap = 2048;         // boundary-bin entries held in shared memory
-constexpr int kWdDirectRank = 128;      // boundary bins up to this size are resolved by direct ranks
 constexpr int kWdRankMax = 128;         // entries of the finest bin resolved by rank counting
 constexpr int kWdUnionUnroll = 8;       // union entries in flight per thread
 constexpr int kWdMaxDirect = 16 * kWdWarps;  // kept rows the resolving CTA attends itself (16 per warp)
@@ -324,18 +323,6 @@ __device__ void wd_select(ForSrc&& for_src, SrcAt&& src_at, int n_src, int n_kee
   if (need > 0 && n_keep > 0) {
     if (n_b == need && n_b <= kWdTieCap) {
       for (int i = tid; i < n_b; i += kWdThreads) wd_keep(bm, ties[i].y, len);
-    } else if (n_b <= kWdDirectRank) {
-      // few entries in the boundary bin: exact ranks among them (key
-      // descending, then token ascending) in one pass
-      for (int i = tid; i < n_b; i += kWdThreads) {
-        const uint2 a = ties[i];
-        int r = 0;
-        for (int j = 0; j < n_b; ++j) {
-          const uint2 c = ties[j];
-          r += (c.x > a.x) || (c.x == a.x && c.y < a.y);
-        }
-        if (r < need) wd_keep(bm, a.y, len);
-      }
     } else if (n_b <= kWdTieCap) {
       // next 8 key bits of the boundary bin's entries, then ranks (or a
       // radix select) among the entries of the boundary sub-bin
