@@ -101,11 +101,6 @@ __device__ __forceinline__ void round_store(__nv_bfloat16* p, double x) { *p = r
 __device__ __forceinline__ void store_f(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_f(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
-// RoPE angular frequency of FC i: base^(-2i/128), float64.
-__device__ __forceinline__ double rope_theta(double base, int i) {
-  return pow(base, -2.0 * (double)i / (double)kD);
-}
-
 // ---------------------------------------------------------- score keys
 
 // Order-preserving map float32 -> uint32 (larger score, larger key); -0.0 is
@@ -173,17 +168,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// 16-byte streaming load through the read-only path, not kept in L1.
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 r;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-// Programmatic dependent launch: wait until the preceding kernel in the
-// stream has completed and its memory is visible (no-op without PDL).
 // Hint: bring [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
 // Safe before griddepcontrol.wait: later loads still see the latest data.
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
@@ -193,6 +177,9 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 __device__ __forceinline__ void prefetch_line_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
+// Programmatic dependent launch: wait until the preceding kernel in the
+// stream has completed and its memory is visible (no-op without PDL); let
+// the next kernel in the stream be scheduled.
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -229,20 +216,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-}  // namespace fasa
-
-namespace fasa {
-
-// Plain mbarrier arrival (count one), release semantics.
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Barrier among a subset of the CTA's warps (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 }  // namespace fasa
