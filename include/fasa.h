@@ -243,12 +243,13 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *    about (SM count / rows) independent CTAs. Each scores its share of the
  *    sketch in registers, keeps its own top-k candidates and publishes them
  *    to the workspace; the row's last CTA to finish (an atomic ticket, no
- *    waiting) selects the exact top-k of the union and, for k_eff <= 512,
- *    attends those rows itself: one launch. Larger budgets add a split-K
- *    attention launch over the kept list.
+ *    waiting) selects the exact top-k of the union and, for k_eff <= 256
+ *    and G <= 8, attends those rows itself: one launch. Larger budgets add
+ *    a split-K attention launch over the kept list.
  *  FASA_DECODE_STAGED  four launches chained with programmatic dependent
  *    launch: the score stream, which also builds a per-row histogram of the
- *    score keys; a filter that marks the certainly-kept tokens and collects
+ *    score keys and, in the row's last CTA, the row's threshold bin; a
+ *    filter that marks the certainly-kept tokens and collects
  *    the tokens of the threshold bin; a per-row exact resolution of that bin
  *    that emits the kept indices in ascending order; and the focused
  *    attention. Scores, histogram and index lists live in the workspace.
@@ -260,18 +261,19 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned
  *            (required whichever plan runs). Zero it once after allocating it
  *            (e.g. cudaMemsetAsync): its first 12 * B * Hkv bytes hold
- *            per-row semaphores that must be zero when a call starts, and
- *            every call leaves them zero again. The rest is scratch. After a
+ *            per-row semaphores, and the staged plan keeps per-row
+ *            histograms, counters and tickets further in; all must be zero
+ *            when a call starts, and every call leaves them zero again. The
+ *            rest is scratch. After a
  *            call that ended in an error (a CUDA error, FASA_ERR_TIMEOUT),
  *            zero it again. A semaphore found non-zero is reported as
  *            FASA_ERR_WORKSPACE in the device status word; no access then
  *            leaves the workspace.
  *  Ordering: the kernels of a plan follow one another with programmatic
  *  dependent launch, but every read of q, the cache and the workspace
- *  happens after all work issued earlier on the stream has completed (the
- *  staged plan starts with a memset; the fused plan waits on the preceding
- *  grid before reading); only L2 prefetch hints of the sketch may run
- *  earlier.
+ *  happens after all work issued earlier on the stream has completed (each
+ *  plan's first kernel waits on the preceding grid before reading); only
+ *  L2 prefetch hints and the kernels' own parameters may be read earlier.
  *  Calls that overlap on the GPU (different streams) must not share a
  *  workspace.
  *  Errors: as fasa_score, fasa_select_topk and fasa_sparse_attend;

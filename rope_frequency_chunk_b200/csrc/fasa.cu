@@ -149,6 +149,23 @@ fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
   return FASA_OK;
 }
 
+// Plain launch with programmatic stream serialization (the kernel waits
+// for its predecessor with griddepcontrol.wait).
+template <typename K, typename P>
+fasa_status launch_pdl(K kern, dim3 grid, int threads, size_t smem, cudaStream_t st, const P& p) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
+}
+
 // ------------------------------------------------------------ score
 
 template <typename T, int LPT, bool kHist>
@@ -163,8 +180,7 @@ fasa_status launch_score_t(const ScoreParams& p, const DevInfo& d, cudaStream_t 
   if (s != FASA_OK) return s;
   const int64_t cap = ceil_div(p.total, 256);  // at least 256 tokens per CTA
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sms, cap));
-  kern<<<grid, kScoreThreads, smem, st>>>(p);
-  return cuda_status(cudaGetLastError());
+  return launch_pdl(kern, dim3((unsigned)grid, 1, 1), kScoreThreads, (size_t)smem, st, p);
 }
 
 template <typename T, bool kHist>
@@ -185,7 +201,8 @@ fasa_status launch_score_lpt(const ScoreParams& p, const DevInfo& d, cudaStream_
 // histogram of the top 12 bits of each score's order-preserving key (added
 // into `hist`, which must be zero).
 fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_t q_pos, float* scores,
-                         int64_t ld, uint32_t* hist, cudaStream_t st) {
+                         int64_t ld, uint32_t* hist, cudaStream_t st, uint32_t* row_done = nullptr,
+                         uint32_t* thr = nullptr, int32_t n_keep = 0) {
   DevInfo d;
   fasa_status s = device_info(&d);
   if (s != FASA_OK) return s;
@@ -196,6 +213,9 @@ fasa_status launch_score(const fasa_cache* c, int32_t len, const void* q, int32_
   p.scores = scores;
   p.ld = ld;
   p.hist = hist;
+  p.row_done = row_done;
+  p.thr = thr;
+  p.n_keep = n_keep;
   p.max_len = c->max_len;
   p.total = (int64_t)c->batch * c->n_kv_heads * len;
   p.len = len;
@@ -484,6 +504,7 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 //   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the fused plan,
 //     the CTAs' published candidates [rows][len + len/64 + 64] u32x2 |
 //   keys [rows][len] u32 (fused plan: every token's score key) | rowk [rows] i32 (varlen: each row's k_eff) |
+//   (staged plan, zero between calls) hist [rows][4096] u32, cnt [rows], thr [rows][2], rdone [rows] |
 //   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
 //   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
 //   part [rows][splits_max][kCcPartStride] f32
@@ -493,7 +514,7 @@ constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
 struct DecodeWs {
-  size_t sem, att_cnt, scores, keys, rowk, hist, cnt, bitmap, cand, ckey, idx, part, total;
+  size_t sem, att_cnt, scores, keys, rowk, hist, cnt, thr, rdone, bitmap, cand, ckey, idx, part, total;
   int64_t ld;
   int cap, words, splits_max;
 };
@@ -522,7 +543,9 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.rowk = al256(w.keys + rows * L * 4);
   w.hist = al256(w.rowk + rows * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
-  w.bitmap = al256(w.cnt + rows * 4);
+  w.thr = w.cnt + rows * 4;
+  w.rdone = w.thr + rows * 8;
+  w.bitmap = al256(w.rdone + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
   w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
   w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
@@ -532,22 +555,6 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
 }
 size_t decode_ws(const fasa_cache* c, int32_t len, int32_t k) { return decode_layout(c, len, k).total; }
 
-// Plain launch with programmatic stream serialization (the kernel waits
-// for its predecessor with griddepcontrol.wait).
-template <typename K, typename P>
-fasa_status launch_pdl(K kern, dim3 grid, int threads, size_t smem, cudaStream_t st, const P& p) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
-}
 
 // Calibration workspace: score planes [rows][n_win][65][len] f32, then the
 // selections [rows][n_win][65][k_eff] i32.
@@ -966,16 +973,19 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   uint32_t* ckey = reinterpret_cast<uint32_t*>(base + w.ckey);
   int32_t* idx = reinterpret_cast<int32_t*>(base + w.idx);
 
-  // 1. TIP scores and the per-row key histogram
-  if ((s = cuda_status(cudaMemsetAsync(base + w.sem, 0, w.scores - w.sem, stream))) != FASA_OK) return s;
-  if ((s = cuda_status(cudaMemsetAsync(hist, 0, w.bitmap - w.hist, stream))) != FASA_OK) return s;
-  if ((s = launch_score(c, len, q, q_pos, scores, w.ld, hist, stream)) != FASA_OK) return s;
+  // 1. TIP scores, the per-row key histogram and its threshold bin (the
+  // histograms, candidate counters and row tickets are zero between calls:
+  // the score kernel and finalize leave them so)
+  uint32_t* thr = reinterpret_cast<uint32_t*>(base + w.thr);
+  if ((s = launch_score(c, len, q, q_pos, scores, w.ld, hist, stream, reinterpret_cast<uint32_t*>(base + w.rdone),
+                        thr, keff)) != FASA_OK)
+    return s;
 
   // 2. filter: certain tokens into the bitmap, threshold-bin tokens into the candidate list
   FilterParams fp{};
   fp.scores = scores;
   fp.ld = w.ld;
-  fp.hist = hist;
+  fp.thr = thr;
   fp.cand_cnt = cnt;
   fp.cand_idx = cand;
   fp.cand_key = ckey;
@@ -995,7 +1005,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   FinalParams np{};
   np.scores = scores;
   np.ld = w.ld;
-  np.hist = hist;
+  np.thr = thr;
   np.cand_cnt = cnt;
   np.cand_idx = cand;
   np.cand_key = ckey;
@@ -1221,9 +1231,12 @@ fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const v
   if (w.total > FASA_STATIC_SCRATCH_BYTES) return FASA_ERR_WORKSPACE;
   void* ws = nullptr;
   if ((s = static_scratch_addr(&ws)) != FASA_OK) return s;
-  // the semaphores start zero at load and every call leaves them zero; clear
-  // them anyway, so that a call that ended in an error cannot poison the next
+  // the semaphores, histograms and counters start zero at load and every
+  // call leaves them zero; clear them anyway, so that a call that ended in an
+  // error cannot poison the next
   if ((s = cuda_status(cudaMemsetAsync(ws, 0, w.scores, stream))) != FASA_OK) return s;
+  if ((s = cuda_status(cudaMemsetAsync(static_cast<char*>(ws) + w.hist, 0, w.bitmap - w.hist, stream))) != FASA_OK)
+    return s;
   return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);
 }
 

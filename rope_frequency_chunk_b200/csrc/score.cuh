@@ -35,6 +35,12 @@ struct ScoreParams {
   float* scores;         // [rows][ld]
   int64_t ld;            // row stride of scores, >= len
   uint32_t* hist;        // [rows][4096] key-histogram counts (added to), or null
+  // with hist: the row's last CTA (a ticket on row_done, zero between calls)
+  // finds the bin of the row's n_keep-th largest key and the count above it
+  // into thr[row] = (bin, above) and leaves the row's histogram zero
+  uint32_t* row_done;    // [rows]
+  uint32_t* thr;         // [rows][2]
+  int32_t n_keep;
   int64_t max_len;
   int64_t total;         // rows * len
   int32_t len;
@@ -48,6 +54,60 @@ struct ScoreParams {
 
 constexpr int kHistBits = 12;                 // key bits of the per-row score histogram
 constexpr int kHistBins = 1 << kHistBits;
+
+// From a 4096-bin histogram of the top 12 key bits (ld(i) = bin i), the bin
+// holding the k-th largest key (1 <= k <= total) and the number of keys in
+// higher bins, for a block of NT threads: thread t owns bins 4095 - BPT*t ..
+// down to 4096 - BPT*(t + 1), then a suffix scan over the threads. scan:
+// 2 * (NT / 32) + 2 words.
+template <int NT, typename Ld>
+__device__ __forceinline__ void hist_bin_of_kth(Ld ld, int k, uint32_t* scan, uint32_t& bin, uint32_t& above) {
+  constexpr int BPT = (kHistBins + NT - 1) / NT, NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t c[BPT], sum = 0u;
+#pragma unroll
+  for (int u = 0; u < BPT; ++u) {
+    const int b = kHistBins - 1 - (BPT * tid + u);
+    c[u] = b >= 0 ? ld(b) : 0u;
+    sum += c[u];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < NW ? scan[lane] : 0u;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, w, off);
+      if (lane >= off) w += v;
+    }
+    if (lane < NW) scan[NW + lane] = w;
+  }
+  __syncthreads();
+  incl += warp > 0 ? scan[NW + warp - 1] : 0u;
+  const uint32_t excl = incl - sum;
+  if (excl < (uint32_t)k && (uint32_t)k <= incl) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) {
+      if (acc + c[u] >= (uint32_t)k) {
+        scan[2 * NW] = (uint32_t)(kHistBins - 1 - (BPT * tid + u));
+        scan[2 * NW + 1] = acc;
+        break;
+      }
+      acc += c[u];
+    }
+  }
+  __syncthreads();
+  bin = scan[2 * NW];
+  above = scan[2 * NW + 1];
+  __syncthreads();
+}
 
 // Shape of the per-token work for sketch rows of LPT 16-byte chunks, with a
 // chunk rotation per lane so that a quarter-warp's 16-byte shared-memory
@@ -127,6 +187,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
   __shared__ float s_q[kD];
   __shared__ __align__(16) T s_qraw[FASA_MAX_GROUP * kD];  // the group's raw queries
   __shared__ int s_dom[kNFC];
+  __shared__ uint32_t s_scan[2 * kScoreWarps + 2];
+  __shared__ uint32_t s_last;
   __shared__ double s_cs[2 * kNFC];  // cos, sin of the query angle
   // the angle table from the parameters (no dependence on the previous
   // launch): read before the wait, so its constant-bank misses overlap it
@@ -202,6 +264,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
         if (v) {
           atomicAdd(p.hist + (int64_t)row * kHistBins + i, v);
           s_hist[i] = 0u;
+        }
+      }
+      if (p.thr) {  // the row's last segment: its threshold bin, once per row
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(p.row_done + row, (uint32_t)n) + (uint32_t)n == (uint32_t)p.len;
+        __syncthreads();
+        if (s_last) {
+          __threadfence();
+          uint32_t* hr = p.hist + (int64_t)row * kHistBins;
+          uint32_t bin, above;
+          hist_bin_of_kth<kScoreThreads>([hr](int i) { return __ldcg(hr + i); }, p.n_keep, s_scan, bin, above);
+          if (tid == 0) {
+            p.thr[2 * row] = bin;
+            p.thr[2 * row + 1] = above;
+            p.row_done[row] = 0u;
+          }
+          for (int i = tid; i < kHistBins; i += kScoreThreads) hr[i] = 0u;  // ready for the next call
         }
       }
     }

@@ -5,9 +5,9 @@
 // §2, FAC first bullet): T_t is the set of the k highest-scoring tokens
 // (ties to the lower index; k_eff = min(k, L)). Two kernels:
 //
-//  filter   (grid: token tiles x rows) The row's 4096-bin histogram of the
-//           top 12 bits of the order-preserving score keys gives the bin b1
-//           holding the k_eff-th key and the count of keys above it. Keys in
+//  filter   (grid: token tiles x rows) The bin b1 holding the k_eff-th key
+//           (found once per row by the score kernel from the row's 4096-bin
+//           histogram of the top 12 key bits) splits the row. Keys in
 //           higher bins are certainly kept: each warp writes the bitmap word
 //           of its 32 consecutive tokens (every word of [0, len) is written
 //           exactly once, so the bitmap needs no clearing). Keys in bin b1
@@ -37,7 +37,7 @@ constexpr int kFilterCands = 2048;  // candidates a CTA gathers in shared memory
 struct FilterParams {
   const float* scores;      // [rows][ld], 16-byte aligned
   int64_t ld;               // row stride of scores, a multiple of 32
-  const uint32_t* hist;     // [rows][4096]
+  const uint32_t* thr;      // [rows][2]: the bin of the k_eff-th key, the keys above it
   uint32_t* cand_cnt;       // [rows], zero before the launch
   int32_t* cand_idx;        // [rows][cap]
   uint32_t* cand_key;       // [rows][cap], the candidates' score keys
@@ -50,7 +50,6 @@ struct FilterParams {
 };
 
 __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterParams p) {
-  __shared__ uint32_t scan[64];
   __shared__ int32_t s_cidx[kFilterCands];
   __shared__ uint32_t s_ckey[kFilterCands];
   __shared__ uint32_t s_n, s_base;
@@ -58,8 +57,8 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_n = 0u;
   grid_dependency_wait();
-  uint32_t bin, above;
-  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);  // its barriers publish s_n
+  const uint32_t bin = __ldcg(p.thr + 2 * row);
+  __syncthreads();  // publishes s_n
   const int t0 = blockIdx.x * p.tile;
   const int t1 = min(p.len, t0 + p.tile);
   const float4* s4 = reinterpret_cast<const float4*>(p.scores + (int64_t)row * p.ld);
@@ -134,8 +133,8 @@ __global__ void __launch_bounds__(kFilterThreads, 4) filter_kernel(const FilterP
 struct FinalParams {
   float* scores;            // [rows][ld]; the slow path turns a row into keys in place
   int64_t ld;
-  const uint32_t* hist;
-  const uint32_t* cand_cnt;
+  const uint32_t* thr;      // [rows][2]
+  uint32_t* cand_cnt;       // [rows]; finalize leaves it zero
   const int32_t* cand_idx;  // [rows][cap]
   const uint32_t* cand_key; // [rows][cap]
   const uint32_t* bitmap;   // [rows][words]
@@ -181,8 +180,7 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
     }
   }
   cp_async_commit();
-  uint32_t bin, above;
-  hist_threshold(p.hist + (int64_t)row * 4096, p.n_keep, scan, bin, above);
+  const uint32_t bin = __ldcg(p.thr + 2 * row), above = __ldcg(p.thr + 2 * row + 1);
   const int krem = p.n_keep - (int)above;
   cp_async_wait<0>();
   __syncthreads();
@@ -289,6 +287,7 @@ __global__ void __launch_bounds__(kSAThreads, 1) finalize_kernel(const FinalPara
       ++pos;
     }
   }
+  if (tid == 0) p.cand_cnt[row] = 0u;  // the workspace is ready for the next call
 }
 
 }  // namespace fasa
