@@ -458,9 +458,12 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   // query's round trip and the float64 work overlap the stream
   const int G = p.group;
   {
-    if (p.n_q == 1) {
+    if (p.n_q == 1) {  // one round trip: both loads in flight before either store
       const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + ((int64_t)(bb * p.n_kv_heads + g) * G) * kD);
-      for (int c = tid; c < G * kD / 8; c += kWdThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+      const uint4 qv = tid < G * kD / 8 ? __ldg(qsrc + tid) : make_uint4(0u, 0u, 0u, 0u);
+      const int dv = tid < p.n_dom ? __ldg(p.dom_idx + g * p.n_dom + tid) : 0;
+      if (tid < G * kD / 8) reinterpret_cast<uint4*>(qraw)[tid] = qv;
+      if (tid < p.n_dom) s_dom[tid] = dv;
     } else {  // rows j * G + h: token j's group queries
       const int hq = p.n_kv_heads * G;
       for (int c = tid; c < p.n_q * G * kD / 8; c += kWdThreads) {
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
             reinterpret_cast<const uint4*>(p.q + (((int64_t)bb * p.n_q + j) * hq + g * G + h) * kD) + c % (kD / 8));
       }
     }
-    if (tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
+    if (p.n_q > 1 && tid < p.n_dom) s_dom[tid] = __ldg(p.dom_idx + g * p.n_dom + tid);
     if (p.n_q > 1) {  // token j at position q_pos0 + j
       for (int e = tid; e < p.n_q * kNFC; e += kWdThreads) {
         const int j = e / kNFC, i = e % kNFC;
