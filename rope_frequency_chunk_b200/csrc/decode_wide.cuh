@@ -533,9 +533,14 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
   }
   __syncthreads();
 
-  // 3. the bin b_loc holding this CTA's n_pub-th key; publish the tokens at
-  // or above it into the CTA's own region: [(count, b_loc)][(key, token) ...],
-  // and every key to the row's key array
+  // 3. every key to the row's key array (for the exact fallback; written
+  // first, so that the stores complete while the rest of this step runs);
+  // the bin b_loc holding this CTA's n_pub-th key; publish the tokens at or
+  // above it into the CTA's own region: [(count, b_loc)][(key, token) ...]
+  {
+    uint32_t* kdst = p.keys + (int64_t)row * p.len + t_beg;
+    for (int i = tid; i < n_tok; i += kWdThreads) kdst[i] = keys[i];
+  }
   uint32_t b_loc = 0u;
   if (n_tok > n_pub) {
     uint32_t above = 0u;
@@ -573,9 +578,6 @@ __global__ void __launch_bounds__(kWdThreads, 1) decode_wide_kernel(const WidePa
       pos += __popc(m);
     }
     if (tid == 0) region[0] = make_uint2(misc[96], b_loc);
-    // every key, for the exact fallback
-    uint32_t* kdst = p.keys + (int64_t)row * p.len + t_beg;
-    for (int i = tid; i < n_tok; i += kWdThreads) kdst[i] = keys[i];
   }
   __threadfence();
   __syncthreads();
