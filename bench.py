@@ -528,7 +528,10 @@ def run_fasa(args, wl):
     fused = plan == F.DECODE_FUSED
     kern = {1: "decode_wide_kernel (score + select + attend, one launch per layer)",
             2: "decode_wide_kernel + attend_mma_kernel (two launches per layer)",
-            4: "score_kernel + filter_kernel + finalize_kernel + attend (four launches per layer)"}[launches]
+            3: "decode_wide_kernel + attend_mma_kernel + attend_merge_kernel (three launches per layer)",
+            4: "score_kernel + filter_kernel + finalize_kernel + attend (four launches per layer)",
+            5: "score_kernel + filter_kernel + finalize_kernel + attend + split merge (five launches per layer)"
+            }[launches]
     roof = {"bound": "hbm", "kernel": kern, "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
             "frac": gbs / world / hbm_peak,
             "traffic": profiled_traffic("decode_wide_kernel", workload_sig(wl, k)) if launches == 1 else None,
@@ -598,7 +601,8 @@ def run_fasa(args, wl):
         "decode_plan": "fused" if fused else "staged",
         "clocks": clocks,
         # kernels of this library per layer (fasa_decode_launches): fused 1, or 2 with the split-K
-        # attention; staged 4 (score, filter, finalize, attend)
+        # attention; staged 4 (score, filter, finalize, attend); +1 when the attention is split
+        # over several CTAs per row (the split merge)
         "gpu_launches": launches * n_layers * args.steps,
         "e2e": e2e,
     }

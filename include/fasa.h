@@ -245,14 +245,16 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *    to the workspace; the row's last CTA to finish (an atomic ticket, no
  *    waiting) selects the exact top-k of the union and, for k_eff <= 256
  *    and G <= 8, attends those rows itself: one launch. Larger budgets add
- *    a split-K attention launch over the kept list.
+ *    a split-K attention launch over the kept list (and, when a row's list
+ *    spans several CTAs, a launch that merges their partial results).
  *  FASA_DECODE_STAGED  four launches chained with programmatic dependent
  *    launch: the score stream, which also builds a per-row histogram of the
  *    score keys and, in the row's last CTA, the row's threshold bin; a
  *    filter that marks the certainly-kept tokens and collects
  *    the tokens of the threshold bin; a per-row exact resolution of that bin
  *    that emits the kept indices in ascending order; and the focused
- *    attention. Scores, histogram and index lists live in the workspace.
+ *    attention (plus the split merge when a row's kept list spans several
+ *    CTAs). Scores, histogram and index lists live in the workspace.
  *
  *  out     : [B][Hq][128] dtype.
  *  idx_out : nullable; [B][Hkv][min(k, len)] int32, the kept tokens in
@@ -300,9 +302,11 @@ fasa_status fasa_set_decode_path(int32_t path);
 int32_t fasa_decode_path(const fasa_cache* cache, int32_t len, int32_t k);
 
 /* Kernels of this library one fasa_decode call launches for this cache, len
- * and k under the current setting (the fused plan: 1, or 2 when the budget
- * needs the split-K attention; the staged plan: 4), or a negative
- * fasa_status for invalid arguments. */
+ * and k under the current setting on the current device (the fused plan: 1,
+ * or 2 when the budget needs the split-K attention; the staged plan: 4; the
+ * split-K attention of a bf16 cache adds 1, the split merge, when a row's
+ * kept list spans several CTAs), or a negative fasa_status for invalid
+ * arguments. */
 int32_t fasa_decode_launches(const fasa_cache* cache, int32_t len, int32_t k);
 
 /*
@@ -487,8 +491,9 @@ size_t fasa_dense_workspace_bytes(const fasa_cache* cache, int32_t len);
  * Dense full-KV decode, the comparison path: the same attention as
  * fasa_sparse_attend over all len cached rows (the upper bound in
  * [tech §4] "Resultados Experimentais", full KV "FKV"). bf16 caches run the
- * decode's split-K tensor-core attention over every row (a one-wave grid of
- * splits, merged by each row's last CTA); f32 caches a cluster kernel.
+ * decode's split-K attention over every row (a one-wave grid of splits,
+ * merged by a second launch; tensor-core products for groups of up to 8
+ * query heads); f32 caches a cluster kernel.
  *
  *  workspace : at least fasa_dense_workspace_bytes(cache, len) bytes,
  *            256-byte aligned, zeroed once after allocation: its first

@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfasa.so")
 SOURCES = ["fasa.cu"]
-DEPS = ["fasa.cu", "fasa_device.cuh", "append.cuh", "score.cuh", "select_attend.cuh", "select_hist.cuh", "decode_wide.cuh", "tip.cuh", "attend_cc.cuh", "attend_tc.cuh", "calibrate.cuh"]
+DEPS = ["fasa.cu", "fasa_device.cuh", "append.cuh", "score.cuh", "select_attend.cuh", "select_hist.cuh", "decode_wide.cuh", "tip.cuh", "attend_cc.cuh", "attend_mma.cuh", "attend_tc.cuh", "calibrate.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fasa.h")
 
 

@@ -278,8 +278,7 @@ struct CcParams {
   const int32_t* idx;       // [rows][n_keep] kept rows, or null: rows 0 .. n_keep-1 (dense)
   const __nv_bfloat16* q;   // [B][Hq][128], pre-RoPE
   __nv_bfloat16* out;       // [B][Hq][128]
-  float* part;              // [rows][splits][kCcPartStride]
-  uint32_t* counter;        // [rows], zero before the launch; the last CTA of a row leaves it zero
+  float* part;              // [rows][splits][kCcPartStride] split partials (attend_merge_kernel merges them)
   int64_t max_len;
   int32_t len;              // kept indices must lie in [0, len)
   int32_t n_keep;
@@ -298,21 +297,168 @@ struct CcParams {
 };
 
 // Shared memory of attend_cc_kernel: group queries (raw), queries (scaled
-// float32), warp scratch, warp partials; the split merge reuses the partials.
+// float32), warp scratch, warp partials.
 __host__ __device__ constexpr int cc_smem_bytes(int MG) {
   return FASA_MAX_GROUP * kD * 2 + MG * kD * 4 + kCcWarps * cc_warp_scratch(MG) * 4 + kCcWarps * MG * kD * 4 +
          kCcWarps * 2 * kCcStep * kD * 2 + 2 * kNFC * 8;
 }
-constexpr int kCcMaxSplits = (kCcWarps * 4 * kD * 4) / (3 * 16 * 4);  // the merge state fits the MG = 4 partials
+constexpr int kCcMaxSplits = 85;  // splits per row at most (the merge kernel holds a quarter of them in registers)
+
+// Prologue of the split-K attention kernels, in two parts called by all NT
+// threads. cc_row_begin: the angle tables to cs (before the launch-
+// dependency wait, so their constant-bank misses overlap it), then the
+// row's length and kept count. cc_row_queries: the group's G pre-RoPE
+// queries to qraw and the rotated, scaled queries qs [MG][128]
+// (cc_queries; rows h >= G zero); varlen rows rotate at their own length
+// with theta_i from the table, unless the queries come rotated. A kernel may
+// start its first row loads between the two.
+template <int NT>
+__device__ __forceinline__ void cc_row_begin(const CcParams& p, int row, double* cs, int& len, int& n_keep) {
+  const int tid = threadIdx.x;
+  if (tid < kNFC) {
+    cs[tid] = p.cosv[tid];
+    cs[kNFC + tid] = p.sinv[tid];
+  } else if (tid < kNFC + 2 * p.group) {  // the group's queries to L2 (a hint)
+    prefetch_line_l2(p.q + (int64_t)row * p.group * kD + (tid - kNFC) * 64);
+  }
+  grid_dependency_wait();
+  len = p.len;
+  n_keep = p.n_keep;
+  if (p.seq_len) {
+    len = min(max(__ldg(p.seq_len + row / p.n_kv_heads), 1), p.len);  // range flagged by the fused kernel
+    n_keep = min(max(p.row_keep[row], 0), p.n_keep);
+  }
+}
+
+// kStaged: the caller has copied the queries to qraw (cc_stage_queries) and
+// waited for that copy; otherwise they are loaded here.
+template <int MG, int NT, bool kStaged = false>
+__device__ __forceinline__ void cc_row_queries(const CcParams& p, int row, int len, __nv_bfloat16* qraw, double* cs,
+                                               float* qs) {
+  const int tid = threadIdx.x;
+  const int G = p.group;
+  if (!kStaged) {
+    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
+    for (int c = tid; c < G * kD / 8; c += NT) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
+  }
+  if (p.seq_len && tid < kNFC) {  // the query of sequence b sits at position len
+    double sn = 0.0, cn = 1.0;
+    if (!p.q_prerot) sincos((double)len * cs[tid], &sn, &cn);
+    cs[tid] = cn;
+    cs[kNFC + tid] = sn;
+  }
+  __syncthreads();
+  cc_queries(qraw, G, MG, cs, cs + kNFC, qs, tid, NT);
+  __syncthreads();
+}
+
+// The group's G query rows to qraw with 16-byte cp.async, committed as one
+// group (so that they can be issued ahead of the row loads and waited for
+// on their own).
+template <int NT>
+__device__ __forceinline__ void cc_stage_queries(const CcParams& p, int row, __nv_bfloat16* qraw) {
+  const int G = p.group;
+  const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
+  for (int c = threadIdx.x; c < G * kD / 8; c += NT) cp_async16(reinterpret_cast<uint4*>(qraw) + c, qsrc + c);
+  cp_async_commit();
+}
+
+// Split merge of the split-K attention: a kernel of its own, launched after
+// the attention (its grid's completion orders the partials before the
+// reads, so there is no ticket or fence). Grid (G, rows), kMgThreads
+// threads: CTA (h, row) merges head h of the row. Warp w takes a contiguous
+// quarter of the splits; lane l owns dims 4l .. 4l+3. Every warp forms the
+// head's maximum M over all splits, the weights w_s = 2^(m_s - M) and the
+// denominator sum_s w_s l_s by one fixed shuffle tree (so all warps agree
+// bit for bit); the warps' weighted sums of o, each in split order, are
+// added in warp order and divided by the denominator.
+constexpr int kMgThreads = 128;
+constexpr int kMgWarps = kMgThreads / 32;
+constexpr int kMgMaxPer = (kCcMaxSplits + kMgWarps - 1) / kMgWarps;  // splits per warp, at most
+
+struct MergeParams {
+  const float* part;   // [rows][splits][kCcPartStride]: m[16], l[16], o[16][128]
+  __nv_bfloat16* out;  // [rows][G][128]
+  int32_t splits;      // 2 .. kCcMaxSplits
+  int32_t group;
+};
+
+__global__ void __launch_bounds__(kMgThreads) attend_merge_kernel(const MergeParams p) {
+  __shared__ float ws[kMgWarps][kCcMaxSplits];
+  __shared__ float4 acc[kMgWarps][32];
+  const int h = blockIdx.x, row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = p.splits;
+  const float* rp = p.part + (int64_t)row * S * kCcPartStride;
+  grid_dependency_wait();
+  const int per = (S + kMgWarps - 1) / kMgWarps;
+  const int s0 = min(S, warp * per), n = min(S, s0 + per) - s0;
+  // the warp's splits' o for the lane's 4 dims, all loads in flight
+  float4 v[kMgMaxPer];
+#pragma unroll
+  for (int i = 0; i < kMgMaxPer; ++i)
+    if (i < n) v[i] = __ldcg(reinterpret_cast<const float4*>(rp + (int64_t)(s0 + i) * kCcPartStride + 32 + h * kD) + lane);
+  // m and l of every split, lanes over the splits
+  constexpr int kLanesPer = (kCcMaxSplits + 31) / 32;
+  float m[kLanesPer], l[kLanesPer];
+#pragma unroll
+  for (int i = 0; i < kLanesPer; ++i) {
+    const int sp = lane + 32 * i;
+    m[i] = sp < S ? __ldcg(rp + (int64_t)sp * kCcPartStride + h) : -INFINITY;
+    l[i] = sp < S ? __ldcg(rp + (int64_t)sp * kCcPartStride + 16 + h) : 0.0f;
+  }
+  float M = m[0];
+#pragma unroll
+  for (int i = 1; i < kLanesPer; ++i) M = fmaxf(M, m[i]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+  float den = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kLanesPer; ++i) {
+    const int sp = lane + 32 * i;
+    const float w = (m[i] == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(m[i] - M);
+    if (sp < S) ws[warp][sp] = w;
+    den += w * l[i];
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, off);
+  __syncwarp();
+  float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < kMgMaxPer; ++i)
+    if (i < n) {
+      const float w = ws[warp][s0 + i];
+      a.x = __fmaf_rn(w, v[i].x, a.x);
+      a.y = __fmaf_rn(w, v[i].y, a.y);
+      a.z = __fmaf_rn(w, v[i].z, a.z);
+      a.w = __fmaf_rn(w, v[i].w, a.w);
+    }
+  acc[warp][lane] = a;
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = acc[0][lane];
+#pragma unroll
+    for (int w = 1; w < kMgWarps; ++w) {
+      const float4 b = acc[w][lane];
+      t.x += b.x;
+      t.y += b.y;
+      t.z += b.z;
+      t.w += b.w;
+    }
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(p.out + ((int64_t)row * p.group + h) * kD + 4 * lane);
+    o2[0] = __floats2bfloat162_rn(den > 0.0f ? t.x / den : 0.0f, den > 0.0f ? t.y / den : 0.0f);
+    o2[1] = __floats2bfloat162_rn(den > 0.0f ? t.z / den : 0.0f, den > 0.0f ? t.w / den : 0.0f);
+  }
+}
 
 // Split-K attention over a row's kept list (or all its rows): grid
 // (splits, rows); CTA `split` takes list positions [split*slice, ...), its
-// 8 warps contiguous eighths of them; the warps merge in shared memory, the
-// CTA writes its partial (m, l, o) and the row's last CTA (atomic ticket, no
-// waiting) merges the splits in a fixed order and writes the output.
+// 8 warps contiguous eighths of them; the warps merge in shared memory and
+// the CTA writes its partial (m, l, o), or with one split the output
+// (attend_merge_kernel merges the partials).
 template <int MG>
 __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(const CcParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
   float* qs = reinterpret_cast<float*>(smem + FASA_MAX_GROUP * kD * 2);
   float* wsall = qs + MG * kD;
@@ -320,35 +466,11 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
   __nv_bfloat16* vball = reinterpret_cast<__nv_bfloat16*>(mo + kCcWarps * MG * kD);
   double* cs = reinterpret_cast<double*>(vball + kCcWarps * 2 * kCcStep * kD);
   const int split = blockIdx.x, row = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = p.group;
-  // the angle table from the parameters, before the wait (its constant-bank
-  // misses overlap it); varlen rows take theta_i and rotate on the device
-  if (tid < kNFC) {
-    cs[tid] = p.cosv[tid];
-    cs[kNFC + tid] = p.sinv[tid];
-  } else if (tid < kNFC + 2 * G) {  // the group's queries to L2 (a hint)
-    prefetch_line_l2(p.q + (int64_t)row * G * kD + (tid - kNFC) * 64);
-  }
-  grid_dependency_wait();
-  int len = p.len, n_keep = p.n_keep;  // the row's length and kept count
-  if (p.seq_len) {
-    len = min(max(__ldg(p.seq_len + row / p.n_kv_heads), 1), p.len);  // range flagged by the fused kernel
-    n_keep = min(max(p.row_keep[row], 0), p.n_keep);
-  }
-  {
-    const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)row * G * kD);
-    for (int c = tid; c < G * kD / 8; c += kCcThreads) reinterpret_cast<uint4*>(qraw)[c] = __ldg(qsrc + c);
-    if (p.seq_len && tid < kNFC) {  // the query of sequence b sits at position len
-      double sn = 0.0, cn = 1.0;
-      if (!p.q_prerot) sincos((double)len * cs[tid], &sn, &cn);
-      cs[tid] = cn;
-      cs[kNFC + tid] = sn;
-    }
-  }
-  __syncthreads();
-  cc_queries(qraw, G, MG, cs, cs + kNFC, qs, tid, kCcThreads);
-  __syncthreads();
+  int len, n_keep;  // the row's length and kept count
+  cc_row_begin<kCcThreads>(p, row, cs, len, n_keep);
+  cc_row_queries<MG, kCcThreads>(p, row, len, qraw, cs, qs);
   float* ws = wsall + warp * cc_warp_scratch(MG);
   CcAcc<MG> acc;
   cc_init<MG>(acc, ws, lane);
@@ -368,6 +490,7 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
     }
     return paged ? paged_row(p.pm, row / p.n_kv_heads, row % p.n_kv_heads, t) : t;
   }, j0, j1, qs, ws, vball + warp * 2 * kCcStep * kD, lane);
+  grid_dependents_launch();  // the merge (or the next kernel) may start its prologue on SMs this grid frees
   __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
   float* pp = p.part + ((int64_t)row * p.splits + split) * kCcPartStride;
   const bool single = p.splits == 1;
@@ -382,55 +505,6 @@ __global__ void __launch_bounds__(kCcThreads, MG <= 8 ? 2 : 1) attend_cc_kernel(
       }
     }
   });
-  if (single) return;
-  // the row's last CTA merges all splits
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(p.counter + row, 1u) == (uint32_t)(p.splits - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* rp = p.part + (int64_t)row * p.splits * kCcPartStride;
-  float* sm_m = mo;                        // [splits][16]
-  float* sm_l = sm_m + p.splits * 16;      // [splits][16]
-  float* sm_w = sm_l + p.splits * 16;      // [splits][16] weights
-  float* sm_den = sm_w + p.splits * 16;    // [16]
-  for (int i = tid; i < p.splits * 16; i += kCcThreads) {
-    sm_m[i] = __ldcg(rp + (i / 16) * kCcPartStride + i % 16);
-    sm_l[i] = __ldcg(rp + (i / 16) * kCcPartStride + 16 + i % 16);
-  }
-  __syncthreads();
-  if (tid < 16) {
-    float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, sm_m[s * 16 + tid]);
-    float den = 0.0f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float ms = sm_m[s * 16 + tid];
-      const float w = (ms == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(ms - M);
-      sm_w[s * 16 + tid] = w;
-      den += w * sm_l[s * 16 + tid];
-    }
-    sm_den[tid] = den;
-  }
-  __syncthreads();
-  for (int e = tid; e < G * kD; e += kCcThreads) {
-    const int h = e / kD;
-    float num = 0.0f;
-    int s = 0;
-    for (; s + 4 <= p.splits; s += 4) {
-      const float v0 = __ldcg(rp + (s + 0) * kCcPartStride + 32 + e);
-      const float v1 = __ldcg(rp + (s + 1) * kCcPartStride + 32 + e);
-      const float v2 = __ldcg(rp + (s + 2) * kCcPartStride + 32 + e);
-      const float v3 = __ldcg(rp + (s + 3) * kCcPartStride + 32 + e);
-      num += sm_w[(s + 0) * 16 + h] * v0 + sm_w[(s + 1) * 16 + h] * v1 + sm_w[(s + 2) * 16 + h] * v2 +
-             sm_w[(s + 3) * 16 + h] * v3;
-    }
-    for (; s < p.splits; ++s) num += sm_w[s * 16 + h] * __ldcg(rp + s * kCcPartStride + 32 + e);
-    const float den = sm_den[h];
-    out[e] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
-  }
-  if (tid == 0) p.counter[row] = 0u;
 }
 
 }  // namespace fasa

@@ -15,6 +15,7 @@
 #include "select_attend.cuh"
 #include "select_hist.cuh"
 #include "attend_cc.cuh"
+#include "attend_mma.cuh"
 #include "attend_tc.cuh"
 #include "decode_wide.cuh"
 #include "calibrate.cuh"
@@ -588,35 +589,60 @@ fasa_status launch_cal_scores(const fasa_cache* c, int32_t len, const void* q_wi
   return cuda_status(cudaGetLastError());
 }
 
-// Split-K attention (attend_cc_kernel) of every row over its kept list idx
-// [rows][n_keep], or over rows 0 .. n_keep-1 when idx is null (the dense
-// decode); every CTA forms its group's queries from q. part [rows][splits_max]
-// [kCcPartStride] holds the split partials; counter [rows] must be zero (the
-// kernel leaves it zero).
-template <int MG>
-fasa_status launch_attend_t(CcParams& ap, int rows, int splits_max, const DevInfo& d, cudaStream_t st) {
-  auto kern = attend_cc_kernel<MG>;
-  const int smem = cc_smem_bytes(MG);
+// Split-K attention of every row over its kept list idx [rows][n_keep], or
+// over rows 0 .. n_keep-1 when idx is null (the dense decode): the
+// tensor-core kernel (attend_mma_kernel) for groups of up to 8 query heads,
+// the CUDA-core one (attend_cc_kernel) for larger groups. Every CTA forms its
+// group's queries from q. A row whose list is split over several CTAs leaves
+// partials in part [rows][splits_max][kCcPartStride], and a second launch
+// (attend_merge_kernel) merges them.
+struct AttendKernel {
+  const void* fn;
+  int threads, smem;
+};
+AttendKernel attend_kernel(int group) {
+  if (group <= 8) return {(const void*)attend_mma_kernel, kAmThreads, am_smem_bytes()};
+  return {(const void*)attend_cc_kernel<16>, kCcThreads, cc_smem_bytes(16)};
+}
+
+// Splits per row of the attention over n_keep list positions: one wave of
+// resident CTAs at most, each with at least one step per warp; sets the
+// slice (list positions per CTA) too.
+fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const DevInfo& d, int* splits, int* slice) {
+  const AttendKernel k = attend_kernel(group);
   int per_sm = 0;
-  fasa_status s = cached_int((const void*)kern, 7, &per_sm, [&](int* v) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kern, kCcThreads, (size_t)smem);
+  fasa_status s = cached_int(k.fn, 7, &per_sm, [&](int* v) {
+    cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, k.fn, k.threads, (size_t)k.smem);
     return cuda_status(e);
   });
   if (s != FASA_OK) return s;
   per_sm = std::max(1, per_sm);
-  // one wave of resident CTAs at most, each with at least one step per warp
   constexpr int kUnit = kCcWarps * kCcStep;
-  const int64_t units = ceil_div(ap.n_keep, kUnit);
-  int64_t splits = std::min<int64_t>(units, std::max<int64_t>(1, (int64_t)per_sm * d.sms / rows));
-  splits = std::min<int64_t>(splits, std::min<int64_t>(splits_max, kCcMaxSplits));
-  ap.slice = (int)(ceil_div(units, splits) * kUnit);
-  ap.splits = (int)ceil_div(ap.n_keep, ap.slice);
-  return launch_pdl(kern, dim3((unsigned)ap.splits, (unsigned)rows, 1), kCcThreads, (size_t)smem, st, ap);
+  const int64_t units = std::max<int64_t>(1, ceil_div(n_keep, kUnit));
+  int64_t sp = std::min<int64_t>(units, std::max<int64_t>(1, (int64_t)per_sm * d.sms / rows));
+  sp = std::min<int64_t>(sp, std::min<int64_t>(splits_max, kCcMaxSplits));
+  sp = std::max<int64_t>(sp, 1);
+  *slice = (int)(ceil_div(units, sp) * kUnit);
+  *splits = (int)ceil_div(std::max(n_keep, 1), *slice);
+  return FASA_OK;
+}
+
+fasa_status launch_attend_k(CcParams& ap, int rows, int splits_max, const DevInfo& d, cudaStream_t st) {
+  fasa_status s = attend_split(ap.group, rows, ap.n_keep, splits_max, d, &ap.splits, &ap.slice);
+  if (s != FASA_OK) return s;
+  const dim3 grid((unsigned)ap.splits, (unsigned)rows, 1);
+  if (ap.group <= 8)
+    s = launch_pdl(attend_mma_kernel, grid, kAmThreads, (size_t)am_smem_bytes(), st, ap);
+  else
+    s = launch_pdl(attend_cc_kernel<16>, grid, kCcThreads, (size_t)cc_smem_bytes(16), st, ap);
+  if (s != FASA_OK || ap.splits == 1) return s;
+  MergeParams mp{ap.part, ap.out, ap.splits, ap.group};
+  return launch_pdl(attend_merge_kernel, dim3((unsigned)ap.group, (unsigned)rows, 1), kMgThreads, 0, st, mp);
 }
 
 fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* out, const int32_t* idx,
-                          const void* q, int32_t q_pos, float* part, uint32_t* counter, int splits_max,
+                          const void* q, int32_t q_pos, float* part, int splits_max,
                           const DevInfo& d, cudaStream_t st, const fasa_varlen* vl = nullptr,
                           const int32_t* row_keep = nullptr, const fasa_paged* pg = nullptr) {
   const int rows = c->batch * c->n_kv_heads;
@@ -627,7 +653,6 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
   ap.q = static_cast<const __nv_bfloat16*>(q);
   ap.out = static_cast<__nv_bfloat16*>(out);
   ap.part = part;
-  ap.counter = counter;
   ap.max_len = c->max_len;
   ap.len = len;
   ap.n_keep = n_keep;
@@ -642,9 +667,7 @@ fasa_status launch_attend(const fasa_cache* c, int32_t len, int n_keep, void* ou
   } else {
     fill_query_angle(ap.cosv, ap.sinv, c->rope_base, q_pos);
   }
-  if (ap.group <= 4) return launch_attend_t<4>(ap, rows, splits_max, d, st);
-  if (ap.group <= 8) return launch_attend_t<8>(ap, rows, splits_max, d, st);
-  return launch_attend_t<16>(ap, rows, splits_max, d, st);
+  return launch_attend_k(ap, rows, splits_max, d, st);
 }
 
 // The decode's attention over the kept lists in the workspace.
@@ -652,8 +675,8 @@ fasa_status launch_attend_ws(const fasa_cache* c, int32_t len, int keff, const v
                              const DecodeWs& w, char* base, const DevInfo& d, cudaStream_t st,
                              const fasa_varlen* vl = nullptr, const fasa_paged* pg = nullptr) {
   return launch_attend(c, len, keff, out, reinterpret_cast<const int32_t*>(base + w.idx), q, q_pos,
-                       reinterpret_cast<float*>(base + w.part), reinterpret_cast<uint32_t*>(base + w.att_cnt),
-                       w.splits_max, d, st, vl, reinterpret_cast<const int32_t*>(base + w.rowk), pg);
+                       reinterpret_cast<float*>(base + w.part), w.splits_max, d, st, vl,
+                       reinterpret_cast<const int32_t*>(base + w.rowk), pg);
 }
 
 // Dense decode workspace: att_cnt [rows] u32 (zero between calls) | part
@@ -1069,12 +1092,28 @@ int32_t fasa_decode_path(const fasa_cache* c, int32_t len, int32_t k) {
 int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
   const int32_t path = fasa_decode_path(c, len, k);
   if (path < 0) return path;
-  if (path == FASA_DECODE_STAGED) return 4;
   DevInfo d;
   if (device_info(&d) != FASA_OK) return -FASA_ERR_CUDA;
+  // the split-K attention of bf16 caches adds the split merge when a row's
+  // kept list spans several CTAs
+  auto merge = [&]() -> int32_t {
+    if (c->dtype != FASA_BF16) return 0;
+    int splits = 1, slice = 0;
+    const DecodeWs w = decode_layout(c, len, k);
+    if (attend_split(c->n_q_heads / c->n_kv_heads, c->batch * c->n_kv_heads, std::min(k, len), w.splits_max, d,
+                     &splits, &slice) != FASA_OK)
+      return -1;
+    return splits > 1 ? 1 : 0;
+  };
+  if (path == FASA_DECODE_STAGED) {
+    const int32_t m = merge();
+    return m < 0 ? -FASA_ERR_CUDA : 4 + m;
+  }
   WidePlan pl;
   if (!wide_plan(c, len, std::min(k, len), d, &pl)) return -FASA_ERR_UNSUPPORTED;
-  return pl.direct ? 1 : 2;
+  if (pl.direct) return 1;
+  const int32_t m = merge();
+  return m < 0 ? -FASA_ERR_CUDA : 2 + m;
 }
 
 }  // extern "C"
@@ -1258,8 +1297,8 @@ fasa_status fasa_dense_decode(const fasa_cache* c, int32_t len, const void* q, i
     DevInfo d;
     if ((s = device_info(&d)) != FASA_OK) return s;
     char* base = static_cast<char*>(workspace);
-    return launch_attend(c, len, len, out, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part),
-                         reinterpret_cast<uint32_t*>(base + w.att_cnt), w.splits_max, d, stream);
+    return launch_attend(c, len, len, out, nullptr, q, q_pos, reinterpret_cast<float*>(base + w.part), w.splits_max,
+                         d, stream);
   }
   // the f32 dense kernel stages K and V with bulk copies, which are kept to
   // device memory: a FASA-M cache (host-resident K/V) is refused here
