@@ -262,11 +262,12 @@ size_t fasa_decode_workspace_bytes(const fasa_cache* cache, int32_t len, int32_t
  *  workspace : caller-owned device memory of at least
  *            fasa_decode_workspace_bytes(cache, len, k) bytes, 256-byte aligned
  *            (required whichever plan runs). Zero it once after allocating it
- *            (e.g. cudaMemsetAsync): its first 12 * B * Hkv bytes hold
- *            per-row semaphores, and the staged plan keeps per-row
- *            histograms, counters and tickets further in; all must be zero
- *            when a call starts, and every call leaves them zero again. The
- *            rest is scratch. After a
+ *            (e.g. cudaMemsetAsync): it starts with per-row semaphores,
+ *            histograms, counters and tickets, at offsets that depend on
+ *            B * Hkv only, which must be zero when a call starts and which
+ *            every call leaves zero again; the rest is scratch. So one
+ *            workspace sized for the largest len and k serves calls at any
+ *            smaller len and k on the same cache. After a
  *            call that ended in an error (a CUDA error, FASA_ERR_TIMEOUT),
  *            zero it again. A semaphore found non-zero is reported as
  *            FASA_ERR_WORKSPACE in the device status word; no access then

@@ -203,6 +203,36 @@ __device__ __forceinline__ void am_step(AmState& st, const AmQuery& Q, uint32_t 
   }
 }
 
+// Merge of NW warps' states in shared memory: wm, wl [NW][8] the maxima and
+// sums, wo(w) warp w's o [8][128]. Threads tid < NW * 8 form the weight of
+// (warp w, head h) = 2^(m_wh - M_h) into wf [NW][8]; after a barrier every
+// output element e = h * 128 + d of the G heads (e = tid, tid + NT, ...)
+// sums its warps' weighted o and l in warp order and calls emit(e, O, L).
+// Called by all NT threads after a barrier that follows the state writes.
+template <int NW, int NT, typename WoAt, typename Emit>
+__device__ __forceinline__ void am_merge_warps(const float* wm, const float* wl, float* wf, WoAt wo, int G, Emit emit) {
+  const int tid = threadIdx.x;
+  if (tid < NW * 8) {
+    const int h = tid & 7;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w * 8 + h]);
+    wf[tid] = (wm[tid] == -INFINITY) ? 0.0f : exp2f(wm[tid] - M);
+  }
+  __syncthreads();
+  for (int e = tid; e < G * kD; e += NT) {
+    const int h = e / kD;
+    float L = 0.0f, O = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = wf[w * 8 + h];
+      L += f * wl[w * 8 + h];
+      O += f * wo(w)[e];
+    }
+    emit(e, O, L);
+  }
+}
+
 // Split-K attention over a row's kept list (or all its rows) for G <= 8:
 // grid (splits, rows); CTA `split` takes list positions [split*slice, ...),
 // its 4 warps contiguous quarters of them in steps of 16 rows; the warps
@@ -314,10 +344,11 @@ __global__ void __launch_bounds__(kAmThreads, 2) attend_mma_kernel(const CcParam
   st.l += __shfl_xor_sync(0xFFFFFFFFu, st.l, 2);
   __syncthreads();  // every warp is past its ring: the states reuse it
 
-  // warp states: m, l [kAmWarps][8], o [kAmWarps][8][128]
+  // warp states: m, l [kAmWarps][8], merge weights [kAmWarps][8], o [kAmWarps][8][128]
   float* wm = reinterpret_cast<float*>(ring);
   float* wl = wm + kAmWarps * 8;
-  float* wo = wl + kAmWarps * 8;
+  float* wf = wl + kAmWarps * 8;
+  float* wo = wf + kAmWarps * 8;
   const int g = lane >> 2, q = lane & 3;
   if (q == 0) {
     wm[warp * 8 + g] = st.m;
@@ -331,29 +362,22 @@ __global__ void __launch_bounds__(kAmThreads, 2) attend_mma_kernel(const CcParam
   __nv_bfloat16* out = p.out + (int64_t)row * G * kD;
   float* pp = p.part + ((int64_t)row * p.splits + split) * kCcPartStride;
   const bool single = p.splits == 1;
-  for (int e = tid; e < G * kD; e += kAmThreads) {
-    const int h = e / kD, d = e % kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kAmWarps; ++w) M = fmaxf(M, wm[w * 8 + h]);
-    float L = 0.0f, O = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kAmWarps; ++w) {
-      const float mw = wm[w * 8 + h];
-      const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
-      L += f * wl[w * 8 + h];
-      O += f * wo[(w * 8 + h) * kD + d];
-    }
+  am_merge_warps<kAmWarps, kAmThreads>(wm, wl, wf, [&](int w) { return wo + w * 8 * kD; }, G,
+                                       [&](int e, float O, float L) {
     if (single) {
       out[e] = __float2bfloat16_rn(L > 0.0f ? O / L : 0.0f);
     } else {
       pp[32 + e] = O;
-      if (d == 0) {
+      if (e % kD == 0) {  // the head's maximum and sum
+        const int h = e / kD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAmWarps; ++w) M = fmaxf(M, wm[w * 8 + h]);
         pp[h] = M;
         pp[16 + h] = L;
       }
     }
-  }
+  });
 }
 
 }  // namespace fasa

@@ -474,11 +474,15 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
 }
 
 // The plan fasa_decode picks by itself: the fused plan while each row can
-// have about eight or more SMs (measured on B200: c2, 8 rows, 21 us against
-// 35 us staged; 16 rows even; 64 and 512 rows 20% faster staged, where the
-// fused plan's per-row resolving CTAs and two launches no longer pay).
-inline bool fused_preferred(const fasa_cache* c, const DevInfo& d) {
-  return (int64_t)c->batch * c->n_kv_heads * 8 <= d.sms;
+// have about eight or more SMs and its budget stays small enough for the
+// one resolving CTA of a row to select it quickly (measured on B200: c2, 8
+// rows, 21.3 us fused against 35 us staged at k 256, 27.9 against 30.7 at
+// k 1024; 64 and 512 rows 20% faster staged, where the fused plan's
+// per-row resolving CTAs no longer pay; 16 rows at k 6193 58.7 us fused
+// against 52.2 staged).
+constexpr int kFusedMaxKeep = 1024;
+inline bool fused_preferred(const fasa_cache* c, int keff, const DevInfo& d) {
+  return (int64_t)c->batch * c->n_kv_heads * 8 <= d.sms && keff <= kFusedMaxKeep;
 }
 
 template <int LPT, int MG>
@@ -500,17 +504,14 @@ fasa_status launch_wide_t(const WideParams& p, int rows, const WidePlan& pl, cud
 }
 
 // Decode workspace, each part 256-byte aligned:
-//   sem [rows] u64 | att_cnt [rows] u32          (zero between calls: every
-//                                                 call leaves them zero)
+//   zero between calls (every call leaves them zero), at offsets fixed by
+//   the row count: sem [rows] u64 | att_cnt [rows] u32 |
+//     hist [rows][4096] u32, cnt [rows], thr [rows][2], rdone [rows] (staged plan) |
 //   scores [rows][ld] f32 (ld = len rounded up to 32), or, in the fused plan,
 //     the CTAs' published candidates [rows][len + len/64 + 64] u32x2 |
 //   keys [rows][len] u32 (fused plan: every token's score key) | rowk [rows] i32 (varlen: each row's k_eff) |
-//   (staged plan, zero between calls) hist [rows][4096] u32, cnt [rows], thr [rows][2], rdone [rows] |
-//   hist [rows][4096] u32 | cand_cnt [rows] u32 | bitmap [rows][ceil(len/32)] u32 |
-//   cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 | idx [rows][k_eff] i32 |
-//   part [rows][splits_max][kCcPartStride] f32
-// The staged plan clears the first two parts and hist, cand_cnt at the start
-// of every call; the wide plan relies on them being zero.
+//   bitmap [rows][ceil(len/32)] u32 | cand_idx [rows][cap] i32 | cand_key [rows][cap] u32 |
+//   idx [rows][k_eff] i32 | part [rows][splits_max][kCcPartStride] f32
 constexpr int kAssumedMaxSms = 256;  // sizes the split-K partials for any GPU
 constexpr int kAttMaxPerSm = 4;      // attention CTAs resident per SM, an upper bound
 constexpr int kAttUnit = kCcWarps * kCcStep;  // kept rows per CTA step of the attention
@@ -537,16 +538,19 @@ DecodeWs decode_layout(const fasa_cache* c, int32_t len, int32_t k) {
   w.cap = (int)std::min<size_t>(std::max<size_t>(L, 1), 8192);
   w.splits_max = att_splits((int)rows, std::max(keff, 1), kAssumedMaxSms, kAttMaxPerSm);
   w.ld = (int64_t)((L + 31) / 32 * 32);
+  // the parts that must be zero between calls first, at offsets that depend
+  // on the row count only: a workspace sized for the largest len and k
+  // serves calls at any smaller len and k
   w.sem = 0;
   w.att_cnt = rows * 8;
-  w.scores = al256(w.att_cnt + rows * 4);
-  w.keys = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
-  w.rowk = al256(w.keys + rows * L * 4);
-  w.hist = al256(w.rowk + rows * 4);
+  w.hist = al256(w.att_cnt + rows * 4);
   w.cnt = w.hist + rows * kHistBins * 4;
   w.thr = w.cnt + rows * 4;
   w.rdone = w.thr + rows * 8;
-  w.bitmap = al256(w.rdone + rows * 4);
+  w.scores = al256(w.rdone + rows * 4);
+  w.keys = al256(w.scores + rows * std::max<size_t>((size_t)w.ld * 4, (size_t)wide_region_slots((int64_t)L) * 8));
+  w.rowk = al256(w.keys + rows * L * 4);
+  w.bitmap = al256(w.rowk + rows * 4);
   w.cand = al256(w.bitmap + rows * (size_t)w.words * 4);
   w.ckey = al256(w.cand + rows * (size_t)w.cap * 4);
   w.idx = al256(w.ckey + rows * (size_t)w.cap * 4);
@@ -983,7 +987,7 @@ fasa_status fasa_decode(const fasa_cache* c, int32_t len, const void* q, int32_t
   const int keff = std::min(k, len);
   const int path = g_decode_path.load();
   char* base = static_cast<char*>(workspace);
-  if ((path == FASA_DECODE_AUTO && fused_preferred(c, d)) || path == FASA_DECODE_FUSED) {
+  if ((path == FASA_DECODE_AUTO && fused_preferred(c, keff, d)) || path == FASA_DECODE_FUSED) {
     WidePlan pl;
     if (wide_plan(c, len, keff, d, &pl)) return launch_wide(c, len, q, q_pos, keff, out, idx_out, w, base, pl, d, stream);
     if (path == FASA_DECODE_FUSED) return FASA_ERR_UNSUPPORTED;
@@ -1086,7 +1090,8 @@ int32_t fasa_decode_path(const fasa_cache* c, int32_t len, int32_t k) {
   const int path = g_decode_path.load();
   if (path != FASA_DECODE_AUTO) return path;
   WidePlan pl;
-  return fused_preferred(c, d) && wide_plan(c, len, std::min(k, len), d, &pl) ? FASA_DECODE_FUSED : FASA_DECODE_STAGED;
+  const int keff = std::min(k, len);
+  return fused_preferred(c, keff, d) && wide_plan(c, len, keff, d, &pl) ? FASA_DECODE_FUSED : FASA_DECODE_STAGED;
 }
 
 int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
@@ -1274,8 +1279,6 @@ fasa_status fasa_decode_static_scratch(const fasa_cache* c, int32_t len, const v
   // call leaves them zero; clear them anyway, so that a call that ended in an
   // error cannot poison the next
   if ((s = cuda_status(cudaMemsetAsync(ws, 0, w.scores, stream))) != FASA_OK) return s;
-  if ((s = cuda_status(cudaMemsetAsync(static_cast<char*>(ws) + w.hist, 0, w.bitmap - w.hist, stream))) != FASA_OK)
-    return s;
   return fasa_decode(c, len, q, q_pos, k, out, idx_out, ws, FASA_STATIC_SCRATCH_BYTES, stream);
 }
 

@@ -325,6 +325,10 @@ def test_decode_path_setting_and_choice():
     wl = C["c2"].replace(ctx_len=4096)
     _, cache, _ = U.build(wl)
     assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_FUSED
+    # a budget above 1024 takes the staged plan
+    assert F.fasa_decode_path(cache, wl.ctx_len, 1024) == F.DECODE_FUSED
+    assert F.fasa_decode_path(cache, wl.ctx_len, 1025) == F.DECODE_STAGED
+    assert F.fasa_decode_launches(cache, wl.ctx_len, 1025) in (4, 5)
     F.fasa_set_decode_path(F.DECODE_STAGED)
     try:
         assert F.fasa_decode_path(cache, wl.ctx_len, wl.k) == F.DECODE_STAGED
@@ -332,6 +336,32 @@ def test_decode_path_setting_and_choice():
         F.fasa_set_decode_path(F.DECODE_AUTO)
     with pytest.raises(F.FasaError):
         F.fasa_set_decode_path(7)
+
+
+def test_one_workspace_serves_smaller_lengths_and_budgets():
+    """A workspace zeroed once and sized for the largest len and k serves
+    decodes at smaller len and k on the same cache, in either plan: the parts
+    that must stay zero between calls sit at offsets fixed by the row count.
+    Each decode equals the same decode with a fresh workspace."""
+    wl = C["c2"].replace(name="wsr", batch=2, ctx_len=3000)
+    _, cache, q = U.build(wl)
+    ws = F.fasa_decode_workspace(cache, 3000, 700)
+    rows = wl.batch * wl.n_kv_heads
+    for path in (F.DECODE_STAGED, F.DECODE_FUSED):
+        F.fasa_set_decode_path(path)
+        try:
+            for L, k in [(3000, 700), (1000, 190), (2500, 300), (640, 640), (3000, 257), (3000, 700)]:
+                idx = torch.empty((wl.batch, wl.n_kv_heads, k), dtype=torch.int32, device="cuda")
+                out = F.fasa_decode(cache, L, q, L, k, idx_out=idx, workspace=ws)
+                idx_f = torch.empty_like(idx)
+                out_f = F.fasa_decode(cache, L, q, L, k, idx_out=idx_f, workspace=F.fasa_decode_workspace(cache, L, k))
+                torch.cuda.synchronize()
+                assert F.fasa_device_status(clear=True) == 0, (path, L, k)
+                assert torch.equal(idx, idx_f), (path, L, k)
+                assert torch.equal(out, out_f), (path, L, k)
+                assert idx.reshape(rows, k).max().item() < L
+        finally:
+            F.fasa_set_decode_path(F.DECODE_AUTO)
 
 
 def test_fused_decode_rejects_f32_when_forced():
