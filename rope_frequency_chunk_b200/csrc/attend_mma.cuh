@@ -43,18 +43,18 @@
 
 namespace fasa {
 
-constexpr int kAmWarps = 4;
-constexpr int kAmThreads = kAmWarps * 32;
 constexpr int kAmStages = 3;                    // steps in flight per warp
 constexpr int kAmRows = 16;                     // rows per warp step
 constexpr int kAmTile = kAmRows * kD * 2;       // bytes of one K (or V) step
-static_assert(kAmWarps * kAmRows == kCcWarps * kCcStep, "the attention launchers share one list unit");
+// A CTA has 4 warps, two CTAs per SM; with many rows and one split each, 2
+// warps, four CTAs per SM (one wave of rows, twice the steps per warp).
+static_assert(4 * kAmRows == kCcWarps * kCcStep, "the attention launchers share one list unit");
 
-// Shared memory: raw queries, scaled queries [8][128] f32, angle tables,
+// Shared memory: raw queries [8][128] bf16, scaled queries [8][128] f32, angle tables,
 // then the per-warp rings (K step, V step per stage); the warps' states
 // reuse the rings after the last step.
-__host__ __device__ constexpr int am_smem_bytes() {
-  return FASA_MAX_GROUP * kD * 2 + 8 * kD * 4 + 2 * kNFC * 8 + kAmWarps * kAmStages * 2 * kAmTile;
+__host__ __device__ constexpr int am_smem_bytes(int NW) {
+  return 8 * kD * 2 + 8 * kD * 4 + 2 * kNFC * 8 + NW * kAmStages * 2 * kAmTile;
 }
 
 __device__ __forceinline__ uint32_t am_pack(float lo_elem, float hi_elem) {
@@ -238,10 +238,12 @@ __device__ __forceinline__ void am_merge_warps(const float* wm, const float* wl,
 // its 4 warps contiguous quarters of them in steps of 16 rows; the warps
 // merge in shared memory and the CTA writes its partial (m, l, o), or with
 // one split the output (attend_merge_kernel merges the partials).
-__global__ void __launch_bounds__(kAmThreads, 2) attend_mma_kernel(const CcParams p) {
+template <int NW>
+__global__ void __launch_bounds__(NW * 32, 8 / NW) attend_mma_kernel(const CcParams p) {
+  constexpr int kAmWarps = NW, kAmThreads = NW * 32;
   extern __shared__ __align__(128) unsigned char smem[];
   __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
-  float* qs = reinterpret_cast<float*>(smem + FASA_MAX_GROUP * kD * 2);
+  float* qs = reinterpret_cast<float*>(smem + 8 * kD * 2);  // the raw queries: G <= 8 rows
   double* cs = reinterpret_cast<double*>(qs + 8 * kD);
   unsigned char* ring = reinterpret_cast<unsigned char*>(cs + 2 * kNFC);
   const int split = blockIdx.x, row = blockIdx.y;

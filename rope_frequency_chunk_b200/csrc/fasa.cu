@@ -604,24 +604,32 @@ struct AttendKernel {
   const void* fn;
   int threads, smem;
 };
-AttendKernel attend_kernel(int group) {
-  if (group <= 8) return {(const void*)attend_mma_kernel, kAmThreads, am_smem_bytes()};
-  return {(const void*)attend_cc_kernel<16>, kCcThreads, cc_smem_bytes(16)};
+AttendKernel attend_kernel(int group, int nw) {
+  if (group > 8) return {(const void*)attend_cc_kernel<16>, kCcThreads, cc_smem_bytes(16)};
+  if (nw == 2) return {(const void*)attend_mma_kernel<2>, 64, am_smem_bytes(2)};
+  return {(const void*)attend_mma_kernel<4>, 128, am_smem_bytes(4)};
 }
 
-// Splits per row of the attention over n_keep list positions: one wave of
-// resident CTAs at most, each with at least one step per warp; sets the
-// slice (list positions per CTA) too.
-fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const DevInfo& d, int* splits, int* slice) {
-  const AttendKernel k = attend_kernel(group);
-  int per_sm = 0;
-  fasa_status s = cached_int(k.fn, 7, &per_sm, [&](int* v) {
+fasa_status attend_per_sm(const AttendKernel& k, int* per_sm) {
+  fasa_status s = cached_int(k.fn, 7, per_sm, [&](int* v) {
     cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
     if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, k.fn, k.threads, (size_t)k.smem);
     return cuda_status(e);
   });
+  *per_sm = std::max(1, *per_sm);
+  return s;
+}
+
+// Splits per row of the attention over n_keep list positions: one wave of
+// resident CTAs at most, each with at least one step per warp; sets the
+// slice (list positions per CTA) too. *nw: warps per CTA of the tensor-core
+// kernel, 2 when the rows alone (one split each) would overfill a wave of
+// 4-warp CTAs but fill one of 2-warp CTAs.
+fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const DevInfo& d, int* splits, int* slice,
+                         int* nw) {
+  int per_sm = 0;
+  fasa_status s = attend_per_sm(attend_kernel(group, 4), &per_sm);
   if (s != FASA_OK) return s;
-  per_sm = std::max(1, per_sm);
   constexpr int kUnit = kCcWarps * kCcStep;
   const int64_t units = std::max<int64_t>(1, ceil_div(n_keep, kUnit));
   int64_t sp = std::min<int64_t>(units, std::max<int64_t>(1, (int64_t)per_sm * d.sms / rows));
@@ -629,17 +637,26 @@ fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const 
   sp = std::max<int64_t>(sp, 1);
   *slice = (int)(ceil_div(units, sp) * kUnit);
   *splits = (int)ceil_div(std::max(n_keep, 1), *slice);
+  *nw = 4;
+  if (group <= 8 && *splits == 1 && (int64_t)rows > (int64_t)per_sm * d.sms) {
+    int per_sm2 = 0;
+    if ((s = attend_per_sm(attend_kernel(group, 2), &per_sm2)) != FASA_OK) return s;
+    if ((int64_t)rows <= (int64_t)per_sm2 * d.sms) *nw = 2;
+  }
   return FASA_OK;
 }
 
 fasa_status launch_attend_k(CcParams& ap, int rows, int splits_max, const DevInfo& d, cudaStream_t st) {
-  fasa_status s = attend_split(ap.group, rows, ap.n_keep, splits_max, d, &ap.splits, &ap.slice);
+  int nw = 4;
+  fasa_status s = attend_split(ap.group, rows, ap.n_keep, splits_max, d, &ap.splits, &ap.slice, &nw);
   if (s != FASA_OK) return s;
   const dim3 grid((unsigned)ap.splits, (unsigned)rows, 1);
-  if (ap.group <= 8)
-    s = launch_pdl(attend_mma_kernel, grid, kAmThreads, (size_t)am_smem_bytes(), st, ap);
-  else
+  if (ap.group > 8)
     s = launch_pdl(attend_cc_kernel<16>, grid, kCcThreads, (size_t)cc_smem_bytes(16), st, ap);
+  else if (nw == 2)
+    s = launch_pdl(attend_mma_kernel<2>, grid, 64, (size_t)am_smem_bytes(2), st, ap);
+  else
+    s = launch_pdl(attend_mma_kernel<4>, grid, 128, (size_t)am_smem_bytes(4), st, ap);
   if (s != FASA_OK || ap.splits == 1) return s;
   MergeParams mp{ap.part, ap.out, ap.splits, ap.group};
   return launch_pdl(attend_merge_kernel, dim3((unsigned)ap.group, (unsigned)rows, 1), kMgThreads, 0, st, mp);
@@ -1103,10 +1120,10 @@ int32_t fasa_decode_launches(const fasa_cache* c, int32_t len, int32_t k) {
   // kept list spans several CTAs
   auto merge = [&]() -> int32_t {
     if (c->dtype != FASA_BF16) return 0;
-    int splits = 1, slice = 0;
+    int splits = 1, slice = 0, nw = 4;
     const DecodeWs w = decode_layout(c, len, k);
     if (attend_split(c->n_q_heads / c->n_kv_heads, c->batch * c->n_kv_heads, std::min(k, len), w.splits_max, d,
-                     &splits, &slice) != FASA_OK)
+                     &splits, &slice, &nw) != FASA_OK)
       return -1;
     return splits > 1 ? 1 : 0;
   };
