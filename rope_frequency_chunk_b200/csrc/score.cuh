@@ -206,9 +206,39 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
   if (kHist)
     for (int i = tid; i < kHistBins; i += kScoreThreads) s_hist[i] = 0u;
 
+  // a segment: the CTA's tokens of one row. Its first D ring slots are
+  // requested before the row's coefficients are formed (and, for every
+  // segment after the first, before the previous row's histogram is
+  // flushed), so the stream's first round trip overlaps that work.
+  int row = 0, t0 = 0, n = 0, mine = 0;
+  const char* src = nullptr;
+  auto begin_seg = [&](int64_t seg) {
+    row = (int)(seg / p.len);
+    t0 = (int)(seg % p.len);
+    n = (int)min((int64_t)(p.len - t0), f_end - seg);
+    src = static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
+    const int nblk = (n + S::TPW - 1) / S::TPW;
+    mine = nblk > warp ? (nblk - warp + kScoreWarps - 1) / kScoreWarps : 0;
+  };
+  // warp w takes the steps w, w + kScoreWarps, ... of TPW consecutive tokens
+  auto issue = [&](int j) {
+    if (j < mine) {
+      const int tok = (j * kScoreWarps + warp) * S::TPW + tl;
+      if (tok < n) {
+        unsigned char* slot = ring + (j % D) * R::kSlot + tl * S::ROWB;
+#pragma unroll
+        for (int c = 0; c < S::CPL; ++c)
+          cp_async16(slot + (sub * S::CPL + c) * 16, src + (int64_t)tok * S::ROWB + (sub * S::CPL + c) * 16);
+      }
+    }
+    cp_async_commit();
+  };
+  if (f_beg < f_end) {
+    begin_seg(f_beg);
+#pragma unroll
+    for (int j = 0; j < D; ++j) issue(j);
+  }
   for (int64_t seg = f_beg; seg < f_end;) {
-    const int row = (int)(seg / p.len), t0 = (int)(seg % p.len);
-    const int n = (int)min((int64_t)(p.len - t0), f_end - seg);
     // the row's query coefficients (float64), every thread taking part
     __syncthreads();
     {
@@ -225,25 +255,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
     float qr[S::EPL];
     load_coefs<T, LPT>(qr, s_q, lane);
 
-    // warp w takes the steps w, w + kScoreWarps, ... of TPW consecutive tokens
-    const char* src = static_cast<const char*>(p.sketch) + ((int64_t)row * p.max_len + t0) * S::ROWB;
     float* out = p.scores + (int64_t)row * p.ld + t0;
-    const int nblk = (n + S::TPW - 1) / S::TPW;
-    const int mine = nblk > warp ? (nblk - warp + kScoreWarps - 1) / kScoreWarps : 0;
-    auto issue = [&](int j) {
-      if (j < mine) {
-        const int tok = (j * kScoreWarps + warp) * S::TPW + tl;
-        if (tok < n) {
-          unsigned char* slot = ring + (j % D) * R::kSlot + tl * S::ROWB;
-#pragma unroll
-          for (int c = 0; c < S::CPL; ++c)
-            cp_async16(slot + (sub * S::CPL + c) * 16, src + (int64_t)tok * S::ROWB + (sub * S::CPL + c) * 16);
-        }
-      }
-      cp_async_commit();
-    };
-#pragma unroll
-    for (int j = 0; j < D; ++j) issue(j);
     for (int j = 0; j < mine; ++j) {
       cp_async_wait<D - 1>();
       __syncwarp();
@@ -257,35 +269,43 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const ScorePara
       issue(j + D);
     }
     cp_async_wait<0>();
+    __syncwarp();  // the warp's ring is consumed: the next segment may fill it
+    const int cur_row = row, cur_n = n;
+    const int64_t next = seg + n;
+    if (next < f_end) {
+      begin_seg(next);
+#pragma unroll
+      for (int j = 0; j < D; ++j) issue(j);
+    }
     if (kHist) {
       __syncthreads();
       for (int i = tid; i < kHistBins; i += kScoreThreads) {
         const uint32_t v = s_hist[i];
         if (v) {
-          atomicAdd(p.hist + (int64_t)row * kHistBins + i, v);
+          atomicAdd(p.hist + (int64_t)cur_row * kHistBins + i, v);
           s_hist[i] = 0u;
         }
       }
       if (p.thr) {  // the row's last segment: its threshold bin, once per row
         __threadfence();
         __syncthreads();
-        if (tid == 0) s_last = atomicAdd(p.row_done + row, (uint32_t)n) + (uint32_t)n == (uint32_t)p.len;
+        if (tid == 0) s_last = atomicAdd(p.row_done + cur_row, (uint32_t)cur_n) + (uint32_t)cur_n == (uint32_t)p.len;
         __syncthreads();
         if (s_last) {
           __threadfence();
-          uint32_t* hr = p.hist + (int64_t)row * kHistBins;
+          uint32_t* hr = p.hist + (int64_t)cur_row * kHistBins;
           uint32_t bin, above;
           hist_bin_of_kth<kScoreThreads>([hr](int i) { return __ldcg(hr + i); }, p.n_keep, s_scan, bin, above);
           if (tid == 0) {
-            p.thr[2 * row] = bin;
-            p.thr[2 * row + 1] = above;
-            p.row_done[row] = 0u;
+            p.thr[2 * cur_row] = bin;
+            p.thr[2 * cur_row + 1] = above;
+            p.row_done[cur_row] = 0u;
           }
           for (int i = tid; i < kHistBins; i += kScoreThreads) hr[i] = 0u;  // ready for the next call
         }
       }
     }
-    seg += n;
+    seg = next;
   }
 }
 
