@@ -61,6 +61,9 @@ def default_layers(wl: W.Workload) -> int:
     return n
 
 
+HBM_NOMINAL_GBS = 7700.0  # B200 HBM3e, the HGX figure (context beside the measured peak)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -536,6 +539,7 @@ def run_fasa(args, wl):
             "frac": gbs / world / hbm_peak,
             "traffic": profiled_traffic("decode_wide_kernel", workload_sig(wl, k)) if launches == 1 else None,
             "bytes_per_launch": per_layer_bytes, "peak_kind": peak_kind, "us_per_launch": us_layer,
+            "nominal_peak": HBM_NOMINAL_GBS, "frac_nominal": gbs / world / HBM_NOMINAL_GBS,
             "us_per_layer_percentiles": us_dist}
     if not fused:
         ms_score = time_graph(score_step, args.steps, args.warmup, stream, dist) / args.steps
