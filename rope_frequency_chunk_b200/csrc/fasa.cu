@@ -150,6 +150,19 @@ fasa_status cached_int(const void* kernel, uint64_t key, int* out, F fn) {
   return FASA_OK;
 }
 
+// True when a cache's K or V lies in host memory (FASA-M), cached per
+// pointer (a reused address of the other kind would only change the plan's
+// speed, not its result).
+bool kv_on_host(const fasa_cache* c) {
+  int h = 0;
+  if (cached_int(c->k, 11, &h, [&](int* v) {
+        *v = host_resident(c->k) || host_resident(c->v) ? 1 : 0;
+        return FASA_OK;
+      }) != FASA_OK)
+    return false;
+  return h != 0;
+}
+
 // Plain launch with programmatic stream serialization (the kernel waits
 // for its predecessor with griddepcontrol.wait).
 template <typename K, typename P>
@@ -452,7 +465,11 @@ bool wide_plan(const fasa_cache* c, int32_t len, int32_t keff, const DevInfo& d,
   const int G = c->n_q_heads / c->n_kv_heads;
   // n_q > 0: the multi-query decode (n_q tokens, the attention in its own launch)
   const int nq = n_q > 0 ? n_q : 1;
-  for (int direct = (keff <= kWdMaxDirect && G <= 8 && n_q == 0) ? 1 : 0; direct >= 0; --direct) {
+  // K and V in host memory (FASA-M): the kept rows cross the host link
+  // faster from the split-K attention's many CTAs than through the one
+  // resolving CTA (measured at c2: 51.5 us against 62.1 us per layer)
+  const bool in_cta = keff <= kWdMaxDirect && G <= 8 && n_q == 0 && !kv_on_host(c);
+  for (int direct = in_cta ? 1 : 0; direct >= 0; --direct) {
     const WdLayout base = wd_layout(pl->n_loc, len, keff, direct, G, pl->n_split, 0, paged, nq);
     if (base.total > d.smem_optin) continue;
     // entries of each CTA's region the resolving CTA stages in shared memory:

@@ -1,8 +1,11 @@
 """GPU parity of FASA-M, the memory-optimised variant: K and V in pinned
 host memory read across the host link, only the dominant-FC sketch on the
-device. The same kernels run on both kinds of cache, so every result must be
-bit-identical to the device-resident cache's, and it is also checked against
-the CPU oracle."""
+device. The kept sets must be identical to the device-resident cache's, and
+so must the outputs wherever both caches run the same attention kernel; the
+fused plan attends a host-resident cache's kept rows with the split-K
+launch even where a device-resident cache is attended inside the fused
+kernel, and those outputs agree within the two kernels' rounding. Every
+result is also checked against the CPU oracle."""
 import ctypes
 
 import numpy as np
@@ -60,7 +63,12 @@ def test_decode_on_host_resident_cache(path, k):
             res.append((idx, out))
     finally:
         F.fasa_set_decode_path(F.DECODE_AUTO)
-    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert torch.equal(res[0][0], res[1][0])
+    if path == F.DECODE_FUSED and k <= 256:  # in-CTA attention on the device cache, split-K on the host one
+        assert F.fasa_decode_launches(dev, wl.ctx_len, k) == 1 and F.fasa_decode_launches(host, wl.ctx_len, k) > 1
+        U.check_gpu_pair(wl, U.stored(res[0][1]), U.stored(res[1][1]))
+    else:
+        assert torch.equal(res[0][1], res[1][1])
     U.check_decode_heads(wl, inp, host, q, k, U.all_heads(wl), res[1][1], res[1][0])
 
 
