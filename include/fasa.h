@@ -148,7 +148,10 @@ fasa_status fasa_check_dom_idx(const int32_t* dom_idx_host, int32_t n_kv_heads, 
  *    to device memory.
  *  - A decode streams the sketch from HBM, selects, and then reads only the
  *    k_eff kept K and V rows of each (b, g) across the host link, 2 * 128 *
- *    es bytes per kept token.
+ *    es bytes per kept token. The fused plan reads them with its split-K
+ *    attention launch (many CTAs keep more requests on the link) also for
+ *    budgets it would attend inside the fused kernel on a device-resident
+ *    cache, so fasa_decode_launches counts 2 or 3 there.
  *  - fasa_dense_decode reads all of K and V across the link (correct, slow;
  *    bf16 caches only: FASA_ERR_UNSUPPORTED for an f32 FASA-M cache).
  *
