@@ -235,15 +235,16 @@ __device__ __forceinline__ void am_merge_warps(const float* wm, const float* wl,
 
 // Split-K attention over a row's kept list (or all its rows) for G <= 8:
 // grid (splits, rows); CTA `split` takes list positions [split*slice, ...),
-// its 4 warps contiguous quarters of them in steps of 16 rows; the warps
-// merge in shared memory and the CTA writes its partial (m, l, o), or with
-// one split the output (attend_merge_kernel merges the partials).
+// its NW warps (4, or 2 for many rows of one split each) contiguous parts of
+// them in steps of 16 rows; the warps merge in shared memory and the CTA
+// writes its partial (m, l, o), or with one split the output
+// (attend_merge_kernel merges the partials).
 template <int NW>
 __global__ void __launch_bounds__(NW * 32, 8 / NW) attend_mma_kernel(const CcParams p) {
   constexpr int kAmWarps = NW, kAmThreads = NW * 32;
   extern __shared__ __align__(128) unsigned char smem[];
   __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem);
-  float* qs = reinterpret_cast<float*>(smem + 8 * kD * 2);  // the raw queries: G <= 8 rows
+  float* qs = reinterpret_cast<float*>(smem + 8 * kD * 2);  // after the raw queries (G <= 8 rows)
   double* cs = reinterpret_cast<double*>(qs + 8 * kD);
   unsigned char* ring = reinterpret_cast<unsigned char*>(cs + 2 * kNFC);
   const int split = blockIdx.x, row = blockIdx.y;
