@@ -293,8 +293,8 @@ fasa_status fasa_decode(const fasa_cache* cache, int32_t len, const void* q, int
 
 /* Launch plan of fasa_decode (library code, no counterpart in the paper). */
 #define FASA_DECODE_AUTO 0   /* chosen from the shape (default) */
-#define FASA_DECODE_FUSED 1  /* row-split decode: one launch (two for k_eff > 512) */
-#define FASA_DECODE_STAGED 2 /* four-launch decode */
+#define FASA_DECODE_FUSED 1  /* row-split decode: one launch (k_eff <= 256, G <= 8), else 2-3 */
+#define FASA_DECODE_STAGED 2 /* score, filter, finalize, attend (and the split merge): 4-5 launches */
 
 /* Sets the plan every later fasa_decode call of this process uses (a
  * process-wide setting; FASA_ERR_INVALID_ARG for an unknown value). */
