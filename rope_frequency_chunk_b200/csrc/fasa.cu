@@ -641,7 +641,10 @@ fasa_status attend_per_sm(const AttendKernel& k, int* per_sm) {
 // resident CTAs at most, each with at least one step per warp; sets the
 // slice (list positions per CTA) too. *nw: warps per CTA of the tensor-core
 // kernel, 2 when the rows alone (one split each) would overfill a wave of
-// 4-warp CTAs but fill one of 2-warp CTAs.
+// 4-warp CTAs but fill one of 2-warp CTAs, for short lists (at most
+// kAm2MaxKeep positions: c5's kept lists; the dense decode's 16K-row lists
+// stream faster from 4-warp CTAs, 596 against 658 us).
+constexpr int kAm2MaxKeep = 2048;
 fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const DevInfo& d, int* splits, int* slice,
                          int* nw) {
   int per_sm = 0;
@@ -655,7 +658,7 @@ fasa_status attend_split(int group, int rows, int n_keep, int splits_max, const 
   *slice = (int)(ceil_div(units, sp) * kUnit);
   *splits = (int)ceil_div(std::max(n_keep, 1), *slice);
   *nw = 4;
-  if (group <= 8 && *splits == 1 && (int64_t)rows > (int64_t)per_sm * d.sms) {
+  if (group <= 8 && *splits == 1 && n_keep <= kAm2MaxKeep && (int64_t)rows > (int64_t)per_sm * d.sms) {
     int per_sm2 = 0;
     if ((s = attend_per_sm(attend_kernel(group, 2), &per_sm2)) != FASA_OK) return s;
     if ((int64_t)rows <= (int64_t)per_sm2 * d.sms) *nw = 2;
